@@ -1,0 +1,421 @@
+#!/usr/bin/env python
+"""Benchmark: MoE-layer decode tokens/s and achieved HBM GB/s for one
+512-expert, hidden-4096, 4-bit MoE layer at decode batch 1 on one B200.
+
+One step = one call of the whole expert forward (router, top-k, gate/up
+dequant + SwiGLU, down dequant, combine + shared gate + residual + RMSNorm)
+for one fresh token. Inputs are seeded synthetic tensors of the layer's shape
+(no model weights exist here); the routed-expert pool is 3.4 GB and each step
+uses one of 48 copies of the router, shared expert, gate vector and RMSNorm
+weight (~11 MB each, 0.5 GB in all), so no step finds its inputs in the 126 MB L2.
+
+--impl reference times the CPU oracle (plain C, double precision) on the
+same workload; it is the deliberately slow baseline arm.
+
+Prints one JSON line (rank 0). Multi-GPU (torchrun): independent replicas,
+one per GPU, no data-path collective; time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer decode tokens/s and achieved HBM GB/s (% of 8 TB/s), 4-bit experts, 1 B200"
+UNIT = "tokens/s"
+NOMINAL_HBM = 8000.0  # GB/s
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=120000)
+    ap.add_argument("--warmup", type=int, default=480)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="layer_q4", choices=["layer_q4", "layer_q2"])
+    ap.add_argument("--copies", type=int, default=48)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=20000)
+    ap.add_argument("--prof-steps", type=int, default=2000)
+    return ap.parse_args()
+
+
+def dist_info():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
+
+
+# ------------------------------------------------------------------ clocks sampler
+class Clocks:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id, self.proc, self.out = gpu_id, None, None
+
+    def start(self):
+        try:
+            self.out = open(os.devnull, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            text, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            text, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in text.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0])); smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(smax), "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ workload
+def build_workload(cfg, copies, dev):
+    import numpy as np
+    import torch
+
+    import fixtures.gpu as fxg
+    import quantized_expert_decode_moe_b200 as qm
+    from fixtures import gen
+
+    base = fxg.device_layer(cfg, 0, device=dev)
+    routed = [qm.Expert(*[qm.QMat(base["q"][m][e], base["s"][m][e], base["b"][m][e]) for m in range(3)])
+              for e in range(cfg.E)]
+    layers, keep = [], [base]
+    for c in range(copies):
+        t = base if c == 0 else fxg.device_layer(cfg, 100 + c, device=dev, expert_ids=[cfg.E])
+        keep.append(t)
+        j = cfg.E if c == 0 else 0
+        shared = qm.Expert(*[qm.QMat(t["q"][m][j], t["s"][m][j], t["b"][m][j]) for m in range(3)])
+        layers.append(qm.Layer(hidden=cfg.H, inter=cfg.I, top_k=cfg.k, bits=cfg.bits, router_w=t["router_w"],
+                               experts=routed, rms_gamma=t["gamma"], shared=shared, shared_gate_w=t["gate_w"],
+                               router_bias=None, rms_eps=cfg.rms_eps))
+    P = copies * 5
+    x = np.stack([gen.x_tokens(cfg, s, T=1)[0] for s in range(P)])
+    xd = torch.from_numpy(x.view(np.int16)).to(dev)
+    h0 = torch.from_numpy(gen.bf16_bits_to_f32(x).astype(np.float32)).to(dev)
+    return dict(layers=layers, keep=keep, x=xd, h=h0.clone(), h0=h0, P=P, x_host=x)
+
+
+def kernel_src_sha():
+    h = hashlib.sha256()
+    for f in ("common.cuh", "kernels.cu", "kernels.cuh", "api.cu"):
+        p = os.path.join(ROOT, "quantized_expert_decode_moe_b200", "csrc", f)
+        if os.path.exists(p):
+            h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, config: str):
+    """dram bytes per launch from the committed ncu summary, if it was taken on the current sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None
+    sha = kernel_src_sha()
+    for line in open(p):
+        if line.startswith("#") or not line.strip():
+            continue
+        kv = dict(x.split("=", 1) for x in line.split() if "=" in x)
+        if kv.get("kernel") == kernel and kv.get("config") == config and kv.get("src_sha") == sha:
+            return float(kv["dram_bytes_per_launch"])
+    return None
+
+
+# ------------------------------------------------------------------ CPU oracle sample
+def oracle_sample(cfg, seconds: float, max_tokens: int = 10 ** 9):
+    """Times the CPU oracle on decode tokens of this workload; returns (tokens/s, tokens, threads)."""
+    import numpy as np
+
+    import fixtures
+    import oracle
+    from fixtures import gen
+
+    threads = oracle.set_threads(os.cpu_count() or 1)
+    Wr, rb, gs, gamma = fixtures.layer_vectors(cfg, 0)
+    cache = {}
+
+    def expert(e):
+        if e not in cache:
+            cache[e] = fixtures.host_expert(cfg, 0, e)
+        return cache[e]
+
+    shared = expert(cfg.E)
+    done, elapsed = 0, 0.0
+    s = 0
+    while done < max_tokens and (elapsed < seconds or done < 2):
+        x = gen.x_tokens(cfg, s, T=1)
+        s += 1
+        # routing first (untimed) only to regenerate the touched experts on the host
+        idx, _, _ = oracle.route(x, Wr, cfg.k, bias=rb, gs=gs)
+        exps = [expert(int(e)) for e in idx[0]]
+        h = gen.bf16_bits_to_f32(x[0]).astype(np.float64)
+        t0 = time.perf_counter()
+        idx, w, sg = oracle.route(x, Wr, cfg.k, bias=rb, gs=gs)
+        xd = h
+        ys = np.stack([oracle.expert(ex, xd, cfg.H, cfg.I, cfg.G, cfg.bits) for ex in exps])
+        ysh = oracle.expert(shared, xd, cfg.H, cfg.I, cfg.G, cfg.bits)
+        oracle.combine_norm(ys, w[0], ysh, sg[0], h, gamma, cfg.rms_eps)
+        elapsed += time.perf_counter() - t0
+        done += 1
+        if len(cache) > 48:
+            cache.clear()
+    return done / elapsed, done, threads, elapsed
+
+
+def reference_arm(args, cfg):
+    ws_, rank, _ = dist_info()
+    if rank != 0:
+        return
+    budget = max(args.cpu_seconds, 5.0)
+    steps = max(1, min(args.steps, 10 ** 6))
+    rate, n, threads, el = oracle_sample(cfg, budget, max_tokens=steps)
+    sample = (f"{n} decode tokens of the {cfg.name} workload (one token = one step, capped by a "
+              f"{budget:.0f} s budget), experts regenerated on the host before timing")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": rate, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": n, "steps_requested": args.steps, "warmup": 0, "ms_per_step": 1e3 * el / n,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; no model weights)",
+        "config": {"workload": cfg.note, "H": cfg.H, "E": cfg.E, "top_k": cfg.k, "I": cfg.I, "bits": cfg.bits,
+                   "T": 1},
+        "cpu_baseline": {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": rate, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+def ours(args, cfg):
+    import numpy as np
+    import torch
+
+    import quantized_expert_decode_moe_b200 as qm
+
+    world, rank, local = dist_info()
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    qm.lib()
+    W = build_workload(cfg, args.copies, dev)
+    layers, P = W["layers"], W["P"]
+    C = len(layers)
+    ws = qm.new_workspace(layers[0], 1)
+    xo = torch.empty((P, cfg.H), dtype=torch.int16, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    G = P  # steps per graph replay: every (token, copy) pair once
+
+    def step(s):
+        i = s % P
+        qm.moe_layer_forward(layers[s % C], W["x"][i:i + 1], W["h"][i:i + 1], xo[i:i + 1], ws=ws, stream=stream)
+
+    graphs = {}
+
+    def graph_of(n):
+        if n not in graphs:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(stream):
+                for s in range(n):   # eager pass first: lazy kernel attributes are set outside capture
+                    step(s)
+                stream.synchronize()
+                with torch.cuda.graph(g, stream=stream):
+                    for s in range(n):
+                        step(s)
+            graphs[n] = g
+        return graphs[n]
+
+    def run(n):
+        full, rem = divmod(n, G)
+        for _ in range(full):
+            graph_of(G).replay()
+        if rem:
+            graph_of(rem).replay()
+
+    with torch.cuda.stream(stream):
+        graph_of(G)
+        if args.steps % G:
+            graph_of(args.steps % G)
+        if args.warmup % G:
+            graph_of(args.warmup % G)
+        run(max(args.warmup, 3))
+    stream.synchronize()
+    assert qm.moe_poll_status(ws, stream) == 0
+
+    gpu_uuid = str(getattr(torch.cuda.get_device_properties(dev), "uuid", "") or "")
+    clocks = Clocks(("GPU-" + gpu_uuid) if gpu_uuid and not gpu_uuid.startswith("GPU-") else (gpu_uuid or str(local)))
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        run(args.steps)
+        e1.record(stream)
+    e1.synchronize()
+    torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    assert qm.moe_poll_status(ws, stream) == 0
+
+    # per-kernel durations (events between the kernels, no overlap)
+    nk = 4
+    prof_n = min(args.prof_steps, args.steps)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(prof_n)]
+    with torch.cuda.stream(stream):
+        for row in evs:            # torch creates the CUDA event on its first record
+            for e in row:
+                e.record(stream)
+        for s in range(prof_n):
+            i = s % P
+            qm.moe_layer_forward_timed(layers[s % C], W["x"][i:i + 1], W["h"][i:i + 1], xo[i:i + 1], ws=ws,
+                                       events=evs[s], stream=stream)
+    stream.synchronize()
+    names = ["route_logits_kernel", "gateup_decode_kernel", "down_decode_kernel", "norm_kernel"]
+    dur = [sum(evs[s][j].elapsed_time(evs[s][j + 1]) for s in range(prof_n)) / prof_n for j in range(nk)]
+    chain_ms = sum(evs[s][0].elapsed_time(evs[s][nk]) for s in range(prof_n)) / prof_n
+
+    # end to end through the public API with host buffers
+    e2e_n = min(args.e2e_steps, args.steps)
+    xh = torch.from_numpy(W["x_host"].view(np.int16)).pin_memory()
+    hh = W["h0"].cpu().pin_memory()
+    outh = torch.empty((P, cfg.H), dtype=torch.int16).pin_memory()
+    xdev = torch.empty((1, cfg.H), dtype=torch.int16, device=dev)
+    hdev = torch.empty((1, cfg.H), dtype=torch.float32, device=dev)
+    odev = torch.empty((1, cfg.H), dtype=torch.int16, device=dev)
+    with torch.cuda.stream(stream):
+        for s in range(8):
+            i = s % P
+            xdev.copy_(xh[i:i + 1], non_blocking=True); hdev.copy_(hh[i:i + 1], non_blocking=True)
+            qm.moe_layer_forward(layers[s % C], xdev, hdev, odev, ws=ws, stream=stream)
+            outh[i:i + 1].copy_(odev, non_blocking=True)
+        stream.synchronize()
+        if dist:
+            dist.barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for s in range(e2e_n):
+            i = s % P
+            xdev.copy_(xh[i:i + 1], non_blocking=True)
+            hdev.copy_(hh[i:i + 1], non_blocking=True)
+            qm.moe_layer_forward(layers[s % C], xdev, hdev, odev, ws=ws, stream=stream)
+            outh[i:i + 1].copy_(odev, non_blocking=True)
+        f1.record(stream)
+    f1.synchronize()
+    e2e_ms = f0.elapsed_time(f1)
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    peaks, peak_kind = measured_peaks()
+    active = cfg.active_bytes_per_token                      # expert bytes per token (4 experts)
+    router_bytes = cfg.E * cfg.H * 2
+    tok_s = world * args.steps / (ms * 1e-3)
+    per_tok_s = args.steps / (ms * 1e-3)
+    gbs = active * per_tok_s / 1e9
+    # dominant kernel: the gate/up dequant GEMV, 2/3 of the expert bytes
+    j_dom = max(range(nk), key=lambda j: dur[j])
+    gu_bytes = (cfg.k + 1) * 2 * (cfg.I * cfg.H * cfg.bits // 8 + 2 * 2 * cfg.I * (cfg.H // cfg.G)) + 2 * cfg.H
+    dom_bytes = {1: gu_bytes}.get(j_dom)
+    if dom_bytes is None:
+        dn = (cfg.k + 1) * (cfg.H * cfg.I * cfg.bits // 8 + 2 * 2 * cfg.H * (cfg.I // cfg.G))
+        dom_bytes = {0: router_bytes + 2 * cfg.H, 2: dn, 3: 6 * cfg.H * 4}[j_dom]
+    achieved = dom_bytes / (dur[j_dom] * 1e-3) / 1e9
+    traffic = recorded_traffic(names[j_dom], cfg.name)
+    line = {
+        "metric": METRIC, "value": tok_s, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int4 codes, fp16 tensor-core products, fp32 accumulate",
+        "data": "synthetic (seeded; no model weights)",
+        "config": {"workload": cfg.note, "H": cfg.H, "E": cfg.E, "top_k": cfg.k, "shared": 1, "I": cfg.I,
+                   "bits": cfg.bits, "group": cfg.G, "T": 1, "parallelism": f"replicas x{world}",
+                   "l2": f"inputs larger than L2: 3.4 GB routed-expert pool, {C} rotating router/shared copies"},
+        "hbm_gbs": gbs, "pct_of_8tbs": 100.0 * gbs / NOMINAL_HBM,
+        "pct_of_measured_copy": 100.0 * gbs / peaks["hbm_gbs"],
+        "active_bytes_per_token": active, "router_bytes_per_token": router_bytes,
+        "kernel_ms": dict(zip(names, dur)), "chain_ms_serialised": chain_ms,
+        "roofline": {"bound": "hbm", "kernel": names[j_dom], "achieved": achieved, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                     "algorithmic_bytes": dom_bytes, "peak_kind": peak_kind},
+        "e2e": {"value": world * e2e_n / (e2e_ms * 1e-3), "unit": UNIT, "steps": e2e_n,
+                "h2d_bytes_per_step": cfg.H * 2 + cfg.H * 4, "d2h_bytes_per_step": cfg.H * 2},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        rate, n, threads, el = oracle_sample(cfg, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                "sample": f"{n} decode tokens of this workload ({el:.1f} s of oracle time)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    for g in graphs.values():
+        del g
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    import fixtures
+    cfg = fixtures.CONFIGS[args.config]
+    if args.impl == "reference":
+        reference_arm(args, cfg)
+    else:
+        ours(args, cfg)
+
+
+if __name__ == "__main__":
+    main()

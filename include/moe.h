@@ -1,0 +1,203 @@
+/*
+ * moe.h — C ABI of the B200 (sm_100a) quantized MoE expert-forward library.
+ *
+ * The library computes the per-token MoE expert forward of the Flash-MoE
+ * engine ("Flash-MoE: running a 397B parameter model on a laptop", summary
+ * pages): a router picks K=4 active experts per token including one shared
+ * expert ("Model architecture"); each expert's gate/up/down projections are
+ * 4-bit or 2-bit group-affine dequantising matrix-vector products, w = q*s + b
+ * ("Key technologies > FMA-optimised dequant kernel"); SwiGLU joins gate and
+ * up; the expert outputs are combined with the router weights and the shared
+ * expert's gate, added to the residual and RMS-normalised on the device before
+ * the next layer ("Key technologies > Metal compute shaders" and "Deferred GPU
+ * expert compute").
+ *
+ * Conventions for every entry point
+ *  - Tensor pointers are CUDA device memory owned by the caller. The library
+ *    never allocates, frees or synchronises on these calls (moe_poll_status is
+ *    the one call that synchronises, by design).
+ *  - bf16 values are passed as their uint16_t bit patterns; fp32 as float.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream). Every call is asynchronous on that stream.
+ *  - Argument and shape errors are detected on the host before anything is
+ *    launched and returned as MOE_ERR_INVALID_ARGUMENT / MOE_ERR_UNSUPPORTED /
+ *    MOE_ERR_WORKSPACE; a failed launch returns MOE_ERR_CUDA. Device-side
+ *    errors (an expert id out of range) are latched in the workspace status
+ *    word and read back with moe_poll_status.
+ *  - Device pointers must be 16-byte aligned; H, I must be multiples of 128
+ *    (one 128-element k-span) and of the quantisation group; the group is 64.
+ *  - No global state: calls on different streams with different workspaces
+ *    may run concurrently.
+ *
+ * Packed matrix layout (the pages fix the affine form, not the packing; this
+ * is the plain reading used throughout):
+ *  - q: uint32 [R][K*bits/32], row-major; element k of row r sits in word
+ *    k/(32/bits) at bit offset bits*(k % (32/bits)), least significant first.
+ *  - scales, biases: bf16 [R][K/group]; group = `group` consecutive k of a row.
+ *  - dequantised weight w[r][k] = q * scales[r][k/group] + biases[r][k/group].
+ *  - gate and up are [I][H] (R = I, K = H); down is [H][I].
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARGUMENT = 1, /* NULL pointer, bad shape, misalignment   */
+  MOE_ERR_UNSUPPORTED = 2,      /* bits not in {2,4}, group != 64, ...    */
+  MOE_ERR_WORKSPACE = 3,        /* workspace missing or too small          */
+  MOE_ERR_CUDA = 4,             /* a CUDA launch or runtime call failed    */
+  MOE_ERR_TIMEOUT = 5,          /* a bounded device-side wait gave up      */
+  MOE_ERR_DEVICE_FAULT = 6      /* a kernel saw an out-of-range expert id  */
+} moe_status;
+
+/* One packed matrix (device pointers). */
+typedef struct {
+  const uint32_t* q;
+  const uint16_t* scales;
+  const uint16_t* biases;
+} moe_qmat;
+
+/* One expert: gate [I][H], up [I][H], down [H][I]. */
+typedef struct {
+  moe_qmat gate, up, down;
+} moe_expert;
+
+/*
+ * One MoE layer. Host struct; its pointers are device memory.
+ *   hidden H, inter I, n_experts E (routed), top_k k (routed, k <= 8),
+ *   bits in {2,4}, group = 64, has_shared in {0,1}, rms_eps > 0.
+ *   router_w    bf16 [E][H]
+ *   router_bias fp32 [E] or NULL: added to the logits before softmax/top-k
+ *   experts     device array [E] of moe_expert
+ *   shared      the shared expert (ignored when has_shared == 0)
+ *   shared_gate_w bf16 [H] (required when has_shared): gate = sigmoid(g_s . x)
+ *   rms_gamma   bf16 [H]
+ */
+typedef struct {
+  int32_t hidden, inter, n_experts, top_k, bits, group, has_shared;
+  float rms_eps;
+  const uint16_t* router_w;
+  const float* router_bias;
+  const moe_expert* experts;
+  moe_expert shared;
+  const uint16_t* shared_gate_w;
+  const uint16_t* rms_gamma;
+} moe_layer;
+
+/* Bytes of workspace that calls on `layer` need for up to max_tokens tokens.
+ * The workspace is caller-owned device memory; it must be zeroed once
+ * (moe_workspace_init) before its first use and may be reused by later calls
+ * on the same stream. */
+moe_status moe_workspace_size(const moe_layer* layer, int32_t max_tokens, size_t* bytes);
+
+/* Clears the workspace status word (async on `stream`). */
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Router ("Model architecture": K=4 active per token incl. one shared;
+ * the router results select the experts to load — HN thread, Table 3 comment).
+ *   logits = router_w . x (+ router_bias), accumulated in fp64;
+ *   topk_idx [T][k]: the k largest logits, descending, ties to the lower index;
+ *   topk_w [T][k]: softmax over all E renormalised over the chosen k (fp32);
+ *   shared_gate [T] (nullable): sigmoid(shared_gate_w . x), 0 if no shared expert.
+ * x: bf16 [T][H]. Uses the workspace for the logits.
+ */
+moe_status moe_route(const moe_layer* layer, const uint16_t* x, int32_t T, int32_t* topk_idx,
+                     float* topk_w, float* shared_gate, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Dequantising matrix-vector product y = W x for one packed matrix
+ * ("FMA-optimised dequant kernel": (q*s + b)*x summed over k).
+ *   W: host struct of device pointers, R rows (a multiple of 16), K columns
+ *   (a multiple of 128), group 64.
+ *   x: fp32 [K]; y: fp32 [R] (overwritten). 4-bit and 2-bit variants.
+ */
+moe_status moe_expert_gemv_q4(const moe_qmat* W, int32_t R, int32_t K, int32_t group,
+                              const float* x, float* y, void* stream);
+moe_status moe_expert_gemv_q2(const moe_qmat* W, int32_t R, int32_t K, int32_t group,
+                              const float* x, float* y, void* stream);
+
+/*
+ * Combine + residual + RMSNorm ("MoE combine + residual + gate", "normalisation +
+ * residual ... passed directly to the next layer"):
+ *   h'[t] = h[t] + sum_i topk_w[t][i] * y_routed[t][i] + shared_gate[t] * y_shared[t]
+ *   x_out[t] = h'[t] / sqrt(mean(h'[t]^2) + eps) * gamma
+ *   y_routed fp32 [T][k][H]; topk_w fp32 [T][k]; y_shared fp32 [T][H] or NULL
+ *   (then shared_gate is ignored and may be NULL); h fp32 [T][H] in/out (h');
+ *   gamma bf16 [H]; x_out bf16 [T][H]; x_out_f32 fp32 [T][H] or NULL.
+ */
+moe_status moe_combine_residual_norm(int32_t T, int32_t H, int32_t k, const float* y_routed,
+                                     const float* topk_w, const float* y_shared,
+                                     const float* shared_gate, float* h, const uint16_t* gamma,
+                                     float eps, uint16_t* x_out, float* x_out_f32, void* stream);
+
+/*
+ * Prefill grouping of routed (token, rank) pairs by expert:
+ *   counts [E], offsets [E+1] (exclusive scan of counts), perm [T*k] where
+ *   perm[offsets[e] + n] is the n-th flattened index t*k + r routed to e, in
+ *   increasing order (a stable sort by expert). topk_idx int32 [T][k].
+ */
+moe_status moe_group_tokens(int32_t T, int32_t k, int32_t E, const int32_t* topk_idx,
+                            int32_t* counts, int32_t* offsets, int32_t* perm, void* ws,
+                            size_t ws_bytes, void* stream);
+
+/*
+ * Whole MoE layer for T tokens: router, expert gate/up + SwiGLU, down, combine
+ * with the shared-expert gate, residual and RMSNorm, all on the device with
+ * no host round trip. T = 1..8 runs the decode kernels; larger T runs the
+ * prefill kernels (grouping by expert, grouped dequant GEMM).
+ *   x_in bf16 [T][H]; h fp32 [T][H] residual in, h' out; x_out bf16 [T][H];
+ *   x_out_f32 fp32 [T][H] or NULL; topk_idx int32 [T][k] or NULL;
+ *   topk_w fp32 [T][k] or NULL.
+ */
+moe_status moe_layer_forward(const moe_layer* layer, const uint16_t* x_in, float* h, int32_t T,
+                             uint16_t* x_out, float* x_out_f32, int32_t* topk_idx, float* topk_w,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * L layers in sequence for one decode token: layer l's x_out feeds layer l+1
+ * and h is carried in fp32 ("Deferred GPU expert compute").
+ *   layers: host array [L]; x_in bf16 [H]; h fp32 [H] in/out; x_out bf16 [H];
+ *   topk_idx_all int32 [L][k] or NULL; layer_inputs bf16 [L][H] or NULL and
+ *   layer_h fp32 [L][H] or NULL: each layer's input x and residual h (for
+ *   teacher-forced checks). Every layer must have the same H, I, E, k, bits.
+ */
+moe_status moe_stack_forward(const moe_layer* layers, int32_t L, const uint16_t* x_in, float* h,
+                             uint16_t* x_out, int32_t* topk_idx_all, uint16_t* layer_inputs,
+                             float* layer_h, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Profiling variant of moe_layer_forward: the same kernels with a CUDA event
+ * recorded before the first and after each of the kernels of the layer, so a
+ * caller can time them one by one. events: host array of n_events created
+ * cudaEvent_t handles (passed as void*); n_events must be at least the number
+ * of kernels of the chosen path + 1 (decode: 5). The kernels run without
+ * programmatic overlap between them. Same arguments and errors otherwise.
+ */
+moe_status moe_layer_forward_timed(const moe_layer* layer, const uint16_t* x_in, float* h, int32_t T,
+                                   uint16_t* x_out, float* x_out_f32, int32_t* topk_idx, float* topk_w,
+                                   void* ws, size_t ws_bytes, void* const* events, int32_t n_events,
+                                   void* stream);
+
+/* Synchronises `stream` and returns the status latched in the workspace by
+ * earlier calls (MOE_OK if none), then clears it. */
+moe_status moe_poll_status(void* ws, void* stream);
+
+/* Static string naming a status code. */
+const char* moe_status_string(moe_status s);
+
+/* Library ABI version (this header: 1). */
+int32_t moe_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

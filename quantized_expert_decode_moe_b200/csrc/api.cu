@@ -1,0 +1,317 @@
+// C-ABI entry points of the quantized MoE expert forward: argument checks on
+// the host, then asynchronous launches on the caller's stream.
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+#include "moe.h"
+
+using namespace qmoe;
+
+namespace {
+
+constexpr int kMaxE = 4096;
+constexpr int kMaxHI = 8192;
+constexpr int kDecodeMaxT = 8;
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Bound of every device-side wait (a staged copy that never lands): 20 ms, or
+// MOE_WAIT_TIMEOUT_NS from the environment (read once).
+unsigned long long wait_bound_ns() {
+  static unsigned long long v = 0;
+  if (!v) {
+    const char* e = getenv("MOE_WAIT_TIMEOUT_NS");
+    unsigned long long x = e ? strtoull(e, nullptr, 10) : 0ull;
+    v = x ? x : 20000000ull;
+  }
+  return v;
+}
+
+moe_status check_qmat(const moe_qmat& m) {
+  if (!m.q || !m.scales || !m.biases) return MOE_ERR_INVALID_ARGUMENT;
+  if (!aligned16(m.q) || !aligned16(m.scales) || !aligned16(m.biases)) return MOE_ERR_INVALID_ARGUMENT;
+  return MOE_OK;
+}
+
+moe_status check_layer(const moe_layer* L) {
+  if (!L) return MOE_ERR_INVALID_ARGUMENT;
+  if (L->bits != 2 && L->bits != 4) return MOE_ERR_UNSUPPORTED;
+  if (L->group != kGroup) return MOE_ERR_UNSUPPORTED;
+  if (L->hidden <= 0 || L->inter <= 0 || L->hidden % kSpan || L->inter % kSpan) return MOE_ERR_INVALID_ARGUMENT;
+  if (L->hidden > kMaxHI || L->inter > kMaxHI) return MOE_ERR_UNSUPPORTED;
+  if (L->n_experts <= 0 || L->n_experts > kMaxE) return MOE_ERR_INVALID_ARGUMENT;
+  if (L->top_k <= 0 || L->top_k > kMaxTopK || L->top_k > L->n_experts) return MOE_ERR_INVALID_ARGUMENT;
+  if (L->has_shared != 0 && L->has_shared != 1) return MOE_ERR_INVALID_ARGUMENT;
+  if (!(L->rms_eps > 0.f) || !isfinite(L->rms_eps)) return MOE_ERR_INVALID_ARGUMENT;
+  if (!L->router_w || !L->experts || !L->rms_gamma) return MOE_ERR_INVALID_ARGUMENT;
+  if (!aligned16(L->router_w) || !aligned16(L->experts) || !aligned16(L->rms_gamma)) return MOE_ERR_INVALID_ARGUMENT;
+  if (L->router_bias && !aligned16(L->router_bias)) return MOE_ERR_INVALID_ARGUMENT;
+  if (L->has_shared) {
+    if (!L->shared_gate_w || !aligned16(L->shared_gate_w)) return MOE_ERR_INVALID_ARGUMENT;
+    moe_status s;
+    if ((s = check_qmat(L->shared.gate)) || (s = check_qmat(L->shared.up)) || (s = check_qmat(L->shared.down))) return s;
+  }
+  return MOE_OK;
+}
+
+int slots_of(const moe_layer* L) { return L->top_k + (L->has_shared ? 1 : 0); }
+
+WsLayout layout_of(const moe_layer* L, int T) {
+  return ws_layout(L->hidden, L->inter, L->n_experts, L->top_k, slots_of(L), T);
+}
+
+moe_status ws_check(const moe_layer* L, int T, void* ws, size_t ws_bytes) {
+  if (!ws) return MOE_ERR_WORKSPACE;
+  if (((uintptr_t)ws & 255u) != 0) return MOE_ERR_INVALID_ARGUMENT;
+  if (ws_bytes < layout_of(L, T).total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+template <class T> T* at(void* ws, size_t off) { return (T*)((char*)ws + off); }
+
+moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// The four-kernel decode chain of one layer for T <= 8 tokens: router logits;
+// gate/up dequant MMAs (top-k recomputed per CTA); down dequant MMAs (SwiGLU
+// applied while building its B fragments); combine + residual + RMSNorm.
+moe_status decode_chain(const moe_layer* L, const uint16_t* x_in, float* h, int T, uint16_t* x_out, float* x_out_f32,
+                        int32_t* topk_idx, float* topk_w, void* ws, cudaStream_t s,
+                        void* const* events = nullptr) {
+  const bool pdl = events == nullptr;
+  auto mark = [&](int i) { if (events) cudaEventRecord((cudaEvent_t)events[i], s); };
+  mark(0);
+  const int H = L->hidden, I = L->inter, E = L->n_experts, k = L->top_k, S = slots_of(L);
+  const WsLayout W = layout_of(L, T);
+  RouteParams rp{};
+  rp.H = H; rp.E = E; rp.T = T; rp.has_shared = L->has_shared;
+  rp.x = x_in; rp.router_w = L->router_w; rp.router_bias = L->router_bias; rp.gate_w = L->shared_gate_w;
+  rp.logits = at<double>(ws, W.logits);
+  rp.zero_buf = at<float>(ws, W.gu);
+  rp.zero_n = (W.y + sizeof(float) * (size_t)T * S * H - W.gu) / sizeof(float);
+  rp.shared = L->shared; rp.I = I; rp.bits = L->bits; rp.prefetch_shared = 0;
+  cudaError_t e = launch_route(rp, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  mark(1);
+
+  GateUpParams gp{};
+  gp.H = H; gp.I = I; gp.E = E; gp.k = k; gp.S = S; gp.has_shared = L->has_shared;
+  gp.nspans = H / kSpan; gp.ntiles = I / 8;
+  const long long gtiles = (long long)S * gp.ntiles;
+  gp.U = gtiles * gp.nspans; gp.nCTA = choose_ncta(gtiles, gp.nspans);
+  gp.x = x_in; gp.logits = rp.logits; gp.experts = L->experts; gp.shared = L->shared;
+  gp.gu = at<float>(ws, W.gu);
+  gp.idx_ws = at<int32_t>(ws, W.idx); gp.w_ws = at<float>(ws, W.w); gp.sg_ws = at<float>(ws, W.sg);
+  gp.slots_ws = at<moe_expert>(ws, W.slots);
+  gp.idx_out = topk_idx; gp.w_out = topk_w;
+  gp.status = at<uint32_t>(ws, W.status);
+  gp.prefetch_down = 0; gp.prefetch_self = 0;
+  gp.wait_ns = wait_bound_ns();
+  if ((e = launch_gateup(gp, L->bits, T, pdl, s)) != cudaSuccess)
+    return e == cudaErrorInvalidConfiguration ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
+  mark(2);
+
+  DownParams dp{};
+  dp.H = H; dp.I = I; dp.E = E; dp.k = k; dp.S = S; dp.has_shared = L->has_shared;
+  dp.nspans = I / kSpan; dp.ntiles = H / 16;
+  const long long dtiles = (long long)S * dp.ntiles;
+  dp.U = dtiles * dp.nspans; dp.nCTA = choose_ncta(dtiles, dp.nspans);
+  dp.gu = gp.gu; dp.idx_ws = gp.idx_ws; dp.slots_ws = gp.slots_ws; dp.experts = L->experts; dp.shared = L->shared;
+  dp.y = at<float>(ws, W.y);
+  dp.status = gp.status; dp.wait_ns = gp.wait_ns;
+  if ((e = launch_down(dp, L->bits, T, pdl, s)) != cudaSuccess)
+    return e == cudaErrorInvalidConfiguration ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
+  mark(3);
+
+  NormParams np{};
+  np.H = H; np.k = k; np.T = T;
+  np.y_routed = dp.y; np.y_routed_tok_stride = (long long)S * H; np.y_routed_slot_stride = H;
+  np.w = gp.w_ws;
+  np.y_shared = L->has_shared ? dp.y + (size_t)k * H : nullptr;
+  np.y_shared_tok_stride = (long long)S * H;
+  np.sg = gp.sg_ws;
+  np.h = h; np.gamma = L->rms_gamma; np.eps = L->rms_eps; np.x_out = x_out; np.x_out_f32 = x_out_f32;
+  if ((e = launch_norm(np, pdl, s)) != cudaSuccess) return MOE_ERR_CUDA;
+  mark(4);
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t moe_abi_version(void) { return 1; }
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_TIMEOUT: return "device wait timed out";
+    case MOE_ERR_DEVICE_FAULT: return "device-side fault (expert id out of range)";
+  }
+  return "unknown status";
+}
+
+moe_status moe_workspace_size(const moe_layer* layer, int32_t max_tokens, size_t* bytes) {
+  moe_status st = check_layer(layer);
+  if (st) return st;
+  if (!bytes || max_tokens <= 0) return MOE_ERR_INVALID_ARGUMENT;
+  *bytes = layout_of(layer, max_tokens).total;
+  return MOE_OK;
+}
+
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || ws_bytes < 256) return MOE_ERR_WORKSPACE;
+  return cuda_status(cudaMemsetAsync(ws, 0, 256, (cudaStream_t)stream));
+}
+
+moe_status moe_route(const moe_layer* layer, const uint16_t* x, int32_t T, int32_t* topk_idx, float* topk_w,
+                     float* shared_gate, void* ws, size_t ws_bytes, void* stream) {
+  moe_status st = check_layer(layer);
+  if (st) return st;
+  if (T <= 0 || !x || !topk_idx || !topk_w || !aligned16(x)) return MOE_ERR_INVALID_ARGUMENT;
+  if ((st = ws_check(layer, T, ws, ws_bytes))) return st;
+  const WsLayout W = layout_of(layer, T);
+  cudaStream_t s = (cudaStream_t)stream;
+  RouteParams rp{};
+  rp.H = layer->hidden; rp.E = layer->n_experts; rp.T = T; rp.has_shared = layer->has_shared;
+  rp.x = x; rp.router_w = layer->router_w; rp.router_bias = layer->router_bias; rp.gate_w = layer->shared_gate_w;
+  rp.logits = at<double>(ws, W.logits);
+  if (launch_route(rp, s) != cudaSuccess) return MOE_ERR_CUDA;
+  TopkParams tp{};
+  tp.E = layer->n_experts; tp.k = layer->top_k; tp.T = T; tp.has_shared = layer->has_shared;
+  tp.logits = rp.logits; tp.idx = topk_idx; tp.w = topk_w; tp.sg = shared_gate;
+  return cuda_status(launch_topk(tp, s));
+}
+
+static moe_status gemv_common(const moe_qmat* W, int32_t R, int32_t K, int32_t group, const float* x, float* y,
+                              int bits, void* stream) {
+  if (!W || !x || !y) return MOE_ERR_INVALID_ARGUMENT;
+  if (group != kGroup) return MOE_ERR_UNSUPPORTED;
+  if (R <= 0 || R % 16 || K <= 0 || K % kSpan || K > 65536) return MOE_ERR_INVALID_ARGUMENT;
+  moe_status st = check_qmat(*W);
+  if (st) return st;
+  if (!aligned16(x) || !aligned16(y)) return MOE_ERR_INVALID_ARGUMENT;
+  cudaStream_t s = (cudaStream_t)stream;
+  GemvParams p{};
+  p.R = R; p.K = K; p.nspans = K / kSpan; p.ntiles = (R + 15) / 16;
+  p.U = (long long)p.ntiles * p.nspans; p.nCTA = choose_ncta(p.ntiles, p.nspans);
+  p.W = *W; p.x = x; p.y = y; p.status = nullptr; p.wait_ns = wait_bound_ns();
+  if (cudaMemsetAsync(y, 0, sizeof(float) * (size_t)R, s) != cudaSuccess) return MOE_ERR_CUDA;
+  const cudaError_t e = launch_gemv(p, bits, s);
+  return e == cudaErrorInvalidConfiguration ? MOE_ERR_UNSUPPORTED : cuda_status(e);
+}
+
+moe_status moe_expert_gemv_q4(const moe_qmat* W, int32_t R, int32_t K, int32_t group, const float* x, float* y,
+                              void* stream) {
+  return gemv_common(W, R, K, group, x, y, 4, stream);
+}
+
+moe_status moe_expert_gemv_q2(const moe_qmat* W, int32_t R, int32_t K, int32_t group, const float* x, float* y,
+                              void* stream) {
+  return gemv_common(W, R, K, group, x, y, 2, stream);
+}
+
+moe_status moe_combine_residual_norm(int32_t T, int32_t H, int32_t k, const float* y_routed, const float* topk_w,
+                                     const float* y_shared, const float* shared_gate, float* h,
+                                     const uint16_t* gamma, float eps, uint16_t* x_out, float* x_out_f32,
+                                     void* stream) {
+  if (T <= 0 || H <= 0 || k < 0 || k > kMaxTopK || H > 65536) return MOE_ERR_INVALID_ARGUMENT;
+  if ((k > 0 && (!y_routed || !topk_w)) || !h || !gamma || !x_out) return MOE_ERR_INVALID_ARGUMENT;
+  if (y_shared && !shared_gate) return MOE_ERR_INVALID_ARGUMENT;
+  if (!(eps > 0.f) || !isfinite(eps)) return MOE_ERR_INVALID_ARGUMENT;
+  NormParams np{};
+  np.H = H; np.k = k; np.T = T;
+  np.y_routed = y_routed; np.y_routed_tok_stride = (long long)k * H; np.y_routed_slot_stride = H;
+  np.w = topk_w; np.y_shared = y_shared; np.y_shared_tok_stride = H; np.sg = shared_gate;
+  np.h = h; np.gamma = gamma; np.eps = eps; np.x_out = x_out; np.x_out_f32 = x_out_f32;
+  return cuda_status(launch_norm(np, false, (cudaStream_t)stream));
+}
+
+moe_status moe_group_tokens(int32_t T, int32_t k, int32_t E, const int32_t* topk_idx, int32_t* counts,
+                            int32_t* offsets, int32_t* perm, void* ws, size_t ws_bytes, void* stream) {
+  (void)ws; (void)ws_bytes;
+  if (T <= 0 || k <= 0 || k > kMaxTopK || E <= 0 || E > kMaxE) return MOE_ERR_INVALID_ARGUMENT;
+  if (!topk_idx || !counts || !offsets || !perm) return MOE_ERR_INVALID_ARGUMENT;
+  GroupParams p{};
+  p.T = T; p.k = k; p.E = E; p.idx = topk_idx; p.counts = counts; p.offsets = offsets; p.perm = perm;
+  return cuda_status(launch_group(p, (cudaStream_t)stream));
+}
+
+moe_status moe_layer_forward(const moe_layer* layer, const uint16_t* x_in, float* h, int32_t T, uint16_t* x_out,
+                             float* x_out_f32, int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes,
+                             void* stream) {
+  moe_status st = check_layer(layer);
+  if (st) return st;
+  if (T <= 0 || !x_in || !h || !x_out) return MOE_ERR_INVALID_ARGUMENT;
+  if (!aligned16(x_in) || !aligned16(h) || !aligned16(x_out)) return MOE_ERR_INVALID_ARGUMENT;
+  if ((st = ws_check(layer, T, ws, ws_bytes))) return st;
+  if (T > kDecodeMaxT) return MOE_ERR_UNSUPPORTED;
+  return decode_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, (cudaStream_t)stream);
+}
+
+moe_status moe_layer_forward_timed(const moe_layer* layer, const uint16_t* x_in, float* h, int32_t T,
+                                   uint16_t* x_out, float* x_out_f32, int32_t* topk_idx, float* topk_w, void* ws,
+                                   size_t ws_bytes, void* const* events, int32_t n_events, void* stream) {
+  moe_status st = check_layer(layer);
+  if (st) return st;
+  if (T <= 0 || !x_in || !h || !x_out) return MOE_ERR_INVALID_ARGUMENT;
+  if (!aligned16(x_in) || !aligned16(h) || !aligned16(x_out)) return MOE_ERR_INVALID_ARGUMENT;
+  if ((st = ws_check(layer, T, ws, ws_bytes))) return st;
+  if (T > kDecodeMaxT) return MOE_ERR_UNSUPPORTED;
+  if (!events || n_events < 5) return MOE_ERR_INVALID_ARGUMENT;
+  for (int i = 0; i < 5; ++i)
+    if (!events[i]) return MOE_ERR_INVALID_ARGUMENT;
+  return decode_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, (cudaStream_t)stream, events);
+}
+
+moe_status moe_stack_forward(const moe_layer* layers, int32_t L, const uint16_t* x_in, float* h, uint16_t* x_out,
+                             int32_t* topk_idx_all, uint16_t* layer_inputs, float* layer_h, void* ws,
+                             size_t ws_bytes, void* stream) {
+  if (!layers || L <= 0 || !x_in || !h || !x_out) return MOE_ERR_INVALID_ARGUMENT;
+  if (!aligned16(x_in) || !aligned16(h) || !aligned16(x_out)) return MOE_ERR_INVALID_ARGUMENT;
+  moe_status st;
+  for (int l = 0; l < L; ++l) {
+    if ((st = check_layer(&layers[l]))) return st;
+    const moe_layer& a = layers[l], &b = layers[0];
+    if (a.hidden != b.hidden || a.inter != b.inter || a.n_experts != b.n_experts || a.top_k != b.top_k ||
+        a.bits != b.bits || a.has_shared != b.has_shared)
+      return MOE_ERR_INVALID_ARGUMENT;
+  }
+  if ((st = ws_check(&layers[0], 1, ws, ws_bytes))) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int H = layers[0].hidden, k = layers[0].top_k;
+  for (int l = 0; l < L; ++l) {
+    const uint16_t* xin = l == 0 ? x_in : x_out;
+    if (layer_inputs && cudaMemcpyAsync(layer_inputs + (size_t)l * H, xin, sizeof(uint16_t) * H,
+                                        cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (layer_h && cudaMemcpyAsync(layer_h + (size_t)l * H, h, sizeof(float) * H, cudaMemcpyDeviceToDevice, s) !=
+                       cudaSuccess)
+      return MOE_ERR_CUDA;
+    if ((st = decode_chain(&layers[l], xin, h, 1, x_out, nullptr, topk_idx_all ? topk_idx_all + (size_t)l * k : nullptr,
+                           nullptr, ws, s)))
+      return st;
+  }
+  return MOE_OK;
+}
+
+moe_status moe_poll_status(void* ws, void* stream) {
+  if (!ws) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  uint32_t v = 0;
+  if (cudaMemcpy(&v, ws, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (v) {
+    if (cudaMemsetAsync(ws, 0, sizeof v, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  return (moe_status)v;
+}
+
+}  // extern "C"

@@ -1,0 +1,128 @@
+"""Host-side checks of the C-ABI library (no GPU needed): it loads, exports
+every entry point the header declares, its struct layouts match the header,
+and argument errors are returned before anything is launched."""
+import ctypes as C
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+import quantized_expert_decode_moe_b200 as qm
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_entry_point():
+    L = qm.lib()
+    names = header_functions()
+    assert len(names) >= 12
+    missing = [n for n in names if not hasattr(L, n)]
+    assert not missing, missing
+    assert qm.moe_abi_version() == 1
+
+
+def test_struct_layout_matches_header():
+    src = r'''
+#include <stdio.h>
+#include <stddef.h>
+#include "moe.h"
+int main(void) {
+  printf("%zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(moe_qmat), sizeof(moe_expert), sizeof(moe_layer),
+         offsetof(moe_layer, rms_eps), offsetof(moe_layer, router_w), offsetof(moe_layer, experts),
+         offsetof(moe_layer, shared), offsetof(moe_layer, rms_gamma));
+  return 0;
+}'''
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "a.c")
+        open(c, "w").write(src)
+        exe = os.path.join(d, "a")
+        subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), "-o", exe, c])
+        got = list(map(int, subprocess.check_output([exe]).split()))
+    L = qm._Layer
+    want = [C.sizeof(qm._QMat), C.sizeof(qm._Expert), C.sizeof(L), L.rms_eps.offset, L.router_w.offset,
+            L.experts.offset, L.shared.offset, L.rms_gamma.offset]
+    assert got == want
+
+
+def test_status_strings():
+    for code in range(7):
+        assert qm.moe_status_string(code)
+    assert qm.moe_status_string(99) == "unknown status"
+
+
+def fake_layer(**kw):
+    """A descriptor with fake (never dereferenced) aligned device pointers."""
+    p = 0x100000
+    ex = qm._Expert(*[qm._QMat(p, p, p) for _ in range(3)])
+    f = dict(hidden=4096, inter=1024, n_experts=512, top_k=3, bits=4, group=64, has_shared=1, rms_eps=1e-6,
+             router_w=p, router_bias=None, experts=p, shared=ex, shared_gate_w=p, rms_gamma=p)
+    f.update(kw)
+    return qm._Layer(**f)
+
+
+def ws_size(layer, T=1):
+    n = C.c_size_t(0)
+    rc = qm.lib().moe_workspace_size(C.byref(layer), T, C.byref(n))
+    return rc, n.value
+
+
+def test_workspace_size_and_layer_validation():
+    rc, n = ws_size(fake_layer())
+    assert rc == 0 and n > 0
+    rc4, n4 = ws_size(fake_layer(), T=4)
+    assert rc4 == 0 and n4 > n
+    assert ws_size(fake_layer(bits=3))[0] == 2            # unsupported bits
+    assert ws_size(fake_layer(group=32))[0] == 2          # unsupported group
+    assert ws_size(fake_layer(top_k=9))[0] == 1           # k > 8
+    assert ws_size(fake_layer(n_experts=2, top_k=3))[0] == 1   # k > E
+    assert ws_size(fake_layer(hidden=4000))[0] == 1       # not a multiple of 128
+    assert ws_size(fake_layer(inter=0))[0] == 1
+    assert ws_size(fake_layer(rms_eps=0.0))[0] == 1
+    assert ws_size(fake_layer(router_w=0x100008))[0] == 1  # misaligned
+    assert ws_size(fake_layer(shared_gate_w=None))[0] == 1
+    assert ws_size(fake_layer(shared_gate_w=None, has_shared=0))[0] == 0
+    assert ws_size(fake_layer(experts=None))[0] == 1
+    assert qm.lib().moe_workspace_size(None, 1, None) == 1
+
+
+def test_entry_points_reject_bad_arguments_before_launch():
+    L = qm.lib()
+    lay = fake_layer()
+    p = C.c_void_p(0x200000)
+    _, n = ws_size(lay)
+    ws = C.c_void_p(0x400000)
+    # layer forward: null input, T = 0, workspace too small, misaligned h
+    assert L.moe_layer_forward(C.byref(lay), None, p, 1, p, None, None, None, ws, n, None) == 1
+    assert L.moe_layer_forward(C.byref(lay), p, p, 0, p, None, None, None, ws, n, None) == 1
+    assert L.moe_layer_forward(C.byref(lay), p, p, 1, p, None, None, None, ws, n - 1, None) == 3
+    assert L.moe_layer_forward(C.byref(lay), p, p, 1, p, None, None, None, None, n, None) == 3
+    assert L.moe_layer_forward(C.byref(lay), p, C.c_void_p(0x200004), 1, p, None, None, None, ws, n, None) == 1
+    assert L.moe_layer_forward(C.byref(lay), p, p, 1, p, None, None, None, C.c_void_p(0x400010), n, None) == 1
+    # route: null outputs
+    assert L.moe_route(C.byref(lay), p, 1, None, p, None, ws, n, None) == 1
+    # gemv: bad group, K not a multiple of 128, R = 0, null matrix
+    W = qm._QMat(0x100000, 0x100000, 0x100000)
+    assert L.moe_expert_gemv_q4(C.byref(W), 16, 256, 32, p, p, None) == 2
+    assert L.moe_expert_gemv_q4(C.byref(W), 16, 200, 64, p, p, None) == 1
+    assert L.moe_expert_gemv_q2(C.byref(W), 0, 256, 64, p, p, None) == 1
+    assert L.moe_expert_gemv_q4(C.byref(W), 300, 256, 64, p, p, None) == 1   # rows not a multiple of 16
+    assert L.moe_expert_gemv_q2(None, 16, 256, 64, p, p, None) == 1
+    # combine: eps <= 0, shared output without gate
+    assert L.moe_combine_residual_norm(1, 256, 2, p, p, None, None, p, p, C.c_float(0.0), p, None, None) == 1
+    assert L.moe_combine_residual_norm(1, 256, 2, p, p, p, None, p, p, C.c_float(1e-6), p, None, None) == 1
+    # grouping: k > 8, E <= 0
+    assert L.moe_group_tokens(4, 9, 16, p, p, p, p, None, 0, None) == 1
+    assert L.moe_group_tokens(4, 2, 0, p, p, p, p, None, 0, None) == 1
+    # stack: mismatched layers
+    lays = (qm._Layer * 2)(fake_layer(), fake_layer(inter=2048))
+    assert L.moe_stack_forward(lays, 2, p, p, p, None, None, None, ws, n, None) == 1
+    assert L.moe_poll_status(None, None) == 3
