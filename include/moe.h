@@ -186,6 +186,34 @@ moe_status moe_layer_forward_timed(const moe_layer* layer, const uint16_t* x_in,
                                    void* ws, size_t ws_bytes, void* const* events, int32_t n_events,
                                    void* stream);
 
+/*
+ * moe_layer_forward without a caller-provided workspace, for callers that
+ * cannot allocate device memory themselves: for example a plug-in running
+ * inside a host application that owns every device allocation and hands the
+ * plug-in only its input and output buffers, or a latency-critical loop in
+ * which cudaMalloc (and the device-wide synchronisation it can imply) is not
+ * allowed. The Flash-MoE pages have no counterpart to this entry point; it is
+ * a deployment convenience of this library.
+ *
+ * The scratch lives in one static device array of MOE_NOALLOC_SCRATCH_BYTES
+ * inside the library; every GPU that loads the library holds it until the
+ * process exits. The call allocates and frees nothing. The first call on a
+ * device looks up that array's device address (once per device, with that
+ * device current); make that first call before any stream capture.
+ * Layers and token counts whose workspace (moe_workspace_size) exceeds
+ * MOE_NOALLOC_SCRATCH_BYTES are rejected with MOE_ERR_WORKSPACE.
+ * All calls share the array and it keeps the last call's contents; the call
+ * clears what has to start at zero. Calls whose kernels overlap on the GPU
+ * (different streams, or different host threads) race on the array: order
+ * them on one stream. Device-side status latched by this call cannot be read
+ * with moe_poll_status. Arguments and errors are otherwise those of
+ * moe_layer_forward.
+ */
+#define MOE_NOALLOC_SCRATCH_BYTES (4u << 20)
+moe_status moe_layer_forward_noalloc(const moe_layer* layer, const uint16_t* x_in, float* h, int32_t T,
+                                     uint16_t* x_out, float* x_out_f32, int32_t* topk_idx, float* topk_w,
+                                     void* stream);
+
 /* Synchronises `stream` and returns the status latched in the workspace by
  * earlier calls (MOE_OK if none), then clears it. */
 moe_status moe_poll_status(void* ws, void* stream);

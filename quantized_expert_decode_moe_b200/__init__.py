@@ -15,7 +15,7 @@ __all__ = [
     "MoeError", "QMat", "Expert", "Layer", "lib", "build",
     "moe_abi_version", "moe_status_string", "moe_workspace_size", "moe_workspace_init", "moe_route",
     "moe_expert_gemv_q4", "moe_expert_gemv_q2", "moe_combine_residual_norm", "moe_group_tokens",
-    "moe_layer_forward", "moe_layer_forward_timed", "moe_stack_forward", "moe_poll_status", "new_workspace",
+    "moe_layer_forward", "moe_layer_forward_noalloc", "moe_layer_forward_timed", "moe_stack_forward", "moe_poll_status", "new_workspace",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -76,6 +76,7 @@ def lib():
         L.moe_group_tokens.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, C.c_size_t, vp]
         L.moe_layer_forward.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp, C.c_size_t, vp]
         L.moe_layer_forward_timed.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp, C.c_size_t, vp, i32, vp]
+        L.moe_layer_forward_noalloc.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp]
         L.moe_stack_forward.argtypes = [vp, i32, vp, vp, vp, vp, vp, vp, vp, C.c_size_t, vp]
         L.moe_poll_status.argtypes = [vp, vp]
         _lib = L
@@ -216,6 +217,14 @@ def moe_layer_forward(layer: Layer, x_in, h, x_out, x_out_f32=None, topk_idx=Non
     _ok(lib().moe_layer_forward(layer.cref(), _ptr(x_in), _ptr(h), x_in.shape[0], _ptr(x_out), _ptr(x_out_f32),
                                 _ptr(topk_idx), _ptr(topk_w), _ptr(ws), ws.numel(), _stream(stream)),
         "moe_layer_forward")
+
+
+def moe_layer_forward_noalloc(layer: Layer, x_in, h, x_out, x_out_f32=None, topk_idx=None, topk_w=None, stream=None):
+    """moe_layer_forward with the library's own static scratch instead of a workspace, for callers that
+    cannot allocate device memory (see include/moe.h). Calls must not overlap on the GPU."""
+    _ok(lib().moe_layer_forward_noalloc(layer.cref(), _ptr(x_in), _ptr(h), x_in.shape[0], _ptr(x_out),
+                                        _ptr(x_out_f32), _ptr(topk_idx), _ptr(topk_w), _stream(stream)),
+        "moe_layer_forward_noalloc")
 
 
 def moe_layer_forward_timed(layer: Layer, x_in, h, x_out, x_out_f32=None, topk_idx=None, topk_w=None, *, ws, events,

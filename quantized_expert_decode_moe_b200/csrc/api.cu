@@ -4,6 +4,8 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.cuh"
 #include "moe.h"
@@ -299,6 +301,52 @@ moe_status moe_stack_forward(const moe_layer* layers, int32_t L, const uint16_t*
       return st;
   }
   return MOE_OK;
+}
+
+}  // extern "C"
+
+// Scratch of moe_layer_forward_noalloc: one file-scope device array, so that
+// callers that cannot allocate still get a workspace. Host code only sees a
+// host-side stand-in under this name; the device address is looked up once
+// per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[MOE_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (nullptr on failure).
+void* noalloc_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return nullptr;
+    g_noalloc_ptr[dev] = p;
+  }
+  return g_noalloc_ptr[dev];
+}
+}  // namespace
+
+extern "C" {
+
+moe_status moe_layer_forward_noalloc(const moe_layer* layer, const uint16_t* x_in, float* h, int32_t T,
+                                     uint16_t* x_out, float* x_out_f32, int32_t* topk_idx, float* topk_w,
+                                     void* stream) {
+  moe_status st = check_layer(layer);
+  if (st) return st;
+  if (T <= 0 || !x_in || !h || !x_out) return MOE_ERR_INVALID_ARGUMENT;
+  if (!aligned16(x_in) || !aligned16(h) || !aligned16(x_out)) return MOE_ERR_INVALID_ARGUMENT;
+  if (T > kDecodeMaxT) return MOE_ERR_UNSUPPORTED;
+  if (layout_of(layer, T).total > (size_t)MOE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_WORKSPACE;
+  void* ws = noalloc_scratch();
+  if (!ws) return MOE_ERR_CUDA;
+  cudaStream_t s = (cudaStream_t)stream;
+  // the status word must start clear; the accumulators are cleared by the chain itself
+  if (cudaMemsetAsync(ws, 0, 256, s) != cudaSuccess) return MOE_ERR_CUDA;
+  return decode_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, s);
 }
 
 moe_status moe_poll_status(void* ws, void* stream) {
