@@ -377,7 +377,7 @@ def ours(args, cfg):
     line = {
         "metric": METRIC, "value": tok_s, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "int4 codes, fp16 tensor-core products, fp32 accumulate",
+        "scaling": "weak", "vs_baseline": None, "dtype": "u4 codes x s8 activation digits on int8 tensor cores (s32), fp32 scale+accumulate",
         "data": "synthetic (seeded; no model weights)",
         "config": {"workload": cfg.note, "H": cfg.H, "E": cfg.E, "top_k": cfg.k, "shared": 1, "I": cfg.I,
                    "bits": cfg.bits, "group": cfg.G, "T": 1, "parallelism": f"replicas x{world}",

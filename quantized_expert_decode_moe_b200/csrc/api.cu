@@ -76,66 +76,60 @@ template <class T> T* at(void* ws, size_t off) { return (T*)((char*)ws + off); }
 
 moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
-// The four-kernel decode chain of one layer for T <= 8 tokens: router logits;
-// gate/up dequant MMAs (top-k recomputed per CTA); down dequant MMAs (SwiGLU
-// applied while building its B fragments); combine + residual + RMSNorm.
+// The four-kernel decode chain of one layer for T <= 8 tokens, linked by
+// programmatic dependent launch. Every kernel lets its successor launch only
+// after its own dependency wait, so a kernel's pre-wait part may read what the
+// kernel two places before it wrote:
+//   1. router logits (weights loaded before the wait, x after it);
+//   2. gate/up + SwiGLU (B tables of x and the shared expert before the wait;
+//      then top-k of the logits in every CTA and the routed experts);
+//   3. down + combine (top-k, residual rows and the bulk copies of its rows of
+//      every chosen expert before the wait; a -> B tables and
+//      hacc = h + weighted expert outputs after it);
+//   4. RMSNorm of hacc into x_out, h.
 moe_status decode_chain(const moe_layer* L, const uint16_t* x_in, float* h, int T, uint16_t* x_out, float* x_out_f32,
                         int32_t* topk_idx, float* topk_w, void* ws, cudaStream_t s,
-                        void* const* events = nullptr) {
+                        void* const* events = nullptr, uint16_t* x_rec = nullptr, float* h_rec = nullptr) {
   const bool pdl = events == nullptr;
   auto mark = [&](int i) { if (events) cudaEventRecord((cudaEvent_t)events[i], s); };
   mark(0);
   const int H = L->hidden, I = L->inter, E = L->n_experts, k = L->top_k, S = slots_of(L);
   const WsLayout W = layout_of(L, T);
+  uint32_t* status = at<uint32_t>(ws, W.status);
   RouteParams rp{};
   rp.H = H; rp.E = E; rp.T = T; rp.has_shared = L->has_shared;
   rp.x = x_in; rp.router_w = L->router_w; rp.router_bias = L->router_bias; rp.gate_w = L->shared_gate_w;
   rp.logits = at<double>(ws, W.logits);
-  rp.zero_buf = at<float>(ws, W.gu);
-  rp.zero_n = (W.y + sizeof(float) * (size_t)T * S * H - W.gu) / sizeof(float);
-  rp.shared = L->shared; rp.I = I; rp.bits = L->bits; rp.prefetch_shared = 0;
-  cudaError_t e = launch_route(rp, s);
+  rp.h = h; rp.x_rec = x_rec; rp.h_rec = h_rec;
+  cudaError_t e = launch_route(rp, s, pdl);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   mark(1);
 
   GateUpParams gp{};
   gp.H = H; gp.I = I; gp.E = E; gp.k = k; gp.S = S; gp.has_shared = L->has_shared;
-  gp.nspans = H / kSpan; gp.ntiles = I / 8;
-  const long long gtiles = (long long)S * gp.ntiles;
-  gp.U = gtiles * gp.nspans; gp.nCTA = choose_ncta(gtiles, gp.nspans);
+  gp.nCTA = gateup_ctas(I);
   gp.x = x_in; gp.logits = rp.logits; gp.experts = L->experts; gp.shared = L->shared;
-  gp.gu = at<float>(ws, W.gu);
-  gp.idx_ws = at<int32_t>(ws, W.idx); gp.w_ws = at<float>(ws, W.w); gp.sg_ws = at<float>(ws, W.sg);
-  gp.slots_ws = at<moe_expert>(ws, W.slots);
+  gp.a = at<float>(ws, W.a);
   gp.idx_out = topk_idx; gp.w_out = topk_w;
-  gp.status = at<uint32_t>(ws, W.status);
-  gp.prefetch_down = 0; gp.prefetch_self = 0;
-  gp.wait_ns = wait_bound_ns();
+  gp.status = status; gp.wait_ns = wait_bound_ns();
   if ((e = launch_gateup(gp, L->bits, T, pdl, s)) != cudaSuccess)
     return e == cudaErrorInvalidConfiguration ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
   mark(2);
 
   DownParams dp{};
   dp.H = H; dp.I = I; dp.E = E; dp.k = k; dp.S = S; dp.has_shared = L->has_shared;
-  dp.nspans = I / kSpan; dp.ntiles = H / 16;
-  const long long dtiles = (long long)S * dp.ntiles;
-  dp.U = dtiles * dp.nspans; dp.nCTA = choose_ncta(dtiles, dp.nspans);
-  dp.gu = gp.gu; dp.idx_ws = gp.idx_ws; dp.slots_ws = gp.slots_ws; dp.experts = L->experts; dp.shared = L->shared;
-  dp.y = at<float>(ws, W.y);
-  dp.status = gp.status; dp.wait_ns = gp.wait_ns;
+  dp.nCTA = down_ctas(H);
+  dp.logits = rp.logits; dp.a = gp.a; dp.h = h; dp.experts = L->experts; dp.shared = L->shared;
+  dp.hacc = at<float>(ws, W.hacc);
+  dp.status = status; dp.wait_ns = gp.wait_ns;
   if ((e = launch_down(dp, L->bits, T, pdl, s)) != cudaSuccess)
     return e == cudaErrorInvalidConfiguration ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
   mark(3);
 
-  NormParams np{};
-  np.H = H; np.k = k; np.T = T;
-  np.y_routed = dp.y; np.y_routed_tok_stride = (long long)S * H; np.y_routed_slot_stride = H;
-  np.w = gp.w_ws;
-  np.y_shared = L->has_shared ? dp.y + (size_t)k * H : nullptr;
-  np.y_shared_tok_stride = (long long)S * H;
-  np.sg = gp.sg_ws;
-  np.h = h; np.gamma = L->rms_gamma; np.eps = L->rms_eps; np.x_out = x_out; np.x_out_f32 = x_out_f32;
-  if ((e = launch_norm(np, pdl, s)) != cudaSuccess) return MOE_ERR_CUDA;
+  NormDecodeParams np{};
+  np.H = H; np.T = T;
+  np.hacc = dp.hacc; np.h = h; np.gamma = L->rms_gamma; np.eps = L->rms_eps; np.x_out = x_out; np.x_out_f32 = x_out_f32;
+  if ((e = launch_norm_decode(np, pdl, s)) != cudaSuccess) return MOE_ERR_CUDA;
   mark(4);
   return MOE_OK;
 }
@@ -184,7 +178,7 @@ moe_status moe_route(const moe_layer* layer, const uint16_t* x, int32_t T, int32
   rp.H = layer->hidden; rp.E = layer->n_experts; rp.T = T; rp.has_shared = layer->has_shared;
   rp.x = x; rp.router_w = layer->router_w; rp.router_bias = layer->router_bias; rp.gate_w = layer->shared_gate_w;
   rp.logits = at<double>(ws, W.logits);
-  if (launch_route(rp, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_route(rp, s, false) != cudaSuccess) return MOE_ERR_CUDA;
   TopkParams tp{};
   tp.E = layer->n_experts; tp.k = layer->top_k; tp.T = T; tp.has_shared = layer->has_shared;
   tp.logits = rp.logits; tp.idx = topk_idx; tp.w = topk_w; tp.sg = shared_gate;
@@ -290,14 +284,9 @@ moe_status moe_stack_forward(const moe_layer* layers, int32_t L, const uint16_t*
   const int H = layers[0].hidden, k = layers[0].top_k;
   for (int l = 0; l < L; ++l) {
     const uint16_t* xin = l == 0 ? x_in : x_out;
-    if (layer_inputs && cudaMemcpyAsync(layer_inputs + (size_t)l * H, xin, sizeof(uint16_t) * H,
-                                        cudaMemcpyDeviceToDevice, s) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    if (layer_h && cudaMemcpyAsync(layer_h + (size_t)l * H, h, sizeof(float) * H, cudaMemcpyDeviceToDevice, s) !=
-                       cudaSuccess)
-      return MOE_ERR_CUDA;
     if ((st = decode_chain(&layers[l], xin, h, 1, x_out, nullptr, topk_idx_all ? topk_idx_all + (size_t)l * k : nullptr,
-                           nullptr, ws, s)))
+                           nullptr, ws, s, nullptr, layer_inputs ? layer_inputs + (size_t)l * H : nullptr,
+                           layer_h ? layer_h + (size_t)l * H : nullptr)))
       return st;
   }
   return MOE_OK;

@@ -4,14 +4,16 @@
 // a weight is code*scale + bias, applied as (q*s + b)*x). The pages fold the
 // scale and bias into the activation per element, fma(q, s*x, b*x). Here the
 // same sum is regrouped once more, per quantisation group g of G=64 elements:
-//     sum_k (q_k s + b) x_k = s * sum_k (q_k - z) x_k + (b + z s) * X_g,
-// with X_g = sum_{k in g} x_k computed once per vector and z a code offset
-// (8 for 4-bit, 2 for 2-bit). The inner sum sum_k (q_k - z) x_k runs on the
-// tensor cores: (q - z) is a small integer, exact in fp16, and x is split into
-// fp16 hi + lo parts, so an m16n8k16 MMA with fp32 accumulation computes it
-// to ~22 bits. The MMA's N=8 columns carry {group 0, group 1} x {hi, lo} of
-// one 128-element span, so each group's partial sum comes out separately and
-// its scale is applied in fp32 after the MMA.
+//     sum_k (q_k s + b) x_k = s * sum_k q_k x_k + b * X_g,
+// with X_g = sum_{k in g} x_k computed once per vector. The inner sum
+// sum_k q_k x_k runs on the integer tensor cores (m16n8k32, u8 x s8 -> s32):
+// the codes are used as unsigned bytes straight from the packed words (one
+// AND per four codes), and each activation group is held in fixed point,
+// x = X * 2^-p_g with |X| < 2^22, split exactly into three signed 8-bit
+// digits. The MMA's N=8 columns carry the digits of the two quantisation
+// groups of one 128-element span (columns 0..2 and 4..6), so each group's
+// exact integer partial sums come out separately; the group's scale and
+// 2^-p_g are applied in fp32 after the MMA.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -111,114 +113,110 @@ __device__ __forceinline__ float warp_max(float v) {
 }
 
 // ------------------------------------------------------------------ tensor-core MMA
-__device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                          uint32_t b0, uint32_t b1) {
-  asm(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+// D = A (16x32 u8, row) * B (32x8 s8, col) + C, s32 accumulate
+__device__ __forceinline__ void mma_u8s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// ------------------------------------------------------------------ code unpack (exact fp16 pairs)
-// (a & mask) | magic: places a code field in the mantissa of the fp16 1024.
-__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t magic) {
-  uint32_t r;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(mask), "r"(magic));
-  return r;
-}
-__device__ __forceinline__ uint32_t hsub2_u(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
-__device__ __forceinline__ uint32_t hfma2_u(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t r;
-  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
-  return r;
-}
-
-// One 4-bit word (codes n0..n7, n_i at bits 4i) -> 4 fp16x2 pairs of (n - 8):
-// p[0] = (n0, n4), p[1] = (n1, n5), p[2] = (n2, n6), p[3] = (n3, n7); first element in the low half.
-__device__ __forceinline__ void unpack_q4(uint32_t w, uint32_t (&p)[4]) {
-  const uint32_t kMagic = 0x64006400u;   // fp16 1024, 1024
-  const uint32_t k1032 = 0x64086408u;    // 1024 + 8
-  const uint32_t kSixteenth = 0x2C002C00u;
-  const uint32_t kMinus72 = 0xD480D480u; // -(64 + 8)
-  const uint32_t w2 = w >> 8;
-  p[0] = hsub2_u(lop3_and_or(w, 0x000F000Fu, kMagic), k1032);
-  p[1] = hfma2_u(lop3_and_or(w, 0x00F000F0u, kMagic), kSixteenth, kMinus72);
-  p[2] = hsub2_u(lop3_and_or(w2, 0x000F000Fu, kMagic), k1032);
-  p[3] = hfma2_u(lop3_and_or(w2, 0x00F000F0u, kMagic), kSixteenth, kMinus72);
-}
-// One 2-bit word (codes c0..c15, c_i at bits 2i) -> 8 fp16x2 pairs of (c - 2):
-// p[i] = (c_i, c_{i+8}) for i = 0..7.
-__device__ __forceinline__ void unpack_q2(uint32_t w, uint32_t (&p)[8]) {
-  const uint32_t kMagic = 0x64006400u;
-  const uint32_t w2 = w >> 8;
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const uint32_t v = h ? w2 : w;
-    p[4 * h + 0] = hsub2_u(lop3_and_or(v, 0x00030003u, kMagic), 0x64026402u);                  // -(1024+2)
-    p[4 * h + 1] = hfma2_u(lop3_and_or(v, 0x000C000Cu, kMagic), 0x34003400u, 0xDC08DC08u);      // /4, -(256+2)
-    p[4 * h + 2] = hfma2_u(lop3_and_or(v, 0x00300030u, kMagic), 0x2C002C00u, 0xD420D420u);      // /16, -(64+2)
-    p[4 * h + 3] = hfma2_u(lop3_and_or(v, 0x00C000C0u, kMagic), 0x24002400u, 0xCC80CC80u);      // /64, -(16+2)
-  }
+// ------------------------------------------------------------------ code bytes for the A operand
+// For MMA j (32 k-slots) a thread supplies two registers per row, each four
+// unsigned code bytes: slots 4t..4t+3 (half 0) and 16+4t..16+4t+3 (half 1).
+// 4-bit: word j of the thread's window, even nibbles (half 0) / odd (half 1).
+// 2-bit: word j>>1, crumb fields s, s+4, s+8, s+12 with s = 2(j&1) + half.
+template <int BITS>
+__device__ __forceinline__ uint32_t code_bytes(const uint32_t* w, int j, int half) {
+  if constexpr (BITS == 4) return (half ? (w[j] >> 4) : w[j]) & 0x0F0F0F0Fu;
+  else return (w[j >> 1] >> (2 * (2 * (j & 1) + half))) & 0x03030303u;
 }
 
 template <int BITS> struct QTraits;
 template <> struct QTraits<4> {
   static constexpr int kWordsPerThread = 4;  // per row per span: 32 codes
-  static constexpr float kZ = 8.f;
-  // k offset (within the thread's 32-element window) of element e of pair p
-  __host__ __device__ static constexpr int koff(int p, int e) { return 8 * (p >> 2) + (p & 3) + 4 * e; }
+  // window offset of byte i (0..3) of half h of MMA j
+  __host__ __device__ static constexpr int koff(int j, int h, int i) { return 8 * j + 2 * i + h; }
 };
 template <> struct QTraits<2> {
   static constexpr int kWordsPerThread = 2;
-  static constexpr float kZ = 2.f;
-  __host__ __device__ static constexpr int koff(int p, int e) { return 16 * (p >> 3) + (p & 7) + 8 * e; }
+  __host__ __device__ static constexpr int koff(int j, int h, int i) { return 16 * (j >> 1) + 2 * (j & 1) + h + 4 * i; }
 };
 
 // ------------------------------------------------------------------ B-fragment table
-// For one vector (one token) x' (prescaled fp32) of length K, the table holds,
-// per span s and MMA j (0..7), the two f16x2 B registers of the 8 lanes that
-// carry data. Column n = lane>>2 of the MMA is {grp = (n>>1)&1, lo = n&1} for
-// n < 4 (columns 4..7 are zero: one token). Lane (g', t) supplies the rows
-// k = s*128 + 32t + koff(2j+i, e) of column n; they are nonzero only when the
-// thread's 32-element window lies in group grp, i.e. (t>>1) == grp. Those 8
-// lanes are stored compactly at c = 2n + (t&1); every other lane reads zeros.
-constexpr int kBtabPerSpan = 8 * 8;   // MMAs x live lanes (uint2 each)
+// For one vector of length K: per quantisation group g a power of two 2^p_g
+// with X_k = rint(x_k 2^p_g), |X_k| < 2^22, split as X = d0 + 2^8 d1 + 2^16 d2
+// with signed bytes d_i. Per span s and MMA j (0..3) the table holds the two
+// B registers (4 s8 each) of the lanes that carry data: MMA column n =
+// lane>>2 is {grp = n>>2, digit = n&3 (< 3)}; lane (g', t) supplies the rows
+// k = s*128 + 32t + koff(j, h, i) of column n, nonzero only when the thread's
+// 32-element window lies in group grp, i.e. (t>>1) == grp. 12 live lanes per
+// MMA are stored compactly.
+constexpr int kDigits = 3;
+constexpr int kBtLanes = 4 * kDigits;          // live lanes per MMA
+constexpr int kBtPerSpan = 4 * kBtLanes;       // uint2 entries per span
 
-__device__ __forceinline__ int btab_lane(int lane) {
+__device__ __forceinline__ int bt_lane_index(int lane) {
   const int n = lane >> 2, t = lane & 3;
-  return (n < 4 && ((n >> 1) & 1) == (t >> 1)) ? 2 * n + (t & 1) : -1;
+  const int grp = n >> 2, d = n & 3;
+  if (d >= kDigits || grp != (t >> 1)) return -1;
+  return (grp * kDigits + d) * 2 + (t & 1);
 }
 
+// power-of-two prescale of a group with max |x| = m: m * 2^p in [2^21, 2^22)
+__device__ __forceinline__ float group_prescale(float m) {
+  if (!(m > 0.f) || !isfinite(m)) return 1.f;
+  int sh = 21 - ilogbf(m);
+  sh = sh > 120 ? 120 : (sh < -120 ? -120 : sh);
+  return ldexpf(1.f, sh);
+}
+__device__ __forceinline__ uint32_t digit_byte(float v, float sc, int d) {
+  int X = __float2int_rn(v * sc);
+  const int d0 = ((X + 128) & 255) - 128;
+  if (d == 0) return (uint32_t)d0 & 255u;
+  X = (X - d0) >> 8;
+  const int d1 = ((X + 128) & 255) - 128;
+  if (d == 1) return (uint32_t)d1 & 255u;
+  return (uint32_t)((X - d1) >> 8) & 255u;
+}
+// entry i (= s * kBtPerSpan + j * kBtLanes + c) of the table of vector xs with
+// per-group prescale gsc[g]
 template <int BITS>
-__device__ __forceinline__ uint2 btab_entry(const float* xs, int s, int j, int c) {
-  const int n = c >> 1, t = 2 * ((n >> 1) & 1) + (c & 1);
-  const int lo = n & 1;
+__device__ __forceinline__ uint2 btab_at(const float* xs, const float* gsc, int i) {
+  const int s = i / kBtPerSpan, j = (i % kBtPerSpan) / kBtLanes, c = i % kBtLanes;
+  const int gd = c >> 1, grp = gd / kDigits, d = gd % kDigits;
+  const int t = 2 * grp + (c & 1);
   const float* w = xs + s * kSpan + 32 * t;
+  const float sc = gsc[2 * s + grp];
   uint32_t r[2];
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const float v0 = w[QTraits<BITS>::koff(2 * j + i, 0)];
-    const float v1 = w[QTraits<BITS>::koff(2 * j + i, 1)];
-    r[i] = lo ? pack_half2(half_lo(v0), half_lo(v1)) : pack_half2(half_hi(v0), half_hi(v1));
+  for (int h = 0; h < 2; ++h) {
+    uint32_t v = 0;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) v |= digit_byte(w[QTraits<BITS>::koff(j, h, b)], sc, d) << (8 * b);
+    r[h] = v;
   }
   return make_uint2(r[0], r[1]);
 }
-
-// Prescale exponent so that max|x * 2^p| lies in [2^14, 2^15): keeps the fp16
-// hi part in range and the lo part meaningful. Exact (power of two).
-__device__ __forceinline__ float prescale_for(float amax) {
-  if (!(amax > 0.f) || !isfinite(amax)) return 1.f;
-  int e = ilogbf(amax);
-  int sh = 14 - e;
-  sh = sh > 100 ? 100 : (sh < -100 ? -100 : sh);
-  return ldexpf(1.f, sh);
+// Per-group prescale gsc[g], its inverse igsc[g] and sums Xg[g] of xs (one warp per group).
+__device__ __forceinline__ void group_stats(const float* xs, int ngroups, float* gsc, float* igsc, float* Xg, int warp,
+                                            int lane, int nwarps) {
+  for (int gi = warp; gi < ngroups; gi += nwarps) {
+    const float a = xs[gi * kGroup + lane], b = xs[gi * kGroup + 32 + lane];
+    float sum = a + b, m = fmaxf(fabsf(a), fabsf(b));
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    }
+    if (lane == 0) {
+      const float sc = group_prescale(m);
+      gsc[gi] = sc;
+      igsc[gi] = 1.f / sc;
+      Xg[gi] = sum;
+    }
+  }
 }
-
-
 
 // ------------------------------------------------------------------ per-warp staging with cp.async
 // Each warp stages exactly the units it will compute: every lane issues its
@@ -255,7 +253,6 @@ template <int BITS>
 struct SpanBytes { static constexpr int v = kSpan * BITS / 8; };   // code bytes of one row over one span
 template <int BITS>
 struct UnitSmem { static constexpr int bytes = 16 * SpanBytes<BITS>::v + 16 * 4 * 2; };
-constexpr int kUnitSlots = 8;   // staged units per warp in flight
 
 // The 16 source rows of one tile: row r (0..15) of codes / scales / biases.
 struct RowSrc { const uint32_t* q; const uint16_t* s; const uint16_t* b; };
@@ -329,58 +326,36 @@ __device__ __forceinline__ void frag_load(Frag<BITS>& F, const unsigned char* sl
   F.ba = sc[16 + g]; F.bb = sc[16 + g + 8];
 }
 
-// 8 MMAs over one span, two independent accumulator chains:
-// c[0..1] = row g (cols 2t, 2t+1), c[2..3] = row g+8.
+// 4 integer MMAs over one span: c[0..1] = row g (cols 2t, 2t+1), c[2..3] = row g+8.
 template <int BITS>
-__device__ __forceinline__ void mma_frag(const Frag<BITS>& F, const uint2* __restrict__ bt, int bl, float (&c)[4]) {
-  float d[4] = {0.f, 0.f, 0.f, 0.f};
-  float e[4] = {0.f, 0.f, 0.f, 0.f};
-  if constexpr (BITS == 4) {
+__device__ __forceinline__ void mma_frag(const Frag<BITS>& F, const uint2* __restrict__ bt, int bl, int (&c)[4]) {
+  c[0] = c[1] = c[2] = c[3] = 0;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      uint32_t pa[4], pb[4];
-      unpack_q4(F.wa[u], pa);
-      unpack_q4(F.wb[u], pb);
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int j = 2 * u + h;
-        const uint2 b = bl >= 0 ? bt[j * 8 + bl] : make_uint2(0u, 0u);
-        if (h == 0) mma_16816(d, pa[0], pb[0], pa[1], pb[1], b.x, b.y);
-        else mma_16816(e, pa[2], pb[2], pa[3], pb[3], b.x, b.y);
-      }
-    }
-  } else {
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      uint32_t pa[8], pb[8];
-      unpack_q2(F.wa[u], pa);
-      unpack_q2(F.wb[u], pb);
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        const int j = 4 * u + h;
-        const uint2 b = bl >= 0 ? bt[j * 8 + bl] : make_uint2(0u, 0u);
-        if (h & 1) mma_16816(e, pa[2 * h], pb[2 * h], pa[2 * h + 1], pb[2 * h + 1], b.x, b.y);
-        else mma_16816(d, pa[2 * h], pb[2 * h], pa[2 * h + 1], pb[2 * h + 1], b.x, b.y);
-      }
-    }
+  for (int j = 0; j < 4; ++j) {
+    const uint2 b = bl >= 0 ? bt[j * kBtLanes + bl] : make_uint2(0u, 0u);
+    mma_u8s8(c, code_bytes<BITS>(F.wa, j, 0), code_bytes<BITS>(F.wb, j, 0), code_bytes<BITS>(F.wa, j, 1),
+             code_bytes<BITS>(F.wb, j, 1), b.x, b.y);
   }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) c[i] = d[i] + e[i];
 }
 
-// Applies the group scales: thread t (< 2) owns group 2*span + t (hi + lo columns).
-template <int BITS>
-__device__ __forceinline__ void scale_frag(const Frag<BITS>& F, const float (&c)[4], const float* Xg, int span, int t,
-                                           float& acc_a, float& acc_b) {
-  if (t < 2) {
-    const float xg = Xg[2 * span + t];
-    const float s_a = t ? bf16hi(F.sa) : bf16lo(F.sa);
-    const float s_b = t ? bf16hi(F.sb) : bf16lo(F.sb);
-    const float b_a = t ? bf16hi(F.ba) : bf16lo(F.ba);
-    const float b_b = t ? bf16hi(F.bb) : bf16lo(F.bb);
-    acc_a = fmaf(s_a, c[0] + c[1], fmaf(fmaf(QTraits<BITS>::kZ, s_a, b_a), xg, acc_a));
-    acc_b = fmaf(s_b, c[2] + c[3], fmaf(fmaf(QTraits<BITS>::kZ, s_b, b_b), xg, acc_b));
-  }
+// Applies the group scales. Thread t holds columns 2t, 2t+1: digits of group
+// grp = t>>1 (t even: d0, d1; t odd: d2), so each thread scales its own part;
+// the even thread adds the bias term b * X_g. The four threads of a quad are
+// summed when the tile is flushed.
+__device__ __forceinline__ void scale_frag_i(uint32_t sa, uint32_t sb, uint32_t ba, uint32_t bb, const int (&c)[4],
+                                             const float* igsc, const float* Xg, int span, int t, float& acc_a,
+                                             float& acc_b) {
+  const int grp = t >> 1, gi = 2 * span + grp;
+  const bool odd = t & 1;
+  const float fa = odd ? 65536.f * (float)c[0] : fmaf(256.f, (float)c[1], (float)c[0]);
+  const float fb = odd ? 65536.f * (float)c[2] : fmaf(256.f, (float)c[3], (float)c[2]);
+  const float ip = igsc[gi], xg = odd ? 0.f : Xg[gi];
+  const float s_a = grp ? bf16hi(sa) : bf16lo(sa);
+  const float s_b = grp ? bf16hi(sb) : bf16lo(sb);
+  const float b_a = grp ? bf16hi(ba) : bf16lo(ba);
+  const float b_b = grp ? bf16hi(bb) : bf16lo(bb);
+  acc_a = fmaf(s_a * ip, fa, fmaf(b_a, xg, acc_a));
+  acc_b = fmaf(s_b * ip, fb, fmaf(b_b, xg, acc_b));
 }
 
 // ------------------------------------------------------------------ split-unit schedule
@@ -404,53 +379,95 @@ struct PartialSmem {
   int tile[kWarps][2];
 };
 
-// Unit loop of one warp: stages up to kUnitSlots units at a time with
-// cp.async, then MMAs them in order as they land. Partials go to `ps`.
-// (tile, span) of consecutive units are tracked incrementally; the lanes'
-// copy sources are recomputed only when the tile changes.
-template <int BITS, class RowFn, class BtFn, class XgFn>
-__device__ __forceinline__ void run_units(Range wr, int nspans, unsigned char* wslots, RowFn row, BtFn bt_of,
-                                          XgFn xg_of, PartialSmem& ps, int warp, int lane) {
+// Rolling per-warp pipeline over the units of a warp range. The range meets
+// at most two tiles (host guarantee); the units of each tile form a
+// sub-range, and a pass selects which sub-ranges it runs (e.g. the shared
+// expert's before the routing is known, the routed ones after). Up to NS
+// units (a template argument) are in flight (cp.async, one commit group per
+// unit); the oldest is computed when it lands and its slot is refilled.
+struct SubRange { int tile, s0, s1, si; };
+
+template <int BITS>
+struct WarpPipe {
+  SubRange sr[2];
+  int n;              // sub-ranges of this pass
+  int is, ispan;      // next unit to issue: sub-range index, span
+  int cs, cspan;      // next unit to compute
+  int issued, computed;
+  LaneCopy<BITS> lc;
+  int lc_tile;
+};
+
+// Sub-ranges of the warp range wr (tile = u / nspans) whose tile satisfies `take`.
+template <int BITS, class TakeFn>
+__device__ __forceinline__ void pipe_init(WarpPipe<BITS>& P, Range wr, int nspans, TakeFn take) {
+  P.n = 0;
+  P.is = P.cs = 0;
+  P.issued = P.computed = 0;
+  P.lc_tile = -1;
+  if (wr.a >= wr.b) return;
+  const int t0 = wr.a / nspans, t1 = (wr.b - 1) / nspans;
+  for (int tile = t0; tile <= t1; ++tile) {
+    const int lo = wr.a > tile * nspans ? wr.a - tile * nspans : 0;
+    const int hi = wr.b < (tile + 1) * nspans ? wr.b - tile * nspans : nspans;
+    if (take(tile)) P.sr[P.n++] = SubRange{tile, lo, hi, tile - t0};
+  }
+  if (P.n) { P.ispan = P.sr[0].s0; P.cspan = P.sr[0].s0; }
+}
+
+// Issues units until NS (<= 8) are in flight or the pass is exhausted.
+template <int BITS, int NS, class RowFn>
+__device__ __forceinline__ void pipe_issue(WarpPipe<BITS>& P, unsigned char* wslots, RowFn row, int lane) {
+  static_assert(NS >= 1 && NS <= 8, "slots per warp");
+  while (P.is < P.n && P.issued - P.computed < NS) {
+    const SubRange& r = P.sr[P.is];
+    if (P.lc_tile != r.tile) { P.lc = lane_copy<BITS>(row, r.tile, lane); P.lc_tile = r.tile; }
+    stage_unit<BITS>(wslots + (P.issued % NS) * UnitSmem<BITS>::bytes, P.lc, P.ispan);
+    cp_async_commit();
+    ++P.issued;
+    if (++P.ispan == r.s1 && ++P.is < P.n) P.ispan = P.sr[P.is].s0;
+  }
+}
+
+// Computes every unit of the pass (issuing more as slots free up); partials of
+// each sub-range go to ps.v[warp][si] / ps.tile[warp][si].
+// bt_of(tile) gives the B table of the tile's vector, gs_of(tile) a pointer
+// G with G[g] = 2^-p_g and G[gstride + g] = X_g for that vector.
+template <int BITS, int NS, class RowFn, class BtFn, class GsFn>
+__device__ __forceinline__ void pipe_run(WarpPipe<BITS>& P, unsigned char* wslots, RowFn row, BtFn bt_of, GsFn gs_of,
+                                         int gstride, PartialSmem& ps, int warp, int lane) {
   const int g = lane >> 2, t = lane & 3;
-  const int bl = btab_lane(lane);
+  const int bl = bt_lane_index(lane);
+  float acc_a = 0.f, acc_b = 0.f;
+  while (P.cs < P.n) {
+    pipe_issue<BITS, NS>(P, wslots, row, lane);
+    const SubRange& r = P.sr[P.cs];
+    cp_async_wait_dyn(P.issued - P.computed - 1);
+    __syncwarp();
+    Frag<BITS> F;
+    frag_load<BITS>(F, wslots + (P.computed % NS) * UnitSmem<BITS>::bytes, g, t);
+    int c[4];
+    mma_frag<BITS>(F, bt_of(r.tile) + P.cspan * kBtPerSpan, bl, c);
+    const float* G = gs_of(r.tile);
+    scale_frag_i(F.sa, F.sb, F.ba, F.bb, c, G, G + gstride, P.cspan, t, acc_a, acc_b);
+    __syncwarp();   // every lane has read the slot before it is refilled
+    ++P.computed;
+    if (++P.cspan == r.s1) {
+      acc_a += __shfl_xor_sync(0xffffffffu, acc_a, 1);
+      acc_b += __shfl_xor_sync(0xffffffffu, acc_b, 1);
+      acc_a += __shfl_xor_sync(0xffffffffu, acc_a, 2);
+      acc_b += __shfl_xor_sync(0xffffffffu, acc_b, 2);
+      if (t == 0) { ps.v[warp][r.si][g] = acc_a; ps.v[warp][r.si][g + 8] = acc_b; }
+      if (lane == 0) ps.tile[warp][r.si] = r.tile;
+      acc_a = acc_b = 0.f;
+      if (++P.cs < P.n) P.cspan = P.sr[P.cs].s0;
+    }
+  }
+}
+
+__device__ __forceinline__ void partials_clear(PartialSmem& ps, int warp, int lane) {
   if (lane == 0) { ps.tile[warp][0] = -1; ps.tile[warp][1] = -1; }
   __syncwarp();
-  if (wr.a >= wr.b) return;
-  int si = 0;
-  float acc_a = 0.f, acc_b = 0.f;
-  int tile_s = wr.a / nspans, span_s = wr.a - tile_s * nspans;   // staging cursor
-  int tile_c = tile_s, span_c = span_s;                           // compute cursor
-  LaneCopy<BITS> lc = lane_copy<BITS>(row, tile_s, lane);
-  const uint2* bt = bt_of(tile_c);
-  const float* xg = xg_of(tile_c);
-  for (int u0 = wr.a; u0 < wr.b; u0 += kUnitSlots) {
-    const int n = wr.b - u0 < kUnitSlots ? wr.b - u0 : kUnitSlots;
-    for (int i = 0; i < n; ++i) {
-      stage_unit<BITS>(wslots + i * UnitSmem<BITS>::bytes, lc, span_s);
-      cp_async_commit();
-      if (++span_s == nspans && u0 + i + 1 < wr.b) { span_s = 0; ++tile_s; lc = lane_copy<BITS>(row, tile_s, lane); }
-    }
-    for (int i = 0; i < n; ++i) {
-      cp_async_wait_dyn(n - 1 - i);
-      __syncwarp();
-      Frag<BITS> F;
-      frag_load<BITS>(F, wslots + i * UnitSmem<BITS>::bytes, g, t);
-      float c[4];
-      mma_frag<BITS>(F, bt + span_c * kBtabPerSpan, bl, c);
-      scale_frag<BITS>(F, c, xg, span_c, t, acc_a, acc_b);
-      const bool last = u0 + i + 1 >= wr.b;
-      if (++span_c == nspans || last) {
-        acc_a += __shfl_xor_sync(0xffffffffu, acc_a, 1);
-        acc_b += __shfl_xor_sync(0xffffffffu, acc_b, 1);
-        if (t == 0) { ps.v[warp][si][g] = acc_a; ps.v[warp][si][g + 8] = acc_b; }
-        if (lane == 0) ps.tile[warp][si] = tile_c;
-        si++;
-        acc_a = acc_b = 0.f;
-        if (!last) { span_c = 0; ++tile_c; bt = bt_of(tile_c); xg = xg_of(tile_c); }
-      }
-    }
-    __syncwarp();
-  }
 }
 
 // After __syncthreads: sums the partials of every tile the CTA met, in warp

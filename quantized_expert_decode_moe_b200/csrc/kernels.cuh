@@ -12,12 +12,8 @@ namespace qmoe {
 struct WsLayout {
   size_t status;      // uint32 status word (+ padding)
   size_t logits;      // double [T][E+1]; column E = shared-gate logit
-  size_t gu;          // float [T][S][2][I]  gate/up pre-activations
-  size_t y;           // float [T][S][H]     expert outputs (unweighted)
-  size_t w;           // float [T][k]        routing weights
-  size_t sg;          // float [T]           shared gate
-  size_t idx;         // int32 [T][k]        routed expert ids
-  size_t slots;       // moe_expert [T][9]   chosen experts of each token
+  size_t a;           // float [T][S][I]  silu(gate) * up of each slot (slot S-1 = shared expert)
+  size_t hacc;        // float [T][H]     h + weighted expert outputs
   // prefill
   size_t counts;      // int32 [E]
   size_t offsets;     // int32 [E+1]
@@ -33,9 +29,8 @@ struct RouteParams {
   const float* router_bias;     // [E] or null
   const uint16_t* gate_w;       // [H] or null
   double* logits;               // [T][E+1]
-  // side jobs of the decode chain (null when unused)
-  float* zero_buf; size_t zero_n;   // accumulators cleared for the next kernels
-  moe_expert shared; int I, bits; int prefetch_shared;
+  // side job of the decode chain (null when unused): copies of the layer's inputs x, h ([T][H])
+  const float* h; uint16_t* x_rec; float* h_rec;
 };
 
 struct TopkParams {
@@ -45,34 +40,33 @@ struct TopkParams {
 };
 
 struct GateUpParams {
-  int H, I, E, k, S, has_shared, nspans, ntiles, nCTA;
-  long long U;
+  int H, I, E, k, S, has_shared, nCTA;
   const uint16_t* x;           // [T][H]
   const double* logits;        // [T][E+1]
   const moe_expert* experts;   // device [E]
   moe_expert shared;
-  float* gu;                   // [T][S][2][I]
-  int32_t* idx_ws; float* w_ws; float* sg_ws;   // [T][k], [T][k], [T]
-  moe_expert* slots_ws;                         // [T][kMaxSlots] chosen experts (routed, then shared)
-  int32_t* idx_out; float* w_out;               // user copies, nullable
+  float* a;                    // [T][S][I]
+  int32_t* idx_out; float* w_out;   // user copies of the routing, nullable
   uint32_t* status;
-  int prefetch_down, prefetch_self;
-  size_t stage_bytes;          // set by the launcher
   unsigned long long wait_ns;  // bound of every device-side wait
 };
 
 struct DownParams {
-  int H, I, E, k, S, has_shared, nspans, ntiles, nCTA;
-  long long U;
-  const float* gu;             // [T][S][2][I]
-  const int32_t* idx_ws;       // [T][k]
-  const moe_expert* slots_ws;  // [T][kMaxSlots]
+  int H, I, E, k, S, has_shared, nCTA;
+  const double* logits;        // [T][E+1]
+  const float* a;              // [T][S][I]
+  const float* h;              // [T][H] residual
   const moe_expert* experts;
   moe_expert shared;
-  float* y;                    // [T][S][H]
+  float* hacc;                 // [T][H]
   uint32_t* status;
-  size_t stage_bytes;
   unsigned long long wait_ns;
+};
+
+struct NormDecodeParams {
+  int H, T;
+  const float* hacc; float* h; const uint16_t* gamma; float eps;
+  uint16_t* x_out; float* x_out_f32;
 };
 
 struct NormParams {
@@ -101,11 +95,16 @@ struct GroupParams {
 };
 
 // launchers (return the launch's cudaError_t)
-cudaError_t launch_route(const RouteParams& p, cudaStream_t s);
+cudaError_t launch_route(const RouteParams& p, cudaStream_t s, bool pdl);
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t s);
 cudaError_t launch_gateup(const GateUpParams& p, int bits, int T, bool pdl, cudaStream_t s);
 cudaError_t launch_down(const DownParams& p, int bits, int T, bool pdl, cudaStream_t s);
 cudaError_t launch_norm(const NormParams& p, bool pdl, cudaStream_t s);
+cudaError_t launch_norm_decode(const NormDecodeParams& p, bool pdl, cudaStream_t s);
+size_t gateup_smem_bytes(int H, int bits);
+size_t down_smem_bytes(int I, int S, int bits);
+int gateup_ctas(int I);
+int down_ctas(int H);
 cudaError_t launch_gemv(const GemvParams& p, int bits, cudaStream_t s);
 cudaError_t launch_group(const GroupParams& p, cudaStream_t s);
 int num_sms();

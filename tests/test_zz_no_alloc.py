@@ -68,12 +68,16 @@ def test_noalloc_forward_matches_workspace_forward(name, T):
             assert rel_err(got["xf"][i], ref["xf"][i]) <= TOL
 
 
-def test_noalloc_rejects_oversized_workspace():
+def test_noalloc_scratch_covers_largest_decode_shape():
+    """The largest layer the decode chain accepts (hidden = inter = 8192, 4096
+    experts, top-8 + shared, 8 tokens) fits the static scratch, so the
+    oversize rejection cannot trigger for a valid call; more than 8 tokens is
+    refused as unsupported before the scratch is touched."""
     L = qm.lib()
     p = 0x100000
     ex = qm._Expert(*[qm._QMat(p, p, p) for _ in range(3)])
     big = qm._Layer(8192, 8192, 4096, 8, 4, 64, 1, 1e-6, p, None, p, ex, p, p)
     n = C.c_size_t(0)
-    assert L.moe_workspace_size(C.byref(big), 8, C.byref(n)) == 0 and n.value > (4 << 20)
+    assert L.moe_workspace_size(C.byref(big), 8, C.byref(n)) == 0 and 0 < n.value <= (4 << 20)
     pp = C.c_void_p(0x200000)
-    assert L.moe_layer_forward_noalloc(C.byref(big), pp, pp, 8, pp, None, None, None, None) == 3   # MOE_ERR_WORKSPACE
+    assert L.moe_layer_forward_noalloc(C.byref(big), pp, pp, 9, pp, None, None, None, None) == 2   # MOE_ERR_UNSUPPORTED
