@@ -218,6 +218,79 @@ __device__ __forceinline__ void group_stats(const float* xs, int ngroups, float*
   }
 }
 
+// ------------------------------------------------------------------ B tables from registers
+// The table builder's thread holds the EPT consecutive elements that feed its
+// own B entries: 8 (4-bit: MMA j of window t takes elements 8j..8j+7) or 16
+// (2-bit: MMAs 2jj, 2jj+1 take elements 16jj..16jj+15).
+template <int BITS> struct TabTraits { static constexpr int kEPT = BITS == 4 ? 8 : 16; };
+
+// Exponent sh of the power-of-two prescale of a group with max |x| = m:
+// m * 2^sh in [2^21, 2^22) for normal m; 0 for zero or non-finite m;
+// clamped to [-120, 120].
+__device__ __forceinline__ int prescale_shift(float m) {
+  const int eb = (int)((__float_as_uint(m) >> 23) & 0xFFu);
+  if (eb == 0xFF || !(m > 0.f)) return 0;
+  const int sh = 148 - eb;
+  return sh > 120 ? 120 : (sh < -120 ? -120 : sh);
+}
+// signed-digit byte d (0..2) of X = d0 + 2^8 d1 + 2^16 d2, |X| <= 2^22
+__device__ __forceinline__ uint32_t sdigit(int X, int d) {
+  if (d > 0) X = (X - (int)(signed char)(X & 0xFF)) >> 8;
+  if (d > 1) X = (X - (int)(signed char)(X & 0xFF)) >> 8;
+  return (uint32_t)X & 0xFFu;
+}
+template <int EPT>
+__device__ __forceinline__ uint32_t pack_digits(const int (&X)[EPT], int o, int st, int d) {
+  return sdigit(X[o], d) | (sdigit(X[o + st], d) << 8) | (sdigit(X[o + 2 * st], d) << 16) |
+         (sdigit(X[o + 3 * st], d) << 24);
+}
+
+// v = elements e0 .. e0+EPT-1 of a vector (e0 a multiple of EPT). The
+// 64/EPT threads of a quantisation group are consecutive lanes, and all 32
+// lanes of the warp call together (valid = false: no elements, v ignored).
+// Writes the thread's B entries into bt (the vector's table) and, from the
+// group's first thread, gs[g] = 2^-p_g and gs[ng + g] = X_g (the group sum).
+template <int BITS>
+__device__ __forceinline__ void build_tables(const float (&v)[TabTraits<BITS>::kEPT], int e0, bool valid, uint2* bt,
+                                             float* gs, int ng) {
+  constexpr int EPT = TabTraits<BITS>::kEPT, TPG = kGroup / EPT;
+  float m = 0.f, sum = 0.f;
+#pragma unroll
+  for (int i = 0; i < EPT; ++i) { m = fmaxf(m, fabsf(v[i])); sum += v[i]; }
+#pragma unroll
+  for (int o = 1; o < TPG; o <<= 1) {
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  }
+  if (!valid) return;
+  const int sh = prescale_shift(m);
+  const float sc = __uint_as_float((uint32_t)(127 + sh) << 23);
+  int X[EPT];
+#pragma unroll
+  for (int i = 0; i < EPT; ++i) X[i] = __float2int_rn(v[i] * sc);
+  const int s = e0 / kSpan, w = e0 % kSpan, t = w / 32, grp = t >> 1;
+  const int c0 = grp * kDigits * 2 + (t & 1);   // entry of digit d: c0 + 2d
+  if constexpr (BITS == 4) {
+    uint2* e = bt + s * kBtPerSpan + ((w % 32) / 8) * kBtLanes + c0;
+#pragma unroll
+    for (int d = 0; d < kDigits; ++d) e[2 * d] = make_uint2(pack_digits(X, 0, 2, d), pack_digits(X, 1, 2, d));
+  } else {
+    const int jj = (w % 32) / 16;
+#pragma unroll
+    for (int jl = 0; jl < 2; ++jl) {
+      uint2* e = bt + s * kBtPerSpan + (2 * jj + jl) * kBtLanes + c0;
+#pragma unroll
+      for (int d = 0; d < kDigits; ++d)
+        e[2 * d] = make_uint2(pack_digits(X, 2 * jl, 4, d), pack_digits(X, 2 * jl + 1, 4, d));
+    }
+  }
+  if (e0 % kGroup == 0) {
+    const int g = e0 / kGroup;
+    gs[g] = __uint_as_float((uint32_t)(127 - sh) << 23);
+    gs[ng + g] = sum;
+  }
+}
+
 // ------------------------------------------------------------------ per-warp staging with cp.async
 // Each warp stages exactly the units it will compute: every lane issues its
 // own 16-byte asynchronous copies (codes) and 4-byte copies (the span's

@@ -90,13 +90,37 @@ __device__ __forceinline__ void frag_codes(Frag<BITS>& F, const unsigned char* r
   }
 }
 
+// Loads the table builder's elements of chunk q of a bf16 vector.
+template <int BITS>
+__device__ __forceinline__ void load_chunk_bf16(const uint16_t* x, int q, float (&v)[TabTraits<BITS>::kEPT]) {
+  constexpr int EPT = TabTraits<BITS>::kEPT;
+  const uint4* p = (const uint4*)(x + (size_t)q * EPT);
+#pragma unroll
+  for (int u = 0; u < EPT / 8; ++u) {
+    const uint4 r = __ldcg(p + u);
+    const uint32_t w4[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) { v[8 * u + 2 * i] = bf16lo(w4[i]); v[8 * u + 2 * i + 1] = bf16hi(w4[i]); }
+  }
+}
+template <int BITS>
+__device__ __forceinline__ void load_chunk_f32(const float* a, int q, float (&v)[TabTraits<BITS>::kEPT]) {
+  constexpr int EPT = TabTraits<BITS>::kEPT;
+  const float4* p = (const float4*)(a + (size_t)q * EPT);
+#pragma unroll
+  for (int u = 0; u < EPT / 4; ++u) {
+    const float4 r = __ldcg(p + u);
+    v[4 * u] = r.x; v[4 * u + 1] = r.y; v[4 * u + 2] = r.z; v[4 * u + 3] = r.w;
+  }
+}
+
 // ------------------------------------------------------------------ gate/up + SwiGLU
-constexpr int kGuBufs = 2;      // expert tiles in flight per CTA
+constexpr int kGuBufs = 3;      // expert tiles staged per CTA (the shared expert's buffer is reused)
 constexpr int kGuMaxRows = 8;   // intermediate rows per CTA
 
 struct GuLayout {
   int RB, SRB, SBR, GB;   // code bytes per row, scale bytes per row, scale region, buffer bytes
-  size_t buf, btab, gsc, gs, part, slots, topk, bars, total;
+  size_t buf, btab, gs, part, slots, topk, bars, total;
 };
 __host__ __device__ inline GuLayout gu_layout(int H, int bits) {
   GuLayout L;
@@ -107,10 +131,9 @@ __host__ __device__ inline GuLayout gu_layout(int H, int bits) {
   size_t o = 0;
   L.buf = o; o += (size_t)kGuBufs * L.GB;
   L.btab = o; o += sizeof(uint2) * (size_t)(H / kSpan) * kBtPerSpan;
-  L.gsc = o; o += sizeof(float) * (size_t)(H / kGroup);
   L.gs = o; o += sizeof(float) * 2 * (size_t)(H / kGroup);   // [2^-p_g | X_g]
   o = (o + 15) & ~(size_t)15;
-  L.part = o; o += sizeof(float) * 2 * kWarps * 16;
+  L.part = o; o += sizeof(float) * kWarps * 16;
   L.slots = o; o += sizeof(moe_expert) * kMaxSlots;
   o = (o + 15) & ~(size_t)15;
   L.topk = o; o += sizeof(TopkSmem);
@@ -122,15 +145,16 @@ __host__ __device__ inline GuLayout gu_layout(int H, int bits) {
 
 // grid (nCTA, T), block 512. Items: the shared expert first (its copies and
 // MMAs run before the dependency wait: this kernel starts only after every
-// router CTA has passed its own wait, so x is final), then the k routed
-// experts, which every CTA ranks itself from the router's logits.
+// router CTA has passed its own wait, so x is final; its a values are stored
+// and fenced before this kernel lets the down kernel launch), then the k
+// routed experts, which every CTA ranks itself from the router's logits and
+// computes side by side, each on its own group of warps.
 template <int BITS>
 __global__ void __launch_bounds__(kThreads, 2) gateup_decode_kernel(GateUpParams p) {
   extern __shared__ __align__(128) unsigned char smem[];
   const GuLayout L = gu_layout(p.H, BITS);
   unsigned char* bufs = smem + L.buf;
   uint2* btab = (uint2*)(smem + L.btab);
-  float* gsc = (float*)(smem + L.gsc);
   float* gs = (float*)(smem + L.gs);
   float* part = (float*)(smem + L.part);
   moe_expert* slot_ex = (moe_expert*)(smem + L.slots);
@@ -149,42 +173,37 @@ __global__ void __launch_bounds__(kThreads, 2) gateup_decode_kernel(GateUpParams
   const unsigned item_bytes = 2u * n * L.RB + 4u * sbw;
   bool ok = true;
 
-  // the byte count of item `it` on its buffer's barrier (thread 0, before the
-  // barrier that precedes the copies; the buffer's previous phase has completed)
-  auto arm = [&](int it) {
-    if (tid == 0 && n) mbar_expect_tx(&bars[it % kGuBufs], item_bytes);
+  auto arm = [&](int it) {   // thread 0, before the barrier that precedes the item's copies
+    if (tid == 0) mbar_expect_tx(&bars[it % kGuBufs], item_bytes);
   };
-  // copies of item `it` into buffer it % kGuBufs: lane 0 of warps 0-5, one copy each
-  auto issue = [&](int it) {
-    if (lane != 0 || warp >= 6 || n == 0) return;
+  // copies of item `it` into buffer it % kGuBufs: one copy per thread listed below
+  auto issue = [&](int it, int c) {   // c = copy 0..5: gate codes, up codes, gate/up scales, gate/up biases
     const int b = it % kGuBufs;
     unsigned char* buf = bufs + (size_t)b * L.GB;
     const moe_expert& ex = slot_ex[item_slot(it)];
     fence_proxy_async();
-    if (warp < 2) {
-      const moe_qmat& m = warp == 0 ? ex.gate : ex.up;
-      bulk_g2s(buf + (size_t)warp * kGuMaxRows * L.RB, (const char*)m.q + (size_t)j0 * L.RB, (unsigned)n * L.RB,
-               &bars[b]);
+    if (c < 2) {
+      const moe_qmat& m = c == 0 ? ex.gate : ex.up;
+      bulk_g2s(buf + (size_t)c * kGuMaxRows * L.RB, (const char*)m.q + (size_t)j0 * L.RB, (unsigned)n * L.RB, &bars[b]);
     } else {
-      const int w = warp - 2;   // 0 gate scales, 1 up scales, 2 gate biases, 3 up biases
+      const int w = c - 2;   // 0 gate scales, 1 up scales, 2 gate biases, 3 up biases
       const moe_qmat& m = (w & 1) ? ex.up : ex.gate;
       const uint16_t* src = w < 2 ? m.scales : m.biases;
-      bulk_g2s(buf + 2 * kGuMaxRows * L.RB + w * L.SBR, (const char*)src + (((size_t)j0 * L.SRB) & ~(size_t)15),
-               sbw, &bars[b]);
+      bulk_g2s(buf + 2 * kGuMaxRows * L.RB + w * L.SBR, (const char*)src + (((size_t)j0 * L.SRB) & ~(size_t)15), sbw,
+               &bars[b]);
     }
   };
-  // MMAs of one item: warp w takes spans [nspans*w/16, nspans*(w+1)/16); row sums to pt[w][16]
-  auto compute = [&](int b, float* pt) {
+  // MMAs of spans [s0, s1) of the item in buffer b; row sums of rows g, g+8 returned in acc_a, acc_b (quad-reduced)
+  auto compute = [&](int b, int s0, int s1, float& acc_a, float& acc_b) {
     const unsigned char* buf = bufs + (size_t)b * L.GB;
     const int g = lane >> 2, tq = lane & 3;
     const int bl = bt_lane_index(lane);
-    const int s0 = nspans * warp / kWarps, s1 = nspans * (warp + 1) / kWarps;
     constexpr int SB = SpanBytes<BITS>::v;
     constexpr int WB = QTraits<BITS>::kWordsPerThread * 4;
     const unsigned char* ra = buf + (size_t)g * L.RB + tq * WB;
     const unsigned char* rb = buf + (size_t)(kGuMaxRows + g) * L.RB + tq * WB;
     const unsigned char* sc = buf + 2 * kGuMaxRows * L.RB + pre + g * L.SRB;
-    float acc_a = 0.f, acc_b = 0.f;
+    acc_a = 0.f; acc_b = 0.f;
     for (int s = s0; s < s1; ++s) {
       Frag<BITS> F;
       frag_codes<BITS>(F, ra + s * SB, rb + s * SB);
@@ -200,14 +219,9 @@ __global__ void __launch_bounds__(kThreads, 2) gateup_decode_kernel(GateUpParams
     acc_b += __shfl_xor_sync(0xffffffffu, acc_b, 1);
     acc_a += __shfl_xor_sync(0xffffffffu, acc_a, 2);
     acc_b += __shfl_xor_sync(0xffffffffu, acc_b, 2);
-    if (tq == 0) { pt[warp * 16 + g] = acc_a; pt[warp * 16 + 8 + g] = acc_b; }
   };
-  auto finalize = [&](int it, const float* pt) {
-    if (tid < n) {
-      float gsum = 0.f, usum = 0.f;
-      for (int w = 0; w < kWarps; ++w) { gsum += pt[w * 16 + tid]; usum += pt[w * 16 + 8 + tid]; }
-      p.a[((size_t)t * S + item_slot(it)) * I + j0 + tid] = silu_f32(gsum) * usum;
-    }
+  auto store_a = [&](int it, int i, float gsum, float usum) {
+    p.a[((size_t)t * S + item_slot(it)) * I + j0 + i] = silu_f32(gsum) * usum;
   };
 
   if (tid == 0) {
@@ -217,30 +231,33 @@ __global__ void __launch_bounds__(kThreads, 2) gateup_decode_kernel(GateUpParams
   }
   if (p.has_shared) arm(0);
   __syncthreads();
-  if (p.has_shared) issue(0);
-  // activation -> fp32 (exact; staged in buffer 1, free until the routed copies), group prescales and sums,
-  // B-fragment table
-  float* xs = (float*)(bufs + (size_t)1 * L.GB);
-  const uint4* xt = (const uint4*)(p.x + (size_t)t * H);
-  for (int i = tid; i < H / 8; i += kThreads) {
-    const uint4 v = __ldcg(xt + i);
-    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) { xs[8 * i + 2 * q] = bf16lo(w4[q]); xs[8 * i + 2 * q + 1] = bf16hi(w4[q]); }
+  if (p.has_shared && warp < 6 && lane == 0) issue(0, warp);
+  // B tables of x, straight from registers
+  {
+    constexpr int EPT = TabTraits<BITS>::kEPT;
+    const int nq = H / EPT;
+    for (int q0 = 0; q0 < nq; q0 += kThreads) {
+      const int q = q0 + tid;
+      float v[EPT];
+      if (q < nq) load_chunk_bf16<BITS>(p.x + (size_t)t * H, q, v);
+      build_tables<BITS>(v, q * EPT, q < nq, btab, gs, ng);
+    }
   }
   __syncthreads();
-  group_stats(xs, ng, gsc, gs, gs + ng, warp, lane, kWarps);
-  __syncthreads();
-  for (int i = tid; i < nspans * kBtPerSpan; i += kThreads) btab[i] = btab_at<BITS>(xs, gsc, i);
-  fence_proxy_async();   // buffer 1 (x staging) is refilled by bulk copies later
-  __syncthreads();
   int it0 = 0;
-  if (p.has_shared) {
-    if (n) ok &= mbar_wait_bounded(&bars[0], 0, p.wait_ns, p.status);
-    compute(0, part);
+  if (p.has_shared) {   // all warps: spans [nspans*w/16, nspans*(w+1)/16)
+    ok &= mbar_wait_bounded(&bars[0], 0, p.wait_ns, p.status);
+    float aa, ab;
+    compute(0, nspans * warp / kWarps, nspans * (warp + 1) / kWarps, aa, ab);
+    if ((lane & 3) == 0) { part[warp * 16 + (lane >> 2)] = aa; part[warp * 16 + 8 + (lane >> 2)] = ab; }
     fence_proxy_async();
     __syncthreads();
-    finalize(0, part);
+    if (tid < n) {
+      float gsum = 0.f, usum = 0.f;
+      for (int w = 0; w < kWarps; ++w) { gsum += part[w * 16 + tid]; usum += part[w * 16 + 8 + tid]; }
+      store_a(0, tid, gsum, usum);
+    }
+    __threadfence();   // the down kernel reads the shared expert's a before its own dependency wait
     it0 = 1;
   }
 
@@ -253,23 +270,35 @@ __global__ void __launch_bounds__(kThreads, 2) gateup_decode_kernel(GateUpParams
     if (p.idx_out) p.idx_out[(size_t)t * k + tid] = ts.idx[tid];
     if (p.w_out) p.w_out[(size_t)t * k + tid] = ts.w[tid];
   }
-  for (int it = it0; it < nitems && it < it0 + kGuBufs; ++it) arm(it);
-  __syncthreads();
-  for (int it = it0; it < nitems && it < it0 + kGuBufs; ++it) issue(it);
-  for (int it = it0; it < nitems; ++it) {
-    const int b = it % kGuBufs;
-    float* pt = part + (it & 1) * kWarps * 16;
-    if (n) ok &= mbar_wait_bounded(&bars[b], (unsigned)(it / kGuBufs) & 1u, p.wait_ns, p.status);
-    compute(b, pt);
+  // routed items in waves of up to kGuBufs, each item on its own group of warps
+  for (int w0 = it0; w0 < nitems; w0 += kGuBufs) {
+    const int nw = nitems - w0 < kGuBufs ? nitems - w0 : kGuBufs;
+    for (int i = 0; i < nw; ++i) arm(w0 + i);
+    __syncthreads();   // slots loaded (first wave) / previous wave's buffers read
+    if (lane == 0)
+      for (int c = warp; c < 6 * nw; c += kWarps) issue(w0 + c / 6, c % 6);
+    const int wi = warp * nw / kWarps;                       // this warp's item in the wave
+    const int wf = (wi * kWarps + nw - 1) / nw;               // first warp of that item
+    const int wc = ((wi + 1) * kWarps + nw - 1) / nw - wf;    // warps of that item
+    const int it = w0 + wi, r = warp - wf;
+    ok &= mbar_wait_bounded(&bars[it % kGuBufs], (unsigned)(it / kGuBufs) & 1u, p.wait_ns, p.status);
+    float aa, ab;
+    compute(it % kGuBufs, nspans * r / wc, nspans * (r + 1) / wc, aa, ab);
+    __syncthreads();   // part of the previous wave is consumed
+    if ((lane & 3) == 0) { part[warp * 16 + (lane >> 2)] = aa; part[warp * 16 + 8 + (lane >> 2)] = ab; }
     fence_proxy_async();
-    if (it + kGuBufs < nitems) arm(it + kGuBufs);
     __syncthreads();
-    if (it + kGuBufs < nitems) issue(it + kGuBufs);
-    finalize(it, pt);
+    if (tid < nw * n) {
+      const int iw = tid / n, i = tid - iw * n;
+      const int f = (iw * kWarps + nw - 1) / nw, c = ((iw + 1) * kWarps + nw - 1) / nw - f;
+      float gsum = 0.f, usum = 0.f;
+      for (int w = f; w < f + c; ++w) { gsum += part[w * 16 + i]; usum += part[w * 16 + 8 + i]; }
+      store_a(w0 + iw, i, gsum, usum);
+    }
   }
   if (!ok) {   // a copy never landed: give the copies in flight one more bound before leaving
     for (int it = (nitems > kGuBufs ? nitems - kGuBufs : 0); it < nitems; ++it)
-      if (n) mbar_wait_bounded(&bars[it % kGuBufs], (unsigned)(it / kGuBufs) & 1u, p.wait_ns, nullptr);
+      mbar_wait_bounded(&bars[it % kGuBufs], (unsigned)(it / kGuBufs) & 1u, p.wait_ns, nullptr);
   }
 }
 
@@ -279,7 +308,7 @@ constexpr int kDnMaxRows = 32;  // hidden rows per CTA
 
 struct DnLayout {
   int RB, SRB, SBR, GB, nsp, ng;
-  size_t buf, as, btab, gsc, gs, part, yacc, wsl, slots, topk, bars, total;
+  size_t buf, btab, gs, part, yacc, wsl, slots, topk, bars, total;
 };
 __host__ __device__ inline DnLayout dn_layout(int I, int S, int bits) {
   DnLayout L;
@@ -292,12 +321,10 @@ __host__ __device__ inline DnLayout dn_layout(int I, int S, int bits) {
   const int nb = S < kDnBufs ? S : kDnBufs;
   size_t o = 0;
   L.buf = o; o += (size_t)nb * L.GB;
-  L.as = o; o += sizeof(float) * (size_t)S * I;
   L.btab = o; o += sizeof(uint2) * (size_t)S * L.nsp * kBtPerSpan;
-  L.gsc = o; o += sizeof(float) * (size_t)S * L.ng;
-  L.gs = o; o += sizeof(float) * 2 * (size_t)S * L.ng;
+  L.gs = o; o += sizeof(float) * 2 * (size_t)S * L.ng;     // per slot [2^-p_g | X_g]
   o = (o + 15) & ~(size_t)15;
-  L.part = o; o += sizeof(float) * 2 * (kDnMaxRows / 16) * L.nsp * 16;
+  L.part = o; o += sizeof(float) * (size_t)nb * (kDnMaxRows / 16) * L.nsp * 16;
   L.yacc = o; o += sizeof(float) * kDnMaxRows;
   L.wsl = o; o += sizeof(float) * kMaxSlots;
   o = (o + 15) & ~(size_t)15;
@@ -311,20 +338,18 @@ __host__ __device__ inline DnLayout dn_layout(int I, int S, int bits) {
 }
 
 // grid (nCTA, T), block 512. This kernel starts once every gate/up CTA has
-// passed its dependency wait, so the router's logits and the residual h are
-// final: before its own wait it ranks the logits and starts the copies of its
-// rows of every chosen expert's down matrix. After the wait it turns a into
-// per-expert B tables and forms hacc = h + sum_i w_i y_i + sg * y_shared for
-// its rows.
+// passed its dependency wait, so the router's logits, the residual h and the
+// shared expert's a are final: before its own wait it ranks the logits,
+// starts the copies of its rows of every chosen expert's down matrix and
+// applies the shared expert. After the wait it turns the routed experts' a
+// into B tables and forms hacc = h + sum_i w_i y_i + sg * y_shared for its rows.
 template <int BITS>
 __global__ void __launch_bounds__(kThreads, 2) down_decode_kernel(DownParams p) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int S = p.S;
   const DnLayout L = dn_layout(p.I, S, BITS);
   unsigned char* bufs = smem + L.buf;
-  float* as = (float*)(smem + L.as);
   uint2* btab = (uint2*)(smem + L.btab);
-  float* gsc = (float*)(smem + L.gsc);
   float* gs = (float*)(smem + L.gs);
   float* part = (float*)(smem + L.part);
   float* yacc = (float*)(smem + L.yacc);
@@ -344,13 +369,94 @@ __global__ void __launch_bounds__(kThreads, 2) down_decode_kernel(DownParams p) 
   int pre;
   const unsigned sbw = sb_window(h0, n, L.SRB, pre);
   const unsigned item_bytes = (unsigned)n * L.RB + 2u * sbw;
+  const int per = nsp * kBtPerSpan;
+  const int ppart = (kDnMaxRows / 16) * nsp * 16;   // floats of part per item
   bool ok = true;
+
+  auto issue = [&](int it, int c) {   // c = 0 codes, 1 scales, 2 biases
+    const int b = it % nb;
+    unsigned char* buf = bufs + (size_t)b * L.GB;
+    const moe_qmat& m = slot_ex[item_slot(it)].down;
+    fence_proxy_async();
+    if (c == 0) {
+      bulk_g2s(buf, (const char*)m.q + (size_t)h0 * L.RB, (unsigned)n * L.RB, &bars[b]);
+    } else {
+      const uint16_t* src = c == 1 ? m.scales : m.biases;
+      bulk_g2s(buf + kDnMaxRows * L.RB + (c - 1) * L.SBR, (const char*)src + (((size_t)h0 * L.SRB) & ~(size_t)15),
+               sbw, &bars[b]);
+    }
+  };
+  // B tables of slots [sl0, sl1) from a
+  auto tables = [&](int sl0, int sl1) {
+    constexpr int EPT = TabTraits<BITS>::kEPT;
+    const int qs = I / EPT, nq = (sl1 - sl0) * qs;
+    for (int q0 = 0; q0 < nq; q0 += kThreads) {
+      const int q = q0 + tid, sl = sl0 + q / qs, e = (q - (q / qs) * qs) * EPT;
+      const bool valid = q < nq;
+      float v[EPT];
+      if (valid) load_chunk_f32<BITS>(p.a + ((size_t)t * S + sl) * I, e / EPT, v);
+      build_tables<BITS>(v, e, valid, btab + (size_t)(valid ? sl : 0) * per, gs + (size_t)(valid ? sl : 0) * 2 * ng, ng);
+    }
+  };
+  // unit u = (tile, span) of item it: row sums to pt[u][16]
+  auto unit = [&](int it, int u, float* pt) {
+    const int b = it % nb, slot = item_slot(it);
+    const unsigned char* buf = bufs + (size_t)b * L.GB;
+    const int g = lane >> 2, tq = lane & 3;
+    const int bl = bt_lane_index(lane);
+    constexpr int SB = SpanBytes<BITS>::v;
+    constexpr int WB = QTraits<BITS>::kWordsPerThread * 4;
+    const int tile = u / nsp, s = u - tile * nsp;
+    const int r = tile * 16 + g;
+    Frag<BITS> F;
+    frag_codes<BITS>(F, buf + (size_t)r * L.RB + s * SB + tq * WB, buf + (size_t)(r + 8) * L.RB + s * SB + tq * WB);
+    const unsigned char* sc = buf + kDnMaxRows * L.RB + pre + s * 4;
+    F.sa = *(const uint32_t*)(sc + r * L.SRB);
+    F.sb = *(const uint32_t*)(sc + (r + 8) * L.SRB);
+    F.ba = *(const uint32_t*)(sc + L.SBR + r * L.SRB);
+    F.bb = *(const uint32_t*)(sc + L.SBR + (r + 8) * L.SRB);
+    int c[4];
+    mma_frag<BITS>(F, btab + (size_t)slot * per + s * kBtPerSpan, bl, c);
+    const float* gsl = gs + (size_t)slot * 2 * ng;
+    float acc_a = 0.f, acc_b = 0.f;
+    scale_frag_i(F.sa, F.sb, F.ba, F.bb, c, gsl, gsl + ng, s, tq, acc_a, acc_b);
+    acc_a += __shfl_xor_sync(0xffffffffu, acc_a, 1);
+    acc_b += __shfl_xor_sync(0xffffffffu, acc_b, 1);
+    acc_a += __shfl_xor_sync(0xffffffffu, acc_a, 2);
+    acc_b += __shfl_xor_sync(0xffffffffu, acc_b, 2);
+    if (tq == 0) { pt[u * 16 + g] = acc_a; pt[u * 16 + 8 + g] = acc_b; }
+  };
+  // items [i0, i1) (all staged): units spread over the warps, then yacc += w * y
+  auto run = [&](int i0, int i1) {
+    const int U = ntile * nsp, UT = (i1 - i0) * U;
+    int waited = -1;
+    for (int x = UT * warp / kWarps; x < UT * (warp + 1) / kWarps; ++x) {
+      const int it = i0 + x / U;
+      if (it != waited) {
+        ok &= mbar_wait_bounded(&bars[it % nb], (unsigned)(it / nb) & 1u, p.wait_ns, p.status);
+        waited = it;
+      }
+      unit(it, x - (it - i0) * U, part + (size_t)(it % nb) * ppart);
+    }
+    fence_proxy_async();
+    __syncthreads();
+    if (tid < n) {
+      const int tile = tid >> 4, rr = tid & 15;
+      float acc = yacc[tid];
+      for (int it = i0; it < i1; ++it) {
+        const float* pt = part + (size_t)(it % nb) * ppart;
+        float y = 0.f;
+        for (int s = 0; s < nsp; ++s) y += pt[(tile * nsp + s) * 16 + rr];
+        acc = fmaf(wsl[item_slot(it)], y, acc);
+      }
+      yacc[tid] = acc;
+    }
+  };
 
   if (tid == 0) {
     for (int b = 0; b < nb; ++b) mbar_init(&bars[b], 1);
     fence_mbar_init();
-    for (int b = 0; b < nb; ++b)
-      if (n) mbar_expect_tx(&bars[b], item_bytes);   // items 0..nb-1
+    for (int b = 0; b < nb; ++b) mbar_expect_tx(&bars[b], item_bytes);   // items 0..nb-1
     if (p.has_shared) slot_ex[S - 1] = p.shared;
   }
   block_topk(p.logits + (size_t)t * (p.E + 1), p.E, k, p.has_shared, ts);
@@ -359,93 +465,38 @@ __global__ void __launch_bounds__(kThreads, 2) down_decode_kernel(DownParams p) 
   if (tid == 0 && p.has_shared) wsl[S - 1] = ts.sg;
   if (tid < n) yacc[tid] = __ldcg(p.h + (size_t)t * H + h0 + tid);
   __syncthreads();
-
-  auto issue = [&](int it) {   // lane 0 of warps 0-2, one copy each
-    if (lane != 0 || warp >= 3 || n == 0) return;
-    const int b = it % nb;
-    unsigned char* buf = bufs + (size_t)b * L.GB;
-    const moe_qmat& m = slot_ex[item_slot(it)].down;
-    fence_proxy_async();
-    if (warp == 0) {
-      bulk_g2s(buf, (const char*)m.q + (size_t)h0 * L.RB, (unsigned)n * L.RB, &bars[b]);
-    } else {
-      const uint16_t* src = warp == 1 ? m.scales : m.biases;
-      bulk_g2s(buf + kDnMaxRows * L.RB + (warp - 1) * L.SBR, (const char*)src + (((size_t)h0 * L.SRB) & ~(size_t)15),
-               sbw, &bars[b]);
-    }
-  };
-  for (int it = 0; it < nb; ++it) issue(it);
+  if (lane == 0)
+    for (int c = warp; c < 3 * nb; c += kWarps) issue(c / 3, c % 3);
+  int issued = nb;   // items [0, issued) have their copies in flight or landed
+  int it0 = 0;
+  if (p.has_shared) {   // the shared expert's a is final: apply it before the wait
+    tables(S - 1, S);
+    __syncthreads();
+    run(0, 1);
+    it0 = 1;
+  }
 
   griddep_wait();
   griddep_launch_dependents();
-  // a = silu(g) * u of every slot -> per-slot group prescales, sums and B tables
-  const float4* ag = (const float4*)(p.a + (size_t)t * S * I);
-  for (int i = tid; i < S * I / 4; i += kThreads) ((float4*)as)[i] = __ldcg(ag + i);
+  tables(0, k);
   __syncthreads();
-  group_stats(as, S * ng, gsc, gs, gs + S * ng, warp, lane, kWarps);   // [slot*ng + g]
-  __syncthreads();
-  const int per = nsp * kBtPerSpan;
-  for (int i = tid; i < S * per; i += kThreads) {
-    const int sl = i / per;
-    btab[i] = btab_at<BITS>(as + (size_t)sl * I, gsc + (size_t)sl * ng, i - sl * per);
-  }
-  __syncthreads();
-
-  // units of an item: (tile, span), warp w takes [U*w/16, U*(w+1)/16); row sums to pt[tile][span][16]
-  const int U = ntile * nsp;
-  auto compute = [&](int b, int slot, float* pt) {
-    const unsigned char* buf = bufs + (size_t)b * L.GB;
-    const int g = lane >> 2, tq = lane & 3;
-    const int bl = bt_lane_index(lane);
-    constexpr int SB = SpanBytes<BITS>::v;
-    constexpr int WB = QTraits<BITS>::kWordsPerThread * 4;
-    const uint2* bt = btab + (size_t)slot * per;
-    const float* gsl = gs + (size_t)slot * ng;          // 2^-p_g of this slot
-    const float* xgl = gs + (size_t)S * ng + (size_t)slot * ng;   // X_g of this slot
-    for (int u = U * warp / kWarps; u < U * (warp + 1) / kWarps; ++u) {
-      const int tile = u / nsp, s = u - tile * nsp;
-      const int r = tile * 16 + g;
-      Frag<BITS> F;
-      frag_codes<BITS>(F, buf + (size_t)r * L.RB + s * SB + tq * WB, buf + (size_t)(r + 8) * L.RB + s * SB + tq * WB);
-      const unsigned char* sc = buf + kDnMaxRows * L.RB + pre + s * 4;
-      F.sa = *(const uint32_t*)(sc + r * L.SRB);
-      F.sb = *(const uint32_t*)(sc + (r + 8) * L.SRB);
-      F.ba = *(const uint32_t*)(sc + L.SBR + r * L.SRB);
-      F.bb = *(const uint32_t*)(sc + L.SBR + (r + 8) * L.SRB);
-      int c[4];
-      mma_frag<BITS>(F, bt + s * kBtPerSpan, bl, c);
-      float acc_a = 0.f, acc_b = 0.f;
-      scale_frag_i(F.sa, F.sb, F.ba, F.bb, c, gsl, xgl, s, tq, acc_a, acc_b);
-      acc_a += __shfl_xor_sync(0xffffffffu, acc_a, 1);
-      acc_b += __shfl_xor_sync(0xffffffffu, acc_b, 1);
-      acc_a += __shfl_xor_sync(0xffffffffu, acc_a, 2);
-      acc_b += __shfl_xor_sync(0xffffffffu, acc_b, 2);
-      if (tq == 0) { pt[u * 16 + g] = acc_a; pt[u * 16 + 8 + g] = acc_b; }
+  for (int w0 = it0; w0 < nitems; w0 += nb) {
+    const int w1 = nitems - w0 < nb ? nitems : w0 + nb;
+    if (issued < w1) {   // refill buffers whose previous items are done
+      if (tid == 0)
+        for (int it = issued; it < w1; ++it) mbar_expect_tx(&bars[it % nb], item_bytes);
+      __syncthreads();
+      if (lane == 0)
+        for (int c = warp; c < 3 * (w1 - issued); c += kWarps) issue(issued + c / 3, c % 3);
+      issued = w1;
     }
-  };
-  auto finalize = [&](int slot, const float* pt) {
-    if (tid < n) {
-      const int tile = tid >> 4, r = tid & 15;
-      float y = 0.f;
-      for (int s = 0; s < nsp; ++s) y += pt[(tile * nsp + s) * 16 + r];
-      yacc[tid] = fmaf(wsl[slot], y, yacc[tid]);
-    }
-  };
-  for (int it = 0; it < nitems; ++it) {
-    const int b = it % nb, slot = item_slot(it);
-    float* pt = part + (it & 1) * (kDnMaxRows / 16) * nsp * 16;
-    if (n) ok &= mbar_wait_bounded(&bars[b], (unsigned)(it / nb) & 1u, p.wait_ns, p.status);
-    compute(b, slot, pt);
-    fence_proxy_async();
-    if (tid == 0 && n && it + nb < nitems) mbar_expect_tx(&bars[b], item_bytes);
+    run(w0, w1);
     __syncthreads();
-    if (it + nb < nitems) issue(it + nb);
-    finalize(slot, pt);
   }
   if (tid < n) p.hacc[(size_t)t * H + h0 + tid] = yacc[tid];
   if (!ok) {
     for (int it = (nitems > nb ? nitems - nb : 0); it < nitems; ++it)
-      if (n) mbar_wait_bounded(&bars[it % nb], (unsigned)(it / nb) & 1u, p.wait_ns, nullptr);
+      mbar_wait_bounded(&bars[it % nb], (unsigned)(it / nb) & 1u, p.wait_ns, nullptr);
   }
 }
 

@@ -9,11 +9,13 @@ namespace qmoe {
 // k largest logits, descending, ties to the lower index; weights = softmax over
 // all E renormalised over the chosen k = exp(l_i - l_max) / sum_chosen exp(l_j - l_max);
 // shared gate = sigmoid(logit E). Logits are compared through an
-// order-preserving 64-bit integer key of their double bits (NaN ranks lowest).
-// Every warp ranks its slice (one logit per lane per pass, in registers);
-// warp 0 merges the warps' candidates. Exact: every global top-k entry is in
-// its slice's top-k.
-constexpr int kTopkPer = 8;   // logits per lane: E <= kTopkPer * 32 * warps
+// order-preserving 64-bit integer key of their double bits (key 0 = NaN or
+// already taken, ranks lowest). Thread i holds logits i, i + blockDim, ...;
+// every warp takes its k best in k rounds (one warp reduction of the key's
+// high half per round; the low half and the index only on ties), warp 0 then
+// takes the k best of the warps' candidates. Exact: every global top-k entry
+// is among its warp's top-k.
+constexpr int kTopkPer = 8;   // logits per thread: E <= kTopkPer * blockDim
 
 struct TopkSmem {
   unsigned long long ck[kWarps][kMaxTopK];   // candidate keys
@@ -32,88 +34,104 @@ __device__ __forceinline__ double key_value(unsigned long long k) {
   const unsigned long long u = (k >> 63) ? (k & 0x7fffffffffffffffull) : ~k;
   return __longlong_as_double((long long)u);
 }
-// warp-wide argmax of (key desc, id asc) with three warp reductions
-__device__ __forceinline__ void warp_argmax(unsigned long long& bk, int& be) {
-  const unsigned hi = (unsigned)(bk >> 32), lo = (unsigned)bk;
-  const unsigned mh = __reduce_max_sync(0xffffffffu, hi);
-  const unsigned ml = __reduce_max_sync(0xffffffffu, hi == mh ? lo : 0u);
-  const bool cand = hi == mh && lo == ml;
-  const unsigned me = __reduce_min_sync(0xffffffffu, cand ? (unsigned)be : 0xffffffffu);
-  bk = ((unsigned long long)mh << 32) | ml;
-  be = (int)me;
+
+// Warp-wide best of (key desc, id asc) over the lanes' (key, id); returns the
+// winning lane (uniform) and the winner's key and id in wk, wi.
+__device__ __forceinline__ int warp_best(unsigned long long key, int id, unsigned long long& wk, int& wi) {
+  const unsigned full = 0xffffffffu;
+  const unsigned hi = (unsigned)(key >> 32), lo = (unsigned)key;
+  const unsigned mh = __reduce_max_sync(full, hi);
+  bool c = hi == mh;
+  unsigned bal = __ballot_sync(full, c);
+  if (bal & (bal - 1)) {   // several lanes share the high half
+    const unsigned ml = __reduce_max_sync(full, c ? lo : 0u);
+    c = c && lo == ml;
+    bal = __ballot_sync(full, c);
+    if (bal & (bal - 1)) {   // equal keys: lowest id
+      const unsigned mi = __reduce_min_sync(full, c ? (unsigned)id : 0xffffffffu);
+      c = c && (unsigned)id == mi;
+      bal = __ballot_sync(full, c);
+    }
+  }
+  const int wl = __ffs(bal) - 1;
+  wk = ((unsigned long long)mh << 32) | __shfl_sync(full, lo, wl);
+  wi = __shfl_sync(full, id, wl);
+  return wl;
 }
 
 // Block-wide top-k of lg[0..E) (+ shared gate from lg[E] when has_shared),
 // global memory written by an earlier kernel. All threads of the block call
-// it; results in ts (valid after the call, which ends with __syncthreads).
+// it (blockDim = 32 * kWarps); results in ts, valid after the call, which ends
+// with __syncthreads. Ids of missing entries (all logits NaN) are -1.
 __device__ __noinline__ static void block_topk(const double* lg, int E, int k, int has_shared, TopkSmem& ts) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  constexpr int kNone = 0x7fffffff;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nt = blockDim.x;
   unsigned long long key[kTopkPer];
 #pragma unroll
   for (int j = 0; j < kTopkPer; ++j) {
-    const int e = (j * nw + warp) * 32 + lane;
+    const int e = tid + j * nt;
     key[j] = e < E ? order_key(__ldcg(lg + e)) : 0ull;
   }
-  double gl = 0.0;
-  if (warp == 0 && lane == 0 && has_shared) gl = __ldcg(lg + E);
-  for (int r = 0; r < k; ++r) {
-    unsigned long long bk = 0ull;
-    int be = kNone, bj = -1;
+  float gl = 0.f;
+  if (warp == 0 && lane == 0 && has_shared) gl = (float)__ldcg(lg + E);
+  // this thread's best (lowest index among equal keys: j ascending, strict >)
+  auto local_best = [&](unsigned long long& bk, int& bj) {
+    bk = 0ull; bj = 0;
 #pragma unroll
-    for (int j = 0; j < kTopkPer; ++j) {
-      const int e = (j * nw + warp) * 32 + lane;
-      if (e < E && key[j] > bk) { bk = key[j]; be = e; bj = j; }
-    }
-    unsigned long long wk = bk;
-    int we = be;
-    warp_argmax(wk, we);
-    if (be == we && we != kNone) {
+    for (int j = 0; j < kTopkPer; ++j)
+      if (key[j] > bk) { bk = key[j]; bj = j; }
+  };
+  unsigned long long bk;
+  int bj;
+  local_best(bk, bj);
+  for (int r = 0; r < k; ++r) {
+    unsigned long long wk;
+    int wi;
+    const int wl = warp_best(bk, tid + bj * nt, wk, wi);
+    if (lane == 0) { ts.ck[warp][r] = wk; ts.ce[warp][r] = wk ? wi : -1; }
+    if (lane == wl && wk) {
 #pragma unroll
       for (int j = 0; j < kTopkPer; ++j)
         if (j == bj) key[j] = 0ull;
+      local_best(bk, bj);
     }
-    if (lane == 0) { ts.ck[warp][r] = wk; ts.ce[warp][r] = we; }
   }
   __syncthreads();
   if (warp == 0) {
-    // candidates c = lane + 32 q (q < 4), c = warp' * kMaxTopK + r'
+    const int nw = nt >> 5, nc = nw * k;
     unsigned long long ck[4];
     int ce[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const int c = lane + 32 * q, w = c / kMaxTopK, r = c % kMaxTopK;
-      const bool ok = w < nw && r < k;
+      const int c = lane + 32 * q, w = c / k, r = c - w * k;
+      const bool ok = c < nc;
       ck[q] = ok ? ts.ck[w][r] : 0ull;
-      ce[q] = ok ? ts.ce[w][r] : kNone;
+      ce[q] = ok ? ts.ce[w][r] : -1;
     }
-    double lv0 = 0.0, z = 0.0;
-    float ex[kMaxTopK];
+    unsigned long long mine = 0ull, first = 0ull;
+    int mid = -1;
     for (int r = 0; r < k; ++r) {
-      unsigned long long bk = 0ull;
-      int be = kNone, bq = -1;
+      unsigned long long b = 0ull;
+      int bq = 0, bid = -1;
 #pragma unroll
       for (int q = 0; q < 4; ++q)
-        if (ce[q] != kNone && (ck[q] > bk || (ck[q] == bk && ce[q] < be))) { bk = ck[q]; be = ce[q]; bq = q; }
-      unsigned long long wk = bk;
-      int we = be;
-      warp_argmax(wk, we);
-      if (be == we && we != kNone) {
+        if (ck[q] > b || (ck[q] == b && b && (unsigned)ce[q] < (unsigned)bid)) { b = ck[q]; bq = q; bid = ce[q]; }
+      unsigned long long wk;
+      int wi;
+      const int wl = warp_best(b, bid, wk, wi);
+      if (lane == wl && wk) {
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-          if (q == bq) { ck[q] = 0ull; ce[q] = kNone; }
+          if (q == bq) { ck[q] = 0ull; ce[q] = -1; }
       }
-      const double lv = key_value(wk);
-      if (r == 0) lv0 = lv;
-      ex[r] = expf((float)(lv - lv0));
-      z += ex[r];
-      if (lane == 0) ts.idx[r] = we == kNone ? -1 : we;
+      if (r == 0) first = wk;
+      if (lane == r) { mine = wk; mid = wk ? wi : -1; }
     }
-    if (lane == 0) {
-      const float iz = (float)(1.0 / z);
-      for (int r = 0; r < k; ++r) ts.w[r] = ex[r] * iz;
-      ts.sg = has_shared ? 1.f / (1.f + expf(-(float)gl)) : 0.f;
-    }
+    // weights over the chosen k
+    const float ex = (lane < k && mine) ? expf((float)(key_value(mine) - key_value(first))) : 0.f;
+    const float z = warp_sum(ex);
+    if (lane < k) { ts.idx[lane] = mid; ts.w[lane] = ex / z; }
+    if (lane == 0) ts.sg = has_shared ? 1.f / (1.f + expf(-gl)) : 0.f;
   }
   __syncthreads();
 }
