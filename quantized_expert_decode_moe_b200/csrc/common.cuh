@@ -264,17 +264,21 @@ __device__ __forceinline__ void build_tables(const float (&v)[TabTraits<BITS>::k
   }
   if (!valid) return;
   const int sh = prescale_shift(m);
-  const float sc = __uint_as_float((uint32_t)(127 + sh) << 23);
-  int X[EPT];
-#pragma unroll
-  for (int i = 0; i < EPT; ++i) X[i] = __float2int_rn(v[i] * sc);
   const int s = e0 / kSpan, w = e0 % kSpan, t = w / 32, grp = t >> 1;
   const int c0 = grp * kDigits * 2 + (t & 1);   // entry of digit d: c0 + 2d
+  // Element o of the window enters the MMA as code << (BITS * q) (masked in
+  // place, q = its field in the byte), so its fixed point is scaled down by
+  // 2^(BITS q): X = rint(x * 2^(sh - BITS q)).
+  int X[EPT];
   if constexpr (BITS == 4) {
+#pragma unroll
+    for (int i = 0; i < EPT; ++i) X[i] = __float2int_rn(v[i] * __uint_as_float((uint32_t)(127 + sh - 4 * (i & 1)) << 23));
     uint2* e = bt + s * kBtPerSpan + ((w % 32) / 8) * kBtLanes + c0;
 #pragma unroll
     for (int d = 0; d < kDigits; ++d) e[2 * d] = make_uint2(pack_digits(X, 0, 2, d), pack_digits(X, 1, 2, d));
   } else {
+#pragma unroll
+    for (int i = 0; i < EPT; ++i) X[i] = __float2int_rn(v[i] * __uint_as_float((uint32_t)(127 + sh - 2 * (i & 3)) << 23));
     const int jj = (w % 32) / 16;
 #pragma unroll
     for (int jl = 0; jl < 2; ++jl) {
@@ -289,6 +293,61 @@ __device__ __forceinline__ void build_tables(const float (&v)[TabTraits<BITS>::k
     gs[g] = __uint_as_float((uint32_t)(127 - sh) << 23);
     gs[ng + g] = sum;
   }
+}
+
+// Code bytes of MMA j, half h, with each field left in place in its byte
+// (the B table holds the matching scaled-down digits): 4-bit: low / high
+// nibble; 2-bit: field 2(j&1)+h of word j>>1.
+template <int BITS>
+__device__ __forceinline__ uint32_t code_bytes_m(const uint32_t* w, int j, int half) {
+  if constexpr (BITS == 4) return w[j] & (half ? 0xF0F0F0F0u : 0x0F0F0F0Fu);
+  else return w[j >> 1] & (0x03030303u << (2 * (2 * (j & 1) + half)));
+}
+
+// B operand of one span of a vector, loaded once and reused for every row tile.
+struct BFrag {
+  uint2 b[4];
+  float ip, xg;   // 2^-p of the lane's group; X_g on even lanes (bias term), 0 on odd lanes
+};
+__device__ __forceinline__ void load_bfrag(BFrag& B, const uint2* bt_span, int bl, const float* gs, int ng, int span,
+                                           int t) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) B.b[j] = bl >= 0 ? bt_span[j * kBtLanes + bl] : make_uint2(0u, 0u);
+  const int gi = 2 * span + (t >> 1);
+  B.ip = gs[gi];
+  B.xg = (t & 1) ? 0.f : gs[ng + gi];
+}
+// Lane constants of the epilogue: thread t holds MMA columns 2t, 2t+1 = the
+// digits of group t>>1 (t even: d0, d1; t odd: d2).
+struct LaneK {
+  float m0, m1;   // f = c0 * m0 + c1 * m1
+  int shl;        // bf16 of the lane's group: (word << shl) & 0xFFFF0000
+};
+__device__ __forceinline__ LaneK lane_consts(int t) {
+  LaneK K;
+  const bool odd = t & 1;
+  K.m0 = odd ? 65536.f : 1.f;
+  K.m1 = odd ? 0.f : 256.f;
+  K.shl = (t >> 1) ? 0 : 16;
+  return K;
+}
+__device__ __forceinline__ float bf16_sel(uint32_t wd, int shl) { return __uint_as_float((wd << shl) & 0xFFFF0000u); }
+
+// One span of one 16-row tile: A codes of rows g (wa) and g+8 (wb), scale and
+// bias words of those rows (bf16 pairs of the span's two groups); adds the
+// dequantised products to acc_a (row g) and acc_b (row g+8).
+template <int BITS>
+__device__ __forceinline__ void tile_span(const uint32_t* wa, const uint32_t* wb, uint32_t sa, uint32_t sb, uint32_t ba,
+                                          uint32_t bb, const BFrag& B, const LaneK& K, float& acc_a, float& acc_b) {
+  int c[4] = {0, 0, 0, 0};
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    mma_u8s8(c, code_bytes_m<BITS>(wa, j, 0), code_bytes_m<BITS>(wb, j, 0), code_bytes_m<BITS>(wa, j, 1),
+             code_bytes_m<BITS>(wb, j, 1), B.b[j].x, B.b[j].y);
+  const float fa = fmaf((float)c[1], K.m1, (float)c[0] * K.m0);
+  const float fb = fmaf((float)c[3], K.m1, (float)c[2] * K.m0);
+  acc_a = fmaf(bf16_sel(sa, K.shl) * B.ip, fa, fmaf(bf16_sel(ba, K.shl), B.xg, acc_a));
+  acc_b = fmaf(bf16_sel(sb, K.shl) * B.ip, fb, fmaf(bf16_sel(bb, K.shl), B.xg, acc_b));
 }
 
 // ------------------------------------------------------------------ per-warp staging with cp.async

@@ -50,9 +50,8 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
 }
 // Waits for the phase of parity `parity` of bar, for at most bound_ns; on
 // timeout latches MOE_ERR_TIMEOUT in *status and returns false.
-__device__ __noinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity, unsigned long long bound_ns,
-                                               uint32_t* status) {
-  if (mbar_try_wait(bar, parity)) return true;
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, unsigned parity, unsigned long long bound_ns,
+                                            uint32_t* status) {
   const unsigned long long t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
     if (globaltimer_ns() - t0 > bound_ns) {
@@ -61,6 +60,10 @@ __device__ __noinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity, u
     }
   }
   return true;
+}
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity, unsigned long long bound_ns,
+                                                  uint32_t* status) {
+  return mbar_try_wait(bar, parity) || mbar_wait_slow(bar, parity, bound_ns, status);
 }
 
 // 16-byte aligned window of rows [r0, r0+n) of a per-row array of SRB bytes
@@ -114,29 +117,47 @@ __device__ __forceinline__ void load_chunk_f32(const float* a, int q, float (&v)
   }
 }
 
+// 16 bytes of scale or bias data (4 spans x a bf16 pair) at p: one 16-byte
+// load when the per-row arrays keep 16-byte alignment, else four 4-byte loads.
+__device__ __forceinline__ uint4 lds_chunk(const unsigned char* p, bool al16) {
+  if (al16) return *(const uint4*)p;
+  const uint32_t* q = (const uint32_t*)p;
+  return make_uint4(q[0], q[1], q[2], q[3]);
+}
+__device__ __forceinline__ uint32_t chunk_word(const uint4& v, int i) {
+  return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+}
+// Code rows in shared memory are padded so that MMA rows g and g+1 (read by
+// the same 8-lane phase of a 16-byte load, or 16-lane phase of an 8-byte
+// load) fall in different banks.
+template <int BITS>
+__host__ __device__ inline int padded_row(int RB) { return RB % 128 == 0 ? RB + (BITS == 4 ? 64 : 32) : RB; }
+
 // ------------------------------------------------------------------ gate/up + SwiGLU
 constexpr int kGuBufs = 3;      // expert tiles staged per CTA (the shared expert's buffer is reused)
 constexpr int kGuMaxRows = 8;   // intermediate rows per CTA
 
 struct GuLayout {
-  int RB, SRB, SBR, GB;   // code bytes per row, scale bytes per row, scale region, buffer bytes
+  int RB, P, SRB, SBR, GB;   // code bytes per row, padded row pitch, scale bytes per row, scale region, buffer bytes
   size_t buf, btab, gs, part, slots, topk, bars, total;
 };
 __host__ __device__ inline GuLayout gu_layout(int H, int bits) {
   GuLayout L;
   L.RB = H * bits / 8;
+  L.P = L.RB;   // rows land contiguously (one bulk copy per row block)
   L.SRB = H / 32;
   L.SBR = sb_region(kGuMaxRows, L.SRB);
-  L.GB = (2 * kGuMaxRows * L.RB + 4 * L.SBR + 127) & ~127;
+  L.GB = (2 * kGuMaxRows * L.P + 4 * L.SBR + 127) & ~127;
   size_t o = 0;
   L.buf = o; o += (size_t)kGuBufs * L.GB;
   L.btab = o; o += sizeof(uint2) * (size_t)(H / kSpan) * kBtPerSpan;
   L.gs = o; o += sizeof(float) * 2 * (size_t)(H / kGroup);   // [2^-p_g | X_g]
   o = (o + 15) & ~(size_t)15;
-  L.part = o; o += sizeof(float) * kWarps * 16;
-  L.slots = o; o += sizeof(moe_expert) * kMaxSlots;
+  const size_t part = sizeof(float) * kGuBufs * kWarps * 16;
+  L.part = o; L.topk = o;   // the top-k scratch is dead before the partial sums are written
+  o += part > sizeof(TopkSmem) ? part : sizeof(TopkSmem);
   o = (o + 15) & ~(size_t)15;
-  L.topk = o; o += sizeof(TopkSmem);
+  L.slots = o; o += sizeof(moe_expert) * kMaxSlots;
   o = (o + 15) & ~(size_t)15;
   L.bars = o; o += 8 * kGuBufs;
   L.total = o;
@@ -164,8 +185,8 @@ __global__ void __launch_bounds__(kThreads, 2) gateup_decode_kernel(GateUpParams
   const int t = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = p.H, I = p.I, S = p.S, k = p.k;
   const int ng = H / kGroup, nspans = H / kSpan;
-  const int j0 = (int)((long long)I * blockIdx.x / gridDim.x);
-  const int n = (int)((long long)I * (blockIdx.x + 1) / gridDim.x) - j0;
+  const int j0 = (int)((unsigned)I * blockIdx.x / gridDim.x);
+  const int n = (int)((unsigned)I * (blockIdx.x + 1) / gridDim.x) - j0;
   const int nitems = k + (p.has_shared ? 1 : 0);
   auto item_slot = [&](int it) { return p.has_shared ? (it == 0 ? S - 1 : it - 1) : it; };
   int pre;
@@ -176,53 +197,99 @@ __global__ void __launch_bounds__(kThreads, 2) gateup_decode_kernel(GateUpParams
   auto arm = [&](int it) {   // thread 0, before the barrier that precedes the item's copies
     if (tid == 0) mbar_expect_tx(&bars[it % kGuBufs], item_bytes);
   };
-  // copies of item `it` into buffer it % kGuBufs: one copy per thread listed below
-  auto issue = [&](int it, int c) {   // c = copy 0..5: gate codes, up codes, gate/up scales, gate/up biases
+  // copies of item `it` into buffer it % kGuBufs, one per call: c = 0 gate
+  // code rows, 1 up code rows (row blocks), 2..5 gate/up scales, gate/up biases
+  const int ncp = 6;
+  auto issue = [&](int it, int c) {
     const int b = it % kGuBufs;
     unsigned char* buf = bufs + (size_t)b * L.GB;
     const moe_expert& ex = slot_ex[item_slot(it)];
     fence_proxy_async();
     if (c < 2) {
       const moe_qmat& m = c == 0 ? ex.gate : ex.up;
-      bulk_g2s(buf + (size_t)c * kGuMaxRows * L.RB, (const char*)m.q + (size_t)j0 * L.RB, (unsigned)n * L.RB, &bars[b]);
+      bulk_g2s(buf + (size_t)c * kGuMaxRows * L.P, (const char*)m.q + (size_t)j0 * L.RB, (unsigned)n * L.RB, &bars[b]);
     } else {
       const int w = c - 2;   // 0 gate scales, 1 up scales, 2 gate biases, 3 up biases
       const moe_qmat& m = (w & 1) ? ex.up : ex.gate;
       const uint16_t* src = w < 2 ? m.scales : m.biases;
-      bulk_g2s(buf + 2 * kGuMaxRows * L.RB + w * L.SBR, (const char*)src + (((size_t)j0 * L.SRB) & ~(size_t)15), sbw,
+      bulk_g2s(buf + 2 * kGuMaxRows * L.P + w * L.SBR, (const char*)src + (((size_t)j0 * L.SRB) & ~(size_t)15), sbw,
                &bars[b]);
     }
   };
-  // MMAs of spans [s0, s1) of the item in buffer b; row sums of rows g, g+8 returned in acc_a, acc_b (quad-reduced)
-  auto compute = [&](int b, int s0, int s1, float& acc_a, float& acc_b) {
-    const unsigned char* buf = bufs + (size_t)b * L.GB;
-    const int g = lane >> 2, tq = lane & 3;
+  // MMAs of this warp's spans [nspans*w/16, nspans*(w+1)/16) for the items
+  // [i0, i1) (at most kGuBufs, each one 16-row tile in buffer it % kGuBufs):
+  // the B fragments of a span are loaded once for all items. Lane tq of a
+  // quad loads 4 spans of one of the row's four scale/bias arrays (gate
+  // scales, up scales, gate biases, up biases) and the quad shares them by
+  // shuffles. Row sums go to part[(it - i0)][warp][16].
+  const bool al16 = L.SRB % 16 == 0;
+  auto compute_items = [&](int i0, int i1) {
+    const int g = lane >> 2, tq = lane & 3, qb = lane & ~3;
     const int bl = bt_lane_index(lane);
+    const LaneK K = lane_consts(tq);
     constexpr int SB = SpanBytes<BITS>::v;
-    constexpr int WB = QTraits<BITS>::kWordsPerThread * 4;
-    const unsigned char* ra = buf + (size_t)g * L.RB + tq * WB;
-    const unsigned char* rb = buf + (size_t)(kGuMaxRows + g) * L.RB + tq * WB;
-    const unsigned char* sc = buf + 2 * kGuMaxRows * L.RB + pre + g * L.SRB;
-    acc_a = 0.f; acc_b = 0.f;
-    for (int s = s0; s < s1; ++s) {
-      Frag<BITS> F;
-      frag_codes<BITS>(F, ra + s * SB, rb + s * SB);
-      F.sa = *(const uint32_t*)(sc + s * 4);
-      F.sb = *(const uint32_t*)(sc + L.SBR + s * 4);
-      F.ba = *(const uint32_t*)(sc + 2 * L.SBR + s * 4);
-      F.bb = *(const uint32_t*)(sc + 3 * L.SBR + s * 4);
-      int c[4];
-      mma_frag<BITS>(F, btab + s * kBtPerSpan, bl, c);
-      scale_frag_i(F.sa, F.sb, F.ba, F.bb, c, gs, gs + ng, s, tq, acc_a, acc_b);
+    constexpr int W = QTraits<BITS>::kWordsPerThread;
+    const int s0 = nspans * warp / kWarps, s1 = nspans * (warp + 1) / kWarps;
+    for (int sp = s0; sp < s1; sp += 2) {   // span pairs: B fragments loaded once for all items
+      BFrag B[2];
+      load_bfrag(B[0], btab + sp * kBtPerSpan, bl, gs, ng, sp, tq);
+      if (sp + 1 < s1) load_bfrag(B[1], btab + (sp + 1) * kBtPerSpan, bl, gs, ng, sp + 1, tq);
+      for (int it = i0; it < i1; ++it) {
+        if (sp == s0) ok &= mbar_wait_bounded(&bars[it % kGuBufs], (unsigned)(it / kGuBufs) & 1u, p.wait_ns, p.status);
+        const unsigned char* buf = bufs + (size_t)(it % kGuBufs) * L.GB;
+        const uint4 sv = lds_chunk(buf + 2 * kGuMaxRows * L.P + tq * L.SBR + pre + g * L.SRB + 16 * (sp >> 2), al16);
+        float aa = 0.f, ab = 0.f;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int s = sp + q;
+          if (s < s1) {
+            const uint32_t w = chunk_word(sv, s & 3);
+            uint32_t wa[W], wb[W];
+            const unsigned char* ra = buf + (size_t)g * L.P + s * SB + tq * W * 4;
+            const unsigned char* rb = ra + (size_t)kGuMaxRows * L.P;
+            if constexpr (W == 4) {
+              const uint4 va = *(const uint4*)ra, vb = *(const uint4*)rb;
+              wa[0] = va.x; wa[1] = va.y; wa[2] = va.z; wa[3] = va.w;
+              wb[0] = vb.x; wb[1] = vb.y; wb[2] = vb.z; wb[3] = vb.w;
+            } else {
+              const uint2 va = *(const uint2*)ra, vb = *(const uint2*)rb;
+              wa[0] = va.x; wa[1] = va.y;
+              wb[0] = vb.x; wb[1] = vb.y;
+            }
+            const uint32_t sa = __shfl_sync(0xffffffffu, w, qb), sb = __shfl_sync(0xffffffffu, w, qb + 1);
+            const uint32_t ba = __shfl_sync(0xffffffffu, w, qb + 2), bb = __shfl_sync(0xffffffffu, w, qb + 3);
+            tile_span<BITS>(wa, wb, sa, sb, ba, bb, B[q], K, aa, ab);
+          }
+        }
+        aa += __shfl_xor_sync(0xffffffffu, aa, 1);
+        ab += __shfl_xor_sync(0xffffffffu, ab, 1);
+        aa += __shfl_xor_sync(0xffffffffu, aa, 2);
+        ab += __shfl_xor_sync(0xffffffffu, ab, 2);
+        float* pt = part + ((size_t)(it - i0) * kWarps + warp) * 16;
+        if (tq == 0) {
+          if (sp == s0) { pt[g] = aa; pt[8 + g] = ab; }
+          else { pt[g] += aa; pt[8 + g] += ab; }
+        }
+      }
     }
-    acc_a += __shfl_xor_sync(0xffffffffu, acc_a, 1);
-    acc_b += __shfl_xor_sync(0xffffffffu, acc_b, 1);
-    acc_a += __shfl_xor_sync(0xffffffffu, acc_a, 2);
-    acc_b += __shfl_xor_sync(0xffffffffu, acc_b, 2);
+    if (s0 == s1) {   // no spans: zero contributions
+      for (int it = i0; it < i1; ++it)
+        if (lane < 16) part[((size_t)(it - i0) * kWarps + warp) * 16 + lane] = 0.f;
+    }
   };
-  auto store_a = [&](int it, int i, float gsum, float usum) {
-    p.a[((size_t)t * S + item_slot(it)) * I + j0 + i] = silu_f32(gsum) * usum;
+  // a = silu(g) * u of the items [i0, i1) from the partial sums (after a barrier)
+  auto finalize = [&](int i0, int i1) {
+    if (tid < (i1 - i0) * n) {
+      const int i = tid / n, r = tid - i * n;
+      const float* pt = part + (size_t)i * kWarps * 16;
+      float gsum = 0.f, usum = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) { gsum += pt[w * 16 + r]; usum += pt[w * 16 + 8 + r]; }
+      p.a[((size_t)t * S + item_slot(i0 + i)) * I + j0 + r] = silu_f32(gsum) * usum;
+      if (i0 == 0 && p.has_shared) __threadfence();   // the down kernel reads the shared expert's a before its own wait
+    }
   };
+
 
   if (tid == 0) {
     for (int b = 0; b < kGuBufs; ++b) mbar_init(&bars[b], 1);
@@ -231,7 +298,8 @@ __global__ void __launch_bounds__(kThreads, 2) gateup_decode_kernel(GateUpParams
   }
   if (p.has_shared) arm(0);
   __syncthreads();
-  if (p.has_shared && warp < 6 && lane == 0) issue(0, warp);
+  if (p.has_shared && lane == 0)
+    for (int c = warp; c < ncp; c += kWarps) issue(0, c);
   // B tables of x, straight from registers
   {
     constexpr int EPT = TabTraits<BITS>::kEPT;
@@ -245,19 +313,12 @@ __global__ void __launch_bounds__(kThreads, 2) gateup_decode_kernel(GateUpParams
   }
   __syncthreads();
   int it0 = 0;
-  if (p.has_shared) {   // all warps: spans [nspans*w/16, nspans*(w+1)/16)
-    ok &= mbar_wait_bounded(&bars[0], 0, p.wait_ns, p.status);
-    float aa, ab;
-    compute(0, nspans * warp / kWarps, nspans * (warp + 1) / kWarps, aa, ab);
-    if ((lane & 3) == 0) { part[warp * 16 + (lane >> 2)] = aa; part[warp * 16 + 8 + (lane >> 2)] = ab; }
+  if (p.has_shared) {   // the shared expert, before the dependency wait
+    compute_items(0, 1);
     fence_proxy_async();
     __syncthreads();
-    if (tid < n) {
-      float gsum = 0.f, usum = 0.f;
-      for (int w = 0; w < kWarps; ++w) { gsum += part[w * 16 + tid]; usum += part[w * 16 + 8 + tid]; }
-      store_a(0, tid, gsum, usum);
-    }
-    __threadfence();   // the down kernel reads the shared expert's a before its own dependency wait
+    finalize(0, 1);
+    __syncthreads();   // ... so no thread signals the dependent launch before those stores are fenced
     it0 = 1;
   }
 
@@ -270,31 +331,17 @@ __global__ void __launch_bounds__(kThreads, 2) gateup_decode_kernel(GateUpParams
     if (p.idx_out) p.idx_out[(size_t)t * k + tid] = ts.idx[tid];
     if (p.w_out) p.w_out[(size_t)t * k + tid] = ts.w[tid];
   }
-  // routed items in waves of up to kGuBufs, each item on its own group of warps
+  // routed items in waves of up to kGuBufs; every warp takes its spans of all items of the wave
   for (int w0 = it0; w0 < nitems; w0 += kGuBufs) {
-    const int nw = nitems - w0 < kGuBufs ? nitems - w0 : kGuBufs;
-    for (int i = 0; i < nw; ++i) arm(w0 + i);
-    __syncthreads();   // slots loaded (first wave) / previous wave's buffers read
+    const int w1 = nitems - w0 < kGuBufs ? nitems : w0 + kGuBufs;
+    for (int it = w0; it < w1; ++it) arm(it);
+    __syncthreads();   // slots loaded (first wave) / previous wave's buffers and partial sums consumed
     if (lane == 0)
-      for (int c = warp; c < 6 * nw; c += kWarps) issue(w0 + c / 6, c % 6);
-    const int wi = warp * nw / kWarps;                       // this warp's item in the wave
-    const int wf = (wi * kWarps + nw - 1) / nw;               // first warp of that item
-    const int wc = ((wi + 1) * kWarps + nw - 1) / nw - wf;    // warps of that item
-    const int it = w0 + wi, r = warp - wf;
-    ok &= mbar_wait_bounded(&bars[it % kGuBufs], (unsigned)(it / kGuBufs) & 1u, p.wait_ns, p.status);
-    float aa, ab;
-    compute(it % kGuBufs, nspans * r / wc, nspans * (r + 1) / wc, aa, ab);
-    __syncthreads();   // part of the previous wave is consumed
-    if ((lane & 3) == 0) { part[warp * 16 + (lane >> 2)] = aa; part[warp * 16 + 8 + (lane >> 2)] = ab; }
+      for (int c = warp; c < ncp * (w1 - w0); c += kWarps) issue(w0 + c / ncp, c % ncp);
+    compute_items(w0, w1);
     fence_proxy_async();
     __syncthreads();
-    if (tid < nw * n) {
-      const int iw = tid / n, i = tid - iw * n;
-      const int f = (iw * kWarps + nw - 1) / nw, c = ((iw + 1) * kWarps + nw - 1) / nw - f;
-      float gsum = 0.f, usum = 0.f;
-      for (int w = f; w < f + c; ++w) { gsum += part[w * 16 + i]; usum += part[w * 16 + 8 + i]; }
-      store_a(w0 + iw, i, gsum, usum);
-    }
+    finalize(w0, w1);
   }
   if (!ok) {   // a copy never landed: give the copies in flight one more bound before leaving
     for (int it = (nitems > kGuBufs ? nitems - kGuBufs : 0); it < nitems; ++it)
@@ -307,15 +354,16 @@ constexpr int kDnBufs = 4;      // expert row blocks staged per CTA
 constexpr int kDnMaxRows = 32;  // hidden rows per CTA
 
 struct DnLayout {
-  int RB, SRB, SBR, GB, nsp, ng;
+  int RB, P, SRB, SBR, GB, nsp, ng;
   size_t buf, btab, gs, part, yacc, wsl, slots, topk, bars, total;
 };
 __host__ __device__ inline DnLayout dn_layout(int I, int S, int bits) {
   DnLayout L;
   L.RB = I * bits / 8;
+  L.P = L.RB;   // rows land contiguously (one bulk copy per row block)
   L.SRB = I / 32;
   L.SBR = sb_region(kDnMaxRows, L.SRB);
-  L.GB = (kDnMaxRows * L.RB + 2 * L.SBR + 127) & ~127;
+  L.GB = (kDnMaxRows * L.P + 2 * L.SBR + 127) & ~127;
   L.nsp = I / kSpan;
   L.ng = I / kGroup;
   const int nb = S < kDnBufs ? S : kDnBufs;
@@ -324,13 +372,13 @@ __host__ __device__ inline DnLayout dn_layout(int I, int S, int bits) {
   L.btab = o; o += sizeof(uint2) * (size_t)S * L.nsp * kBtPerSpan;
   L.gs = o; o += sizeof(float) * 2 * (size_t)S * L.ng;     // per slot [2^-p_g | X_g]
   o = (o + 15) & ~(size_t)15;
-  L.part = o; o += sizeof(float) * (size_t)nb * (kDnMaxRows / 16) * L.nsp * 16;
+  const size_t part = sizeof(float) * kWarps * (kDnMaxRows / 16) * 16;   // [segment][tile][16]
+  L.part = o; L.topk = o;   // the top-k scratch is dead before the partial sums are written
+  o += part > sizeof(TopkSmem) ? part : sizeof(TopkSmem);
   L.yacc = o; o += sizeof(float) * kDnMaxRows;
   L.wsl = o; o += sizeof(float) * kMaxSlots;
   o = (o + 15) & ~(size_t)15;
   L.slots = o; o += sizeof(moe_expert) * kMaxSlots;
-  o = (o + 15) & ~(size_t)15;
-  L.topk = o; o += sizeof(TopkSmem);
   o = (o + 15) & ~(size_t)15;
   L.bars = o; o += 8 * kDnBufs;
   L.total = o;
@@ -361,8 +409,8 @@ __global__ void __launch_bounds__(kThreads, 2) down_decode_kernel(DownParams p) 
   const int t = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = p.H, I = p.I, k = p.k, nsp = L.nsp, ng = L.ng;
   const int nb = S < kDnBufs ? S : kDnBufs;
-  const int h0 = (int)((long long)H * blockIdx.x / gridDim.x);
-  const int n = (int)((long long)H * (blockIdx.x + 1) / gridDim.x) - h0;
+  const int h0 = (int)((unsigned)H * blockIdx.x / gridDim.x);
+  const int n = (int)((unsigned)H * (blockIdx.x + 1) / gridDim.x) - h0;
   const int ntile = (n + 15) / 16;
   const int nitems = S;
   auto item_slot = [&](int it) { return p.has_shared ? (it == 0 ? S - 1 : it - 1) : it; };
@@ -370,10 +418,11 @@ __global__ void __launch_bounds__(kThreads, 2) down_decode_kernel(DownParams p) 
   const unsigned sbw = sb_window(h0, n, L.SRB, pre);
   const unsigned item_bytes = (unsigned)n * L.RB + 2u * sbw;
   const int per = nsp * kBtPerSpan;
-  const int ppart = (kDnMaxRows / 16) * nsp * 16;   // floats of part per item
   bool ok = true;
 
-  auto issue = [&](int it, int c) {   // c = 0 codes, 1 scales, 2 biases
+  // copies of item `it`, one per call: c = 0 code rows, 1 scales, 2 biases (row blocks)
+  const int ncp = 3;
+  auto issue = [&](int it, int c) {
     const int b = it % nb;
     unsigned char* buf = bufs + (size_t)b * L.GB;
     const moe_qmat& m = slot_ex[item_slot(it)].down;
@@ -382,8 +431,8 @@ __global__ void __launch_bounds__(kThreads, 2) down_decode_kernel(DownParams p) 
       bulk_g2s(buf, (const char*)m.q + (size_t)h0 * L.RB, (unsigned)n * L.RB, &bars[b]);
     } else {
       const uint16_t* src = c == 1 ? m.scales : m.biases;
-      bulk_g2s(buf + kDnMaxRows * L.RB + (c - 1) * L.SBR, (const char*)src + (((size_t)h0 * L.SRB) & ~(size_t)15),
-               sbw, &bars[b]);
+      bulk_g2s(buf + kDnMaxRows * L.P + (c - 1) * L.SBR, (const char*)src + (((size_t)h0 * L.SRB) & ~(size_t)15), sbw,
+               &bars[b]);
     }
   };
   // B tables of slots [sl0, sl1) from a
@@ -398,56 +447,96 @@ __global__ void __launch_bounds__(kThreads, 2) down_decode_kernel(DownParams p) 
       build_tables<BITS>(v, e, valid, btab + (size_t)(valid ? sl : 0) * per, gs + (size_t)(valid ? sl : 0) * 2 * ng, ng);
     }
   };
-  // unit u = (tile, span) of item it: row sums to pt[u][16]
-  auto unit = [&](int it, int u, float* pt) {
-    const int b = it % nb, slot = item_slot(it);
-    const unsigned char* buf = bufs + (size_t)b * L.GB;
-    const int g = lane >> 2, tq = lane & 3;
+  // MMAs of spans [s0, s1) of every row tile of item it, the span's B
+  // fragments loaded once for the tiles; row sums of tile tl, rows g / g+8
+  // to pt[tl][16] (quad-reduced). Lane tq of a quad loads 4 spans of one
+  // scale/bias row of each tile (tq = 0 scales of row r, 1 scales of row
+  // r+8, 2 biases of row r, 3 biases of row r+8); the quad shares them by
+  // shuffles.
+  constexpr int kTiles = kDnMaxRows / 16;
+  const bool al16 = L.SRB % 16 == 0;
+  auto seg_compute = [&](int it, int s0, int s1, float* pt) {
+    const int slot = item_slot(it);
+    const unsigned char* buf = bufs + (size_t)(it % nb) * L.GB;
+    const int g = lane >> 2, tq = lane & 3, qb = lane & ~3;
     const int bl = bt_lane_index(lane);
+    const LaneK K = lane_consts(tq);
     constexpr int SB = SpanBytes<BITS>::v;
-    constexpr int WB = QTraits<BITS>::kWordsPerThread * 4;
-    const int tile = u / nsp, s = u - tile * nsp;
-    const int r = tile * 16 + g;
-    Frag<BITS> F;
-    frag_codes<BITS>(F, buf + (size_t)r * L.RB + s * SB + tq * WB, buf + (size_t)(r + 8) * L.RB + s * SB + tq * WB);
-    const unsigned char* sc = buf + kDnMaxRows * L.RB + pre + s * 4;
-    F.sa = *(const uint32_t*)(sc + r * L.SRB);
-    F.sb = *(const uint32_t*)(sc + (r + 8) * L.SRB);
-    F.ba = *(const uint32_t*)(sc + L.SBR + r * L.SRB);
-    F.bb = *(const uint32_t*)(sc + L.SBR + (r + 8) * L.SRB);
-    int c[4];
-    mma_frag<BITS>(F, btab + (size_t)slot * per + s * kBtPerSpan, bl, c);
+    constexpr int W = QTraits<BITS>::kWordsPerThread;
+    const uint2* bt = btab + (size_t)slot * per;
     const float* gsl = gs + (size_t)slot * 2 * ng;
-    float acc_a = 0.f, acc_b = 0.f;
-    scale_frag_i(F.sa, F.sb, F.ba, F.bb, c, gsl, gsl + ng, s, tq, acc_a, acc_b);
-    acc_a += __shfl_xor_sync(0xffffffffu, acc_a, 1);
-    acc_b += __shfl_xor_sync(0xffffffffu, acc_b, 1);
-    acc_a += __shfl_xor_sync(0xffffffffu, acc_a, 2);
-    acc_b += __shfl_xor_sync(0xffffffffu, acc_b, 2);
-    if (tq == 0) { pt[u * 16 + g] = acc_a; pt[u * 16 + 8 + g] = acc_b; }
+    float aa[kTiles], ab[kTiles];
+    uint4 sv[kTiles];
+#pragma unroll
+    for (int tl = 0; tl < kTiles; ++tl) { aa[tl] = 0.f; ab[tl] = 0.f; sv[tl] = make_uint4(0u, 0u, 0u, 0u); }
+    for (int s = s0; s < s1; ++s) {
+      BFrag B;
+      load_bfrag(B, bt + s * kBtPerSpan, bl, gsl, ng, s, tq);
+#pragma unroll
+      for (int tl = 0; tl < kTiles; ++tl) {
+        if (tl < ntile) {
+          const int r = tl * 16 + g;
+          if (s == s0 || (s & 3) == 0)
+            sv[tl] = lds_chunk(buf + kDnMaxRows * L.P + pre + (tq >> 1) * L.SBR + (r + 8 * (tq & 1)) * L.SRB +
+                                   16 * (s >> 2), al16);
+          const uint32_t w = chunk_word(sv[tl], s & 3);
+          uint32_t wa[W], wb[W];
+          const unsigned char* ra = buf + (size_t)r * L.P + s * SB + tq * W * 4;
+          const unsigned char* rb = ra + (size_t)8 * L.P;
+          if constexpr (W == 4) {
+            const uint4 va = *(const uint4*)ra, vb = *(const uint4*)rb;
+            wa[0] = va.x; wa[1] = va.y; wa[2] = va.z; wa[3] = va.w;
+            wb[0] = vb.x; wb[1] = vb.y; wb[2] = vb.z; wb[3] = vb.w;
+          } else {
+            const uint2 va = *(const uint2*)ra, vb = *(const uint2*)rb;
+            wa[0] = va.x; wa[1] = va.y;
+            wb[0] = vb.x; wb[1] = vb.y;
+          }
+          const uint32_t sa = __shfl_sync(0xffffffffu, w, qb), sb = __shfl_sync(0xffffffffu, w, qb + 1);
+          const uint32_t ba = __shfl_sync(0xffffffffu, w, qb + 2), bb = __shfl_sync(0xffffffffu, w, qb + 3);
+          tile_span<BITS>(wa, wb, sa, sb, ba, bb, B, K, aa[tl], ab[tl]);
+        }
+      }
+    }
+#pragma unroll
+    for (int tl = 0; tl < kTiles; ++tl) {
+      if (tl < ntile) {
+        float a = aa[tl], b = ab[tl];
+        a += __shfl_xor_sync(0xffffffffu, a, 1);
+        b += __shfl_xor_sync(0xffffffffu, b, 1);
+        a += __shfl_xor_sync(0xffffffffu, a, 2);
+        b += __shfl_xor_sync(0xffffffffu, b, 2);
+        if (tq == 0) { pt[tl * 16 + g] = a; pt[tl * 16 + 8 + g] = b; }
+      }
+    }
   };
-  // items [i0, i1) (all staged): units spread over the warps, then yacc += w * y
+  // items [i0, i1) (all staged): segments (item, span part) spread over the
+  // warps, each covering all row tiles; then, in item order, yacc += w * y
   auto run = [&](int i0, int i1) {
-    const int U = ntile * nsp, UT = (i1 - i0) * U;
+    const int ni = i1 - i0;
+    int nsplit = kWarps / ni;
+    nsplit = nsplit < 1 ? 1 : (nsplit > nsp ? nsp : nsplit);
+    const int nseg = ni * nsplit;
     int waited = -1;
-    for (int x = UT * warp / kWarps; x < UT * (warp + 1) / kWarps; ++x) {
-      const int it = i0 + x / U;
+    for (int sg = warp; sg < nseg; sg += kWarps) {
+      const int itr = sg / nsplit, pr = sg - itr * nsplit;
+      const int it = i0 + itr;
       if (it != waited) {
         ok &= mbar_wait_bounded(&bars[it % nb], (unsigned)(it / nb) & 1u, p.wait_ns, p.status);
         waited = it;
       }
-      unit(it, x - (it - i0) * U, part + (size_t)(it % nb) * ppart);
+      seg_compute(it, nsp * pr / nsplit, nsp * (pr + 1) / nsplit, part + (size_t)sg * kTiles * 16);
     }
     fence_proxy_async();
     __syncthreads();
     if (tid < n) {
-      const int tile = tid >> 4, rr = tid & 15;
+      const int tl = tid >> 4, rr = tid & 15;
       float acc = yacc[tid];
-      for (int it = i0; it < i1; ++it) {
-        const float* pt = part + (size_t)(it % nb) * ppart;
+      for (int itr = 0; itr < ni; ++itr) {
+        const float* pt = part + (size_t)itr * nsplit * kTiles * 16 + tl * 16 + rr;
         float y = 0.f;
-        for (int s = 0; s < nsp; ++s) y += pt[(tile * nsp + s) * 16 + rr];
-        acc = fmaf(wsl[item_slot(it)], y, acc);
+        for (int pr = 0; pr < nsplit; ++pr) y += pt[pr * kTiles * 16];
+        acc = fmaf(wsl[item_slot(i0 + itr)], y, acc);
       }
       yacc[tid] = acc;
     }
@@ -466,7 +555,7 @@ __global__ void __launch_bounds__(kThreads, 2) down_decode_kernel(DownParams p) 
   if (tid < n) yacc[tid] = __ldcg(p.h + (size_t)t * H + h0 + tid);
   __syncthreads();
   if (lane == 0)
-    for (int c = warp; c < 3 * nb; c += kWarps) issue(c / 3, c % 3);
+    for (int c = warp; c < ncp * nb; c += kWarps) issue(c / ncp, c % ncp);
   int issued = nb;   // items [0, issued) have their copies in flight or landed
   int it0 = 0;
   if (p.has_shared) {   // the shared expert's a is final: apply it before the wait
@@ -487,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 2) down_decode_kernel(DownParams p) 
         for (int it = issued; it < w1; ++it) mbar_expect_tx(&bars[it % nb], item_bytes);
       __syncthreads();
       if (lane == 0)
-        for (int c = warp; c < 3 * (w1 - issued); c += kWarps) issue(issued + c / 3, c % 3);
+        for (int c = warp; c < ncp * (w1 - issued); c += kWarps) issue(issued + c / ncp, c % ncp);
       issued = w1;
     }
     run(w0, w1);

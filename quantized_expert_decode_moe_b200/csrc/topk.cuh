@@ -18,8 +18,8 @@ namespace qmoe {
 constexpr int kTopkPer = 8;   // logits per thread: E <= kTopkPer * blockDim
 
 struct TopkSmem {
-  unsigned long long ck[kWarps][kMaxTopK];   // candidate keys
-  int ce[kWarps][kMaxTopK];                  // candidate expert ids
+  unsigned long long ck[kWarps * kMaxTopK];   // candidate keys, [warp * k + round]
+  int ce[kWarps * kMaxTopK];                  // candidate expert ids
   int idx[kMaxTopK];
   float w[kMaxTopK];
   float sg;
@@ -59,80 +59,98 @@ __device__ __forceinline__ int warp_best(unsigned long long key, int id, unsigne
   return wl;
 }
 
+// Merge by warp 0 of the warps' candidates ts.ck/ce [nw][k], then the
+// weights and the shared gate (lane 0 holds gl).
+__device__ __forceinline__ void topk_merge(int k, int nw, int has_shared, float gl, TopkSmem& ts) {
+  const int lane = threadIdx.x & 31, nc = nw * k;
+  // each lane's candidates c = lane + 32q, sorted best first (keys desc, ids asc)
+  unsigned long long ck[4];
+  int ci[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int c = lane + 32 * q;
+    ck[q] = c < nc ? ts.ck[c] : 0ull;
+    ci[q] = c < nc ? ts.ce[c] : -1;
+  }
+  auto cx = [&](int a, int b) {   // compare-exchange: better one to a
+    const bool sw = ck[b] > ck[a] || (ck[b] == ck[a] && ck[a] && (unsigned)ci[b] < (unsigned)ci[a]);
+    if (sw) {
+      const unsigned long long tk = ck[a]; ck[a] = ck[b]; ck[b] = tk;
+      const int ti = ci[a]; ci[a] = ci[b]; ci[b] = ti;
+    }
+  };
+  cx(0, 1); cx(2, 3); cx(0, 2); cx(1, 3); cx(1, 2);
+  unsigned long long mine = 0ull, first = 0ull;
+  int mid = -1;
+  for (int r = 0; r < k; ++r) {
+    unsigned long long wk;
+    int wi;
+    const int wl = warp_best(ck[0], ci[0], wk, wi);
+    if (lane == wl) {
+      ck[0] = ck[1]; ci[0] = ci[1]; ck[1] = ck[2]; ci[1] = ci[2]; ck[2] = ck[3]; ci[2] = ci[3];
+      ck[3] = 0ull; ci[3] = -1;
+    }
+    if (r == 0) first = wk;
+    if (lane == r) { mine = wk; mid = wk ? wi : -1; }
+  }
+  const float ex = (lane < k && mine) ? expf((float)(key_value(mine) - key_value(first))) : 0.f;
+  const float z = warp_sum(ex);
+  if (lane < k) { ts.idx[lane] = mid; ts.w[lane] = ex / z; }
+  if (lane == 0) ts.sg = has_shared ? 1.f / (1.f + expf(-gl)) : 0.f;
+}
+
 // Block-wide top-k of lg[0..E) (+ shared gate from lg[E] when has_shared),
 // global memory written by an earlier kernel. All threads of the block call
 // it (blockDim = 32 * kWarps); results in ts, valid after the call, which ends
 // with __syncthreads. Ids of missing entries (all logits NaN) are -1.
-__device__ __noinline__ static void block_topk(const double* lg, int E, int k, int has_shared, TopkSmem& ts) {
+// k <= 8 and (candidates per warp) * warps <= 128.
+__device__ __forceinline__ void block_topk(const double* lg, int E, int k, int has_shared, TopkSmem& ts) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nt = blockDim.x;
-  unsigned long long key[kTopkPer];
-#pragma unroll
-  for (int j = 0; j < kTopkPer; ++j) {
-    const int e = tid + j * nt;
-    key[j] = e < E ? order_key(__ldcg(lg + e)) : 0ull;
-  }
   float gl = 0.f;
-  if (warp == 0 && lane == 0 && has_shared) gl = (float)__ldcg(lg + E);
-  // this thread's best (lowest index among equal keys: j ascending, strict >)
-  auto local_best = [&](unsigned long long& bk, int& bj) {
-    bk = 0ull; bj = 0;
+  if (E <= nt) {   // one logit per thread
+    unsigned long long key = tid < E ? order_key(__ldcg(lg + tid)) : 0ull;
+    if (warp == 0 && lane == 0 && has_shared) gl = (float)__ldcg(lg + E);
+    for (int r = 0; r < k; ++r) {
+      unsigned long long wk;
+      int wi;
+      const int wl = warp_best(key, tid, wk, wi);
+      if (lane == wl) key = 0ull;
+      if (lane == 0) { ts.ck[warp * k + r] = wk; ts.ce[warp * k + r] = wk ? wi : -1; }
+    }
+  } else {
+    unsigned long long key[kTopkPer];
 #pragma unroll
-    for (int j = 0; j < kTopkPer; ++j)
-      if (key[j] > bk) { bk = key[j]; bj = j; }
-  };
-  unsigned long long bk;
-  int bj;
-  local_best(bk, bj);
-  for (int r = 0; r < k; ++r) {
-    unsigned long long wk;
-    int wi;
-    const int wl = warp_best(bk, tid + bj * nt, wk, wi);
-    if (lane == 0) { ts.ck[warp][r] = wk; ts.ce[warp][r] = wk ? wi : -1; }
-    if (lane == wl && wk) {
+    for (int j = 0; j < kTopkPer; ++j) {
+      const int e = tid + j * nt;
+      key[j] = e < E ? order_key(__ldcg(lg + e)) : 0ull;
+    }
+    if (warp == 0 && lane == 0 && has_shared) gl = (float)__ldcg(lg + E);
+    // this thread's best (lowest index among equal keys: j ascending, strict >)
+    auto local_best = [&](unsigned long long& bk, int& bj) {
+      bk = 0ull; bj = 0;
 #pragma unroll
       for (int j = 0; j < kTopkPer; ++j)
-        if (j == bj) key[j] = 0ull;
-      local_best(bk, bj);
+        if (key[j] > bk) { bk = key[j]; bj = j; }
+    };
+    unsigned long long bk;
+    int bj;
+    local_best(bk, bj);
+    for (int r = 0; r < k; ++r) {
+      unsigned long long wk;
+      int wi;
+      const int wl = warp_best(bk, tid + bj * nt, wk, wi);
+      if (lane == 0) { ts.ck[warp * k + r] = wk; ts.ce[warp * k + r] = wk ? wi : -1; }
+      if (lane == wl && wk) {
+#pragma unroll
+        for (int j = 0; j < kTopkPer; ++j)
+          if (j == bj) key[j] = 0ull;
+        local_best(bk, bj);
+      }
     }
   }
   __syncthreads();
-  if (warp == 0) {
-    const int nw = nt >> 5, nc = nw * k;
-    unsigned long long ck[4];
-    int ce[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int c = lane + 32 * q, w = c / k, r = c - w * k;
-      const bool ok = c < nc;
-      ck[q] = ok ? ts.ck[w][r] : 0ull;
-      ce[q] = ok ? ts.ce[w][r] : -1;
-    }
-    unsigned long long mine = 0ull, first = 0ull;
-    int mid = -1;
-    for (int r = 0; r < k; ++r) {
-      unsigned long long b = 0ull;
-      int bq = 0, bid = -1;
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        if (ck[q] > b || (ck[q] == b && b && (unsigned)ce[q] < (unsigned)bid)) { b = ck[q]; bq = q; bid = ce[q]; }
-      unsigned long long wk;
-      int wi;
-      const int wl = warp_best(b, bid, wk, wi);
-      if (lane == wl && wk) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          if (q == bq) { ck[q] = 0ull; ce[q] = -1; }
-      }
-      if (r == 0) first = wk;
-      if (lane == r) { mine = wk; mid = wk ? wi : -1; }
-    }
-    // weights over the chosen k
-    const float ex = (lane < k && mine) ? expf((float)(key_value(mine) - key_value(first))) : 0.f;
-    const float z = warp_sum(ex);
-    if (lane < k) { ts.idx[lane] = mid; ts.w[lane] = ex / z; }
-    if (lane == 0) ts.sg = has_shared ? 1.f / (1.f + expf(-gl)) : 0.f;
-  }
+  if (warp == 0) topk_merge(k, nt >> 5, has_shared, gl, ts);
   __syncthreads();
 }
 
