@@ -200,10 +200,9 @@ __global__ void __launch_bounds__(kThreads, 2) gateup_decode_kernel(GateUpParams
   // copies of item `it` into buffer it % kGuBufs, one per call: c = 0 gate
   // code rows, 1 up code rows (row blocks), 2..5 gate/up scales, gate/up biases
   const int ncp = 6;
-  auto issue = [&](int it, int c) {
+  auto issue_ex = [&](const moe_expert& ex, int it, int c) {
     const int b = it % kGuBufs;
     unsigned char* buf = bufs + (size_t)b * L.GB;
-    const moe_expert& ex = slot_ex[item_slot(it)];
     fence_proxy_async();
     if (c < 2) {
       const moe_qmat& m = c == 0 ? ex.gate : ex.up;
@@ -216,6 +215,7 @@ __global__ void __launch_bounds__(kThreads, 2) gateup_decode_kernel(GateUpParams
                &bars[b]);
     }
   };
+  auto issue = [&](int it, int c) { issue_ex(slot_ex[item_slot(it)], it, c); };
   // MMAs of this warp's spans [nspans*w/16, nspans*(w+1)/16) for the items
   // [i0, i1) (at most kGuBufs, each one 16-row tile in buffer it % kGuBufs):
   // the B fragments of a span are loaded once for all items. Lane tq of a
@@ -296,10 +296,13 @@ __global__ void __launch_bounds__(kThreads, 2) gateup_decode_kernel(GateUpParams
     fence_mbar_init();
     if (p.has_shared) slot_ex[S - 1] = p.shared;
   }
-  if (p.has_shared) arm(0);
-  __syncthreads();
-  if (p.has_shared && lane == 0)
-    for (int c = warp; c < ncp; c += kWarps) issue(0, c);
+  if (p.has_shared) {   // the shared expert's copies go out first, from the kernel parameters
+    arm(0);
+    if (warp < ncp) {
+      asm volatile("bar.sync 1, %0;" :: "r"(ncp * 32) : "memory");   // barriers initialised (warps 0..ncp-1)
+      if (lane == 0) issue_ex(p.shared, 0, warp);
+    }
+  }
   // B tables of x, straight from registers
   {
     constexpr int EPT = TabTraits<BITS>::kEPT;

@@ -75,12 +75,13 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
 }
 
 // ------------------------------------------------------------------ router logits
-// grid (ceil(rows / 4), T), block 256: two warps per router row (row E = the
-// shared-expert gate), each over one half of H; every lane keeps its 16-byte
-// chunks of the row in registers.
-constexpr int kRouteRows = 4;
-constexpr int kRouteThreads = kRouteRows * 2 * 32;
-constexpr int kRouteChunks = 8;   // 16-byte weight chunks per lane per pass
+// grid (ceil(rows / 2), T), block 256: four warps per router row (row E = the
+// shared-expert gate), each over one quarter of H; every lane keeps its
+// 16-byte chunks of the row in registers.
+constexpr int kRouteRows = 2;
+constexpr int kRouteSplit = 4;
+constexpr int kRouteThreads = kRouteRows * kRouteSplit * 32;
+constexpr int kRouteChunks = 4;   // 16-byte weight chunks per lane per pass
 
 // s + c += x with the rounding error of the addition kept in c (Knuth's TwoSum).
 __device__ __forceinline__ void two_sum_acc(float& s, float& c, float x) {
@@ -108,14 +109,14 @@ __device__ __forceinline__ void dot8_bf16_comp(uint4 w, uint4 x, float (&s)[4], 
 __global__ void __launch_bounds__(kRouteThreads) route_logits_kernel(RouteParams p) {
   extern __shared__ __align__(128) unsigned char smem[];
   uint4* xs = (uint4*)smem;                                  // [H/8]
-  __shared__ float part[kRouteRows][2];
+  __shared__ float part[kRouteRows][kRouteSplit][2];
   const int t = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nch = p.H / 8, half = nch / 2;
+  const int nch = p.H / 8, half = nch / kRouteSplit;   // chunks per warp's part of the row
   const int nrows = p.E + (p.has_shared ? 1 : 0);
-  const int rl = warp >> 1, hs = warp & 1;
+  const int rl = warp / kRouteSplit, hs = warp % kRouteSplit;
   const int e = blockIdx.x * kRouteRows + rl;
   const uint16_t* wrow = e < p.E ? p.router_w + (size_t)e * p.H : p.gate_w;
-  const int cb = hs * half;   // first chunk of this warp's half
+  const int cb = hs * half;   // first chunk of this warp's part
   float cs[4] = {0.f, 0.f, 0.f, 0.f}, cc[4] = {0.f, 0.f, 0.f, 0.f};
   for (int c0 = 0; c0 < half; c0 += 32 * kRouteChunks) {
     uint4 wv[kRouteChunks];
@@ -166,11 +167,14 @@ __global__ void __launch_bounds__(kRouteThreads) route_logits_kernel(RouteParams
     ac_ += oc;
     two_sum_acc(as_, ac_, os);
   }
-  if (lane == 0 && hs == 1) { part[rl][0] = as_; part[rl][1] = ac_; }
+  if (lane == 0 && hs != 0) { part[rl][hs][0] = as_; part[rl][hs][1] = ac_; }
   __syncthreads();
   if (lane == 0 && hs == 0 && e < nrows) {
-    ac_ += part[rl][1];
-    two_sum_acc(as_, ac_, part[rl][0]);
+#pragma unroll
+    for (int q = 1; q < kRouteSplit; ++q) {
+      ac_ += part[rl][q][1];
+      two_sum_acc(as_, ac_, part[rl][q][0]);
+    }
     double acc = (double)as_ + (double)ac_;
     if (e < p.E && p.router_bias) acc += (double)p.router_bias[e];
     p.logits[(size_t)t * (p.E + 1) + e] = acc;
