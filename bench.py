@@ -139,7 +139,7 @@ def build_workload(cfg, copies, dev):
 
 def kernel_src_sha():
     h = hashlib.sha256()
-    for f in ("common.cuh", "kernels.cu", "kernels.cuh", "api.cu"):
+    for f in ("common.cuh", "kernels.cu", "kernels.cuh", "api.cu", "decode.cu", "topk.cuh"):
         p = os.path.join(ROOT, "quantized_expert_decode_moe_b200", "csrc", f)
         if os.path.exists(p):
             h.update(open(p, "rb").read())
