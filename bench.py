@@ -224,6 +224,22 @@ def reference_arm(args, cfg):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ replicas
+def max_over_ranks(value: float, dist, device) -> float:
+    """The slowest rank's time: every rank contributes its own, all get the max."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, steps_per_rank: int, ms: float) -> float:
+    """Whole-job tokens/s: every rank decodes steps_per_rank tokens in ms (the max over ranks)."""
+    return world * steps_per_rank / (ms * 1e-3)
+
+
 # ------------------------------------------------------------------ our arm
 def ours(args, cfg):
     import numpy as np
@@ -302,11 +318,7 @@ def ours(args, cfg):
     if dist:
         dist.barrier()
     clk = clocks.stop()
-    ms = e0.elapsed_time(e1)
-    if dist:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
     assert qm.moe_poll_status(ws, stream) == 0
 
     # per-kernel durations (events between the kernels, no overlap)
@@ -353,16 +365,12 @@ def ours(args, cfg):
             outh[i:i + 1].copy_(odev, non_blocking=True)
         f1.record(stream)
     f1.synchronize()
-    e2e_ms = f0.elapsed_time(f1)
-    if dist:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1), dist, dev)
 
     peaks, peak_kind = measured_peaks()
     active = cfg.active_bytes_per_token                      # expert bytes per token (4 experts)
     router_bytes = cfg.E * cfg.H * 2
-    tok_s = world * args.steps / (ms * 1e-3)
+    tok_s = job_throughput(world, args.steps, ms)
     per_tok_s = args.steps / (ms * 1e-3)
     gbs = active * per_tok_s / 1e9
     # dominant kernel: the gate/up dequant GEMV, 2/3 of the expert bytes
@@ -389,7 +397,7 @@ def ours(args, cfg):
         "roofline": {"bound": "hbm", "kernel": names[j_dom], "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
                      "algorithmic_bytes": dom_bytes, "peak_kind": peak_kind},
-        "e2e": {"value": world * e2e_n / (e2e_ms * 1e-3), "unit": UNIT, "steps": e2e_n,
+        "e2e": {"value": job_throughput(world, e2e_n, e2e_ms), "unit": UNIT, "steps": e2e_n,
                 "h2d_bytes_per_step": cfg.H * 2 + cfg.H * 4, "d2h_bytes_per_step": cfg.H * 2},
         "gpu_launches": 4 * args.steps,
         "clocks": clk,
