@@ -134,6 +134,56 @@ moe_status decode_chain(const moe_layer* L, const uint16_t* x_in, float* h, int 
   return MOE_OK;
 }
 
+// Prefill (T > 8): router logits for all tokens, top-k, grouping of the
+// (token, rank) pairs by expert, grouped dequant GEMMs (gate/up + SwiGLU,
+// then down) on the fp16 tensor cores, combine + residual + RMSNorm.
+moe_status prefill_chain(const moe_layer* L, const uint16_t* x_in, float* h, int T, uint16_t* x_out,
+                         float* x_out_f32, int32_t* topk_idx, float* topk_w, void* ws, cudaStream_t s,
+                         void* const* events = nullptr) {
+  auto mark = [&](int i) { if (events) cudaEventRecord((cudaEvent_t)events[i], s); };
+  mark(0);
+  const int H = L->hidden, I = L->inter, E = L->n_experts, k = L->top_k;
+  const WsLayout W = layout_of(L, T);
+  uint32_t* status = at<uint32_t>(ws, W.status);
+  RouteParams rp{};
+  rp.H = H; rp.E = E; rp.T = T; rp.has_shared = L->has_shared;
+  rp.x = x_in; rp.router_w = L->router_w; rp.router_bias = L->router_bias; rp.gate_w = L->shared_gate_w;
+  rp.logits = at<double>(ws, W.logits);
+  cudaError_t e = launch_route(rp, s, false);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  mark(1);
+  TopkParams tp{};
+  tp.E = E; tp.k = k; tp.T = T; tp.has_shared = L->has_shared;
+  tp.logits = rp.logits; tp.idx = at<int32_t>(ws, W.pidx); tp.w = at<float>(ws, W.pw); tp.sg = at<float>(ws, W.psg);
+  if ((e = launch_topk(tp, s)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (topk_idx && cudaMemcpyAsync(topk_idx, tp.idx, sizeof(int32_t) * (size_t)T * k, cudaMemcpyDeviceToDevice, s))
+    return MOE_ERR_CUDA;
+  if (topk_w && cudaMemcpyAsync(topk_w, tp.w, sizeof(float) * (size_t)T * k, cudaMemcpyDeviceToDevice, s))
+    return MOE_ERR_CUDA;
+  GroupParams gp{};
+  gp.T = T; gp.k = k; gp.E = E; gp.idx = tp.idx;
+  gp.counts = at<int32_t>(ws, W.counts); gp.offsets = at<int32_t>(ws, W.offsets); gp.perm = at<int32_t>(ws, W.perm);
+  if ((e = launch_group(gp, s)) != cudaSuccess) return MOE_ERR_CUDA;
+  mark(2);
+  PrefillParams pp{};
+  pp.H = H; pp.I = I; pp.E = E; pp.k = k; pp.T = T; pp.has_shared = L->has_shared;
+  pp.x = x_in; pp.xh = at<__half>(ws, W.xh); pp.a16 = at<__half>(ws, W.a16); pp.y = at<float>(ws, W.y);
+  pp.offsets = gp.offsets; pp.perm = gp.perm; pp.experts = L->experts; pp.shared = L->shared;
+  pp.status = status; pp.wait_ns = wait_bound_ns();
+  if ((e = launch_prefill(pp, L->bits, s)) != cudaSuccess) return MOE_ERR_CUDA;
+  mark(3);
+  NormParams np{};
+  np.H = H; np.k = k; np.T = T;
+  np.y_routed = pp.y; np.y_routed_tok_stride = (long long)k * H; np.y_routed_slot_stride = H;
+  np.w = tp.w;
+  np.y_shared = L->has_shared ? pp.y + (size_t)T * k * H : nullptr; np.y_shared_tok_stride = H;
+  np.sg = tp.sg;
+  np.h = h; np.gamma = L->rms_gamma; np.eps = L->rms_eps; np.x_out = x_out; np.x_out_f32 = x_out_f32;
+  if ((e = launch_norm(np, false, s)) != cudaSuccess) return MOE_ERR_CUDA;
+  mark(4);
+  return MOE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -247,7 +297,8 @@ moe_status moe_layer_forward(const moe_layer* layer, const uint16_t* x_in, float
   if (T <= 0 || !x_in || !h || !x_out) return MOE_ERR_INVALID_ARGUMENT;
   if (!aligned16(x_in) || !aligned16(h) || !aligned16(x_out)) return MOE_ERR_INVALID_ARGUMENT;
   if ((st = ws_check(layer, T, ws, ws_bytes))) return st;
-  if (T > kDecodeMaxT) return MOE_ERR_UNSUPPORTED;
+  if (T > kDecodeMaxT)
+    return prefill_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, (cudaStream_t)stream);
   return decode_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, (cudaStream_t)stream);
 }
 
@@ -259,10 +310,11 @@ moe_status moe_layer_forward_timed(const moe_layer* layer, const uint16_t* x_in,
   if (T <= 0 || !x_in || !h || !x_out) return MOE_ERR_INVALID_ARGUMENT;
   if (!aligned16(x_in) || !aligned16(h) || !aligned16(x_out)) return MOE_ERR_INVALID_ARGUMENT;
   if ((st = ws_check(layer, T, ws, ws_bytes))) return st;
-  if (T > kDecodeMaxT) return MOE_ERR_UNSUPPORTED;
   if (!events || n_events < 5) return MOE_ERR_INVALID_ARGUMENT;
   for (int i = 0; i < 5; ++i)
     if (!events[i]) return MOE_ERR_INVALID_ARGUMENT;
+  if (T > kDecodeMaxT)
+    return prefill_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, (cudaStream_t)stream, events);
   return decode_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, (cudaStream_t)stream, events);
 }
 

@@ -26,6 +26,13 @@ WsLayout ws_layout(int H, int I, int E, int k, int S, int T) {
   L.counts = o; o = align256(o + sizeof(int32_t) * (size_t)E);
   L.offsets = o; o = align256(o + sizeof(int32_t) * (size_t)(E + 1));
   L.perm = o; o = align256(o + sizeof(int32_t) * (size_t)T * k);
+  L.pidx = o; o = align256(o + sizeof(int32_t) * (size_t)T * k);
+  L.pw = o; o = align256(o + sizeof(float) * (size_t)T * k);
+  L.psg = o; o = align256(o + sizeof(float) * (size_t)T);
+  const size_t prows = T > 8 ? (size_t)T * k + T : 0;   // the prefill buffers exist only for T > 8
+  L.xh = o; o = align256(o + (T > 8 ? sizeof(uint16_t) * (size_t)T * H : 0));
+  L.a16 = o; o = align256(o + sizeof(uint16_t) * prows * I);
+  L.y = o; o = align256(o + sizeof(float) * prows * H);
   L.total = o;
   return L;
 }

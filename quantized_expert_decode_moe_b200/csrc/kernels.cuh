@@ -1,6 +1,7 @@
 // Kernel parameter blocks and launchers of the quantized MoE expert forward.
 #pragma once
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -18,6 +19,12 @@ struct WsLayout {
   size_t counts;      // int32 [E]
   size_t offsets;     // int32 [E+1]
   size_t perm;        // int32 [T*k]
+  size_t pidx;        // int32 [T][k]   routed expert ids
+  size_t pw;          // float [T][k]   routing weights
+  size_t psg;         // float [T]      shared-expert gate
+  size_t xh;          // fp16 [T][H]    activations for the tensor cores
+  size_t a16;         // fp16 [T*k + T][I]  SwiGLU outputs per pair (t*k + r), then per token (shared)
+  size_t y;           // float [T*k + T][H] expert outputs, same rows
   size_t total;
 };
 WsLayout ws_layout(int H, int I, int E, int k, int S, int T);
@@ -88,6 +95,20 @@ struct GemvParams {
   unsigned long long wait_ns;
 };
 
+struct PrefillParams {
+  int H, I, E, k, T, has_shared;
+  const uint16_t* x;           // [T][H] bf16
+  __half* xh;                  // [T][H]
+  __half* a16;                 // [T*k + T][I]
+  float* y;                    // [T*k + T][H]
+  const int32_t* offsets;      // [E+1]
+  const int32_t* perm;         // [T*k]
+  const moe_expert* experts;
+  moe_expert shared;
+  uint32_t* status;
+  unsigned long long wait_ns;
+};
+
 struct GroupParams {
   int T, k, E;
   const int32_t* idx;
@@ -107,6 +128,7 @@ int gateup_ctas(int I);
 int down_ctas(int H);
 cudaError_t launch_gemv(const GemvParams& p, int bits, cudaStream_t s);
 cudaError_t launch_group(const GroupParams& p, cudaStream_t s);
+cudaError_t launch_prefill(const PrefillParams& p, int bits, cudaStream_t s);
 int num_sms();
 int choose_ncta(long long ntiles, int nspans);
 

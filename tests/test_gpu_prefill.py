@@ -1,0 +1,109 @@
+"""GPU parity of the prefill path (T > 8 tokens: grouping by expert, grouped
+dequant GEMMs on the fp16 tensor cores, combine + residual + RMSNorm) against
+the CPU oracle, through moe_layer_forward.
+
+Routing ids bit-exact for every token; h and x_out within max relative error
+2e-3 (max|gpu - oracle| / max|oracle|) per token; bf16 x_out within one ulp
+of the oracle's rounding or the normwise bar.
+"""
+import numpy as np
+import pytest
+import torch
+
+import fixtures
+import fixtures.gpu as fxg
+import oracle
+import quantized_expert_decode_moe_b200 as qm
+from fixtures import gen
+from refs import oracle_tokens, rel_err
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-3
+
+
+def _np16(t):
+    return t.cpu().numpy().view(np.uint16)
+
+
+def _check_bf16(xb, ref, ref_b):
+    ulp = np.abs(xb.astype(np.int32) - ref_b.astype(np.int32))
+    close = np.abs(gen.bf16_bits_to_f32(xb).astype(np.float64) - ref) <= TOL * np.max(np.abs(ref))
+    assert np.all((ulp <= 1) | close)
+
+
+def _run(cfg, layer, x_bits, dev):
+    T = x_bits.shape[0]
+    ws = qm.new_workspace(layer, T)
+    xo = torch.empty((T, cfg.H), dtype=torch.int16, device=dev)
+    xf = torch.empty((T, cfg.H), dtype=torch.float32, device=dev)
+    idx = torch.empty((T, cfg.k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, cfg.k), dtype=torch.float32, device=dev)
+    h0 = gen.bf16_bits_to_f32(x_bits).astype(np.float32)
+    h = torch.from_numpy(h0.copy()).to(dev)
+    qm.moe_layer_forward(layer, torch.from_numpy(x_bits.view(np.int16)).to(dev), h, xo, xf, idx, w, ws=ws)
+    assert qm.moe_poll_status(ws) == 0
+    return h0, idx.cpu().numpy(), w.cpu().numpy(), h.cpu().numpy(), xf.cpu().numpy(), _np16(xo)
+
+
+def _compare(cfg, x_bits, h0, idx, w, h, xf, xo, sample):
+    ref = oracle_tokens(cfg, 0, x_bits[sample], h0[sample].astype(np.float64))
+    np.testing.assert_array_equal(idx[sample], ref["idx"])
+    np.testing.assert_allclose(w[sample], ref["w"], rtol=1e-6, atol=1e-7)
+    worst = 0.0
+    for n, i in enumerate(sample):
+        eh, ex = rel_err(h[i], ref["h_out"][n]), rel_err(xf[i], ref["x_out"][n])
+        assert eh <= TOL and ex <= TOL, (i, eh, ex)
+        np.testing.assert_array_equal(xo[i], gen.f32_to_bf16_bits(xf[i]))
+        _check_bf16(xo[i], ref["x_out"][n], ref["x_out_bf16"][n])
+        worst = max(worst, eh, ex)
+    print(f"{cfg.name} prefill T={x_bits.shape[0]}: max rel err {worst:.3e} over {len(sample)} tokens")
+    return worst
+
+
+@pytest.fixture(scope="module")
+def dev():
+    assert torch.cuda.is_available()
+    qm.lib()
+    return torch.device("cuda")
+
+
+@pytest.mark.parametrize("T", [9, 40])
+def test_prefill_tiny_matches_oracle(dev, T):
+    cfg = fixtures.CONFIGS["tiny"]
+    t = fxg.device_layer(cfg, 0)
+    layer = qm.layer_from_tensors(cfg, t)
+    x = gen.x_tokens(cfg, 21, T=T)
+    out = _run(cfg, layer, x, dev)
+    _compare(cfg, x, *out, sample=list(range(T)))
+
+
+@pytest.mark.parametrize("bits,shared", [(2, True), (4, False)])
+def test_prefill_small_layers(dev, bits, shared):
+    cfg = fixtures.Config(f"pf{bits}{'s' if shared else 'n'}", H=512, E=24, k=3, I=256, bits=bits,
+                          scale_sigma=0.05 if bits == 2 else 0.02, has_shared=shared)
+    t = fxg.device_layer(cfg, 0)
+    layer = qm.layer_from_tensors(cfg, t)
+    x = gen.x_tokens(cfg, 4, T=33)
+    out = _run(cfg, layer, x, dev)
+    _compare(cfg, x, *out, sample=list(range(33)))
+
+
+def test_prefill_full_size_512_tokens(dev):
+    """The 512-token prefill of the 4-bit layer (hidden 4096, 512 experts,
+    top-3 + shared): routing of all 512 tokens bit-exact, outputs of a
+    sample of tokens (regenerating every expert the whole batch touches on
+    the host is too slow for a test)."""
+    cfg = fixtures.CONFIGS["prefill_q4"]
+    t = fxg.device_layer(cfg, 0)
+    layer = qm.layer_from_tensors(cfg, t)
+    x = gen.x_tokens(cfg, 0, T=cfg.T)
+    h0, idx, w, h, xf, xo = _run(cfg, layer, x, dev)
+    Wr, rb, gs, _ = fixtures.layer_vectors(cfg, 0)
+    ridx, rw, _ = oracle.route(x, Wr, cfg.k, bias=rb, gs=gs)
+    np.testing.assert_array_equal(idx, ridx)
+    np.testing.assert_allclose(w, rw, rtol=1e-6, atol=1e-7)
+    assert len(np.unique(idx)) > 400   # the batch touches most of the 512 experts
+    sample = [0, 1, 2, 63, 64, 200, 255, 256, 300, 447, 510, 511]
+    _compare(cfg, x, h0, idx, w, h, xf, xo, sample=sample)
+    del t, layer
+    torch.cuda.empty_cache()
