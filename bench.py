@@ -39,7 +39,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=120000)
     ap.add_argument("--warmup", type=int, default=480)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="layer_q4", choices=["layer_q4", "layer_q2"])
+    ap.add_argument("--config", default="layer_q4", choices=["layer_q4", "layer_q2", "prefill_q4"],
+                    help="prefill_q4: one step = one 512-token forward of the layer (the prefill path)")
     ap.add_argument("--copies", type=int, default=48)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -415,12 +416,123 @@ def ours(args, cfg):
         dist.destroy_process_group()
 
 
+# ------------------------------------------------------------------ prefill arm (--config prefill_q4)
+def ours_prefill(args, cfg):
+    import numpy as np
+    import torch
+
+    import fixtures.gpu as fxg
+    import quantized_expert_decode_moe_b200 as qm
+    from fixtures import gen
+
+    world, rank, local = dist_info()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    qm.lib()
+    t = fxg.device_layer(cfg, 0, dev)
+    layer = qm.layer_from_tensors(cfg, t)
+    T, NB = cfg.T, 4
+    xs_host = [gen.x_tokens(cfg, 100 + b, T=T) for b in range(NB)]
+    xs = [torch.from_numpy(x.view(np.int16)).to(dev) for x in xs_host]
+    hs = [torch.from_numpy(gen.bf16_bits_to_f32(x).astype(np.float32)).to(dev) for x in xs_host]
+    ws = qm.new_workspace(layer, T)
+    xo = torch.empty((T, cfg.H), dtype=torch.int16, device=dev)
+    idx = torch.empty((NB, T, cfg.k), dtype=torch.int32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        for b in range(NB):   # eager pass (lazy attributes), and the routing of every batch
+            qm.moe_layer_forward(layer, xs[b], hs[b].clone(), xo, None, idx[b], None, ws=ws, stream=stream)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for b in range(NB):
+                qm.moe_layer_forward(layer, xs[b], hs[b], xo, ws=ws, stream=stream)
+    steps = max(NB, (args.steps // NB) * NB)
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 3) // NB + 1):
+            g.replay()
+    stream.synchronize()
+    assert qm.moe_poll_status(ws, stream) == 0
+    gpu_uuid = str(getattr(torch.cuda.get_device_properties(dev), "uuid", "") or "")
+    clocks = Clocks(("GPU-" + gpu_uuid) if gpu_uuid and not gpu_uuid.startswith("GPU-") else (gpu_uuid or str(local)))
+    clocks.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(steps // NB):
+            g.replay()
+        e1.record(stream)
+    e1.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    assert qm.moe_poll_status(ws, stream) == 0
+    # stages, timed one by one: router, top-k + grouping, gate/up, down, combine + norm
+    nst, reps = 5, 8
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for _ in range(reps)]
+    with torch.cuda.stream(stream):
+        for row in evs:
+            for e in row:
+                e.record(stream)
+        for r in range(reps):
+            qm.moe_layer_forward_timed(layer, xs[r % NB], hs[r % NB], xo, ws=ws, events=evs[r], stream=stream)
+    stream.synchronize()
+    names = ["route_logits", "topk+group", "gateup_grouped", "down_grouped", "combine_norm"]
+    dur = [sum(evs[r][j].elapsed_time(evs[r][j + 1]) for r in range(reps)) / reps for j in range(nst)]
+    # end to end with host buffers: x, h in; x_out back, every step
+    xh = torch.from_numpy(np.stack(xs_host).view(np.int16)).pin_memory()
+    hh = torch.stack([h.cpu() for h in hs]).pin_memory()
+    outh = torch.empty((T, cfg.H), dtype=torch.int16).pin_memory()
+    xd = torch.empty((T, cfg.H), dtype=torch.int16, device=dev)
+    hd = torch.empty((T, cfg.H), dtype=torch.float32, device=dev)
+    e2e_n = min(steps, 32)
+    with torch.cuda.stream(stream):
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for i in range(e2e_n):
+            xd.copy_(xh[i % NB], non_blocking=True)
+            hd.copy_(hh[i % NB], non_blocking=True)
+            qm.moe_layer_forward(layer, xd, hd, xo, ws=ws, stream=stream)
+            outh.copy_(xo, non_blocking=True)
+        f1.record(stream)
+    f1.synchronize()
+    e2e_ms = f0.elapsed_time(f1)
+    peaks, peak_kind = measured_peaks()
+    touched = [len(np.unique(idx[b].cpu().numpy())) for b in range(NB)]
+    bytes_mat = cfg.I * cfg.H * cfg.bits // 8 + 2 * 2 * cfg.I * (cfg.H // cfg.G)   # one matrix: codes, scales, biases
+    gu_bytes = (np.mean(touched) + 1) * 2 * bytes_mat + 2 * T * cfg.H * 2
+    flops = 2.0 * (T * cfg.k + T) * 3 * cfg.H * cfg.I
+    achieved = gu_bytes / (dur[2] * 1e-3) / 1e9
+    line = {
+        "metric": "MoE-layer prefill tokens/s (512-token batch), 4-bit experts, 1 B200", "value": T * steps / (ms * 1e-3),
+        "unit": "tokens/s", "n_gpus": world, "steps": steps, "warmup": max(args.warmup, 3),
+        "ms_per_step": ms / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "u4 codes dequantised to f16, f16 tensor-core MMA, f32 accumulate",
+        "data": "synthetic (seeded; no model weights)",
+        "config": {"workload": cfg.note, "H": cfg.H, "E": cfg.E, "top_k": cfg.k, "I": cfg.I, "bits": cfg.bits,
+                   "T": T, "experts_touched_per_step": float(np.mean(touched)),
+                   "l2": "inputs larger than L2: every step streams the ~3.3 GB of touched experts"},
+        "stage_ms": dict(zip(names, dur)),
+        "tflops": flops / (ms / steps * 1e-3) / 1e12,
+        "roofline": {"bound": "hbm", "kernel": "gateup_grouped", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "algorithmic_bytes": gu_bytes, "peak_kind": peak_kind},
+        "e2e": {"value": T * e2e_n / (e2e_ms * 1e-3), "unit": "tokens/s", "steps": e2e_n,
+                "h2d_bytes_per_step": T * cfg.H * (2 + 4), "d2h_bytes_per_step": T * cfg.H * 2},
+        "gpu_launches": 7 * steps, "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     import fixtures
     cfg = fixtures.CONFIGS[args.config]
     if args.impl == "reference":
         reference_arm(args, cfg)
+    elif cfg.T > 1:
+        ours_prefill(args, cfg)
     else:
         ours(args, cfg)
 

@@ -178,8 +178,10 @@ moe_status moe_stack_forward(const moe_layer* layers, int32_t L, const uint16_t*
  * recorded before the first and after each of the kernels of the layer, so a
  * caller can time them one by one. events: host array of n_events created
  * cudaEvent_t handles (passed as void*); n_events must be at least the number
- * of kernels of the chosen path + 1 (decode: 5). The kernels run without
- * programmatic overlap between them. Same arguments and errors otherwise.
+ * of recorded stages + 1: decode (T <= 8) 5 (router, gate/up, down, norm);
+ * prefill 6 (router, top-k + grouping, gate/up, down, combine + norm). The
+ * kernels run without programmatic overlap between them. Same arguments and
+ * errors otherwise.
  */
 moe_status moe_layer_forward_timed(const moe_layer* layer, const uint16_t* x_in, float* h, int32_t T,
                                    uint16_t* x_out, float* x_out_f32, int32_t* topk_idx, float* topk_w,

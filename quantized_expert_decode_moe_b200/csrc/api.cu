@@ -170,8 +170,10 @@ moe_status prefill_chain(const moe_layer* L, const uint16_t* x_in, float* h, int
   pp.x = x_in; pp.xh = at<__half>(ws, W.xh); pp.a16 = at<__half>(ws, W.a16); pp.y = at<float>(ws, W.y);
   pp.offsets = gp.offsets; pp.perm = gp.perm; pp.experts = L->experts; pp.shared = L->shared;
   pp.status = status; pp.wait_ns = wait_bound_ns();
-  if ((e = launch_prefill(pp, L->bits, s)) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((e = launch_prefill_gateup(pp, L->bits, s)) != cudaSuccess) return MOE_ERR_CUDA;
   mark(3);
+  if ((e = launch_prefill_down(pp, L->bits, s)) != cudaSuccess) return MOE_ERR_CUDA;
+  mark(4);
   NormParams np{};
   np.H = H; np.k = k; np.T = T;
   np.y_routed = pp.y; np.y_routed_tok_stride = (long long)k * H; np.y_routed_slot_stride = H;
@@ -180,7 +182,7 @@ moe_status prefill_chain(const moe_layer* L, const uint16_t* x_in, float* h, int
   np.sg = tp.sg;
   np.h = h; np.gamma = L->rms_gamma; np.eps = L->rms_eps; np.x_out = x_out; np.x_out_f32 = x_out_f32;
   if ((e = launch_norm(np, false, s)) != cudaSuccess) return MOE_ERR_CUDA;
-  mark(4);
+  mark(5);
   return MOE_OK;
 }
 
@@ -310,8 +312,9 @@ moe_status moe_layer_forward_timed(const moe_layer* layer, const uint16_t* x_in,
   if (T <= 0 || !x_in || !h || !x_out) return MOE_ERR_INVALID_ARGUMENT;
   if (!aligned16(x_in) || !aligned16(h) || !aligned16(x_out)) return MOE_ERR_INVALID_ARGUMENT;
   if ((st = ws_check(layer, T, ws, ws_bytes))) return st;
-  if (!events || n_events < 5) return MOE_ERR_INVALID_ARGUMENT;
-  for (int i = 0; i < 5; ++i)
+  const int need = T > kDecodeMaxT ? 6 : 5;   // kernels (or kernel groups) of the path + 1
+  if (!events || n_events < need) return MOE_ERR_INVALID_ARGUMENT;
+  for (int i = 0; i < need; ++i)
     if (!events[i]) return MOE_ERR_INVALID_ARGUMENT;
   if (T > kDecodeMaxT)
     return prefill_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, (cudaStream_t)stream, events);

@@ -128,7 +128,8 @@ int gateup_ctas(int I);
 int down_ctas(int H);
 cudaError_t launch_gemv(const GemvParams& p, int bits, cudaStream_t s);
 cudaError_t launch_group(const GroupParams& p, cudaStream_t s);
-cudaError_t launch_prefill(const PrefillParams& p, int bits, cudaStream_t s);
+cudaError_t launch_prefill_gateup(const PrefillParams& p, int bits, cudaStream_t s);   // activations to fp16 + gate/up
+cudaError_t launch_prefill_down(const PrefillParams& p, int bits, cudaStream_t s);
 int num_sms();
 int choose_ncta(long long ntiles, int nspans);
 

@@ -305,31 +305,29 @@ static cudaError_t pf_prepare(const void* fn, size_t bytes) {
   return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
-cudaError_t launch_prefill(const PrefillParams& p, int bits, cudaStream_t s) {
+cudaError_t launch_prefill_gateup(const PrefillParams& p, int bits, cudaStream_t s) {
   PrefillParams q = p;
   void* args[] = {&q};
   const int groups = p.E + (p.has_shared ? 1 : 0);
-  {
-    const size_t n = (size_t)p.T * p.H;
-    to_f16_kernel<<<(unsigned)((n + 1023) / 1024 < 4096 ? (n + 1023) / 1024 : 4096), 1024, 0, s>>>(p.x, p.xh, n);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
-  {
-    const size_t sm = pf_layout(p.H, bits).total;
-    const void* fn = bits == 4 ? (const void*)prefill_gateup_kernel<4> : (const void*)prefill_gateup_kernel<2>;
-    cudaError_t e = pf_prepare(fn, sm);
-    if (e != cudaSuccess) return e;
-    if ((e = cudaLaunchKernel(fn, dim3(p.I / 8, groups), dim3(kPfThreads), args, sm, s)) != cudaSuccess) return e;
-  }
-  {
-    const size_t sm = pf_layout(p.I, bits).total;
-    const void* fn = bits == 4 ? (const void*)prefill_down_kernel<4> : (const void*)prefill_down_kernel<2>;
-    cudaError_t e = pf_prepare(fn, sm);
-    if (e != cudaSuccess) return e;
-    if ((e = cudaLaunchKernel(fn, dim3(p.H / 16, groups), dim3(kPfThreads), args, sm, s)) != cudaSuccess) return e;
-  }
-  return cudaSuccess;
+  const size_t n = (size_t)p.T * p.H;
+  to_f16_kernel<<<(unsigned)((n + 1023) / 1024 < 4096 ? (n + 1023) / 1024 : 4096), 1024, 0, s>>>(p.x, p.xh, n);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t sm = pf_layout(p.H, bits).total;
+  const void* fn = bits == 4 ? (const void*)prefill_gateup_kernel<4> : (const void*)prefill_gateup_kernel<2>;
+  if ((e = pf_prepare(fn, sm)) != cudaSuccess) return e;
+  return cudaLaunchKernel(fn, dim3(p.I / 8, groups), dim3(kPfThreads), args, sm, s);
+}
+
+cudaError_t launch_prefill_down(const PrefillParams& p, int bits, cudaStream_t s) {
+  PrefillParams q = p;
+  void* args[] = {&q};
+  const int groups = p.E + (p.has_shared ? 1 : 0);
+  const size_t sm = pf_layout(p.I, bits).total;
+  const void* fn = bits == 4 ? (const void*)prefill_down_kernel<4> : (const void*)prefill_down_kernel<2>;
+  cudaError_t e = pf_prepare(fn, sm);
+  if (e != cudaSuccess) return e;
+  return cudaLaunchKernel(fn, dim3(p.H / 16, groups), dim3(kPfThreads), args, sm, s);
 }
 
 }  // namespace qmoe
