@@ -65,22 +65,9 @@ __device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1,
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Two consecutive codes (elements k, k+1; k even) of a packed row as an exact
-// fp16 pair, from the row's bytes `rb` (4-bit: one byte; 2-bit: two fields
-// of one byte).
-template <int BITS>
-__device__ __forceinline__ uint32_t code_pair(const unsigned char* rb, int k) {
-  uint32_t lo, hi;
-  if constexpr (BITS == 4) {
-    const uint32_t b = rb[k >> 1];
-    lo = b & 0xFu;
-    hi = b >> 4;
-  } else {
-    const uint32_t b = rb[k >> 2] >> (2 * (k & 3));
-    lo = b & 3u;
-    hi = (b >> 2) & 3u;
-  }
-  // 0x6400 is fp16 1024: (1024 + q) - 1024 = q exactly
+// Two codes (lo, hi in 0..15) as an exact fp16 pair: 0x6400 is fp16 1024,
+// (1024 + q) - 1024 = q exactly.
+__device__ __forceinline__ uint32_t codes_h2(uint32_t lo, uint32_t hi) {
   const uint32_t v = 0x64006400u | lo | (hi << 16);
   const __half2 q = __hsub2(*(const __half2*)&v, __halves2half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400)));
   return *(const uint32_t*)&q;
@@ -115,24 +102,55 @@ __host__ __device__ inline PfLayout pf_layout(int K, int bits) {
 }
 
 // Accumulates, for the rows of the block (rows 0-15 of `codes`) and up to 64
-// tokens, the warp's K-slice [k0, k1) into acc[tile][4]; B operands come from
-// `act` (fp16 [*][K], row of token i = act + row_of[i] * K).
+// tokens, the warp's K-slice [k0, k1) (multiples of 16) into acc[tile][4]; B
+// operands come from `act` (fp16 [*][K], row of token i = act + row_of[i] * K).
+// Codes are read once per 64 columns: lane t of a quad loads one quarter of
+// its row's bytes for those columns and the quad shares them by shuffles.
 template <int BITS>
 __device__ __forceinline__ void pf_block_mma(const unsigned char* codes, const uint16_t* sc, const uint16_t* bi,
                                              int K, const __half* act, const int* row_of, int ntok, int k0, int k1,
                                              float (&acc)[kPfTiles][4]) {
-  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3, qb = lane & ~3;
   const int RB = K * BITS / 8, ng = K / kGroup;
   const unsigned char* ra = codes + (size_t)g * RB;
   const unsigned char* rb = codes + (size_t)(g + 8) * RB;
+  constexpr int CB = 64 * BITS / 8 / 4;   // bytes per lane per 64 columns: 8 (4-bit) or 4 (2-bit)
+  uint2 ca = make_uint2(0u, 0u), cb = make_uint2(0u, 0u);
+  __half2 sa, ba, sb, bb;
   for (int k = k0; k < k1; k += 16) {
-    const int grp = k / kGroup;
-    const __half2 sa = bf16_to_h2(sc[g * ng + grp]), ba = bf16_to_h2(bi[g * ng + grp]);
-    const __half2 sb = bf16_to_h2(sc[(g + 8) * ng + grp]), bb = bf16_to_h2(bi[(g + 8) * ng + grp]);
-    const uint32_t a0 = deq_pair(code_pair<BITS>(ra, k + 2 * t), sa, ba);
-    const uint32_t a1 = deq_pair(code_pair<BITS>(rb, k + 2 * t), sb, bb);
-    const uint32_t a2 = deq_pair(code_pair<BITS>(ra, k + 8 + 2 * t), sa, ba);
-    const uint32_t a3 = deq_pair(code_pair<BITS>(rb, k + 8 + 2 * t), sb, bb);
+    if (k == k0 || (k & 63) == 0) {
+      const int grp = k / kGroup;
+      sa = bf16_to_h2(sc[g * ng + grp]); ba = bf16_to_h2(bi[g * ng + grp]);
+      sb = bf16_to_h2(sc[(g + 8) * ng + grp]); bb = bf16_to_h2(bi[(g + 8) * ng + grp]);
+    }
+    const int kc = k & ~63;   // first column of this 64-column chunk
+    if (k == k0 || (k & 63) == 0) {
+      const int off = kc * BITS / 8 + CB * t;
+      if constexpr (BITS == 4) { ca = *(const uint2*)(ra + off); cb = *(const uint2*)(rb + off); }
+      else { ca.x = *(const uint32_t*)(ra + off); cb.x = *(const uint32_t*)(rb + off); }
+    }
+    const int st = (k - kc) >> 4;   // step inside the chunk: its bytes are held by quad lane st
+    uint32_t a0, a1, a2, a3;
+    if constexpr (BITS == 4) {
+      // step bytes [8 st, 8 st + 8): lo word -> columns k..k+7, hi word -> k+8..k+15; lane t takes byte t
+      const uint32_t la = __shfl_sync(0xffffffffu, ca.x, qb + st) >> (8 * t);
+      const uint32_t ha = __shfl_sync(0xffffffffu, ca.y, qb + st) >> (8 * t);
+      const uint32_t lb = __shfl_sync(0xffffffffu, cb.x, qb + st) >> (8 * t);
+      const uint32_t hb = __shfl_sync(0xffffffffu, cb.y, qb + st) >> (8 * t);
+      a0 = deq_pair(codes_h2(la & 0xFu, (la >> 4) & 0xFu), sa, ba);
+      a1 = deq_pair(codes_h2(lb & 0xFu, (lb >> 4) & 0xFu), sb, bb);
+      a2 = deq_pair(codes_h2(ha & 0xFu, (ha >> 4) & 0xFu), sa, ba);
+      a3 = deq_pair(codes_h2(hb & 0xFu, (hb >> 4) & 0xFu), sb, bb);
+    } else {
+      // step bytes [4 st, 4 st + 4): columns k + 4i .. k + 4i + 3 in byte i; lane t needs columns 2t, 2t+1
+      // (byte t>>1, fields 2(t&1), +1) and 8+2t, 9+2t (byte 2 + (t>>1))
+      const uint32_t wa = __shfl_sync(0xffffffffu, ca.x, qb + st), wb = __shfl_sync(0xffffffffu, cb.x, qb + st);
+      const int s0 = 8 * (t >> 1) + 4 * (t & 1), s1 = s0 + 16;
+      a0 = deq_pair(codes_h2((wa >> s0) & 3u, (wa >> (s0 + 2)) & 3u), sa, ba);
+      a1 = deq_pair(codes_h2((wb >> s0) & 3u, (wb >> (s0 + 2)) & 3u), sb, bb);
+      a2 = deq_pair(codes_h2((wa >> s1) & 3u, (wa >> (s1 + 2)) & 3u), sa, ba);
+      a3 = deq_pair(codes_h2((wb >> s1) & 3u, (wb >> (s1 + 2)) & 3u), sb, bb);
+    }
 #pragma unroll
     for (int nt = 0; nt < kPfTiles; ++nt) {
       if (nt * 8 < ntok) {
@@ -200,14 +218,15 @@ __global__ void __launch_bounds__(kPfThreads) prefill_gateup_kernel(PrefillParam
   if (tid == 0) {
     pf_mbar_init(bar);
     pf_expect(bar, 2u * 8 * RB + 4u * 8 * SRB);
-    pf_bulk(codes, (const char*)ex.gate.q + (size_t)j0 * RB, 8u * RB, bar);
-    pf_bulk(codes + (size_t)8 * RB, (const char*)ex.up.q + (size_t)j0 * RB, 8u * RB, bar);
-    pf_bulk(sc, (const char*)ex.gate.scales + (size_t)j0 * SRB, 8u * SRB, bar);
-    pf_bulk((char*)sc + 8 * SRB, (const char*)ex.up.scales + (size_t)j0 * SRB, 8u * SRB, bar);
-    pf_bulk(bi, (const char*)ex.gate.biases + (size_t)j0 * SRB, 8u * SRB, bar);
-    pf_bulk((char*)bi + 8 * SRB, (const char*)ex.up.biases + (size_t)j0 * SRB, 8u * SRB, bar);
   }
   __syncthreads();
+  if ((tid & 31) == 0 && warp < 6) {   // one copy per warp: gate/up codes, scales, biases (8-row blocks)
+    const moe_qmat& m = (warp & 1) ? ex.up : ex.gate;
+    const int half = warp & 1;
+    if (warp < 2) pf_bulk(codes + (size_t)half * 8 * RB, (const char*)m.q + (size_t)j0 * RB, 8u * RB, bar);
+    else if (warp < 4) pf_bulk((char*)sc + half * 8 * SRB, (const char*)m.scales + (size_t)j0 * SRB, 8u * SRB, bar);
+    else pf_bulk((char*)bi + half * 8 * SRB, (const char*)m.biases + (size_t)j0 * SRB, 8u * SRB, bar);
+  }
   pf_wait(bar, p.wait_ns, p.status);
   const int ks = H / kPfWarps;   // K-slice per warp (multiple of 16)
   for (int pass = 0; pass < G.n; pass += kPfTokens) {
@@ -262,11 +281,13 @@ __global__ void __launch_bounds__(kPfThreads) prefill_down_kernel(PrefillParams 
   if (tid == 0) {
     pf_mbar_init(bar);
     pf_expect(bar, 16u * RB + 2u * 16 * SRB);
-    pf_bulk(codes, (const char*)ex.down.q + (size_t)h0 * RB, 16u * RB, bar);
-    pf_bulk(sc, (const char*)ex.down.scales + (size_t)h0 * SRB, 16u * SRB, bar);
-    pf_bulk(bi, (const char*)ex.down.biases + (size_t)h0 * SRB, 16u * SRB, bar);
   }
   __syncthreads();
+  if ((tid & 31) == 0 && warp < 3) {   // one copy per warp: codes, scales, biases (16-row blocks)
+    if (warp == 0) pf_bulk(codes, (const char*)ex.down.q + (size_t)h0 * RB, 16u * RB, bar);
+    else if (warp == 1) pf_bulk(sc, (const char*)ex.down.scales + (size_t)h0 * SRB, 16u * SRB, bar);
+    else pf_bulk(bi, (const char*)ex.down.biases + (size_t)h0 * SRB, 16u * SRB, bar);
+  }
   pf_wait(bar, p.wait_ns, p.status);
   const int ks = I / kPfWarps;
   for (int pass = 0; pass < G.n; pass += kPfTokens) {
