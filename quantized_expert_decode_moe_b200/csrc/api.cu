@@ -135,8 +135,9 @@ moe_status decode_chain(const moe_layer* L, const uint16_t* x_in, float* h, int 
 }
 
 // Prefill (T > 8): router logits for all tokens, top-k, grouping of the
-// (token, rank) pairs by expert, grouped dequant GEMMs (gate/up + SwiGLU,
-// then down) on the fp16 tensor cores, combine + residual + RMSNorm.
+// (token, rank) pairs by expert into chunks, grouped GEMMs (gate/up + SwiGLU,
+// then down) of the packed codes against fixed-point activation digits on the
+// integer tensor cores, combine + residual + RMSNorm.
 moe_status prefill_chain(const moe_layer* L, const uint16_t* x_in, float* h, int T, uint16_t* x_out,
                          float* x_out_f32, int32_t* topk_idx, float* topk_w, void* ws, cudaStream_t s,
                          void* const* events = nullptr) {
@@ -161,18 +162,26 @@ moe_status prefill_chain(const moe_layer* L, const uint16_t* x_in, float* h, int
   if (topk_w && cudaMemcpyAsync(topk_w, tp.w, sizeof(float) * (size_t)T * k, cudaMemcpyDeviceToDevice, s))
     return MOE_ERR_CUDA;
   GroupParams gp{};
-  gp.T = T; gp.k = k; gp.E = E; gp.idx = tp.idx;
+  gp.T = T; gp.k = k; gp.E = E; gp.has_shared = L->has_shared; gp.chunk = pf_chunk_tokens(H, I); gp.idx = tp.idx;
   gp.counts = at<int32_t>(ws, W.counts); gp.offsets = at<int32_t>(ws, W.offsets); gp.perm = at<int32_t>(ws, W.perm);
+  gp.chunks = at<int4>(ws, W.chunks); gp.nchunks = at<int32_t>(ws, W.nchunks);
   if ((e = launch_group(gp, s)) != cudaSuccess) return MOE_ERR_CUDA;
   mark(2);
   PrefillParams pp{};
   pp.H = H; pp.I = I; pp.E = E; pp.k = k; pp.T = T; pp.has_shared = L->has_shared;
-  pp.x = x_in; pp.xh = at<__half>(ws, W.xh); pp.a16 = at<__half>(ws, W.a16); pp.y = at<float>(ws, W.y);
-  pp.offsets = gp.offsets; pp.perm = gp.perm; pp.experts = L->experts; pp.shared = L->shared;
+  pp.x = x_in;
+  pp.xd = at<unsigned char>(ws, W.xd); pp.xX = at<float>(ws, W.xX); pp.xrs = at<float>(ws, W.xrs);
+  pp.a = at<float>(ws, W.a);
+  pp.ad = at<unsigned char>(ws, W.ad); pp.aX = at<float>(ws, W.aX); pp.ars = at<float>(ws, W.ars);
+  pp.y = at<float>(ws, W.y);
+  pp.chunks = gp.chunks; pp.nchunks = gp.nchunks; pp.perm = gp.perm;
+  pp.experts = L->experts; pp.shared = L->shared;
   pp.status = status; pp.wait_ns = wait_bound_ns();
-  if ((e = launch_prefill_gateup(pp, L->bits, s)) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((e = launch_prefill_gateup(pp, L->bits, s)) != cudaSuccess)
+    return e == cudaErrorInvalidConfiguration ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
   mark(3);
-  if ((e = launch_prefill_down(pp, L->bits, s)) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((e = launch_prefill_down(pp, L->bits, s)) != cudaSuccess)
+    return e == cudaErrorInvalidConfiguration ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
   mark(4);
   NormParams np{};
   np.H = H; np.k = k; np.T = T;

@@ -30,8 +30,15 @@ WsLayout ws_layout(int H, int I, int E, int k, int S, int T) {
   L.pw = o; o = align256(o + sizeof(float) * (size_t)T * k);
   L.psg = o; o = align256(o + sizeof(float) * (size_t)T);
   const size_t prows = T > 8 ? (size_t)T * k + T : 0;   // the prefill buffers exist only for T > 8
-  L.xh = o; o = align256(o + (T > 8 ? sizeof(uint16_t) * (size_t)T * H : 0));
-  L.a16 = o; o = align256(o + sizeof(uint16_t) * prows * I);
+  const size_t trows = T > 8 ? (size_t)T : 0;
+  L.xd = o; o = align256(o + 2 * trows * H);
+  L.xX = o; o = align256(o + sizeof(float) * trows * (H / kGroup));
+  L.xrs = o; o = align256(o + sizeof(float) * trows);
+  L.ad = o; o = align256(o + 2 * prows * I);
+  L.aX = o; o = align256(o + sizeof(float) * prows * (I / kGroup));
+  L.ars = o; o = align256(o + sizeof(float) * prows);
+  L.chunks = o; o = align256(o + (T > 8 ? sizeof(int4) * pf_max_chunks(T, k, E, pf_chunk_tokens(H, I)) : 0));
+  L.nchunks = o; o = align256(o + (T > 8 ? sizeof(int32_t) : 0));
   L.y = o; o = align256(o + sizeof(float) * prows * H);
   L.total = o;
   return L;
@@ -390,59 +397,81 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GemvParams p) {
 }
 
 // ------------------------------------------------------------------ grouping by expert
-// One CTA: histogram, exclusive scan, then a stable scatter by one warp that
-// walks the pairs in order 32 at a time (ranks of equal experts inside a chunk
-// from __match_any_sync).
+// Exclusive scan of v[0..n) in place (one block); returns the total.
+__device__ int block_exclusive_scan(int* v, int n, int* warp_tot) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  int carry = 0;
+  for (int base = 0; base < n; base += blockDim.x) {
+    const int e = base + tid;
+    const int x = e < n ? v[e] : 0;
+    int incl = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      int wv = lane < nw ? warp_tot[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, wv, o);
+        if (lane >= o) wv += y;
+      }
+      if (lane < nw) warp_tot[lane] = wv;
+    }
+    __syncthreads();
+    if (e < n) v[e] = carry + (warp ? warp_tot[warp - 1] : 0) + incl - x;
+    const int tot = warp_tot[nw - 1];
+    __syncthreads();
+    carry += tot;
+  }
+  return carry;
+}
+
+// Prefill grouping in one CTA: histogram of the chosen experts, exclusive
+// scan, then a stable scatter of the flattened (token, rank) pairs by one warp
+// that walks them in order 32 at a time (ranks of equal experts from
+// __match_any_sync). Also the chunk list of the grouped GEMMs: expert e's
+// pairs in runs of `chunk`, then the shared expert's tokens in runs of `chunk`.
 __global__ void __launch_bounds__(1024) group_kernel(GroupParams p) {
   extern __shared__ __align__(128) unsigned char smem[];
   int* cnt = (int*)smem;            // [E]
   int* fill = cnt + p.E;            // [E]
+  int* cb = fill + p.E;             // [E] first chunk of each expert
   __shared__ int warp_tot[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int N = p.T * p.k;
-  for (int e = tid; e < p.E; e += blockDim.x) { cnt[e] = 0; fill[e] = 0; }
+  const int N = p.T * p.k, C = p.chunk;
+  for (int e = tid; e < p.E; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
   for (int i = tid; i < N; i += blockDim.x) {
     const int e = p.idx[i];
     if (e >= 0 && e < p.E) atomicAdd(&cnt[e], 1);
   }
   __syncthreads();
-  // exclusive scan of cnt into fill (blockDim-wide chunks)
-  int carry = 0;
-  for (int base = 0; base < p.E; base += blockDim.x) {
-    const int e = base + tid;
-    const int v = e < p.E ? cnt[e] : 0;
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int n = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += n;
-    }
-    if (lane == 31) warp_tot[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-      const int nw = blockDim.x >> 5;
-      int wv = lane < nw ? warp_tot[lane] : 0;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, wv, o);
-        if (lane >= o) wv += n;
-      }
-      if (lane < nw) warp_tot[lane] = wv;
-    }
-    __syncthreads();
-    const int wbase = warp ? warp_tot[warp - 1] : 0;
-    const int excl = carry + wbase + incl - v;
-    if (e < p.E) {
-      fill[e] = excl;
-      p.counts[e] = v;
-      p.offsets[e] = excl;
-    }
-    const int tot = warp_tot[(blockDim.x >> 5) - 1];
-    __syncthreads();
-    carry += tot;
+  for (int e = tid; e < p.E; e += blockDim.x) {
+    p.counts[e] = cnt[e];
+    fill[e] = cnt[e];
+    cb[e] = C > 0 ? (cnt[e] + C - 1) / C : 0;
   }
-  if (tid == 0) p.offsets[p.E] = carry;
+  __syncthreads();
+  const int total = block_exclusive_scan(fill, p.E, warp_tot);
+  const int nrouted = block_exclusive_scan(cb, p.E, warp_tot);
+  const bool chunked = p.chunks != nullptr && p.nchunks != nullptr && C > 0;   // the grouped GEMMs' list
+  for (int e = tid; e < p.E; e += blockDim.x) {
+    p.offsets[e] = fill[e];
+    if (chunked)
+      for (int c = 0; c * C < cnt[e]; ++c)
+        p.chunks[cb[e] + c] = make_int4(e, fill[e] + c * C, min(C, cnt[e] - c * C), 0);
+  }
+  const int nshared = chunked && p.has_shared ? (p.T + C - 1) / C : 0;
+  for (int c = tid; c < nshared; c += blockDim.x)
+    p.chunks[nrouted + c] = make_int4(p.E, c * C, min(C, p.T - c * C), 0);
+  if (tid == 0) {
+    p.offsets[p.E] = total;
+    if (chunked) *p.nchunks = nrouted + nshared;
+  }
   __syncthreads();
   if (warp == 0) {
     for (int base = 0; base < N; base += 32) {
@@ -548,8 +577,15 @@ cudaError_t launch_gemv(const GemvParams& p, int bits, cudaStream_t s) {
   return launch_ex(fn, dim3(p.nCTA), dim3(kThreads), sm, s, false, args);
 }
 
+size_t pf_max_chunks(int T, int k, int E, int chunk) {
+  // sum over experts of ceil(n_e / chunk) <= min(T*k, T*k / chunk + E), plus the shared expert's
+  const size_t pairs = (size_t)T * k;
+  const size_t routed = pairs / chunk + (size_t)E < pairs ? pairs / chunk + (size_t)E : pairs;
+  return routed + ((size_t)T + chunk - 1) / chunk;
+}
+
 cudaError_t launch_group(const GroupParams& p, cudaStream_t s) {
-  const size_t sm = sizeof(int) * 2 * (size_t)p.E;
+  const size_t sm = sizeof(int) * 3 * (size_t)p.E;
   cudaError_t e = set_smem((const void*)group_kernel, sm);
   if (e != cudaSuccess) return e;
   GroupParams q = p;

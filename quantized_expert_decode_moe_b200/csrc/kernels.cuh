@@ -22,8 +22,12 @@ struct WsLayout {
   size_t pidx;        // int32 [T][k]   routed expert ids
   size_t pw;          // float [T][k]   routing weights
   size_t psg;         // float [T]      shared-expert gate
-  size_t xh;          // fp16 [T][H]    activations for the tensor cores
-  size_t a16;         // fp16 [T*k + T][I]  SwiGLU outputs per pair (t*k + r), then per token (shared)
+  size_t xd;          // u8 [T][2H]     digit tables of x (+ xX float [T][H/64], xrs float [T])
+  size_t xX, xrs;
+  size_t ad;          // u8 [T*k + T][2I]  digit tables of the SwiGLU outputs (+ aX, ars)
+  size_t aX, ars;
+  size_t chunks;      // int4 [max chunks] (expert, first position, tokens, 0)
+  size_t nchunks;     // int32
   size_t y;           // float [T*k + T][H] expert outputs, same rows
   size_t total;
 };
@@ -97,11 +101,18 @@ struct GemvParams {
 
 struct PrefillParams {
   int H, I, E, k, T, has_shared;
+  int nst;                     // shared-memory stages of the grouped kernels (set by their launcher)
   const uint16_t* x;           // [T][H] bf16
-  __half* xh;                  // [T][H]
-  __half* a16;                 // [T*k + T][I]
+  unsigned char* xd;           // [T][2H]   digit tables of x
+  float* xX;                   // [T][H/64] group sums of x
+  float* xrs;                  // [T]       2^-p of each row of x
+  float* a;                    // [T*k + T][I] silu(gate) * up per pair (t*k + r), then per token (shared)
+  unsigned char* ad;           // [T*k + T][2I] digit tables of a
+  float* aX;                   // [T*k + T][I/64]
+  float* ars;                  // [T*k + T]
   float* y;                    // [T*k + T][H]
-  const int32_t* offsets;      // [E+1]
+  const int4* chunks;          // {expert, first position (perm index, or token for the shared expert), tokens, 0}
+  const int32_t* nchunks;      // [1]
   const int32_t* perm;         // [T*k]
   const moe_expert* experts;
   moe_expert shared;
@@ -110,9 +121,11 @@ struct PrefillParams {
 };
 
 struct GroupParams {
-  int T, k, E;
+  int T, k, E, has_shared;
+  int chunk;                   // tokens per chunk of the grouped GEMMs
   const int32_t* idx;
   int32_t* counts; int32_t* offsets; int32_t* perm;
+  int4* chunks; int32_t* nchunks;
 };
 
 // launchers (return the launch's cudaError_t)
@@ -128,9 +141,11 @@ int gateup_ctas(int I);
 int down_ctas(int H);
 cudaError_t launch_gemv(const GemvParams& p, int bits, cudaStream_t s);
 cudaError_t launch_group(const GroupParams& p, cudaStream_t s);
-cudaError_t launch_prefill_gateup(const PrefillParams& p, int bits, cudaStream_t s);   // activations to fp16 + gate/up
-cudaError_t launch_prefill_down(const PrefillParams& p, int bits, cudaStream_t s);
+cudaError_t launch_prefill_gateup(const PrefillParams& p, int bits, cudaStream_t s);   // digit tables of x + gate/up
+cudaError_t launch_prefill_down(const PrefillParams& p, int bits, cudaStream_t s);     // digit tables of a + down
 int num_sms();
+int pf_chunk_tokens(int H, int I);   // tokens per chunk of the grouped GEMMs
+size_t pf_max_chunks(int T, int k, int E, int chunk);
 int choose_ncta(long long ntiles, int nspans);
 
 }  // namespace qmoe

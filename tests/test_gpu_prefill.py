@@ -1,6 +1,7 @@
-"""GPU parity of the prefill path (T > 8 tokens: grouping by expert, grouped
-dequant GEMMs on the fp16 tensor cores, combine + residual + RMSNorm) against
-the CPU oracle, through moe_layer_forward.
+"""GPU parity of the prefill path (T > 8 tokens: grouping by expert into
+chunks, grouped GEMMs of the packed codes against fixed-point activation
+digits on the integer tensor cores, combine + residual + RMSNorm) against the
+CPU oracle, through moe_layer_forward.
 
 Routing ids bit-exact for every token; h and x_out within max relative error
 2e-3 (max|gpu - oracle| / max|oracle|) per token; bf16 x_out within one ulp
@@ -86,6 +87,17 @@ def test_prefill_small_layers(dev, bits, shared):
     x = gen.x_tokens(cfg, 4, T=33)
     out = _run(cfg, layer, x, dev)
     _compare(cfg, x, *out, sample=list(range(33)))
+
+
+def test_prefill_wide_hidden(dev):
+    """Hidden 8192 (the widest layer the library takes): 4-token chunks and
+    8 quantisation groups per warp in the gate/up kernel."""
+    cfg = fixtures.Config("pfwide", H=8192, E=8, k=2, I=256, bits=4, has_shared=True)
+    t = fxg.device_layer(cfg, 0)
+    layer = qm.layer_from_tensors(cfg, t)
+    x = gen.x_tokens(cfg, 7, T=12)
+    out = _run(cfg, layer, x, dev)
+    _compare(cfg, x, *out, sample=list(range(12)))
 
 
 def test_prefill_full_size_512_tokens(dev):
