@@ -24,9 +24,9 @@
 // meets only a few chunks and keeps their B fragments in registers. Each
 // item's 16 code rows (padded in shared memory so that the 8 rows a warp
 // reads fall in different banks), scales and biases arrive with bulk copies
-// into a ring of stages, issued nst items ahead by one warp right after the
-// block barrier that frees a stage; the 16 warps each take 1/16 of K and
-// their partial sums are added in a fixed order.
+// into a ring of stages, issued nst items ahead by all warps (one row each)
+// right after the block barrier that frees a stage; the 16 warps each take
+// 1/16 of K and their partial sums are added in a fixed order.
 #include <math.h>
 
 #include <type_traits>
@@ -38,7 +38,6 @@ namespace qmoe {
 
 constexpr int kPfWarps = 16;                            // each owns 1/16 of K
 constexpr int kPfThreads = kPfWarps * 32;
-constexpr int kPfIssuer = kPfWarps - 1;                 // the warp that issues the bulk copies
 constexpr int kPfMaxStages = 8;
 constexpr int kPfDigitThreads = 256;
 
@@ -182,19 +181,22 @@ __global__ void __launch_bounds__(kPfDigitThreads) pf_digitize_kernel(const void
 }
 
 // ------------------------------------------------------------------ grouped GEMM geometry
-// Shared memory: nst stages of {codes [16][stride], scales [16][ng], biases
-// [16][ng]} (stride = row bytes + 8*bits, so the rows a warp reads at one
-// column start 8*bits bytes apart in the banks), partial sums [2][16 warps]
-// [16 rows][C], output rows [2][C], one barrier per stage.
+// An item holds RT tiles of 16 weight rows (gate/up: tile r = 8 gate rows and
+// the 8 up rows of the same intermediate indices). Shared memory: nst stages
+// of {codes [16 RT][stride], scales [16 RT][ng], biases [16 RT][ng]} (stride =
+// row bytes + 8*bits, so the rows a warp reads at one column start 8*bits
+// bytes apart in the banks; gate/up scales and biases are [gate 8 RT][up 8 RT]),
+// partial sums [2][256 rows of (K-slice, tile row)][C], output rows [2][C],
+// one barrier per stage.
 struct PfGeom { int RB, SRB, stride, nst; size_t stage, sc, bi, part, rows, bars, total; };
-__host__ __device__ inline PfGeom pf_geom(int K, int bits, int C, int nst) {
+__host__ __device__ inline PfGeom pf_geom(int K, int bits, int C, int RT, int nst) {
   PfGeom G;
   G.RB = K * bits / 8;
   G.SRB = (K / kGroup) * 2;
   G.stride = G.RB + 8 * bits;
-  G.sc = (size_t)16 * G.stride;
-  G.bi = G.sc + (size_t)16 * G.SRB;
-  G.stage = (G.bi + (size_t)16 * G.SRB + 127) & ~(size_t)127;
+  G.sc = (size_t)16 * RT * G.stride;
+  G.bi = G.sc + (size_t)16 * RT * G.SRB;
+  G.stage = (G.bi + (size_t)16 * RT * G.SRB + 127) & ~(size_t)127;
   G.nst = nst;
   size_t o = G.stage * nst;
   G.part = o; o += sizeof(float) * 2 * kPfWarps * 16 * C;
@@ -203,6 +205,11 @@ __host__ __device__ inline PfGeom pf_geom(int K, int bits, int C, int nst) {
   G.bars = o; o += sizeof(uint64_t) * kPfMaxStages;
   G.total = o;
   return G;
+}
+// row tiles per item: enough that every warp owns up to 4 groups of its K-slice
+__host__ __device__ inline int pf_row_tiles(int K) {
+  const int ng = K / kGroup;
+  return ng >= 64 ? 1 : (ng >= 32 ? 2 : 4);
 }
 
 // activation row of token j of a chunk {e, pos, n}: x row (gate/up) or pair row (down)
@@ -222,15 +229,20 @@ __device__ __forceinline__ moe_qmat pf_mat(const PrefillParams& p, int e, int wh
 }
 
 // Persistent grouped GEMM (GU: gate/up + SwiGLU -> a; else down -> y).
-// GPW: most groups per warp; TILES: 4-token tiles per chunk.
+// GPW: most groups per warp; TILES: 4-token tiles per chunk. Warp w takes row
+// tile w / NS of the item and K-slice w % NS (NS = 16 / RT slices of ng / NS
+// groups each).
 template <int BITS, bool GU, int GPW, int TILES>
 __global__ void __launch_bounds__(kPfThreads, 1) prefill_grouped_kernel(PrefillParams p) {
   extern __shared__ __align__(128) unsigned char smem[];
   constexpr int C = 4 * TILES;
   const int K = GU ? p.H : p.I;
-  const int R = GU ? p.I / 8 : p.H / 16;   // 16-row blocks per expert
+  const int RT = p.rt;                                 // row tiles per item (1, 2 or 4)
+  const int rshift = RT == 1 ? 0 : (RT == 2 ? 1 : 2);
+  const int NS = kPfWarps >> rshift;                   // K-slices
+  const int R = GU ? p.I / (8 * RT) : p.H / (16 * RT); // items per chunk
   const int ng = K / kGroup;
-  const PfGeom G = pf_geom(K, BITS, C, p.nst);
+  const PfGeom G = pf_geom(K, BITS, C, RT, p.nst);
   const int nst = G.nst;
   uint64_t* full = (uint64_t*)(smem + G.bars);
   float* part = (float*)(smem + G.part);
@@ -244,57 +256,69 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_grouped_kernel(PrefillP
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  const unsigned item_bytes = 16u * G.RB + 32u * G.SRB;
-  // Copies of local item i into stage i % nst (issuer warp: lane 0 arms the
-  // barrier, one lane per copy).
-  int icur = -1, ie = 0;
-  auto issue = [&](int i) {
-    const int st = i % nst;
-    const long long item = lo + i;
-    const int ci = (int)(item / R), rb = (int)(item - (long long)ci * R);
-    if (ci != icur) { icur = ci; ie = __ldg(&p.chunks[ci].x); }
-    const int e = ie;
-    unsigned char* sb = smem + (size_t)st * G.stage;
-    if (lane == 0) pf_expect(&full[st], item_bytes);
-    __syncwarp();
-    if (GU) {
-      if (lane < 16) {   // code rows: gate rows rb*8.. -> 0..7, up rows -> 8..15
-        const moe_qmat m = pf_mat(p, e, lane >> 3);
-        pf_bulk(sb + (size_t)lane * G.stride, (const char*)m.q + (size_t)(rb * 8 + (lane & 7)) * G.RB, G.RB,
-                &full[st]);
-      } else if (lane < 20) {   // 16 gate scales, 17 up scales, 18 gate biases, 19 up biases
-        const int c = lane - 16;
-        const moe_qmat m = pf_mat(p, e, c & 1);
-        pf_bulk(sb + (c < 2 ? G.sc : G.bi) + (size_t)(c & 1) * 8 * G.SRB,
-                (const char*)(c < 2 ? m.scales : m.biases) + (size_t)rb * 8 * G.SRB, 8u * G.SRB, &full[st]);
+  const unsigned item_bytes = 16u * RT * G.RB + 32u * RT * G.SRB;
+  const int ci0 = (int)(lo / R), rb0 = (int)(lo - (long long)ci0 * R);
+
+  // Copies of the next item to issue (cursor ici, irb) into stage st. Lane 0
+  // of warp w copies code rows w, w+16, ... of the item; warps 0-3 (gate/up)
+  // or 0-1 (down) also one scale or bias block. The stage's barrier is armed
+  // by thread 0 before the block barrier that precedes these copies.
+  int ici = ci0, irb = rb0, icur = -1, ie = -1;
+  const char* mq = nullptr;    // this warp's code rows (gate/up: gate for warps 0-7, up for 8-15)
+  const char* msb = nullptr;   // this warp's scale or bias block (warps 0-3 / 0-1)
+  auto issue = [&](int st) {
+    if (ici != icur) {
+      icur = ici;
+      const int e = __ldg(&p.chunks[ici].x);
+      if (e != ie) {
+        ie = e;
+        const moe_qmat m = pf_mat(p, e, GU ? (warp >> 3) : 2);
+        mq = (const char*)m.q;
+        if (GU && warp < 4) {
+          const moe_qmat ms = pf_mat(p, e, warp & 1);
+          msb = (const char*)(warp < 2 ? ms.scales : ms.biases);
+        } else if (!GU && warp < 2) {
+          msb = (const char*)(warp == 0 ? m.scales : m.biases);
+        }
       }
-    } else if (lane < 18) {   // 16 code rows, then scales and biases
-      const moe_qmat m = pf_mat(p, e, 2);
-      if (lane < 16)
-        pf_bulk(sb + (size_t)lane * G.stride, (const char*)m.q + (size_t)(rb * 16 + lane) * G.RB, G.RB, &full[st]);
-      else
-        pf_bulk(sb + (lane == 16 ? G.sc : G.bi),
-                (const char*)(lane == 16 ? m.scales : m.biases) + (size_t)rb * 16 * G.SRB, 16u * G.SRB, &full[st]);
     }
+    unsigned char* sb = smem + (size_t)st * G.stage;
+    for (int r = warp; r < 16 * RT; r += kPfWarps) {
+      const int tr = r >> 4, q = r & 15;
+      const int src = GU ? irb * 8 * RT + 8 * tr + (q & 7) : irb * 16 * RT + r;
+      pf_bulk(sb + (size_t)r * G.stride, mq + (size_t)src * G.RB, G.RB, &full[st]);
+    }
+    if (GU && warp < 4)   // 0 gate scales, 1 up scales, 2 gate biases, 3 up biases
+      pf_bulk(sb + (warp < 2 ? G.sc : G.bi) + (size_t)(warp & 1) * 8 * RT * G.SRB,
+              msb + (size_t)irb * 8 * RT * G.SRB, 8u * RT * G.SRB, &full[st]);
+    else if (!GU && warp < 2)
+      pf_bulk(sb + (warp == 0 ? G.sc : G.bi), msb + (size_t)irb * 16 * RT * G.SRB, 16u * RT * G.SRB, &full[st]);
+    if (++irb == R) { irb = 0; ++ici; }
   };
-  if (warp == kPfIssuer)
+  if (tid == 0)
+    for (int i = 0; i < nloc && i < nst; ++i) pf_expect(&full[i], item_bytes);
+  __syncthreads();
+  if (lane == 0)
     for (int i = 0; i < nloc && i < nst; ++i) issue(i);
 
   const int g = lane >> 2, t = lane & 3;
-  const int gpw = (ng + kPfWarps - 1) / kPfWarps;
-  const int g0 = warp * gpw;
+  const int tr = warp >> (4 - rshift), ks = warp & (NS - 1);   // row tile, K-slice
+  const int gpw = (ng + NS - 1) / NS;
+  const int g0 = ks * gpw;
   const int mg = max(0, min(gpw, ng - g0));   // groups of this warp
   const unsigned char* dig = GU ? p.xd : p.ad;
   const float* Xt = GU ? p.xX : p.aX;
   const float* rst = GU ? p.xrs : p.ars;
   const bool vec_sb = (mg == GPW) && (ng % GPW == 0);   // the warp's scales in one load per row
+  // shared-memory rows of this warp's tile: A rows g (gate / first 8) and g+8 (up / last 8)
+  const int crA = 16 * tr + g, crB = 16 * tr + 8 + g;
+  const int srA = GU ? 8 * tr + g : crA, srB = GU ? 8 * RT + 8 * tr + g : crB;
   uint4 bq[TILES][GPW];
   float xg[TILES][GPW], rsc[TILES];
   int cur = -1, n = 0, orow = -1;
+  int ci = ci0, rb = rb0, st = 0;
+  unsigned phase = 0;
   for (int i = 0; i < nloc; ++i) {
-    const int st = i % nst;
-    const long long item = lo + i;
-    const int ci = (int)(item / R), rb = (int)(item - (long long)ci * R);
     if (ci != cur) {   // new chunk: B fragments and group sums of its tokens
       cur = ci;
       const int4 ch = __ldg(&p.chunks[ci]);
@@ -316,16 +340,16 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_grouped_kernel(PrefillP
       if (warp == 0 && lane < C) orow = lane < n ? pf_out_row(p, ch, lane) : -1;
     }
     if (warp == 0 && lane < C) rows_out[(i & 1) * C + lane] = orow;
-    pf_wait(&full[st], (unsigned)(i / nst) & 1u, p.wait_ns, p.status);
+    pf_wait(&full[st], phase, p.wait_ns, p.status);
     const unsigned char* sb = smem + (size_t)st * G.stage;
     const uint16_t* ssc = (const uint16_t*)(sb + G.sc);
     const uint16_t* sbi = (const uint16_t*)(sb + G.bi);
-    // scales / biases of rows g and g+8 for the warp's groups
+    // scales / biases of the warp's two rows for its groups
     float sA[GPW], sB[GPW], bA[GPW], bB[GPW];
     if (vec_sb) {
       using V = typename std::conditional<GPW == 4, uint2, uint4>::type;
-      const V va = *(const V*)(ssc + (size_t)g * ng + g0), vb = *(const V*)(ssc + (size_t)(g + 8) * ng + g0);
-      const V wa = *(const V*)(sbi + (size_t)g * ng + g0), wb = *(const V*)(sbi + (size_t)(g + 8) * ng + g0);
+      const V va = *(const V*)(ssc + (size_t)srA * ng + g0), vb = *(const V*)(ssc + (size_t)srB * ng + g0);
+      const V wa = *(const V*)(sbi + (size_t)srA * ng + g0), wb = *(const V*)(sbi + (size_t)srB * ng + g0);
       const uint32_t* pa = (const uint32_t*)&va;
       const uint32_t* pb = (const uint32_t*)&vb;
       const uint32_t* qa = (const uint32_t*)&wa;
@@ -340,16 +364,19 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_grouped_kernel(PrefillP
     } else {
 #pragma unroll
       for (int gi = 0; gi < GPW; ++gi) {
-        const int gg = gi < mg ? g0 + gi : 0;
-        sA[gi] = bf16_lo(ssc[(size_t)g * ng + gg]); sB[gi] = bf16_lo(ssc[(size_t)(g + 8) * ng + gg]);
-        bA[gi] = bf16_lo(sbi[(size_t)g * ng + gg]); bB[gi] = bf16_lo(sbi[(size_t)(g + 8) * ng + gg]);
+        sA[gi] = sB[gi] = bA[gi] = bB[gi] = 0.f;
+        if (gi < mg) {
+          const int gg = g0 + gi;
+          sA[gi] = bf16_lo(ssc[(size_t)srA * ng + gg]); sB[gi] = bf16_lo(ssc[(size_t)srB * ng + gg]);
+          bA[gi] = bf16_lo(sbi[(size_t)srA * ng + gg]); bB[gi] = bf16_lo(sbi[(size_t)srB * ng + gg]);
+        }
       }
     }
     float sacc[TILES][2], bacc[TILES][2];
 #pragma unroll
     for (int tau = 0; tau < TILES; ++tau) sacc[tau][0] = sacc[tau][1] = bacc[tau][0] = bacc[tau][1] = 0.f;
-    const unsigned char* ra = sb + (size_t)g * G.stride;
-    const unsigned char* rbp = sb + (size_t)(g + 8) * G.stride;
+    const unsigned char* ra = sb + (size_t)crA * G.stride;
+    const unsigned char* rbp = sb + (size_t)crB * G.stride;
 #pragma unroll
     for (int gi = 0; gi < GPW; ++gi) {
       if (gi < mg) {
@@ -384,49 +411,47 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_grouped_kernel(PrefillP
         }
       }
     }
-    float* pw = part + ((size_t)(i & 1) * kPfWarps + warp) * 16 * C;
+    // partials: part[buf][ks][tile row][token]
+    float* pw = part + ((size_t)(i & 1) * kPfWarps * 16 + (size_t)ks * 16 * RT) * C;
 #pragma unroll
     for (int tau = 0; tau < TILES; ++tau) {
-      pw[g * C + 4 * tau + t] = fmaf(sacc[tau][0], rsc[tau], bacc[tau][0]);
-      pw[(g + 8) * C + 4 * tau + t] = fmaf(sacc[tau][1], rsc[tau], bacc[tau][1]);
+      pw[crA * C + 4 * tau + t] = fmaf(sacc[tau][0], rsc[tau], bacc[tau][0]);
+      pw[crB * C + 4 * tau + t] = fmaf(sacc[tau][1], rsc[tau], bacc[tau][1]);
     }
-    pf_fence_proxy();   // this thread's reads of the stage precede the copies that refill it
+    if (tid == 0 && i + nst < nloc) pf_expect(&full[st], item_bytes);   // its phase for item i is complete
     __syncthreads();
-    if (warp == kPfIssuer && i + nst < nloc) issue(i + nst);   // stage st is free again
-    // outputs: the 16 warps' partials added in a fixed order, L lanes per output
+    if (lane == 0 && i + nst < nloc) {   // stage st is free again: item i + nst
+      pf_fence_proxy();   // the block's reads of the stage (ordered by the barrier) precede the refill
+      issue(st);
+    }
+    // outputs: one thread per output adds the NS slices' partials in slice order
     const float* pr = part + (size_t)(i & 1) * kPfWarps * 16 * C;
     const int* ro = rows_out + (i & 1) * C;
+    const int slice = 16 * RT * C;   // floats per slice
     if (GU) {
-      constexpr int L = kPfWarps * 32 / (8 * C), PW = kPfWarps / L;   // lanes per output, warps per lane
-      const int o = tid / L, s = tid - o * L;   // o = x * 8 + j
-      const int x = o >> 3, j = o & 7;
-      float gs = 0.f, us = 0.f;
-#pragma unroll
-      for (int w = 0; w < PW; ++w) {
-        const float* pq = pr + (size_t)(s * PW + w) * 16 * C;
-        gs += pq[j * C + x];
-        us += pq[(8 + j) * C + x];
+      if (tid < 8 * RT * C) {   // tid = x * 8 RT + jj
+        const int x = tid >> (3 + rshift), jj = tid & (8 * RT - 1);
+        const int prow = 16 * (jj >> 3) + (jj & 7);
+        const float* pq = pr + prow * C + x;
+        float gs = 0.f, us = 0.f;
+        for (int w = 0; w < NS; ++w) {
+          gs += pq[w * slice];
+          us += pq[w * slice + 8 * C];
+        }
+        if (x < n) p.a[(size_t)ro[x] * p.I + rb * 8 * RT + jj] = gs / (1.f + expf(-gs)) * us;
       }
-#pragma unroll
-      for (int off = 1; off < L; off <<= 1) {
-        gs += __shfl_xor_sync(0xffffffffu, gs, off);
-        us += __shfl_xor_sync(0xffffffffu, us, off);
-      }
-      if (s == 0 && x < n) p.a[(size_t)ro[x] * p.I + rb * 8 + j] = gs / (1.f + expf(-gs)) * us;
-    } else {
-      constexpr int L = kPfWarps * 32 / (16 * C), PW = kPfWarps / L;
-      const int o = tid / L, s = tid - o * L;   // o = x * 16 + r
-      const int x = o >> 4, r = o & 15;
+    } else if (tid < 16 * RT * C) {   // tid = x * 16 RT + rr
+      const int x = tid >> (4 + rshift), rr = tid & (16 * RT - 1);
+      const float* pq = pr + rr * C + x;
       float y = 0.f;
-#pragma unroll
-      for (int w = 0; w < PW; ++w) y += pr[(size_t)(s * PW + w) * 16 * C + r * C + x];
-#pragma unroll
-      for (int off = 1; off < L; off <<= 1) y += __shfl_xor_sync(0xffffffffu, y, off);
-      if (s == 0 && x < n) p.y[(size_t)ro[x] * p.H + rb * 16 + r] = y;
+      for (int w = 0; w < NS; ++w) y += pq[w * slice];
+      if (x < n) p.y[(size_t)ro[x] * p.H + rb * 16 * RT + rr] = y;
     }
+    if (++st == nst) { st = 0; phase ^= 1u; }
+    if (++rb == R) { rb = 0; ++ci; }
   }
   // every copy this CTA issued has landed before it exits (immediate unless a wait above gave up)
-  if (warp == kPfIssuer)
+  if (lane == 0)
     for (int i = nloc - nst < 0 ? 0 : nloc - nst; i < nloc; ++i)
       pf_wait(&full[i % nst], (unsigned)(i / nst) & 1u, p.wait_ns, nullptr);
 }
@@ -444,19 +469,22 @@ template <int BITS, bool GU>
 static cudaError_t pf_grouped(const PrefillParams& p, cudaStream_t s) {
   const int K = GU ? p.H : p.I;
   const int C = pf_chunk_tokens(p.H, p.I);
-  const int ng = K / kGroup, gpw = (ng + kPfWarps - 1) / kPfWarps;
+  const int RT = C == 8 ? pf_row_tiles(K) : 1;
+  const int ng = K / kGroup, NS = kPfWarps / RT, gpw = (ng + NS - 1) / NS;
+  if (gpw > (C == 8 ? 4 : 8)) return cudaErrorInvalidConfiguration;
+  if ((GU ? p.I % (8 * RT) : p.H % (16 * RT)) != 0) return cudaErrorInvalidConfiguration;
   int optin = 0, dev = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-  const size_t fixed = pf_geom(K, BITS, C, 0).total;
-  const size_t stage = pf_geom(K, BITS, C, 1).stage;
+  const size_t fixed = pf_geom(K, BITS, C, RT, 0).total;
+  const size_t stage = pf_geom(K, BITS, C, RT, 1).stage;
   if ((size_t)optin < fixed + 2 * stage) return cudaErrorInvalidConfiguration;
   int nst = (int)(((size_t)optin - fixed) / stage);
   if (nst > kPfMaxStages) nst = kPfMaxStages;
-  if (gpw > (C == 8 ? 4 : 8)) return cudaErrorInvalidConfiguration;
   PrefillParams q = p;
   q.nst = nst;
-  const size_t sm = pf_geom(K, BITS, C, nst).total;
+  q.rt = RT;
+  const size_t sm = pf_geom(K, BITS, C, RT, nst).total;
   const void* fn = C == 8 ? (const void*)prefill_grouped_kernel<BITS, GU, 4, 2>
                           : (const void*)prefill_grouped_kernel<BITS, GU, 8, 1>;
   cudaError_t e = pf_prepare(fn, sm);
