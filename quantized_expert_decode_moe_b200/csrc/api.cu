@@ -150,7 +150,7 @@ moe_status prefill_chain(const moe_layer* L, const uint16_t* x_in, float* h, int
   rp.H = H; rp.E = E; rp.T = T; rp.has_shared = L->has_shared;
   rp.x = x_in; rp.router_w = L->router_w; rp.router_bias = L->router_bias; rp.gate_w = L->shared_gate_w;
   rp.logits = at<double>(ws, W.logits);
-  cudaError_t e = launch_route(rp, s, false);
+  cudaError_t e = launch_route_gemm(rp, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   mark(1);
   TopkParams tp{};
@@ -239,7 +239,7 @@ moe_status moe_route(const moe_layer* layer, const uint16_t* x, int32_t T, int32
   rp.H = layer->hidden; rp.E = layer->n_experts; rp.T = T; rp.has_shared = layer->has_shared;
   rp.x = x; rp.router_w = layer->router_w; rp.router_bias = layer->router_bias; rp.gate_w = layer->shared_gate_w;
   rp.logits = at<double>(ws, W.logits);
-  if (launch_route(rp, s, false) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((T > kDecodeMaxT ? launch_route_gemm(rp, s) : launch_route(rp, s, false)) != cudaSuccess) return MOE_ERR_CUDA;
   TopkParams tp{};
   tp.E = layer->n_experts; tp.k = layer->top_k; tp.T = T; tp.has_shared = layer->has_shared;
   tp.logits = rp.logits; tp.idx = topk_idx; tp.w = topk_w; tp.sg = shared_gate;

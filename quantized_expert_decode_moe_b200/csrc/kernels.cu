@@ -195,6 +195,99 @@ __global__ void __launch_bounds__(kRouteThreads) route_logits_kernel(RouteParams
   }
 }
 
+// Router logits of many tokens (prefill): a tiled GEMM in fp64. Every
+// product of two bf16 values is exact in fp64, and each logit is accumulated
+// over k in index order from 0 by one thread, then the bias is added: the
+// same sequence of roundings as the plain fp64 loop of the definition
+// (logits l = W_r x + b, "Model architecture" of the Flash-MoE write-up), so
+// the logits are reproduced exactly. Tile: 32 tokens x 64 router rows per
+// CTA; thread (ty, tx) holds tokens 2ty, 2ty+1 and rows 8tx..8tx+7; operands
+// are staged in shared memory as doubles, k-major.
+constexpr int kRgTok = 32, kRgRows = 64, kRgK = 32, kRgThreads = 128;
+__global__ void __launch_bounds__(kRgThreads) route_gemm_kernel(RouteParams p) {
+  __shared__ __align__(16) double xs[kRgK][kRgTok];    // [k][token]
+  __shared__ __align__(16) double ws[kRgK][kRgRows];   // [k][row pair b/2][tx][b%2]
+  const int tid = threadIdx.x, tx = tid & 7, ty = tid >> 3;
+  const int e0 = blockIdx.x * kRgRows, t0 = blockIdx.y * kRgTok;
+  const int nrows = p.E + (p.has_shared ? 1 : 0);
+  double acc[2][8];
+#pragma unroll
+  for (int a = 0; a < 2; ++a)
+#pragma unroll
+    for (int b = 0; b < 8; ++b) acc[a][b] = 0.0;
+  // global tile: x 32 tokens x 32 k (one uint4 of 8 k per thread), W 64 rows x 32 k (two per thread)
+  const int xr = tid >> 2, xc = tid & 3;
+  const uint16_t* xrow = t0 + xr < p.T ? p.x + (size_t)(t0 + xr) * p.H : nullptr;
+  const uint16_t* wrow[2];
+  int wr[2], wc[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int idx = tid + kRgThreads * j;
+    wr[j] = idx >> 2; wc[j] = idx & 3;
+    const int e = e0 + wr[j];
+    wrow[j] = e < p.E ? p.router_w + (size_t)e * p.H : (e < nrows ? p.gate_w : nullptr);
+  }
+  auto load = [&](int k0, uint4& xv, uint4 (&wv)[2]) {
+    xv = xrow ? __ldg((const uint4*)(xrow + k0 + 8 * xc)) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+      wv[j] = wrow[j] ? __ldg((const uint4*)(wrow[j] + k0 + 8 * wc[j])) : make_uint4(0u, 0u, 0u, 0u);
+  };
+  uint4 xv, wv[2];
+  load(0, xv, wv);
+  for (int k0 = 0; k0 < p.H; k0 += kRgK) {
+    __syncthreads();   // the previous tile has been read
+    {
+      const uint32_t u[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        xs[8 * xc + 2 * i][xr] = (double)bf16lo(u[i]);
+        xs[8 * xc + 2 * i + 1][xr] = (double)bf16hi(u[i]);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const uint32_t u[4] = {wv[j].x, wv[j].y, wv[j].z, wv[j].w};
+      const int r = wr[j], pos = ((r & 7) >> 1) * 16 + (r >> 3) * 2 + (r & 1);   // row 8 tx + b at (b/2, tx, b%2)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        ws[8 * wc[j] + 2 * i][pos] = (double)bf16lo(u[i]);
+        ws[8 * wc[j] + 2 * i + 1][pos] = (double)bf16hi(u[i]);
+      }
+    }
+    __syncthreads();
+    if (k0 + kRgK < p.H) load(k0 + kRgK, xv, wv);   // next tile in flight during the products
+#pragma unroll 8
+    for (int kk = 0; kk < kRgK; ++kk) {
+      const double2 xa = *(const double2*)&xs[kk][2 * ty];
+      double w8[8];
+#pragma unroll
+      for (int bp = 0; bp < 4; ++bp) {
+        const double2 v = *(const double2*)&ws[kk][bp * 16 + tx * 2];
+        w8[2 * bp] = v.x; w8[2 * bp + 1] = v.y;
+      }
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        acc[0][b] = fma(w8[b], xa.x, acc[0][b]);
+        acc[1][b] = fma(w8[b], xa.y, acc[1][b]);
+      }
+    }
+  }
+#pragma unroll
+  for (int a = 0; a < 2; ++a) {
+    const int t = t0 + 2 * ty + a;
+    if (t >= p.T) continue;
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+      const int e = e0 + 8 * tx + b;
+      if (e >= nrows) continue;
+      double v = acc[a][b];
+      if (e < p.E && p.router_bias) v += (double)p.router_bias[e];
+      p.logits[(size_t)t * (p.E + 1) + e] = v;
+    }
+  }
+}
+
 // grid T, block 512: top-k of logits already in the workspace (moe_route).
 __global__ void __launch_bounds__(kThreads) topk_kernel(TopkParams p) {
   __shared__ TopkSmem ts;
@@ -529,6 +622,14 @@ cudaError_t launch_route(const RouteParams& p, cudaStream_t s, bool pdl) {
   cudaError_t e = set_smem((const void*)route_logits_kernel, sm);
   if (e != cudaSuccess) return e;
   return launch_ex((const void*)route_logits_kernel, grid, dim3(kRouteThreads), sm, s, pdl, args);
+}
+
+cudaError_t launch_route_gemm(const RouteParams& p, cudaStream_t s) {
+  const int rows = p.E + (p.has_shared ? 1 : 0);
+  dim3 grid((rows + kRgRows - 1) / kRgRows, (p.T + kRgTok - 1) / kRgTok);
+  RouteParams q = p;
+  void* args[] = {&q};
+  return launch_ex((const void*)route_gemm_kernel, grid, dim3(kRgThreads), 0, s, false, args);
 }
 
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t s) {

@@ -130,6 +130,7 @@ struct GroupParams {
 
 // launchers (return the launch's cudaError_t)
 cudaError_t launch_route(const RouteParams& p, cudaStream_t s, bool pdl);
+cudaError_t launch_route_gemm(const RouteParams& p, cudaStream_t s);   // many tokens: tiled fp64
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t s);
 cudaError_t launch_gateup(const GateUpParams& p, int bits, int T, bool pdl, cudaStream_t s);
 cudaError_t launch_down(const DownParams& p, int bits, int T, bool pdl, cudaStream_t s);
