@@ -138,21 +138,25 @@ def build_workload(cfg, copies, dev):
     return dict(layers=layers, keep=keep, x=xd, h=h0.clone(), h0=h0, P=P, x_host=x)
 
 
-def kernel_src_sha():
+DECODE_SOURCES = ("common.cuh", "kernels.cu", "kernels.cuh", "api.cu", "decode.cu", "topk.cuh")
+PREFILL_SOURCES = ("common.cuh", "kernels.cuh", "prefill.cu")   # the grouped GEMM kernels
+
+
+def kernel_src_sha(files=DECODE_SOURCES):
     h = hashlib.sha256()
-    for f in ("common.cuh", "kernels.cu", "kernels.cuh", "api.cu", "decode.cu", "topk.cuh"):
+    for f in files:
         p = os.path.join(ROOT, "quantized_expert_decode_moe_b200", "csrc", f)
         if os.path.exists(p):
             h.update(open(p, "rb").read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel: str, config: str):
+def recorded_traffic(kernel: str, config: str, files=DECODE_SOURCES):
     """dram bytes per launch from the committed ncu summary, if it was taken on the current sources."""
     p = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(p):
         return None
-    sha = kernel_src_sha()
+    sha = kernel_src_sha(files)
     for line in open(p):
         if line.startswith("#") or not line.strip():
             continue
@@ -507,7 +511,8 @@ def ours_prefill(args, cfg):
         "metric": "MoE-layer prefill tokens/s (512-token batch), 4-bit experts, 1 B200", "value": T * steps / (ms * 1e-3),
         "unit": "tokens/s", "n_gpus": world, "steps": steps, "warmup": max(args.warmup, 3),
         "ms_per_step": ms / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "u4 codes dequantised to f16, f16 tensor-core MMA, f32 accumulate",
+        "dtype": "u4 codes x s8 digits of 16-bit fixed-point activations on int8 tensor cores (s32), "
+                 "fp32 scale+accumulate; router logits f64",
         "data": "synthetic (seeded; no model weights)",
         "config": {"workload": cfg.note, "H": cfg.H, "E": cfg.E, "top_k": cfg.k, "I": cfg.I, "bits": cfg.bits,
                    "T": T, "experts_touched_per_step": float(np.mean(touched)),
@@ -515,11 +520,13 @@ def ours_prefill(args, cfg):
         "stage_ms": dict(zip(names, dur)),
         "tflops": flops / (ms / steps * 1e-3) / 1e12,
         "roofline": {"bound": "hbm", "kernel": "gateup_grouped", "achieved": achieved, "peak": peaks["hbm_gbs"],
-                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": recorded_traffic("prefill_grouped_gateup", cfg.name, PREFILL_SOURCES),
                      "algorithmic_bytes": gu_bytes, "peak_kind": peak_kind},
         "e2e": {"value": T * e2e_n / (e2e_ms * 1e-3), "unit": "tokens/s", "steps": e2e_n,
                 "h2d_bytes_per_step": T * cfg.H * (2 + 4), "d2h_bytes_per_step": T * cfg.H * 2},
-        "gpu_launches": 7 * steps, "clocks": clk,
+        # route, top-k, grouping, digits of x, gate/up, digits of a, down, combine + norm
+        "gpu_launches": 8 * steps, "clocks": clk,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
