@@ -103,11 +103,15 @@ moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
 /*
  * Router ("Model architecture": K=4 active per token incl. one shared;
  * the router results select the experts to load — HN thread, Table 3 comment).
- *   logits = router_w . x (+ router_bias), accumulated in fp64;
+ *   logits = router_w . x (+ router_bias): for T > 8 in fp64, each logit
+ *   accumulated in index order from 0 with the bias added last, which with
+ *   exact bf16 x bf16 products is the plain fp64 sum itself; for T <= 8 as
+ *   compensated fp32 (about 2^-44 relative to sum |w x|), rounded to fp64;
  *   topk_idx [T][k]: the k largest logits, descending, ties to the lower index;
  *   topk_w [T][k]: softmax over all E renormalised over the chosen k (fp32);
  *   shared_gate [T] (nullable): sigmoid(shared_gate_w . x), 0 if no shared expert.
- * x: bf16 [T][H]. Uses the workspace for the logits.
+ * x: bf16 [T][H]. The logits stay in the workspace after the call: double
+ * [T][E+1] at byte offset 256, column E holding shared_gate_w . x.
  */
 moe_status moe_route(const moe_layer* layer, const uint16_t* x, int32_t T, int32_t* topk_idx,
                      float* topk_w, float* shared_gate, void* ws, size_t ws_bytes, void* stream);

@@ -195,99 +195,6 @@ __global__ void __launch_bounds__(kRouteThreads) route_logits_kernel(RouteParams
   }
 }
 
-// Router logits of many tokens (prefill): a tiled GEMM in fp64. Every
-// product of two bf16 values is exact in fp64, and each logit is accumulated
-// over k in index order from 0 by one thread, then the bias is added: the
-// same sequence of roundings as the plain fp64 loop of the definition
-// (logits l = W_r x + b, "Model architecture" of the Flash-MoE write-up), so
-// the logits are reproduced exactly. Tile: 32 tokens x 64 router rows per
-// CTA; thread (ty, tx) holds tokens 2ty, 2ty+1 and rows 8tx..8tx+7; operands
-// are staged in shared memory as doubles, k-major.
-constexpr int kRgTok = 32, kRgRows = 64, kRgK = 32, kRgThreads = 128;
-__global__ void __launch_bounds__(kRgThreads) route_gemm_kernel(RouteParams p) {
-  __shared__ __align__(16) double xs[kRgK][kRgTok];    // [k][token]
-  __shared__ __align__(16) double ws[kRgK][kRgRows];   // [k][row pair b/2][tx][b%2]
-  const int tid = threadIdx.x, tx = tid & 7, ty = tid >> 3;
-  const int e0 = blockIdx.x * kRgRows, t0 = blockIdx.y * kRgTok;
-  const int nrows = p.E + (p.has_shared ? 1 : 0);
-  double acc[2][8];
-#pragma unroll
-  for (int a = 0; a < 2; ++a)
-#pragma unroll
-    for (int b = 0; b < 8; ++b) acc[a][b] = 0.0;
-  // global tile: x 32 tokens x 32 k (one uint4 of 8 k per thread), W 64 rows x 32 k (two per thread)
-  const int xr = tid >> 2, xc = tid & 3;
-  const uint16_t* xrow = t0 + xr < p.T ? p.x + (size_t)(t0 + xr) * p.H : nullptr;
-  const uint16_t* wrow[2];
-  int wr[2], wc[2];
-#pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const int idx = tid + kRgThreads * j;
-    wr[j] = idx >> 2; wc[j] = idx & 3;
-    const int e = e0 + wr[j];
-    wrow[j] = e < p.E ? p.router_w + (size_t)e * p.H : (e < nrows ? p.gate_w : nullptr);
-  }
-  auto load = [&](int k0, uint4& xv, uint4 (&wv)[2]) {
-    xv = xrow ? __ldg((const uint4*)(xrow + k0 + 8 * xc)) : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-    for (int j = 0; j < 2; ++j)
-      wv[j] = wrow[j] ? __ldg((const uint4*)(wrow[j] + k0 + 8 * wc[j])) : make_uint4(0u, 0u, 0u, 0u);
-  };
-  uint4 xv, wv[2];
-  load(0, xv, wv);
-  for (int k0 = 0; k0 < p.H; k0 += kRgK) {
-    __syncthreads();   // the previous tile has been read
-    {
-      const uint32_t u[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        xs[8 * xc + 2 * i][xr] = (double)bf16lo(u[i]);
-        xs[8 * xc + 2 * i + 1][xr] = (double)bf16hi(u[i]);
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const uint32_t u[4] = {wv[j].x, wv[j].y, wv[j].z, wv[j].w};
-      const int r = wr[j], pos = ((r & 7) >> 1) * 16 + (r >> 3) * 2 + (r & 1);   // row 8 tx + b at (b/2, tx, b%2)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        ws[8 * wc[j] + 2 * i][pos] = (double)bf16lo(u[i]);
-        ws[8 * wc[j] + 2 * i + 1][pos] = (double)bf16hi(u[i]);
-      }
-    }
-    __syncthreads();
-    if (k0 + kRgK < p.H) load(k0 + kRgK, xv, wv);   // next tile in flight during the products
-#pragma unroll 8
-    for (int kk = 0; kk < kRgK; ++kk) {
-      const double2 xa = *(const double2*)&xs[kk][2 * ty];
-      double w8[8];
-#pragma unroll
-      for (int bp = 0; bp < 4; ++bp) {
-        const double2 v = *(const double2*)&ws[kk][bp * 16 + tx * 2];
-        w8[2 * bp] = v.x; w8[2 * bp + 1] = v.y;
-      }
-#pragma unroll
-      for (int b = 0; b < 8; ++b) {
-        acc[0][b] = fma(w8[b], xa.x, acc[0][b]);
-        acc[1][b] = fma(w8[b], xa.y, acc[1][b]);
-      }
-    }
-  }
-#pragma unroll
-  for (int a = 0; a < 2; ++a) {
-    const int t = t0 + 2 * ty + a;
-    if (t >= p.T) continue;
-#pragma unroll
-    for (int b = 0; b < 8; ++b) {
-      const int e = e0 + 8 * tx + b;
-      if (e >= nrows) continue;
-      double v = acc[a][b];
-      if (e < p.E && p.router_bias) v += (double)p.router_bias[e];
-      p.logits[(size_t)t * (p.E + 1) + e] = v;
-    }
-  }
-}
-
 // grid T, block 512: top-k of logits already in the workspace (moe_route).
 __global__ void __launch_bounds__(kThreads) topk_kernel(TopkParams p) {
   __shared__ TopkSmem ts;
@@ -489,103 +396,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GemvParams p) {
   reduce_partials(cr, p.nspans, ps, [&](int tile, int r, float v) { atomicAdd(p.y + (size_t)tile * 16 + r, v); });
 }
 
-// ------------------------------------------------------------------ grouping by expert
-// Exclusive scan of v[0..n) in place (one block); returns the total.
-__device__ int block_exclusive_scan(int* v, int n, int* warp_tot) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
-  int carry = 0;
-  for (int base = 0; base < n; base += blockDim.x) {
-    const int e = base + tid;
-    const int x = e < n ? v[e] : 0;
-    int incl = x;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    if (lane == 31) warp_tot[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-      int wv = lane < nw ? warp_tot[lane] : 0;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, wv, o);
-        if (lane >= o) wv += y;
-      }
-      if (lane < nw) warp_tot[lane] = wv;
-    }
-    __syncthreads();
-    if (e < n) v[e] = carry + (warp ? warp_tot[warp - 1] : 0) + incl - x;
-    const int tot = warp_tot[nw - 1];
-    __syncthreads();
-    carry += tot;
-  }
-  return carry;
-}
-
-// Prefill grouping in one CTA: histogram of the chosen experts, exclusive
-// scan, then a stable scatter of the flattened (token, rank) pairs by one warp
-// that walks them in order 32 at a time (ranks of equal experts from
-// __match_any_sync). Also the chunk list of the grouped GEMMs: expert e's
-// pairs in runs of `chunk`, then the shared expert's tokens in runs of `chunk`.
-__global__ void __launch_bounds__(1024) group_kernel(GroupParams p) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  int* cnt = (int*)smem;            // [E]
-  int* fill = cnt + p.E;            // [E]
-  int* cb = fill + p.E;             // [E] first chunk of each expert
-  __shared__ int warp_tot[32];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int N = p.T * p.k, C = p.chunk;
-  for (int e = tid; e < p.E; e += blockDim.x) cnt[e] = 0;
-  __syncthreads();
-  for (int i = tid; i < N; i += blockDim.x) {
-    const int e = p.idx[i];
-    if (e >= 0 && e < p.E) atomicAdd(&cnt[e], 1);
-  }
-  __syncthreads();
-  for (int e = tid; e < p.E; e += blockDim.x) {
-    p.counts[e] = cnt[e];
-    fill[e] = cnt[e];
-    cb[e] = C > 0 ? (cnt[e] + C - 1) / C : 0;
-  }
-  __syncthreads();
-  const int total = block_exclusive_scan(fill, p.E, warp_tot);
-  const int nrouted = block_exclusive_scan(cb, p.E, warp_tot);
-  const bool chunked = p.chunks != nullptr && p.nchunks != nullptr && C > 0;   // the grouped GEMMs' list
-  for (int e = tid; e < p.E; e += blockDim.x) {
-    p.offsets[e] = fill[e];
-    if (chunked)
-      for (int c = 0; c * C < cnt[e]; ++c)
-        p.chunks[cb[e] + c] = make_int4(e, fill[e] + c * C, min(C, cnt[e] - c * C), 0);
-  }
-  const int nshared = chunked && p.has_shared ? (p.T + C - 1) / C : 0;
-  for (int c = tid; c < nshared; c += blockDim.x)
-    p.chunks[nrouted + c] = make_int4(p.E, c * C, min(C, p.T - c * C), 0);
-  if (tid == 0) {
-    p.offsets[p.E] = total;
-    if (chunked) *p.nchunks = nrouted + nshared;
-  }
-  __syncthreads();
-  if (warp == 0) {
-    for (int base = 0; base < N; base += 32) {
-      const int i = base + lane;
-      const bool valid = i < N;
-      const int e = valid ? p.idx[i] : -1;
-      const unsigned mask = __ballot_sync(0xffffffffu, valid);
-      const unsigned peers = __match_any_sync(0xffffffffu, e);
-      const int rank = __popc(peers & ((1u << lane) - 1u));
-      const int leader = __ffs(peers) - 1;
-      int basepos = 0;
-      if (valid && e >= 0 && e < p.E && lane == leader) basepos = fill[e];
-      basepos = __shfl_sync(0xffffffffu, basepos, leader);
-      if (valid && e >= 0 && e < p.E) p.perm[basepos + rank] = i;
-      __syncwarp();
-      if (valid && e >= 0 && e < p.E && lane == leader) fill[e] = basepos + __popc(peers & mask);
-      __syncwarp();
-    }
-  }
-}
-
 // ------------------------------------------------------------------ launchers
 static cudaError_t launch_ex(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl, void** args) {
   cudaLaunchConfig_t cfg = {};
@@ -622,14 +432,6 @@ cudaError_t launch_route(const RouteParams& p, cudaStream_t s, bool pdl) {
   cudaError_t e = set_smem((const void*)route_logits_kernel, sm);
   if (e != cudaSuccess) return e;
   return launch_ex((const void*)route_logits_kernel, grid, dim3(kRouteThreads), sm, s, pdl, args);
-}
-
-cudaError_t launch_route_gemm(const RouteParams& p, cudaStream_t s) {
-  const int rows = p.E + (p.has_shared ? 1 : 0);
-  dim3 grid((rows + kRgRows - 1) / kRgRows, (p.T + kRgTok - 1) / kRgTok);
-  RouteParams q = p;
-  void* args[] = {&q};
-  return launch_ex((const void*)route_gemm_kernel, grid, dim3(kRgThreads), 0, s, false, args);
 }
 
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t s) {
@@ -676,22 +478,6 @@ cudaError_t launch_gemv(const GemvParams& p, int bits, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   void* args[] = {&q};
   return launch_ex(fn, dim3(p.nCTA), dim3(kThreads), sm, s, false, args);
-}
-
-size_t pf_max_chunks(int T, int k, int E, int chunk) {
-  // sum over experts of ceil(n_e / chunk) <= min(T*k, T*k / chunk + E), plus the shared expert's
-  const size_t pairs = (size_t)T * k;
-  const size_t routed = pairs / chunk + (size_t)E < pairs ? pairs / chunk + (size_t)E : pairs;
-  return routed + ((size_t)T + chunk - 1) / chunk;
-}
-
-cudaError_t launch_group(const GroupParams& p, cudaStream_t s) {
-  const size_t sm = sizeof(int) * 3 * (size_t)p.E;
-  cudaError_t e = set_smem((const void*)group_kernel, sm);
-  if (e != cudaSuccess) return e;
-  GroupParams q = p;
-  void* args[] = {&q};
-  return launch_ex((const void*)group_kernel, dim3(1), dim3(1024), sm, s, false, args);
 }
 
 }  // namespace qmoe

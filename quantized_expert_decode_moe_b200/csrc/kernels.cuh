@@ -101,7 +101,7 @@ struct GemvParams {
 
 struct PrefillParams {
   int H, I, E, k, T, has_shared;
-  int nst, rt;                 // stages and row tiles per item of the grouped kernels (set by their launcher)
+  int nst, rt, rw;             // stages, tile groups and tiles per warp of the grouped kernels (set by their launcher)
   const uint16_t* x;           // [T][H] bf16
   unsigned char* xd;           // [T][2H]   digit tables of x
   float* xX;                   // [T][H/64] group sums of x

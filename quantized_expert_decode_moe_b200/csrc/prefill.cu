@@ -181,25 +181,27 @@ __global__ void __launch_bounds__(kPfDigitThreads) pf_digitize_kernel(const void
 }
 
 // ------------------------------------------------------------------ grouped GEMM geometry
-// An item holds RT tiles of 16 weight rows (gate/up: tile r = 8 gate rows and
-// the 8 up rows of the same intermediate indices). Shared memory: nst stages
-// of {codes [16 RT][stride], scales [16 RT][ng], biases [16 RT][ng]} (stride =
-// row bytes + 8*bits, so the rows a warp reads at one column start 8*bits
-// bytes apart in the banks; gate/up scales and biases are [gate 8 RT][up 8 RT]),
-// partial sums [2][256 rows of (K-slice, tile row)][C], output rows [2][C],
-// one barrier per stage.
+// An item holds TT = RT * RW tiles of 16 weight rows (gate/up: tile r = 8
+// gate rows and the 8 up rows of the same intermediate indices): the 16 warps
+// form RT groups of NS = 16 / RT K-slices, and each warp takes RW consecutive
+// tiles of its slice. Shared memory: nst stages of {codes [16 TT][stride],
+// scales [16 TT][ng], biases [16 TT][ng]} (stride = row bytes + 8*bits, so the
+// rows a warp reads at one column start 8*bits bytes apart in the banks;
+// gate/up scales and biases are [gate 8 TT][up 8 TT]), partial sums
+// [2][NS][16 TT rows][C], output rows [2][C], one barrier per stage.
 struct PfGeom { int RB, SRB, stride, nst; size_t stage, sc, bi, part, rows, bars, total; };
-__host__ __device__ inline PfGeom pf_geom(int K, int bits, int C, int RT, int nst) {
+__host__ __device__ inline PfGeom pf_geom(int K, int bits, int C, int RT, int RW, int nst) {
   PfGeom G;
+  const int TT = RT * RW;   // 16-row tiles per item
   G.RB = K * bits / 8;
   G.SRB = (K / kGroup) * 2;
   G.stride = G.RB + 8 * bits;
-  G.sc = (size_t)16 * RT * G.stride;
-  G.bi = G.sc + (size_t)16 * RT * G.SRB;
-  G.stage = (G.bi + (size_t)16 * RT * G.SRB + 127) & ~(size_t)127;
+  G.sc = (size_t)16 * TT * G.stride;
+  G.bi = G.sc + (size_t)16 * TT * G.SRB;
+  G.stage = (G.bi + (size_t)16 * TT * G.SRB + 127) & ~(size_t)127;
   G.nst = nst;
   size_t o = G.stage * nst;
-  G.part = o; o += sizeof(float) * 2 * kPfWarps * 16 * C;
+  G.part = o; o += sizeof(float) * 2 * kPfWarps * 16 * RW * C;   // [2][NS slices][16 TT rows][C]
   G.rows = o; o += sizeof(int) * 2 * C;
   o = (o + 15) & ~(size_t)15;
   G.bars = o; o += sizeof(uint64_t) * kPfMaxStages;
@@ -237,12 +239,15 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_grouped_kernel(PrefillP
   extern __shared__ __align__(128) unsigned char smem[];
   constexpr int C = 4 * TILES;
   const int K = GU ? p.H : p.I;
-  const int RT = p.rt;                                 // row tiles per item (1, 2 or 4)
+  const int RT = p.rt;                                 // tile groups per item (1, 2 or 4)
+  const int RW = p.rw;                                 // tiles per warp (1 or 2)
+  const int TT = RT * RW;                              // 16-row tiles per item
   const int rshift = RT == 1 ? 0 : (RT == 2 ? 1 : 2);
+  const int tshift = rshift + (RW == 2 ? 1 : 0);       // log2 TT
   const int NS = kPfWarps >> rshift;                   // K-slices
-  const int R = GU ? p.I / (8 * RT) : p.H / (16 * RT); // items per chunk
+  const int R = GU ? p.I / (8 * TT) : p.H / (16 * TT); // items per chunk
   const int ng = K / kGroup;
-  const PfGeom G = pf_geom(K, BITS, C, RT, p.nst);
+  const PfGeom G = pf_geom(K, BITS, C, RT, RW, p.nst);
   const int nst = G.nst;
   uint64_t* full = (uint64_t*)(smem + G.bars);
   float* part = (float*)(smem + G.part);
@@ -256,7 +261,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_grouped_kernel(PrefillP
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  const unsigned item_bytes = 16u * RT * G.RB + 32u * RT * G.SRB;
+  const unsigned item_bytes = 16u * TT * G.RB + 32u * TT * G.SRB;
   const int ci0 = (int)(lo / R), rb0 = (int)(lo - (long long)ci0 * R);
 
   // Copies of the next item to issue (cursor ici, irb) into stage st. Lane 0
@@ -283,16 +288,16 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_grouped_kernel(PrefillP
       }
     }
     unsigned char* sb = smem + (size_t)st * G.stage;
-    for (int r = warp; r < 16 * RT; r += kPfWarps) {
+    for (int r = warp; r < 16 * TT; r += kPfWarps) {
       const int tr = r >> 4, q = r & 15;
-      const int src = GU ? irb * 8 * RT + 8 * tr + (q & 7) : irb * 16 * RT + r;
+      const int src = GU ? irb * 8 * TT + 8 * tr + (q & 7) : irb * 16 * TT + r;
       pf_bulk(sb + (size_t)r * G.stride, mq + (size_t)src * G.RB, G.RB, &full[st]);
     }
     if (GU && warp < 4)   // 0 gate scales, 1 up scales, 2 gate biases, 3 up biases
-      pf_bulk(sb + (warp < 2 ? G.sc : G.bi) + (size_t)(warp & 1) * 8 * RT * G.SRB,
-              msb + (size_t)irb * 8 * RT * G.SRB, 8u * RT * G.SRB, &full[st]);
+      pf_bulk(sb + (warp < 2 ? G.sc : G.bi) + (size_t)(warp & 1) * 8 * TT * G.SRB,
+              msb + (size_t)irb * 8 * TT * G.SRB, 8u * TT * G.SRB, &full[st]);
     else if (!GU && warp < 2)
-      pf_bulk(sb + (warp == 0 ? G.sc : G.bi), msb + (size_t)irb * 16 * RT * G.SRB, 16u * RT * G.SRB, &full[st]);
+      pf_bulk(sb + (warp == 0 ? G.sc : G.bi), msb + (size_t)irb * 16 * TT * G.SRB, 16u * TT * G.SRB, &full[st]);
     if (++irb == R) { irb = 0; ++ici; }
   };
   if (tid == 0)
@@ -302,7 +307,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_grouped_kernel(PrefillP
     for (int i = 0; i < nloc && i < nst; ++i) issue(i);
 
   const int g = lane >> 2, t = lane & 3;
-  const int tr = warp >> (4 - rshift), ks = warp & (NS - 1);   // row tile, K-slice
+  const int tg = warp >> (4 - rshift), ks = warp & (NS - 1);   // tile group, K-slice
   const int gpw = (ng + NS - 1) / NS;
   const int g0 = ks * gpw;
   const int mg = max(0, min(gpw, ng - g0));   // groups of this warp
@@ -310,9 +315,6 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_grouped_kernel(PrefillP
   const float* Xt = GU ? p.xX : p.aX;
   const float* rst = GU ? p.xrs : p.ars;
   const bool vec_sb = (mg == GPW) && (ng % GPW == 0);   // the warp's scales in one load per row
-  // shared-memory rows of this warp's tile: A rows g (gate / first 8) and g+8 (up / last 8)
-  const int crA = 16 * tr + g, crB = 16 * tr + 8 + g;
-  const int srA = GU ? 8 * tr + g : crA, srB = GU ? 8 * RT + 8 * tr + g : crB;
   uint4 bq[TILES][GPW];
   float xg[TILES][GPW], rsc[TILES];
   int cur = -1, n = 0, orow = -1;
@@ -344,79 +346,85 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_grouped_kernel(PrefillP
     const unsigned char* sb = smem + (size_t)st * G.stage;
     const uint16_t* ssc = (const uint16_t*)(sb + G.sc);
     const uint16_t* sbi = (const uint16_t*)(sb + G.bi);
-    // scales / biases of the warp's two rows for its groups
-    float sA[GPW], sB[GPW], bA[GPW], bB[GPW];
-    if (vec_sb) {
-      using V = typename std::conditional<GPW == 4, uint2, uint4>::type;
-      const V va = *(const V*)(ssc + (size_t)srA * ng + g0), vb = *(const V*)(ssc + (size_t)srB * ng + g0);
-      const V wa = *(const V*)(sbi + (size_t)srA * ng + g0), wb = *(const V*)(sbi + (size_t)srB * ng + g0);
-      const uint32_t* pa = (const uint32_t*)&va;
-      const uint32_t* pb = (const uint32_t*)&vb;
-      const uint32_t* qa = (const uint32_t*)&wa;
-      const uint32_t* qb = (const uint32_t*)&wb;
+    float* pw = part + ((size_t)(i & 1) * NS + ks) * 16 * TT * C;   // part[buf][ks][tile row][token]
+#pragma unroll 1
+    for (int rr = 0; rr < RW; ++rr) {   // the warp's tiles, one at a time
+      const int tr = tg * RW + rr;
+      // shared-memory rows of the tile: A rows g (gate / first 8) and g+8 (up / last 8)
+      const int crA = 16 * tr + g, crB = 16 * tr + 8 + g;
+      const int srA = GU ? 8 * tr + g : crA, srB = GU ? 8 * TT + 8 * tr + g : crB;
+      // scales / biases of the warp's two rows for its groups
+      float sA[GPW], sB[GPW], bA[GPW], bB[GPW];
+      if (vec_sb) {
+        using V = typename std::conditional<GPW == 4, uint2, uint4>::type;
+        const V va = *(const V*)(ssc + (size_t)srA * ng + g0), vb = *(const V*)(ssc + (size_t)srB * ng + g0);
+        const V wa = *(const V*)(sbi + (size_t)srA * ng + g0), wb = *(const V*)(sbi + (size_t)srB * ng + g0);
+        const uint32_t* pa = (const uint32_t*)&va;
+        const uint32_t* pb = (const uint32_t*)&vb;
+        const uint32_t* qa = (const uint32_t*)&wa;
+        const uint32_t* qb = (const uint32_t*)&wb;
 #pragma unroll
-      for (int h = 0; h < GPW / 2; ++h) {
-        sA[2 * h] = bf16_lo(pa[h]); sA[2 * h + 1] = bf16_hi(pa[h]);
-        sB[2 * h] = bf16_lo(pb[h]); sB[2 * h + 1] = bf16_hi(pb[h]);
-        bA[2 * h] = bf16_lo(qa[h]); bA[2 * h + 1] = bf16_hi(qa[h]);
-        bB[2 * h] = bf16_lo(qb[h]); bB[2 * h + 1] = bf16_hi(qb[h]);
-      }
-    } else {
-#pragma unroll
-      for (int gi = 0; gi < GPW; ++gi) {
-        sA[gi] = sB[gi] = bA[gi] = bB[gi] = 0.f;
-        if (gi < mg) {
-          const int gg = g0 + gi;
-          sA[gi] = bf16_lo(ssc[(size_t)srA * ng + gg]); sB[gi] = bf16_lo(ssc[(size_t)srB * ng + gg]);
-          bA[gi] = bf16_lo(sbi[(size_t)srA * ng + gg]); bB[gi] = bf16_lo(sbi[(size_t)srB * ng + gg]);
+        for (int h = 0; h < GPW / 2; ++h) {
+          sA[2 * h] = bf16_lo(pa[h]); sA[2 * h + 1] = bf16_hi(pa[h]);
+          sB[2 * h] = bf16_lo(pb[h]); sB[2 * h + 1] = bf16_hi(pb[h]);
+          bA[2 * h] = bf16_lo(qa[h]); bA[2 * h + 1] = bf16_hi(qa[h]);
+          bB[2 * h] = bf16_lo(qb[h]); bB[2 * h + 1] = bf16_hi(qb[h]);
         }
-      }
-    }
-    float sacc[TILES][2], bacc[TILES][2];
+      } else {
 #pragma unroll
-    for (int tau = 0; tau < TILES; ++tau) sacc[tau][0] = sacc[tau][1] = bacc[tau][0] = bacc[tau][1] = 0.f;
-    const unsigned char* ra = sb + (size_t)crA * G.stride;
-    const unsigned char* rbp = sb + (size_t)crB * G.stride;
-#pragma unroll
-    for (int gi = 0; gi < GPW; ++gi) {
-      if (gi < mg) {
-        const int grp = g0 + gi;
-        uint32_t A[2][4];   // per MMA m: a0 (row g, h 0), a1 (row g+8, h 0), a2 (row g, h 1), a3 (row g+8, h 1)
-        if constexpr (BITS == 4) {
-          const uint2 ua = *(const uint2*)(ra + grp * 32 + 8 * t), ub = *(const uint2*)(rbp + grp * 32 + 8 * t);
-          A[0][0] = ua.x & 0x0F0F0F0Fu; A[0][2] = (ua.x >> 4) & 0x0F0F0F0Fu;
-          A[0][1] = ub.x & 0x0F0F0F0Fu; A[0][3] = (ub.x >> 4) & 0x0F0F0F0Fu;
-          A[1][0] = ua.y & 0x0F0F0F0Fu; A[1][2] = (ua.y >> 4) & 0x0F0F0F0Fu;
-          A[1][1] = ub.y & 0x0F0F0F0Fu; A[1][3] = (ub.y >> 4) & 0x0F0F0F0Fu;
-        } else {
-          const uint32_t ua = *(const uint32_t*)(ra + grp * 16 + 4 * t);
-          const uint32_t ub = *(const uint32_t*)(rbp + grp * 16 + 4 * t);
-#pragma unroll
-          for (int m = 0; m < 2; ++m) {
-            A[m][0] = (ua >> (4 * m)) & 0x03030303u; A[m][2] = (ua >> (4 * m + 2)) & 0x03030303u;
-            A[m][1] = (ub >> (4 * m)) & 0x03030303u; A[m][3] = (ub >> (4 * m + 2)) & 0x03030303u;
+        for (int gi = 0; gi < GPW; ++gi) {
+          sA[gi] = sB[gi] = bA[gi] = bB[gi] = 0.f;
+          if (gi < mg) {
+            const int gg = g0 + gi;
+            sA[gi] = bf16_lo(ssc[(size_t)srA * ng + gg]); sB[gi] = bf16_lo(ssc[(size_t)srB * ng + gg]);
+            bA[gi] = bf16_lo(sbi[(size_t)srA * ng + gg]); bB[gi] = bf16_lo(sbi[(size_t)srB * ng + gg]);
           }
         }
+      }
+      float sacc[TILES][2], bacc[TILES][2];
 #pragma unroll
-        for (int tau = 0; tau < TILES; ++tau) {
-          int c[4] = {0, 0, 0, 0};
-          const uint4 b = bq[tau][gi];
-          mma_u8s8(c, A[0][0], A[0][1], A[0][2], A[0][3], b.x, b.y);
-          mma_u8s8(c, A[1][0], A[1][1], A[1][2], A[1][3], b.z, b.w);
-          // columns 2t, 2t+1 of the tile: token t's high- and low-digit sums
-          sacc[tau][0] = fmaf(sA[gi], (float)(c[0] * 256 + c[1]), sacc[tau][0]);
-          sacc[tau][1] = fmaf(sB[gi], (float)(c[2] * 256 + c[3]), sacc[tau][1]);
-          bacc[tau][0] = fmaf(bA[gi], xg[tau][gi], bacc[tau][0]);
-          bacc[tau][1] = fmaf(bB[gi], xg[tau][gi], bacc[tau][1]);
+      for (int tau = 0; tau < TILES; ++tau) sacc[tau][0] = sacc[tau][1] = bacc[tau][0] = bacc[tau][1] = 0.f;
+      const unsigned char* ra = sb + (size_t)crA * G.stride;
+      const unsigned char* rbp = sb + (size_t)crB * G.stride;
+#pragma unroll
+      for (int gi = 0; gi < GPW; ++gi) {
+        if (gi < mg) {
+          const int grp = g0 + gi;
+          uint32_t A[2][4];   // per MMA m: a0 (row g, h 0), a1 (row g+8, h 0), a2 (row g, h 1), a3 (row g+8, h 1)
+          if constexpr (BITS == 4) {
+            const uint2 ua = *(const uint2*)(ra + grp * 32 + 8 * t), ub = *(const uint2*)(rbp + grp * 32 + 8 * t);
+            A[0][0] = ua.x & 0x0F0F0F0Fu; A[0][2] = (ua.x >> 4) & 0x0F0F0F0Fu;
+            A[0][1] = ub.x & 0x0F0F0F0Fu; A[0][3] = (ub.x >> 4) & 0x0F0F0F0Fu;
+            A[1][0] = ua.y & 0x0F0F0F0Fu; A[1][2] = (ua.y >> 4) & 0x0F0F0F0Fu;
+            A[1][1] = ub.y & 0x0F0F0F0Fu; A[1][3] = (ub.y >> 4) & 0x0F0F0F0Fu;
+          } else {
+            const uint32_t ua = *(const uint32_t*)(ra + grp * 16 + 4 * t);
+            const uint32_t ub = *(const uint32_t*)(rbp + grp * 16 + 4 * t);
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+              A[m][0] = (ua >> (4 * m)) & 0x03030303u; A[m][2] = (ua >> (4 * m + 2)) & 0x03030303u;
+              A[m][1] = (ub >> (4 * m)) & 0x03030303u; A[m][3] = (ub >> (4 * m + 2)) & 0x03030303u;
+            }
+          }
+#pragma unroll
+          for (int tau = 0; tau < TILES; ++tau) {
+            int c[4] = {0, 0, 0, 0};
+            const uint4 b = bq[tau][gi];
+            mma_u8s8(c, A[0][0], A[0][1], A[0][2], A[0][3], b.x, b.y);
+            mma_u8s8(c, A[1][0], A[1][1], A[1][2], A[1][3], b.z, b.w);
+            // columns 2t, 2t+1 of the tile: token t's high- and low-digit sums
+            sacc[tau][0] = fmaf(sA[gi], (float)(c[0] * 256 + c[1]), sacc[tau][0]);
+            sacc[tau][1] = fmaf(sB[gi], (float)(c[2] * 256 + c[3]), sacc[tau][1]);
+            bacc[tau][0] = fmaf(bA[gi], xg[tau][gi], bacc[tau][0]);
+            bacc[tau][1] = fmaf(bB[gi], xg[tau][gi], bacc[tau][1]);
+          }
         }
       }
-    }
-    // partials: part[buf][ks][tile row][token]
-    float* pw = part + ((size_t)(i & 1) * kPfWarps * 16 + (size_t)ks * 16 * RT) * C;
 #pragma unroll
-    for (int tau = 0; tau < TILES; ++tau) {
-      pw[crA * C + 4 * tau + t] = fmaf(sacc[tau][0], rsc[tau], bacc[tau][0]);
-      pw[crB * C + 4 * tau + t] = fmaf(sacc[tau][1], rsc[tau], bacc[tau][1]);
+      for (int tau = 0; tau < TILES; ++tau) {
+        pw[crA * C + 4 * tau + t] = fmaf(sacc[tau][0], rsc[tau], bacc[tau][0]);
+        pw[crB * C + 4 * tau + t] = fmaf(sacc[tau][1], rsc[tau], bacc[tau][1]);
+      }
     }
     if (tid == 0 && i + nst < nloc) pf_expect(&full[st], item_bytes);   // its phase for item i is complete
     __syncthreads();
@@ -425,12 +433,12 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_grouped_kernel(PrefillP
       issue(st);
     }
     // outputs: one thread per output adds the NS slices' partials in slice order
-    const float* pr = part + (size_t)(i & 1) * kPfWarps * 16 * C;
+    const float* pr = part + (size_t)(i & 1) * NS * 16 * TT * C;
     const int* ro = rows_out + (i & 1) * C;
-    const int slice = 16 * RT * C;   // floats per slice
+    const int slice = 16 * TT * C;   // floats per slice
     if (GU) {
-      if (tid < 8 * RT * C) {   // tid = x * 8 RT + jj
-        const int x = tid >> (3 + rshift), jj = tid & (8 * RT - 1);
+      for (int o = tid; o < 8 * TT * C; o += kPfThreads) {   // o = x * 8 TT + jj
+        const int x = o >> (3 + tshift), jj = o & (8 * TT - 1);
         const int prow = 16 * (jj >> 3) + (jj & 7);
         const float* pq = pr + prow * C + x;
         float gs = 0.f, us = 0.f;
@@ -438,14 +446,16 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_grouped_kernel(PrefillP
           gs += pq[w * slice];
           us += pq[w * slice + 8 * C];
         }
-        if (x < n) p.a[(size_t)ro[x] * p.I + rb * 8 * RT + jj] = gs / (1.f + expf(-gs)) * us;
+        if (x < n) p.a[(size_t)ro[x] * p.I + rb * 8 * TT + jj] = gs / (1.f + expf(-gs)) * us;
       }
-    } else if (tid < 16 * RT * C) {   // tid = x * 16 RT + rr
-      const int x = tid >> (4 + rshift), rr = tid & (16 * RT - 1);
-      const float* pq = pr + rr * C + x;
-      float y = 0.f;
-      for (int w = 0; w < NS; ++w) y += pq[w * slice];
-      if (x < n) p.y[(size_t)ro[x] * p.H + rb * 16 * RT + rr] = y;
+    } else {
+      for (int o = tid; o < 16 * TT * C; o += kPfThreads) {   // o = x * 16 TT + rr
+        const int x = o >> (4 + tshift), rr = o & (16 * TT - 1);
+        const float* pq = pr + rr * C + x;
+        float y = 0.f;
+        for (int w = 0; w < NS; ++w) y += pq[w * slice];
+        if (x < n) p.y[(size_t)ro[x] * p.H + rb * 16 * TT + rr] = y;
+      }
     }
     if (++st == nst) { st = 0; phase ^= 1u; }
     if (++rb == R) { rb = 0; ++ci; }
@@ -456,7 +466,217 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_grouped_kernel(PrefillP
       pf_wait(&full[i % nst], (unsigned)(i / nst) & 1u, p.wait_ns, nullptr);
 }
 
+// ------------------------------------------------------------------ router of many tokens
+// Router logits of many tokens (prefill): a tiled GEMM in fp64. Every
+// product of two bf16 values is exact in fp64, and each logit is accumulated
+// over k in index order from 0 by one thread, then the bias is added: the
+// same sequence of roundings as the plain fp64 loop of the definition
+// (logits l = W_r x + b, "Model architecture" of the Flash-MoE write-up), so
+// the logits are reproduced exactly. That order makes each logit a chain of
+// H dependent fp64 FMAs, so the kernel's time is about H times the FMA
+// latency once every chain is in flight (2 x 4 per thread here). Tile: 32
+// tokens x 32 router rows per CTA; thread (ty, tx) holds tokens 2ty, 2ty+1
+// and rows 4tx..4tx+3; operands are staged in shared memory as doubles,
+// k-major.
+constexpr int kRgTok = 32, kRgRows = 32, kRgK = 32, kRgThreads = 128;
+
+// bf16 bit pattern -> double, exactly: normal values and zeros by moving the
+// fields (exponent bias 127 -> 1023), the rest through float.
+__device__ __forceinline__ double bf16_to_f64(uint32_t b) {
+  const uint32_t e = (b >> 7) & 0xFFu;
+  uint32_t hi = ((b & 0x8000u) << 16) | ((e + 896u) << 20) | ((b & 0x7Fu) << 13);
+  if ((b & 0x7FFFu) == 0u) hi = (b & 0x8000u) << 16;
+  else if (e == 0u || e == 0xFFu) return (double)__uint_as_float(b << 16);
+  return __hiloint2double((int)hi, 0);
+}
+
+__global__ void __launch_bounds__(kRgThreads) route_gemm_kernel(RouteParams p) {
+  __shared__ __align__(16) double xs[kRgK][kRgTok];    // [k][token]
+  __shared__ __align__(16) double ws[kRgK][kRgRows];   // [k][row pair b/2][tx][b%2]
+  const int tid = threadIdx.x, tx = tid & 7, ty = tid >> 3;
+  const int e0 = blockIdx.x * kRgRows, t0 = blockIdx.y * kRgTok;
+  const int nrows = p.E + (p.has_shared ? 1 : 0);
+  double acc[2][4];
+#pragma unroll
+  for (int a = 0; a < 2; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
+  // global tiles: x 32 tokens x 32 k and W 32 rows x 32 k, one uint4 (8 k) of each per thread
+  const int lr = tid >> 2, lc = tid & 3;
+  const uint16_t* xrow = t0 + lr < p.T ? p.x + (size_t)(t0 + lr) * p.H : nullptr;
+  const int we = e0 + lr;
+  const uint16_t* wrow = we < p.E ? p.router_w + (size_t)we * p.H : (we < nrows ? p.gate_w : nullptr);
+  const int wpos = ((lr & 3) >> 1) * 16 + (lr >> 2) * 2 + (lr & 1);   // row 4 tx + b at (b/2, tx, b%2)
+  auto load = [&](int k0, uint4& xv, uint4& wv) {
+    xv = xrow ? __ldg((const uint4*)(xrow + k0 + 8 * lc)) : make_uint4(0u, 0u, 0u, 0u);
+    wv = wrow ? __ldg((const uint4*)(wrow + k0 + 8 * lc)) : make_uint4(0u, 0u, 0u, 0u);
+  };
+  uint4 xv, wv;
+  load(0, xv, wv);
+  for (int k0 = 0; k0 < p.H; k0 += kRgK) {
+    __syncthreads();   // the previous tile has been read
+    {
+      const uint32_t u[4] = {xv.x, xv.y, xv.z, xv.w}, v[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        xs[8 * lc + 2 * i][lr] = bf16_to_f64(u[i] & 0xFFFFu);
+        xs[8 * lc + 2 * i + 1][lr] = bf16_to_f64(u[i] >> 16);
+        ws[8 * lc + 2 * i][wpos] = bf16_to_f64(v[i] & 0xFFFFu);
+        ws[8 * lc + 2 * i + 1][wpos] = bf16_to_f64(v[i] >> 16);
+      }
+    }
+    __syncthreads();
+    if (k0 + kRgK < p.H) load(k0 + kRgK, xv, wv);   // next tile in flight during the products
+#pragma unroll 8
+    for (int kk = 0; kk < kRgK; ++kk) {
+      const double2 xa = *(const double2*)&xs[kk][2 * ty];
+      const double2 w0 = *(const double2*)&ws[kk][tx * 2];
+      const double2 w1 = *(const double2*)&ws[kk][16 + tx * 2];
+      const double w4[4] = {w0.x, w0.y, w1.x, w1.y};
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        acc[0][b] = fma(w4[b], xa.x, acc[0][b]);
+        acc[1][b] = fma(w4[b], xa.y, acc[1][b]);
+      }
+    }
+  }
+#pragma unroll
+  for (int a = 0; a < 2; ++a) {
+    const int t = t0 + 2 * ty + a;
+    if (t >= p.T) continue;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int e = e0 + 4 * tx + b;
+      if (e >= nrows) continue;
+      double v = acc[a][b];
+      if (e < p.E && p.router_bias) v += (double)p.router_bias[e];
+      p.logits[(size_t)t * (p.E + 1) + e] = v;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ grouping by expert
+// Exclusive scan of v[0..n) in place (one block); returns the total.
+__device__ int block_exclusive_scan(int* v, int n, int* warp_tot) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  int carry = 0;
+  for (int base = 0; base < n; base += blockDim.x) {
+    const int e = base + tid;
+    const int x = e < n ? v[e] : 0;
+    int incl = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      int wv = lane < nw ? warp_tot[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, wv, o);
+        if (lane >= o) wv += y;
+      }
+      if (lane < nw) warp_tot[lane] = wv;
+    }
+    __syncthreads();
+    if (e < n) v[e] = carry + (warp ? warp_tot[warp - 1] : 0) + incl - x;
+    const int tot = warp_tot[nw - 1];
+    __syncthreads();
+    carry += tot;
+  }
+  return carry;
+}
+
+// Prefill grouping in one CTA: histogram of the chosen experts, exclusive
+// scan, then a stable scatter of the flattened (token, rank) pairs by one warp
+// that walks them in order 32 at a time (ranks of equal experts from
+// __match_any_sync). Also the chunk list of the grouped GEMMs: expert e's
+// pairs in runs of `chunk`, then the shared expert's tokens in runs of `chunk`.
+__global__ void __launch_bounds__(1024) group_kernel(GroupParams p) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  int* cnt = (int*)smem;            // [E]
+  int* fill = cnt + p.E;            // [E]
+  int* cb = fill + p.E;             // [E] first chunk of each expert
+  __shared__ int warp_tot[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int N = p.T * p.k, C = p.chunk;
+  for (int e = tid; e < p.E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  for (int i = tid; i < N; i += blockDim.x) {
+    const int e = p.idx[i];
+    if (e >= 0 && e < p.E) atomicAdd(&cnt[e], 1);
+  }
+  __syncthreads();
+  for (int e = tid; e < p.E; e += blockDim.x) {
+    p.counts[e] = cnt[e];
+    fill[e] = cnt[e];
+    cb[e] = C > 0 ? (cnt[e] + C - 1) / C : 0;
+  }
+  __syncthreads();
+  const int total = block_exclusive_scan(fill, p.E, warp_tot);
+  const int nrouted = block_exclusive_scan(cb, p.E, warp_tot);
+  const bool chunked = p.chunks != nullptr && p.nchunks != nullptr && C > 0;   // the grouped GEMMs' list
+  for (int e = tid; e < p.E; e += blockDim.x) {
+    p.offsets[e] = fill[e];
+    if (chunked)
+      for (int c = 0; c * C < cnt[e]; ++c)
+        p.chunks[cb[e] + c] = make_int4(e, fill[e] + c * C, min(C, cnt[e] - c * C), 0);
+  }
+  const int nshared = chunked && p.has_shared ? (p.T + C - 1) / C : 0;
+  for (int c = tid; c < nshared; c += blockDim.x)
+    p.chunks[nrouted + c] = make_int4(p.E, c * C, min(C, p.T - c * C), 0);
+  if (tid == 0) {
+    p.offsets[p.E] = total;
+    if (chunked) *p.nchunks = nrouted + nshared;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    for (int base = 0; base < N; base += 32) {
+      const int i = base + lane;
+      const bool valid = i < N;
+      const int e = valid ? p.idx[i] : -1;
+      const unsigned mask = __ballot_sync(0xffffffffu, valid);
+      const unsigned peers = __match_any_sync(0xffffffffu, e);
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      const int leader = __ffs(peers) - 1;
+      int basepos = 0;
+      if (valid && e >= 0 && e < p.E && lane == leader) basepos = fill[e];
+      basepos = __shfl_sync(0xffffffffu, basepos, leader);
+      if (valid && e >= 0 && e < p.E) p.perm[basepos + rank] = i;
+      __syncwarp();
+      if (valid && e >= 0 && e < p.E && lane == leader) fill[e] = basepos + __popc(peers & mask);
+      __syncwarp();
+    }
+  }
+}
+
 // ------------------------------------------------------------------ launchers
+size_t pf_max_chunks(int T, int k, int E, int chunk) {
+  // sum over experts of ceil(n_e / chunk) <= min(T*k, T*k / chunk + E), plus the shared expert's
+  const size_t pairs = (size_t)T * k;
+  const size_t routed = pairs / chunk + (size_t)E < pairs ? pairs / chunk + (size_t)E : pairs;
+  return routed + ((size_t)T + chunk - 1) / chunk;
+}
+
+cudaError_t launch_group(const GroupParams& p, cudaStream_t s) {
+  const size_t sm = sizeof(int) * 3 * (size_t)p.E;
+  cudaError_t e = cudaFuncSetAttribute((const void*)group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (e != cudaSuccess) return e;
+  GroupParams q = p;
+  void* args[] = {&q};
+  return cudaLaunchKernel((const void*)group_kernel, dim3(1), dim3(1024), args, sm, s);
+}
+
+cudaError_t launch_route_gemm(const RouteParams& p, cudaStream_t s) {
+  const int rows = p.E + (p.has_shared ? 1 : 0);
+  dim3 grid((rows + kRgRows - 1) / kRgRows, (p.T + kRgTok - 1) / kRgTok);
+  RouteParams q = p;
+  void* args[] = {&q};
+  return cudaLaunchKernel((const void*)route_gemm_kernel, grid, dim3(kRgThreads), args, 0, s);
+}
+
 int pf_chunk_tokens(int H, int I) { return (H > 4096 || I > 4096) ? 4 : 8; }
 
 static cudaError_t pf_prepare(const void* fn, size_t bytes) {
@@ -472,19 +692,26 @@ static cudaError_t pf_grouped(const PrefillParams& p, cudaStream_t s) {
   const int RT = C == 8 ? pf_row_tiles(K) : 1;
   const int ng = K / kGroup, NS = kPfWarps / RT, gpw = (ng + NS - 1) / NS;
   if (gpw > (C == 8 ? 4 : 8)) return cudaErrorInvalidConfiguration;
-  if ((GU ? p.I % (8 * RT) : p.H % (16 * RT)) != 0) return cudaErrorInvalidConfiguration;
+  const int rows = GU ? p.I / 8 : p.H / 16;   // 16-row tiles per expert matrix
+  if (rows % RT != 0) return cudaErrorInvalidConfiguration;
   int optin = 0, dev = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-  const size_t fixed = pf_geom(K, BITS, C, RT, 0).total;
-  const size_t stage = pf_geom(K, BITS, C, RT, 1).stage;
-  if ((size_t)optin < fixed + 2 * stage) return cudaErrorInvalidConfiguration;
-  int nst = (int)(((size_t)optin - fixed) / stage);
-  if (nst > kPfMaxStages) nst = kPfMaxStages;
+  auto stages = [&](int rw) {
+    const size_t fixed = pf_geom(K, BITS, C, RT, rw, 0).total, stage = pf_geom(K, BITS, C, RT, rw, 1).stage;
+    if ((size_t)optin < fixed + 2 * stage) return 0;
+    const int n = (int)(((size_t)optin - fixed) / stage);
+    return n > kPfMaxStages ? kPfMaxStages : n;
+  };
+  // two tiles per warp where the shapes divide and two stages still fit
+  const int RW = (C == 8 && rows % (2 * RT) == 0 && stages(2) >= 2) ? 2 : 1;
+  const int nst = stages(RW);
+  if (nst < 2) return cudaErrorInvalidConfiguration;
   PrefillParams q = p;
   q.nst = nst;
   q.rt = RT;
-  const size_t sm = pf_geom(K, BITS, C, RT, nst).total;
+  q.rw = RW;
+  const size_t sm = pf_geom(K, BITS, C, RT, RW, nst).total;
   const void* fn = C == 8 ? (const void*)prefill_grouped_kernel<BITS, GU, 4, 2>
                           : (const void*)prefill_grouped_kernel<BITS, GU, 8, 1>;
   cudaError_t e = pf_prepare(fn, sm);

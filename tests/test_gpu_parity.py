@@ -135,6 +135,35 @@ def test_route_matches_oracle(dev, name):
     np.testing.assert_allclose(sg.cpu().numpy(), rsg, rtol=1e-6, atol=1e-7)
 
 
+def test_route_logits_equal_fp64_definition(dev):
+    """Many tokens (T > 8): every logit equals the plain fp64 loop of the
+    definition bit for bit (bf16 products are exact in fp64; each logit is
+    accumulated in index order and the bias added last). moe_route leaves the
+    logits in the workspace: double [T][E+1] at byte 256, column E the
+    shared-gate logit."""
+    cfg = fixtures.CONFIGS["stack_q4"]   # the biased router
+    Wr, rb, gs, gamma = fixtures.layer_vectors(cfg, 0)
+    dummy = torch.zeros(64, dtype=torch.int32, device=dev)
+    ex = qm.Expert(*[qm.QMat(dummy, dummy, dummy)] * 3)
+    layer = qm.Layer(hidden=cfg.H, inter=cfg.I, top_k=cfg.k, bits=cfg.bits,
+                     router_w=torch.from_numpy(Wr.view(np.int16)).to(dev), experts=[ex] * cfg.E,
+                     rms_gamma=torch.from_numpy(gamma.view(np.int16)).to(dev), shared=ex,
+                     shared_gate_w=torch.from_numpy(gs.view(np.int16)).to(dev),
+                     router_bias=torch.from_numpy(rb).to(dev))
+    T = 40
+    x = gen.x_tokens(cfg, 5, T=T)
+    ws = qm.new_workspace(layer, T)
+    idx = torch.empty((T, cfg.k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, cfg.k), dtype=torch.float32, device=dev)
+    qm.moe_route(layer, torch.from_numpy(x.view(np.int16)).to(dev), idx, w, ws=ws)
+    torch.cuda.synchronize()
+    got = ws[256:256 + 8 * T * (cfg.E + 1)].cpu().numpy().view(np.float64).reshape(T, cfg.E + 1)
+    _, _, _, ref = oracle.route(x, Wr, cfg.k, bias=rb, want_logits=True)
+    np.testing.assert_array_equal(got[:, :cfg.E], ref)
+    _, _, _, ref_g = oracle.route(x, gs[None, :], 1, want_logits=True)
+    np.testing.assert_array_equal(got[:, cfg.E], ref_g[:, 0])
+
+
 @pytest.mark.parametrize("E,k", [(512, 8), (4096, 8), (4096, 3), (100, 5)])
 def test_route_wide_pools_and_top8(dev, E, k):
     """Random router, with exact duplicate rows 37 apart (equal logits that land
