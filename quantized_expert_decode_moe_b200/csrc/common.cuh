@@ -56,40 +56,9 @@ __device__ __forceinline__ uint4 ldg_stream_v4(const void* p) {
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
   return r;
 }
-__device__ __forceinline__ uint2 ldg_stream_v2(const void* p) {
-  uint2 r;
-  asm("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
-  return r;
-}
-__device__ __forceinline__ uint32_t ldg_stream_u32(const void* p) {
-  uint32_t r;
-  asm("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(r) : "l"(p));
-  return r;
-}
 // coherent (L2) loads of data written by an earlier kernel of the same chain
-__device__ __forceinline__ double ldcg_f64(const double* p) { return __ldcg(p); }
 __device__ __forceinline__ float ldcg_f32(const float* p) { return __ldcg(p); }
 __device__ __forceinline__ int ldcg_i32(const int* p) { return __ldcg(p); }
-
-// Hint HBM -> L2 for [p, p+bytes); only whole 16-byte pieces inside the range.
-__device__ __forceinline__ void prefetch_l2_range(const void* p, size_t bytes) {
-  uintptr_t a = (uintptr_t)p;
-  uintptr_t lo = (a + 15) & ~(uintptr_t)15;
-  uintptr_t hi = (a + bytes) & ~(uintptr_t)15;
-  while (lo < hi) {
-    uint32_t n = (uint32_t)((hi - lo) < 65536 ? (hi - lo) : 65536);
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(lo), "r"(n) : "memory");
-    lo += n;
-  }
-}
-// Part `part` of `nparts` of [p, p+bytes), for spreading one prefetch over CTAs.
-__device__ __forceinline__ void prefetch_l2_part(const void* p, size_t bytes, int part, int nparts) {
-  size_t per = ((bytes + nparts - 1) / nparts + 15) & ~(size_t)15;
-  size_t lo = per * (size_t)part;
-  if (lo >= bytes) return;
-  size_t hi = lo + per < bytes ? lo + per : bytes;
-  prefetch_l2_range((const char*)p + lo, hi - lo);
-}
 
 // ------------------------------------------------------------------ programmatic dependent launch
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }

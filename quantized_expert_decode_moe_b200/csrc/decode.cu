@@ -79,20 +79,6 @@ __host__ __device__ __forceinline__ int sb_region(int rows, int SRB) { return (r
 
 __device__ __forceinline__ float silu_f32(float z) { return z / (1.f + expf(-z)); }
 
-// A fragments of one span for MMA rows g (from ra) and g+8 (from rb), t = lane & 3.
-template <int BITS>
-__device__ __forceinline__ void frag_codes(Frag<BITS>& F, const unsigned char* ra, const unsigned char* rb) {
-  if constexpr (BITS == 4) {
-    const uint4 va = *(const uint4*)ra, vb = *(const uint4*)rb;
-    F.wa[0] = va.x; F.wa[1] = va.y; F.wa[2] = va.z; F.wa[3] = va.w;
-    F.wb[0] = vb.x; F.wb[1] = vb.y; F.wb[2] = vb.z; F.wb[3] = vb.w;
-  } else {
-    const uint2 va = *(const uint2*)ra, vb = *(const uint2*)rb;
-    F.wa[0] = va.x; F.wa[1] = va.y;
-    F.wb[0] = vb.x; F.wb[1] = vb.y;
-  }
-}
-
 // Loads the table builder's elements of chunk q of a bf16 vector.
 template <int BITS>
 __device__ __forceinline__ void load_chunk_bf16(const uint16_t* x, int q, float (&v)[TabTraits<BITS>::kEPT]) {
@@ -127,11 +113,6 @@ __device__ __forceinline__ uint4 lds_chunk(const unsigned char* p, bool al16) {
 __device__ __forceinline__ uint32_t chunk_word(const uint4& v, int i) {
   return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
 }
-// Code rows in shared memory are padded so that MMA rows g and g+1 (read by
-// the same 8-lane phase of a 16-byte load, or 16-lane phase of an 8-byte
-// load) fall in different banks.
-template <int BITS>
-__host__ __device__ inline int padded_row(int RB) { return RB % 128 == 0 ? RB + (BITS == 4 ? 64 : 32) : RB; }
 
 // ------------------------------------------------------------------ gate/up + SwiGLU
 constexpr int kGuBufs = 3;      // expert tiles staged per CTA (the shared expert's buffer is reused)
