@@ -39,7 +39,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=120000)
     ap.add_argument("--warmup", type=int, default=480)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="layer_q4", choices=["layer_q4", "layer_q2", "prefill_q4"],
+    ap.add_argument("--config", default="layer_q4", choices=["layer_q4", "layer_q2", "prefill_q4", "stack_q4"],
                     help="prefill_q4: one step = one 512-token forward of the layer (the prefill path)")
     ap.add_argument("--copies", type=int, default=48)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-oracle sample")
@@ -533,6 +533,128 @@ def ours_prefill(args, cfg):
         print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ 24-layer stack (--config stack_q4)
+def ours_stack(args, cfg):
+    """One step = moe_stack_forward of one fresh token through all 24 resident layers."""
+    import numpy as np
+    import torch
+
+    import fixtures.gpu as fxg
+    import quantized_expert_decode_moe_b200 as qm
+    from fixtures import gen
+
+    world, rank, local = dist_info()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    qm.lib()
+    tensors = [fxg.device_layer(cfg, l, dev) for l in range(cfg.layers)]
+    layers = [qm.layer_from_tensors(cfg, t) for t in tensors]
+    arr = qm.stack_array(layers)
+    P, G = 64, 16                                   # distinct tokens; steps per graph
+    x_host = np.stack([gen.x_tokens(cfg, s, T=1)[0] for s in range(P)])
+    xs = torch.from_numpy(x_host.view(np.int16)).to(dev)
+    h0 = torch.from_numpy(gen.bf16_bits_to_f32(x_host).astype(np.float32)).to(dev)
+    hs = h0.clone()
+    xo = torch.empty((P, cfg.H), dtype=torch.int16, device=dev)
+    ws = qm.new_workspace(layers[0], 1)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(s):
+        i = s % P
+        qm.moe_stack_forward(arr, xs[i], hs[i], xo[i], ws=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for s in range(G):   # eager pass (lazy kernel attributes)
+            step(s)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for s in range(G):
+                step(s)
+        for _ in range(max(args.warmup, 3) // G + 1):
+            g.replay()
+    stream.synchronize()
+    assert qm.moe_poll_status(ws, stream) == 0
+    steps = max(G, (min(args.steps, 4096) // G) * G)
+    gpu_uuid = str(getattr(torch.cuda.get_device_properties(dev), "uuid", "") or "")
+    clocks = Clocks(("GPU-" + gpu_uuid) if gpu_uuid and not gpu_uuid.startswith("GPU-") else (gpu_uuid or str(local)))
+    clocks.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(steps // G):
+            g.replay()
+        e1.record(stream)
+    e1.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    assert qm.moe_poll_status(ws, stream) == 0
+    # the dominant kernel, timed alone on the stack's layers (events between the kernels, no overlap)
+    nk, prof_n = 4, 48
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(prof_n)]
+    x1 = torch.empty((1, cfg.H), dtype=torch.int16, device=dev)
+    with torch.cuda.stream(stream):
+        for row in evs:
+            for e in row:
+                e.record(stream)
+        for s in range(prof_n):
+            i = s % P
+            qm.moe_layer_forward_timed(layers[s % cfg.layers], xs[i:i + 1], hs[i:i + 1], x1, ws=ws, events=evs[s],
+                                       stream=stream)
+    stream.synchronize()
+    names = ["route_logits_kernel", "gateup_decode_kernel", "down_decode_kernel", "norm_kernel"]
+    dur = [sum(evs[s][j].elapsed_time(evs[s][j + 1]) for s in range(prof_n)) / prof_n for j in range(nk)]
+    # end to end with host buffers: x, h in; x_out back, every step
+    xh = torch.from_numpy(x_host.view(np.int16)).pin_memory()
+    hh = h0.cpu().pin_memory()
+    outh = torch.empty((P, cfg.H), dtype=torch.int16).pin_memory()
+    xd = torch.empty(cfg.H, dtype=torch.int16, device=dev)
+    hd = torch.empty(cfg.H, dtype=torch.float32, device=dev)
+    od = torch.empty(cfg.H, dtype=torch.int16, device=dev)
+    e2e_n = min(steps, 256)
+    with torch.cuda.stream(stream):
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for s in range(e2e_n):
+            i = s % P
+            xd.copy_(xh[i], non_blocking=True)
+            hd.copy_(hh[i], non_blocking=True)
+            qm.moe_stack_forward(arr, xd, hd, od, ws=ws, stream=stream)
+            outh[i].copy_(od, non_blocking=True)
+        f1.record(stream)
+    f1.synchronize()
+    e2e_ms = f0.elapsed_time(f1)
+    peaks, peak_kind = measured_peaks()
+    active = cfg.active_bytes_per_token               # 24 layers x 4 experts
+    tok_s = steps / (ms * 1e-3)
+    gbs = active * tok_s / 1e9
+    gu_bytes = (cfg.k + 1) * 2 * (cfg.I * cfg.H * cfg.bits // 8 + 2 * 2 * cfg.I * (cfg.H // cfg.G)) + 2 * cfg.H
+    achieved = gu_bytes / (dur[1] * 1e-3) / 1e9
+    line = {
+        "metric": "24-layer MoE decode tokens/s and achieved HBM GB/s (% of 8 TB/s), 4-bit experts, 1 B200",
+        "value": tok_s, "unit": UNIT, "n_gpus": world, "steps": steps, "warmup": max(args.warmup, 3),
+        "ms_per_step": ms / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "u4 codes x s8 activation digits on int8 tensor cores (s32), fp32 scale+accumulate",
+        "data": "synthetic (seeded; no model weights)",
+        "config": {"workload": cfg.note, "H": cfg.H, "E": cfg.E, "top_k": cfg.k, "shared": 1, "I": cfg.I,
+                   "bits": cfg.bits, "layers": cfg.layers, "T": 1,
+                   "l2": "inputs larger than L2: every step streams 24 layers' experts (679 MB) from an 87 GB stack"},
+        "hbm_gbs": gbs, "pct_of_8tbs": 100.0 * gbs / NOMINAL_HBM, "pct_of_measured_copy": 100.0 * gbs / peaks["hbm_gbs"],
+        "active_bytes_per_token": active, "us_per_layer": ms / steps / cfg.layers * 1e3,
+        "kernel_ms": dict(zip(names, dur)),
+        "roofline": {"bound": "hbm", "kernel": "gateup_decode_kernel", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "algorithmic_bytes": gu_bytes, "peak_kind": peak_kind},
+        "e2e": {"value": e2e_n / (e2e_ms * 1e-3), "unit": UNIT, "steps": e2e_n,
+                "h2d_bytes_per_step": cfg.H * (2 + 4), "d2h_bytes_per_step": cfg.H * 2},
+        "gpu_launches": 4 * cfg.layers * steps, "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del g
+
+
 def main():
     args = parse()
     import fixtures
@@ -541,6 +663,8 @@ def main():
         reference_arm(args, cfg)
     elif cfg.T > 1:
         ours_prefill(args, cfg)
+    elif cfg.layers > 1:
+        ours_stack(args, cfg)
     else:
         ours(args, cfg)
 
