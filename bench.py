@@ -168,8 +168,9 @@ def recorded_traffic(kernel: str, config: str, files=DECODE_SOURCES):
 
 
 # ------------------------------------------------------------------ CPU oracle sample
-def oracle_sample(cfg, seconds: float, max_tokens: int = 10 ** 9):
-    """Times the CPU oracle on decode tokens of this workload; returns (tokens/s, tokens, threads)."""
+def oracle_sample(cfg, seconds: float, max_tokens: int = 10 ** 9, warmup: int = 3):
+    """Times the CPU oracle on decode tokens of this workload after `warmup` untimed tokens;
+    returns (tokens/s, tokens, threads, seconds)."""
     import numpy as np
 
     import fixtures
@@ -187,6 +188,15 @@ def oracle_sample(cfg, seconds: float, max_tokens: int = 10 ** 9):
 
     shared = expert(cfg.E)
     done, elapsed = 0, 0.0
+    s = 0
+    for _ in range(warmup):   # untimed: the same work on tokens that are not counted
+        x = gen.x_tokens(cfg, 10 ** 6 + s, T=1)
+        s += 1
+        idx, w, sg = oracle.route(x, Wr, cfg.k, bias=rb, gs=gs)
+        h = gen.bf16_bits_to_f32(x[0]).astype(np.float64)
+        ys = np.stack([oracle.expert(expert(int(e)), h, cfg.H, cfg.I, cfg.G, cfg.bits) for e in idx[0]])
+        oracle.combine_norm(ys, w[0], oracle.expert(shared, h, cfg.H, cfg.I, cfg.G, cfg.bits), sg[0], h, gamma,
+                            cfg.rms_eps)
     s = 0
     while done < max_tokens and (elapsed < seconds or done < 2):
         x = gen.x_tokens(cfg, s, T=1)
@@ -214,12 +224,13 @@ def reference_arm(args, cfg):
         return
     budget = max(args.cpu_seconds, 5.0)
     steps = max(1, min(args.steps, 10 ** 6))
-    rate, n, threads, el = oracle_sample(cfg, budget, max_tokens=steps)
+    warm = max(args.warmup, 3)
+    rate, n, threads, el = oracle_sample(cfg, budget, max_tokens=steps, warmup=warm)
     sample = (f"{n} decode tokens of the {cfg.name} workload (one token = one step, capped by a "
               f"{budget:.0f} s budget), experts regenerated on the host before timing")
     line = {
         "impl": "reference", "metric": METRIC, "value": rate, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": n, "steps_requested": args.steps, "warmup": 0, "ms_per_step": 1e3 * el / n,
+        "steps": n, "steps_requested": args.steps, "warmup": warm, "ms_per_step": 1e3 * el / n,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded; no model weights)",
         "config": {"workload": cfg.note, "H": cfg.H, "E": cfg.E, "top_k": cfg.k, "I": cfg.I, "bits": cfg.bits,
