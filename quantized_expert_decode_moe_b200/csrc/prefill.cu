@@ -386,39 +386,43 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_grouped_kernel(PrefillP
       for (int tau = 0; tau < TILES; ++tau) sacc[tau][0] = sacc[tau][1] = bacc[tau][0] = bacc[tau][1] = 0.f;
       const unsigned char* ra = sb + (size_t)crA * G.stride;
       const unsigned char* rbp = sb + (size_t)crB * G.stride;
+      // one quantisation group of the warp's K-slice; the groups go in pairs,
+      // so two groups' MMA chains share a basic block and interleave
+      auto group = [&](int gi) {
+        const int grp = g0 + gi;
+        uint32_t A[2][4];   // per MMA m: a0 (row g, h 0), a1 (row g+8, h 0), a2 (row g, h 1), a3 (row g+8, h 1)
+        if constexpr (BITS == 4) {
+          const uint2 ua = *(const uint2*)(ra + grp * 32 + 8 * t), ub = *(const uint2*)(rbp + grp * 32 + 8 * t);
+          A[0][0] = ua.x & 0x0F0F0F0Fu; A[0][2] = (ua.x >> 4) & 0x0F0F0F0Fu;
+          A[0][1] = ub.x & 0x0F0F0F0Fu; A[0][3] = (ub.x >> 4) & 0x0F0F0F0Fu;
+          A[1][0] = ua.y & 0x0F0F0F0Fu; A[1][2] = (ua.y >> 4) & 0x0F0F0F0Fu;
+          A[1][1] = ub.y & 0x0F0F0F0Fu; A[1][3] = (ub.y >> 4) & 0x0F0F0F0Fu;
+        } else {
+          const uint32_t ua = *(const uint32_t*)(ra + grp * 16 + 4 * t);
+          const uint32_t ub = *(const uint32_t*)(rbp + grp * 16 + 4 * t);
 #pragma unroll
-      for (int gi = 0; gi < GPW; ++gi) {
-        if (gi < mg) {
-          const int grp = g0 + gi;
-          uint32_t A[2][4];   // per MMA m: a0 (row g, h 0), a1 (row g+8, h 0), a2 (row g, h 1), a3 (row g+8, h 1)
-          if constexpr (BITS == 4) {
-            const uint2 ua = *(const uint2*)(ra + grp * 32 + 8 * t), ub = *(const uint2*)(rbp + grp * 32 + 8 * t);
-            A[0][0] = ua.x & 0x0F0F0F0Fu; A[0][2] = (ua.x >> 4) & 0x0F0F0F0Fu;
-            A[0][1] = ub.x & 0x0F0F0F0Fu; A[0][3] = (ub.x >> 4) & 0x0F0F0F0Fu;
-            A[1][0] = ua.y & 0x0F0F0F0Fu; A[1][2] = (ua.y >> 4) & 0x0F0F0F0Fu;
-            A[1][1] = ub.y & 0x0F0F0F0Fu; A[1][3] = (ub.y >> 4) & 0x0F0F0F0Fu;
-          } else {
-            const uint32_t ua = *(const uint32_t*)(ra + grp * 16 + 4 * t);
-            const uint32_t ub = *(const uint32_t*)(rbp + grp * 16 + 4 * t);
-#pragma unroll
-            for (int m = 0; m < 2; ++m) {
-              A[m][0] = (ua >> (4 * m)) & 0x03030303u; A[m][2] = (ua >> (4 * m + 2)) & 0x03030303u;
-              A[m][1] = (ub >> (4 * m)) & 0x03030303u; A[m][3] = (ub >> (4 * m + 2)) & 0x03030303u;
-            }
-          }
-#pragma unroll
-          for (int tau = 0; tau < TILES; ++tau) {
-            int c[4] = {0, 0, 0, 0};
-            const uint4 b = bq[tau][gi];
-            mma_u8s8(c, A[0][0], A[0][1], A[0][2], A[0][3], b.x, b.y);
-            mma_u8s8(c, A[1][0], A[1][1], A[1][2], A[1][3], b.z, b.w);
-            // columns 2t, 2t+1 of the tile: token t's high- and low-digit sums
-            sacc[tau][0] = fmaf(sA[gi], (float)(c[0] * 256 + c[1]), sacc[tau][0]);
-            sacc[tau][1] = fmaf(sB[gi], (float)(c[2] * 256 + c[3]), sacc[tau][1]);
-            bacc[tau][0] = fmaf(bA[gi], xg[tau][gi], bacc[tau][0]);
-            bacc[tau][1] = fmaf(bB[gi], xg[tau][gi], bacc[tau][1]);
+          for (int m = 0; m < 2; ++m) {
+            A[m][0] = (ua >> (4 * m)) & 0x03030303u; A[m][2] = (ua >> (4 * m + 2)) & 0x03030303u;
+            A[m][1] = (ub >> (4 * m)) & 0x03030303u; A[m][3] = (ub >> (4 * m + 2)) & 0x03030303u;
           }
         }
+#pragma unroll
+        for (int tau = 0; tau < TILES; ++tau) {
+          int c[4] = {0, 0, 0, 0};
+          const uint4 b = bq[tau][gi];
+          mma_u8s8(c, A[0][0], A[0][1], A[0][2], A[0][3], b.x, b.y);
+          mma_u8s8(c, A[1][0], A[1][1], A[1][2], A[1][3], b.z, b.w);
+          // columns 2t, 2t+1 of the tile: token t's high- and low-digit sums
+          sacc[tau][0] = fmaf(sA[gi], (float)(c[0] * 256 + c[1]), sacc[tau][0]);
+          sacc[tau][1] = fmaf(sB[gi], (float)(c[2] * 256 + c[3]), sacc[tau][1]);
+          bacc[tau][0] = fmaf(bA[gi], xg[tau][gi], bacc[tau][0]);
+          bacc[tau][1] = fmaf(bB[gi], xg[tau][gi], bacc[tau][1]);
+        }
+      };
+#pragma unroll
+      for (int gp = 0; gp < GPW; gp += 2) {
+        if (gp + 1 < mg) { group(gp); group(gp + 1); }
+        else if (gp < mg) group(gp);
       }
 #pragma unroll
       for (int tau = 0; tau < TILES; ++tau) {
