@@ -94,6 +94,28 @@ def test_workspace_size_and_layer_validation():
     assert qm.lib().moe_workspace_size(None, 1, None) == 1
 
 
+def test_prefill_workspace_holds_the_grouped_buffers():
+    """Above 8 tokens the workspace also holds the prefill path's buffers: the
+    expert outputs y [T(k+1)][H] fp32, the activation digit tables of x
+    ([T][2H] bytes) and of the SwiGLU outputs ([T(k+1)][2I] bytes) and the fp64
+    logits [T][E+1]; a call whose workspace was sized for fewer tokens is
+    rejected before anything is launched."""
+    lay = fake_layer()
+    H, I, E, k = 4096, 1024, 512, 3
+    _, n8 = ws_size(lay, T=8)
+    _, n9 = ws_size(lay, T=9)
+    _, n512 = ws_size(lay, T=512)
+    T = 512
+    need = T * (k + 1) * H * 4 + T * 2 * H + T * (k + 1) * 2 * I + T * (E + 1) * 8
+    assert n512 >= need
+    assert n9 - n8 >= 9 * (k + 1) * H * 4   # the prefill buffers appear at T = 9
+    L = qm.lib()
+    p = C.c_void_p(0x200000)
+    ws = C.c_void_p(0x400000)
+    assert L.moe_layer_forward(C.byref(lay), p, p, 9, p, None, None, None, ws, n8, None) == 3
+    assert L.moe_route(C.byref(lay), p, 12, p, p, None, ws, n8, None) == 3
+
+
 def test_entry_points_reject_bad_arguments_before_launch():
     L = qm.lib()
     lay = fake_layer()
