@@ -224,6 +224,17 @@ moe_status moe_layer_forward_noalloc(const moe_layer* layer, const uint16_t* x_i
  * earlier calls (MOE_OK if none), then clears it. */
 moe_status moe_poll_status(void* ws, void* stream);
 
+/* Diagnostics for the device-side failure path. Launches one warp that waits,
+ * through the library's bounded wait, on a barrier phase that nothing
+ * completes (no copy is issued, so nothing is in flight). After bound_ns
+ * (1 ns .. 10 s) the wait gives up, MOE_ERR_TIMEOUT is latched in the
+ * workspace status word, and the kernel returns normally. The timeout is
+ * read back with moe_poll_status, and later calls on the same context work
+ * as before. Asynchronous on `stream`.
+ * Errors: MOE_ERR_WORKSPACE (ws NULL or under 256 bytes),
+ * MOE_ERR_INVALID_ARGUMENT (ws not 256-byte aligned, bound out of range). */
+moe_status moe_selftest_wait_timeout(void* ws, size_t ws_bytes, uint64_t bound_ns, void* stream);
+
 /* Static string naming a status code. */
 const char* moe_status_string(moe_status s);
 

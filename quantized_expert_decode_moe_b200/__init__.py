@@ -15,7 +15,8 @@ __all__ = [
     "MoeError", "QMat", "Expert", "Layer", "lib", "build",
     "moe_abi_version", "moe_status_string", "moe_workspace_size", "moe_workspace_init", "moe_route",
     "moe_expert_gemv_q4", "moe_expert_gemv_q2", "moe_combine_residual_norm", "moe_group_tokens",
-    "moe_layer_forward", "moe_layer_forward_noalloc", "moe_layer_forward_timed", "moe_stack_forward", "moe_poll_status", "new_workspace",
+    "moe_layer_forward", "moe_layer_forward_noalloc", "moe_layer_forward_timed", "moe_stack_forward", "moe_poll_status",
+    "moe_selftest_wait_timeout", "new_workspace",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -79,6 +80,7 @@ def lib():
         L.moe_layer_forward_noalloc.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp]
         L.moe_stack_forward.argtypes = [vp, i32, vp, vp, vp, vp, vp, vp, vp, C.c_size_t, vp]
         L.moe_poll_status.argtypes = [vp, vp]
+        L.moe_selftest_wait_timeout.argtypes = [vp, C.c_size_t, C.c_uint64, vp]
         _lib = L
     return _lib
 
@@ -257,3 +259,9 @@ def stack_array(layers) -> _LayerArray:
 
 def moe_poll_status(ws, stream=None) -> int:
     return lib().moe_poll_status(_ptr(ws), _stream(stream))
+
+
+def moe_selftest_wait_timeout(ws, bound_ns: int, stream=None):
+    """A bounded device wait that runs out (see moe.h): latches MOE_ERR_TIMEOUT in ws."""
+    _ok(lib().moe_selftest_wait_timeout(_ptr(ws), ws.numel() * ws.element_size(), int(bound_ns), _stream(stream)),
+        "moe_selftest_wait_timeout")

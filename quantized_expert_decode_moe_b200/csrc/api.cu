@@ -402,6 +402,13 @@ moe_status moe_layer_forward_noalloc(const moe_layer* layer, const uint16_t* x_i
   return decode_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, s);
 }
 
+moe_status moe_selftest_wait_timeout(void* ws, size_t ws_bytes, uint64_t bound_ns, void* stream) {
+  if (!ws || ws_bytes < 256) return MOE_ERR_WORKSPACE;
+  if (((uintptr_t)ws & 255u) != 0) return MOE_ERR_INVALID_ARGUMENT;
+  if (bound_ns == 0 || bound_ns > 10000000000ull) return MOE_ERR_INVALID_ARGUMENT;
+  return cuda_status(launch_selftest_wait((uint32_t*)ws, (unsigned long long)bound_ns, (cudaStream_t)stream));
+}
+
 moe_status moe_poll_status(void* ws, void* stream) {
   if (!ws) return MOE_ERR_WORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;

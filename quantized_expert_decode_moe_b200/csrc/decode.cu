@@ -573,6 +573,22 @@ __global__ void __launch_bounds__(kThreads, 2) down_decode_kernel(DownParams p) 
   }
 }
 
+// ------------------------------------------------------------------ diagnostics
+// One warp waits, through the same bounded wait as every kernel above, on an
+// mbarrier phase that nothing completes (16 bytes expected, no copy issued):
+// the wait gives up after bound_ns, latches MOE_ERR_TIMEOUT in *status and the
+// kernel returns. Nothing is in flight when it gives up.
+__global__ void __launch_bounds__(32) selftest_wait_kernel(uint32_t* status, unsigned long long bound_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_expect_tx(&bar, 16);
+  }
+  __syncthreads();
+  mbar_wait_bounded(&bar, 0u, bound_ns, status);
+}
+
 // ------------------------------------------------------------------ launchers
 static cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
                               void** args) {
@@ -646,6 +662,11 @@ cudaError_t launch_down(const DownParams& p, int bits, int T, bool pdl, cudaStre
   if (e != cudaSuccess) return e;
   void* args[] = {&q};
   return launch_pdl(fn, dim3(p.nCTA, T), dim3(kThreads), sm, s, pdl, args);
+}
+
+cudaError_t launch_selftest_wait(uint32_t* status, unsigned long long bound_ns, cudaStream_t s) {
+  selftest_wait_kernel<<<1, 32, 0, s>>>(status, bound_ns);
+  return cudaGetLastError();
 }
 
 }  // namespace qmoe

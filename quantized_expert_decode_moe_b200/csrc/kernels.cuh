@@ -144,6 +144,7 @@ cudaError_t launch_gemv(const GemvParams& p, int bits, cudaStream_t s);
 cudaError_t launch_group(const GroupParams& p, cudaStream_t s);
 cudaError_t launch_prefill_gateup(const PrefillParams& p, int bits, cudaStream_t s);   // digit tables of x + gate/up
 cudaError_t launch_prefill_down(const PrefillParams& p, int bits, cudaStream_t s);     // digit tables of a + down
+cudaError_t launch_selftest_wait(uint32_t* status, unsigned long long bound_ns, cudaStream_t s);
 int num_sms();
 int pf_chunk_tokens(int H, int I);   // tokens per chunk of the grouped GEMMs
 size_t pf_max_chunks(int T, int k, int E, int chunk);

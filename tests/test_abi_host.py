@@ -148,3 +148,8 @@ def test_entry_points_reject_bad_arguments_before_launch():
     lays = (qm._Layer * 2)(fake_layer(), fake_layer(inter=2048))
     assert L.moe_stack_forward(lays, 2, p, p, p, None, None, None, ws, n, None) == 1
     assert L.moe_poll_status(None, None) == 3
+    # failure-path diagnostics: no workspace, misaligned, bound out of range
+    assert L.moe_selftest_wait_timeout(None, n, 1000, None) == 3
+    assert L.moe_selftest_wait_timeout(C.c_void_p(0x400010), n, 1000, None) == 1
+    assert L.moe_selftest_wait_timeout(ws, n, 0, None) == 1
+    assert L.moe_selftest_wait_timeout(ws, n, 20 * 10 ** 9, None) == 1
