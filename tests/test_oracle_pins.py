@@ -342,15 +342,16 @@ def test_expert_vs_torch_composition(bits):
     np.testing.assert_allclose(y, y_ref, rtol=1e-11, atol=1e-12)
 
 
-def test_tiny_layer_vs_torch_composition():
+@pytest.mark.parametrize("with_shared", [True, False])
+def test_tiny_layer_vs_torch_composition(with_shared):
     cfg = fixtures.CONFIGS["tiny"]
     Wr, _, gsv, gamma = fixtures.layer_vectors(cfg, 0)
     experts = [fixtures.host_expert(cfg, 0, e) for e in range(cfg.E)]
-    shared = fixtures.host_expert(cfg, 0, cfg.E)
+    shared = fixtures.host_expert(cfg, 0, cfg.E) if with_shared else None
     x = gen.x_tokens(cfg, 0, T=2)
     h = gen.bf16_bits_to_f32(x).astype(np.float64)
     out = oracle.layer(x, h, Wr, gamma, experts, shared, I=cfg.I, k=cfg.k, G=cfg.G, bits=cfg.bits,
-                       eps=cfg.rms_eps, gs=gsv)
+                       eps=cfg.rms_eps, gs=gsv if with_shared else None)
     xf = torch.from_numpy(h)
     logits = xf @ torch.from_numpy(gen.bf16_bits_to_f32(Wr).astype(np.float64)).T
     p = torch.softmax(logits, dim=-1)
@@ -361,7 +362,8 @@ def test_tiny_layer_vs_torch_composition():
         np.testing.assert_array_equal(out["idx"][t], top)
         wt = p[t, top] / p[t, top].sum()
         moe = sum(float(wt[i]) * _torch_expert(experts[e], h[t], cfg.H, cfg.I, cfg.G, 4)[0] for i, e in enumerate(top))
-        moe = moe + float(sgate[t]) * _torch_expert(shared, h[t], cfg.H, cfg.I, cfg.G, 4)[0]
+        if with_shared:
+            moe = moe + float(sgate[t]) * _torch_expert(shared, h[t], cfg.H, cfg.I, cfg.G, 4)[0]
         h_ref = h[t] + moe
         np.testing.assert_allclose(out["h_out"][t], h_ref, rtol=1e-11, atol=1e-11)
         x_ref = torch.nn.functional.rms_norm(torch.from_numpy(h_ref), (cfg.H,), weight=gf, eps=cfg.rms_eps).numpy()
