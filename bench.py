@@ -168,16 +168,16 @@ def recorded_traffic(kernel: str, config: str, files=DECODE_SOURCES):
 
 
 # ------------------------------------------------------------------ CPU oracle sample
-def oracle_sample(cfg, seconds: float, max_tokens: int = 10 ** 9, warmup: int = 3):
-    """Times the CPU oracle on decode tokens of this workload after `warmup` untimed tokens;
-    returns (tokens/s, tokens, threads, seconds)."""
+def oracle_sample(cfg, seconds: float, max_tokens: int = 10 ** 9, warmup: int = 3, threads: int = 0):
+    """Times the CPU oracle on decode tokens of this workload after `warmup` untimed tokens, on
+    `threads` host threads (0: all cores); returns (tokens/s, tokens, threads, seconds)."""
     import numpy as np
 
     import fixtures
     import oracle
     from fixtures import gen
 
-    threads = oracle.set_threads(os.cpu_count() or 1)
+    threads = oracle.set_threads(threads if threads > 0 else (os.cpu_count() or 1))
     Wr, rb, gs, gamma = fixtures.layer_vectors(cfg, 0)
     cache = {}
 
@@ -421,8 +421,11 @@ def ours(args, cfg):
     }
     if rank == 0 and not args.no_cpu_baseline:
         rate, n, threads, el = oracle_sample(cfg, args.cpu_seconds)
+        rate1, n1, _, el1 = oracle_sample(cfg, max(2.0, args.cpu_seconds / 4), threads=1)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
-                                "sample": f"{n} decode tokens of this workload ({el:.1f} s of oracle time)"}
+                                "sample": f"{n} decode tokens of this workload ({el:.1f} s of oracle time)",
+                                "single_thread": {"value": rate1, "unit": UNIT, "cores": 1,
+                                                  "sample": f"{n1} decode tokens ({el1:.1f} s)"}}
     if rank == 0:
         print(json.dumps(line), flush=True)
     for g in graphs.values():
@@ -540,6 +543,11 @@ def ours_prefill(args, cfg):
         # route, top-k, grouping, digits of x, gate/up, digits of a, down, combine + norm
         "gpu_launches": 8 * steps, "clocks": clk,
     }
+    if rank == 0 and not args.no_cpu_baseline:
+        rate, n, threads, el = oracle_sample(cfg, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                "sample": f"{n} tokens of the batch, one at a time as the oracle has no batching "
+                                          f"({el:.1f} s of oracle time)"}
     if rank == 0:
         print(json.dumps(line), flush=True)
 
