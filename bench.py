@@ -110,6 +110,27 @@ class Clocks:
         return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(smax), "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ------------------------------------------------------------------ host buffers
+def packed_inputs(x_bits, h, dev):
+    """Pinned host rows holding a step's x (bf16 bits) and h (fp32) back to back, and a device twin
+    with x and h views: one host->device copy per step carries both inputs (both views 16-byte
+    aligned). x_bits: uint16 [N, ...]; h: float32 [N, ...] of the same shape; returns
+    (host [N, bytes], device [bytes], x view, h view)."""
+    import numpy as np
+    import torch
+
+    n = x_bits.shape[0]
+    shape = x_bits.shape[1:]
+    xb = np.ascontiguousarray(x_bits).view(np.uint8).reshape(n, -1)
+    hb = np.ascontiguousarray(h, dtype=np.float32).view(np.uint8).reshape(n, -1)
+    host = torch.from_numpy(np.concatenate([xb, hb], axis=1)).pin_memory()
+    devbuf = torch.empty(host.shape[1], dtype=torch.uint8, device=dev)
+    nx = xb.shape[1]
+    xv = devbuf[:nx].view(torch.int16).view(*shape)
+    hv = devbuf[nx:].view(torch.float32).view(*shape)
+    return host, devbuf, xv, hv
+
+
 # ------------------------------------------------------------------ workload
 def build_workload(cfg, copies, dev):
     import numpy as np
@@ -357,16 +378,14 @@ def ours(args, cfg):
 
     # end to end through the public API with host buffers
     e2e_n = min(args.e2e_steps, args.steps)
-    xh = torch.from_numpy(W["x_host"].view(np.int16)).pin_memory()
-    hh = W["h0"].cpu().pin_memory()
+    inh, ind, xdev, hdev = packed_inputs(W["x_host"].reshape(P, 1, cfg.H),
+                                         W["h0"].cpu().numpy().reshape(P, 1, cfg.H), dev)
     outh = torch.empty((P, cfg.H), dtype=torch.int16).pin_memory()
-    xdev = torch.empty((1, cfg.H), dtype=torch.int16, device=dev)
-    hdev = torch.empty((1, cfg.H), dtype=torch.float32, device=dev)
     odev = torch.empty((1, cfg.H), dtype=torch.int16, device=dev)
     with torch.cuda.stream(stream):
         for s in range(8):
             i = s % P
-            xdev.copy_(xh[i:i + 1], non_blocking=True); hdev.copy_(hh[i:i + 1], non_blocking=True)
+            ind.copy_(inh[i], non_blocking=True)
             qm.moe_layer_forward(layers[s % C], xdev, hdev, odev, ws=ws, stream=stream)
             outh[i:i + 1].copy_(odev, non_blocking=True)
         stream.synchronize()
@@ -376,8 +395,7 @@ def ours(args, cfg):
         f0.record(stream)
         for s in range(e2e_n):
             i = s % P
-            xdev.copy_(xh[i:i + 1], non_blocking=True)
-            hdev.copy_(hh[i:i + 1], non_blocking=True)
+            ind.copy_(inh[i], non_blocking=True)   # x and h of the step, one copy
             qm.moe_layer_forward(layers[s % C], xdev, hdev, odev, ws=ws, stream=stream)
             outh[i:i + 1].copy_(odev, non_blocking=True)
         f1.record(stream)
@@ -499,18 +517,14 @@ def ours_prefill(args, cfg):
     names = ["route_logits", "topk+group", "gateup_grouped", "down_grouped", "combine_norm"]
     dur = [sum(evs[r][j].elapsed_time(evs[r][j + 1]) for r in range(reps)) / reps for j in range(nst)]
     # end to end with host buffers: x, h in; x_out back, every step
-    xh = torch.from_numpy(np.stack(xs_host).view(np.int16)).pin_memory()
-    hh = torch.stack([h.cpu() for h in hs]).pin_memory()
+    inh, ind, xd, hd = packed_inputs(np.stack(xs_host), np.stack([h.cpu().numpy() for h in hs]), dev)
     outh = torch.empty((T, cfg.H), dtype=torch.int16).pin_memory()
-    xd = torch.empty((T, cfg.H), dtype=torch.int16, device=dev)
-    hd = torch.empty((T, cfg.H), dtype=torch.float32, device=dev)
     e2e_n = min(steps, 32)
     with torch.cuda.stream(stream):
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         f0.record(stream)
         for i in range(e2e_n):
-            xd.copy_(xh[i % NB], non_blocking=True)
-            hd.copy_(hh[i % NB], non_blocking=True)
+            ind.copy_(inh[i % NB], non_blocking=True)   # x and h of the batch, one copy
             qm.moe_layer_forward(layer, xd, hd, xo, ws=ws, stream=stream)
             outh.copy_(xo, non_blocking=True)
         f1.record(stream)
@@ -625,11 +639,8 @@ def ours_stack(args, cfg):
     names = ["route_logits_kernel", "gateup_decode_kernel", "down_decode_kernel", "norm_kernel"]
     dur = [sum(evs[s][j].elapsed_time(evs[s][j + 1]) for s in range(prof_n)) / prof_n for j in range(nk)]
     # end to end with host buffers: x, h in; x_out back, every step
-    xh = torch.from_numpy(x_host.view(np.int16)).pin_memory()
-    hh = h0.cpu().pin_memory()
+    inh, ind, xd, hd = packed_inputs(x_host, h0.cpu().numpy(), dev)
     outh = torch.empty((P, cfg.H), dtype=torch.int16).pin_memory()
-    xd = torch.empty(cfg.H, dtype=torch.int16, device=dev)
-    hd = torch.empty(cfg.H, dtype=torch.float32, device=dev)
     od = torch.empty(cfg.H, dtype=torch.int16, device=dev)
     e2e_n = min(steps, 256)
     with torch.cuda.stream(stream):
@@ -637,8 +648,7 @@ def ours_stack(args, cfg):
         f0.record(stream)
         for s in range(e2e_n):
             i = s % P
-            xd.copy_(xh[i], non_blocking=True)
-            hd.copy_(hh[i], non_blocking=True)
+            ind.copy_(inh[i], non_blocking=True)   # x and h of the step, one copy
             qm.moe_stack_forward(arr, xd, hd, od, ws=ws, stream=stream)
             outh[i].copy_(od, non_blocking=True)
         f1.record(stream)
