@@ -22,8 +22,32 @@
  *  - Argument and shape errors are detected on the host before anything is
  *    launched and returned as MOE_ERR_INVALID_ARGUMENT / MOE_ERR_UNSUPPORTED /
  *    MOE_ERR_WORKSPACE; a failed launch returns MOE_ERR_CUDA. Device-side
- *    errors (an expert id out of range) are latched in the workspace status
- *    word and read back with moe_poll_status.
+ *    errors (an expert id out of range, a bounded wait that ran out) are
+ *    latched in the workspace status word and read back with moe_poll_status.
+ *  - Every device-side wait (a staged copy, a grid-wide barrier of the fused
+ *    decode kernel) gives up after 100 ms, or MOE_WAIT_TIMEOUT_NS from the
+ *    environment (read once, clamped to 1 ms .. 10 s), latches
+ *    MOE_ERR_TIMEOUT and skips the remaining waits of the call: the outputs
+ *    of a call that latched a timeout are invalid.
+ *  - Supported shapes. The decode kernels stage each CTA's rows of the active
+ *    experts in shared memory, one CTA per SM. A layer call is rejected with
+ *    MOE_ERR_UNSUPPORTED, before any launch, when no kernel path fits the
+ *    device:
+ *      T = 1     the fused single-kernel layer: H <= 4096, top_k <= 3
+ *                (top_k + shared <= 4), E <= 4096, I <= 8 n and H <= 32 n
+ *                with n = min(SMs, I, H) (148 SMs: I <= 1152); otherwise
+ *                the chain below;
+ *      T <= 8    the four-kernel chain: gate/up stages 3 experts x 8 rows x H
+ *                and down up to 4 experts x 32 rows x I in one CTA (227 KB
+ *                per CTA, top_k 3 + shared: H <= 7552 and I <= 2688 at 4
+ *                bits, I <= 4352 at 2 bits);
+ *      T > 8     the grouped prefill kernels (two stages of their ring of
+ *                weight tiles must fit and their row tiles must divide the
+ *                matrices);
+ *    and H, I <= 8192 throughout.
+ *    moe_layer_forward_noalloc and moe_stack_forward apply the same rules
+ *    (T = 1 for the stack), and moe_workspace_size applies the rule of
+ *    T = max_tokens.
  *  - Device pointers must be 16-byte aligned; H, I must be multiples of 128
  *    (one 128-element k-span) and of the quantisation group; the group is 64.
  *  - No global state: calls on different streams with different workspaces
@@ -103,15 +127,23 @@ moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
 /*
  * Router ("Model architecture": K=4 active per token incl. one shared;
  * the router results select the experts to load — HN thread, Table 3 comment).
- *   logits = router_w . x (+ router_bias): for T > 8 in fp64, each logit
- *   accumulated in index order from 0 with the bias added last, which with
- *   exact bf16 x bf16 products is the plain fp64 sum itself; for T <= 8 as
- *   compensated fp32 (about 2^-44 relative to sum |w x|), rounded to fp64;
+ *   logits = router_w . x (+ router_bias). The ranking is that of the plain
+ *   fp64 definition (exact bf16 x bf16 products summed in index order from
+ *   0, bias added last). For T > 8 the logits are computed exactly so. For
+ *   T <= 8 they are compensated fp32 sums (about 2^-44 relative to
+ *   sum |w x|) with a rigorous bound on their distance to the definition;
+ *   the top-k is certified against that bound, and when two candidates are
+ *   closer than it, every candidate near the k-th is recomputed as the
+ *   definition and ranked again, so the indices are those of the definition;
  *   topk_idx [T][k]: the k largest logits, descending, ties to the lower index;
  *   topk_w [T][k]: softmax over all E renormalised over the chosen k (fp32);
  *   shared_gate [T] (nullable): sigmoid(shared_gate_w . x), 0 if no shared expert.
  * x: bf16 [T][H]. The logits stay in the workspace after the call: double
- * [T][E+1] at byte offset 256, column E holding shared_gate_w . x.
+ * [T][E+1] at byte offset 256, column E holding shared_gate_w . x. The
+ * uint32 at byte offset 16 of the workspace counts the selections (by this
+ * and the decode layer calls) that needed the exact recheck; it wraps, and
+ * moe_workspace_init clears it.
+ * Requires E <= 4096 and k <= 8; |w x| products must be finite in fp32.
  */
 moe_status moe_route(const moe_layer* layer, const uint16_t* x, int32_t T, int32_t* topk_idx,
                      float* topk_w, float* shared_gate, void* ws, size_t ws_bytes, void* stream);
@@ -155,8 +187,10 @@ moe_status moe_group_tokens(int32_t T, int32_t k, int32_t E, const int32_t* topk
 /*
  * Whole MoE layer for T tokens: router, expert gate/up + SwiGLU, down, combine
  * with the shared-expert gate, residual and RMSNorm, all on the device with
- * no host round trip. T = 1..8 runs the decode kernels; larger T runs the
- * prefill kernels (grouping by expert, grouped dequant GEMM).
+ * no host round trip. T = 1 runs the fused decode kernel (the whole layer in
+ * one persistent launch, grid-wide barriers between its phases); T = 2..8
+ * the four-kernel decode chain; larger T the prefill kernels (grouping by
+ * expert, grouped dequant GEMM). See "Supported shapes" above.
  *   x_in bf16 [T][H]; h fp32 [T][H] residual in, h' out; x_out bf16 [T][H];
  *   x_out_f32 fp32 [T][H] or NULL; topk_idx int32 [T][k] or NULL;
  *   topk_w fp32 [T][k] or NULL.
@@ -167,7 +201,10 @@ moe_status moe_layer_forward(const moe_layer* layer, const uint16_t* x_in, float
 
 /*
  * L layers in sequence for one decode token: layer l's x_out feeds layer l+1
- * and h is carried in fp32 ("Deferred GPU expert compute").
+ * and h is carried in fp32 ("Deferred GPU expert compute"). With the fused
+ * kernel, up to 24 layers run in one launch: x and h stay on the chip
+ * between layers, and the next layer's router rows and shared expert are
+ * requested while the current layer finishes.
  *   layers: host array [L]; x_in bf16 [H]; h fp32 [H] in/out; x_out bf16 [H];
  *   topk_idx_all int32 [L][k] or NULL; layer_inputs bf16 [L][H] or NULL and
  *   layer_h fp32 [L][H] or NULL: each layer's input x and residual h (for
@@ -178,14 +215,27 @@ moe_status moe_stack_forward(const moe_layer* layers, int32_t L, const uint16_t*
                              float* layer_h, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * The kernel path that serves a call of T tokens on `layer` (host only,
+ * launches nothing): MOE_PATH_FUSED (the fused decode kernel, T = 1),
+ * MOE_PATH_CHAIN (the four-kernel decode chain, T <= 8) or MOE_PATH_PREFILL
+ * (T > 8), and in *n_events the number of events moe_layer_forward_timed
+ * records on that path (its stages + 1). Either output may be NULL.
+ * Errors: those of moe_workspace_size's layer checks; MOE_ERR_UNSUPPORTED
+ * when no path fits (see "Supported shapes").
+ */
+typedef enum { MOE_PATH_FUSED = 1, MOE_PATH_CHAIN = 2, MOE_PATH_PREFILL = 3 } moe_path;
+moe_status moe_layer_path(const moe_layer* layer, int32_t T, int32_t* path, int32_t* n_events);
+
+/*
  * Profiling variant of moe_layer_forward: the same kernels with a CUDA event
  * recorded before the first and after each of the kernels of the layer, so a
  * caller can time them one by one. events: host array of n_events created
  * cudaEvent_t handles (passed as void*); n_events must be at least the number
- * of recorded stages + 1: decode (T <= 8) 5 (router, gate/up, down, norm);
- * prefill 6 (router, top-k + grouping, gate/up, down, combine + norm). The
- * kernels run without programmatic overlap between them. Same arguments and
- * errors otherwise.
+ * of recorded stages + 1: fused decode (T = 1) 2 (the one kernel); decode
+ * chain (T = 2..8, or T = 1 when the fused kernel does not fit) 5 (router,
+ * gate/up, down, norm); prefill 6 (router, top-k + grouping, gate/up, down,
+ * combine + norm). The kernels run without programmatic overlap between
+ * them. Same arguments and errors otherwise.
  */
 moe_status moe_layer_forward_timed(const moe_layer* layer, const uint16_t* x_in, float* h, int32_t T,
                                    uint16_t* x_out, float* x_out_f32, int32_t* topk_idx, float* topk_w,
@@ -206,22 +256,32 @@ moe_status moe_layer_forward_timed(const moe_layer* layer, const uint16_t* x_in,
  * process exits. The call allocates and frees nothing. The first call on a
  * device looks up that array's device address (once per device, with that
  * device current); make that first call before any stream capture.
- * Layers and token counts whose workspace (moe_workspace_size) exceeds
- * MOE_NOALLOC_SCRATCH_BYTES are rejected with MOE_ERR_WORKSPACE.
- * All calls share the array and it keeps the last call's contents; the call
- * clears what has to start at zero. Calls whose kernels overlap on the GPU
- * (different streams, or different host threads) race on the array: order
- * them on one stream. Device-side status latched by this call cannot be read
- * with moe_poll_status. Arguments and errors are otherwise those of
- * moe_layer_forward.
+ * It serves decode only: T = 1..8; T > 8 is rejected with
+ * MOE_ERR_UNSUPPORTED. Layers and token counts whose workspace
+ * (moe_workspace_size) exceeds MOE_NOALLOC_SCRATCH_BYTES are rejected with
+ * MOE_ERR_WORKSPACE.
+ * All calls share the array and it keeps the last call's contents; the
+ * kernels clear what has to start at zero. The array starts zeroed, and a
+ * device-side status latched by a call (MOE_ERR_TIMEOUT,
+ * MOE_ERR_DEVICE_FAULT) stays in it until moe_noalloc_poll_status reads and
+ * clears it. Calls whose kernels overlap on the GPU (different streams, or
+ * different host threads) race on the array: order them on one stream.
+ * Arguments and errors are otherwise those of moe_layer_forward.
  */
 #define MOE_NOALLOC_SCRATCH_BYTES (4u << 20)
 moe_status moe_layer_forward_noalloc(const moe_layer* layer, const uint16_t* x_in, float* h, int32_t T,
                                      uint16_t* x_out, float* x_out_f32, int32_t* topk_idx, float* topk_w,
                                      void* stream);
 
+/* moe_poll_status for the static scratch of moe_layer_forward_noalloc on the
+ * current device: synchronises `stream`, returns the status latched by
+ * earlier no-alloc calls (MOE_OK if none) and clears it. */
+moe_status moe_noalloc_poll_status(void* stream);
+
 /* Synchronises `stream` and returns the status latched in the workspace by
- * earlier calls (MOE_OK if none), then clears it. */
+ * earlier calls (MOE_OK if none). A latched status is cleared together with
+ * the grid-barrier counters of the workspace header (the first 256 bytes),
+ * which a call that ran out of time may have left mid-round. */
 moe_status moe_poll_status(void* ws, void* stream);
 
 /* Diagnostics for the device-side failure path. Launches one warp that waits,
@@ -234,6 +294,15 @@ moe_status moe_poll_status(void* ws, void* stream);
  * Errors: MOE_ERR_WORKSPACE (ws NULL or under 256 bytes),
  * MOE_ERR_INVALID_ARGUMENT (ws not 256-byte aligned, bound out of range). */
 moe_status moe_selftest_wait_timeout(void* ws, size_t ws_bytes, uint64_t bound_ns, void* stream);
+
+/* Diagnostics for the grid-wide barrier of the fused decode kernel. One
+ * thread arrives at a barrier of the workspace header as if the grid had two
+ * CTAs, so the round never completes; after bound_ns (1 ns .. 10 s) its wait
+ * gives up, MOE_ERR_TIMEOUT is latched and the kernel returns. The barrier's
+ * arrival counter is left mid-round, as a real timeout can leave it: read the
+ * status with moe_poll_status, which also clears the counters, before the
+ * workspace serves another call. Errors as for moe_selftest_wait_timeout. */
+moe_status moe_selftest_grid_timeout(void* ws, size_t ws_bytes, uint64_t bound_ns, void* stream);
 
 /* Static string naming a status code. */
 const char* moe_status_string(moe_status s);

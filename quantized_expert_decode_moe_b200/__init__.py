@@ -13,10 +13,10 @@ import os
 
 __all__ = [
     "MoeError", "QMat", "Expert", "Layer", "lib", "build",
-    "moe_abi_version", "moe_status_string", "moe_workspace_size", "moe_workspace_init", "moe_route",
+    "moe_abi_version", "moe_status_string", "moe_workspace_size", "moe_workspace_init", "moe_layer_path", "moe_route",
     "moe_expert_gemv_q4", "moe_expert_gemv_q2", "moe_combine_residual_norm", "moe_group_tokens",
     "moe_layer_forward", "moe_layer_forward_noalloc", "moe_layer_forward_timed", "moe_stack_forward", "moe_poll_status",
-    "moe_selftest_wait_timeout", "new_workspace",
+    "moe_selftest_wait_timeout", "moe_selftest_grid_timeout", "moe_noalloc_poll_status", "new_workspace",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -70,6 +70,7 @@ def lib():
         L.moe_status_string.argtypes = [C.c_int]
         L.moe_workspace_size.argtypes = [vp, i32, C.POINTER(C.c_size_t)]
         L.moe_workspace_init.argtypes = [vp, C.c_size_t, vp]
+        L.moe_layer_path.argtypes = [vp, i32, C.POINTER(i32), C.POINTER(i32)]
         L.moe_route.argtypes = [vp, vp, i32, vp, vp, vp, vp, C.c_size_t, vp]
         L.moe_expert_gemv_q4.argtypes = [vp, i32, i32, i32, vp, vp, vp]
         L.moe_expert_gemv_q2.argtypes = [vp, i32, i32, i32, vp, vp, vp]
@@ -81,6 +82,8 @@ def lib():
         L.moe_stack_forward.argtypes = [vp, i32, vp, vp, vp, vp, vp, vp, vp, C.c_size_t, vp]
         L.moe_poll_status.argtypes = [vp, vp]
         L.moe_selftest_wait_timeout.argtypes = [vp, C.c_size_t, C.c_uint64, vp]
+        L.moe_selftest_grid_timeout.argtypes = [vp, C.c_size_t, C.c_uint64, vp]
+        L.moe_noalloc_poll_status.argtypes = [vp]
         _lib = L
     return _lib
 
@@ -174,6 +177,16 @@ def moe_workspace_size(layer: Layer, max_tokens: int) -> int:
     return n.value
 
 
+PATHS = {1: "fused", 2: "chain", 3: "prefill"}
+
+
+def moe_layer_path(layer: Layer, T: int):
+    """(path name, events moe_layer_forward_timed records) for a call of T tokens on layer."""
+    path, nev = C.c_int32(0), C.c_int32(0)
+    _ok(lib().moe_layer_path(layer.cref(), int(T), C.byref(path), C.byref(nev)), "moe_layer_path")
+    return PATHS[path.value], nev.value
+
+
 def moe_workspace_init(ws, stream=None):
     _ok(lib().moe_workspace_init(_ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "moe_workspace_init")
 
@@ -223,7 +236,8 @@ def moe_layer_forward(layer: Layer, x_in, h, x_out, x_out_f32=None, topk_idx=Non
 
 def moe_layer_forward_noalloc(layer: Layer, x_in, h, x_out, x_out_f32=None, topk_idx=None, topk_w=None, stream=None):
     """moe_layer_forward with the library's own static scratch instead of a workspace, for callers that
-    cannot allocate device memory (see include/moe.h). Calls must not overlap on the GPU."""
+    cannot allocate device memory (see include/moe.h). Decode only (1 <= T <= 8). Calls must not
+    overlap on the GPU; a latched device status is read with moe_noalloc_poll_status."""
     _ok(lib().moe_layer_forward_noalloc(layer.cref(), _ptr(x_in), _ptr(h), x_in.shape[0], _ptr(x_out),
                                         _ptr(x_out_f32), _ptr(topk_idx), _ptr(topk_w), _stream(stream)),
         "moe_layer_forward_noalloc")
@@ -259,6 +273,17 @@ def stack_array(layers) -> _LayerArray:
 
 def moe_poll_status(ws, stream=None) -> int:
     return lib().moe_poll_status(_ptr(ws), _stream(stream))
+
+
+def moe_noalloc_poll_status(stream=None) -> int:
+    """Status latched by earlier moe_layer_forward_noalloc calls on the current device (then cleared)."""
+    return lib().moe_noalloc_poll_status(_stream(stream))
+
+
+def moe_selftest_grid_timeout(ws, bound_ns: int, stream=None):
+    """A grid-barrier wait that runs out (see moe.h): latches MOE_ERR_TIMEOUT in ws."""
+    _ok(lib().moe_selftest_grid_timeout(_ptr(ws), ws.numel() * ws.element_size(), int(bound_ns), _stream(stream)),
+        "moe_selftest_grid_timeout")
 
 
 def moe_selftest_wait_timeout(ws, bound_ns: int, stream=None):

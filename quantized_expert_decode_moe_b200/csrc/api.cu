@@ -20,14 +20,19 @@ constexpr int kDecodeMaxT = 8;
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
-// Bound of every device-side wait (a staged copy that never lands): 20 ms, or
-// MOE_WAIT_TIMEOUT_NS from the environment (read once).
+// Bound of every device-side wait (a staged copy that never lands, a CTA
+// that never reaches a grid barrier): 100 ms, or MOE_WAIT_TIMEOUT_NS from the
+// environment (read once), clamped to [1 ms, 10 s] so that a normal wait on a
+// busy or time-sliced GPU does not run out.
 unsigned long long wait_bound_ns() {
   static unsigned long long v = 0;
   if (!v) {
     const char* e = getenv("MOE_WAIT_TIMEOUT_NS");
     unsigned long long x = e ? strtoull(e, nullptr, 10) : 0ull;
-    v = x ? x : 20000000ull;
+    if (!x) x = 100000000ull;
+    if (x < 1000000ull) x = 1000000ull;
+    if (x > 10000000000ull) x = 10000000000ull;
+    v = x;
   }
   return v;
 }
@@ -60,6 +65,18 @@ moe_status check_layer(const moe_layer* L) {
 }
 
 int slots_of(const moe_layer* L) { return L->top_k + (L->has_shared ? 1 : 0); }
+
+// The kernels that serve T tokens of a layer, chosen on the host before any
+// launch: the fused single-kernel layer for one token, the four-kernel chain
+// for up to 8 tokens, the grouped prefill path above that.
+enum class Path { kNone, kFused, kChain, kPrefill };
+Path path_of(const moe_layer* L, int T) {
+  if (T > kDecodeMaxT) return prefill_supported(L->hidden, L->inter, L->bits) ? Path::kPrefill : Path::kNone;
+  if (T == 1 && fused_supported(L->hidden, L->inter, L->n_experts, L->top_k, L->has_shared, L->bits))
+    return Path::kFused;
+  if (chain_supported(L->hidden, L->inter, L->top_k, L->has_shared, L->bits)) return Path::kChain;
+  return Path::kNone;
+}
 
 WsLayout layout_of(const moe_layer* L, int T) {
   return ws_layout(L->hidden, L->inter, L->n_experts, L->top_k, slots_of(L), T);
@@ -100,6 +117,7 @@ moe_status decode_chain(const moe_layer* L, const uint16_t* x_in, float* h, int 
   rp.H = H; rp.E = E; rp.T = T; rp.has_shared = L->has_shared;
   rp.x = x_in; rp.router_w = L->router_w; rp.router_bias = L->router_bias; rp.gate_w = L->shared_gate_w;
   rp.logits = at<double>(ws, W.logits);
+  rp.bound = at<float>(ws, W.bound);
   rp.h = h; rp.x_rec = x_rec; rp.h_rec = h_rec;
   cudaError_t e = launch_route(rp, s, pdl);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
@@ -108,10 +126,12 @@ moe_status decode_chain(const moe_layer* L, const uint16_t* x_in, float* h, int 
   GateUpParams gp{};
   gp.H = H; gp.I = I; gp.E = E; gp.k = k; gp.S = S; gp.has_shared = L->has_shared;
   gp.nCTA = gateup_ctas(I);
-  gp.x = x_in; gp.logits = rp.logits; gp.experts = L->experts; gp.shared = L->shared;
+  gp.x = x_in; gp.logits = rp.logits; gp.bound = rp.bound; gp.experts = L->experts; gp.shared = L->shared;
+  gp.router_w = L->router_w; gp.router_bias = L->router_bias;
   gp.a = at<float>(ws, W.a);
   gp.idx_out = topk_idx; gp.w_out = topk_w;
   gp.status = status; gp.wait_ns = wait_bound_ns();
+  gp.rechecks = at<uint32_t>(ws, 16);
   if ((e = launch_gateup(gp, L->bits, T, pdl, s)) != cudaSuccess)
     return e == cudaErrorInvalidConfiguration ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
   mark(2);
@@ -119,7 +139,8 @@ moe_status decode_chain(const moe_layer* L, const uint16_t* x_in, float* h, int 
   DownParams dp{};
   dp.H = H; dp.I = I; dp.E = E; dp.k = k; dp.S = S; dp.has_shared = L->has_shared;
   dp.nCTA = down_ctas(H);
-  dp.logits = rp.logits; dp.a = gp.a; dp.h = h; dp.experts = L->experts; dp.shared = L->shared;
+  dp.x = x_in; dp.logits = rp.logits; dp.bound = rp.bound; dp.a = gp.a; dp.h = h; dp.experts = L->experts;
+  dp.shared = L->shared; dp.router_w = L->router_w; dp.router_bias = L->router_bias;
   dp.hacc = at<float>(ws, W.hacc);
   dp.status = status; dp.wait_ns = gp.wait_ns;
   if ((e = launch_down(dp, L->bits, T, pdl, s)) != cudaSuccess)
@@ -132,6 +153,30 @@ moe_status decode_chain(const moe_layer* L, const uint16_t* x_in, float* h, int 
   if ((e = launch_norm_decode(np, pdl, s)) != cudaSuccess) return MOE_ERR_CUDA;
   mark(4);
   return MOE_OK;
+}
+
+// The fused decode kernel over layers [0, n) of `layers` (one token, n <= kFuMaxLayers).
+moe_status fused_forward(const moe_layer* layers, int n, const uint16_t* x_in, float* h, uint16_t* x_out,
+                         float* x_out_f32, int32_t* idx_out, float* w_out, uint16_t* x_rec, float* h_rec, void* ws,
+                         cudaStream_t s) {
+  const moe_layer& L0 = layers[0];
+  const WsLayout W = layout_of(&L0, 1);
+  FusedParams p{};
+  p.H = L0.hidden; p.I = L0.inter; p.E = L0.n_experts; p.k = L0.top_k; p.S = slots_of(&L0);
+  p.has_shared = L0.has_shared; p.nCTA = fused_ctas(L0.hidden, L0.inter); p.L = n;
+  p.x_in = x_in; p.h = h; p.x_out = x_out; p.x_out_f32 = x_out_f32;
+  p.idx_out = idx_out; p.w_out = w_out; p.x_rec = x_rec; p.h_rec = h_rec;
+  p.status = at<uint32_t>(ws, W.status); p.hdr = at<unsigned>(ws, 0);
+  p.logits = at<double>(ws, W.logits); p.bound = at<float>(ws, W.bound);
+  p.a = at<float>(ws, W.a); p.hacc = at<float>(ws, W.hacc); p.gpart = at<float>(ws, W.gpart);
+  p.wait_ns = wait_bound_ns();
+  for (int l = 0; l < n; ++l) {
+    const moe_layer& Ly = layers[l];
+    FuLayer& f = p.layer[l];
+    f.router_w = Ly.router_w; f.router_bias = Ly.router_bias; f.experts = Ly.experts; f.shared = Ly.shared;
+    f.gate_w = Ly.shared_gate_w; f.gamma = Ly.rms_gamma; f.eps = Ly.rms_eps;
+  }
+  return cuda_status(launch_fused(p, L0.bits, s));
 }
 
 // Prefill (T > 8): router logits for all tokens, top-k, grouping of the
@@ -154,8 +199,10 @@ moe_status prefill_chain(const moe_layer* L, const uint16_t* x_in, float* h, int
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   mark(1);
   TopkParams tp{};
-  tp.E = E; tp.k = k; tp.T = T; tp.has_shared = L->has_shared;
-  tp.logits = rp.logits; tp.idx = at<int32_t>(ws, W.pidx); tp.w = at<float>(ws, W.pw); tp.sg = at<float>(ws, W.psg);
+  tp.E = E; tp.k = k; tp.T = T; tp.has_shared = L->has_shared; tp.H = H;
+  tp.logits = rp.logits; tp.bound = nullptr;   // the fp64 router GEMM's logits are the definition's values
+  tp.x = x_in; tp.router_w = L->router_w; tp.router_bias = L->router_bias;
+  tp.idx = at<int32_t>(ws, W.pidx); tp.w = at<float>(ws, W.pw); tp.sg = at<float>(ws, W.psg);
   if ((e = launch_topk(tp, s)) != cudaSuccess) return MOE_ERR_CUDA;
   if (topk_idx && cudaMemcpyAsync(topk_idx, tp.idx, sizeof(int32_t) * (size_t)T * k, cudaMemcpyDeviceToDevice, s))
     return MOE_ERR_CUDA;
@@ -218,7 +265,25 @@ moe_status moe_workspace_size(const moe_layer* layer, int32_t max_tokens, size_t
   moe_status st = check_layer(layer);
   if (st) return st;
   if (!bytes || max_tokens <= 0) return MOE_ERR_INVALID_ARGUMENT;
+  if (path_of(layer, max_tokens) == Path::kNone) return MOE_ERR_UNSUPPORTED;
   *bytes = layout_of(layer, max_tokens).total;
+  return MOE_OK;
+}
+
+moe_status moe_layer_path(const moe_layer* layer, int32_t T, int32_t* path, int32_t* n_events) {
+  moe_status st = check_layer(layer);
+  if (st) return st;
+  if (T <= 0) return MOE_ERR_INVALID_ARGUMENT;
+  const Path pa = path_of(layer, T);
+  int32_t code = 0, ev = 0;
+  switch (pa) {
+    case Path::kFused: code = MOE_PATH_FUSED; ev = 2; break;
+    case Path::kChain: code = MOE_PATH_CHAIN; ev = 5; break;
+    case Path::kPrefill: code = MOE_PATH_PREFILL; ev = 6; break;
+    default: return MOE_ERR_UNSUPPORTED;
+  }
+  if (path) *path = code;
+  if (n_events) *n_events = ev;
   return MOE_OK;
 }
 
@@ -239,10 +304,14 @@ moe_status moe_route(const moe_layer* layer, const uint16_t* x, int32_t T, int32
   rp.H = layer->hidden; rp.E = layer->n_experts; rp.T = T; rp.has_shared = layer->has_shared;
   rp.x = x; rp.router_w = layer->router_w; rp.router_bias = layer->router_bias; rp.gate_w = layer->shared_gate_w;
   rp.logits = at<double>(ws, W.logits);
+  rp.bound = T > kDecodeMaxT ? nullptr : at<float>(ws, W.bound);
   if ((T > kDecodeMaxT ? launch_route_gemm(rp, s) : launch_route(rp, s, false)) != cudaSuccess) return MOE_ERR_CUDA;
   TopkParams tp{};
-  tp.E = layer->n_experts; tp.k = layer->top_k; tp.T = T; tp.has_shared = layer->has_shared;
-  tp.logits = rp.logits; tp.idx = topk_idx; tp.w = topk_w; tp.sg = shared_gate;
+  tp.E = layer->n_experts; tp.k = layer->top_k; tp.T = T; tp.has_shared = layer->has_shared; tp.H = layer->hidden;
+  tp.logits = rp.logits; tp.bound = rp.bound;
+  tp.x = x; tp.router_w = layer->router_w; tp.router_bias = layer->router_bias;
+  tp.idx = topk_idx; tp.w = topk_w; tp.sg = shared_gate;
+  tp.rechecks = at<uint32_t>(ws, 16);
   return cuda_status(launch_topk(tp, s));
 }
 
@@ -308,9 +377,15 @@ moe_status moe_layer_forward(const moe_layer* layer, const uint16_t* x_in, float
   if (T <= 0 || !x_in || !h || !x_out) return MOE_ERR_INVALID_ARGUMENT;
   if (!aligned16(x_in) || !aligned16(h) || !aligned16(x_out)) return MOE_ERR_INVALID_ARGUMENT;
   if ((st = ws_check(layer, T, ws, ws_bytes))) return st;
-  if (T > kDecodeMaxT)
-    return prefill_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, (cudaStream_t)stream);
-  return decode_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, (cudaStream_t)stream);
+  const Path path = path_of(layer, T);
+  cudaStream_t s = (cudaStream_t)stream;
+  switch (path) {
+    case Path::kPrefill: return prefill_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, s);
+    case Path::kFused:
+      return fused_forward(layer, 1, x_in, h, x_out, x_out_f32, topk_idx, topk_w, nullptr, nullptr, ws, s);
+    case Path::kChain: return decode_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, s);
+    default: return MOE_ERR_UNSUPPORTED;
+  }
 }
 
 moe_status moe_layer_forward_timed(const moe_layer* layer, const uint16_t* x_in, float* h, int32_t T,
@@ -321,13 +396,23 @@ moe_status moe_layer_forward_timed(const moe_layer* layer, const uint16_t* x_in,
   if (T <= 0 || !x_in || !h || !x_out) return MOE_ERR_INVALID_ARGUMENT;
   if (!aligned16(x_in) || !aligned16(h) || !aligned16(x_out)) return MOE_ERR_INVALID_ARGUMENT;
   if ((st = ws_check(layer, T, ws, ws_bytes))) return st;
-  const int need = T > kDecodeMaxT ? 6 : 5;   // kernels (or kernel groups) of the path + 1
+  const Path path = path_of(layer, T);
+  if (path == Path::kNone) return MOE_ERR_UNSUPPORTED;
+  // kernels (or kernel groups) of the path + 1
+  const int need = path == Path::kPrefill ? 6 : (path == Path::kFused ? 2 : 5);
   if (!events || n_events < need) return MOE_ERR_INVALID_ARGUMENT;
   for (int i = 0; i < need; ++i)
     if (!events[i]) return MOE_ERR_INVALID_ARGUMENT;
-  if (T > kDecodeMaxT)
-    return prefill_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, (cudaStream_t)stream, events);
-  return decode_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, (cudaStream_t)stream, events);
+  cudaStream_t s = (cudaStream_t)stream;
+  if (path == Path::kPrefill)
+    return prefill_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, s, events);
+  if (path == Path::kFused) {
+    if (cudaEventRecord((cudaEvent_t)events[0], s) != cudaSuccess) return MOE_ERR_CUDA;
+    if ((st = fused_forward(layer, 1, x_in, h, x_out, x_out_f32, topk_idx, topk_w, nullptr, nullptr, ws, s)))
+      return st;
+    return cuda_status(cudaEventRecord((cudaEvent_t)events[1], s));
+  }
+  return decode_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, s, events);
 }
 
 moe_status moe_stack_forward(const moe_layer* layers, int32_t L, const uint16_t* x_in, float* h, uint16_t* x_out,
@@ -344,8 +429,21 @@ moe_status moe_stack_forward(const moe_layer* layers, int32_t L, const uint16_t*
       return MOE_ERR_INVALID_ARGUMENT;
   }
   if ((st = ws_check(&layers[0], 1, ws, ws_bytes))) return st;
+  const Path path = path_of(&layers[0], 1);   // every layer has the first one's shape
+  if (path == Path::kNone) return MOE_ERR_UNSUPPORTED;
   cudaStream_t s = (cudaStream_t)stream;
   const int H = layers[0].hidden, k = layers[0].top_k;
+  if (path == Path::kFused) {   // up to kFuMaxLayers layers per launch, x and h stay on chip in between
+    for (int l0 = 0; l0 < L; l0 += kFuMaxLayers) {
+      const int n = L - l0 < kFuMaxLayers ? L - l0 : kFuMaxLayers;
+      if ((st = fused_forward(layers + l0, n, l0 == 0 ? x_in : x_out, h, x_out, nullptr,
+                              topk_idx_all ? topk_idx_all + (size_t)l0 * k : nullptr, nullptr,
+                              layer_inputs ? layer_inputs + (size_t)l0 * H : nullptr,
+                              layer_h ? layer_h + (size_t)l0 * H : nullptr, ws, s)))
+        return st;
+    }
+    return MOE_OK;
+  }
   for (int l = 0; l < L; ++l) {
     const uint16_t* xin = l == 0 ? x_in : x_out;
     if ((st = decode_chain(&layers[l], xin, h, 1, x_out, nullptr, topk_idx_all ? topk_idx_all + (size_t)l * k : nullptr,
@@ -393,13 +491,24 @@ moe_status moe_layer_forward_noalloc(const moe_layer* layer, const uint16_t* x_i
   if (T <= 0 || !x_in || !h || !x_out) return MOE_ERR_INVALID_ARGUMENT;
   if (!aligned16(x_in) || !aligned16(h) || !aligned16(x_out)) return MOE_ERR_INVALID_ARGUMENT;
   if (T > kDecodeMaxT) return MOE_ERR_UNSUPPORTED;
+  const Path path = path_of(layer, T);
+  if (path == Path::kNone) return MOE_ERR_UNSUPPORTED;
   if (layout_of(layer, T).total > (size_t)MOE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_WORKSPACE;
   void* ws = noalloc_scratch();
   if (!ws) return MOE_ERR_CUDA;
   cudaStream_t s = (cudaStream_t)stream;
-  // the status word must start clear; the accumulators are cleared by the chain itself
-  if (cudaMemsetAsync(ws, 0, 256, s) != cudaSuccess) return MOE_ERR_CUDA;
+  // The scratch starts zeroed (a static device array), so its status word and
+  // grid-barrier counters start clear; a latched error stays until
+  // moe_noalloc_poll_status reads it. The kernels clear their own accumulators.
+  if (path == Path::kFused)
+    return fused_forward(layer, 1, x_in, h, x_out, x_out_f32, topk_idx, topk_w, nullptr, nullptr, ws, s);
   return decode_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, s);
+}
+
+moe_status moe_noalloc_poll_status(void* stream) {
+  void* ws = noalloc_scratch();
+  if (!ws) return MOE_ERR_CUDA;
+  return moe_poll_status(ws, stream);
 }
 
 moe_status moe_selftest_wait_timeout(void* ws, size_t ws_bytes, uint64_t bound_ns, void* stream) {
@@ -409,14 +518,21 @@ moe_status moe_selftest_wait_timeout(void* ws, size_t ws_bytes, uint64_t bound_n
   return cuda_status(launch_selftest_wait((uint32_t*)ws, (unsigned long long)bound_ns, (cudaStream_t)stream));
 }
 
+moe_status moe_selftest_grid_timeout(void* ws, size_t ws_bytes, uint64_t bound_ns, void* stream) {
+  if (!ws || ws_bytes < 256) return MOE_ERR_WORKSPACE;
+  if (((uintptr_t)ws & 255u) != 0) return MOE_ERR_INVALID_ARGUMENT;
+  if (bound_ns == 0 || bound_ns > 10000000000ull) return MOE_ERR_INVALID_ARGUMENT;
+  return cuda_status(launch_selftest_grid((unsigned*)ws, (unsigned long long)bound_ns, (cudaStream_t)stream));
+}
+
 moe_status moe_poll_status(void* ws, void* stream) {
   if (!ws) return MOE_ERR_WORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;
   if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
   uint32_t v = 0;
   if (cudaMemcpy(&v, ws, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
-  if (v) {
-    if (cudaMemsetAsync(ws, 0, sizeof v, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (v) {   // clear the status word and the grid-barrier counters a failed call may have left mid-round
+    if (cudaMemsetAsync(ws, 0, 256, s) != cudaSuccess) return MOE_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
   }
   return (moe_status)v;

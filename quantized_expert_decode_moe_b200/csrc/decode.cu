@@ -17,102 +17,11 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "stage.cuh"
+#include "sync.cuh"
 #include "topk.cuh"
 
 namespace qmoe {
-
-// ------------------------------------------------------------------ mbarrier and bulk copies
-__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(smem_u32(bar)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
-// orders this thread's earlier generic-proxy accesses of shared memory before its later bulk copies
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, unsigned bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(smem_u32(bar)), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
-  return ok != 0;
-}
-// global -> shared bulk copy of `bytes` (multiple of 16; both addresses 16-byte aligned), counted on bar
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-               :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ unsigned long long globaltimer_ns() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-// Waits for the phase of parity `parity` of bar, for at most bound_ns; on
-// timeout latches MOE_ERR_TIMEOUT in *status and returns false.
-__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, unsigned parity, unsigned long long bound_ns,
-                                            uint32_t* status) {
-  const unsigned long long t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > bound_ns) {
-      if (status) atomicCAS(status, 0u, (uint32_t)MOE_ERR_TIMEOUT);
-      return false;
-    }
-  }
-  return true;
-}
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity, unsigned long long bound_ns,
-                                                  uint32_t* status) {
-  return mbar_try_wait(bar, parity) || mbar_wait_slow(bar, parity, bound_ns, status);
-}
-
-// 16-byte aligned window of rows [r0, r0+n) of a per-row array of SRB bytes
-// per row; `pre` = offset of row r0 inside the window. The window ends inside
-// the array: its size R*SRB is a multiple of 16 (R a multiple of 16, SRB of 4).
-__host__ __device__ __forceinline__ unsigned sb_window(int r0, int n, int SRB, int& pre) {
-  const unsigned o = (unsigned)r0 * (unsigned)SRB, e = o + (unsigned)n * (unsigned)SRB;
-  const unsigned oa = o & ~15u, ea = (e + 15u) & ~15u;
-  pre = (int)(o - oa);
-  return ea - oa;
-}
-__host__ __device__ __forceinline__ int sb_region(int rows, int SRB) { return (rows * SRB + 32 + 15) & ~15; }
-
-__device__ __forceinline__ float silu_f32(float z) { return z / (1.f + expf(-z)); }
-
-// Loads the table builder's elements of chunk q of a bf16 vector.
-template <int BITS>
-__device__ __forceinline__ void load_chunk_bf16(const uint16_t* x, int q, float (&v)[TabTraits<BITS>::kEPT]) {
-  constexpr int EPT = TabTraits<BITS>::kEPT;
-  const uint4* p = (const uint4*)(x + (size_t)q * EPT);
-#pragma unroll
-  for (int u = 0; u < EPT / 8; ++u) {
-    const uint4 r = __ldcg(p + u);
-    const uint32_t w4[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) { v[8 * u + 2 * i] = bf16lo(w4[i]); v[8 * u + 2 * i + 1] = bf16hi(w4[i]); }
-  }
-}
-template <int BITS>
-__device__ __forceinline__ void load_chunk_f32(const float* a, int q, float (&v)[TabTraits<BITS>::kEPT]) {
-  constexpr int EPT = TabTraits<BITS>::kEPT;
-  const float4* p = (const float4*)(a + (size_t)q * EPT);
-#pragma unroll
-  for (int u = 0; u < EPT / 4; ++u) {
-    const float4 r = __ldcg(p + u);
-    v[4 * u] = r.x; v[4 * u + 1] = r.y; v[4 * u + 2] = r.z; v[4 * u + 3] = r.w;
-  }
-}
-
-// 16 bytes of scale or bias data (4 spans x a bf16 pair) at p: one 16-byte
-// load when the per-row arrays keep 16-byte alignment, else four 4-byte loads.
-__device__ __forceinline__ uint4 lds_chunk(const unsigned char* p, bool al16) {
-  if (al16) return *(const uint4*)p;
-  const uint32_t* q = (const uint32_t*)p;
-  return make_uint4(q[0], q[1], q[2], q[3]);
-}
-__device__ __forceinline__ uint32_t chunk_word(const uint4& v, int i) {
-  return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
-}
 
 // ------------------------------------------------------------------ gate/up + SwiGLU
 constexpr int kGuBufs = 3;      // expert tiles staged per CTA (the shared expert's buffer is reused)
@@ -309,26 +218,35 @@ __global__ void __launch_bounds__(kThreads, 2) gateup_decode_kernel(GateUpParams
   // the router's logits are complete after the wait
   griddep_wait();
   griddep_launch_dependents();
-  block_topk(p.logits + (size_t)t * (p.E + 1), p.E, k, p.has_shared, ts);
+  {
+    const RouterRef rr{p.x + (size_t)t * H, p.router_w, p.router_bias, H};
+    block_topk(p.logits + (size_t)t * (p.E + 1), p.bound + (size_t)t * (p.E + 1), p.E, k, p.has_shared, rr, ts);
+  }
   load_slots(ts, k, p.E, p.experts, slot_ex, p.status);
+  if (blockIdx.x == 0 && tid == 0 && p.rechecks && ts.rechecked) atomicAdd(p.rechecks, 1u);
   if (blockIdx.x == 0 && tid < k) {
     if (p.idx_out) p.idx_out[(size_t)t * k + tid] = ts.idx[tid];
     if (p.w_out) p.w_out[(size_t)t * k + tid] = ts.w[tid];
   }
   // routed items in waves of up to kGuBufs; every warp takes its spans of all items of the wave
+  int issued = it0;   // items [0, issued) have had their copies issued
   for (int w0 = it0; w0 < nitems; w0 += kGuBufs) {
     const int w1 = nitems - w0 < kGuBufs ? nitems : w0 + kGuBufs;
+    // after a wait ran out, nothing more is armed or issued (a new phase on a
+    // buffer whose copies may still be landing would mix two phases)
+    if (!__syncthreads_and(ok)) break;
     for (int it = w0; it < w1; ++it) arm(it);
     __syncthreads();   // slots loaded (first wave) / previous wave's buffers and partial sums consumed
     if (lane == 0)
       for (int c = warp; c < ncp * (w1 - w0); c += kWarps) issue(w0 + c / ncp, c % ncp);
+    issued = w1;
     compute_items(w0, w1);
     fence_proxy_async();
     __syncthreads();
     finalize(w0, w1);
   }
-  if (!ok) {   // a copy never landed: give the copies in flight one more bound before leaving
-    for (int it = (nitems > kGuBufs ? nitems - kGuBufs : 0); it < nitems; ++it)
+  if (!__syncthreads_and(ok) && tid == 0) {   // drain: no copy may still be landing when the CTA exits
+    for (int it = (issued > kGuBufs ? issued - kGuBufs : 0); it < issued; ++it)
       mbar_wait_bounded(&bars[it % kGuBufs], (unsigned)(it / kGuBufs) & 1u, p.wait_ns, nullptr);
   }
 }
@@ -532,7 +450,10 @@ __global__ void __launch_bounds__(kThreads, 2) down_decode_kernel(DownParams p) 
     for (int b = 0; b < nb; ++b) mbar_expect_tx(&bars[b], item_bytes);   // items 0..nb-1
     if (p.has_shared) slot_ex[S - 1] = p.shared;
   }
-  block_topk(p.logits + (size_t)t * (p.E + 1), p.E, k, p.has_shared, ts);
+  {
+    const RouterRef rr{p.x + (size_t)t * H, p.router_w, p.router_bias, H};
+    block_topk(p.logits + (size_t)t * (p.E + 1), p.bound + (size_t)t * (p.E + 1), p.E, k, p.has_shared, rr, ts);
+  }
   load_slots(ts, k, p.E, p.experts, slot_ex, p.status);
   if (tid < k) wsl[tid] = ts.w[tid];
   if (tid == 0 && p.has_shared) wsl[S - 1] = ts.sg;
@@ -556,6 +477,8 @@ __global__ void __launch_bounds__(kThreads, 2) down_decode_kernel(DownParams p) 
   for (int w0 = it0; w0 < nitems; w0 += nb) {
     const int w1 = nitems - w0 < nb ? nitems : w0 + nb;
     if (issued < w1) {   // refill buffers whose previous items are done
+      // after a wait ran out, nothing more is armed or issued
+      if (!__syncthreads_and(ok)) break;
       if (tid == 0)
         for (int it = issued; it < w1; ++it) mbar_expect_tx(&bars[it % nb], item_bytes);
       __syncthreads();
@@ -567,8 +490,8 @@ __global__ void __launch_bounds__(kThreads, 2) down_decode_kernel(DownParams p) 
     __syncthreads();
   }
   if (tid < n) p.hacc[(size_t)t * H + h0 + tid] = yacc[tid];
-  if (!ok) {
-    for (int it = (nitems > nb ? nitems - nb : 0); it < nitems; ++it)
+  if (!__syncthreads_and(ok) && tid == 0) {   // drain: no copy may still be landing when the CTA exits
+    for (int it = (issued > nb ? issued - nb : 0); it < issued; ++it)
       mbar_wait_bounded(&bars[it % nb], (unsigned)(it / nb) & 1u, p.wait_ns, nullptr);
   }
 }
@@ -625,6 +548,11 @@ static int optin_smem() {
 }
 
 size_t gateup_smem_bytes(int H, int bits) { return gu_layout(H, bits).total; }
+
+bool chain_supported(int H, int I, int k, int has_shared, int bits) {
+  const int S = k + (has_shared ? 1 : 0);
+  return gu_layout(H, bits).total <= (size_t)optin_smem() && dn_layout(I, S, bits).total <= (size_t)optin_smem();
+}
 size_t down_smem_bytes(int I, int S, int bits) { return dn_layout(I, S, bits).total; }
 
 int gateup_ctas(int I) {

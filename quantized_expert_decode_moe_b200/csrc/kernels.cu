@@ -21,6 +21,8 @@ WsLayout ws_layout(int H, int I, int E, int k, int S, int T) {
   size_t o = 0;
   L.status = o; o = align256(o + 256);
   L.logits = o; o = align256(o + sizeof(double) * (size_t)T * (E + 1));
+  L.bound = o; o = align256(o + sizeof(float) * (size_t)T * (E + 1));
+  L.gpart = o; o = align256(o + sizeof(float) * (size_t)kMaxCtas);
   L.a = o; o = align256(o + sizeof(float) * (size_t)T * S * I);
   L.hacc = o; o = align256(o + sizeof(float) * (size_t)T * H);
   L.counts = o; o = align256(o + sizeof(int32_t) * (size_t)E);
@@ -97,33 +99,13 @@ constexpr int kRouteSplit = 4;
 constexpr int kRouteThreads = kRouteRows * kRouteSplit * 32;
 constexpr int kRouteChunks = 4;   // 16-byte weight chunks per lane per pass
 
-// s + c += x with the rounding error of the addition kept in c (Knuth's TwoSum).
-__device__ __forceinline__ void two_sum_acc(float& s, float& c, float x) {
-  const float t = s + x;
-  const float bp = t - s;
-  c += (s - (t - bp)) + (x - bp);
-  s = t;
-}
-// Dot product of 8 bf16 pairs accumulated as unevaluated sums s[i] + c[i]
-// over 4 independent chains: each bf16 x bf16 product is exact in fp32 and
-// every addition error is carried, so the sum of the chains holds the dot
-// product to about 2^-44 relative to sum |w x|.
-__device__ __forceinline__ void dot8_bf16_comp(uint4 w, uint4 x, float (&s)[4], float (&c)[4]) {
-  const uint32_t wv[4] = {w.x, w.y, w.z, w.w}, xv[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    two_sum_acc(s[i], c[i], bf16lo(wv[i]) * bf16lo(xv[i]));
-    two_sum_acc(s[i], c[i], bf16hi(wv[i]) * bf16hi(xv[i]));
-  }
-}
-
 // The router's weights do not depend on the previous kernel and are loaded
 // before griddepcontrol.wait; x after it. Side job of the decode chain (CTAs
 // of token row 0): optionally record the layer's inputs x and h.
 __global__ void __launch_bounds__(kRouteThreads) route_logits_kernel(RouteParams p) {
   extern __shared__ __align__(128) unsigned char smem[];
   uint4* xs = (uint4*)smem;                                  // [H/8]
-  __shared__ float part[kRouteRows][kRouteSplit][2];
+  __shared__ float part[kRouteRows][kRouteSplit][3];
   const int t = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nch = p.H / 8, half = nch / kRouteSplit;   // chunks per warp's part of the row
   const int nrows = p.E + (p.has_shared ? 1 : 0);
@@ -131,7 +113,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_logits_kernel(RouteParams
   const int e = blockIdx.x * kRouteRows + rl;
   const uint16_t* wrow = e < p.E ? p.router_w + (size_t)e * p.H : p.gate_w;
   const int cb = hs * half;   // first chunk of this warp's part
-  float cs[4] = {0.f, 0.f, 0.f, 0.f}, cc[4] = {0.f, 0.f, 0.f, 0.f};
+  float cs[4] = {0.f, 0.f, 0.f, 0.f}, cc[4] = {0.f, 0.f, 0.f, 0.f}, sa = 0.f;
   for (int c0 = 0; c0 < half; c0 += 32 * kRouteChunks) {
     uint4 wv[kRouteChunks];
 #pragma unroll
@@ -168,7 +150,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_logits_kernel(RouteParams
 #pragma unroll
     for (int i = 0; i < kRouteChunks; ++i) {
       const int c = c0 + lane + 32 * i;
-      if (c < half) dot8_bf16_comp(wv[i], xs[cb + c], cs, cc);
+      if (c < half) dot8_bf16_comp(wv[i], xs[cb + c], cs, cc, sa);
     }
   }
   float as_ = cs[0], ac_ = cc[0] + cc[1] + cc[2] + cc[3];
@@ -181,17 +163,21 @@ __global__ void __launch_bounds__(kRouteThreads) route_logits_kernel(RouteParams
     ac_ += oc;
     two_sum_acc(as_, ac_, os);
   }
-  if (lane == 0 && hs != 0) { part[rl][hs][0] = as_; part[rl][hs][1] = ac_; }
+  sa = warp_sum(sa);
+  if (lane == 0 && hs != 0) { part[rl][hs][0] = as_; part[rl][hs][1] = ac_; part[rl][hs][2] = sa; }
   __syncthreads();
   if (lane == 0 && hs == 0 && e < nrows) {
 #pragma unroll
     for (int q = 1; q < kRouteSplit; ++q) {
       ac_ += part[rl][q][1];
       two_sum_acc(as_, ac_, part[rl][q][0]);
+      sa += part[rl][q][2];
     }
     double acc = (double)as_ + (double)ac_;
-    if (e < p.E && p.router_bias) acc += (double)p.router_bias[e];
+    const double bias = (e < p.E && p.router_bias) ? (double)p.router_bias[e] : 0.0;
+    acc += bias;
     p.logits[(size_t)t * (p.E + 1) + e] = acc;
+    if (p.bound && e < p.E) p.bound[(size_t)t * (p.E + 1) + e] = logit_bound(p.H, sa, acc, bias);
   }
 }
 
@@ -199,12 +185,15 @@ __global__ void __launch_bounds__(kRouteThreads) route_logits_kernel(RouteParams
 __global__ void __launch_bounds__(kThreads) topk_kernel(TopkParams p) {
   __shared__ TopkSmem ts;
   const int t = blockIdx.x, tid = threadIdx.x;
-  block_topk(p.logits + (size_t)t * (p.E + 1), p.E, p.k, p.has_shared, ts);
+  const RouterRef rr{p.x + (size_t)t * p.H, p.router_w, p.router_bias, p.H};
+  block_topk(p.logits + (size_t)t * (p.E + 1), p.bound ? p.bound + (size_t)t * (p.E + 1) : nullptr, p.E, p.k,
+             p.has_shared, rr, ts);
   if (tid < p.k) {
     p.idx[(size_t)t * p.k + tid] = ts.idx[tid];
     p.w[(size_t)t * p.k + tid] = ts.w[tid];
   }
   if (tid == 0 && p.sg) p.sg[t] = ts.sg;
+  if (tid == 0 && p.rechecks && ts.rechecked) atomicAdd(p.rechecks, 1u);
 }
 
 // ------------------------------------------------------------------ RMSNorm of the accumulated h' (decode)

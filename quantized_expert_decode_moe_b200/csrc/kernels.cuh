@@ -9,10 +9,17 @@
 
 namespace qmoe {
 
-// Workspace carve-up for T tokens of one layer shape.
+constexpr int kMaxCtas = 1024;   // CTAs of the fused decode kernel at most
+
+// Workspace carve-up for T tokens of one layer shape. The first 256 bytes are
+// the header: the status word (word 0), the count of top-k selections that
+// needed the exact recheck (word 4), the grid-barrier arrival counters
+// (words 16..19) and generations (words 32, 40, 48, 56).
 struct WsLayout {
   size_t status;      // uint32 status word (+ padding)
   size_t logits;      // double [T][E+1]; column E = shared-gate logit
+  size_t bound;       // float [T][E+1]  error bounds of fast logits
+  size_t gpart;       // float [kMaxCtas] per-CTA partial sums (fused decode)
   size_t a;           // float [T][S][I]  silu(gate) * up of each slot (slot S-1 = shared expert)
   size_t hacc;        // float [T][H]     h + weighted expert outputs
   // prefill
@@ -40,31 +47,43 @@ struct RouteParams {
   const float* router_bias;     // [E] or null
   const uint16_t* gate_w;       // [H] or null
   double* logits;               // [T][E+1]
+  float* bound;                 // [T][E+1]: bound on |logit - fp64 definition| (null: not written)
   // side job of the decode chain (null when unused): copies of the layer's inputs x, h ([T][H])
   const float* h; uint16_t* x_rec; float* h_rec;
 };
 
 struct TopkParams {
-  int E, k, T, has_shared;
+  int E, k, T, has_shared, H;
   const double* logits;        // [T][E+1]
+  const float* bound;          // [T][E+1] error bounds of fast logits, or null (logits exact)
+  const uint16_t* x;           // [T][H]  } what an exact recheck of a logit reads
+  const uint16_t* router_w;    // [E][H]  }
+  const float* router_bias;    // [E] or null
   int32_t* idx; float* w; float* sg;   // outputs (sg nullable)
+  uint32_t* rechecks;          // counter of selections that needed the exact recheck, or null
 };
 
 struct GateUpParams {
   int H, I, E, k, S, has_shared, nCTA;
   const uint16_t* x;           // [T][H]
   const double* logits;        // [T][E+1]
+  const float* bound;          // [T][E+1] error bounds of the logits
+  const uint16_t* router_w; const float* router_bias;   // for an exact recheck of near ties
   const moe_expert* experts;   // device [E]
   moe_expert shared;
   float* a;                    // [T][S][I]
   int32_t* idx_out; float* w_out;   // user copies of the routing, nullable
+  uint32_t* rechecks;          // counter of selections that needed the exact recheck, or null
   uint32_t* status;
   unsigned long long wait_ns;  // bound of every device-side wait
 };
 
 struct DownParams {
   int H, I, E, k, S, has_shared, nCTA;
+  const uint16_t* x;           // [T][H]
   const double* logits;        // [T][E+1]
+  const float* bound;          // [T][E+1] error bounds of the logits
+  const uint16_t* router_w; const float* router_bias;   // for an exact recheck of near ties
   const float* a;              // [T][S][I]
   const float* h;              // [T][H] residual
   const moe_expert* experts;
@@ -128,6 +147,36 @@ struct GroupParams {
   int4* chunks; int32_t* nchunks;
 };
 
+// One layer of the fused decode kernel (device pointers).
+struct FuLayer {
+  const uint16_t* router_w;    // [E][H]
+  const float* router_bias;    // [E] or null
+  const moe_expert* experts;   // device [E]
+  moe_expert shared;
+  const uint16_t* gate_w;      // [H] or null
+  const uint16_t* gamma;       // [H]
+  float eps;
+};
+constexpr int kFuMaxLayers = 24;   // layers per launch of the fused kernel (kernel parameter space)
+
+struct FusedParams {
+  int H, I, E, k, S, has_shared, nCTA, L;
+  const uint16_t* x_in;        // [H] bf16, the first layer's input
+  float* h;                    // [H] residual in, h' of the last layer out
+  uint16_t* x_out;             // [H] bf16, the last layer's output
+  float* x_out_f32;            // [H] or null
+  int32_t* idx_out; float* w_out;   // [L][k] routing of every layer, nullable
+  uint16_t* x_rec; float* h_rec;    // [L][H] inputs x, h of every layer, nullable
+  uint32_t* status;            // workspace status word
+  unsigned* hdr;               // workspace header (grid barrier counters at words 16.., generations at 32..)
+  double* logits; float* bound;     // [E+1]
+  float* a;                    // [S][I]
+  float* hacc;                 // [H]
+  float* gpart;                // [nCTA] partial sums of squares
+  unsigned long long wait_ns;
+  FuLayer layer[kFuMaxLayers];
+};
+
 // launchers (return the launch's cudaError_t)
 cudaError_t launch_route(const RouteParams& p, cudaStream_t s, bool pdl);
 cudaError_t launch_route_gemm(const RouteParams& p, cudaStream_t s);   // many tokens: tiled fp64
@@ -145,7 +194,14 @@ cudaError_t launch_group(const GroupParams& p, cudaStream_t s);
 cudaError_t launch_prefill_gateup(const PrefillParams& p, int bits, cudaStream_t s);   // digit tables of x + gate/up
 cudaError_t launch_prefill_down(const PrefillParams& p, int bits, cudaStream_t s);     // digit tables of a + down
 cudaError_t launch_selftest_wait(uint32_t* status, unsigned long long bound_ns, cudaStream_t s);
+cudaError_t launch_selftest_grid(unsigned* hdr, unsigned long long bound_ns, cudaStream_t s);
 int num_sms();
+bool fused_supported(int H, int I, int E, int k, int has_shared, int bits);
+int fused_ctas(int H, int I);
+size_t fused_smem_bytes(int H, int I, int S, int bits);
+cudaError_t launch_fused(const FusedParams& p, int bits, cudaStream_t s);
+bool chain_supported(int H, int I, int k, int has_shared, int bits);
+bool prefill_supported(int H, int I, int bits);
 int pf_chunk_tokens(int H, int I);   // tokens per chunk of the grouped GEMMs
 size_t pf_max_chunks(int T, int k, int E, int chunk);
 int choose_ncta(long long ntiles, int nspans);

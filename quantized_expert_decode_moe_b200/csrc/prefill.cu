@@ -689,20 +689,25 @@ static cudaError_t pf_prepare(const void* fn, size_t bytes) {
   return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
-template <int BITS, bool GU>
-static cudaError_t pf_grouped(const PrefillParams& p, cudaStream_t s) {
-  const int K = GU ? p.H : p.I;
-  const int C = pf_chunk_tokens(p.H, p.I);
+// Launch configuration of a grouped kernel (gate/up or down) of a layer shape:
+// row tile groups per item, tiles per warp, stages; false when the shape
+// cannot run (too many groups per warp, row tiles that do not divide, or
+// fewer than two stages in the shared memory of one CTA).
+struct PfConfig { int rt, rw, nst; };
+static bool pf_config(int H, int I, int bits, bool gu, PfConfig& cf) {
+  const int K = gu ? H : I;
+  const int C = pf_chunk_tokens(H, I);
   const int RT = C == 8 ? pf_row_tiles(K) : 1;
   const int ng = K / kGroup, NS = kPfWarps / RT, gpw = (ng + NS - 1) / NS;
-  if (gpw > (C == 8 ? 4 : 8)) return cudaErrorInvalidConfiguration;
-  const int rows = GU ? p.I / 8 : p.H / 16;   // 16-row tiles per expert matrix
-  if (rows % RT != 0) return cudaErrorInvalidConfiguration;
+  if (gpw > (C == 8 ? 4 : 8)) return false;
+  const int rows = gu ? I / 8 : H / 16;   // 16-row tiles per expert matrix
+  if (rows % RT != 0) return false;
   int optin = 0, dev = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (optin <= 0) optin = 227 * 1024;
   auto stages = [&](int rw) {
-    const size_t fixed = pf_geom(K, BITS, C, RT, rw, 0).total, stage = pf_geom(K, BITS, C, RT, rw, 1).stage;
+    const size_t fixed = pf_geom(K, bits, C, RT, rw, 0).total, stage = pf_geom(K, bits, C, RT, rw, 1).stage;
     if ((size_t)optin < fixed + 2 * stage) return 0;
     const int n = (int)(((size_t)optin - fixed) / stage);
     return n > kPfMaxStages ? kPfMaxStages : n;
@@ -710,12 +715,27 @@ static cudaError_t pf_grouped(const PrefillParams& p, cudaStream_t s) {
   // two tiles per warp where the shapes divide and two stages still fit
   const int RW = (C == 8 && rows % (2 * RT) == 0 && stages(2) >= 2) ? 2 : 1;
   const int nst = stages(RW);
-  if (nst < 2) return cudaErrorInvalidConfiguration;
+  if (nst < 2) return false;
+  cf.rt = RT; cf.rw = RW; cf.nst = nst;
+  return true;
+}
+
+bool prefill_supported(int H, int I, int bits) {
+  PfConfig a, b;
+  return pf_config(H, I, bits, true, a) && pf_config(H, I, bits, false, b);
+}
+
+template <int BITS, bool GU>
+static cudaError_t pf_grouped(const PrefillParams& p, cudaStream_t s) {
+  const int K = GU ? p.H : p.I;
+  const int C = pf_chunk_tokens(p.H, p.I);
+  PfConfig cf;
+  if (!pf_config(p.H, p.I, BITS, GU, cf)) return cudaErrorInvalidConfiguration;
   PrefillParams q = p;
-  q.nst = nst;
-  q.rt = RT;
-  q.rw = RW;
-  const size_t sm = pf_geom(K, BITS, C, RT, RW, nst).total;
+  q.nst = cf.nst;
+  q.rt = cf.rt;
+  q.rw = cf.rw;
+  const size_t sm = pf_geom(K, BITS, C, cf.rt, cf.rw, cf.nst).total;
   const void* fn = C == 8 ? (const void*)prefill_grouped_kernel<BITS, GU, 4, 2>
                           : (const void*)prefill_grouped_kernel<BITS, GU, 8, 1>;
   cudaError_t e = pf_prepare(fn, sm);

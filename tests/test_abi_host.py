@@ -153,3 +153,44 @@ def test_entry_points_reject_bad_arguments_before_launch():
     assert L.moe_selftest_wait_timeout(C.c_void_p(0x400010), n, 1000, None) == 1
     assert L.moe_selftest_wait_timeout(ws, n, 0, None) == 1
     assert L.moe_selftest_wait_timeout(ws, n, 20 * 10 ** 9, None) == 1
+
+
+def test_unlaunchable_decode_shapes_are_rejected_before_launch():
+    """Hidden 8192, intermediate 3072, 4-bit, top-3 + shared: the decode
+    kernels' staging of a CTA's rows does not fit one CTA's shared memory, so
+    every decode entry point refuses the layer with MOE_ERR_UNSUPPORTED for
+    every token count from 1 to 8. On a machine without a GPU any launch
+    would fail with MOE_ERR_CUDA instead, so these codes also show that
+    nothing was launched. The grouped prefill path (T > 8) still takes the
+    layer, and the largest shapes each decode path accepts pass the checks."""
+    L = qm.lib()
+    bad = fake_layer(hidden=8192, inter=3072)
+    p = C.c_void_p(0x200000)
+    ws = C.c_void_p(0x400000)
+    for T in (1, 8):
+        assert ws_size(bad, T)[0] == 2
+    rc, n = ws_size(bad, 9)
+    assert rc == 0 and n > 0
+    ev = (C.c_void_p * 6)(*[0x1000] * 6)
+    for T in range(1, 9):
+        assert L.moe_layer_forward(C.byref(bad), p, p, T, p, None, None, None, ws, n, None) == 2
+        assert L.moe_layer_forward_timed(C.byref(bad), p, p, T, p, None, None, None, ws, n, ev, 6, None) == 2
+        assert L.moe_layer_forward_noalloc(C.byref(bad), p, p, T, p, None, None, None, None) == 2
+    lays = (qm._Layer * 3)(bad, bad, bad)
+    assert L.moe_stack_forward(lays, 3, p, p, p, None, None, None, ws, n, None) == 2
+    # the limits: fused (T = 1) up to hidden 4096 / inter 1152; the chain up to hidden 7552 / inter 2688 (4-bit)
+    assert ws_size(fake_layer(hidden=4096, inter=1152), 1)[0] == 0
+    assert ws_size(fake_layer(hidden=7552, inter=2688), 1)[0] == 0
+    assert ws_size(fake_layer(hidden=7552, inter=2688), 8)[0] == 0
+    assert ws_size(fake_layer(hidden=7680, inter=1024), 8)[0] == 2
+    assert ws_size(fake_layer(hidden=4096, inter=2816), 8)[0] == 2
+    assert ws_size(fake_layer(hidden=8192, inter=2048, bits=2), 8)[0] == 0
+
+
+def test_wait_bound_and_header_words_documented():
+    """The header states the default bound of device-side waits and the
+    workspace header words the tests read (status, recheck count, grid-barrier
+    counters)."""
+    text = open(HEADER).read()
+    assert "100 ms" in text and "MOE_WAIT_TIMEOUT_NS" in text
+    assert "byte offset 16" in text and "moe_noalloc_poll_status" in text

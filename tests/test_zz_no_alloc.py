@@ -66,18 +66,30 @@ def test_noalloc_forward_matches_workspace_forward(name, T):
         for i in range(T):
             assert rel_err(got["h"][i], ref["h"][i]) <= TOL
             assert rel_err(got["xf"][i], ref["xf"][i]) <= TOL
+    assert qm.moe_noalloc_poll_status() == 0     # nothing latched in the static scratch
 
 
 def test_noalloc_scratch_covers_largest_decode_shape():
-    """The largest layer the decode chain accepts (hidden = inter = 8192, 4096
-    experts, top-8 + shared, 8 tokens) fits the static scratch, so the
-    oversize rejection cannot trigger for a valid call; more than 8 tokens is
-    refused as unsupported before the scratch is touched."""
+    """Every decode shape the library accepts fits the static scratch, so the
+    oversize rejection cannot trigger for a call that could otherwise run:
+    the workspace for 8 tokens stays within MOE_NOALLOC_SCRATCH_BYTES at the
+    largest hidden and intermediate sizes the decode kernels take (4 and 2
+    bits, top-3 and top-8 with a shared expert, 4096 experts). A shape the
+    decode kernels cannot run, and more than 8 tokens, are refused as
+    unsupported before the scratch is touched."""
     L = qm.lib()
     p = 0x100000
     ex = qm._Expert(*[qm._QMat(p, p, p) for _ in range(3)])
-    big = qm._Layer(8192, 8192, 4096, 8, 4, 64, 1, 1e-6, p, None, p, ex, p, p)
-    n = C.c_size_t(0)
-    assert L.moe_workspace_size(C.byref(big), 8, C.byref(n)) == 0 and 0 < n.value <= (4 << 20)
+    cases = [(4, 3, 7552, 2688), (4, 8, 7552, 2176), (2, 3, 8192, 4352), (2, 8, 8192, 3328)]
+    for bits, k, H, I in cases:
+        lay = qm._Layer(H, I, 4096, k, bits, 64, 1, 1e-6, p, None, p, ex, p, p)
+        n = C.c_size_t(0)
+        assert L.moe_workspace_size(C.byref(lay), 8, C.byref(n)) == 0, (bits, k, H, I)
+        assert 0 < n.value <= (4 << 20)
+        big = qm._Layer(H, I + 128 * (1 if bits == 4 else 8), 4096, k, bits, 64, 1, 1e-6, p, None, p, ex, p, p)
+        assert L.moe_workspace_size(C.byref(big), 8, C.byref(n)) == 2   # one span more: no longer fits
     pp = C.c_void_p(0x200000)
-    assert L.moe_layer_forward_noalloc(C.byref(big), pp, pp, 9, pp, None, None, None, None) == 2   # MOE_ERR_UNSUPPORTED
+    lay = qm._Layer(4096, 1024, 512, 3, 4, 64, 1, 1e-6, p, None, p, ex, p, p)
+    assert L.moe_layer_forward_noalloc(C.byref(lay), pp, pp, 9, pp, None, None, None, None) == 2   # MOE_ERR_UNSUPPORTED
+    bad = qm._Layer(8192, 3072, 512, 3, 4, 64, 1, 1e-6, p, None, p, ex, p, p)
+    assert L.moe_layer_forward_noalloc(C.byref(bad), pp, pp, 1, pp, None, None, None, None) == 2
