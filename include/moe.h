@@ -33,18 +33,18 @@
  *    experts in shared memory, one CTA per SM. A layer call is rejected with
  *    MOE_ERR_UNSUPPORTED, before any launch, when no kernel path fits the
  *    device:
- *      T = 1     the fused single-kernel layer: H <= 4096, top_k <= 3
- *                (top_k + shared <= 4), E <= 4096, I <= 8 n and H <= 32 n
- *                with n = min(SMs, I, H) (148 SMs: I <= 1152); otherwise
- *                the chain below;
- *      T <= 8    the four-kernel chain: gate/up stages 3 experts x 8 rows x H
+ *      T <= 8    the four-kernel decode chain (also for T = 1, by default): gate/up stages 3 experts x 8 rows x H
  *                and down up to 4 experts x 32 rows x I in one CTA (227 KB
  *                per CTA, top_k 3 + shared: H <= 7552 and I <= 2688 at 4
  *                bits, I <= 4352 at 2 bits);
  *      T > 8     the grouped prefill kernels (two stages of their ring of
  *                weight tiles must fit and their row tiles must divide the
  *                matrices);
- *    and H, I <= 8192 throughout.
+ *    and H, I <= 8192 throughout. With MOE_DECODE_KERNEL=fused in the
+ *    environment (read once), single-token calls and stacks take the fused
+ *    single-kernel layer where it fits: H <= 4096, top_k <= 3 (top_k +
+ *    shared <= 4), E <= 4096, I <= 8 n and H <= 32 n with n = min(SMs, I, H)
+ *    (148 SMs: I <= 1152); otherwise the chain.
  *    moe_layer_forward_noalloc and moe_stack_forward apply the same rules
  *    (T = 1 for the stack), and moe_workspace_size applies the rule of
  *    T = max_tokens.
@@ -187,10 +187,12 @@ moe_status moe_group_tokens(int32_t T, int32_t k, int32_t E, const int32_t* topk
 /*
  * Whole MoE layer for T tokens: router, expert gate/up + SwiGLU, down, combine
  * with the shared-expert gate, residual and RMSNorm, all on the device with
- * no host round trip. T = 1 runs the fused decode kernel (the whole layer in
- * one persistent launch, grid-wide barriers between its phases); T = 2..8
- * the four-kernel decode chain; larger T the prefill kernels (grouping by
- * expert, grouped dequant GEMM). See "Supported shapes" above.
+ * no host round trip. T = 1..8 runs the four-kernel decode chain (router,
+ * gate/up + SwiGLU, down + combine, RMSNorm, linked by programmatic
+ * dependent launch), or for T = 1 on request the fused decode kernel (the
+ * whole layer in one persistent launch, grid-wide barriers between its
+ * phases); larger T the prefill kernels (grouping by expert, grouped dequant
+ * GEMM). See "Supported shapes" above.
  *   x_in bf16 [T][H]; h fp32 [T][H] residual in, h' out; x_out bf16 [T][H];
  *   x_out_f32 fp32 [T][H] or NULL; topk_idx int32 [T][k] or NULL;
  *   topk_w fp32 [T][k] or NULL.
@@ -202,9 +204,9 @@ moe_status moe_layer_forward(const moe_layer* layer, const uint16_t* x_in, float
 /*
  * L layers in sequence for one decode token: layer l's x_out feeds layer l+1
  * and h is carried in fp32 ("Deferred GPU expert compute"). With the fused
- * kernel, up to 24 layers run in one launch: x and h stay on the chip
- * between layers, and the next layer's router rows and shared expert are
- * requested while the current layer finishes.
+ * kernel (MOE_DECODE_KERNEL=fused), up to 24 layers run in one launch: x and
+ * h stay on the chip between layers, and the next layer's router rows and
+ * shared expert are requested while the current layer finishes.
  *   layers: host array [L]; x_in bf16 [H]; h fp32 [H] in/out; x_out bf16 [H];
  *   topk_idx_all int32 [L][k] or NULL; layer_inputs bf16 [L][H] or NULL and
  *   layer_h fp32 [L][H] or NULL: each layer's input x and residual h (for
@@ -231,9 +233,8 @@ moe_status moe_layer_path(const moe_layer* layer, int32_t T, int32_t* path, int3
  * recorded before the first and after each of the kernels of the layer, so a
  * caller can time them one by one. events: host array of n_events created
  * cudaEvent_t handles (passed as void*); n_events must be at least the number
- * of recorded stages + 1: fused decode (T = 1) 2 (the one kernel); decode
- * chain (T = 2..8, or T = 1 when the fused kernel does not fit) 5 (router,
- * gate/up, down, norm); prefill 6 (router, top-k + grouping, gate/up, down,
+ * of recorded stages + 1 (moe_layer_path reports it): decode chain 5
+ * (router, gate/up, down, norm); fused decode 2 (the one kernel); prefill 6 (router, top-k + grouping, gate/up, down,
  * combine + norm). The kernels run without programmatic overlap between
  * them. Same arguments and errors otherwise.
  */

@@ -127,13 +127,17 @@ __global__ void __launch_bounds__(kThreads, 2) gateup_decode_kernel(GateUpParams
       for (int it = i0; it < i1; ++it) {
         if (sp == s0) ok &= mbar_wait_bounded(&bars[it % kGuBufs], (unsigned)(it / kGuBufs) & 1u, p.wait_ns, p.status);
         const unsigned char* buf = bufs + (size_t)(it % kGuBufs) * L.GB;
-        const uint4 sv = lds_chunk(buf + 2 * kGuMaxRows * L.P + tq * L.SBR + pre + g * L.SRB + 16 * (sp >> 2), al16);
+        // 16-byte chunk of 4 spans' scale (or bias) words; a pair that starts on the last span of a
+        // chunk (odd first span of the warp) takes its second span from the next chunk
+        const unsigned char* sc = buf + 2 * kGuMaxRows * L.P + tq * L.SBR + pre + g * L.SRB;
+        const uint4 sv0 = lds_chunk(sc + 16 * (sp >> 2), al16);
+        const uint4 sv1 = ((sp & 3) == 3 && sp + 1 < s1) ? lds_chunk(sc + 16 * ((sp + 1) >> 2), al16) : sv0;
         float aa = 0.f, ab = 0.f;
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           const int s = sp + q;
           if (s < s1) {
-            const uint32_t w = chunk_word(sv, s & 3);
+            const uint32_t w = chunk_word(q == 0 ? sv0 : sv1, s & 3);
             uint32_t wa[W], wb[W];
             const unsigned char* ra = buf + (size_t)g * L.P + s * SB + tq * W * 4;
             const unsigned char* rb = ra + (size_t)kGuMaxRows * L.P;

@@ -93,7 +93,8 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
 // ------------------------------------------------------------------ router logits
 // grid (ceil(rows / 2), T), block 256: four warps per router row (row E = the
 // shared-expert gate), each over one quarter of H; every lane keeps its
-// 16-byte chunks of the row in registers.
+// 16-byte chunks of the row in registers. Products exact in fp32, summed in
+// fp64; each routed logit gets its certified bound (logit_bound).
 constexpr int kRouteRows = 2;
 constexpr int kRouteSplit = 4;
 constexpr int kRouteThreads = kRouteRows * kRouteSplit * 32;
@@ -105,7 +106,8 @@ constexpr int kRouteChunks = 4;   // 16-byte weight chunks per lane per pass
 __global__ void __launch_bounds__(kRouteThreads) route_logits_kernel(RouteParams p) {
   extern __shared__ __align__(128) unsigned char smem[];
   uint4* xs = (uint4*)smem;                                  // [H/8]
-  __shared__ float part[kRouteRows][kRouteSplit][3];
+  __shared__ double part[kRouteRows][kRouteSplit];
+  __shared__ float spart[kRouteRows][kRouteSplit];
   const int t = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nch = p.H / 8, half = nch / kRouteSplit;   // chunks per warp's part of the row
   const int nrows = p.E + (p.has_shared ? 1 : 0);
@@ -113,7 +115,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_logits_kernel(RouteParams
   const int e = blockIdx.x * kRouteRows + rl;
   const uint16_t* wrow = e < p.E ? p.router_w + (size_t)e * p.H : p.gate_w;
   const int cb = hs * half;   // first chunk of this warp's part
-  float cs[4] = {0.f, 0.f, 0.f, 0.f}, cc[4] = {0.f, 0.f, 0.f, 0.f}, sa = 0.f;
+  double acc2[2] = {0.0, 0.0};
+  float sa = 0.f;
   for (int c0 = 0; c0 < half; c0 += 32 * kRouteChunks) {
     uint4 wv[kRouteChunks];
 #pragma unroll
@@ -150,30 +153,20 @@ __global__ void __launch_bounds__(kRouteThreads) route_logits_kernel(RouteParams
 #pragma unroll
     for (int i = 0; i < kRouteChunks; ++i) {
       const int c = c0 + lane + 32 * i;
-      if (c < half) dot8_bf16_comp(wv[i], xs[cb + c], cs, cc, sa);
+      if (c < half) dot8_bf16_f64(wv[i], xs[cb + c], acc2, sa);
     }
   }
-  float as_ = cs[0], ac_ = cc[0] + cc[1] + cc[2] + cc[3];
-  two_sum_acc(as_, ac_, cs[1]);
-  two_sum_acc(as_, ac_, cs[2]);
-  two_sum_acc(as_, ac_, cs[3]);
-#pragma unroll
-  for (int o = 16; o; o >>= 1) {
-    const float os = __shfl_xor_sync(0xffffffffu, as_, o), oc = __shfl_xor_sync(0xffffffffu, ac_, o);
-    ac_ += oc;
-    two_sum_acc(as_, ac_, os);
-  }
+  const double v = warp_sum_f64(acc2[0] + acc2[1]);
   sa = warp_sum(sa);
-  if (lane == 0 && hs != 0) { part[rl][hs][0] = as_; part[rl][hs][1] = ac_; part[rl][hs][2] = sa; }
+  if (lane == 0 && hs != 0) { part[rl][hs] = v; spart[rl][hs] = sa; }
   __syncthreads();
   if (lane == 0 && hs == 0 && e < nrows) {
+    double acc = v;
 #pragma unroll
     for (int q = 1; q < kRouteSplit; ++q) {
-      ac_ += part[rl][q][1];
-      two_sum_acc(as_, ac_, part[rl][q][0]);
-      sa += part[rl][q][2];
+      acc += part[rl][q];
+      sa += spart[rl][q];
     }
-    double acc = (double)as_ + (double)ac_;
     const double bias = (e < p.E && p.router_bias) ? (double)p.router_bias[e] : 0.0;
     acc += bias;
     p.logits[(size_t)t * (p.E + 1) + e] = acc;

@@ -9,15 +9,15 @@
 //
 // The logits that define the ranking are the plain fp64 ones: every bf16 x
 // bf16 product is exact in fp64 and the products are summed in index order,
-// then the bias is added. The decode router computes each logit faster
-// (compensated fp32 over a summation tree) together with a rigorous bound
-// b_e on |fast - definition|. Selection runs on the fast values and is then
-// certified: with theta = min over the chosen of (l - b), the chosen set is
-// certain when no other expert has l + b >= theta, and the order among the
-// chosen is certain when adjacent chosen intervals [l - b, l + b] are
-// disjoint. Otherwise every expert with l + b >= theta (a set that contains
-// the true top k) is recomputed exactly as the definition's index-order fp64
-// sum, and the selection runs again on those exact values.
+// then the bias is added. The decode router computes each logit faster (fp64
+// over a summation tree instead of index order) together with a rigorous
+// bound b_e on |fast - definition|. Selection runs on the fast values and is then
+// certified with beta = max_e b_e: when consecutive selected logits, down to
+// the (k+1)-th, are more than 2 beta apart, the definition's top k and their
+// order are the same. Otherwise every expert whose fast logit is within
+// 2 beta of the k-th (a set that contains the true top k) is recomputed
+// exactly as the definition's index-order fp64 sum, and the selection runs
+// again on those exact values.
 #pragma once
 
 #include "common.cuh"
@@ -27,12 +27,14 @@ namespace qmoe {
 constexpr int kTopkPer = 8;   // logits per thread at most: E <= kTopkPer * blockDim
 
 struct TopkSmem {
-  unsigned long long ck[kWarps * kMaxTopK];   // candidate keys, [warp * k + round]
-  int ce[kWarps * kMaxTopK];                  // candidate expert ids
-  int idx[kMaxTopK];
+  unsigned long long ck[kWarps * (kMaxTopK + 1)];   // each warp's best keys, [warp][round]
+  int ce[kWarps * (kMaxTopK + 1)];                  // their expert ids
+  unsigned wb[kWarps];                              // each warp's largest bound (float bits)
+  double thr;                                       // recheck threshold: k-th logit - 2 beta
+  int sure;                                         // the fast selection is certified
+  int idx[kMaxTopK + 1];                      // the selected, best first (one past k when certifying)
   float w[kMaxTopK];
-  double lsel[kMaxTopK];                      // logits of the chosen (the values ranked on)
-  float bsel[kMaxTopK];                       // their error bounds
+  double lsel[kMaxTopK + 1];                  // their logits (the values ranked on)
   float sg;
   int rechecked;                              // the exact recheck ran
 };
@@ -65,45 +67,37 @@ static __device__ __noinline__ double exact_logit(const RouterRef& r, int e) {
   return acc;
 }
 
-// s + c += x with the rounding error of the addition kept in c (Knuth's TwoSum).
-__device__ __forceinline__ void two_sum_acc(float& s, float& c, float x) {
-  const float t = s + x;
-  const float bp = t - s;
-  c += (s - (t - bp)) + (x - bp);
-  s = t;
-}
-// Dot product of 8 bf16 pairs accumulated as unevaluated sums s[i] + c[i]
-// over 4 independent chains: each bf16 x bf16 product is exact in fp32 and
-// every addition error is carried, so the sum of the chains holds the dot
-// product to about 2^-44 relative to sum |w x|, which goes to a.
-__device__ __forceinline__ void dot8_bf16_comp(uint4 w, uint4 x, float (&s)[4], float (&c)[4], float& a) {
+// Dot product of 8 bf16 pairs for the router: each bf16 x bf16 product is
+// exact in fp32 (bf16 has 8 significant bits); it is converted to fp64
+// (exactly) and added into one of two fp64 chains; sum |w x| goes to a (fp32).
+__device__ __forceinline__ void dot8_bf16_f64(uint4 w, uint4 x, double (&acc)[2], float& a) {
   const uint32_t wv[4] = {w.x, w.y, w.z, w.w}, xv[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const float p0 = bf16lo(wv[i]) * bf16lo(xv[i]), p1 = bf16hi(wv[i]) * bf16hi(xv[i]);
-    two_sum_acc(s[i], c[i], p0);
-    two_sum_acc(s[i], c[i], p1);
+    acc[0] += (double)p0;
+    acc[1] += (double)p1;
     a += fabsf(p0) + fabsf(p1);
   }
 }
 
-// Bound on |fast logit - definition| for a logit of n products computed as
-// the compensated fp32 sum of the decode router (every addition of the main
-// sum an error-free TwoSum, the rounding errors carried in a plain fp32 sum),
-// given sa = the fp32 sum of |w x| over the n products, the fast fp64 logit
-// acc (bias included) and the bias. With u = 2^-24 and S = sum |w x|:
-//  - the TwoSum errors e_j satisfy sum |e_j| <= n u S, and carrying them in a
-//    plain fp32 sum adds at most n u sum |e_j| <= n^2 u^2 S;
-//  - the definition (index-order fp64 sum) is within n 2^-53 S of the exact
-//    sum; three fp64 roundings of the results (s + c, + bias, the
-//    definition's + bias) are within 2^-53 (|acc| + |bias|) each;
-//  - an fp32 product below 2^-126 in magnitude loses at most 2^-150;
-//  - sa underestimates S by at most a factor 1 - n u (n <= 8192).
+// Bound on |fast logit - definition| for a logit of n products summed in
+// fp64 in any order (a summation tree), given sa = the fp32 sum of |w x|
+// over the n products, the fast logit acc (bias included) and the bias.
+// With u = 2^-53 and S = sum |w x|:
+//  - any summation tree of n exact terms is within (n-1) u / (1 - (n-1) u) S
+//    of the exact sum (Higham, Accuracy and Stability of Numerical
+//    Algorithms, sec. 4.2), and so is the definition's index-order sum;
+//  - the roundings of "+ bias" on both sides are within u (|acc| + |bias|)
+//    each (with room to spare);
+//  - an fp32 product below 2^-126 in magnitude loses at most 2^-150 (the
+//    definition forms the products in fp64);
+//  - sa underestimates S by at most a factor 1 - n 2^-24 (n <= 8192).
 // The margins 1.25 and 2^-50 cover the last point and the rounding of the
 // bound itself; the result is rounded up to fp32.
 __device__ __forceinline__ float logit_bound(int n, float sa, double acc, double bias) {
   const double nn = (double)n;
-  const double b = 1.25 * (nn * nn * 0x1p-48 + nn * 0x1p-53) * (double)sa + 0x1p-50 * (fabs(acc) + fabs(bias)) +
+  const double b = 1.25 * 2.0 * (nn + 2.0) * 0x1p-53 * (double)sa + 0x1p-50 * (fabs(acc) + fabs(bias)) +
                    nn * 0x1p-148;
   return __double2float_ru(b);
 }
@@ -143,142 +137,133 @@ __device__ __forceinline__ int warp_best(unsigned long long key, int id, unsigne
   return wl;
 }
 
-// The k best of the block's keys (key desc, id asc). Thread tid holds the
-// keys of e = tid + j * blockDim (j < kTopkPer; key 0 = not a candidate); the
-// keys are consumed. Every warp takes its k best in k rounds, warp 0 merges
-// the warps' candidates (exact: every global top-k entry is among its warp's
-// top k). Results: ts.idx[i] (-1 when there are fewer than k candidates) and
-// ts.lsel[i], valid after the call, which ends with __syncthreads.
-// k <= 8 and k * warps <= 128.
+// Block-wide top-k of lg[0..E) (+ shared gate from lg[E] when has_shared),
+// global memory written by an earlier kernel or CTA (read through L2).
+// bnd: per-logit error bounds of fast logits, or null when lg already holds
+// the definition's values. All threads of the block call it (blockDim =
+// 32 * kWarps); results in ts (idx, w, sg), valid after the call, which ends
+// with __syncthreads. Ids of missing entries (fewer than k logits that are
+// not NaN) are -1. k <= 8, E <= kTopkPer * blockDim.
+//
+// Thread tid holds the order keys of e = tid + j * blockDim (j < PER); a key
+// encodes its logit (key_value); 0 = not a candidate (NaN, or past E). Every
+// warp selects its own best n = k + 1 (k without bounds) by rounds of a warp
+// argmax of (key desc, id asc), with no block barrier; lane 0 stores them
+// with the warp's largest bound. After one __syncthreads, warp 0 merges the
+// warps' lists (each sorted best first) into the block's best n (exact:
+// each of the block's best n is among its warp's best n) and certifies them
+// against beta = the
+// token's largest bound: the top k and their order are those of the
+// definition when consecutive selected logits, down to the (k+1)-th, are more
+// than 2 beta apart. Otherwise (rare) every expert within 2 beta of the k-th
+// and the selected are recomputed exactly and the selection runs again.
 template <int PER>
-__device__ __forceinline__ void topk_select(unsigned long long (&key)[PER], int k, TopkSmem& ts) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nt = blockDim.x;
-  auto local_best = [&](unsigned long long& bk, int& bj) {   // lowest j among equal keys
-    bk = 0ull; bj = 0;
+__device__ __forceinline__ void topk_warp_candidates(unsigned long long (&key)[PER], int n, int nt,
+                                                     TopkSmem& ts, unsigned bmax_bits) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+#pragma unroll 1
+  for (int r = 0; r < n; ++r) {
+    unsigned long long bk = 0ull;
+    int bj = 0;
 #pragma unroll
     for (int j = 0; j < PER; ++j)
       if (key[j] > bk) { bk = key[j]; bj = j; }
-  };
-  unsigned long long bk;
-  int bj;
-  local_best(bk, bj);
-  for (int r = 0; r < k; ++r) {
     unsigned long long wk;
     int wi;
     const int wl = warp_best(bk, tid + bj * nt, wk, wi);
-    if (lane == 0) { ts.ck[warp * k + r] = wk; ts.ce[warp * k + r] = wk ? wi : -1; }
     if (lane == wl && wk) {
 #pragma unroll
       for (int j = 0; j < PER; ++j)
         if (j == bj) key[j] = 0ull;
-      local_best(bk, bj);
     }
+    if (lane == 0) { ts.ck[warp * (kMaxTopK + 1) + r] = wk; ts.ce[warp * (kMaxTopK + 1) + r] = wk ? wi : -1; }
   }
-  __syncthreads();
-  if (warp == 0) {
-    const int nc = (nt >> 5) * k;
-    unsigned long long ck[4];   // each lane's candidates c = lane + 32q, sorted best first
-    int ci[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int c = lane + 32 * q;
-      ck[q] = c < nc ? ts.ck[c] : 0ull;
-      ci[q] = c < nc ? ts.ce[c] : -1;
-    }
-    auto cx = [&](int a, int b) {   // compare-exchange: better one to a
-      const bool sw = ck[b] > ck[a] || (ck[b] == ck[a] && ck[a] && (unsigned)ci[b] < (unsigned)ci[a]);
-      if (sw) {
-        const unsigned long long tk = ck[a]; ck[a] = ck[b]; ck[b] = tk;
-        const int ti = ci[a]; ci[a] = ci[b]; ci[b] = ti;
-      }
-    };
-    cx(0, 1); cx(2, 3); cx(0, 2); cx(1, 3); cx(1, 2);
-    for (int r = 0; r < k; ++r) {
-      unsigned long long wk;
-      int wi;
-      const int wl = warp_best(ck[0], ci[0], wk, wi);
-      if (lane == wl) {
-        ck[0] = ck[1]; ci[0] = ci[1]; ck[1] = ck[2]; ci[1] = ci[2]; ck[2] = ck[3]; ci[2] = ci[3];
-        ck[3] = 0ull; ci[3] = -1;
-      }
-      if (lane == 0) {
-        ts.idx[r] = wk ? wi : -1;
-        ts.lsel[r] = wk ? key_value(wk) : __longlong_as_double(0x7ff8000000000000ll);
-      }
-    }
-  }
-  __syncthreads();
+  if (lane == 0) ts.wb[warp] = bmax_bits;
 }
 
-// Block-wide top-k of lg[0..E) (+ shared gate from lg[E] when has_shared),
-// global memory written by an earlier kernel or CTA (read through L2).
-// bnd: per-logit error bounds of fast logits (certified as described at the
-// top of this file, with an exact recheck through rr when needed), or null
-// when lg already holds the definition's values. All threads of the block
-// call it (blockDim = 32 * kWarps); results in ts (idx, w, sg), valid after
-// the call, which ends with __syncthreads. Ids of missing entries (fewer
-// than k logits that are not NaN) are -1. k <= 8, E <= kTopkPer * blockDim.
 template <int PER>
-__device__ __forceinline__ void block_topk_per(const double* lg, const float* bnd, int E, int k, int has_shared,
-                                               const RouterRef& rr, TopkSmem& ts) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nt = blockDim.x;
+static __device__ __noinline__ void block_topk_per(const double* lg, const float* bnd, int E, int k, int has_shared,
+                                                   const RouterRef& rr, TopkSmem& ts) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nt = blockDim.x, nw = nt >> 5;
+  const int n = bnd && k < E ? k + 1 : k;
   double l[PER];
   float b[PER];
-  unsigned long long key[PER];
 #pragma unroll
   for (int j = 0; j < PER; ++j) {
     const int e = tid + j * nt;
     l[j] = e < E ? __ldcg(lg + e) : 0.0;
     b[j] = (bnd && e < E) ? __ldcg(bnd + e) : 0.f;
-    key[j] = e < E ? order_key(l[j]) : 0ull;
   }
   const float gl = (tid == 0 && has_shared) ? (float)__ldcg(lg + E) : 0.f;
-  topk_select(key, k, ts);
-  if (tid == 0) ts.rechecked = 0;
-  if (bnd) {
-    int sel[kMaxTopK];
+  unsigned long long key[PER];
+  float bm = 0.f;
 #pragma unroll
-    for (int i = 0; i < kMaxTopK; ++i) sel[i] = i < k ? ts.idx[i] : -1;
-    auto chosen = [&](int e) {
-      bool c = false;
-#pragma unroll
-      for (int i = 0; i < kMaxTopK; ++i) c |= sel[i] == e;
-      return c;
-    };
-#pragma unroll
-    for (int j = 0; j < PER; ++j) {   // owners publish the bounds of the chosen
-      const int e = tid + j * nt;
-      if (e < E) {
-#pragma unroll
-        for (int i = 0; i < kMaxTopK; ++i)
-          if (sel[i] == e) ts.bsel[i] = b[j];
+  for (int j = 0; j < PER; ++j) {
+    key[j] = tid + j * nt < E ? order_key(l[j]) : 0ull;
+    bm = fmaxf(bm, b[j]);
+  }
+  // non-negative floats order as their bits
+  topk_warp_candidates<PER>(key, n, nt, ts, __reduce_max_sync(0xffffffffu, __float_as_uint(bm)));
+  __syncthreads();
+#pragma unroll 1
+  for (int pass = 0; pass < 2; ++pass) {
+    if (warp == 0) {   // the best n of the warps' candidates: a merge of nw lists sorted best first
+      int ptr = 0;
+      const int base = lane * (kMaxTopK + 1);
+      unsigned long long hk = lane < nw ? ts.ck[base] : 0ull;
+      int hi = lane < nw ? ts.ce[base] : 0x7fffffff;
+      for (int r = 0; r < n; ++r) {
+        unsigned long long wk;
+        int wi;
+        const int wl = warp_best(hk, hi, wk, wi);
+        if (lane == wl && wk) {   // the winning list moves to its next candidate
+          ++ptr;
+          hk = ptr < n ? ts.ck[base + ptr] : 0ull;
+          hi = ptr < n ? ts.ce[base + ptr] : 0x7fffffff;
+        }
+        if (lane == 0) {
+          ts.idx[r] = wk ? wi : -1;
+          ts.lsel[r] = wk ? key_value(wk) : __longlong_as_double(0x7ff8000000000000ll);
+        }
+      }
+      __syncwarp();
+      // certification (lane 0): consecutive selected logits more than 2 beta apart
+      if (lane == 0) {
+        unsigned bb = 0;
+        for (int w = 0; w < nw; ++w) bb = max(bb, ts.wb[w]);
+        const double twob = 2.0 * (double)__uint_as_float(bb);
+        bool sure = !bnd || pass == 1 || ts.idx[0] >= 0;
+        if (bnd && pass == 0)
+          for (int i = 0; i + 1 < n; ++i) sure = sure && ts.idx[i + 1] >= 0 && ts.lsel[i] - ts.lsel[i + 1] > twob;
+        ts.sure = sure ? 1 : 0;
+        ts.thr = ts.lsel[k - 1] - twob;
       }
     }
     __syncthreads();
-    double theta = ts.lsel[0] - (double)ts.bsel[0];
-    bool unsure = !(theta == theta) || sel[0] < 0;
-    for (int i = 1; i < k; ++i) {
-      const double lo = ts.lsel[i] - (double)ts.bsel[i];
-      unsure |= sel[i] < 0 || !(ts.lsel[i - 1] - (double)ts.bsel[i - 1] > ts.lsel[i] + (double)ts.bsel[i]);
-      theta = lo < theta ? lo : theta;
-    }
-#pragma unroll
+    if (ts.sure) break;
+    // ---- rare: the selected and every expert within 2 beta of the k-th, recomputed as the definition
+    const double thr = ts.thr;
+#pragma unroll 1
     for (int j = 0; j < PER; ++j) {
       const int e = tid + j * nt;
-      if (e < E && !chosen(e) && l[j] + (double)b[j] >= theta) unsure = true;
-    }
-    if (__syncthreads_or(unsure)) {   // rare: recompute the candidates exactly and select again
+      double lj = 0.0;
 #pragma unroll
-      for (int j = 0; j < PER; ++j) {
-        const int e = tid + j * nt;
-        key[j] = (e < E && (l[j] + (double)b[j] >= theta || chosen(e) || !(theta == theta)))
-                     ? order_key(exact_logit(rr, e)) : 0ull;
-      }
-      topk_select(key, k, ts);
-      if (tid == 0) ts.rechecked = 1;
+      for (int q = 0; q < PER; ++q)
+        if (q == j) lj = l[q];
+      bool sel = false;
+      for (int i = 0; i < n; ++i) sel |= ts.idx[i] == e;
+      const bool cand = e < E && (sel || !(thr == thr) || lj >= thr);
+      const unsigned long long nk = cand ? order_key(exact_logit(rr, e)) : 0ull;
+#pragma unroll
+      for (int q = 0; q < PER; ++q)
+        if (q == j) key[q] = nk;
     }
+    __syncthreads();   // every thread has read the first selection
+    topk_warp_candidates<PER>(key, n, nt, ts, 0u);
+    if (tid == 0) ts.rechecked = 1;
+    __syncthreads();
   }
-  if (warp == 0) {   // weights over the chosen, shared gate
+  if (warp == 0) {   // weights over the chosen k, shared gate
     const double first = ts.lsel[0];
     const float ex = (lane < k && ts.idx[lane] >= 0) ? expf((float)(ts.lsel[lane] - first)) : 0.f;
     const float z = warp_sum(ex);
@@ -289,6 +274,7 @@ __device__ __forceinline__ void block_topk_per(const double* lg, const float* bn
 }
 __device__ __forceinline__ void block_topk(const double* lg, const float* bnd, int E, int k, int has_shared,
                                            const RouterRef& rr, TopkSmem& ts) {
+  if (threadIdx.x == 0) ts.rechecked = 0;
   if (E <= (int)blockDim.x) block_topk_per<1>(lg, bnd, E, k, has_shared, rr, ts);
   else block_topk_per<kTopkPer>(lg, bnd, E, k, has_shared, rr, ts);
 }

@@ -16,6 +16,8 @@ The same ids and layer outputs are checked through the fused single-kernel
 layer (T = 1) and the four-kernel chain (T = 2..8), and both paths run at the
 largest shape they accept.
 """
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -259,3 +261,24 @@ def test_chain_at_its_largest_shape(dev):
     cfg = fixtures.Config("chain_max", H=7552, E=8, k=3, I=2688, bits=4)
     _layer_vs_oracle(cfg, 1, dev, calls=1)
     _layer_vs_oracle(cfg, 2, dev, calls=1)
+
+
+@pytest.mark.parametrize("bits", [4, 2])
+def test_odd_span_counts(dev, bits):
+    """hidden 3968 (31 spans of 128) and intermediate 896 (7 spans): warps
+    whose share of the spans starts on an odd span, and span pairs that cross
+    a 16-byte chunk of scale words; T = 1 (fused) and T = 2 (chain)."""
+    cfg = fixtures.Config("odd_spans", H=3968, E=12, k=3, I=896, bits=bits,
+                          scale_sigma=0.02 if bits == 4 else 0.05)
+    _layer_vs_oracle(cfg, 1, dev, calls=1)
+    _layer_vs_oracle(cfg, 2, dev, calls=1)
+
+
+def test_decode_path_is_the_one_requested(dev):
+    """Single-token calls take the four-kernel chain unless MOE_DECODE_KERNEL=fused."""
+    t = fxg.device_layer(NT, 0)
+    layer = qm.layer_from_tensors(NT, t)
+    want = "fused" if os.environ.get("MOE_DECODE_KERNEL") == "fused" else "chain"
+    assert qm.moe_layer_path(layer, 1) == (want, 2 if want == "fused" else 5)
+    assert qm.moe_layer_path(layer, 2) == ("chain", 5)
+    assert qm.moe_layer_path(layer, 9) == ("prefill", 6)

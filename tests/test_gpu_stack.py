@@ -9,6 +9,8 @@ The layers are the full decode shape (hidden 4096, 512 experts + 1 shared,
 intermediate 1024, 4-bit), with the per-expert router bias that skews expert
 reuse, all resident on the device at once (about 83 GB).
 """
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -57,6 +59,12 @@ def _run_step(cfg, layers, step, dev):
     assert qm.moe_poll_status(ws) == 0
     return (x_bits, idx.cpu().numpy(), xin.cpu().numpy().view(np.uint16), hin.cpu().numpy(),
             xo.cpu().numpy().view(np.uint16), h.cpu().numpy())
+
+
+def test_stack_runs_the_requested_decode_path(stack):
+    cfg, _, layers = stack
+    want = "fused" if os.environ.get("MOE_DECODE_KERNEL") == "fused" else "chain"
+    assert qm.moe_layer_path(layers[0], 1)[0] == want
 
 
 @pytest.mark.parametrize("step", [0, 1])
