@@ -129,12 +129,13 @@ moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
  * the router results select the experts to load — HN thread, Table 3 comment).
  *   logits = router_w . x (+ router_bias). The ranking is that of the plain
  *   fp64 definition (exact bf16 x bf16 products summed in index order from
- *   0, bias added last). For T > 8 the logits are computed exactly so. For
- *   T <= 8 they are compensated fp32 sums (about 2^-44 relative to
- *   sum |w x|) with a rigorous bound on their distance to the definition;
- *   the top-k is certified against that bound, and when two candidates are
- *   closer than it, every candidate near the k-th is recomputed as the
- *   definition and ranked again, so the indices are those of the definition;
+ *   0, bias added last). The logits are computed faster, as fp64 sums in
+ *   another order (T <= 8: a summation tree per token; T > 8: a GEMM over
+ *   four slices of H), each with a rigorous bound on its distance to the
+ *   definition (about 2^-40 relative). The top-k is certified against the
+ *   bounds, and when two candidates are closer than them, every candidate
+ *   near the k-th is recomputed as the definition and ranked again, so the
+ *   indices are those of the definition;
  *   topk_idx [T][k]: the k largest logits, descending, ties to the lower index;
  *   topk_w [T][k]: softmax over all E renormalised over the chosen k (fp32);
  *   shared_gate [T] (nullable): sigmoid(shared_gate_w . x), 0 if no shared expert.

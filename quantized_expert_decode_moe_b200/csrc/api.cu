@@ -211,13 +211,16 @@ moe_status prefill_chain(const moe_layer* L, const uint16_t* x_in, float* h, int
   rp.H = H; rp.E = E; rp.T = T; rp.has_shared = L->has_shared;
   rp.x = x_in; rp.router_w = L->router_w; rp.router_bias = L->router_bias; rp.gate_w = L->shared_gate_w;
   rp.logits = at<double>(ws, W.logits);
+  rp.bound = at<float>(ws, W.bound);
+  rp.lpart = at<double>(ws, W.lpart); rp.xn2 = at<double>(ws, W.xn2); rp.wn2 = at<double>(ws, W.wn2);
   cudaError_t e = launch_route_gemm(rp, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   mark(1);
   TopkParams tp{};
   tp.E = E; tp.k = k; tp.T = T; tp.has_shared = L->has_shared; tp.H = H;
-  tp.logits = rp.logits; tp.bound = nullptr;   // the fp64 router GEMM's logits are the definition's values
+  tp.logits = rp.logits; tp.bound = rp.bound;
   tp.x = x_in; tp.router_w = L->router_w; tp.router_bias = L->router_bias;
+  tp.rechecks = at<uint32_t>(ws, 16);
   tp.idx = at<int32_t>(ws, W.pidx); tp.w = at<float>(ws, W.pw); tp.sg = at<float>(ws, W.psg);
   if ((e = launch_topk(tp, s)) != cudaSuccess) return MOE_ERR_CUDA;
   if (topk_idx && cudaMemcpyAsync(topk_idx, tp.idx, sizeof(int32_t) * (size_t)T * k, cudaMemcpyDeviceToDevice, s))
@@ -320,7 +323,8 @@ moe_status moe_route(const moe_layer* layer, const uint16_t* x, int32_t T, int32
   rp.H = layer->hidden; rp.E = layer->n_experts; rp.T = T; rp.has_shared = layer->has_shared;
   rp.x = x; rp.router_w = layer->router_w; rp.router_bias = layer->router_bias; rp.gate_w = layer->shared_gate_w;
   rp.logits = at<double>(ws, W.logits);
-  rp.bound = T > kDecodeMaxT ? nullptr : at<float>(ws, W.bound);
+  rp.bound = at<float>(ws, W.bound);
+  rp.lpart = at<double>(ws, W.lpart); rp.xn2 = at<double>(ws, W.xn2); rp.wn2 = at<double>(ws, W.wn2);
   if ((T > kDecodeMaxT ? launch_route_gemm(rp, s) : launch_route(rp, s, false)) != cudaSuccess) return MOE_ERR_CUDA;
   TopkParams tp{};
   tp.E = layer->n_experts; tp.k = layer->top_k; tp.T = T; tp.has_shared = layer->has_shared; tp.H = layer->hidden;

@@ -35,13 +35,16 @@ WsLayout ws_layout(int H, int I, int E, int k, int S, int T) {
   const size_t trows = T > 8 ? (size_t)T : 0;
   L.xd = o; o = align256(o + 2 * trows * H);
   L.xX = o; o = align256(o + sizeof(float) * trows * (H / kGroup));
-  L.xrs = o; o = align256(o + sizeof(float) * trows);
+  L.xrs = o; o = align256(o + sizeof(float) * trows * (H / kGroup));
   L.ad = o; o = align256(o + 2 * prows * I);
   L.aX = o; o = align256(o + sizeof(float) * prows * (I / kGroup));
-  L.ars = o; o = align256(o + sizeof(float) * prows);
+  L.ars = o; o = align256(o + sizeof(float) * prows * (I / kGroup));
   L.chunks = o; o = align256(o + (T > 8 ? sizeof(int4) * pf_max_chunks(T, k, E, pf_chunk_tokens(H, I)) : 0));
   L.nchunks = o; o = align256(o + (T > 8 ? sizeof(int32_t) : 0));
   L.y = o; o = align256(o + sizeof(float) * prows * H);
+  L.lpart = o; o = align256(o + (T > 8 ? sizeof(double) * kRgSplit * (size_t)T * (E + 1) : 0));
+  L.xn2 = o; o = align256(o + (T > 8 ? sizeof(double) * kRgSplit * (size_t)T : 0));
+  L.wn2 = o; o = align256(o + (T > 8 ? sizeof(double) * kRgSplit * (size_t)(E + 1) : 0));
   L.total = o;
   return L;
 }

@@ -10,6 +10,7 @@
 namespace qmoe {
 
 constexpr int kMaxCtas = 1024;   // CTAs of the fused decode kernel at most
+constexpr int kRgSplit = 4;      // slices of H in the many-token router GEMM
 
 // Workspace carve-up for T tokens of one layer shape. The first 256 bytes are
 // the header: the status word (word 0), the count of top-k selections that
@@ -29,13 +30,15 @@ struct WsLayout {
   size_t pidx;        // int32 [T][k]   routed expert ids
   size_t pw;          // float [T][k]   routing weights
   size_t psg;         // float [T]      shared-expert gate
-  size_t xd;          // u8 [T][2H]     digit tables of x (+ xX float [T][H/64], xrs float [T])
+  size_t xd;          // u8 [T][2H]     digit tables of x (+ xX float [T][H/64], xrs float [T][H/64])
   size_t xX, xrs;
   size_t ad;          // u8 [T*k + T][2I]  digit tables of the SwiGLU outputs (+ aX, ars)
   size_t aX, ars;
   size_t chunks;      // int4 [max chunks] (expert, first position, tokens, 0)
   size_t nchunks;     // int32
   size_t y;           // float [T*k + T][H] expert outputs, same rows
+  size_t lpart;       // double [kRgSplit][T][E+1] partial router logits (T > 8)
+  size_t xn2, wn2;    // double [kRgSplit][T], [kRgSplit][E+1] partial squared norms (T > 8)
   size_t total;
 };
 WsLayout ws_layout(int H, int I, int E, int k, int S, int T);
@@ -48,6 +51,9 @@ struct RouteParams {
   const uint16_t* gate_w;       // [H] or null
   double* logits;               // [T][E+1]
   float* bound;                 // [T][E+1]: bound on |logit - fp64 definition| (null: not written)
+  // many tokens: per-slice partial logits [kRgSplit][T][E+1], squared norms of x [kRgSplit][T] and of the
+  // router rows [kRgSplit][E+1]
+  double* lpart; double* xn2; double* wn2;
   // side job of the decode chain (null when unused): copies of the layer's inputs x, h ([T][H])
   const float* h; uint16_t* x_rec; float* h_rec;
 };
@@ -124,11 +130,11 @@ struct PrefillParams {
   const uint16_t* x;           // [T][H] bf16
   unsigned char* xd;           // [T][2H]   digit tables of x
   float* xX;                   // [T][H/64] group sums of x
-  float* xrs;                  // [T]       2^-p of each row of x
+  float* xrs;                  // [T][H/64] 2^-p of each group of x
   float* a;                    // [T*k + T][I] silu(gate) * up per pair (t*k + r), then per token (shared)
   unsigned char* ad;           // [T*k + T][2I] digit tables of a
   float* aX;                   // [T*k + T][I/64]
-  float* ars;                  // [T*k + T]
+  float* ars;                  // [T*k + T][I/64]
   float* y;                    // [T*k + T][H]
   const int4* chunks;          // {expert, first position (perm index, or token for the shared expert), tokens, 0}
   const int32_t* nchunks;      // [1]

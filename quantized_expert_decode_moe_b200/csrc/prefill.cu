@@ -14,7 +14,7 @@
 // Arithmetic: the codes enter the tensor cores as they are stored (u8 planes
 // masked out of the packed words, no dequantisation); every activation row is
 // written once as a 16-bit fixed-point number v = 2^-p (256 d1 + d0) with one
-// exponent p per row and two s8 digits (pf_digitize_kernel). One
+// exponent p per 64-value group and two s8 digits (pf_digitize_kernel). One
 // mma.sync m16n8k32 (u8 x s8 -> s32) takes 16 weight rows x 32 columns
 // against 4 tokens x 2 digits, so per group the integer sums are exact and
 // the float work is one scale and one bias term per row, token and group.
@@ -100,15 +100,18 @@ __device__ __forceinline__ int pf_digit_slot(int c16) {
   else return ((c16 & 3) >> 1) * 8 + (c16 & 1) * 4 + (c16 >> 2);
 }
 
-// One CTA per activation row: p = the largest exponent with max|v| * 2^p <=
-// 32639 (so both digits fit s8 after rounding), v' = rint(v * 2^p),
-// d1 = floor((v' + 128) / 256), d0 = v' - 256 d1; rs[row] = 2^-p and
-// X[row][g] = the fp32 sum of the row's 64 values of group g.
+// One CTA per activation row, one exponent per quantisation group g of 64
+// values: p_g = the largest exponent with max|v_g| * 2^p_g <= 32639 (so both
+// digits fit s8 after rounding), v' = rint(v * 2^p_g), d1 = floor((v' + 128)
+// / 256), d0 = v' - 256 d1; rs[row][g] = 2^-p_g and X[row][g] = the fp32 sum
+// of the group's values. A group's four 16-value units sit on the four
+// threads of a quad, so its maximum and sum are quad reductions. (A group
+// exponent keeps 16 bits relative to the group's own maximum: a large value
+// elsewhere in the row costs the other groups nothing.)
 template <int BITS, bool BF16>
 __global__ void __launch_bounds__(kPfDigitThreads) pf_digitize_kernel(const void* src, int K, unsigned char* dig,
                                                                       float* X, float* rs) {
-  __shared__ uint32_t red[kPfDigitThreads / 32];
-  const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int row = blockIdx.x, tid = threadIdx.x;
   const int units = K / 16, ng = K / kGroup;
   auto load16 = [&](int u, float (&v)[16]) {
     if constexpr (BF16) {
@@ -126,56 +129,49 @@ __global__ void __launch_bounds__(kPfDigitThreads) pf_digitize_kernel(const void
       }
     }
   };
-  uint32_t mx = 0;
-  for (int u = tid; u < units; u += kPfDigitThreads) {
-    float v[16];
-    load16(u, v);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) mx = max(mx, __float_as_uint(fabsf(v[i])));
-  }
-  mx = __reduce_max_sync(0xffffffffu, mx);
-  if (lane == 0) red[warp] = mx;
-  __syncthreads();
-  mx = 0;
-#pragma unroll
-  for (int w = 0; w < kPfDigitThreads / 32; ++w) mx = max(mx, red[w]);
-  const float m = __uint_as_float(mx);
-  int p = 0;
-  if (m > 0.f) {
-    const int e = (int)(mx >> 23);   // biased exponent (0 for a subnormal m)
-    p = 141 - e;                     // m * 2^p in [2^14, 2^15) for a normal m
-    if (p > 126) p = 126;
-    if (m * __uint_as_float((uint32_t)(127 + p) << 23) > 32639.f) --p;
-  }
-  const float sc = __uint_as_float((uint32_t)(127 + p) << 23);
-  if (tid == 0) rs[row] = __uint_as_float((uint32_t)(127 - p) << 23);
   for (int base = 0; base < units; base += kPfDigitThreads) {   // uniform trips: the quads shuffle below
     const int u = base + tid;
-    const bool live = u < units;   // units is a multiple of 8, so a quad is live or idle as a whole
+    const bool live = u < units;   // units is a multiple of 4, so a quad is live or idle as a whole
     float v[16];
     if (live) load16(u, v);
     else {
 #pragma unroll
       for (int c = 0; c < 16; ++c) v[c] = 0.f;
     }
-    uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};   // high digits [m][h], then low digits [m][h]
+    uint32_t mx = 0;
     float s = 0.f;
 #pragma unroll
+    for (int c = 0; c < 16; ++c) { mx = max(mx, __float_as_uint(fabsf(v[c]))); s += v[c]; }
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    s += __shfl_xor_sync(0xffffffffu, s, 2);
+    const float m = __uint_as_float(mx);
+    int p = 0;
+    if (m > 0.f) {
+      const int e = (int)(mx >> 23);   // biased exponent (0 for a subnormal m)
+      p = 141 - e;                     // m * 2^p in [2^14, 2^15) for a normal m
+      if (p > 126) p = 126;
+      if (m * __uint_as_float((uint32_t)(127 + p) << 23) > 32639.f) --p;
+    }
+    const float sc = __uint_as_float((uint32_t)(127 + p) << 23);
+    uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};   // high digits [m][h], then low digits [m][h]
+#pragma unroll
     for (int c = 0; c < 16; ++c) {
-      s += v[c];
       const int q = __float2int_rn(v[c] * sc);
       const int d1 = (q + 128) >> 8, d0 = q - (d1 << 8);
       const int slot = pf_digit_slot<BITS>(c);
       w[slot >> 2] |= (uint32_t)(d1 & 0xFF) << (8 * (slot & 3));
       w[4 + (slot >> 2)] |= (uint32_t)(d0 & 0xFF) << (8 * (slot & 3));
     }
-    s += __shfl_xor_sync(0xffffffffu, s, 1);
-    s += __shfl_xor_sync(0xffffffffu, s, 2);
     if (live) {
       uint4* o = (uint4*)(dig + (size_t)row * 2 * K + (size_t)(u >> 2) * 128 + (u & 3) * 32);
       o[0] = make_uint4(w[0], w[1], w[2], w[3]);
       o[1] = make_uint4(w[4], w[5], w[6], w[7]);
-      if ((u & 3) == 0) X[(size_t)row * ng + (u >> 2)] = s;
+      if ((u & 3) == 0) {
+        X[(size_t)row * ng + (u >> 2)] = s;
+        rs[(size_t)row * ng + (u >> 2)] = __uint_as_float((uint32_t)(127 - p) << 23);
+      }
     }
   }
 }
@@ -316,7 +312,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_grouped_kernel(PrefillP
   const float* rst = GU ? p.xrs : p.ars;
   const bool vec_sb = (mg == GPW) && (ng % GPW == 0);   // the warp's scales in one load per row
   uint4 bq[TILES][GPW];
-  float xg[TILES][GPW], rsc[TILES];
+  float xg[TILES][GPW], rsg[TILES][GPW];
   int cur = -1, n = 0, orow = -1;
   int ci = ci0, rb = rb0, st = 0;
   unsigned phase = 0;
@@ -336,8 +332,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_grouped_kernel(PrefillP
           bq[tau][gi] = (rB >= 0 && gi < mg) ? __ldg((const uint4*)(db + (size_t)(g0 + gi) * 128))
                                              : make_uint4(0u, 0u, 0u, 0u);
           xg[tau][gi] = (rC >= 0 && gi < mg) ? __ldg(Xt + (size_t)rC * ng + g0 + gi) : 0.f;
+          rsg[tau][gi] = (rC >= 0 && gi < mg) ? __ldg(rst + (size_t)rC * ng + g0 + gi) : 0.f;
         }
-        rsc[tau] = rC >= 0 ? __ldg(rst + rC) : 0.f;
       }
       if (warp == 0 && lane < C) orow = lane < n ? pf_out_row(p, ch, lane) : -1;
     }
@@ -413,8 +409,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_grouped_kernel(PrefillP
           mma_u8s8(c, A[0][0], A[0][1], A[0][2], A[0][3], b.x, b.y);
           mma_u8s8(c, A[1][0], A[1][1], A[1][2], A[1][3], b.z, b.w);
           // columns 2t, 2t+1 of the tile: token t's high- and low-digit sums
-          sacc[tau][0] = fmaf(sA[gi], (float)(c[0] * 256 + c[1]), sacc[tau][0]);
-          sacc[tau][1] = fmaf(sB[gi], (float)(c[2] * 256 + c[3]), sacc[tau][1]);
+          sacc[tau][0] = fmaf(sA[gi] * rsg[tau][gi], (float)(c[0] * 256 + c[1]), sacc[tau][0]);
+          sacc[tau][1] = fmaf(sB[gi] * rsg[tau][gi], (float)(c[2] * 256 + c[3]), sacc[tau][1]);
           bacc[tau][0] = fmaf(bA[gi], xg[tau][gi], bacc[tau][0]);
           bacc[tau][1] = fmaf(bB[gi], xg[tau][gi], bacc[tau][1]);
         }
@@ -426,8 +422,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_grouped_kernel(PrefillP
       }
 #pragma unroll
       for (int tau = 0; tau < TILES; ++tau) {
-        pw[crA * C + 4 * tau + t] = fmaf(sacc[tau][0], rsc[tau], bacc[tau][0]);
-        pw[crB * C + 4 * tau + t] = fmaf(sacc[tau][1], rsc[tau], bacc[tau][1]);
+        pw[crA * C + 4 * tau + t] = sacc[tau][0] + bacc[tau][0];
+        pw[crB * C + 4 * tau + t] = sacc[tau][1] + bacc[tau][1];
       }
     }
     if (tid == 0 && i + nst < nloc) pf_expect(&full[st], item_bytes);   // its phase for item i is complete
@@ -471,17 +467,17 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_grouped_kernel(PrefillP
 }
 
 // ------------------------------------------------------------------ router of many tokens
-// Router logits of many tokens (prefill): a tiled GEMM in fp64. Every
-// product of two bf16 values is exact in fp64, and each logit is accumulated
-// over k in index order from 0 by one thread, then the bias is added: the
-// same sequence of roundings as the plain fp64 loop of the definition
-// (logits l = W_r x + b, "Model architecture" of the Flash-MoE write-up), so
-// the logits are reproduced exactly. That order makes each logit a chain of
-// H dependent fp64 FMAs, so the kernel's time is about H times the FMA
-// latency once every chain is in flight (2 x 4 per thread here). Tile: 32
-// tokens x 32 router rows per CTA; thread (ty, tx) holds tokens 2ty, 2ty+1
-// and rows 4tx..4tx+3; operands are staged in shared memory as doubles,
-// k-major.
+// Router logits of many tokens (prefill): a tiled GEMM in fp64, split over
+// kRgSplit slices of H (blockIdx.z). Every product of two bf16 values is exact
+// in fp64; each CTA sums its slice in k order per logit and writes the
+// partial sum to lpart[slice][token][row]. CTAs of token tile 0 also write
+// the partial sums of the squared router weights of their rows, and CTAs of
+// row tile 0 those of the squared activations of their tokens: the norms
+// that bound each logit's rounding (route_combine_kernel). Tile: 32 tokens x
+// 32 router rows per CTA; thread (ty, tx) holds tokens 2ty, 2ty+1 and rows
+// 4tx..4tx+3; operands are staged in shared memory as doubles, k-major. A
+// slice is a chain of H / kRgSplit dependent fp64 FMAs per logit, and the
+// split gives the GPU kRgSplit times the independent chains.
 constexpr int kRgTok = 32, kRgRows = 32, kRgK = 32, kRgThreads = 128;
 
 // bf16 bit pattern -> double, exactly: normal values and zeros by moving the
@@ -498,9 +494,11 @@ __global__ void __launch_bounds__(kRgThreads) route_gemm_kernel(RouteParams p) {
   __shared__ __align__(16) double xs[kRgK][kRgTok];    // [k][token]
   __shared__ __align__(16) double ws[kRgK][kRgRows];   // [k][row pair b/2][tx][b%2]
   const int tid = threadIdx.x, tx = tid & 7, ty = tid >> 3;
-  const int e0 = blockIdx.x * kRgRows, t0 = blockIdx.y * kRgTok;
+  const int e0 = blockIdx.x * kRgRows, t0 = blockIdx.y * kRgTok, ks = blockIdx.z;
   const int nrows = p.E + (p.has_shared ? 1 : 0);
-  double acc[2][4];
+  const int kbeg = (int)((long long)p.H * ks / kRgSplit) & ~(kRgK - 1);
+  const int kend = ks + 1 == kRgSplit ? p.H : (int)((long long)p.H * (ks + 1) / kRgSplit) & ~(kRgK - 1);
+  double acc[2][4], xn[2] = {0.0, 0.0}, wn[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll
   for (int a = 0; a < 2; ++a)
 #pragma unroll
@@ -515,9 +513,10 @@ __global__ void __launch_bounds__(kRgThreads) route_gemm_kernel(RouteParams p) {
     xv = xrow ? __ldg((const uint4*)(xrow + k0 + 8 * lc)) : make_uint4(0u, 0u, 0u, 0u);
     wv = wrow ? __ldg((const uint4*)(wrow + k0 + 8 * lc)) : make_uint4(0u, 0u, 0u, 0u);
   };
+  const bool do_xn = blockIdx.x == 0 && tx == 0, do_wn = blockIdx.y == 0 && ty == 0;
   uint4 xv, wv;
-  load(0, xv, wv);
-  for (int k0 = 0; k0 < p.H; k0 += kRgK) {
+  if (kbeg < kend) load(kbeg, xv, wv);
+  for (int k0 = kbeg; k0 < kend; k0 += kRgK) {
     __syncthreads();   // the previous tile has been read
     {
       const uint32_t u[4] = {xv.x, xv.y, xv.z, xv.w}, v[4] = {wv.x, wv.y, wv.z, wv.w};
@@ -530,7 +529,7 @@ __global__ void __launch_bounds__(kRgThreads) route_gemm_kernel(RouteParams p) {
       }
     }
     __syncthreads();
-    if (k0 + kRgK < p.H) load(k0 + kRgK, xv, wv);   // next tile in flight during the products
+    if (k0 + kRgK < kend) load(k0 + kRgK, xv, wv);   // next tile in flight during the products
 #pragma unroll 8
     for (int kk = 0; kk < kRgK; ++kk) {
       const double2 xa = *(const double2*)&xs[kk][2 * ty];
@@ -542,8 +541,14 @@ __global__ void __launch_bounds__(kRgThreads) route_gemm_kernel(RouteParams p) {
         acc[0][b] = fma(w4[b], xa.x, acc[0][b]);
         acc[1][b] = fma(w4[b], xa.y, acc[1][b]);
       }
+      if (do_xn) { xn[0] = fma(xa.x, xa.x, xn[0]); xn[1] = fma(xa.y, xa.y, xn[1]); }
+      if (do_wn) {
+#pragma unroll
+        for (int b = 0; b < 4; ++b) wn[b] = fma(w4[b], w4[b], wn[b]);
+      }
     }
   }
+  const size_t ld = (size_t)p.E + 1;
 #pragma unroll
   for (int a = 0; a < 2; ++a) {
     const int t = t0 + 2 * ty + a;
@@ -551,10 +556,47 @@ __global__ void __launch_bounds__(kRgThreads) route_gemm_kernel(RouteParams p) {
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
       const int e = e0 + 4 * tx + b;
-      if (e >= nrows) continue;
-      double v = acc[a][b];
-      if (e < p.E && p.router_bias) v += (double)p.router_bias[e];
-      p.logits[(size_t)t * (p.E + 1) + e] = v;
+      if (e < nrows) p.lpart[((size_t)ks * p.T + t) * ld + e] = acc[a][b];
+    }
+    if (do_xn) p.xn2[(size_t)ks * p.T + t] = xn[a];
+  }
+  if (do_wn)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int e = e0 + 4 * tx + b;
+      if (e < nrows) p.wn2[(size_t)ks * ld + e] = wn[b];
+    }
+}
+
+// Logits of many tokens from the router GEMM's slices: l = sum of the
+// slices' partial sums in slice order + bias (fp64), written to
+// logits[t][e], and a certified bound on |l - definition| to bound[t][e].
+// Every product is exact and every sum a tree of fp64 additions, so with
+// u = 2^-53 both l and the index-order definition are within
+// (H + 1) u / (1 - (H + 1) u) sum |w x| of the exact value, and
+// sum |w x| <= ||w_e|| ||x_t|| (Cauchy-Schwarz). The squared norms are fp64
+// sums of exact squares (relative error below (H + 1) u); the factor 1.25 and
+// the term 2^-50 (|l| + |b|) cover the roundings of the norms, of the bias
+// additions and of the bound itself. Grid T, block 512.
+__global__ void __launch_bounds__(kThreads) route_combine_kernel(RouteParams p) {
+  const int t = blockIdx.x;
+  const size_t ld = (size_t)p.E + 1;
+  double xn = 0.0;
+  for (int q = 0; q < kRgSplit; ++q) xn += p.xn2[(size_t)q * p.T + t];
+  const int nrows = p.E + (p.has_shared ? 1 : 0);
+  for (int e = threadIdx.x; e < nrows; e += blockDim.x) {
+    double l = 0.0, wn = 0.0;
+    for (int q = 0; q < kRgSplit; ++q) {
+      l += p.lpart[((size_t)q * p.T + t) * ld + e];
+      wn += p.wn2[(size_t)q * ld + e];
+    }
+    const double bias = (e < p.E && p.router_bias) ? (double)p.router_bias[e] : 0.0;
+    l += bias;
+    p.logits[(size_t)t * ld + e] = l;
+    if (e < p.E) {
+      const double nn = (double)p.H;
+      const double b = 1.25 * 2.0 * (nn + 2.0) * 0x1p-53 * sqrt(wn * xn) + 0x1p-50 * (fabs(l) + fabs(bias));
+      p.bound[(size_t)t * ld + e] = __double2float_ru(b);
     }
   }
 }
@@ -675,10 +717,12 @@ cudaError_t launch_group(const GroupParams& p, cudaStream_t s) {
 
 cudaError_t launch_route_gemm(const RouteParams& p, cudaStream_t s) {
   const int rows = p.E + (p.has_shared ? 1 : 0);
-  dim3 grid((rows + kRgRows - 1) / kRgRows, (p.T + kRgTok - 1) / kRgTok);
+  dim3 grid((rows + kRgRows - 1) / kRgRows, (p.T + kRgTok - 1) / kRgTok, kRgSplit);
   RouteParams q = p;
   void* args[] = {&q};
-  return cudaLaunchKernel((const void*)route_gemm_kernel, grid, dim3(kRgThreads), args, 0, s);
+  cudaError_t e = cudaLaunchKernel((const void*)route_gemm_kernel, grid, dim3(kRgThreads), args, 0, s);
+  if (e != cudaSuccess) return e;
+  return cudaLaunchKernel((const void*)route_combine_kernel, dim3(p.T), dim3(kThreads), args, 0, s);
 }
 
 int pf_chunk_tokens(int H, int I) { return (H > 4096 || I > 4096) ? 4 : 8; }

@@ -12,9 +12,9 @@ So the ids must equal the oracle's bit for bit:
     element that meets a tiny activation (fp64 logits 2^-44 apart), and an
     exact tie. These must take the exact recheck, which the workspace header
     counts.
-The same ids and layer outputs are checked through the fused single-kernel
-layer (T = 1) and the four-kernel chain (T = 2..8), and both paths run at the
-largest shape they accept.
+The same ids and layer outputs are checked through the decode layer (the
+four-kernel chain, or the fused kernel when MOE_DECODE_KERNEL=fused) and the
+prefill path, and the decode paths run at the largest shapes they accept.
 """
 import os
 
@@ -146,7 +146,7 @@ def test_near_ties_route_like_the_definition(dev):
     assert ridx.tolist() == [[10, 20, 31]]
     gamma = np.zeros(NT.H, dtype=np.uint16)
     layer = _router_layer(Wr, None, None, gamma, NT.H, NT.k, dev)
-    for T in (1, 3):
+    for T in (1, 3, 12):   # the decode router (T <= 8) and the many-token router GEMM
         xs = np.repeat(x, T, axis=0)
         ws = qm.new_workspace(layer, T)
         idx = torch.empty((T, NT.k), dtype=torch.int32, device=dev)
@@ -157,11 +157,12 @@ def test_near_ties_route_like_the_definition(dev):
         assert _rechecks(ws) == T, "the near tie must be decided by the exact recheck"
 
 
-@pytest.mark.parametrize("T", [1, 2])
+@pytest.mark.parametrize("T", [1, 2, 9])
 def test_near_ties_through_the_layer(dev, T):
-    """The same near ties through moe_layer_forward: T = 1 runs the fused
-    kernel, T = 2 the four-kernel chain; ids, weights and outputs against the
-    oracle's layer with the same router."""
+    """The same near ties through moe_layer_forward: T = 1 and 2 take the
+    decode kernels (T = 1 the fused kernel when MOE_DECODE_KERNEL=fused),
+    T = 9 the prefill path; ids, weights and outputs against the oracle's
+    layer with the same router."""
     Wr, x1 = _near_tie_router(2)
     t = fxg.device_layer(NT, 0)
     t["router_w"] = torch.from_numpy(Wr.view(np.int16)).to(dev)
@@ -192,7 +193,7 @@ def test_near_ties_through_the_layer(dev, T):
 
 def test_fused_layer_routes_many_biased_tokens_like_the_oracle(dev):
     """256 single-token calls of the full 512-expert layer with the per-expert
-    router bias (the fused kernel); ids bit-exact against the oracle."""
+    router bias; ids bit-exact against the oracle."""
     cfg = fixtures.CONFIGS["stack_q4"]
     t = fxg.device_layer(cfg, 0)
     layer = qm.layer_from_tensors(cfg, t)
@@ -248,7 +249,8 @@ def _layer_vs_oracle(cfg, T, dev, calls=2):
 @pytest.mark.parametrize("bits", [4, 2])
 def test_fused_layer_at_its_largest_shape(dev, bits):
     """hidden 4096 and intermediate 1152 = 8 rows x 148 SMs (rounded to a span):
-    the largest shape whose per-SM gate/up and down rows fit the fused kernel."""
+    the largest shape whose per-SM gate/up and down rows fit the fused kernel
+    (which runs it when MOE_DECODE_KERNEL=fused; the chain otherwise)."""
     cfg = fixtures.Config("fused_max", H=4096, E=16, k=3, I=1152, bits=bits,
                           scale_sigma=0.02 if bits == 4 else 0.05)
     _layer_vs_oracle(cfg, 1, dev)
@@ -267,7 +269,7 @@ def test_chain_at_its_largest_shape(dev):
 def test_odd_span_counts(dev, bits):
     """hidden 3968 (31 spans of 128) and intermediate 896 (7 spans): warps
     whose share of the spans starts on an odd span, and span pairs that cross
-    a 16-byte chunk of scale words; T = 1 (fused) and T = 2 (chain)."""
+    a 16-byte chunk of scale words; T = 1 and T = 2."""
     cfg = fixtures.Config("odd_spans", H=3968, E=12, k=3, I=896, bits=bits,
                           scale_sigma=0.02 if bits == 4 else 0.05)
     _layer_vs_oracle(cfg, 1, dev, calls=1)

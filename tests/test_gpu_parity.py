@@ -135,12 +135,14 @@ def test_route_matches_oracle(dev, name):
     np.testing.assert_allclose(sg.cpu().numpy(), rsg, rtol=1e-6, atol=1e-7)
 
 
-def test_route_logits_equal_fp64_definition(dev):
-    """Many tokens (T > 8): every logit equals the plain fp64 loop of the
-    definition bit for bit (bf16 products are exact in fp64; each logit is
-    accumulated in index order and the bias added last). moe_route leaves the
-    logits in the workspace: double [T][E+1] at byte 256, column E the
-    shared-gate logit."""
+def test_route_logits_within_their_bound_of_the_fp64_definition(dev):
+    """Many tokens (T > 8): the router GEMM sums four slices of H in fp64, so
+    a logit may differ from the plain index-order fp64 loop of the definition
+    in its last bits; every logit must lie within the certified bound the
+    library stores beside it (2 (H+2) 2^-53 ||w|| ||x|| + 2^-50 (|l| + |b|),
+    with a margin), and the ranking must be the definition's. moe_route leaves
+    the logits in the workspace: double [T][E+1] at byte 256, column E the
+    shared-gate logit; the bounds follow as float [T][E+1]."""
     cfg = fixtures.CONFIGS["stack_q4"]   # the biased router
     Wr, rb, gs, gamma = fixtures.layer_vectors(cfg, 0)
     dummy = torch.zeros(64, dtype=torch.int32, device=dev)
@@ -158,10 +160,16 @@ def test_route_logits_equal_fp64_definition(dev):
     qm.moe_route(layer, torch.from_numpy(x.view(np.int16)).to(dev), idx, w, ws=ws)
     torch.cuda.synchronize()
     got = ws[256:256 + 8 * T * (cfg.E + 1)].cpu().numpy().view(np.float64).reshape(T, cfg.E + 1)
-    _, _, _, ref = oracle.route(x, Wr, cfg.k, bias=rb, want_logits=True)
-    np.testing.assert_array_equal(got[:, :cfg.E], ref)
+    off = 256 + ((8 * T * (cfg.E + 1) + 255) // 256) * 256
+    bnd = ws[off:off + 4 * T * (cfg.E + 1)].cpu().numpy().view(np.float32).reshape(T, cfg.E + 1)[:, :cfg.E]
+    ridx, _, _, ref = oracle.route(x, Wr, cfg.k, bias=rb, want_logits=True)
+    err = np.abs(got[:, :cfg.E] - ref)
+    assert np.all(err <= bnd.astype(np.float64))
+    assert np.all(bnd < 1e-9)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ridx)
     _, _, _, ref_g = oracle.route(x, gs[None, :], 1, want_logits=True)
-    np.testing.assert_array_equal(got[:, cfg.E], ref_g[:, 0])
+    assert np.max(np.abs(got[:, cfg.E] - ref_g[:, 0])) <= 1e-9
+    print(f"many-token router: largest |l - definition| {err.max():.2e}, largest bound {bnd.max():.2e}")
 
 
 @pytest.mark.parametrize("E,k", [(512, 8), (4096, 8), (4096, 3), (100, 5)])
