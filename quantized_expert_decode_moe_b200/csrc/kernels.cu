@@ -43,8 +43,8 @@ WsLayout ws_layout(int H, int I, int E, int k, int S, int T) {
   L.nchunks = o; o = align256(o + (T > 8 ? sizeof(int32_t) : 0));
   L.y = o; o = align256(o + sizeof(float) * prows * H);
   L.lpart = o; o = align256(o + (T > 8 ? sizeof(double) * kRgSplit * (size_t)T * (E + 1) : 0));
-  L.xn2 = o; o = align256(o + (T > 8 ? sizeof(double) * kRgSplit * (size_t)T : 0));
-  L.wn2 = o; o = align256(o + (T > 8 ? sizeof(double) * kRgSplit * (size_t)(E + 1) : 0));
+  L.xn2 = o; o = align256(o + (T > 8 ? sizeof(double) * (size_t)T : 0));
+  L.wn2 = o; o = align256(o + (T > 8 ? sizeof(double) * (size_t)(E + 1) : 0));
   L.total = o;
   return L;
 }

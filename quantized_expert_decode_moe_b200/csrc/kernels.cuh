@@ -38,7 +38,7 @@ struct WsLayout {
   size_t nchunks;     // int32
   size_t y;           // float [T*k + T][H] expert outputs, same rows
   size_t lpart;       // double [kRgSplit][T][E+1] partial router logits (T > 8)
-  size_t xn2, wn2;    // double [kRgSplit][T], [kRgSplit][E+1] partial squared norms (T > 8)
+  size_t xn2, wn2;    // double [T], [E+1] squared norms of x and of the router rows (T > 8)
   size_t total;
 };
 WsLayout ws_layout(int H, int I, int E, int k, int S, int T);
@@ -51,8 +51,8 @@ struct RouteParams {
   const uint16_t* gate_w;       // [H] or null
   double* logits;               // [T][E+1]
   float* bound;                 // [T][E+1]: bound on |logit - fp64 definition| (null: not written)
-  // many tokens: per-slice partial logits [kRgSplit][T][E+1], squared norms of x [kRgSplit][T] and of the
-  // router rows [kRgSplit][E+1]
+  // many tokens: per-slice partial logits [kRgSplit][T][E+1], squared norms of x [T] and of the
+  // router rows [E+1]
   double* lpart; double* xn2; double* wn2;
   // side job of the decode chain (null when unused): copies of the layer's inputs x, h ([T][H])
   const float* h; uint16_t* x_rec; float* h_rec;

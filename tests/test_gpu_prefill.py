@@ -121,16 +121,18 @@ def test_prefill_full_size_512_tokens(dev):
     torch.cuda.empty_cache()
 
 
+@pytest.mark.parametrize("where", ["x", "a"])
 @pytest.mark.parametrize("name,T", [("tiny", 40), ("layer_q4", 16)])
-def test_prefill_outlier_activations(dev, name, T):
-    """Activations as real models have them: every token carries one element
-    2^10 times the rest (in x), and one intermediate row of the shared expert
-    has its up-projection scales raised by 2^10, so the SwiGLU output a holds
-    one value ~2^10 above the others in every token. The prefill path writes
-    activations as 16-bit fixed point with one exponent per 64-value group,
-    so an outlier costs only its own group bits. The experts' contribution
-    h' - h must match the oracle's within the normwise bar; the routing
-    bit for bit."""
+def test_prefill_outlier_activations(dev, name, T, where):
+    """Activations as real models have them, one outlier per row: "x": every
+    token's input carries one element 2^10 times the rest; "a": one
+    intermediate row of the shared expert has its up-projection scales raised
+    by 2^10, so every token's SwiGLU output a holds one value ~2^10 above the
+    others. The prefill path writes activations as 16-bit fixed point with one
+    exponent per 64-value group (each value within 2^-15 of its group's
+    maximum), so an outlier costs only its own group bits. The experts'
+    contribution h' - h must match the oracle's within the normwise bar; the
+    routing bit for bit."""
     cfg = fixtures.CONFIGS[name]
     n = None if name == "tiny" else 32
     c = cfg if n is None else fixtures.Config(cfg.name, H=cfg.H, E=n, k=cfg.k, I=cfg.I, bits=cfg.bits,
@@ -138,23 +140,26 @@ def test_prefill_outlier_activations(dev, name, T):
     t = fxg.device_layer(c, 0, n_experts=n)
     rng = np.random.default_rng(11)
     jstar = int(rng.integers(0, c.I))
-    up_s = t["s"][1][c.E]                      # shared expert (stored at index E), up scales [I][H/64]
-    boosted = up_s[jstar].cpu().numpy().view(np.uint16).astype(np.uint32) + (10 << 7)   # bf16 exponent + 10
-    up_s[jstar] = torch.from_numpy(boosted.astype(np.uint16).view(np.int16)).to(dev)
+    if where == "a":
+        up_s = t["s"][1][c.E]                      # shared expert (stored at index E), up scales [I][H/64]
+        boosted = up_s[jstar].cpu().numpy().view(np.uint16).astype(np.uint32) + (10 << 7)   # bf16 exponent + 10
+        up_s[jstar] = torch.from_numpy(boosted.astype(np.uint16).view(np.int16)).to(dev)
     layer = qm.layer_from_tensors(c, t)
     x = gen.x_tokens(c, 23, T=T)
-    xf = gen.bf16_bits_to_f32(x)
-    for i in range(T):
-        j = int(rng.integers(0, c.H))
-        xf[i, j] = np.float32(1024.0) * np.sign(xf[i, j] if xf[i, j] != 0 else 1.0) * max(abs(xf[i]).max(), 1.0)
-    x = gen.f32_to_bf16_bits(xf.astype(np.float32))
+    if where == "x":
+        xf = gen.bf16_bits_to_f32(x)
+        for i in range(T):
+            j = int(rng.integers(0, c.H))
+            xf[i, j] = np.float32(1024.0) * np.sign(xf[i, j] if xf[i, j] != 0 else 1.0) * max(abs(xf[i]).max(), 1.0)
+        x = gen.f32_to_bf16_bits(xf.astype(np.float32))
     h0, idx, w, h, xfo, xo = _run(c, layer, x, dev)
     Wr, rb, gs, gamma = fixtures.layer_vectors(c, 0)
     experts = [fixtures.host_expert(c, 0, e) for e in range(c.E)]
     shared = [list(m) for m in fixtures.host_expert(c, 0, c.E)]
-    s_up = shared[1][1].copy()
-    s_up[jstar] = (s_up[jstar].astype(np.uint32) + (10 << 7)).astype(np.uint16)
-    shared[1][1] = s_up
+    if where == "a":
+        s_up = shared[1][1].copy()
+        s_up[jstar] = (s_up[jstar].astype(np.uint32) + (10 << 7)).astype(np.uint16)
+        shared[1][1] = s_up
     sample = list(range(0, T, max(1, T // 8)))
     ref = oracle.layer(x[sample], h0[sample].astype(np.float64), Wr, gamma, experts, [tuple(m) for m in shared],
                        I=c.I, k=c.k, G=c.G, bits=c.bits, eps=c.rms_eps, gs=gs, router_bias=rb)
@@ -166,4 +171,4 @@ def test_prefill_outlier_activations(dev, name, T):
         e = float(np.max(np.abs(d_gpu - d_ref)) / np.max(np.abs(d_ref)))
         assert e <= TOL, (i, e)
         worst = max(worst, e)
-    print(f"{name} outliers: max rel err of the experts' contribution {worst:.3e}")
+    print(f"{name} outlier in {where}: max rel err of the experts' contribution {worst:.3e}")
