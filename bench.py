@@ -574,6 +574,8 @@ def ours_prefill(args, cfg):
     f1.synchronize()
     e2e_ms = f0.elapsed_time(f1)
     peaks, peak_kind = measured_peaks()
+    shared_tc = cfg.T >= 64 and os.environ.get("MOE_PREFILL_SHARED", "") != "mma" or \
+        os.environ.get("MOE_PREFILL_SHARED", "") == "tc"
     touched = [len(np.unique(idx[b].cpu().numpy())) for b in range(NB)]
     bytes_mat = cfg.I * cfg.H * cfg.bits // 8 + 2 * 2 * cfg.I * (cfg.H // cfg.G)   # one matrix: codes, scales, biases
     gu_bytes = (np.mean(touched) + 1) * 2 * bytes_mat + 2 * T * cfg.H * 2
@@ -583,7 +585,10 @@ def ours_prefill(args, cfg):
         "metric": "MoE-layer prefill tokens/s (512-token batch), 4-bit experts, 1 B200", "value": T * steps / (ms * 1e-3),
         "unit": "tokens/s", "n_gpus": world, "steps": steps, "warmup": max(args.warmup, 3),
         "ms_per_step": ms / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "u4 codes x s8 digits of 16-bit fixed-point activations on int8 tensor cores (s32), "
+        "dtype": "routed experts: u4 codes x s8 digits of 16-bit fixed-point activations on int8 tensor cores "
+                 "(s32), fp32 scale+accumulate; shared expert: exact fp16 s*(q-8) x fp16 activations on tcgen05 "
+                 "(fp32 accumulate in tensor memory); router logits f64" if shared_tc else
+                 "u4 codes x s8 digits of 16-bit fixed-point activations on int8 tensor cores (s32), "
                  "fp32 scale+accumulate; router logits f64",
         "data": "synthetic (seeded; no model weights)",
         "config": {"workload": cfg.note, "H": cfg.H, "E": cfg.E, "top_k": cfg.k, "I": cfg.I, "bits": cfg.bits,
@@ -597,8 +602,9 @@ def ours_prefill(args, cfg):
                      "algorithmic_bytes": gu_bytes, "peak_kind": peak_kind},
         "e2e": {"value": T * e2e_n / (e2e_ms * 1e-3), "unit": "tokens/s", "steps": e2e_n,
                 "h2d_bytes_per_step": T * cfg.H * (2 + 4), "d2h_bytes_per_step": T * cfg.H * 2},
-        # route, top-k, grouping, digits of x, gate/up, digits of a, down, combine + norm
-        "gpu_launches": 8 * steps, "clocks": clk,
+        # router (GEMM, norms, combine), top-k, grouping, digits of x, gate/up, digits of a, down,
+        # combine + norm; with the shared expert on tcgen05 also its tables of x, gate/up, tables of a, down
+        "gpu_launches": (14 if shared_tc else 10) * steps, "clocks": clk,
     }
     if rank == 0 and not args.no_cpu_baseline:
         rate, n, threads, el = oracle_sample(cfg, args.cpu_seconds)

@@ -94,6 +94,18 @@ Path path_of(const moe_layer* L, int T) {
   return Path::kNone;
 }
 
+// Prefill (T > 8): the shared expert runs as dense GEMMs on the tcgen05 tensor
+// cores (shared_tc.cu) from 64 tokens up, on the grouped integer kernels below
+// that. MOE_PREFILL_SHARED=tc or =mma in the environment (read at every call)
+// forces one of them for every prefill call.
+bool shared_on_tc(const moe_layer* L, int T) {
+  if (!L->has_shared || T <= kDecodeMaxT || !tc_supported(L->hidden, L->inter, L->bits)) return false;
+  const char* e = getenv("MOE_PREFILL_SHARED");
+  if (e && strcmp(e, "tc") == 0) return true;
+  if (e && strcmp(e, "mma") == 0) return false;
+  return T >= 64;
+}
+
 WsLayout layout_of(const moe_layer* L, int T) {
   return ws_layout(L->hidden, L->inter, L->n_experts, L->top_k, slots_of(L), T);
 }
@@ -227,14 +239,15 @@ moe_status prefill_chain(const moe_layer* L, const uint16_t* x_in, float* h, int
     return MOE_ERR_CUDA;
   if (topk_w && cudaMemcpyAsync(topk_w, tp.w, sizeof(float) * (size_t)T * k, cudaMemcpyDeviceToDevice, s))
     return MOE_ERR_CUDA;
+  const bool tc = shared_on_tc(L, T);
   GroupParams gp{};
-  gp.T = T; gp.k = k; gp.E = E; gp.has_shared = L->has_shared; gp.chunk = pf_chunk_tokens(H, I); gp.idx = tp.idx;
+  gp.T = T; gp.k = k; gp.E = E; gp.has_shared = L->has_shared && !tc; gp.chunk = pf_chunk_tokens(H, I); gp.idx = tp.idx;
   gp.counts = at<int32_t>(ws, W.counts); gp.offsets = at<int32_t>(ws, W.offsets); gp.perm = at<int32_t>(ws, W.perm);
   gp.chunks = at<int4>(ws, W.chunks); gp.nchunks = at<int32_t>(ws, W.nchunks);
   if ((e = launch_group(gp, s)) != cudaSuccess) return MOE_ERR_CUDA;
   mark(2);
   PrefillParams pp{};
-  pp.H = H; pp.I = I; pp.E = E; pp.k = k; pp.T = T; pp.has_shared = L->has_shared;
+  pp.H = H; pp.I = I; pp.E = E; pp.k = k; pp.T = T; pp.has_shared = L->has_shared && !tc;
   pp.x = x_in;
   pp.xd = at<unsigned char>(ws, W.xd); pp.xX = at<float>(ws, W.xX); pp.xrs = at<float>(ws, W.xrs);
   pp.a = at<float>(ws, W.a);
@@ -243,9 +256,35 @@ moe_status prefill_chain(const moe_layer* L, const uint16_t* x_in, float* h, int
   pp.chunks = gp.chunks; pp.nchunks = gp.nchunks; pp.perm = gp.perm;
   pp.experts = L->experts; pp.shared = L->shared;
   pp.status = status; pp.wait_ns = wait_bound_ns();
+  // shared expert on the tensor cores: operand tables of x, gate/up partial sums
+  const int Tpad = (T + 15) & ~15;
+  TcConvParams cx{};
+  TcParams tg{};
+  if (tc) {
+    cx.K = H; cx.T = T; cx.Tpad = Tpad; cx.bits = L->bits; cx.x = x_in;
+    cx.b_hi = at<__half>(ws, W.tcbx); cx.tscale = at<float>(ws, W.tcxs);
+    if ((e = launch_tc_conv(cx, s)) != cudaSuccess) return MOE_ERR_CUDA;
+    tg.M = 2 * I; tg.K = H; tg.R0 = I; tg.bits = L->bits; tg.w0 = L->shared.gate; tg.w1 = L->shared.up;
+    tg.T = T; tg.Tpad = Tpad; tg.hilo = 0; tg.b_hi = cx.b_hi; tg.tscale = cx.tscale;
+    tg.part = at<float>(ws, W.tcpart); tg.status = status; tg.wait_ns = pp.wait_ns;
+    if ((e = launch_tc_dense(tg, s)) != cudaSuccess)
+      return e == cudaErrorInvalidConfiguration ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
+  }
   if ((e = launch_prefill_gateup(pp, L->bits, s)) != cudaSuccess)
     return e == cudaErrorInvalidConfiguration ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
   mark(3);
+  if (tc) {   // SwiGLU of the split sums -> hi/lo tables of a, down partial sums
+    TcConvParams ca{};
+    ca.K = I; ca.T = T; ca.Tpad = Tpad; ca.bits = L->bits;
+    ca.part = tg.part; ca.splits = tc_splits(2 * I, T, H); ca.I = I;
+    ca.b_hi = at<__half>(ws, W.tcbah); ca.b_lo = at<__half>(ws, W.tcbal); ca.tscale = at<float>(ws, W.tcas);
+    if ((e = launch_tc_conv(ca, s)) != cudaSuccess) return MOE_ERR_CUDA;
+    TcParams td = tg;
+    td.M = H; td.K = I; td.R0 = H; td.w0 = L->shared.down; td.w1 = L->shared.down;
+    td.hilo = 1; td.b_hi = ca.b_hi; td.b_lo = ca.b_lo; td.tscale = ca.tscale;
+    if ((e = launch_tc_dense(td, s)) != cudaSuccess)
+      return e == cudaErrorInvalidConfiguration ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
+  }
   if ((e = launch_prefill_down(pp, L->bits, s)) != cudaSuccess)
     return e == cudaErrorInvalidConfiguration ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
   mark(4);
@@ -254,6 +293,11 @@ moe_status prefill_chain(const moe_layer* L, const uint16_t* x_in, float* h, int
   np.y_routed = pp.y; np.y_routed_tok_stride = (long long)k * H; np.y_routed_slot_stride = H;
   np.w = tp.w;
   np.y_shared = L->has_shared ? pp.y + (size_t)T * k * H : nullptr; np.y_shared_tok_stride = H;
+  if (tc) {
+    np.y_shared = at<float>(ws, W.tcpart);
+    np.y_shared_splits = tc_splits(H, T, I);
+    np.y_shared_split_stride = (long long)T * H;
+  }
   np.sg = tp.sg;
   np.h = h; np.gamma = L->rms_gamma; np.eps = L->rms_eps; np.x_out = x_out; np.x_out_f32 = x_out_f32;
   if ((e = launch_norm(np, false, s)) != cudaSuccess) return MOE_ERR_CUDA;

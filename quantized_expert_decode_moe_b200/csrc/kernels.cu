@@ -45,6 +45,18 @@ WsLayout ws_layout(int H, int I, int E, int k, int S, int T) {
   L.lpart = o; o = align256(o + (T > 8 ? sizeof(double) * kRgSplit * (size_t)T * (E + 1) : 0));
   L.xn2 = o; o = align256(o + (T > 8 ? sizeof(double) * (size_t)T : 0));
   L.wn2 = o; o = align256(o + (T > 8 ? sizeof(double) * (size_t)(E + 1) : 0));
+  const size_t tpad = T > 8 ? (size_t)((T + 15) & ~15) : 0;
+  L.tcbx = o; o = align256(o + 2 * tpad * tc_cols(H));
+  L.tcxs = o; o = align256(o + sizeof(float) * tpad);
+  L.tcbah = o; o = align256(o + 2 * tpad * tc_cols(I));
+  L.tcbal = o; o = align256(o + 2 * tpad * tc_cols(I));
+  L.tcas = o; o = align256(o + sizeof(float) * tpad);
+  size_t np = 0;
+  if (T > 8) {
+    const size_t gu = (size_t)tc_splits(2 * I, T, H) * 2 * I, dn = (size_t)tc_splits(H, T, I) * H;
+    np = (gu > dn ? gu : dn) * (size_t)T;
+  }
+  L.tcpart = o; o = align256(o + sizeof(float) * np);
   L.total = o;
   return L;
 }
@@ -272,6 +284,7 @@ norm_cluster_kernel(NormParams p) {
   if (tid == 0) wsh[kMaxSlots - 1] = p.y_shared ? ldcg_f32(p.sg + t) : 0.f;
   const float* yr = p.y_routed + (size_t)t * p.y_routed_tok_stride;
   const float* ysh = p.y_shared ? p.y_shared + (size_t)t * p.y_shared_tok_stride : nullptr;
+  const int nsp = p.y_shared_splits > 1 ? p.y_shared_splits : 1;
   float* h = p.h + (size_t)t * p.H;
   float hv[kNormCPer], yv[kNormCPer][kMaxSlots];
 #pragma unroll
@@ -282,7 +295,10 @@ norm_cluster_kernel(NormParams p) {
     hv[u] = in ? h[j] : 0.f;
 #pragma unroll
     for (int i = 0; i < kMaxTopK; ++i) yv[u][i] = (in && i < p.k) ? ldcg_f32(yr + (size_t)i * p.y_routed_slot_stride + j) : 0.f;
-    yv[u][kMaxSlots - 1] = (in && ysh) ? ldcg_f32(ysh + j) : 0.f;
+    float ys = 0.f;
+    if (in && ysh)
+      for (int q = 0; q < nsp; ++q) ys += ldcg_f32(ysh + (size_t)q * p.y_shared_split_stride + j);
+    yv[u][kMaxSlots - 1] = ys;
   }
   __syncthreads();
   float ss = 0.f;

@@ -39,6 +39,9 @@ struct WsLayout {
   size_t y;           // float [T*k + T][H] expert outputs, same rows
   size_t lpart;       // double [kRgSplit][T][E+1] partial router logits (T > 8)
   size_t xn2, wn2;    // double [T], [E+1] squared norms of x and of the router rows (T > 8)
+  // shared expert on the tensor cores (T > 8): fp16 operand tables of x and of its SwiGLU
+  // outputs (hi, lo) [Kx/8][Tpad][8], per-token scales [Tpad], split partial sums
+  size_t tcbx, tcxs, tcbah, tcbal, tcas, tcpart;
   size_t total;
 };
 WsLayout ws_layout(int H, int I, int E, int k, int S, int T);
@@ -109,6 +112,7 @@ struct NormParams {
   int H, k, T;
   const float* y_routed; long long y_routed_tok_stride, y_routed_slot_stride;
   const float* w; const float* y_shared; long long y_shared_tok_stride; const float* sg;
+  int y_shared_splits; long long y_shared_split_stride;   // y_shared = sum of the splits (0 or 1: one)
   float* h; const uint16_t* gamma; float eps;
   uint16_t* x_out; float* x_out_f32;
 };
@@ -151,6 +155,35 @@ struct GroupParams {
   const int32_t* idx;
   int32_t* counts; int32_t* offsets; int32_t* perm;
   int4* chunks; int32_t* nchunks;
+};
+
+// Dense pass of one expert over every token of a batch on the tcgen05 tensor
+// cores (the shared expert in prefill, shared_tc.cu):
+//   part[s][t][m] = sum over the columns of split s of W[m][k] * v_t[k]
+// with W the dequantised (stacked) weight matrix, rows [0, R0) from w0 and
+// [R0, M) from w1, and v_t the token's activations (hi + lo parts when hilo).
+struct TcParams {
+  int M, K, R0, bits;
+  moe_qmat w0, w1;
+  int T, Tpad;                 // tokens, and tokens padded to 16 (rows of the operand tables)
+  int nt;                      // tokens per CTA (multiple of 16, <= 256)
+  int hilo;                    // operand tables carry a lo part (b_lo) beside the hi part
+  const __half* b_hi;          // [Kx/8][Tpad][8] fp16, Kx = K + 64*ceil(K/1024) (tc_cols)
+  const __half* b_lo;          // same, or null
+  const float* tscale;         // [T] 2^-p of each token's table
+  int splits;                  // column splits (gridDim.z)
+  int nst;                     // pipeline stages (set by the launcher)
+  float* part;                 // [splits][T][M]
+  uint32_t* status;
+  unsigned long long wait_ns;
+};
+// Operand tables of a batch's activations for the dense pass (shared_tc.cu).
+struct TcConvParams {
+  int K, T, Tpad, bits;
+  const uint16_t* x;           // bf16 [T][K] (gate/up input) or null
+  const float* part; int splits, I;   // gate/up partial sums [splits][T][2I] (down input) or null
+  __half* b_hi; __half* b_lo;  // [Kx/8][Tpad][8]
+  float* tscale;               // [Tpad]
 };
 
 // One layer of the fused decode kernel (device pointers).
@@ -211,5 +244,12 @@ bool prefill_supported(int H, int I, int bits);
 int pf_chunk_tokens(int H, int I);   // tokens per chunk of the grouped GEMMs
 size_t pf_max_chunks(int T, int k, int E, int chunk);
 int choose_ncta(long long ntiles, int nspans);
+// dense tensor-core pass of the shared expert (prefill)
+// Kx: K data columns plus the bias-term columns (64 per 1024 data columns or part of them)
+__host__ __device__ inline int tc_cols(int K) { return K + 64 * ((K + 1023) / 1024); }
+int tc_splits(int M, int T, int K);                  // column splits of a pass
+bool tc_supported(int H, int I, int bits);
+cudaError_t launch_tc_conv(const TcConvParams& p, cudaStream_t s);
+cudaError_t launch_tc_dense(const TcParams& p, cudaStream_t s);
 
 }  // namespace qmoe

@@ -1,7 +1,9 @@
 """GPU parity of the prefill path (T > 8 tokens: grouping by expert into
 chunks, grouped GEMMs of the packed codes against fixed-point activation
 digits on the integer tensor cores, combine + residual + RMSNorm) against the
-CPU oracle, through moe_layer_forward.
+CPU oracle, through moe_layer_forward. The shared expert runs either on the
+grouped integer kernels or as dense tcgen05 GEMMs on exact fp16 operands
+(MOE_PREFILL_SHARED=mma / tc); the tests marked with `path` run both.
 
 Routing ids bit-exact for every token; h and x_out within max relative error
 2e-3 (max|gpu - oracle| / max|oracle|) per token; bf16 x_out within one ulp
@@ -68,8 +70,10 @@ def dev():
     return torch.device("cuda")
 
 
+@pytest.mark.parametrize("path", ["tc", "mma"])
 @pytest.mark.parametrize("T", [9, 40])
-def test_prefill_tiny_matches_oracle(dev, T):
+def test_prefill_tiny_matches_oracle(dev, T, path, monkeypatch):
+    monkeypatch.setenv("MOE_PREFILL_SHARED", path)
     cfg = fixtures.CONFIGS["tiny"]
     t = fxg.device_layer(cfg, 0)
     layer = qm.layer_from_tensors(cfg, t)
@@ -78,8 +82,9 @@ def test_prefill_tiny_matches_oracle(dev, T):
     _compare(cfg, x, *out, sample=list(range(T)))
 
 
-@pytest.mark.parametrize("bits,shared", [(2, True), (4, False)])
-def test_prefill_small_layers(dev, bits, shared):
+@pytest.mark.parametrize("bits,shared,path", [(2, True, "tc"), (2, True, "mma"), (4, True, "tc"), (4, False, "tc")])
+def test_prefill_small_layers(dev, bits, shared, path, monkeypatch):
+    monkeypatch.setenv("MOE_PREFILL_SHARED", path)
     cfg = fixtures.Config(f"pf{bits}{'s' if shared else 'n'}", H=512, E=24, k=3, I=256, bits=bits,
                           scale_sigma=0.05 if bits == 2 else 0.02, has_shared=shared)
     t = fxg.device_layer(cfg, 0)
@@ -89,9 +94,12 @@ def test_prefill_small_layers(dev, bits, shared):
     _compare(cfg, x, *out, sample=list(range(33)))
 
 
-def test_prefill_wide_hidden(dev):
+@pytest.mark.parametrize("path", ["tc", "mma"])
+def test_prefill_wide_hidden(dev, path, monkeypatch):
     """Hidden 8192 (the widest layer the library takes): 4-token chunks and
-    8 quantisation groups per warp in the gate/up kernel."""
+    8 quantisation groups per warp in the gate/up kernel; 136 column stages
+    (8192 data + 512 bias-term columns) in the tensor-core gate/up pass."""
+    monkeypatch.setenv("MOE_PREFILL_SHARED", path)
     cfg = fixtures.Config("pfwide", H=8192, E=8, k=2, I=256, bits=4, has_shared=True)
     t = fxg.device_layer(cfg, 0)
     layer = qm.layer_from_tensors(cfg, t)
@@ -104,7 +112,9 @@ def test_prefill_full_size_512_tokens(dev):
     """The 512-token prefill of the 4-bit layer (hidden 4096, 512 experts,
     top-3 + shared): routing of all 512 tokens bit-exact, outputs of a
     sample of tokens (regenerating every expert the whole batch touches on
-    the host is too slow for a test)."""
+    the host is too slow for a test). At 512 tokens the shared expert takes
+    the tcgen05 path by default: two 256-token blocks per weight tile and
+    column splits whose partial sums the combine adds."""
     cfg = fixtures.CONFIGS["prefill_q4"]
     t = fxg.device_layer(cfg, 0)
     layer = qm.layer_from_tensors(cfg, t)
@@ -121,9 +131,10 @@ def test_prefill_full_size_512_tokens(dev):
     torch.cuda.empty_cache()
 
 
+@pytest.mark.parametrize("path", ["tc", "mma"])
 @pytest.mark.parametrize("where", ["x", "a"])
 @pytest.mark.parametrize("name,T", [("tiny", 40), ("layer_q4", 16)])
-def test_prefill_outlier_activations(dev, name, T, where):
+def test_prefill_outlier_activations(dev, name, T, where, path, monkeypatch):
     """Activations as real models have them, one outlier per row: "x": every
     token's input carries one element 2^10 times the rest; "a": one
     intermediate row of the shared expert has its up-projection scales raised
@@ -132,7 +143,9 @@ def test_prefill_outlier_activations(dev, name, T, where):
     exponent per 64-value group (each value within 2^-15 of its group's
     maximum), so an outlier costs only its own group bits. The experts'
     contribution h' - h must match the oracle's within the normwise bar; the
-    routing bit for bit."""
+    routing bit for bit. On the tcgen05 path the shared expert's activations
+    are fp16 with one exponent per token (a as hi + lo parts), exact for x."""
+    monkeypatch.setenv("MOE_PREFILL_SHARED", path)
     cfg = fixtures.CONFIGS[name]
     n = None if name == "tiny" else 32
     c = cfg if n is None else fixtures.Config(cfg.name, H=cfg.H, E=n, k=cfg.k, I=cfg.I, bits=cfg.bits,
