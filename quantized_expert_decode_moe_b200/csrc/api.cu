@@ -263,9 +263,15 @@ moe_status prefill_chain(const moe_layer* L, const uint16_t* x_in, float* h, int
   if (tc) {
     cx.K = H; cx.T = T; cx.Tpad = Tpad; cx.bits = L->bits; cx.x = x_in;
     cx.b_hi = at<__half>(ws, W.tcbx); cx.tscale = at<float>(ws, W.tcxs);
+    // the same launch prepares the shared expert's gate/up and down rows
+    cx.nprep = 2;
+    cx.prep[0] = TcRowPrep{2 * I, I, H, L->shared.gate, L->shared.up, at<int>(ws, W.tcrexp), at<__half>(ws, W.tcaext)};
+    cx.prep[1] = TcRowPrep{H, H, I, L->shared.down, L->shared.down, at<int>(ws, W.tcrexp) + 2 * I,
+                           at<__half>(ws, W.tcaext) + (size_t)2 * I * ((H + 1023) / 1024) * 64};
     if ((e = launch_tc_conv(cx, s)) != cudaSuccess) return MOE_ERR_CUDA;
     tg.M = 2 * I; tg.K = H; tg.R0 = I; tg.bits = L->bits; tg.w0 = L->shared.gate; tg.w1 = L->shared.up;
     tg.T = T; tg.Tpad = Tpad; tg.hilo = 0; tg.b_hi = cx.b_hi; tg.tscale = cx.tscale;
+    tg.rexp = cx.prep[0].rexp; tg.aext = cx.prep[0].aext;
     tg.part = at<float>(ws, W.tcpart); tg.status = status; tg.wait_ns = pp.wait_ns;
     if ((e = launch_tc_dense(tg, s)) != cudaSuccess)
       return e == cudaErrorInvalidConfiguration ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
@@ -282,6 +288,7 @@ moe_status prefill_chain(const moe_layer* L, const uint16_t* x_in, float* h, int
     TcParams td = tg;
     td.M = H; td.K = I; td.R0 = H; td.w0 = L->shared.down; td.w1 = L->shared.down;
     td.hilo = 1; td.b_hi = ca.b_hi; td.b_lo = ca.b_lo; td.tscale = ca.tscale;
+    td.rexp = cx.prep[1].rexp; td.aext = cx.prep[1].aext;
     if ((e = launch_tc_dense(td, s)) != cudaSuccess)
       return e == cudaErrorInvalidConfiguration ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
   }

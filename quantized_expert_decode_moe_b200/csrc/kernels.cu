@@ -57,6 +57,9 @@ WsLayout ws_layout(int H, int I, int E, int k, int S, int T) {
     np = (gu > dn ? gu : dn) * (size_t)T;
   }
   L.tcpart = o; o = align256(o + sizeof(float) * np);
+  L.tcrexp = o; o = align256(o + (T > 8 ? sizeof(int) * (size_t)(2 * I + H) : 0));
+  L.tcaext = o;
+  o = align256(o + (T > 8 ? (size_t)128 * (2 * (size_t)I * ((H + 1023) / 1024) + (size_t)H * ((I + 1023) / 1024)) : 0));
   L.total = o;
   return L;
 }

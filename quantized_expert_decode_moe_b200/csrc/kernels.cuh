@@ -42,6 +42,7 @@ struct WsLayout {
   // shared expert on the tensor cores (T > 8): fp16 operand tables of x and of its SwiGLU
   // outputs (hi, lo) [Kx/8][Tpad][8], per-token scales [Tpad], split partial sums
   size_t tcbx, tcxs, tcbah, tcbal, tcas, tcpart;
+  size_t tcrexp, tcaext;   // row exponents [2I + H] int, bias-column tiles of gate/up then down
   size_t total;
 };
 WsLayout ws_layout(int H, int I, int E, int k, int S, int T);
@@ -171,19 +172,32 @@ struct TcParams {
   const __half* b_hi;          // [Kx/8][Tpad][8] fp16, Kx = K + 64*ceil(K/1024) (tc_cols)
   const __half* b_lo;          // same, or null
   const float* tscale;         // [T] 2^-p of each token's table
+  const int* rexp;             // [M] exponent e of each weight row (row values scaled by 2^e)
+  const __half* aext;          // bias-column tiles [M/128][Kx/64 - K/64][8][128][8] fp16
   int splits;                  // column splits (gridDim.z)
   int nst;                     // pipeline stages (set by the launcher)
   float* part;                 // [splits][T][M]
   uint32_t* status;
   unsigned long long wait_ns;
 };
-// Operand tables of a batch's activations for the dense pass (shared_tc.cu).
+// Per-row preparation of a weight matrix for the dense pass: the row exponent
+// and the bias-column tiles (shared_tc.cu).
+struct TcRowPrep {
+  int M, R0, K;
+  moe_qmat w0, w1;
+  int* rexp;                   // [M]
+  __half* aext;                // [M/128][Kx/64 - K/64][8][128][8]
+};
+// Operand tables of a batch's activations for the dense pass (shared_tc.cu),
+// and (row CTAs after the token CTAs) the weight rows' preparation.
 struct TcConvParams {
   int K, T, Tpad, bits;
   const uint16_t* x;           // bf16 [T][K] (gate/up input) or null
   const float* part; int splits, I;   // gate/up partial sums [splits][T][2I] (down input) or null
   __half* b_hi; __half* b_lo;  // [Kx/8][Tpad][8]
   float* tscale;               // [Tpad]
+  int nprep;                   // weight matrices to prepare (0..2)
+  TcRowPrep prep[2];
 };
 
 // One layer of the fused decode kernel (device pointers).

@@ -78,13 +78,6 @@ int tc_splits(int M, int T, int K) {
   return s < 1 ? 1 : s;
 }
 
-// chunk position -> element offset inside the chunk's span (see the file comment)
-template <int BITS>
-__host__ __device__ __forceinline__ int tc_elem(int c, int e) {
-  if (BITS == 4) return 8 * c + (e >> 1) + 4 * (e & 1);
-  return 16 * (c >> 1) + 4 * (c & 1) + (e >> 1) + 8 * (e & 1);
-}
-
 __device__ __forceinline__ float tc_pow2(int e) { return ldexpf(1.f, e); }
 // exponent e with v * 2^e < 2^lim (v > 0), clamped; 0 for v = 0
 __device__ __forceinline__ int tc_exp_below(float v, int lim) {
@@ -96,90 +89,181 @@ __device__ __forceinline__ int tc_exp_below(float v, int lim) {
 }
 
 // ------------------------------------------------------------------ operand tables
-// One CTA per (padded) token. Values v: the bf16 input x, or the SwiGLU of the
-// gate/up pass's split sums (added in split order). Writes the token's fp16
-// columns (hi, and lo when b_lo is given) in chunk order, the group-sum
-// columns, and 2^-p. Padding tokens (t >= T) get zero columns.
+// Token CTAs: tw = min(256, max(32, pow2 >= K/16)) threads per token, 256/tw
+// tokens per CTA; each thread holds 16-element spans of its token's values in
+// registers (span sp = lane-in-token + tw q). Values v: the bf16 input x, or
+// the SwiGLU of the gate/up pass's split sums (added in split order). Writes
+// the token's fp16 columns (hi, and lo when b_lo is given) in chunk order, the
+// group-sum columns, and 2^-p. Padding tokens (T <= t < Tpad) get zero
+// columns. Row CTAs (after the token CTAs, one thread per weight row of the
+// matrices in prep): the row exponent and the bias-column tiles.
+constexpr int kTcConvSpans = 2;   // spans per thread: K <= 16 * 256 * 2
+
+// element of a 16-element span held at position e of its chunk h (0 or 1)
+template <int BITS>
+__host__ __device__ constexpr int tc_span_elem(int h, int e) {
+  return BITS == 4 ? 8 * h + (e >> 1) + 4 * (e & 1) : 4 * h + (e >> 1) + 8 * (e & 1);
+}
+__host__ __device__ inline int tc_token_threads(int K) {
+  int tw = 32;
+  while (tw < K / 16 && tw < kTcConvThreads) tw <<= 1;
+  return tw;
+}
+
+// One weight row: e with max(c|s_g|, |beta_g|) 2^e < 2^14 over all its groups,
+// then its bias columns (beta_hi, beta_lo, beta_hi, beta_lo per group, scaled
+// by 2^e) in the dense kernel's tile layout.
+template <int BITS>
+__device__ void tc_prep_row(const TcRowPrep& P, int m) {
+  constexpr float cq = BITS == 4 ? 8.f : 2.f;
+  const int ng = P.K / kGroup, nxs = tc_cols(P.K) / 64 - ng;
+  const bool second = m >= P.R0;
+  const moe_qmat W = second ? P.w1 : P.w0;
+  const int r = second ? m - P.R0 : m;
+  const uint16_t* srow = W.scales + (size_t)r * ng;
+  const uint16_t* brow = W.biases + (size_t)r * ng;
+  float mx = 0.f;
+#pragma unroll 8
+  for (int g = 0; g < ng; ++g) {
+    const float sv = bf16_to_f32(__ldg(srow + g)), bv = bf16_to_f32(__ldg(brow + g));
+    mx = fmaxf(mx, fmaxf(cq * fabsf(sv), fabsf(fmaf(cq, sv, bv))));
+  }
+  const int e = tc_exp_below(mx, 14);
+  P.rexp[m] = e;
+  const float rsc = tc_pow2(e);
+  uint4* tile = (uint4*)P.aext + (size_t)(m / kTcM) * nxs * 8 * kTcM + (m % kTcM);
+  for (int x = 0; x < nxs; ++x)
+#pragma unroll 2
+    for (int c = 0; c < 8; ++c) {
+      uint32_t v[4];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int g = 16 * x + 2 * c + h;
+        float beta = 0.f;
+        if (g < ng) beta = fmaf(cq, bf16_to_f32(__ldg(srow + g)), bf16_to_f32(__ldg(brow + g))) * rsc;
+        const uint32_t hl = pack_half2(half_hi(beta), half_lo(beta));
+        v[2 * h] = hl;
+        v[2 * h + 1] = hl;
+      }
+      tile[(size_t)(x * 8 + c) * kTcM] = make_uint4(v[0], v[1], v[2], v[3]);
+    }
+}
+
 template <int BITS>
 __global__ void __launch_bounds__(kTcConvThreads) tc_conv_kernel(TcConvParams p) {
-  extern __shared__ __align__(16) float vals[];   // [K], then the group sums [K/64]
   __shared__ float red[kTcConvThreads / 32];
-  const int t = blockIdx.x, tid = threadIdx.x;
-  const int K = p.K, ng = K / kGroup, nck = K / 8, nxk = tc_cols(K) / 8 - nck;
-  float* gsum = vals + K;
-  const bool real = t < p.T;
-  float m = 0.f;
-  if (real && p.x) {
-    const uint16_t* x = p.x + (size_t)t * K;
-    for (int k = tid; k < K; k += blockDim.x) {
-      const float v = bf16_to_f32(x[k]);
-      vals[k] = v;
-      m = fmaxf(m, fabsf(v));
-    }
-  } else if (real) {   // SwiGLU of the gate/up split sums, splits added in order
-    const int I = p.I;
-    for (int i = tid; i < I; i += blockDim.x) {
-      float g = 0.f, u = 0.f;
-      for (int s = 0; s < p.splits; ++s) {
-        const float* row = p.part + ((size_t)s * p.T + t) * (2 * (size_t)I);
-        g += __ldcg(row + i);
-        u += __ldcg(row + I + i);
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int K = p.K, nsp = K / 16, ng = K / kGroup, nck = K / 8, nxk = tc_cols(K) / 8 - nck;
+  const int tw = tc_token_threads(K), tpc = kTcConvThreads / tw;
+  const int ntb = (p.Tpad + tpc - 1) / tpc;   // token CTAs
+  if ((int)blockIdx.x >= ntb) {   // ---------------------------------------- weight rows
+    int m = (blockIdx.x - ntb) * kTcConvThreads + tid;
+    for (int j = 0; j < p.nprep; ++j) {
+      if (m < p.prep[j].M) {
+        tc_prep_row<BITS>(p.prep[j], m);
+        return;
       }
-      const float v = silu_f32(g) * u;
-      vals[i] = v;
-      m = fmaxf(m, fabsf(v));
+      m -= p.prep[j].M;
     }
-  } else {
-    for (int k = tid; k < K; k += blockDim.x) vals[k] = 0.f;
+    return;
   }
-  // block max -> 2^p with max|v| 2^p < 2^9
-  m = warp_max(m);
-  if ((tid & 31) == 0) red[tid >> 5] = m;
-  __syncthreads();
-  if (tid < 32) {
-    float r = tid < (int)(blockDim.x >> 5) ? red[tid] : 0.f;
-    r = warp_max(r);
-    if (tid == 0) red[0] = r;
-  }
-  __syncthreads();
-  const int pe = tc_exp_below(red[0], 9);
-  const float sc = tc_pow2(pe);
-  if (tid == 0) p.tscale[t] = real ? tc_pow2(-pe) : 0.f;
-  // group sums of the scaled values
-  for (int g = tid; g < ng; g += blockDim.x) {
-    float s = 0.f;
-    for (int k = 0; k < kGroup; ++k) s += vals[g * kGroup + k] * sc;
-    gsum[g] = s;
-  }
-  // data columns
-  for (int c = tid; c < nck; c += blockDim.x) {
-    uint32_t hi[4], lo[4];
+  const int sub = tid / tw, lt = tid % tw;
+  const int t = blockIdx.x * tpc + sub;
+  const bool real = t < p.T, live = t < p.Tpad;
+  float v[kTcConvSpans][16];
+  float m = 0.f;
 #pragma unroll
-    for (int e = 0; e < 8; e += 2) {
-      const float v0 = vals[tc_elem<BITS>(c, e)] * sc, v1 = vals[tc_elem<BITS>(c, e + 1)] * sc;
-      hi[e / 2] = pack_half2(half_hi(v0), half_hi(v1));
-      lo[e / 2] = pack_half2(half_lo(v0), half_lo(v1));
+  for (int q = 0; q < kTcConvSpans; ++q) {
+    const int sp = lt + q * tw;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) v[q][e] = 0.f;
+    if (!real || sp >= nsp) continue;
+    if (p.x) {
+      const uint4* src = (const uint4*)(p.x + (size_t)t * K + 16 * sp);
+      const uint4 a = __ldg(src), b = __ldg(src + 1);
+      const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        v[q][2 * j] = bf16lo(w[j]);
+        v[q][2 * j + 1] = bf16hi(w[j]);
+      }
+    } else {   // SwiGLU of the gate/up split sums, splits added in order
+      float g[16], u[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) g[e] = u[e] = 0.f;
+      for (int s = 0; s < p.splits; ++s) {
+        const float* row = p.part + ((size_t)s * p.T + t) * (2 * (size_t)p.I) + 16 * sp;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float4 gg = __ldcg((const float4*)row + j), uu = __ldcg((const float4*)(row + p.I) + j);
+          g[4 * j] += gg.x; g[4 * j + 1] += gg.y; g[4 * j + 2] += gg.z; g[4 * j + 3] += gg.w;
+          u[4 * j] += uu.x; u[4 * j + 1] += uu.y; u[4 * j + 2] += uu.z; u[4 * j + 3] += uu.w;
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 16; ++e) v[q][e] = silu_f32(g[e]) * u[e];
     }
-    const size_t o = ((size_t)c * p.Tpad + t) * 8;
-    *(uint4*)(p.b_hi + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-    if (p.b_lo) *(uint4*)(p.b_lo + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) m = fmaxf(m, fabsf(v[q][e]));
   }
+  // the token's max -> 2^p with max|v| 2^p < 2^9
+  m = warp_max(m);
+  if (lane == 0) red[tid >> 5] = m;
   __syncthreads();
-  // group-sum columns: chunk j holds groups 2j, 2j+1 as (S_hi, S_hi, S_lo, S_lo)
-  for (int j = tid; j < nxk; j += blockDim.x) {
-    uint32_t w[4];
+  float mx = 0.f;
+  for (int w = sub * (tw / 32); w < (sub + 1) * (tw / 32); ++w) mx = fmaxf(mx, red[w]);
+  const int pe = tc_exp_below(mx, 9);
+  const float sc = tc_pow2(pe);
+  if (lt == 0 && live) p.tscale[t] = real ? tc_pow2(-pe) : 0.f;
+#pragma unroll
+  for (int q = 0; q < kTcConvSpans; ++q) {
+    const int sp = lt + q * tw;
+    float ssum = 0.f;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      v[q][e] *= sc;
+      ssum += v[q][e];
+    }
+    // a group is 4 spans = 4 consecutive lanes
+    ssum += __shfl_xor_sync(0xffffffffu, ssum, 1);
+    ssum += __shfl_xor_sync(0xffffffffu, ssum, 2);
+    const float snext = __shfl_down_sync(0xffffffffu, ssum, 4);   // the next group's sum
+    if (sp >= nsp || !live) continue;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const int g = 2 * j + h;
-      const float s = g < ng ? gsum[g] : 0.f;
-      const __half sh = half_hi(s), sl = half_lo(s);
-      w[2 * h] = pack_half2(sh, sh);
-      w[2 * h + 1] = pack_half2(sl, sl);
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        const float v0 = v[q][tc_span_elem<BITS>(h, e)], v1 = v[q][tc_span_elem<BITS>(h, e + 1)];
+        hi[e / 2] = pack_half2(half_hi(v0), half_hi(v1));
+        lo[e / 2] = pack_half2(half_lo(v0), half_lo(v1));
+      }
+      const size_t o = ((size_t)(2 * sp + h) * p.Tpad + t) * 8;
+      *(uint4*)(p.b_hi + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      if (p.b_lo) *(uint4*)(p.b_lo + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
-    const size_t o = ((size_t)(nck + j) * p.Tpad + t) * 8;
-    *(uint4*)(p.b_hi + o) = make_uint4(w[0], w[1], w[2], w[3]);
-    if (p.b_lo) *(uint4*)(p.b_lo + o) = make_uint4(0u, 0u, 0u, 0u);
+    // group-sum columns: chunk j holds groups 2j, 2j+1 as (S_hi, S_hi, S_lo, S_lo)
+    if ((sp & 7) == 0) {
+      uint32_t w[4];
+      const float sg[2] = {ssum, snext};
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const __half sh = half_hi(sg[h]), sl = half_lo(sg[h]);
+        w[2 * h] = pack_half2(sh, sh);
+        w[2 * h + 1] = pack_half2(sl, sl);
+      }
+      const size_t o = ((size_t)(nck + sp / 8) * p.Tpad + t) * 8;
+      *(uint4*)(p.b_hi + o) = make_uint4(w[0], w[1], w[2], w[3]);
+      if (p.b_lo) *(uint4*)(p.b_lo + o) = make_uint4(0u, 0u, 0u, 0u);
+    }
   }
+  // padding group-sum columns (groups ng and above)
+  if (live)
+    for (int j = ng / 2 + lt; j < nxk; j += tw) {
+      const size_t o = ((size_t)(nck + j) * p.Tpad + t) * 8;
+      *(uint4*)(p.b_hi + o) = make_uint4(0u, 0u, 0u, 0u);
+      if (p.b_lo) *(uint4*)(p.b_lo + o) = make_uint4(0u, 0u, 0u, 0u);
+    }
 }
 
 // ------------------------------------------------------------------ dense pass
@@ -266,12 +350,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_dense_kernel(TcParams p) {
   const int i0 = (int)((long long)nstg * split / p.splits);
   const int i1 = (int)((long long)nstg * (split + 1) / p.splits);
   const int n = i1 - i0;
+  // The row blocks of one split start at different stages (the sum order of a
+  // row is still fixed), so that they do not all read the same activation tile
+  // of L2 at the same time.
+  const int rot = (int)(blockIdx.x % (unsigned)n);
+  auto stage_of = [&](int u) { const int v = u + rot; return i0 + (v >= n ? v - n : v); };
   const uint32_t ncols = tc_tmem_cols(p.nt, p.hilo);
   const unsigned long long wns = p.wait_ns;
 
   if (tid == 0) {
     for (int s = 0; s < nst; ++s) {
-      mbar_init(&full_a[s], kTcProducers);
+      mbar_init(&full_a[s], kTcProducers + 1);   // + the copy thread (bias-column tiles)
       mbar_init(&full_b[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -294,57 +383,36 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_dense_kernel(TcParams p) {
     const int r = second ? grow - p.R0 : grow;
     const uint32_t* qrow = W.q + (size_t)r * (p.K * BITS / 32);
     const uint16_t* srow = W.scales + (size_t)r * ng;
-    const uint16_t* brow = W.biases + (size_t)r * ng;
-    constexpr float cq = BITS == 4 ? 8.f : 2.f;
-    // row exponent over the groups this CTA reads: data groups need c|s|, bias-column groups |beta|
-    float mx = 0.f;
-    for (int i = i0; i < i1; ++i) {
-      if (i < ng) {
-        mx = fmaxf(mx, cq * fabsf(bf16_to_f32(__ldg(srow + i))));
-      } else {
-        const int gb = (i - ng) * 16;
-        for (int u = 0; u < 16 && gb + u < ng; ++u) {
-          const float s = bf16_to_f32(__ldg(srow + gb + u)), b = bf16_to_f32(__ldg(brow + gb + u));
-          mx = fmaxf(mx, fabsf(fmaf(cq, s, b)));
-        }
-      }
-    }
-    const int e = tc_exp_below(mx, 14);
+    const int d1 = i1 < ng ? i1 : ng;   // data stages of this CTA: [i0, d1); the rest are bias columns
+    // codes of the next stages in a ring of four register sets, named (no moves between them)
+    TcRaw r0{}, r1{}, r2{}, r3{};
+    if (n > 0 && stage_of(0) < d1) tc_load_raw<BITS>(qrow, srow, stage_of(0), r0);
+    if (n > 1 && stage_of(1) < d1) tc_load_raw<BITS>(qrow, srow, stage_of(1), r1);
+    if (n > 2 && stage_of(2) < d1) tc_load_raw<BITS>(qrow, srow, stage_of(2), r2);
+    const int e = __ldg(p.rexp + grow);
     const float rsc = tc_pow2(e);
-    TcRaw cur{}, nxt{};
-    if (i0 < ng) tc_load_raw<BITS>(qrow, srow, i0, cur);
-    for (int u = 0; u < n; ++u) {
-      const int i = i0 + u, slot = u % nst, use = u / nst;
-      if (i + 1 < i1 && i + 1 < ng) tc_load_raw<BITS>(qrow, srow, i + 1, nxt);
+    auto step = [&](int u, const TcRaw& cur, TcRaw& ahead) -> bool {
+      const int i = stage_of(u), slot = u % nst, use = u / nst;
+      if (u + 3 < n && stage_of(u + 3) < d1) tc_load_raw<BITS>(qrow, srow, stage_of(u + 3), ahead);
       if (use > 0 && !mbar_wait_bounded(&empty[slot], (use - 1) & 1, wns, p.status)) *abort_flag = 1;
-      if (*abort_flag) break;
-      uint4* dst = (uint4*)(sA + (size_t)slot * kTcABytes) + tid;   // chunk c at + c*128 uint4
+      if (*abort_flag) return false;
       if (i < ng) {
+        uint4* dst = (uint4*)(sA + (size_t)slot * kTcABytes) + tid;   // chunk c at + c*128 uint4
         const __half2 s2 = __half2half2(__float2half_rn(cur.s * rsc));
         const uint32_t w[8] = {cur.q0.x, cur.q0.y, cur.q0.z, cur.q0.w, cur.q1.x, cur.q1.y, cur.q1.z, cur.q1.w};
 #pragma unroll
         for (int c = 0; c < 8; ++c)
           dst[c * kTcM] = BITS == 4 ? tc_dequant_chunk<4>(w[c], 0, s2) : tc_dequant_chunk<2>(w[c >> 1], c & 1, s2);
-      } else {   // bias columns: chunk c holds groups gb+2c, gb+2c+1 as (beta_hi, beta_lo, beta_hi, beta_lo)
-        const int gb = (i - ng) * 16;
-#pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          uint32_t v[4];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int g = gb + 2 * c + h;
-            float beta = 0.f;
-            if (g < ng) beta = fmaf(cq, bf16_to_f32(__ldg(srow + g)), bf16_to_f32(__ldg(brow + g))) * rsc;
-            const uint32_t hl = pack_half2(half_hi(beta), half_lo(beta));
-            v[2 * h] = hl;
-            v[2 * h + 1] = hl;
-          }
-          dst[c * kTcM] = make_uint4(v[0], v[1], v[2], v[3]);
-        }
+        fence_proxy_async();
       }
-      fence_proxy_async();
-      mbar_arrive(&full_a[slot]);
-      cur = nxt;
+      mbar_arrive(&full_a[slot]);   // bias-column tiles arrive by bulk copy (warp 5)
+      return true;
+    };
+    for (int u = 0; u < n; u += 4) {
+      if (!step(u, r0, r3)) break;
+      if (u + 1 >= n || !step(u + 1, r1, r0)) break;
+      if (u + 2 >= n || !step(u + 2, r2, r1)) break;
+      if (u + 3 >= n || !step(u + 3, r3, r2)) break;
     }
     // ---------------------------------------------------------------- epilogue
     bool ok = mbar_wait_bounded(done, 0, wns, p.status) && !*abort_flag;
@@ -397,14 +465,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_dense_kernel(TcParams p) {
     mbar_wait_bounded(done, 0, wns, p.status);
   } else if (tid == 5 * 32) {
     // ---------------------------------------------------------------- activation tiles (one thread)
-    int last[kTcMaxStages];
-    for (int s = 0; s < kTcMaxStages; ++s) last[s] = -1;
+    int last[kTcMaxStages], lastx[kTcMaxStages];   // last use of each slot with copies issued (B, bias tile)
+    for (int s = 0; s < kTcMaxStages; ++s) last[s] = lastx[s] = -1;
     const unsigned rows_bytes = (unsigned)npad * 16;
     const unsigned bytes = rows_bytes * (kTcKS / 8) * (p.hilo ? 2u : 1u);
     for (int u = 0; u < n; ++u) {
-      const int i = i0 + u, slot = u % nst, use = u / nst;
+      const int i = stage_of(u), slot = u % nst, use = u / nst;
       if (use > 0 && !mbar_wait_bounded(&empty[slot], (use - 1) & 1, wns, p.status)) *abort_flag = 1;
       if (*abort_flag) break;
+      if (i >= ng) {   // bias columns: the prepared 128 x 64 tile of this row block
+        mbar_expect_tx(&full_a[slot], (unsigned)kTcABytes);
+        bulk_g2s(sA + (size_t)slot * kTcABytes, p.aext + ((size_t)blockIdx.x * (nstg - ng) + (i - ng)) * (kTcABytes / 2),
+                 (unsigned)kTcABytes, &full_a[slot]);
+      } else {
+        mbar_arrive(&full_a[slot]);
+      }
       mbar_expect_tx(&full_b[slot], bytes);
       unsigned char* dst = sB + (size_t)slot * G.stage_b;
 #pragma unroll 1
@@ -414,10 +489,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_dense_kernel(TcParams p) {
         if (p.hilo) bulk_g2s(dst + (size_t)c * G.brows * 16 + (size_t)p.nt * 16, p.b_lo + o, rows_bytes, &full_b[slot]);
       }
       last[slot] = use;
+      lastx[slot] = i >= ng ? use : -1;
     }
     // no copy may land after the CTA has left
     for (int s = 0; s < nst && s < kTcMaxStages; ++s)
-      if (last[s] >= 0) mbar_wait_bounded(&full_b[s], last[s] & 1, wns, p.status);
+      if (last[s] >= 0) {
+        mbar_wait_bounded(&full_b[s], last[s] & 1, wns, p.status);
+        if (lastx[s] >= 0) mbar_wait_bounded(&full_a[s], lastx[s] & 1, wns, p.status);
+      }
   }
   tc_fence_before();
   __syncthreads();
@@ -446,13 +525,15 @@ bool tc_supported(int H, int I, int bits) {
 }
 
 cudaError_t launch_tc_conv(const TcConvParams& p, cudaStream_t s) {
-  const size_t sm = sizeof(float) * ((size_t)p.K + p.K / kGroup);
+  if (p.K % kGroup || p.K > 16 * kTcConvThreads * kTcConvSpans) return cudaErrorInvalidConfiguration;
   const void* fn = p.bits == 4 ? (const void*)tc_conv_kernel<4> : (const void*)tc_conv_kernel<2>;
-  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-  if (e != cudaSuccess) return e;
+  const int tpc = kTcConvThreads / tc_token_threads(p.K);
+  int rows = 0;
+  for (int j = 0; j < p.nprep; ++j) rows += p.prep[j].M;
+  const int nb = (p.Tpad + tpc - 1) / tpc + (rows + kTcConvThreads - 1) / kTcConvThreads;
   TcConvParams q = p;
   void* args[] = {&q};
-  return cudaLaunchKernel(fn, dim3(p.Tpad), dim3(kTcConvThreads), args, sm, s);
+  return cudaLaunchKernel(fn, dim3(nb), dim3(kTcConvThreads), args, 0, s);
 }
 
 // Sets nt, splits and nst from the shapes (callers read the split count with tc_splits).
