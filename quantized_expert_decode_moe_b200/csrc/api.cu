@@ -158,6 +158,8 @@ moe_status decode_chain(const moe_layer* L, const uint16_t* x_in, float* h, int 
   gp.router_w = L->router_w; gp.router_bias = L->router_bias;
   gp.a = at<float>(ws, W.a);
   gp.idx_out = topk_idx; gp.w_out = topk_w;
+  gp.sel_idx = at<int32_t>(ws, W.pidx); gp.sel_w = at<float>(ws, W.pw); gp.sel_sg = at<float>(ws, W.psg);
+  gp.sel_flag = at<unsigned>(ws, kSelFlagOffset);
   gp.status = status; gp.wait_ns = wait_bound_ns();
   gp.rechecks = at<uint32_t>(ws, 16);
   if ((e = launch_gateup(gp, L->bits, T, pdl, s)) != cudaSuccess)
@@ -167,8 +169,8 @@ moe_status decode_chain(const moe_layer* L, const uint16_t* x_in, float* h, int 
   DownParams dp{};
   dp.H = H; dp.I = I; dp.E = E; dp.k = k; dp.S = S; dp.has_shared = L->has_shared;
   dp.nCTA = down_ctas(H);
-  dp.x = x_in; dp.logits = rp.logits; dp.bound = rp.bound; dp.a = gp.a; dp.h = h; dp.experts = L->experts;
-  dp.shared = L->shared; dp.router_w = L->router_w; dp.router_bias = L->router_bias;
+  dp.sel_idx = gp.sel_idx; dp.sel_w = gp.sel_w; dp.sel_sg = gp.sel_sg; dp.sel_flag = gp.sel_flag;
+  dp.a = gp.a; dp.h = h; dp.experts = L->experts; dp.shared = L->shared;
   dp.hacc = at<float>(ws, W.hacc);
   dp.status = status; dp.wait_ns = gp.wait_ns;
   if ((e = launch_down(dp, L->bits, T, pdl, s)) != cudaSuccess)
@@ -178,6 +180,7 @@ moe_status decode_chain(const moe_layer* L, const uint16_t* x_in, float* h, int 
   NormDecodeParams np{};
   np.H = H; np.T = T;
   np.hacc = dp.hacc; np.h = h; np.gamma = L->rms_gamma; np.eps = L->rms_eps; np.x_out = x_out; np.x_out_f32 = x_out_f32;
+  np.sel_flag = gp.sel_flag;
   if ((e = launch_norm_decode(np, pdl, s)) != cudaSuccess) return MOE_ERR_CUDA;
   mark(4);
   return MOE_OK;

@@ -54,12 +54,14 @@ __host__ __device__ inline GuLayout gu_layout(int H, int bits) {
   return L;
 }
 
-// grid (nCTA, T), block 512. Items: the shared expert first (its copies and
-// MMAs run before the dependency wait: this kernel starts only after every
-// router CTA has passed its own wait, so x is final; its a values are stored
-// and fenced before this kernel lets the down kernel launch), then the k
-// routed experts, which every CTA ranks itself from the router's logits and
-// computes side by side, each on its own group of warps.
+// grid (nCTA, T), block 512. Before the dependency wait (this kernel starts
+// only after every router CTA has passed its own wait, so x is final): the
+// shared expert's copies and the B tables of x. After it: every CTA ranks the
+// router's logits itself (the first CTA of each token publishes the selection
+// for the down kernel behind a flag), issues the copies of the routed experts
+// whose buffers are free, computes the shared expert while they land, stores
+// and fences its a, lets the down kernel launch, and computes the routed
+// experts.
 template <int BITS>
 __global__ void __launch_bounds__(kThreads, 2) gateup_decode_kernel(GateUpParams p) {
   extern __shared__ __align__(128) unsigned char smem[];
@@ -209,40 +211,60 @@ __global__ void __launch_bounds__(kThreads, 2) gateup_decode_kernel(GateUpParams
     }
   }
   __syncthreads();
-  int it0 = 0;
-  if (p.has_shared) {   // the shared expert, before the dependency wait
-    compute_items(0, 1);
-    fence_proxy_async();
-    __syncthreads();
-    finalize(0, 1);
-    __syncthreads();   // ... so no thread signals the dependent launch before those stores are fenced
-    it0 = 1;
-  }
 
   // the router's logits are complete after the wait
   griddep_wait();
-  griddep_launch_dependents();
   {
     const RouterRef rr{p.x + (size_t)t * H, p.router_w, p.router_bias, H};
     block_topk(p.logits + (size_t)t * (p.E + 1), p.bound + (size_t)t * (p.E + 1), p.E, k, p.has_shared, rr, ts);
   }
   load_slots(ts, k, p.E, p.experts, slot_ex, p.status);
   if (blockIdx.x == 0 && tid == 0 && p.rechecks && ts.rechecked) atomicAdd(p.rechecks, 1u);
-  if (blockIdx.x == 0 && tid < k) {
-    if (p.idx_out) p.idx_out[(size_t)t * k + tid] = ts.idx[tid];
-    if (p.w_out) p.w_out[(size_t)t * k + tid] = ts.w[tid];
+  if (blockIdx.x == 0) {   // publish the selection for the down kernel (and the user copies)
+    if (tid < k) {
+      p.sel_idx[(size_t)t * k + tid] = ts.idx[tid];
+      p.sel_w[(size_t)t * k + tid] = ts.w[tid];
+      if (p.idx_out) p.idx_out[(size_t)t * k + tid] = ts.idx[tid];
+      if (p.w_out) p.w_out[(size_t)t * k + tid] = ts.w[tid];
+    }
+    if (tid == 0) p.sel_sg[t] = ts.sg;
+    __syncthreads();
+    if (tid == 0) {
+      __threadfence();
+      st_release_u32(p.sel_flag + t, 1u);
+    }
   }
+  // Items: 0 = the shared expert (copies issued before the wait, buffer 0), then the
+  // routed ones. The routed items whose buffers are free go out first; the shared
+  // expert is computed while they land, and its a is stored (and fenced) before the
+  // dependent launch, since the down kernel applies it before its own wait.
+  int it0 = 0, issued = 0;   // items [0, issued) have had their copies issued
+  if (p.has_shared) {
+    const int w1 = nitems < kGuBufs ? nitems : kGuBufs;
+    for (int it = 1; it < w1; ++it) arm(it);
+    __syncthreads();   // slots loaded
+    if (lane == 0)
+      for (int c = warp; c < ncp * (w1 - 1); c += kWarps) issue(1 + c / ncp, c % ncp);
+    compute_items(0, 1);
+    fence_proxy_async();
+    __syncthreads();
+    finalize(0, 1);
+    __syncthreads();   // ... so no thread signals the dependent launch before those stores are fenced
+    it0 = 1;
+    issued = w1;
+  }
+  griddep_launch_dependents();
   // routed items in waves of up to kGuBufs; every warp takes its spans of all items of the wave
-  int issued = it0;   // items [0, issued) have had their copies issued
   for (int w0 = it0; w0 < nitems; w0 += kGuBufs) {
     const int w1 = nitems - w0 < kGuBufs ? nitems : w0 + kGuBufs;
     // after a wait ran out, nothing more is armed or issued (a new phase on a
     // buffer whose copies may still be landing would mix two phases)
     if (!__syncthreads_and(ok)) break;
-    for (int it = w0; it < w1; ++it) arm(it);
+    const int a0 = issued > w0 ? issued : w0;   // the wave's items not yet issued
+    for (int it = a0; it < w1; ++it) arm(it);
     __syncthreads();   // slots loaded (first wave) / previous wave's buffers and partial sums consumed
     if (lane == 0)
-      for (int c = warp; c < ncp * (w1 - w0); c += kWarps) issue(w0 + c / ncp, c % ncp);
+      for (int c = warp; c < ncp * (w1 - a0); c += kWarps) issue(a0 + c / ncp, c % ncp);
     issued = w1;
     compute_items(w0, w1);
     fence_proxy_async();
@@ -454,13 +476,24 @@ __global__ void __launch_bounds__(kThreads, 2) down_decode_kernel(DownParams p) 
     for (int b = 0; b < nb; ++b) mbar_expect_tx(&bars[b], item_bytes);   // items 0..nb-1
     if (p.has_shared) slot_ex[S - 1] = p.shared;
   }
-  {
-    const RouterRef rr{p.x + (size_t)t * H, p.router_w, p.router_bias, H};
-    block_topk(p.logits + (size_t)t * (p.E + 1), p.bound + (size_t)t * (p.E + 1), p.E, k, p.has_shared, rr, ts);
+  // the selection of the gate/up kernel's first CTA: published behind a flag that the norm
+  // kernel clears after this kernel has completed (the wait is bounded)
+  if (tid == 0) {
+    const unsigned long long t0 = globaltimer_ns();
+    while (ld_acquire_u32(p.sel_flag + t) == 0u)
+      if (globaltimer_ns() - t0 > p.wait_ns) {
+        latch_timeout(p.status);
+        break;
+      }
   }
+  __syncthreads();
+  if (tid < k) {
+    ts.idx[tid] = __ldcg(p.sel_idx + (size_t)t * k + tid);
+    wsl[tid] = __ldcg(p.sel_w + (size_t)t * k + tid);
+  }
+  if (tid == 0 && p.has_shared) wsl[S - 1] = __ldcg(p.sel_sg + t);
+  __syncthreads();
   load_slots(ts, k, p.E, p.experts, slot_ex, p.status);
-  if (tid < k) wsl[tid] = ts.w[tid];
-  if (tid == 0 && p.has_shared) wsl[S - 1] = ts.sg;
   if (tid < n) yacc[tid] = __ldcg(p.h + (size_t)t * H + h0 + tid);
   __syncthreads();
   if (lane == 0)

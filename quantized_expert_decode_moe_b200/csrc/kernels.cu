@@ -228,6 +228,7 @@ __global__ void __launch_bounds__(kNormThreads) norm_decode_kernel(NormDecodePar
   }
   griddep_wait();
   griddep_launch_dependents();
+  if (tid == 0 && p.sel_flag) p.sel_flag[t] = 0u;   // the down kernel has completed: no reader is left
   const float4* hr = (const float4*)(p.hacc + (size_t)t * p.H);
   float4 hv[kNormPer / 4];
   float ss = 0.f;

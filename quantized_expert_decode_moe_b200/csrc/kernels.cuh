@@ -11,11 +11,13 @@ namespace qmoe {
 
 constexpr int kMaxCtas = 1024;   // CTAs of the fused decode kernel at most
 constexpr int kRgSplit = 4;      // slices of H in the many-token router GEMM
+constexpr size_t kSelFlagOffset = 80;   // byte offset of the decode chain's selection flags (8 words)
 
 // Workspace carve-up for T tokens of one layer shape. The first 256 bytes are
 // the header: the status word (word 0), the count of top-k selections that
 // needed the exact recheck (word 4), the grid-barrier arrival counters
-// (words 16..19) and generations (words 32, 40, 48, 56).
+// (words 16..19), the decode chain's per-token selection flags (words
+// 20..27) and the grid-barrier generations (words 32, 40, 48, 56).
 struct WsLayout {
   size_t status;      // uint32 status word (+ padding)
   size_t logits;      // double [T][E+1]; column E = shared-gate logit
@@ -84,16 +86,18 @@ struct GateUpParams {
   float* a;                    // [T][S][I]
   int32_t* idx_out; float* w_out;   // user copies of the routing, nullable
   uint32_t* rechecks;          // counter of selections that needed the exact recheck, or null
+  // the first CTA of each token publishes its selection for the down kernel, then sets the flag
+  int32_t* sel_idx; float* sel_w; float* sel_sg;   // [T][k], [T][k], [T]
+  unsigned* sel_flag;          // [T]
   uint32_t* status;
   unsigned long long wait_ns;  // bound of every device-side wait
 };
 
 struct DownParams {
   int H, I, E, k, S, has_shared, nCTA;
-  const uint16_t* x;           // [T][H]
-  const double* logits;        // [T][E+1]
-  const float* bound;          // [T][E+1] error bounds of the logits
-  const uint16_t* router_w; const float* router_bias;   // for an exact recheck of near ties
+  // the selection published by the gate/up kernel's first CTA of each token (behind sel_flag)
+  const int32_t* sel_idx; const float* sel_w; const float* sel_sg;
+  const unsigned* sel_flag;
   const float* a;              // [T][S][I]
   const float* h;              // [T][H] residual
   const moe_expert* experts;
@@ -107,6 +111,7 @@ struct NormDecodeParams {
   int H, T;
   const float* hacc; float* h; const uint16_t* gamma; float eps;
   uint16_t* x_out; float* x_out_f32;
+  unsigned* sel_flag;          // [T] cleared (every reader has passed: the down kernel is complete)
 };
 
 struct NormParams {
