@@ -121,7 +121,10 @@ typedef struct {
  * on the same stream. */
 moe_status moe_workspace_size(const moe_layer* layer, int32_t max_tokens, size_t* bytes);
 
-/* Clears the workspace status word (async on `stream`). */
+/* Clears the workspace header, the first 256 bytes (async on `stream`): the
+ * status word, the recheck counter, and the words the decode kernels keep
+ * there between calls (grid-barrier counters, per-token selection flags;
+ * all 0 between calls). */
 moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
 
 /*
@@ -283,7 +286,7 @@ moe_status moe_noalloc_poll_status(void* stream);
 
 /* Synchronises `stream` and returns the status latched in the workspace by
  * earlier calls (MOE_OK if none). A latched status is cleared together with
- * the grid-barrier counters of the workspace header (the first 256 bytes),
+ * the counters and flags of the workspace header (the first 256 bytes),
  * which a call that ran out of time may have left mid-round. */
 moe_status moe_poll_status(void* ws, void* stream);
 
