@@ -173,6 +173,7 @@ moe_status moe_expert_gemv_q2(const moe_qmat* W, int32_t R, int32_t K, int32_t g
  *   y_routed fp32 [T][k][H]; topk_w fp32 [T][k]; y_shared fp32 [T][H] or NULL
  *   (then shared_gate is ignored and may be NULL); h fp32 [T][H] in/out (h');
  *   gamma bf16 [H]; x_out bf16 [T][H]; x_out_f32 fp32 [T][H] or NULL.
+ *   H a multiple of 8, at most 8192 (else MOE_ERR_UNSUPPORTED).
  */
 moe_status moe_combine_residual_norm(int32_t T, int32_t H, int32_t k, const float* y_routed,
                                      const float* topk_w, const float* y_shared,

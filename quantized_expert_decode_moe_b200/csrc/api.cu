@@ -421,7 +421,8 @@ moe_status moe_combine_residual_norm(int32_t T, int32_t H, int32_t k, const floa
                                      const float* y_shared, const float* shared_gate, float* h,
                                      const uint16_t* gamma, float eps, uint16_t* x_out, float* x_out_f32,
                                      void* stream) {
-  if (T <= 0 || H <= 0 || k < 0 || k > kMaxTopK || H > 65536) return MOE_ERR_INVALID_ARGUMENT;
+  if (T <= 0 || H <= 0 || k < 0 || k > kMaxTopK) return MOE_ERR_INVALID_ARGUMENT;
+  if (H % 8 || H > kMaxHI) return MOE_ERR_UNSUPPORTED;   // eight equal row slices per token, H <= 8192
   if ((k > 0 && (!y_routed || !topk_w)) || !h || !gamma || !x_out) return MOE_ERR_INVALID_ARGUMENT;
   if (y_shared && !shared_gate) return MOE_ERR_INVALID_ARGUMENT;
   if (!(eps > 0.f) || !isfinite(eps)) return MOE_ERR_INVALID_ARGUMENT;

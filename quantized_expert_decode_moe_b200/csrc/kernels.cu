@@ -342,6 +342,71 @@ norm_cluster_kernel(NormParams p) {
   }
 }
 
+// grid T, block 512 (many tokens: a token per CTA, float4 per thread). Same
+// sums as norm_cluster_kernel, element by element: v = h; v = fma(w_i, y_i, v)
+// for the routed slots in rank order; v = fma(sg, y_shared, v) with y_shared
+// the sum of its splits in order.
+constexpr int kNormRThreads = 512;
+constexpr int kNormRPer = 4;   // float4 per thread: H <= 8192
+
+__global__ void __launch_bounds__(kNormRThreads) norm_rows_kernel(NormParams p) {
+  __shared__ float red[kNormRThreads / 32];
+  __shared__ float wsh[kMaxSlots];
+  const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  griddep_wait();
+  griddep_launch_dependents();
+  if (tid < p.k) wsh[tid] = ldcg_f32(p.w + (size_t)t * p.k + tid);
+  if (tid == 0) wsh[kMaxSlots - 1] = p.y_shared ? ldcg_f32(p.sg + t) : 0.f;
+  __syncthreads();
+  const int n4 = p.H / 4, nsp = p.y_shared_splits > 1 ? p.y_shared_splits : 1;
+  const float4* hr = (const float4*)(p.h + (size_t)t * p.H);
+  const float* yr = p.y_routed + (size_t)t * p.y_routed_tok_stride;
+  const float* ysh = p.y_shared ? p.y_shared + (size_t)t * p.y_shared_tok_stride : nullptr;
+  float4 hv[kNormRPer];
+  float ss = 0.f;
+#pragma unroll
+  for (int u = 0; u < kNormRPer; ++u) {
+    const int i = tid + kNormRThreads * u;
+    if (i >= n4) continue;
+    float4 v = hr[i];
+    for (int r = 0; r < p.k; ++r) {
+      const float4 y = __ldcg((const float4*)(yr + (size_t)r * p.y_routed_slot_stride) + i);
+      const float w = wsh[r];
+      v.x = fmaf(w, y.x, v.x); v.y = fmaf(w, y.y, v.y); v.z = fmaf(w, y.z, v.z); v.w = fmaf(w, y.w, v.w);
+    }
+    if (ysh) {
+      float4 ys = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int q = 0; q < nsp; ++q) {
+        const float4 y = __ldcg((const float4*)(ysh + (size_t)q * p.y_shared_split_stride) + i);
+        ys.x += y.x; ys.y += y.y; ys.z += y.z; ys.w += y.w;
+      }
+      const float w = wsh[kMaxSlots - 1];
+      v.x = fmaf(w, ys.x, v.x); v.y = fmaf(w, ys.y, v.y); v.z = fmaf(w, ys.z, v.z); v.w = fmaf(w, ys.w, v.w);
+    }
+    hv[u] = v;
+    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  ss = warp_sum(ss);
+  if (lane == 0) red[warp] = ss;
+  __syncthreads();
+  const float tot = warp_sum(lane < kNormRThreads / 32 ? red[lane] : 0.f);
+  const float inv = 1.f / sqrtf(tot / (float)p.H + p.eps);
+#pragma unroll
+  for (int u = 0; u < kNormRPer; ++u) {
+    const int i = tid + kNormRThreads * u;
+    if (i >= n4) continue;
+    ((float4*)(p.h + (size_t)t * p.H))[i] = hv[u];
+    const uint2 g = *(const uint2*)(p.gamma + 4 * (size_t)i);
+    const float o0 = hv[u].x * inv * bf16lo(g.x), o1 = hv[u].y * inv * bf16hi(g.x);
+    const float o2 = hv[u].z * inv * bf16lo(g.y), o3 = hv[u].w * inv * bf16hi(g.y);
+    uint2 ob;
+    ob.x = (uint32_t)f32_to_bf16(o0) | ((uint32_t)f32_to_bf16(o1) << 16);
+    ob.y = (uint32_t)f32_to_bf16(o2) | ((uint32_t)f32_to_bf16(o3) << 16);
+    *(uint2*)(p.x_out + (size_t)t * p.H + 4 * (size_t)i) = ob;
+    if (p.x_out_f32) ((float4*)(p.x_out_f32 + (size_t)t * p.H))[i] = make_float4(o0, o1, o2, o3);
+  }
+}
+
 // ------------------------------------------------------------------ standalone dequant GEMV
 constexpr int kGemvSlots = 8;
 
@@ -467,6 +532,14 @@ cudaError_t launch_norm_decode(const NormDecodeParams& p, bool pdl, cudaStream_t
 }
 
 cudaError_t launch_norm(const NormParams& p, bool pdl, cudaStream_t s) {
+  auto a16 = [](const void* q) { return ((uintptr_t)q & 15u) == 0; };
+  const bool vec = a16(p.y_routed) && a16(p.y_shared) && a16(p.h) && a16(p.x_out) && a16(p.x_out_f32) &&
+                   a16(p.gamma) && p.H % 4 == 0 && p.y_routed_slot_stride % 4 == 0 && p.y_shared_split_stride % 4 == 0;
+  if (p.T >= 32 && vec) {   // enough tokens to fill the GPU with a CTA each (float4 rows)
+    NormParams q = p;
+    void* args[] = {&q};
+    return launch_ex((const void*)norm_rows_kernel, dim3(p.T), dim3(kNormRThreads), 0, s, pdl, args);
+  }
   cudaError_t e = set_smem((const void*)norm_cluster_kernel, 0);
   if (e != cudaSuccess) return e;
   NormParams q = p;

@@ -110,43 +110,53 @@ __host__ __device__ inline int tc_token_threads(int K) {
   return tw;
 }
 
-// One weight row: e with max(c|s_g|, |beta_g|) 2^e < 2^14 over all its groups,
-// then its bias columns (beta_hi, beta_lo, beta_hi, beta_lo per group, scaled
-// by 2^e) in the dense kernel's tile layout.
+// One weight row, one warp: e with max(c|s_g|, |beta_g|) 2^e < 2^14 over all
+// its groups, then its bias columns (beta_hi, beta_lo, beta_hi, beta_lo per
+// group, scaled by 2^e) in the dense kernel's tile layout. Lane l takes the
+// column chunks j = l + 32 q, chunk j holding groups 2j and 2j+1.
+constexpr int kTcPrepChunks = 2;   // chunks per lane: K <= 64 * 2 * 32 * kTcPrepChunks
 template <int BITS>
 __device__ void tc_prep_row(const TcRowPrep& P, int m) {
   constexpr float cq = BITS == 4 ? 8.f : 2.f;
+  const int lane = threadIdx.x & 31;
   const int ng = P.K / kGroup, nxs = tc_cols(P.K) / 64 - ng;
   const bool second = m >= P.R0;
   const moe_qmat W = second ? P.w1 : P.w0;
   const int r = second ? m - P.R0 : m;
-  const uint16_t* srow = W.scales + (size_t)r * ng;
-  const uint16_t* brow = W.biases + (size_t)r * ng;
+  const uint32_t* srow = (const uint32_t*)(W.scales + (size_t)r * ng);   // ng is even: bf16 pairs
+  const uint32_t* brow = (const uint32_t*)(W.biases + (size_t)r * ng);
+  float beta[kTcPrepChunks][2];
   float mx = 0.f;
-#pragma unroll 8
-  for (int g = 0; g < ng; ++g) {
-    const float sv = bf16_to_f32(__ldg(srow + g)), bv = bf16_to_f32(__ldg(brow + g));
-    mx = fmaxf(mx, fmaxf(cq * fabsf(sv), fabsf(fmaf(cq, sv, bv))));
+#pragma unroll
+  for (int q = 0; q < kTcPrepChunks; ++q) {
+    const int j = lane + 32 * q;
+    const bool in = j < ng / 2;
+    const uint32_t sv = in ? __ldg(srow + j) : 0u, bv = in ? __ldg(brow + j) : 0u;
+    const float s0 = bf16lo(sv), s1 = bf16hi(sv);
+    beta[q][0] = fmaf(cq, s0, bf16lo(bv));
+    beta[q][1] = fmaf(cq, s1, bf16hi(bv));
+    mx = fmaxf(mx, fmaxf(cq * fmaxf(fabsf(s0), fabsf(s1)), fmaxf(fabsf(beta[q][0]), fabsf(beta[q][1]))));
   }
+  mx = warp_max(mx);
   const int e = tc_exp_below(mx, 14);
-  P.rexp[m] = e;
+  if (lane == 0) P.rexp[m] = e;
   const float rsc = tc_pow2(e);
   uint4* tile = (uint4*)P.aext + (size_t)(m / kTcM) * nxs * 8 * kTcM + (m % kTcM);
-  for (int x = 0; x < nxs; ++x)
-#pragma unroll 2
-    for (int c = 0; c < 8; ++c) {
+#pragma unroll
+  for (int q = 0; q < kTcPrepChunks; ++q) {
+    const int j = lane + 32 * q;   // chunk j = stage j / 8, chunk j % 8 of it
+    if (j < nxs * 8) {
       uint32_t v[4];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int g = 16 * x + 2 * c + h;
-        float beta = 0.f;
-        if (g < ng) beta = fmaf(cq, bf16_to_f32(__ldg(srow + g)), bf16_to_f32(__ldg(brow + g))) * rsc;
-        const uint32_t hl = pack_half2(half_hi(beta), half_lo(beta));
+        const float bt = j < ng / 2 ? beta[q][h] * rsc : 0.f;
+        const uint32_t hl = pack_half2(half_hi(bt), half_lo(bt));
         v[2 * h] = hl;
         v[2 * h + 1] = hl;
       }
-      tile[(size_t)(x * 8 + c) * kTcM] = make_uint4(v[0], v[1], v[2], v[3]);
+      tile[(size_t)j * kTcM] = make_uint4(v[0], v[1], v[2], v[3]);
     }
+  }
 }
 
 template <int BITS>
@@ -156,8 +166,8 @@ __global__ void __launch_bounds__(kTcConvThreads) tc_conv_kernel(TcConvParams p)
   const int K = p.K, nsp = K / 16, ng = K / kGroup, nck = K / 8, nxk = tc_cols(K) / 8 - nck;
   const int tw = tc_token_threads(K), tpc = kTcConvThreads / tw;
   const int ntb = (p.Tpad + tpc - 1) / tpc;   // token CTAs
-  if ((int)blockIdx.x >= ntb) {   // ---------------------------------------- weight rows
-    int m = (blockIdx.x - ntb) * kTcConvThreads + tid;
+  if ((int)blockIdx.x >= ntb) {   // ---------------------------------------- weight rows, a warp each
+    int m = (blockIdx.x - ntb) * (kTcConvThreads / 32) + (tid >> 5);
     for (int j = 0; j < p.nprep; ++j) {
       if (m < p.prep[j].M) {
         tc_prep_row<BITS>(p.prep[j], m);
@@ -526,11 +536,13 @@ bool tc_supported(int H, int I, int bits) {
 
 cudaError_t launch_tc_conv(const TcConvParams& p, cudaStream_t s) {
   if (p.K % kGroup || p.K > 16 * kTcConvThreads * kTcConvSpans) return cudaErrorInvalidConfiguration;
+  for (int j = 0; j < p.nprep; ++j)
+    if (p.prep[j].K > 64 * 2 * 32 * kTcPrepChunks || p.prep[j].M % kTcM) return cudaErrorInvalidConfiguration;
   const void* fn = p.bits == 4 ? (const void*)tc_conv_kernel<4> : (const void*)tc_conv_kernel<2>;
   const int tpc = kTcConvThreads / tc_token_threads(p.K);
   int rows = 0;
   for (int j = 0; j < p.nprep; ++j) rows += p.prep[j].M;
-  const int nb = (p.Tpad + tpc - 1) / tpc + (rows + kTcConvThreads - 1) / kTcConvThreads;
+  const int nb = (p.Tpad + tpc - 1) / tpc + (rows + kTcConvThreads / 32 - 1) / (kTcConvThreads / 32);
   TcConvParams q = p;
   void* args[] = {&q};
   return cudaLaunchKernel(fn, dim3(nb), dim3(kTcConvThreads), args, 0, s);

@@ -141,6 +141,9 @@ def test_entry_points_reject_bad_arguments_before_launch():
     # combine: eps <= 0, shared output without gate
     assert L.moe_combine_residual_norm(1, 256, 2, p, p, None, None, p, p, C.c_float(0.0), p, None, None) == 1
     assert L.moe_combine_residual_norm(1, 256, 2, p, p, p, None, p, p, C.c_float(1e-6), p, None, None) == 1
+    # combine: H not a multiple of 8 or above 8192 is unsupported
+    assert L.moe_combine_residual_norm(1, 100, 2, p, p, None, None, p, p, C.c_float(1e-6), p, None, None) == 2
+    assert L.moe_combine_residual_norm(1, 16384, 2, p, p, None, None, p, p, C.c_float(1e-6), p, None, None) == 2
     # grouping: k > 8, E <= 0
     assert L.moe_group_tokens(4, 9, 16, p, p, p, p, None, 0, None) == 1
     assert L.moe_group_tokens(4, 2, 0, p, p, p, p, None, 0, None) == 1

@@ -213,8 +213,11 @@ def test_route_ties_resolve_to_lower_index(dev):
 
 
 # ------------------------------------------------------------------ combine + residual + RMSNorm
-@pytest.mark.parametrize("T,H,k,shared", [(1, 4096, 3, True), (5, 256, 2, True), (3, 384, 1, False)])
+@pytest.mark.parametrize("T,H,k,shared", [(1, 4096, 3, True), (5, 256, 2, True), (3, 384, 1, False),
+                                           (40, 4096, 3, True), (33, 8192, 8, False)])
 def test_combine_norm_matches_oracle(dev, T, H, k, shared):
+    """Up to 31 tokens the combine runs as clusters of eight CTAs per token, from 32 tokens up
+    (16-byte aligned buffers) as one CTA per token."""
     rng = np.random.default_rng(T * H + k)
     y = rng.normal(size=(T, k, H)).astype(np.float32)
     w = rng.dirichlet(np.ones(k), size=T).astype(np.float32)
