@@ -202,10 +202,14 @@ def kernel_bytes(cfg, name: str, layers: int = 1) -> int:
     return per * layers
 
 
-# the files that define each path's kernels (recorded ncu traffic is tied to their hash)
-DECODE_SOURCES = ("common.cuh", "kernels.cu", "kernels.cuh", "decode.cu", "fused.cu", "stage.cuh", "sync.cuh",
-                  "topk.cuh")
+# the files that define each kernel (its translation unit and the headers it includes); recorded
+# ncu traffic is tied to their hash
+DECODE_SOURCES = ("common.cuh", "kernels.cuh", "decode.cu", "stage.cuh", "sync.cuh", "topk.cuh")   # gate/up, down
+ROUTER_SOURCES = ("common.cuh", "kernels.cu", "kernels.cuh", "topk.cuh")                           # router, norm
+FUSED_SOURCES = ("common.cuh", "kernels.cuh", "fused.cu", "stage.cuh", "sync.cuh", "topk.cuh")
 PREFILL_SOURCES = ("common.cuh", "kernels.cuh", "prefill.cu")
+SOURCES_OF = {"route_logits_kernel": ROUTER_SOURCES, "norm_kernel": ROUTER_SOURCES,
+              "fused_decode_kernel": FUSED_SOURCES}
 
 
 def kernel_src_sha(files=DECODE_SOURCES):
@@ -458,7 +462,7 @@ def ours(args, cfg):
     j_dom = max(range(nk), key=lambda j: dur[j])
     dom_bytes = kernel_bytes(cfg, names[j_dom])
     achieved = dom_bytes / (dur[j_dom] * 1e-3) / 1e9
-    traffic = recorded_traffic(names[j_dom], cfg.name)
+    traffic = recorded_traffic(names[j_dom], cfg.name, SOURCES_OF.get(names[j_dom], DECODE_SOURCES))
     line = {
         "metric": METRIC, "value": tok_s, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": ms / args.steps, "higher_is_better": True,
