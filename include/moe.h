@@ -285,6 +285,51 @@ moe_status moe_layer_forward_noalloc(const moe_layer* layer, const uint16_t* x_i
  * earlier no-alloc calls (MOE_OK if none) and clears it. */
 moe_status moe_noalloc_poll_status(void* stream);
 
+/*
+ * Host-resident routed experts with an HBM expert cache ("Key technologies >
+ * SSD expert streaming" and "Trust the OS" of the Flash-MoE write-up: the
+ * experts live outside the GPU and the ones the router picks are loaded for
+ * each token). Here the routed experts live in host memory and HBM holds
+ * `slots` of them; a slot that has to be reused is the least recently used
+ * one (free slots first, the lowest index on ties). All memory is
+ * caller-owned:
+ *   host_experts  host array [E] of moe_expert whose q / scales / biases point
+ *                 to host memory (page-locked memory lets the copies overlap
+ *                 other work); it must stay valid while the cache is used;
+ *   dev           device memory of dev_bytes (256-byte aligned): the expert
+ *                 table [E] the kernels read, then the slots;
+ *   state         host memory of state_bytes (8-byte aligned): the
+ *                 bookkeeping.
+ * moe_cache_size: the two sizes for `layer` and `slots` (layer->experts is not
+ * read). moe_cache_init: empties the cache (host only, no device access).
+ */
+moe_status moe_cache_size(const moe_layer* layer, int32_t slots, size_t* dev_bytes, size_t* state_bytes);
+moe_status moe_cache_init(const moe_layer* layer, const moe_expert* host_experts, int32_t slots, void* dev,
+                          size_t dev_bytes, void* state, size_t state_bytes);
+
+/* The cache's bookkeeping for one call, host only (no copy, no device access):
+ * makes the n expert ids (duplicates allowed) resident and writes, per id, its
+ * slot and whether it had to be loaded (missed = 1 on the first id of each
+ * loaded expert, 0 otherwise). MOE_ERR_UNSUPPORTED when the call names more
+ * distinct experts than there are slots; MOE_ERR_INVALID_ARGUMENT for an id
+ * outside [0, E) or a state that moe_cache_init did not set up. */
+moe_status moe_cache_admit(void* state, const int32_t* ids, int32_t n, int32_t* slot, int32_t* missed);
+
+/* moe_layer_forward with the routed experts served from the cache: routes the
+ * T tokens on the GPU (moe_route), reads the chosen ids back (synchronises
+ * `stream`), admits them, copies each missing expert's nine arrays host -> HBM
+ * (one cudaMemcpyAsync per array) and its entry of the device expert table,
+ * then runs the layer as moe_layer_forward does, with layer->experts replaced
+ * by the cache's table. Arguments, workspace and errors otherwise those of
+ * moe_layer_forward; T * top_k <= 4096. */
+moe_status moe_layer_forward_cached(const moe_layer* layer, void* state, const uint16_t* x_in, float* h, int32_t T,
+                                    uint16_t* x_out, float* x_out_f32, int32_t* topk_idx, float* topk_w, void* ws,
+                                    size_t ws_bytes, void* stream);
+
+/* Counters of the cache since moe_cache_init: distinct experts found resident
+ * and loaded per call, and bytes copied host -> HBM. Pointers may be NULL. */
+moe_status moe_cache_stats(const void* state, uint64_t* hits, uint64_t* misses, uint64_t* bytes_copied);
+
 /* Synchronises `stream` and returns the status latched in the workspace by
  * earlier calls (MOE_OK if none). A latched status is cleared together with
  * the counters and flags of the workspace header (the first 256 bytes),

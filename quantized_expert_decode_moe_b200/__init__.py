@@ -84,6 +84,13 @@ def lib():
         L.moe_selftest_wait_timeout.argtypes = [vp, C.c_size_t, C.c_uint64, vp]
         L.moe_selftest_grid_timeout.argtypes = [vp, C.c_size_t, C.c_uint64, vp]
         L.moe_noalloc_poll_status.argtypes = [vp]
+        sz = C.POINTER(C.c_size_t)
+        u64 = C.POINTER(C.c_uint64)
+        L.moe_cache_size.argtypes = [vp, i32, sz, sz]
+        L.moe_cache_init.argtypes = [vp, vp, i32, vp, C.c_size_t, vp, C.c_size_t]
+        L.moe_cache_admit.argtypes = [vp, vp, i32, vp, vp]
+        L.moe_layer_forward_cached.argtypes = [vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, C.c_size_t, vp]
+        L.moe_cache_stats.argtypes = [vp, u64, u64, u64]
         _lib = L
     return _lib
 
@@ -278,6 +285,60 @@ def moe_poll_status(ws, stream=None) -> int:
 def moe_noalloc_poll_status(stream=None) -> int:
     """Status latched by earlier moe_layer_forward_noalloc calls on the current device (then cleared)."""
     return lib().moe_noalloc_poll_status(_stream(stream))
+
+
+# ------------------------------------------------------------------ host-resident experts, HBM cache
+def moe_cache_size(layer: Layer, slots: int):
+    """(device bytes, host state bytes) of an expert cache with `slots` slots for `layer`."""
+    d, h = C.c_size_t(0), C.c_size_t(0)
+    _ok(lib().moe_cache_size(layer.cref(), int(slots), C.byref(d), C.byref(h)), "moe_cache_size")
+    return d.value, h.value
+
+
+class ExpertCache:
+    """Caller-owned memory of an expert cache (see include/moe.h): the host experts' descriptor
+    array, the device buffer (expert table + slots) and the host bookkeeping. host_experts: list of
+    E Expert whose tensors are host (ideally pinned) memory; they must outlive the cache."""
+
+    def __init__(self, layer: Layer, host_experts, slots: int, device="cuda"):
+        import numpy as np
+        import torch
+        self.host_experts = host_experts
+        self._host_c = (_Expert * len(host_experts))(*[e.c() for e in host_experts])
+        dev_bytes, state_bytes = moe_cache_size(layer, slots)
+        self.dev = torch.zeros(dev_bytes, dtype=torch.uint8, device=device)
+        self.state = np.zeros((state_bytes + 7) // 8, dtype=np.uint64)
+        self.slots = slots
+        _ok(lib().moe_cache_init(layer.cref(), C.cast(self._host_c, C.c_void_p), int(slots), _ptr(self.dev),
+                                 dev_bytes, C.c_void_p(self.state.ctypes.data), self.state.nbytes), "moe_cache_init")
+
+    def state_ptr(self):
+        return C.c_void_p(self.state.ctypes.data)
+
+
+def moe_cache_admit(cache: ExpertCache, ids):
+    """Host bookkeeping of one call: (slot per id, missed per id) as int32 numpy arrays."""
+    import numpy as np
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    slot = np.empty_like(ids)
+    missed = np.empty_like(ids)
+    _ok(lib().moe_cache_admit(cache.state_ptr(), C.c_void_p(ids.ctypes.data), ids.size, C.c_void_p(slot.ctypes.data),
+                              C.c_void_p(missed.ctypes.data)), "moe_cache_admit")
+    return slot, missed
+
+
+def moe_cache_stats(cache: ExpertCache):
+    """(hits, misses, bytes copied) since the cache was set up."""
+    h, m, b = C.c_uint64(0), C.c_uint64(0), C.c_uint64(0)
+    _ok(lib().moe_cache_stats(cache.state_ptr(), C.byref(h), C.byref(m), C.byref(b)), "moe_cache_stats")
+    return h.value, m.value, b.value
+
+
+def moe_layer_forward_cached(layer: Layer, cache: ExpertCache, x_in, h, x_out, x_out_f32=None, topk_idx=None,
+                             topk_w=None, *, ws, stream=None):
+    _ok(lib().moe_layer_forward_cached(layer.cref(), cache.state_ptr(), _ptr(x_in), _ptr(h), x_in.shape[0],
+                                       _ptr(x_out), _ptr(x_out_f32), _ptr(topk_idx), _ptr(topk_w), _ptr(ws),
+                                       ws.numel(), _stream(stream)), "moe_layer_forward_cached")
 
 
 def moe_selftest_grid_timeout(ws, bound_ns: int, stream=None):
