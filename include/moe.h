@@ -132,11 +132,15 @@ moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
  * the router results select the experts to load — HN thread, Table 3 comment).
  *   logits = router_w . x (+ router_bias). The ranking is that of the plain
  *   fp64 definition (exact bf16 x bf16 products summed in index order from
- *   0, bias added last). The logits are computed faster, as fp64 sums in
- *   another order (T <= 8: a summation tree per token; T > 8: a GEMM over
- *   four slices of H), each with a rigorous bound on its distance to the
- *   definition (at H = 4096 about 2^-39 of sum|w x| when T <= 8, and of
- *   ||w||.||x|| when T > 8). The top-k is certified against the
+ *   0, bias added last). The logits are computed faster, each with a
+ *   rigorous bound on its distance to the definition: T <= 8 as fp64 sums
+ *   in a summation tree per token (bound about 2^-39 of sum|w x| at
+ *   H = 4096); T > 8 exactly, in integers on the tensor cores, on 22-bit
+ *   fixed-point forms of every router row and token (one power-of-two
+ *   scale each), the bound made of the rows' own rounding residuals
+ *   sum|v - v~| and the fp64 rounding of the sums (about 1e-7 on unit-scale
+ *   activations); the shared-gate logit is an fp64 sum of the exact
+ *   products. The top-k is certified against the
  *   bounds, and when two candidates are closer than them, every candidate
  *   near the k-th is recomputed as the definition and ranked again, so the
  *   indices are those of the definition;

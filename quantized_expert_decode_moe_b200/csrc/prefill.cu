@@ -466,164 +466,6 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_grouped_kernel(PrefillP
       pf_wait(&full[i % nst], (unsigned)(i / nst) & 1u, p.wait_ns, nullptr);
 }
 
-// ------------------------------------------------------------------ router of many tokens
-// Router logits of many tokens (prefill): a GEMM on the fp64 tensor cores
-// (mma.sync m8n8k4 .f64), split over kRgSplit slices of H (blockIdx.z). Every
-// product of two bf16 values is exact in fp64; each CTA writes its slice's
-// partial sums to lpart[slice][token][row]. Tile: 64 tokens x 64 router rows
-// per CTA of 4 warps, each warp 32 tokens x 32 rows = 4 x 4 MMA tiles;
-// operands staged in shared memory as doubles, k-major, 32 k at a time.
-// (A logit is then a sum over a tree of fp64 roundings; the bound on its
-// distance to the index-order definition is route_combine_kernel's.)
-constexpr int kRgTok = 64, kRgRows = 64, kRgK = 32, kRgThreads = 128;
-constexpr int kRgPad = 4;   // doubles of padding per staged k row
-
-// bf16 bit pattern -> double, exactly: normal values and zeros by moving the
-// fields (exponent bias 127 -> 1023), the rest through float.
-__device__ __forceinline__ double bf16_to_f64(uint32_t b) {
-  const uint32_t e = (b >> 7) & 0xFFu;
-  uint32_t hi = ((b & 0x8000u) << 16) | ((e + 896u) << 20) | ((b & 0x7Fu) << 13);
-  if ((b & 0x7FFFu) == 0u) hi = (b & 0x8000u) << 16;
-  else if (e == 0u || e == 0xFFu) return (double)__uint_as_float(b << 16);
-  return __hiloint2double((int)hi, 0);
-}
-
-// D (8x8) += A (8x4, row-major) * B (4x8, col-major) in fp64. Lane l holds
-// A[l/4][l%4], B[l%4][l/4] and D[l/4][2(l%4)], D[l/4][2(l%4)+1].
-__device__ __forceinline__ void mma_f64(double (&d)[2], double a, double b) {
-  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
-               : "+d"(d[0]), "+d"(d[1]) : "d"(a), "d"(b));
-}
-
-__global__ void __launch_bounds__(kRgThreads) route_gemm_kernel(RouteParams p) {
-  __shared__ __align__(16) double xs[kRgK][kRgTok + kRgPad];    // [k][token]
-  __shared__ __align__(16) double ws[kRgK][kRgRows + kRgPad];   // [k][row]
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int e0 = blockIdx.x * kRgRows, t0 = blockIdx.y * kRgTok, ks = blockIdx.z;
-  const int nrows = p.E + (p.has_shared ? 1 : 0);
-  const int kbeg = (int)((long long)p.H * ks / kRgSplit) & ~(kRgK - 1);
-  const int kend = ks + 1 == kRgSplit ? p.H : (int)((long long)p.H * (ks + 1) / kRgSplit) & ~(kRgK - 1);
-  const int wt = (warp & 1) * 32, we = (warp >> 1) * 32;   // the warp's tokens and rows inside the tile
-  double acc[4][4][2];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j][0] = acc[i][j][1] = 0.0;
-  // staging: thread tid loads one uint4 (8 k) of each of 2 tokens and 2 rows per tile
-  auto src_x = [&](int r) -> const uint16_t* { return t0 + r < p.T ? p.x + (size_t)(t0 + r) * p.H : nullptr; };
-  auto src_w = [&](int r) -> const uint16_t* {
-    const int e = e0 + r;
-    return e < p.E ? p.router_w + (size_t)e * p.H : (e < nrows ? p.gate_w : nullptr);
-  };
-  const int lr = tid >> 2, lc = tid & 3;   // rows lr and lr + 32, k chunk lc
-  const uint16_t* xa = src_x(lr);
-  const uint16_t* xb = src_x(lr + 32);
-  const uint16_t* wa = src_w(lr);
-  const uint16_t* wb = src_w(lr + 32);
-  auto ld = [&](const uint16_t* q, int k0) {
-    return q ? __ldg((const uint4*)(q + k0 + 8 * lc)) : make_uint4(0u, 0u, 0u, 0u);
-  };
-  auto put = [&](double (*dst)[kRgTok + kRgPad], int col, uint4 v) {
-    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      dst[8 * lc + 2 * i][col] = bf16_to_f64(u[i] & 0xFFFFu);
-      dst[8 * lc + 2 * i + 1][col] = bf16_to_f64(u[i] >> 16);
-    }
-  };
-  uint4 v0, v1, v2, v3;
-  if (kbeg < kend) { v0 = ld(xa, kbeg); v1 = ld(xb, kbeg); v2 = ld(wa, kbeg); v3 = ld(wb, kbeg); }
-  for (int k0 = kbeg; k0 < kend; k0 += kRgK) {
-    __syncthreads();   // the previous tile has been read
-    put(xs, lr, v0); put(xs, lr + 32, v1); put(ws, lr, v2); put(ws, lr + 32, v3);
-    __syncthreads();
-    if (k0 + kRgK < kend) {   // next tile in flight during the products
-      v0 = ld(xa, k0 + kRgK); v1 = ld(xb, k0 + kRgK); v2 = ld(wa, k0 + kRgK); v3 = ld(wb, k0 + kRgK);
-    }
-#pragma unroll
-    for (int kk = 0; kk < kRgK; kk += 4) {
-      double af[4], bf[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) af[i] = xs[kk + (lane & 3)][wt + 8 * i + (lane >> 2)];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) bf[j] = ws[kk + (lane & 3)][we + 8 * j + (lane >> 2)];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) mma_f64(acc[i][j], af[i], bf[j]);
-    }
-  }
-  const size_t ldl = (size_t)p.E + 1;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int t = t0 + wt + 8 * i + (lane >> 2);
-    if (t >= p.T) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const int e = e0 + we + 8 * j + 2 * (lane & 3) + c;
-        if (e < nrows) p.lpart[((size_t)ks * p.T + t) * ldl + e] = acc[i][j][c];
-      }
-  }
-}
-
-// Squared norms of the router rows (incl. the shared-gate row) and of the
-// tokens' activations, in fp64 (exact squares): one warp per vector.
-__global__ void __launch_bounds__(256) route_norms_kernel(RouteParams p) {
-  const int v = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-  const int nrows = p.E + (p.has_shared ? 1 : 0);
-  if (v >= nrows + p.T) return;
-  const uint16_t* q = v < p.E ? p.router_w + (size_t)v * p.H : (v < nrows ? p.gate_w : p.x + (size_t)(v - nrows) * p.H);
-  double s = 0.0;
-  for (int c = lane; c < p.H / 8; c += 32) {
-    const uint4 u = __ldg((const uint4*)(q + 8 * c));
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const double lo = bf16_to_f64(w[i] & 0xFFFFu), hi = bf16_to_f64(w[i] >> 16);
-      s = fma(lo, lo, s);
-      s = fma(hi, hi, s);
-    }
-  }
-  s = warp_sum_f64(s);
-  if (lane == 0) {
-    if (v < nrows) p.wn2[v] = s;
-    else p.xn2[v - nrows] = s;
-  }
-}
-
-// Logits of many tokens from the router GEMM's slices: l = sum of the
-// slices' partial sums in slice order + bias (fp64), written to
-// logits[t][e], and a certified bound on |l - definition| to bound[t][e].
-// Every product is exact and every sum a tree of at most H + 1 fp64
-// roundings. Taking u = 2^-52 (twice the unit roundoff, so that the bound
-// holds for a rounding of the tensor cores' fp64 accumulation that is merely
-// faithful), both l and the index-order definition are within
-// (H + 1) u / (1 - (H + 1) u) sum |w x| of the exact value, and
-// sum |w x| <= ||w_e|| ||x_t|| (Cauchy-Schwarz). The squared norms are fp64
-// sums of exact squares (relative error below (H + 1) 2^-53); the factor 1.25
-// and the term 2^-50 (|l| + |b|) cover the roundings of the norms, of the
-// bias additions and of the bound itself. Grid T, block 512.
-__global__ void __launch_bounds__(kThreads) route_combine_kernel(RouteParams p) {
-  const int t = blockIdx.x;
-  const size_t ld = (size_t)p.E + 1;
-  const double xn = p.xn2[t];
-  const int nrows = p.E + (p.has_shared ? 1 : 0);
-  for (int e = threadIdx.x; e < nrows; e += blockDim.x) {
-    double l = 0.0;
-    for (int q = 0; q < kRgSplit; ++q) l += p.lpart[((size_t)q * p.T + t) * ld + e];
-    const double bias = (e < p.E && p.router_bias) ? (double)p.router_bias[e] : 0.0;
-    l += bias;
-    p.logits[(size_t)t * ld + e] = l;
-    if (e < p.E) {
-      const double nn = (double)p.H;
-      const double b = 1.25 * 2.0 * (nn + 2.0) * 0x1p-52 * sqrt(p.wn2[e] * xn) + 0x1p-50 * (fabs(l) + fabs(bias));
-      p.bound[(size_t)t * ld + e] = __double2float_ru(b);
-    }
-  }
-}
-
 // ------------------------------------------------------------------ grouping by expert
 // Exclusive scan of v[0..n) in place (one block); returns the total.
 __device__ int block_exclusive_scan(int* v, int n, int* warp_tot) {
@@ -738,17 +580,6 @@ cudaError_t launch_group(const GroupParams& p, cudaStream_t s) {
   return cudaLaunchKernel((const void*)group_kernel, dim3(1), dim3(1024), args, sm, s);
 }
 
-cudaError_t launch_route_gemm(const RouteParams& p, cudaStream_t s) {
-  const int rows = p.E + (p.has_shared ? 1 : 0);
-  dim3 grid((rows + kRgRows - 1) / kRgRows, (p.T + kRgTok - 1) / kRgTok, kRgSplit);
-  RouteParams q = p;
-  void* args[] = {&q};
-  cudaError_t e = cudaLaunchKernel((const void*)route_gemm_kernel, grid, dim3(kRgThreads), args, 0, s);
-  if (e != cudaSuccess) return e;
-  e = cudaLaunchKernel((const void*)route_norms_kernel, dim3((rows + p.T + 7) / 8), dim3(256), args, 0, s);
-  if (e != cudaSuccess) return e;
-  return cudaLaunchKernel((const void*)route_combine_kernel, dim3(p.T), dim3(kThreads), args, 0, s);
-}
 
 int pf_chunk_tokens(int H, int I) { return (H > 4096 || I > 4096) ? 4 : 8; }
 

@@ -136,11 +136,13 @@ def test_route_matches_oracle(dev, name):
 
 
 def test_route_logits_within_their_bound_of_the_fp64_definition(dev):
-    """Many tokens (T > 8): the router GEMM sums four slices of H in fp64, so
-    a logit may differ from the plain index-order fp64 loop of the definition
-    in its last bits; every logit must lie within the certified bound the
-    library stores beside it (2 (H+2) 2^-53 ||w|| ||x|| + 2^-50 (|l| + |b|),
-    with a margin), and the ranking must be the definition's. moe_route leaves
+    """Many tokens (T > 8): a logit is computed in exact integer arithmetic on
+    22-bit fixed-point forms of w and x (one power-of-two scale per router row
+    and per token), so it differs from the plain index-order fp64 loop of the
+    definition by at most the rounding of that fixed point and of the fp64
+    sums; every logit must lie within the certified bound the library stores
+    beside it, and the ranking must be the definition's. The shared-gate logit
+    is an fp64 sum of exact products. moe_route leaves
     the logits in the workspace: double [T][E+1] at byte 256, column E the
     shared-gate logit; the bounds follow as float [T][E+1]."""
     cfg = fixtures.CONFIGS["stack_q4"]   # the biased router
@@ -165,7 +167,9 @@ def test_route_logits_within_their_bound_of_the_fp64_definition(dev):
     ridx, _, _, ref = oracle.route(x, Wr, cfg.k, bias=rb, want_logits=True)
     err = np.abs(got[:, :cfg.E] - ref)
     assert np.all(err <= bnd.astype(np.float64))
-    assert np.all(bnd < 1e-9)
+    # the bound is built from each row's own rounding residuals sum|v - v~| (most
+    # bf16 values are exact in 22-bit fixed point) and the fp64 sums' rounding
+    assert np.all(bnd < 1e-5)
     np.testing.assert_array_equal(idx.cpu().numpy(), ridx)
     _, _, _, ref_g = oracle.route(x, gs[None, :], 1, want_logits=True)
     assert np.max(np.abs(got[:, cfg.E] - ref_g[:, 0])) <= 1e-9
