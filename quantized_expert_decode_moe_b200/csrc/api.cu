@@ -227,7 +227,7 @@ moe_status prefill_chain(const moe_layer* L, const uint16_t* x_in, float* h, int
   rp.x = x_in; rp.router_w = L->router_w; rp.router_bias = L->router_bias; rp.gate_w = L->shared_gate_w;
   rp.logits = at<double>(ws, W.logits);
   rp.bound = at<float>(ws, W.bound);
-  rp.lpart = at<double>(ws, W.lpart);
+  rp.lpart = at<long long>(ws, W.lpart);
   rp.wdig = at<int8_t>(ws, W.wdig); rp.xdig = at<int8_t>(ws, W.xdig);
   rp.wst = at<double>(ws, W.wst); rp.xst = at<double>(ws, W.xst);
   rp.status = at<uint32_t>(ws, W.status); rp.wait_ns = wait_bound_ns();
@@ -381,7 +381,7 @@ moe_status moe_route(const moe_layer* layer, const uint16_t* x, int32_t T, int32
   rp.x = x; rp.router_w = layer->router_w; rp.router_bias = layer->router_bias; rp.gate_w = layer->shared_gate_w;
   rp.logits = at<double>(ws, W.logits);
   rp.bound = at<float>(ws, W.bound);
-  rp.lpart = at<double>(ws, W.lpart);
+  rp.lpart = at<long long>(ws, W.lpart);
   rp.wdig = at<int8_t>(ws, W.wdig); rp.xdig = at<int8_t>(ws, W.xdig);
   rp.wst = at<double>(ws, W.wst); rp.xst = at<double>(ws, W.xst);
   rp.status = at<uint32_t>(ws, W.status); rp.wait_ns = wait_bound_ns();

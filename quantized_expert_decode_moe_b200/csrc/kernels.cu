@@ -42,12 +42,12 @@ WsLayout ws_layout(int H, int I, int E, int k, int S, int T) {
   L.chunks = o; o = align256(o + (T > 8 ? sizeof(int4) * pf_max_chunks(T, k, E, pf_chunk_tokens(H, I)) : 0));
   L.nchunks = o; o = align256(o + (T > 8 ? sizeof(int32_t) : 0));
   L.y = o; o = align256(o + sizeof(float) * prows * H);
-  L.lpart = o; o = align256(o + (T > 8 ? sizeof(double) * kRgSplit * (size_t)T * (E + 1) : 0));
+  L.lpart = o; o = align256(o + (T > 8 ? sizeof(long long) * kRtSplitMax * (size_t)T * E : 0));
   const size_t rw = T > 8 ? route_tc_rows_w(E) : 0, rx = T > 8 ? route_tc_rows_x(T) : 0;
   L.wdig = o; o = align256(o + 3 * rw * (size_t)H);
   L.xdig = o; o = align256(o + 3 * rx * (size_t)H);
-  L.wst = o; o = align256(o + sizeof(double) * 4 * rw);
-  L.xst = o; o = align256(o + sizeof(double) * 4 * rx);
+  L.wst = o; o = align256(o + sizeof(double) * 8 * rw);
+  L.xst = o; o = align256(o + sizeof(double) * 8 * rx);
   const size_t tpad = T > 8 ? (size_t)((T + 15) & ~15) : 0;
   L.tcbx = o; o = align256(o + 2 * tpad * tc_cols(H));
   L.tcxs = o; o = align256(o + sizeof(float) * tpad);

@@ -10,7 +10,7 @@
 namespace qmoe {
 
 constexpr int kMaxCtas = 1024;   // CTAs of the fused decode kernel at most
-constexpr int kRgSplit = 4;      // slices of H in the many-token router GEMM
+constexpr int kRtSplitMax = 12;  // column splits of the many-token router GEMM at most
 constexpr size_t kSelFlagOffset = 80;   // byte offset of the decode chain's selection flags (8 words)
 
 // Workspace carve-up for T tokens of one layer shape. The first 256 bytes are
@@ -39,9 +39,9 @@ struct WsLayout {
   size_t chunks;      // int4 [max chunks] (expert, first position, tokens, 0)
   size_t nchunks;     // int32
   size_t y;           // float [T*k + T][H] expert outputs, same rows
-  size_t lpart;       // double [kRgSplit][T][E+1] partial router logits (T > 8)
+  size_t lpart;       // int64 [kRtSplitMax][T][E] exact partial router sums (T > 8)
   size_t wdig, xdig;  // int8 digit planes of the router rows and of x (T > 8)
-  size_t wst, xst;    // double [rows][4] their scales, sums, maxima and rounding residuals (T > 8)
+  size_t wst, xst;    // double [rows][8] their scales, sums, maxima, rounding residuals, low digits (T > 8)
   // shared expert on the tensor cores (T > 8): fp16 operand tables of x and of its SwiGLU
   // outputs (hi, lo) [Kx/8][Tpad][8], per-token scales [Tpad], split partial sums
   size_t tcbx, tcxs, tcbah, tcbal, tcas, tcpart;
@@ -58,10 +58,11 @@ struct RouteParams {
   const uint16_t* gate_w;       // [H] or null
   double* logits;               // [T][E+1]
   float* bound;                 // [T][E+1]: bound on |logit - fp64 definition| (null: not written)
-  // many tokens (route_tc.cu): per-split partial logits [kRgSplit][T][E+1]; the router rows' and
-  // tokens' digit planes (3 x [H/16][rows][16] int8, rows padded) and per-row statistics
-  // {2^-p, sum |v|, max |v|, sum |v - V 2^-p|}
-  double* lpart;
+  // many tokens (route_tc.cu): per-split exact partial sums [kRtSplitMax][T][E]; the router
+  // rows' and tokens' digit planes (int8, rows padded to 128, tiled: 128-row tile, 64-column
+  // stage, plane, 16-column chunk, row) and per-row statistics {2^-p, sum |v|, max |v|,
+  // sum |v - V 2^-p|, sum |d0|, max |d0|, 0, 0}
+  long long* lpart;
   int8_t* wdig; int8_t* xdig; double* wst; double* xst;
   uint32_t* status; unsigned long long wait_ns;   // bound of the tcgen05 router's waits
   // side job of the decode chain (null when unused): copies of the layer's inputs x, h ([T][H])
@@ -242,9 +243,9 @@ struct FusedParams {
 // launchers (return the launch's cudaError_t)
 cudaError_t launch_route(const RouteParams& p, cudaStream_t s, bool pdl);
 cudaError_t launch_route_gemm(const RouteParams& p, cudaStream_t s);   // many tokens: exact integer tcgen05
-// router rows (incl. the shared-gate row) and tokens, padded to the tcgen05 router's tiles
-__host__ __device__ inline size_t route_tc_rows_w(int E) { return (size_t)((E + 1 + 127) / 128) * 128; }
-__host__ __device__ inline size_t route_tc_rows_x(int T) { return (size_t)((T + 63) / 64) * 64; }
+// router rows and tokens, padded to the tcgen05 router's 128 x 128 tiles
+__host__ __device__ inline size_t route_tc_rows_w(int E) { return (size_t)((E + 127) / 128) * 128; }
+__host__ __device__ inline size_t route_tc_rows_x(int T) { return (size_t)((T + 127) / 128) * 128; }
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t s);
 cudaError_t launch_gateup(const GateUpParams& p, int bits, int T, bool pdl, cudaStream_t s);
 cudaError_t launch_down(const DownParams& p, int bits, int T, bool pdl, cudaStream_t s);
