@@ -50,6 +50,12 @@ def lib():
         _lib.oracle_silu.argtypes = [C.c_double]
         _lib.oracle_sigmoid.restype = C.c_double
         _lib.oracle_sigmoid.argtypes = [C.c_double]
+        _lib.oracle_e2m1.restype = C.c_double
+        _lib.oracle_e2m1.argtypes = [C.c_uint]
+        _lib.oracle_e8m0.restype = C.c_double
+        _lib.oracle_e8m0.argtypes = [C.c_uint]
+        _lib.oracle_mx_weight.restype = C.c_double
+        _lib.oracle_mx_weight.argtypes = [C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_int]
         _lib.oracle_weight.restype = C.c_double
         _lib.oracle_weight.argtypes = [C.c_void_p, C.c_void_p, C.c_void_p] + [C.c_int] * 5
         _lib.oracle_combine_norm.argtypes = [C.c_int, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p,
@@ -107,6 +113,44 @@ def qgemv(q, s, b, x, K: int, G: int, bits: int) -> np.ndarray:
     if rc:
         raise ValueError("oracle_qgemv: invalid arguments")
     return y
+
+
+def e2m1(code: int) -> float:
+    """Value of a 4-bit FP4 E2M1 code (MXFP4 element)."""
+    return lib().oracle_e2m1(int(code))
+
+
+def e8m0(byte: int) -> float:
+    """Value of an E8M0 scale byte (MXFP4 block scale); NaN for 0xFF."""
+    return lib().oracle_e8m0(int(byte))
+
+
+def mx_dequant(q, e, K: int) -> np.ndarray:
+    """MXFP4 matrix (codes uint32 [R][K/8], scales uint8 [R][K/32]) as double [R][K]."""
+    q = _c(q, np.uint32); e = _c(e, np.uint8)
+    R = e.shape[0]
+    w = np.empty((R, K), dtype=np.float64)
+    if lib().oracle_mx_dequant(R, K, _p(q), _p(e), _p(w)):
+        raise ValueError("oracle_mx_dequant: invalid arguments")
+    return w
+
+
+def mx_gemv(q, e, x, K: int) -> np.ndarray:
+    """y = W x for an MXFP4 matrix W, index-order double sums."""
+    q = _c(q, np.uint32); e = _c(e, np.uint8); x = _c(x, np.float64)
+    R = e.shape[0]
+    y = np.empty(R, dtype=np.float64)
+    if lib().oracle_mx_gemv(R, K, _p(q), _p(e), _p(x), _p(y)):
+        raise ValueError("oracle_mx_gemv: invalid arguments")
+    return y
+
+
+def mx_gemm(q, e, x, K: int) -> np.ndarray:
+    """Y[t] = W x[t] for every row of x (bf16 bits [T][K] or doubles): the dequantised
+    matrix (double) times the activations by one library matrix product."""
+    x = np.asarray(x)
+    xd = bf16_to_f64(x) if x.dtype == np.uint16 else x.astype(np.float64)
+    return xd @ mx_dequant(q, e, K).T
 
 
 def swiglu(g, u) -> np.ndarray:

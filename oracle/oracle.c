@@ -314,3 +314,53 @@ done:
   free(sgate); free(xd); free(yr); free(ys);
   return rc;
 }
+
+/*
+ * MXFP4 expert matrices (page 4, "300b on 32gb MoE-streaming findings +
+ * optimisations": the streamed experts are MXFP4). The pages name the format
+ * only; the reading is the OCP Microscaling Formats (MX) v1.0 definition:
+ *   - a block of 32 consecutive k of a row shares one scale, E8M0: an 8-bit
+ *     biased exponent, value 2^(byte - 127), byte 0xFF = NaN;
+ *   - each element is FP4 E2M1: bit 3 sign, bits 2..1 exponent (bias 1),
+ *     bit 0 mantissa; exponent field 0 is subnormal (0.5 * mantissa),
+ *     otherwise 2^(exponent - 1) * (1 + mantissa / 2); no infinities or NaN;
+ *   - weight = scale * element.
+ * Layout (same packing as the 4-bit codes): codes uint32 [R][K/8], element k
+ * of a row in word k/8 at bits 4*(k%8), LSB first; scales uint8 [R][K/32].
+ */
+double oracle_e2m1(unsigned code) {
+  const unsigned s = (code >> 3) & 1u, e = (code >> 1) & 3u, m = code & 1u;
+  const double mag = e == 0 ? 0.5 * (double)m : ldexp(1.0 + 0.5 * (double)m, (int)e - 1);
+  return s ? -mag : mag;
+}
+
+double oracle_e8m0(unsigned byte) {
+  if ((byte & 0xFFu) == 0xFFu) return NAN;
+  return ldexp(1.0, (int)(byte & 0xFFu) - 127);
+}
+
+/* Weight (r, k) of an MXFP4 matrix, exact in double. */
+double oracle_mx_weight(const uint32_t* q, const uint8_t* e, int K, int r, int k) {
+  const unsigned code = code_at(q, K, 4, r, k);
+  return oracle_e2m1(code) * oracle_e8m0(e[(size_t)r * (size_t)(K / 32) + (size_t)(k / 32)]);
+}
+
+/* Dense dequantisation of an MXFP4 matrix into double [R][K]. */
+int oracle_mx_dequant(int R, int K, const uint32_t* q, const uint8_t* e, double* w) {
+  if (R < 0 || K <= 0 || K % 32) return ORC_EINVAL;
+  for (int r = 0; r < R; ++r)
+    for (int k = 0; k < K; ++k) w[(size_t)r * K + k] = oracle_mx_weight(q, e, K, r, k);
+  return ORC_OK;
+}
+
+/* y[r] = sum_k w[r][k] x[k] for an MXFP4 matrix, naive, index order, in double. */
+int oracle_mx_gemv(int R, int K, const uint32_t* q, const uint8_t* e, const double* x, double* y) {
+  if (R < 0 || K <= 0 || K % 32) return ORC_EINVAL;
+#pragma omp parallel for schedule(static)
+  for (int r = 0; r < R; ++r) {
+    double acc = 0.0;
+    for (int k = 0; k < K; ++k) acc += oracle_mx_weight(q, e, K, r, k) * x[k];
+    y[r] = acc;
+  }
+  return ORC_OK;
+}

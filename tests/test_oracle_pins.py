@@ -378,3 +378,109 @@ def test_fixture_streams_are_counter_based():
     np.testing.assert_array_equal(a[60:], b)
     z = gen.bf16_bits_to_f32(gen.normal_bf16(gen.key_of(0, 0, gen.T_X), 200_000, 1.0))
     assert abs(z.mean()) < 0.01 and abs(z.std() - 1.0) < 0.01
+
+
+# ---------------------------------------------------------------- MXFP4 (third codec)
+def _mx_table():
+    """The MX encodings of tests/golden/mx_formats.txt: {code: Fraction}, {byte: Fraction or None}."""
+    import os
+    e2m1, e8m0, block = {}, {}, None
+    with open(os.path.join(os.path.dirname(__file__), "golden", "mx_formats.txt")) as f:
+        for line in f:
+            t = line.split()
+            if not t or t[0].startswith("#"):
+                continue
+            if t[0] == "block":
+                block = int(t[1])
+            elif t[0] == "e2m1":
+                e2m1[int(t[1].replace(".", ""), 2)] = (t[2].startswith("-"), Fraction(t[2].lstrip("-")))
+            elif t[0] == "e8m0":
+                e8m0[int(t[1])] = None if t[2] == "nan" else Fraction(2) ** int(t[2].split("^")[1])
+    return e2m1, e8m0, block
+
+
+def test_mx_element_and_scale_values_match_the_format():
+    """Every E2M1 code and the tabulated E8M0 bytes decode to the values of the MX format
+    (signed zero included: code 1.00.0 is -0)."""
+    e2m1, e8m0, block = _mx_table()
+    assert block == 32 and len(e2m1) == 16
+    for code, (neg, mag) in e2m1.items():
+        v = oracle.e2m1(code)
+        assert Fraction(abs(v)) == mag and np.signbit(v) == neg, code
+    for byte, val in e8m0.items():
+        v = oracle.e8m0(byte)
+        assert (np.isnan(v) if val is None else Fraction(v) == val), byte
+    for byte in range(255):   # every non-NaN byte: consecutive powers of two
+        assert oracle.e8m0(byte + 1) == 2.0 * oracle.e8m0(byte) or byte == 254
+
+
+def mx_dense_by_table(q, e, K):
+    """MXFP4 matrix as exact Fractions from the format table and a bit-string unpacking."""
+    e2m1, e8m0, block = _mx_table()
+    R = q.shape[0]
+    W = [[None] * K for _ in range(R)]
+    for r in range(R):
+        c = codes_by_bitstring(q[r], 4)
+        for k in range(K):
+            neg, mag = e2m1[int(c[k])]
+            b = int(e[r][k // block])   # bytes between the tabulated ones: consecutive powers of two
+            W[r][k] = (-mag if neg else mag) * e8m0[127] * Fraction(2) ** (b - 127)
+    return W
+
+
+def test_mx_dequant_and_gemv_brute_force():
+    """A small random MXFP4 matrix (all 16 codes, scale bytes 100..140): the oracle's
+    dequantised weights equal the table's exactly, and its mat-vec equals the exact
+    rational dot products within one rounding per term."""
+    rng = np.random.default_rng(11)
+    R, K = 5, 96
+    q = rng.integers(0, 2**32, size=(R, K // 8), dtype=np.uint64).astype(np.uint32)
+    e = rng.integers(100, 141, size=(R, K // 32)).astype(np.uint8)
+    Wt = mx_dense_by_table(q, e, K)
+    Wo = oracle.mx_dequant(q, e, K)
+    for r in range(R):
+        for k in range(K):
+            assert Fraction(Wo[r, k]) == Wt[r][k], (r, k)
+    xb = gen.f32_to_bf16_bits(rng.standard_normal(K).astype(np.float32))
+    x = [bf16_exact(int(b)) for b in xb]
+    y = oracle.mx_gemv(q, e, gen.bf16_bits_to_f32(xb).astype(np.float64), K)
+    for r in range(R):
+        exact = sum(Wt[r][k] * x[k] for k in range(K))
+        mag = sum(abs(Wt[r][k] * x[k]) for k in range(K))
+        assert abs(Fraction(y[r]) - exact) <= mag * Fraction(K, 2**52), r
+
+
+def test_mx_one_code_and_one_scale_land_where_the_layout_says():
+    """A matrix with a single nonzero code (element k of row r) gives y[r] = value * x[k] and
+    zero elsewhere; raising that block's scale byte by one doubles it. A wrong nibble order,
+    word index or block index moves or loses the term."""
+    R, K = 3, 128
+    x = np.arange(1, K + 1, dtype=np.float64)
+    for (r, k, code) in [(0, 0, 0x2), (1, 37, 0xF), (2, 127, 0x5), (1, 64, 0x9)]:
+        q = np.zeros((R, K // 8), dtype=np.uint32)
+        q[r, k // 8] = np.uint32(code << (4 * (k % 8)))
+        e = np.full((R, K // 32), 127, dtype=np.uint8)
+        y = oracle.mx_gemv(q, e, x, K)
+        want = np.zeros(R)
+        want[r] = oracle.e2m1(code) * x[k]
+        np.testing.assert_array_equal(y, want)
+        e[r, k // 32] += 1
+        np.testing.assert_array_equal(oracle.mx_gemv(q, e, x, K), 2 * want)
+        e[r, k // 32] -= 1
+        e[r, (k // 32 + 1) % (K // 32)] += 5   # another block's scale: no effect
+        np.testing.assert_array_equal(oracle.mx_gemv(q, e, x, K), want)
+
+
+def test_mx_gemm_rows_are_the_gemv():
+    """The batched form (dequantised matrix times the tokens by one library product) agrees with
+    the index-order mat-vec on every token, to the rounding of two summation orders."""
+    rng = np.random.default_rng(12)
+    R, K, T = 16, 256, 5
+    q = rng.integers(0, 2**32, size=(R, K // 8), dtype=np.uint64).astype(np.uint32)
+    e = rng.integers(118, 126, size=(R, K // 32)).astype(np.uint8)
+    xb = gen.f32_to_bf16_bits(rng.standard_normal((T, K)).astype(np.float32))
+    Y = oracle.mx_gemm(q, e, xb, K)
+    W = oracle.mx_dequant(q, e, K)
+    for t in range(T):
+        y = oracle.mx_gemv(q, e, gen.bf16_bits_to_f32(xb[t]).astype(np.float64), K)
+        np.testing.assert_allclose(Y[t], y, rtol=0, atol=1e-13 * np.abs(W).sum(1).max() * 8)
