@@ -43,6 +43,8 @@ T_SHARED_GATE = 4
 T_GAMMA = 5
 T_CODES = 16      # + matrix index (0 gate, 1 up, 2 down)
 T_SCALES = 32     # + matrix index
+T_MX_CODES = 48   # MXFP4 matrices
+T_MX_SCALES = 49
 
 
 def _mix64_int(z: int) -> int:
@@ -244,3 +246,18 @@ def host_expert(cfg: Config, layer: int, expert: int):
         b = biases_from_scales(s, cfg.bits)
         out.append((q, s, b))
     return tuple(out)
+
+
+def mx_matrix(seed: int, R: int, K: int, scale_lo: int = 118, scale_hi: int = 124):
+    """A synthetic MXFP4 matrix (no model weights): codes uint32 [R][K/8], one uniform 32-bit word
+    per eight 4-bit codes (all sixteen E2M1 codes equally likely), and E8M0 scale bytes uint8
+    [R][K/32] uniform in [scale_lo, scale_hi] (default 2^-9 .. 2^-3)."""
+    q = codes_words(key_of(seed, 0, T_MX_CODES), R * K // 8).reshape(R, K // 8)
+    u = u64_stream(key_of(seed, 0, T_MX_SCALES), 0, R * K // 32)
+    e = (np.uint64(scale_lo) + u % np.uint64(scale_hi - scale_lo + 1)).astype(np.uint8).reshape(R, K // 32)
+    return q, e
+
+
+def mx_tokens(seed: int, T: int, K: int, sigma: float = 1.0) -> np.ndarray:
+    """T rows of K normal bf16 activations (bit patterns, uint16 [T][K])."""
+    return normal_bf16(key_of(seed, 0, T_X, 7), T * K, sigma).reshape(T, K)

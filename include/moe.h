@@ -170,6 +170,53 @@ moe_status moe_expert_gemv_q2(const moe_qmat* W, int32_t R, int32_t K, int32_t g
                               const float* x, float* y, void* stream);
 
 /*
+ * MXFP4 expert matrices (the experts' format on "300b on 32gb MoE-streaming
+ * findings + optimisations"), read as the OCP Microscaling (MX) v1.0 format:
+ * FP4 E2M1 elements (values 0, 0.5, 1, 1.5, 2, 3, 4, 6 and negatives), one
+ * E8M0 scale 2^(byte - 127) per 32 consecutive k of a row (byte 0xFF: NaN);
+ * weight = scale * element.
+ *   q: uint32 [R][K/8], element k of a row in word k/8 at bits 4*(k%8), LSB
+ *      first (the 4-bit packing); 16-byte aligned.
+ *   scales: uint8 [R][K/32].
+ */
+typedef struct {
+  const uint32_t* q;
+  const uint8_t* scales;
+} moe_mxmat;
+
+/*
+ * y = W x for one MXFP4 matrix (decode). R >= 1, K a multiple of 32 and at
+ * most 8192 (MOE_ERR_UNSUPPORTED above); x fp32 [K] (16-byte aligned); y fp32
+ * [R], overwritten. Element products and block sums in fp32, each block sum
+ * times its scale. Asynchronous on `stream`; no workspace.
+ */
+moe_status moe_expert_gemv_mxfp4(const moe_mxmat* W, int32_t R, int32_t K, const float* x, float* y,
+                                 void* stream);
+
+/* Bytes of workspace moe_expert_gemm_mxfp4 needs for R x K and T tokens
+ * (R and K multiples of 128, K <= 8192: else MOE_ERR_UNSUPPORTED). */
+moe_status moe_mxfp4_workspace_size(int32_t R, int32_t K, int32_t T, size_t* bytes);
+
+/*
+ * Y[t][r] = sum_k W[r][k] x[t][k] for T tokens (prefill-shaped expert GEMM) on
+ * the tcgen05 tensor cores with block scaling (kind::mxf4): the codes are used
+ * as stored and the hardware applies the E8M0 scales. Each token's bf16 row is
+ * written as a sum of five E2M1 terms, each with its own E8M0 scale per
+ * 32-block, exact up to a residual below 4^-4/3 of the block's largest
+ * |x| (about 5e-5 of the output's norm on unit-scale activations); fp32
+ * accumulation in tensor memory.
+ *   R, K multiples of 128, K <= 8192; x bf16 [T][K] (16-byte aligned); y fp32
+ *   [T][R], overwritten; W.q 16-byte aligned, W.scales 4-byte aligned.
+ *   ws: caller-owned device memory of moe_mxfp4_workspace_size bytes, 256-byte
+ *   aligned, header cleared by moe_workspace_init; a bounded wait that runs out
+ *   latches MOE_ERR_TIMEOUT there (moe_poll_status), and Y is then invalid.
+ *   Errors before any launch: MOE_ERR_INVALID_ARGUMENT, MOE_ERR_UNSUPPORTED,
+ *   MOE_ERR_WORKSPACE (ws_bytes too small).
+ */
+moe_status moe_expert_gemm_mxfp4(const moe_mxmat* W, int32_t R, int32_t K, const uint16_t* x, int32_t T,
+                                 float* y, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Combine + residual + RMSNorm ("MoE combine + residual + gate", "normalisation +
  * residual ... passed directly to the next layer"):
  *   h'[t] = h[t] + sum_i topk_w[t][i] * y_routed[t][i] + shared_gate[t] * y_shared[t]

@@ -17,6 +17,7 @@ __all__ = [
     "moe_expert_gemv_q4", "moe_expert_gemv_q2", "moe_combine_residual_norm", "moe_group_tokens",
     "moe_layer_forward", "moe_layer_forward_noalloc", "moe_layer_forward_timed", "moe_stack_forward", "moe_poll_status",
     "moe_selftest_wait_timeout", "moe_selftest_grid_timeout", "moe_noalloc_poll_status", "new_workspace",
+    "MxMat", "moe_expert_gemv_mxfp4", "moe_mxfp4_workspace_size", "moe_expert_gemm_mxfp4", "new_mx_workspace",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -39,6 +40,10 @@ class _QMat(C.Structure):
 
 class _Expert(C.Structure):
     _fields_ = [("gate", _QMat), ("up", _QMat), ("down", _QMat)]
+
+
+class _MxMat(C.Structure):
+    _fields_ = [("q", C.c_void_p), ("scales", C.c_void_p)]
 
 
 class _Layer(C.Structure):
@@ -91,6 +96,9 @@ def lib():
         L.moe_cache_admit.argtypes = [vp, vp, i32, vp, vp]
         L.moe_layer_forward_cached.argtypes = [vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, C.c_size_t, vp]
         L.moe_cache_stats.argtypes = [vp, u64, u64, u64]
+        L.moe_expert_gemv_mxfp4.argtypes = [vp, i32, i32, vp, vp, vp]
+        L.moe_mxfp4_workspace_size.argtypes = [i32, i32, i32, sz]
+        L.moe_expert_gemm_mxfp4.argtypes = [vp, i32, i32, vp, i32, vp, vp, C.c_size_t, vp]
         _lib = L
     return _lib
 
@@ -218,6 +226,43 @@ def moe_expert_gemv_q4(W: QMat, R: int, K: int, group: int, x, y, stream=None):
 def moe_expert_gemv_q2(W: QMat, R: int, K: int, group: int, x, y, stream=None):
     w = W.c()
     _ok(lib().moe_expert_gemv_q2(C.byref(w), R, K, group, _ptr(x), _ptr(y), _stream(stream)), "moe_expert_gemv_q2")
+
+
+class MxMat:
+    """One MXFP4 matrix: codes int32 [R][K/8] (E2M1 nibbles), scales uint8 [R][K/32] (E8M0)."""
+
+    def __init__(self, q, scales):
+        self.q, self.scales = q, scales
+
+    def c(self) -> _MxMat:
+        return _MxMat(self.q.data_ptr(), self.scales.data_ptr())
+
+
+def moe_expert_gemv_mxfp4(W: MxMat, x, y, stream=None):
+    """y = W x (fp32 [K] -> fp32 [R])."""
+    w = W.c()
+    R, K = W.scales.shape[0], W.scales.shape[1] * 32
+    _ok(lib().moe_expert_gemv_mxfp4(C.byref(w), R, K, _ptr(x), _ptr(y), _stream(stream)), "moe_expert_gemv_mxfp4")
+
+
+def moe_mxfp4_workspace_size(R: int, K: int, T: int) -> int:
+    n = C.c_size_t(0)
+    _ok(lib().moe_mxfp4_workspace_size(int(R), int(K), int(T), C.byref(n)), "moe_mxfp4_workspace_size")
+    return n.value
+
+
+def new_mx_workspace(R: int, K: int, T: int, device="cuda"):
+    """A zero-initialised workspace for moe_expert_gemm_mxfp4 (caller-owned device memory)."""
+    import torch
+    return torch.zeros(moe_mxfp4_workspace_size(R, K, T), dtype=torch.uint8, device=device)
+
+
+def moe_expert_gemm_mxfp4(W: MxMat, x, y, *, ws, stream=None):
+    """Y[t] = W x[t]: x bf16 bits int16 [T][K], y fp32 [T][R]."""
+    w = W.c()
+    R, K = W.scales.shape[0], W.scales.shape[1] * 32
+    _ok(lib().moe_expert_gemm_mxfp4(C.byref(w), R, K, _ptr(x), x.shape[0], _ptr(y), _ptr(ws), ws.numel(),
+                                    _stream(stream)), "moe_expert_gemm_mxfp4")
 
 
 def moe_combine_residual_norm(y_routed, topk_w, y_shared, shared_gate, h, gamma, eps: float, x_out, x_out_f32=None,

@@ -16,7 +16,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libmoe_b200.so")
-SOURCES = ["api.cu", "kernels.cu", "decode.cu", "fused.cu", "prefill.cu", "shared_tc.cu", "cache.cu", "route_tc.cu"]
+SOURCES = ["api.cu", "kernels.cu", "decode.cu", "fused.cu", "prefill.cu", "shared_tc.cu", "cache.cu", "route_tc.cu", "mx.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -423,6 +423,32 @@ moe_status moe_expert_gemv_q2(const moe_qmat* W, int32_t R, int32_t K, int32_t g
   return gemv_common(W, R, K, group, x, y, 2, stream);
 }
 
+moe_status moe_expert_gemv_mxfp4(const moe_mxmat* W, int32_t R, int32_t K, const float* x, float* y, void* stream) {
+  if (!W || !W->q || !W->scales || !x || !y || R <= 0 || K <= 0 || K % 32) return MOE_ERR_INVALID_ARGUMENT;
+  if (K > kMaxHI) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(W->q) || !aligned16(x)) return MOE_ERR_INVALID_ARGUMENT;
+  return cuda_status(launch_mx_gemv(W->q, W->scales, R, K, x, y, (cudaStream_t)stream));
+}
+
+moe_status moe_mxfp4_workspace_size(int32_t R, int32_t K, int32_t T, size_t* bytes) {
+  if (!bytes || R <= 0 || K <= 0 || T <= 0) return MOE_ERR_INVALID_ARGUMENT;
+  if (R % 128 || K % 128 || K > kMaxHI) return MOE_ERR_UNSUPPORTED;
+  *bytes = mx_gemm_ws_bytes(R, K, T);
+  return MOE_OK;
+}
+
+moe_status moe_expert_gemm_mxfp4(const moe_mxmat* W, int32_t R, int32_t K, const uint16_t* x, int32_t T, float* y,
+                                 void* ws, size_t ws_bytes, void* stream) {
+  size_t need = 0;
+  moe_status st = moe_mxfp4_workspace_size(R, K, T, &need);
+  if (st) return st;
+  if (!W || !W->q || !W->scales || !x || !y || !ws) return MOE_ERR_INVALID_ARGUMENT;
+  if (!aligned16(W->q) || ((uintptr_t)W->scales & 3) || !aligned16(x) || ((uintptr_t)ws & 255))
+    return MOE_ERR_INVALID_ARGUMENT;
+  if (ws_bytes < need) return MOE_ERR_WORKSPACE;
+  return cuda_status(launch_mx_gemm(W->q, W->scales, R, K, x, T, y, ws, wait_bound_ns(), (cudaStream_t)stream));
+}
+
 moe_status moe_combine_residual_norm(int32_t T, int32_t H, int32_t k, const float* y_routed, const float* topk_w,
                                      const float* y_shared, const float* shared_gate, float* h,
                                      const uint16_t* gamma, float eps, uint16_t* x_out, float* x_out_f32,

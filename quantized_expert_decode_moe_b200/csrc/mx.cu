@@ -1,0 +1,455 @@
+// MXFP4 expert matrices: the third codec. The page on running a 300B MoE from
+// a 32 GB laptop ("300b on 32gb MoE-streaming findings + optimisations")
+// streams MXFP4 experts; the format is read as the OCP Microscaling (MX) v1.0
+// definition: FP4 E2M1 elements (sign, two exponent bits with bias 1, one
+// mantissa bit; values 0, 0.5, 1, 1.5, 2, 3, 4, 6 and their negatives), one
+// E8M0 scale 2^(byte - 127) per 32 consecutive k (byte 0xFF is NaN). Codes use
+// the 4-bit packing (element k of a row in word k/8 at bits 4(k%8), LSB first),
+// scales are uint8 [R][K/32].
+//
+// Two entry points:
+//  * mx_gemv_kernel: y = W x (decode). A warp per row, a lane per 32-element
+//    block: the 16 code bytes of the block in one load, each nibble decoded to
+//    2|v| by a byte permutation (the eight magnitudes 0..12 as a byte table),
+//    the sign bit moved into the float, an fp32 FMA with x (staged in shared
+//    memory), the block sum times 2^(byte - 128).
+//  * mx_gemm_kernel: Y = X W^T for many tokens on the tcgen05 tensor cores,
+//    kind::mxf4 with block scaling: the weight codes go from HBM to shared
+//    memory unchanged (TMA tiles of 16 bytes x 128 rows, i.e. one MX block of
+//    128 rows) and the MMA applies the weight's E8M0 scales itself. The bf16
+//    activations are written as a sum of kMxTerms E2M1 terms, each with its
+//    own E8M0 scale per 32-block (mx_prep_kernel): term j is the residual's
+//    block maximum scaled to at most 6, rounded to the nearest E2M1 value, and
+//    subtracted exactly (the rounded value lies within a factor of two of the
+//    residual, so the fp32 subtraction is exact). Each term cuts the largest
+//    residual of a block by a factor of at least four; after five terms it is
+//    below 4^-4 / 3 of the block's maximum (about 5e-5 of the output's norm in
+//    practice). All terms accumulate into one fp32 accumulator in tensor
+//    memory, since each carries its own scales.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+#include "sync.cuh"
+#include "tc.cuh"
+
+namespace qmoe {
+
+// ------------------------------------------------------------------ mat-vec (decode)
+constexpr int kMvWarps = 8;
+constexpr int kMvXStride = 36;   // floats per 32-element block of x in shared memory (padded)
+
+// 2^(byte - 128): the block scale times 1/2, as the nibbles decode to 2|v|; NaN for 0xFF
+__device__ __forceinline__ float mx_half_scale(unsigned byte) {
+  return byte == 0xFFu ? __int_as_float(0x7FC00000) : ldexpf(1.0f, (int)byte - 128);
+}
+
+// sum over one 32-element block of (2 e2m1(code_k)) x_k; xs: the block's 32 values of x
+__device__ __forceinline__ float mx_block_dot(const uint4 c, const float* xs) {
+  const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float4 xa = *(const float4*)(xs + 8 * i), xb = *(const float4*)(xs + 8 * i + 4);
+    const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+    // byte table of 2|v| for the magnitude fields 0..7: 0, 1, 2, 3, 4, 6, 8, 12
+    const uint32_t lo = __byte_perm(0x03020100u, 0x0C080604u, w[i] & 0x7777u);
+    const uint32_t hi = __byte_perm(0x03020100u, 0x0C080604u, (w[i] >> 16) & 0x7777u);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t mag = ((j < 4 ? lo : hi) >> (8 * (j & 3))) & 0xFFu;
+      const uint32_t sgn = (w[i] << (28 - 4 * j)) & 0x80000000u;   // bit 4j+3 -> bit 31
+      s = fmaf(__uint_as_float(__float_as_uint((float)mag) ^ sgn), xv[j], s);
+    }
+  }
+  return s;
+}
+
+// grid ceil(R / kMvWarps), block 32 kMvWarps: warp w of CTA b computes row b kMvWarps + w.
+__global__ void __launch_bounds__(kMvWarps * 32) mx_gemv_kernel(const uint32_t* __restrict__ q,
+                                                                const uint8_t* __restrict__ e, int R, int K,
+                                                                const float* __restrict__ x, float* __restrict__ y) {
+  extern __shared__ __align__(16) float xs[];   // [K/32][kMvXStride]
+  const int nb = K / 32;
+  for (int i = threadIdx.x; i < K / 4; i += blockDim.x) {
+    const float4 v = __ldg((const float4*)x + i);
+    *(float4*)(xs + (i >> 3) * kMvXStride + 4 * (i & 7)) = v;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, r = blockIdx.x * kMvWarps + (threadIdx.x >> 5);
+  if (r >= R) return;
+  const uint4* qr = (const uint4*)(q + (size_t)r * (K / 8));
+  const uint8_t* er = e + (size_t)r * nb;
+  float acc = 0.f;
+  for (int b0 = 0; b0 < nb; b0 += 4 * 32) {   // four blocks per lane in flight
+    uint4 c[4];
+    unsigned sb[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int b = b0 + 32 * u + lane;
+      c[u] = b < nb ? __ldg(qr + b) : make_uint4(0u, 0u, 0u, 0u);
+      sb[u] = b < nb ? __ldg(er + b) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int b = b0 + 32 * u + lane;
+      if (b < nb) acc = fmaf(mx_block_dot(c[u], xs + b * kMvXStride), mx_half_scale(sb[u]), acc);
+    }
+  }
+  acc = warp_sum(acc);
+  if (lane == 0) y[r] = acc;
+}
+
+cudaError_t launch_mx_gemv(const uint32_t* q, const uint8_t* e, int R, int K, const float* x, float* y,
+                           cudaStream_t s) {
+  const size_t sm = sizeof(float) * (size_t)(K / 32) * kMvXStride;
+  cudaError_t err = cudaFuncSetAttribute((const void*)mx_gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)sm);
+  if (err != cudaSuccess) return err;
+  mx_gemv_kernel<<<(R + kMvWarps - 1) / kMvWarps, kMvWarps * 32, sm, s>>>(q, e, R, K, x, y);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ many tokens (tcgen05 kind::mxf4)
+constexpr int kMxTerms = 5;                      // E2M1 terms of an activation block
+constexpr int kMxM = 128, kMxN = 128;            // weight rows, tokens per CTA
+constexpr int kMxKS = 128;                       // columns per stage: four MX blocks
+constexpr int kMxStages = 4;
+constexpr int kMxChunk = 128 * 16;               // one MX block (16 bytes of codes) of 128 rows
+constexpr int kMxTileA = 4 * kMxChunk;           // 8 KB
+constexpr int kMxTileB = kMxTerms * 4 * kMxChunk;   // 40 KB: the terms of 128 tokens
+constexpr int kMxSf = 512;                       // scales of 128 rows x 4 blocks
+constexpr int kMxStageBytes = kMxTileA + kMxTileB + kMxSf * (1 + kMxTerms);
+constexpr int kMxSfCols = 4 * (1 + kMxTerms);    // tensor-memory columns of one stage's scales
+constexpr int kMxPrepThreads = 128;
+constexpr int kMxSplitMax = 8;                   // column splits of the product at most
+constexpr int kMxWaveCtas = 148;                 // CTAs of one wave (one per SM of a B200)
+
+static_assert(kMxStageBytes % 1024 == 0, "stages stay 1 KB aligned");
+static_assert(kMxN + kMxStages * kMxSfCols <= 256, "accumulator and scales fit 256 tensor-memory columns");
+
+// Byte offset of a scale in a 512-byte block of 128 rows x 4 blocks: row m =
+// m0 + 32 m1 and block j at m0 16 + m1 4 + j. Copied to tensor memory by
+// tcgen05.cp 32x128b.warpx4, that puts the four scales of row m0 + 32 m1 in
+// column m1 of lane m0 of every 32-lane group, the layout the block-scaled
+// MMA reads (scale j of the word selected by the descriptor's scale id).
+__host__ __device__ __forceinline__ int mx_sf_off(int m, int j) { return (m & 31) * 16 + (m >> 5) * 4 + j; }
+
+// 2^n for n in [-149, 127], from its bits (subnormal below 2^-126)
+__device__ __forceinline__ float mx_pow2(int n) {
+  return n >= -126 ? __int_as_float((n + 127) << 23) : __int_as_float(1 << (n + 149));
+}
+
+// grid T_pad + ceil(R nstg / kMxPrepThreads), block kMxPrepThreads.
+//  CTA t < T_pad: token row t (zeros beyond T); thread i takes the 32-element
+//   blocks b = i + kMxPrepThreads n and writes, per term, the 16 code bytes at
+//   bq[(((t/128) nstg + b/4) kMxTerms + term) kMxChunk 4 + (b%4) kMxChunk + (t%128) 16]
+//   and the scale byte at bsf[(((t/128) nstg + b/4) kMxTerms + term) 512 + mx_sf_off(t%128, b%4)].
+//  CTA T_pad + s: scale words i = s kMxPrepThreads + thread (row i / nstg, stage
+//   i % nstg: the row's four scales of that stage), rearranged into the same
+//   512-byte blocks, asf[((row/128) nstg + stage) 512 + mx_sf_off(row%128, 0)].
+__global__ void __launch_bounds__(kMxPrepThreads) mx_prep_kernel(const uint16_t* __restrict__ x, int T, int Tpad,
+                                                                 const uint8_t* __restrict__ e, int R, int K,
+                                                                 uint8_t* __restrict__ bq, uint8_t* __restrict__ bsf,
+                                                                 uint8_t* __restrict__ asf) {
+  const int nb = K / 32, nstg = K / kMxKS;
+  if ((int)blockIdx.x >= Tpad) {   // weight scales: one 4-byte word (4 blocks, K % 128 == 0) per thread
+    const size_t i = (size_t)(blockIdx.x - Tpad) * kMxPrepThreads + threadIdx.x;
+    if (i >= (size_t)R * nstg) return;
+    const int r = (int)(i / nstg), g = (int)(i % nstg);
+    const uint32_t w = __ldg((const uint32_t*)e + i);
+    *(uint32_t*)(asf + ((size_t)(r / kMxM) * nstg + g) * kMxSf + mx_sf_off(r % kMxM, 0)) = w;
+    return;
+  }
+  const int t = blockIdx.x, tt = t / kMxN, rr = t % kMxN;
+  for (int b = threadIdx.x; b < nb; b += kMxPrepThreads) {
+    float v[32];
+    if (t < T) {
+      const uint4* src = (const uint4*)(x + (size_t)t * K + 32 * b);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint4 u = __ldg(src + i);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          v[8 * i + 2 * h] = bf16lo(w[h]);
+          v[8 * i + 2 * h + 1] = bf16hi(w[h]);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < 32; ++k) v[k] = 0.f;
+    }
+    const int g = b / 4, c = b % 4;
+#pragma unroll 1
+    for (int term = 0; term < kMxTerms; ++term) {
+      float m = 0.f;
+#pragma unroll
+      for (int k = 0; k < 32; ++k) m = fmaxf(m, fabsf(v[k]));
+      // the smallest power 2^u with m <= 6 2^u, no smaller than 2^-127 (every m below 2^-126 takes
+      // u = -127): with m = f 2^E, f in [0.5, 1), u = E - 3 if f <= 0.75, else E - 2
+      int u = -127;
+      if (m >= 0x1p-126f) {
+        const uint32_t bits = __float_as_uint(m);
+        const int E = (int)((bits >> 23) & 0xFFu) - 126;
+        u = max(-127, (bits & 0x7FFFFFu) <= 0x400000u ? E - 3 : E - 2);
+      }
+      const float down = mx_pow2(-u), up = mx_pow2(u - 1);   // 2^-u; 2^(u-1), the unit of 2|E2M1 value|
+      uint32_t code[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        const float a = fabsf(v[k] * down);   // exact unless it underflows, far below 0.25
+        const int idx = (a > 0.25f) + (a > 0.75f) + (a > 1.25f) + (a > 1.75f) + (a > 2.5f) + (a > 3.5f) + (a > 5.f);
+        const int twice = idx <= 4 ? idx : (idx == 5 ? 6 : (idx == 6 ? 8 : 12));   // 2 |E2M1 value|
+        const bool neg = v[k] < 0.f;
+        const float val = (float)(neg ? -twice : twice) * up;   // exact: a small integer times 2^(u-1)
+        v[k] -= val;   // exact: 0, or within a factor of two of v[k]
+        code[k >> 3] |= (uint32_t)(idx | (neg ? 8 : 0)) << (4 * (k & 7));
+      }
+      const size_t blk = ((size_t)tt * nstg + g) * kMxTerms + term;
+      *(uint4*)(bq + blk * kMxTileA + (size_t)c * kMxChunk + (size_t)rr * 16) =
+          make_uint4(code[0], code[1], code[2], code[3]);
+      bsf[blk * kMxSf + mx_sf_off(rr, c)] = (uint8_t)(u + 127);
+    }
+  }
+}
+
+// grid (R/128, T_pad/128), block 128. Stage u (columns 128u .. 128u+127):
+// the weight codes by four TMA tiles (16 bytes x 128 rows each, one MX block,
+// at byte c kMxChunk), then the tokens' terms (one bulk copy of kMxTileB) and
+// the scales of the weight rows and of the terms (512 bytes each). Thread 0
+// loads; thread 32 copies the stage's scales into tensor memory (tcgen05.cp)
+// and issues per term two MMAs of K = 64 (blocks 2h, 2h+1: scale id 2h); all
+// four warps read the accumulator (lane = weight row) and write Y[t][r].
+struct MxSmem {
+  uint64_t full[kMxStages], empty[kMxStages], done;
+  uint32_t tslot;
+  int abort;
+};
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      :: "r"(smem_u32(dst)), "l"((uint64_t)map), "r"(x), "r"(y), "r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" :: "r"(taddr), "l"(sdesc) : "memory");
+}
+
+// kind::mxf4 instruction descriptor: E2M1 A and B (format 1), both K-major,
+// N >> 3 at bit 17, E8M0 scales (bit 23), M >> 4 at bit 24, scale ids of B
+// (bits 4-5) and A (bits 29-30), K = 64.
+__device__ __forceinline__ uint32_t mx_idesc(int sf_id) {
+  return ((uint32_t)sf_id << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kMxN >> 3) << 17) | (1u << 23) |
+         ((uint32_t)(kMxM >> 4) << 24) | ((uint32_t)sf_id << 29);
+}
+
+struct MxGemmParams {
+  int R, K, T, splits;
+  float* part;         // [splits][T][R] partial products when splits > 1
+  const uint8_t* bq;   // the tokens' terms (prep layout)
+  const uint8_t* bsf;  // their scales
+  const uint8_t* asf;  // the weight scales, rearranged
+  float* y;            // [T][R]
+  uint32_t* status;
+  unsigned long long wait_ns;
+};
+
+__global__ void __launch_bounds__(128, 1) mx_gemm_kernel(const __grid_constant__ CUtensorMap wmap, MxGemmParams p) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  MxSmem& S = *(MxSmem*)(smem + kMxStages * kMxStageBytes);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int mt = blockIdx.x, nt = blockIdx.y, nstg = p.K / kMxKS;
+  const int i0 = (int)((long long)nstg * blockIdx.z / p.splits), n = (int)((long long)nstg * (blockIdx.z + 1) / p.splits) - i0;
+  const unsigned long long wait_ns = p.wait_ns;
+  uint32_t* status = p.status;
+  if (tid == 0) {
+    for (int s = 0; s < kMxStages; ++s) {
+      mbar_init(&S.full[s], 1);
+      mbar_init(&S.empty[s], 1);
+    }
+    mbar_init(&S.done, 1);
+    S.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) tc_alloc(&S.tslot, 256);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = S.tslot;
+  volatile int* abort_flag = &S.abort;
+
+  if (tid == 0) {   // ---------------------------------------------------- loads
+    int last[kMxStages];
+    for (int s = 0; s < kMxStages; ++s) last[s] = -1;
+    for (int u = 0; u < n; ++u) {
+      const int slot = u % kMxStages, use = u / kMxStages, g = i0 + u;
+      if (use > 0 && !mbar_wait_bounded(&S.empty[slot], (use - 1) & 1, wait_ns, status)) *abort_flag = 1;
+      if (*abort_flag) break;
+      unsigned char* st = smem + (size_t)slot * kMxStageBytes;
+      mbar_expect_tx(&S.full[slot], (unsigned)kMxStageBytes);
+      for (int c = 0; c < 4; ++c) tma_load_2d(st + c * kMxChunk, &wmap, g * (kMxKS / 2) + 16 * c, mt * kMxM, &S.full[slot]);
+      const size_t bstage = (size_t)nt * nstg + g;
+      bulk_g2s(st + kMxTileA, p.bq + bstage * kMxTileB, kMxTileB, &S.full[slot]);
+      bulk_g2s(st + kMxTileA + kMxTileB, p.asf + ((size_t)mt * nstg + g) * kMxSf, kMxSf, &S.full[slot]);
+      bulk_g2s(st + kMxTileA + kMxTileB + kMxSf, p.bsf + bstage * kMxTerms * kMxSf, kMxTerms * kMxSf, &S.full[slot]);
+      last[slot] = use;
+    }
+    for (int s = 0; s < kMxStages; ++s)   // no copy may land after the CTA has left
+      if (last[s] >= 0) mbar_wait_bounded(&S.full[s], last[s] & 1, wait_ns, status);
+  } else if (tid == 32) {   // --------------------------------------------- scales to tensor memory, MMAs
+    bool started = false;
+    for (int u = 0; u < n; ++u) {
+      const int slot = u % kMxStages, ph = (u / kMxStages) & 1;
+      if (!mbar_wait_bounded(&S.full[slot], ph, wait_ns, status)) *abort_flag = 1;
+      if (*abort_flag) break;
+      tc_fence_after();
+      const uint32_t a0 = smem_u32(smem + (size_t)slot * kMxStageBytes), b0 = a0 + kMxTileA;
+      const uint32_t sf0 = b0 + kMxTileB;
+      const uint32_t tsf = tbase + (uint32_t)(kMxN + slot * kMxSfCols);
+      for (int i = 0; i < 1 + kMxTerms; ++i)   // weight scales, then each term's: 4 columns each
+        tc_cp_sf(tsf + 4 * i, tc_smem_desc(sf0 + i * kMxSf, 128, 128));
+#pragma unroll
+      for (int term = 0; term < kMxTerms; ++term)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint64_t ad = tc_smem_desc(a0 + 2 * h * kMxChunk, kMxChunk, 128);
+          const uint64_t bd = tc_smem_desc(b0 + term * kMxTileA + 2 * h * kMxChunk, kMxChunk, 128);
+          const uint32_t sfa = (tsf) | ((uint32_t)(2 * h) << 30);
+          const uint32_t sfb = (tsf + 4 * (1 + term)) | ((uint32_t)(2 * h) << 30);
+          const uint32_t acc = started ? 1u : 0u;
+          asm volatile("{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+                       " tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%5], [%6], p;\n}\n"
+                       :: "r"(tbase), "l"(ad), "l"(bd), "r"(mx_idesc(2 * h)), "r"(acc), "r"(sfa), "r"(sfb)
+                       : "memory");
+          started = true;
+        }
+      tc_commit(&S.empty[slot]);
+    }
+    tc_commit(&S.done);
+    mbar_wait_bounded(&S.done, 0, wait_ns, status);
+  }
+  // -------------------------------------------------------------------- epilogue (all warps)
+  __syncwarp();
+  bool ok = mbar_wait_bounded(&S.done, 0, wait_ns, status) && !*abort_flag;
+  ok = __all_sync(0xffffffffu, ok);
+  tc_fence_after();
+  if (ok) {
+    const int r = mt * kMxM + tid;
+    const uint32_t lane_addr = tbase + ((uint32_t)(warp * 32) << 16);
+    float* out = p.splits > 1 ? p.part + (size_t)blockIdx.z * p.T * p.R : p.y;
+    for (int c0 = 0; c0 < kMxN; c0 += 16) {
+      uint32_t v[16];
+      tc_ld16(lane_addr + c0, v);
+      tc_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int t = nt * kMxN + c0 + j;
+        if (t < p.T && r < p.R) out[(size_t)t * p.R + r] = __uint_as_float(v[j]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tc_dealloc(tbase, 256);
+}
+
+// grid ceil(T R / 4 / 256), block 256: Y = the splits' partial products summed in split order.
+__global__ void __launch_bounds__(256) mx_reduce_kernel(const float* __restrict__ part, int splits, size_t n4,
+                                                        float* __restrict__ y) {
+  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n4) return;
+  float4 a = __ldcg((const float4*)part + i);
+  for (int q = 1; q < splits; ++q) {
+    const float4 b = __ldcg((const float4*)part + (size_t)q * n4 + i);
+    a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+  }
+  *((float4*)y + i) = a;
+}
+
+// ------------------------------------------------------------------ host side
+// Workspace of the many-token product: a 256-byte header (status word first),
+// then the tokens' terms, their scales and the rearranged weight scales.
+struct MxWs {
+  size_t bq, bsf, asf, part, total;
+  int splits;
+};
+// Column splits: as many as keep the CTAs within one wave, at most kMxSplitMax, at least two
+// stages each; a function of the shape alone, so the workspace size is known without a device.
+static int mx_splits(int R, int K, int T) {
+  const int tiles = (R / kMxM) * ((T + kMxN - 1) / kMxN), nstg = K / kMxKS;
+  int s = kMxWaveCtas / tiles;
+  s = s > kMxSplitMax ? kMxSplitMax : s;
+  s = s > nstg / 2 ? nstg / 2 : s;
+  return s < 1 ? 1 : s;
+}
+static MxWs mx_ws(int R, int K, int T) {
+  const size_t tpad = (size_t)(T + kMxN - 1) / kMxN * kMxN;
+  MxWs w;
+  w.splits = mx_splits(R, K, T);
+  size_t o = 256;
+  w.bq = o; o = (o + tpad * (size_t)K / 2 * kMxTerms + 255) / 256 * 256;
+  w.bsf = o; o = (o + tpad * (size_t)K / 32 * kMxTerms + 255) / 256 * 256;
+  w.asf = o; o = (o + (size_t)R * K / 32 + 255) / 256 * 256;
+  w.part = o; o = (o + (w.splits > 1 ? sizeof(float) * w.splits * (size_t)T * R : 0) + 255) / 256 * 256;
+  w.total = o;
+  return w;
+}
+
+size_t mx_gemm_ws_bytes(int R, int K, int T) { return mx_ws(R, K, T).total; }
+
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (PFN_cuTensorMapEncodeTiled_v12000)ptr;
+  }
+  return fn;
+}
+
+cudaError_t launch_mx_gemm(const uint32_t* q, const uint8_t* e, int R, int K, const uint16_t* x, int T, float* y,
+                           void* ws, unsigned long long wait_ns, cudaStream_t s) {
+  const MxWs W = mx_ws(R, K, T);
+  const int tpad = (T + kMxN - 1) / kMxN * kMxN;
+  uint8_t* base = (uint8_t*)ws;
+  const int nscale = (int)(((size_t)R * (K / kMxKS) + kMxPrepThreads - 1) / kMxPrepThreads);
+  mx_prep_kernel<<<tpad + nscale, kMxPrepThreads, 0, s>>>(x, T, tpad, e, R, K, base + W.bq, base + W.bsf,
+                                                             base + W.asf);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {(cuuint64_t)K / 2, (cuuint64_t)R};   // bytes of a row, rows
+  const cuuint64_t strides[1] = {(cuuint64_t)K / 2};
+  const cuuint32_t box[2] = {16, (cuuint32_t)kMxM};
+  const cuuint32_t estr[2] = {1, 1};
+  if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, (void*)q, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+      CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  MxGemmParams p;
+  p.R = R; p.K = K; p.T = T; p.splits = W.splits;
+  p.part = (float*)(base + W.part);
+  p.bq = base + W.bq; p.bsf = base + W.bsf; p.asf = base + W.asf;
+  p.y = y;
+  p.status = (uint32_t*)ws;
+  p.wait_ns = wait_ns;
+  const size_t sm = (size_t)kMxStages * kMxStageBytes + sizeof(MxSmem);
+  err = cudaFuncSetAttribute((const void*)mx_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (err != cudaSuccess) return err;
+  mx_gemm_kernel<<<dim3(R / kMxM, tpad / kMxN, W.splits), 128, sm, s>>>(map, p);
+  err = cudaGetLastError();
+  if (err != cudaSuccess || W.splits == 1) return err;
+  const size_t n4 = (size_t)T * R / 4;   // R % 128 == 0
+  mx_reduce_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, s>>>(p.part, W.splits, n4, y);
+  return cudaGetLastError();
+}
+
+}  // namespace qmoe

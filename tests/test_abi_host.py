@@ -197,3 +197,29 @@ def test_wait_bound_and_header_words_documented():
     text = open(HEADER).read()
     assert "100 ms" in text and "MOE_WAIT_TIMEOUT_NS" in text
     assert "byte offset 16" in text and "moe_noalloc_poll_status" in text
+
+
+def test_mxfp4_entry_points_check_arguments_on_the_host():
+    """The MXFP4 calls reject bad shapes, missing pointers and small workspaces before any CUDA
+    call (so this runs without a GPU)."""
+    L = qm.lib()
+    n = C.c_size_t(0)
+    assert L.moe_mxfp4_workspace_size(256, 4096, 512, C.byref(n)) == 0 and n.value > 256
+    assert L.moe_mxfp4_workspace_size(200, 4096, 1, C.byref(n)) == 2      # R % 128
+    assert L.moe_mxfp4_workspace_size(128, 4000, 1, C.byref(n)) == 2      # K % 128
+    assert L.moe_mxfp4_workspace_size(128, 16384, 1, C.byref(n)) == 2     # K > 8192
+    assert L.moe_mxfp4_workspace_size(128, 128, 0, C.byref(n)) == 1
+    assert L.moe_mxfp4_workspace_size(128, 128, 1, None) == 1
+    W = qm._MxMat(0x1000, 0x1000)
+    assert L.moe_expert_gemv_mxfp4(None, 16, 64, C.c_void_p(0x1000), C.c_void_p(0x1000), None) == 1
+    assert L.moe_expert_gemv_mxfp4(C.byref(W), 16, 48, C.c_void_p(0x1000), C.c_void_p(0x1000), None) == 1   # K % 32
+    assert L.moe_expert_gemv_mxfp4(C.byref(W), 16, 16384, C.c_void_p(0x1000), C.c_void_p(0x1000), None) == 2
+    assert L.moe_expert_gemv_mxfp4(C.byref(W), 16, 64, C.c_void_p(0x1008), C.c_void_p(0x1000), None) == 1   # x align
+    L.moe_mxfp4_workspace_size(128, 128, 4, C.byref(n))
+    need = n.value
+    args = (C.c_void_p(0x1000), 4, C.c_void_p(0x1000), C.c_void_p(0x10000))
+    assert L.moe_expert_gemm_mxfp4(C.byref(W), 128, 128, *args, need - 1, None) == 3
+    assert L.moe_expert_gemm_mxfp4(C.byref(W), 100, 128, *args, need, None) == 2
+    assert L.moe_expert_gemm_mxfp4(None, 128, 128, *args, need, None) == 1
+    assert L.moe_expert_gemm_mxfp4(C.byref(W), 128, 128, C.c_void_p(0x1000), 4, C.c_void_p(0x1000),
+                                   C.c_void_p(0x10010), need, None) == 1      # workspace not 256-byte aligned

@@ -1,0 +1,141 @@
+"""GPU: MXFP4 expert matrices (E2M1 codes, E8M0 scale per 32) against the oracle.
+
+moe_expert_gemv_mxfp4 (decode mat-vec, fp32 block sums) and
+moe_expert_gemm_mxfp4 (many tokens on tcgen05 kind::mxf4 with block scaling;
+the bf16 activations as five E2M1 terms) are compared with the oracle's
+double-precision products on the same seeded inputs, at sizes spanning
+several tiles with ragged tails, the expert shapes of the 4-bit layer
+(hidden 4096, intermediate 1024), the largest accepted K, and the degenerate
+cases (zero activations, an outlier element, the NaN scale byte)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import quantized_expert_decode_moe_b200 as qm
+from fixtures import gen
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dev():
+    assert torch.cuda.is_available()
+    qm.lib()
+    return torch.device("cuda")
+
+
+def normwise(got, ref):
+    return float(np.abs(got - ref).max() / max(np.abs(ref).max(), 1e-300))
+
+
+def mat(q, e, dev):
+    return qm.MxMat(torch.from_numpy(q.view(np.int32)).to(dev), torch.from_numpy(e).to(dev))
+
+
+def gemv(q, e, x, dev):
+    W = mat(q, e, dev)
+    xd = torch.from_numpy(x.astype(np.float32)).to(dev)
+    y = torch.empty(q.shape[0], dtype=torch.float32, device=dev)
+    qm.moe_expert_gemv_mxfp4(W, xd, y)
+    return y.cpu().numpy()
+
+
+def gemm(q, e, xb, dev):
+    R, K = q.shape[0], q.shape[1] * 8
+    W = mat(q, e, dev)
+    ws = qm.new_mx_workspace(R, K, xb.shape[0])
+    y = torch.full((xb.shape[0], R), float("nan"), dtype=torch.float32, device=dev)
+    qm.moe_expert_gemm_mxfp4(W, torch.from_numpy(xb.view(np.int16)).to(dev), y, ws=ws)
+    assert qm.moe_poll_status(ws) == 0
+    return y.cpu().numpy()
+
+
+# ------------------------------------------------------------------ mat-vec
+@pytest.mark.parametrize("R,K", [(16, 64), (40, 96), (1024, 4096), (4096, 1024), (24, 8192), (3, 32)])
+def test_gemv_matches_oracle(dev, R, K):
+    q, e = gen.mx_matrix(R + K, R, K)
+    x = gen.bf16_bits_to_f32(gen.mx_tokens(R, 1, K)[0]).astype(np.float64)
+    got = gemv(q, e, x, dev)
+    ref = oracle.mx_gemv(q, e, x, K)
+    err = normwise(got, ref)
+    # fp32 products and sums over at most 8192 terms: far inside the 2e-3 contract
+    assert err <= 1e-5, err
+
+
+def test_gemv_nan_scale_and_zero_codes(dev):
+    """Scale byte 0xFF is NaN in the format: that row's output is NaN; an all-zero row is 0."""
+    R, K = 8, 128
+    q, e = gen.mx_matrix(5, R, K)
+    q[2] = 0
+    e[5, 1] = 0xFF
+    x = np.linspace(-1, 1, K)
+    got = gemv(q, e, x, dev)
+    ref = oracle.mx_gemv(q, e, x, K)
+    assert np.isnan(got[5]) and np.isnan(ref[5])
+    assert got[2] == 0.0
+    keep = [i for i in range(R) if i != 5]
+    assert normwise(got[keep], ref[keep]) <= 1e-5
+
+
+# ------------------------------------------------------------------ many tokens (tcgen05)
+@pytest.mark.parametrize("R,K,T", [(128, 128, 1), (128, 256, 9), (256, 1024, 40), (384, 512, 130),
+                                   (2048, 4096, 512), (4096, 1024, 64), (128, 8192, 33)])
+def test_gemm_matches_oracle(dev, R, K, T):
+    """One 128 x 128 tile up to the shared expert's gate/up (2048 x 4096, 512 tokens); ragged token
+    tails (1, 9, 33, 40, 130); one 128-column stage up to 64 stages."""
+    q, e = gen.mx_matrix(R * 7 + K, R, K)
+    xb = gen.mx_tokens(T + K, T, K)
+    got = gemm(q, e, xb, dev)
+    ref = oracle.mx_gemm(q, e, xb, K)
+    err = normwise(got, ref)
+    # five E2M1 terms leave a residual below 4^-4/3 of each block's largest |x|; about 5e-5 normwise
+    assert err <= 5e-4, err
+    print(f"mxfp4 gemm R={R} K={K} T={T}: normwise error {err:.2e}")
+
+
+def test_gemm_rows_equal_gemv_within_the_term_error(dev):
+    """The tensor-core product of one token against the mat-vec of the same token (two
+    independent kernels, different arithmetic), both against the oracle."""
+    R, K = 1024, 4096
+    q, e = gen.mx_matrix(77, R, K)
+    xb = gen.mx_tokens(78, 1, K)
+    x = gen.bf16_bits_to_f32(xb[0]).astype(np.float64)
+    a = gemm(q, e, xb, dev)[0]
+    b = gemv(q, e, x, dev)
+    ref = oracle.mx_gemv(q, e, x, K)
+    assert normwise(a, ref) <= 5e-4 and normwise(b, ref) <= 1e-5
+
+
+def test_gemm_degenerate_activations(dev):
+    """Zero tokens give exactly zero; a token whose one element is 2^10 times the rest costs only
+    its own block; tokens of very different magnitudes in one tile keep their own scales."""
+    R, K, T = 256, 1024, 6
+    q, e = gen.mx_matrix(9, R, K)
+    x = gen.bf16_bits_to_f32(gen.mx_tokens(10, T, K)).astype(np.float32)
+    x[0] = 0.0
+    x[1, 100] *= 1024.0
+    x[2] *= 2.0 ** -40
+    x[3] *= 2.0 ** 40
+    x[4, ::2] = 0.0
+    xb = gen.f32_to_bf16_bits(x)
+    got = gemm(q, e, xb, dev)
+    ref = oracle.mx_gemm(q, e, xb, K)
+    assert np.all(got[0] == 0.0)
+    for t in range(1, T):
+        assert normwise(got[t], ref[t]) <= 5e-4, t
+
+
+def test_gemm_rejects_bad_shapes_before_launch(dev):
+    q, e = gen.mx_matrix(1, 256, 256)
+    W = mat(q, e, dev)
+    x = torch.zeros((4, 256), dtype=torch.int16, device=dev)
+    y = torch.empty((4, 256), dtype=torch.float32, device=dev)
+    ws = qm.new_mx_workspace(256, 256, 4)
+    with pytest.raises(qm.MoeError) as ex:   # workspace for fewer tokens than the call has
+        qm.moe_expert_gemm_mxfp4(W, torch.zeros((400, 256), dtype=torch.int16, device=dev),
+                                 torch.empty((400, 256), dtype=torch.float32, device=dev), ws=ws)
+    assert ex.value.code == 3
+    with pytest.raises(qm.MoeError) as ex:   # R not a multiple of 128
+        qm.moe_expert_gemm_mxfp4(qm.MxMat(W.q[:200], W.scales[:200]), x, y, ws=ws)
+    assert ex.value.code == 2
