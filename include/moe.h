@@ -40,6 +40,8 @@
  *      T > 8     the grouped prefill kernels (two stages of their ring of
  *                weight tiles must fit and their row tiles must divide the
  *                matrices);
+ *      MXFP4    (group 32) T <= 8: the down kernel stages every slot's SwiGLU
+ *                output in shared memory: (top_k + shared) * I <= 51,200;
  *    and H, I <= 8192 throughout. With MOE_DECODE_KERNEL=fused in the
  *    environment (read once), single-token calls and stacks take the fused
  *    single-kernel layer where it fits: H <= 4096, top_k <= 3 (top_k +
@@ -97,6 +99,11 @@ typedef struct {
  * One MoE layer. Host struct; its pointers are device memory.
  *   hidden H, inter I, n_experts E (routed), top_k k (routed, k <= 8),
  *   bits in {2,4}, group = 64, has_shared in {0,1}, rms_eps > 0.
+ *   bits = 4 with group = 32 selects MXFP4 experts (see moe_mxmat): each
+ *   moe_qmat's q holds the E2M1 codes, its scales pointer the E8M0 bytes
+ *   uint8 [R][K/32], its biases are not read (may be NULL); decode only
+ *   (T <= 8; MOE_ERR_UNSUPPORTED above), through moe_layer_forward,
+ *   moe_layer_forward_timed, moe_layer_forward_noalloc and moe_stack_forward.
  *   router_w    bf16 [E][H]
  *   router_bias fp32 [E] or NULL: added to the logits before softmax/top-k
  *   experts     device array [E] of moe_expert
@@ -267,7 +274,7 @@ moe_status moe_layer_forward(const moe_layer* layer, const uint16_t* x_in, float
  *   layers: host array [L]; x_in bf16 [H]; h fp32 [H] in/out; x_out bf16 [H];
  *   topk_idx_all int32 [L][k] or NULL; layer_inputs bf16 [L][H] or NULL and
  *   layer_h fp32 [L][H] or NULL: each layer's input x and residual h (for
- *   teacher-forced checks). Every layer must have the same H, I, E, k, bits.
+ *   teacher-forced checks). Every layer must have the same H, I, E, k, bits, group.
  */
 moe_status moe_stack_forward(const moe_layer* layers, int32_t L, const uint16_t* x_in, float* h,
                              uint16_t* x_out, int32_t* topk_idx_all, uint16_t* layer_inputs,
@@ -276,13 +283,14 @@ moe_status moe_stack_forward(const moe_layer* layers, int32_t L, const uint16_t*
 /*
  * The kernel path that serves a call of T tokens on `layer` (host only,
  * launches nothing): MOE_PATH_FUSED (the fused decode kernel, T = 1),
- * MOE_PATH_CHAIN (the four-kernel decode chain, T <= 8) or MOE_PATH_PREFILL
- * (T > 8), and in *n_events the number of events moe_layer_forward_timed
+ * MOE_PATH_CHAIN (the four-kernel decode chain, T <= 8), MOE_PATH_PREFILL
+ * (T > 8) or MOE_PATH_MXFP4 (a layer of MXFP4 experts: router, top-k,
+ * gate/up + SwiGLU and down + combine, RMSNorm), and in *n_events the number of events moe_layer_forward_timed
  * records on that path (its stages + 1). Either output may be NULL.
  * Errors: those of moe_workspace_size's layer checks; MOE_ERR_UNSUPPORTED
  * when no path fits (see "Supported shapes").
  */
-typedef enum { MOE_PATH_FUSED = 1, MOE_PATH_CHAIN = 2, MOE_PATH_PREFILL = 3 } moe_path;
+typedef enum { MOE_PATH_FUSED = 1, MOE_PATH_CHAIN = 2, MOE_PATH_PREFILL = 3, MOE_PATH_MXFP4 = 4 } moe_path;
 moe_status moe_layer_path(const moe_layer* layer, int32_t T, int32_t* path, int32_t* n_events);
 
 /*

@@ -202,6 +202,33 @@ def combine_norm(y_routed, w, y_shared, sg: float, h_in, gamma, eps: float):
     return h_out, x_out, xb
 
 
+def mx_layer(x, h_in, Wr, gamma, experts, shared, *, k: int, eps: float, router_bias=None, gs=None):
+    """One layer with MXFP4 experts, composed of the oracle's steps: route; per token, for each
+    chosen expert (rank order) and then the shared one, g = G x and u = U x (mx_gemv), a =
+    swiglu(g, u), y = D a; then combine + residual + RMSNorm.
+    experts: list of E ((qg, eg), (qu, eu), (qd, ed)); shared: one such tuple or None.
+    Returns dict(h_out, x_out, x_out_bf16, idx, w, shared_gate)."""
+    x = _c(np.atleast_2d(x), np.uint16); h_in = np.atleast_2d(np.asarray(h_in, dtype=np.float64))
+    T, H = x.shape
+    idx, w, sg = route(x, Wr, k, bias=router_bias, gs=gs if shared is not None else None)
+
+    def run(ex, xt):
+        (qg, eg), (qu, eu), (qd, ed) = ex
+        g = mx_gemv(qg, eg, xt, H)
+        u = mx_gemv(qu, eu, xt, H)
+        return mx_gemv(qd, ed, swiglu(g, u), g.shape[0])
+
+    out = {"h_out": np.empty((T, H)), "x_out": np.empty((T, H)), "x_out_bf16": np.empty((T, H), dtype=np.uint16),
+           "idx": idx, "w": w, "shared_gate": sg}
+    for t in range(T):
+        xt = bf16_to_f64(x[t])
+        yr = np.stack([run(experts[e], xt) for e in idx[t]])
+        ys = run(shared, xt) if shared is not None else None
+        out["h_out"][t], out["x_out"][t], out["x_out_bf16"][t] = combine_norm(
+            yr, w[t], ys, sg[t] if shared is not None else 0.0, h_in[t], gamma, eps)
+    return out
+
+
 def group_by_expert(idx, E: int):
     idx = _c(idx, np.int32)
     T, k = idx.shape

@@ -121,13 +121,14 @@ def _ok(rc: int, where: str):
 
 
 class QMat:
-    """One packed matrix: codes int32 [R][K*bits/32], scales/biases int16 (bf16 bits) [R][K/64]."""
+    """One packed matrix: codes int32 [R][K*bits/32], scales/biases int16 (bf16 bits) [R][K/64].
+    In a layer of MXFP4 experts (group 32): codes int32 [R][K/8], scales uint8 E8M0 [R][K/32], biases None."""
 
     def __init__(self, q, scales, biases):
         self.q, self.scales, self.biases = q, scales, biases
 
     def c(self) -> _QMat:
-        return _QMat(self.q.data_ptr(), self.scales.data_ptr(), self.biases.data_ptr())
+        return _QMat(self.q.data_ptr(), self.scales.data_ptr(), self.biases.data_ptr() if self.biases is not None else None)
 
 
 class Expert:
@@ -153,7 +154,7 @@ class Layer:
         table = []
         for ex in experts:
             for m in (ex.gate, ex.up, ex.down):
-                table += [m.q.data_ptr(), m.scales.data_ptr(), m.biases.data_ptr()]
+                table += [m.q.data_ptr(), m.scales.data_ptr(), m.biases.data_ptr() if m.biases is not None else 0]
         self.expert_table = torch.tensor(table, dtype=torch.int64).to(router_w.device)
         self._c = _Layer(hidden, inter, self.n_experts, top_k, bits, group, 1 if shared is not None else 0,
                          float(rms_eps), router_w.data_ptr(), router_bias.data_ptr() if router_bias is not None else None,

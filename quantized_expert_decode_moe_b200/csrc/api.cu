@@ -43,10 +43,18 @@ moe_status check_qmat(const moe_qmat& m) {
   return MOE_OK;
 }
 
+// group 32 selects the MXFP4 codec (E2M1 codes, E8M0 scale bytes in moe_qmat.scales, no biases)
+bool is_mx(const moe_layer* L) { return L->group == 32; }
+
+moe_status check_mxmat(const moe_qmat& m) {
+  if (!m.q || !m.scales) return MOE_ERR_INVALID_ARGUMENT;
+  return aligned16(m.q) ? MOE_OK : MOE_ERR_INVALID_ARGUMENT;
+}
+
 moe_status check_layer(const moe_layer* L) {
   if (!L) return MOE_ERR_INVALID_ARGUMENT;
   if (L->bits != 2 && L->bits != 4) return MOE_ERR_UNSUPPORTED;
-  if (L->group != kGroup) return MOE_ERR_UNSUPPORTED;
+  if (is_mx(L) ? L->bits != 4 : L->group != kGroup) return MOE_ERR_UNSUPPORTED;
   if (L->hidden <= 0 || L->inter <= 0 || L->hidden % kSpan || L->inter % kSpan) return MOE_ERR_INVALID_ARGUMENT;
   if (L->hidden > kMaxHI || L->inter > kMaxHI) return MOE_ERR_UNSUPPORTED;
   if (L->n_experts <= 0 || L->n_experts > kMaxE) return MOE_ERR_INVALID_ARGUMENT;
@@ -59,7 +67,8 @@ moe_status check_layer(const moe_layer* L) {
   if (L->has_shared) {
     if (!L->shared_gate_w || !aligned16(L->shared_gate_w)) return MOE_ERR_INVALID_ARGUMENT;
     moe_status s;
-    if ((s = check_qmat(L->shared.gate)) || (s = check_qmat(L->shared.up)) || (s = check_qmat(L->shared.down))) return s;
+    auto chk = is_mx(L) ? check_mxmat : check_qmat;
+    if ((s = chk(L->shared.gate)) || (s = chk(L->shared.up)) || (s = chk(L->shared.down))) return s;
   }
   return MOE_OK;
 }
@@ -76,7 +85,7 @@ int slots_of(const moe_layer* L) { return L->top_k + (L->has_shared ? 1 : 0); }
 // them across kernels. MOE_DECODE_KERNEL=fused in the environment (read
 // once) selects the fused kernel for single-token calls and stacks wherever
 // it fits.
-enum class Path { kNone, kFused, kChain, kPrefill };
+enum class Path { kNone, kFused, kChain, kPrefill, kMx };
 bool fused_requested() {
   static int v = -1;
   if (v < 0) {
@@ -85,7 +94,14 @@ bool fused_requested() {
   }
   return v == 1;
 }
+// MXFP4 layers: decode (up to 8 tokens); the down kernel stages every slot's
+// SwiGLU output (S I floats, padded by 9/8) in shared memory.
+bool mx_supported(const moe_layer* L, int T) {
+  return T <= kDecodeMaxT && (size_t)slots_of(L) * (L->inter / 32) * 36 * sizeof(float) <= 227 * 1024;
+}
+
 Path path_of(const moe_layer* L, int T) {
+  if (is_mx(L)) return mx_supported(L, T) ? Path::kMx : Path::kNone;
   if (T > kDecodeMaxT) return prefill_supported(L->hidden, L->inter, L->bits) ? Path::kPrefill : Path::kNone;
   const bool fused = fused_supported(L->hidden, L->inter, L->n_experts, L->top_k, L->has_shared, L->bits);
   const bool chain = chain_supported(L->hidden, L->inter, L->top_k, L->has_shared, L->bits);
@@ -182,6 +198,49 @@ moe_status decode_chain(const moe_layer* L, const uint16_t* x_in, float* h, int 
   np.hacc = dp.hacc; np.h = h; np.gamma = L->rms_gamma; np.eps = L->rms_eps; np.x_out = x_out; np.x_out_f32 = x_out_f32;
   np.sel_flag = gp.sel_flag;
   if ((e = launch_norm_decode(np, pdl, s)) != cudaSuccess) return MOE_ERR_CUDA;
+  mark(4);
+  return MOE_OK;
+}
+
+// A decode layer of MXFP4 experts: router, certified top-k, gate/up with SwiGLU, down with the
+// weighted combine and the residual (mx.cu), RMSNorm.
+moe_status mx_chain(const moe_layer* L, const uint16_t* x_in, float* h, int T, uint16_t* x_out, float* x_out_f32,
+                    int32_t* topk_idx, float* topk_w, void* ws, cudaStream_t s, void* const* events = nullptr,
+                    uint16_t* x_rec = nullptr, float* h_rec = nullptr) {
+  auto mark = [&](int i) { if (events) cudaEventRecord((cudaEvent_t)events[i], s); };
+  mark(0);
+  const int H = L->hidden, I = L->inter, E = L->n_experts, k = L->top_k, S = slots_of(L);
+  const WsLayout W = layout_of(L, T);
+  RouteParams rp{};
+  rp.H = H; rp.E = E; rp.T = T; rp.has_shared = L->has_shared;
+  rp.x = x_in; rp.router_w = L->router_w; rp.router_bias = L->router_bias; rp.gate_w = L->shared_gate_w;
+  rp.logits = at<double>(ws, W.logits);
+  rp.bound = at<float>(ws, W.bound);
+  rp.h = h; rp.x_rec = x_rec; rp.h_rec = h_rec;
+  if (launch_route(rp, s, false) != cudaSuccess) return MOE_ERR_CUDA;
+  mark(1);
+  TopkParams tp{};
+  tp.E = E; tp.k = k; tp.T = T; tp.has_shared = L->has_shared; tp.H = H;
+  tp.logits = rp.logits; tp.bound = rp.bound;
+  tp.x = x_in; tp.router_w = L->router_w; tp.router_bias = L->router_bias;
+  tp.idx = at<int32_t>(ws, W.pidx); tp.w = at<float>(ws, W.pw); tp.sg = L->has_shared ? at<float>(ws, W.psg) : nullptr;
+  tp.rechecks = at<uint32_t>(ws, 16);
+  if (launch_topk(tp, s) != cudaSuccess) return MOE_ERR_CUDA;
+  const size_t sel = sizeof(int32_t) * (size_t)T * k;
+  if (topk_idx && cudaMemcpyAsync(topk_idx, tp.idx, sel, cudaMemcpyDeviceToDevice, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (topk_w && cudaMemcpyAsync(topk_w, tp.w, sel, cudaMemcpyDeviceToDevice, s) != cudaSuccess) return MOE_ERR_CUDA;
+  mark(2);
+  MxLayerParams mp{};
+  mp.H = H; mp.I = I; mp.k = k; mp.S = S; mp.T = T;
+  mp.x = x_in; mp.experts = L->experts; mp.shared = L->shared;
+  mp.idx = tp.idx; mp.w = tp.w; mp.sg = tp.sg;
+  mp.a = at<float>(ws, W.a); mp.h = h;
+  if (launch_mx_layer(mp, s) != cudaSuccess) return MOE_ERR_CUDA;
+  mark(3);
+  NormParams np{};
+  np.H = H; np.k = 0; np.T = T;
+  np.h = h; np.gamma = L->rms_gamma; np.eps = L->rms_eps; np.x_out = x_out; np.x_out_f32 = x_out_f32;
+  if (launch_norm(np, false, s) != cudaSuccess) return MOE_ERR_CUDA;
   mark(4);
   return MOE_OK;
 }
@@ -356,6 +415,7 @@ moe_status moe_layer_path(const moe_layer* layer, int32_t T, int32_t* path, int3
     case Path::kFused: code = MOE_PATH_FUSED; ev = 2; break;
     case Path::kChain: code = MOE_PATH_CHAIN; ev = 5; break;
     case Path::kPrefill: code = MOE_PATH_PREFILL; ev = 6; break;
+    case Path::kMx: code = MOE_PATH_MXFP4; ev = 5; break;
     default: return MOE_ERR_UNSUPPORTED;
   }
   if (path) *path = code;
@@ -491,6 +551,7 @@ moe_status moe_layer_forward(const moe_layer* layer, const uint16_t* x_in, float
     case Path::kFused:
       return fused_forward(layer, 1, x_in, h, x_out, x_out_f32, topk_idx, topk_w, nullptr, nullptr, ws, s);
     case Path::kChain: return decode_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, s);
+    case Path::kMx: return mx_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, s);
     default: return MOE_ERR_UNSUPPORTED;
   }
 }
@@ -513,6 +574,7 @@ moe_status moe_layer_forward_timed(const moe_layer* layer, const uint16_t* x_in,
   cudaStream_t s = (cudaStream_t)stream;
   if (path == Path::kPrefill)
     return prefill_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, s, events);
+  if (path == Path::kMx) return mx_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, s, events);
   if (path == Path::kFused) {
     if (cudaEventRecord((cudaEvent_t)events[0], s) != cudaSuccess) return MOE_ERR_CUDA;
     if ((st = fused_forward(layer, 1, x_in, h, x_out, x_out_f32, topk_idx, topk_w, nullptr, nullptr, ws, s)))
@@ -532,7 +594,7 @@ moe_status moe_stack_forward(const moe_layer* layers, int32_t L, const uint16_t*
     if ((st = check_layer(&layers[l]))) return st;
     const moe_layer& a = layers[l], &b = layers[0];
     if (a.hidden != b.hidden || a.inter != b.inter || a.n_experts != b.n_experts || a.top_k != b.top_k ||
-        a.bits != b.bits || a.has_shared != b.has_shared)
+        a.bits != b.bits || a.group != b.group || a.has_shared != b.has_shared)
       return MOE_ERR_INVALID_ARGUMENT;
   }
   if ((st = ws_check(&layers[0], 1, ws, ws_bytes))) return st;
@@ -553,6 +615,13 @@ moe_status moe_stack_forward(const moe_layer* layers, int32_t L, const uint16_t*
   }
   for (int l = 0; l < L; ++l) {
     const uint16_t* xin = l == 0 ? x_in : x_out;
+    if (path == Path::kMx) {
+      if ((st = mx_chain(&layers[l], xin, h, 1, x_out, nullptr, topk_idx_all ? topk_idx_all + (size_t)l * k : nullptr,
+                         nullptr, ws, s, nullptr, layer_inputs ? layer_inputs + (size_t)l * H : nullptr,
+                         layer_h ? layer_h + (size_t)l * H : nullptr)))
+        return st;
+      continue;
+    }
     if ((st = decode_chain(&layers[l], xin, h, 1, x_out, nullptr, topk_idx_all ? topk_idx_all + (size_t)l * k : nullptr,
                            nullptr, ws, s, nullptr, layer_inputs ? layer_inputs + (size_t)l * H : nullptr,
                            layer_h ? layer_h + (size_t)l * H : nullptr)))
@@ -609,6 +678,7 @@ moe_status moe_layer_forward_noalloc(const moe_layer* layer, const uint16_t* x_i
   // moe_noalloc_poll_status reads it. The kernels clear their own accumulators.
   if (path == Path::kFused)
     return fused_forward(layer, 1, x_in, h, x_out, x_out_f32, topk_idx, topk_w, nullptr, nullptr, ws, s);
+  if (path == Path::kMx) return mx_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, s);
   return decode_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, s);
 }
 

@@ -252,6 +252,17 @@ cudaError_t launch_mx_gemv(const uint32_t* q, const uint8_t* e, int R, int K, co
 cudaError_t launch_mx_gemm(const uint32_t* q, const uint8_t* e, int R, int K, const uint16_t* x, int T, float* y,
                            void* ws, unsigned long long wait_ns, cudaStream_t s);
 size_t mx_gemm_ws_bytes(int R, int K, int T);
+// a decode layer of MXFP4 experts, after the router and the top-k
+struct MxLayerParams {
+  int H, I, k, S, T;
+  const uint16_t* x;           // [T][H] bf16
+  const moe_expert* experts;   // device [E]: q codes, scales E8M0 bytes [R][K/32]
+  moe_expert shared;           // slot k when S > k
+  const int32_t* idx; const float* w; const float* sg;   // [T][k], [T][k], [T]
+  float* a;                    // [T][S][I]
+  float* h;                    // [T][H], in place: h + the weighted expert outputs
+};
+cudaError_t launch_mx_layer(const MxLayerParams& p, cudaStream_t s);
 cudaError_t launch_gateup(const GateUpParams& p, int bits, int T, bool pdl, cudaStream_t s);
 cudaError_t launch_down(const DownParams& p, int bits, int T, bool pdl, cudaStream_t s);
 cudaError_t launch_norm(const NormParams& p, bool pdl, cudaStream_t s);

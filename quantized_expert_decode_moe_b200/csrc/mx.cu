@@ -452,4 +452,140 @@ cudaError_t launch_mx_gemm(const uint32_t* q, const uint8_t* e, int R, int K, co
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ a decode layer of MXFP4 experts
+// After the router and the top-k (kernels.cu): gate/up with SwiGLU, then down
+// with the weighted combine and the residual, then the RMSNorm (kernels.cu).
+// The expert descriptors are the layer's: moe_qmat.q the codes, moe_qmat.scales
+// the E8M0 bytes [R][K/32] (uint8), biases unused.
+constexpr int kMxLWarps = 8;
+constexpr int kMxGuItems = 1;    // (slot, row) pairs per warp in gate/up
+constexpr int kMxDnRows = 1;     // hidden rows per warp in down
+constexpr int kMxMaxSlots = kMaxSlots;
+
+// dots of two MXFP4 rows (nb blocks each) with one staged vector (blocks of kMvXStride floats):
+// each lane's blocks of both rows are loaded before any is used; all lanes get both sums
+__device__ __forceinline__ float2 mx_row_dot2(const uint32_t* qa, const uint8_t* ea, const uint32_t* qb,
+                                              const uint8_t* eb, int nb, const float* xs, int lane) {
+  float2 acc = make_float2(0.f, 0.f);
+  for (int b0 = 0; b0 < nb; b0 += 4 * 32) {
+    uint4 ca[4], cb[4];
+    unsigned sa[4], sb[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int b = b0 + 32 * u + lane;
+      const bool in = b < nb;
+      ca[u] = in ? __ldg((const uint4*)qa + b) : make_uint4(0u, 0u, 0u, 0u);
+      cb[u] = in ? __ldg((const uint4*)qb + b) : make_uint4(0u, 0u, 0u, 0u);
+      sa[u] = in ? __ldg(ea + b) : 0u;
+      sb[u] = in ? __ldg(eb + b) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int b = b0 + 32 * u + lane;
+      if (b < nb) {
+        acc.x = fmaf(mx_block_dot(ca[u], xs + b * kMvXStride), mx_half_scale(sa[u]), acc.x);
+        acc.y = fmaf(mx_block_dot(cb[u], xs + b * kMvXStride), mx_half_scale(sb[u]), acc.y);
+      }
+    }
+  }
+  return make_float2(warp_sum(acc.x), warp_sum(acc.y));
+}
+
+__device__ __forceinline__ void mx_stage(float* dst, const float* src, int n) {   // n floats, n % 32 == 0
+  for (int i = threadIdx.x; i < n / 4; i += blockDim.x)
+    *(float4*)(dst + (i >> 3) * kMvXStride + 4 * (i & 7)) = *(const float4*)(src + 4 * i);
+}
+
+// grid (ceil(S I / (kMxLWarps kMxGuItems)), T), block 32 kMxLWarps: a[t][s][i] = silu(G x_t)_i (U x_t)_i
+// for the expert of slot s (slot k = the shared expert).
+__global__ void __launch_bounds__(kMxLWarps * 32) mx_gateup_kernel(MxLayerParams p) {
+  extern __shared__ __align__(16) float xs[];   // x_t, [H/32][kMvXStride]
+  const int t = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint16_t* xt = p.x + (size_t)t * p.H;
+  for (int i = threadIdx.x; i < p.H / 8; i += blockDim.x) {   // bf16 -> fp32, 8 values per thread
+    const uint4 v = __ldg((const uint4*)xt + i);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float* d = xs + (i >> 2) * kMvXStride + 8 * (i & 3);
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      d[2 * h] = bf16lo(w[h]);
+      d[2 * h + 1] = bf16hi(w[h]);
+    }
+  }
+  __syncthreads();
+  const int nb = p.H / 32;
+  for (int j = 0; j < kMxGuItems; ++j) {
+    const int item = (blockIdx.x * kMxLWarps + warp) * kMxGuItems + j;
+    if (item >= p.S * p.I) break;
+    const int sl = item / p.I, i = item % p.I;
+    const moe_expert* ex = sl < p.k ? p.experts + p.idx[t * p.k + sl] : &p.shared;
+    const moe_qmat G = ex->gate, U = ex->up;
+    const size_t qo = (size_t)i * (p.H / 8), eo = (size_t)i * nb;
+    const float2 gu = mx_row_dot2(G.q + qo, (const uint8_t*)G.scales + eo, U.q + qo, (const uint8_t*)U.scales + eo,
+                                  nb, xs, lane);
+    if (lane == 0) p.a[((size_t)t * p.S + sl) * p.I + i] = gu.x / (1.f + expf(-gu.x)) * gu.y;
+  }
+}
+
+// grid (ceil(H / (kMxLWarps kMxDnRows)), T), block 32 kMxLWarps:
+// h[t][j] += sum_{s<k} w[t][s] (D_s a[t][s])_j + sg[t] (D_shared a[t][k])_j, in that order.
+__global__ void __launch_bounds__(kMxLWarps * 32) mx_down_kernel(MxLayerParams p) {
+  extern __shared__ __align__(16) float as[];   // a[t][s], s < S: [S][I/32][kMvXStride]
+  const int t = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nb = p.I / 32, sstride = nb * kMvXStride;
+  for (int sl = 0; sl < p.S; ++sl) mx_stage(as + sl * sstride, p.a + ((size_t)t * p.S + sl) * p.I, p.I);
+  __syncthreads();
+  for (int j = 0; j < kMxDnRows; ++j) {
+    const int row = (blockIdx.x * kMxLWarps + warp) * kMxDnRows + j;
+    if (row >= p.H) break;
+    const uint4* q[kMxMaxSlots];
+    const uint8_t* e[kMxMaxSlots];
+#pragma unroll
+    for (int sl = 0; sl < kMxMaxSlots; ++sl)
+      if (sl < p.S) {
+        const moe_qmat D = sl < p.k ? p.experts[p.idx[t * p.k + sl]].down : p.shared.down;
+        q[sl] = (const uint4*)(D.q + (size_t)row * (p.I / 8));
+        e[sl] = (const uint8_t*)D.scales + (size_t)row * nb;
+      }
+    float y[kMxMaxSlots];
+#pragma unroll
+    for (int sl = 0; sl < kMxMaxSlots; ++sl) y[sl] = 0.f;
+    for (int b0 = 0; b0 < nb; b0 += 32) {   // every slot's block b in flight at once
+      const int b = b0 + lane;
+      uint4 c[kMxMaxSlots];
+      unsigned sc[kMxMaxSlots];
+#pragma unroll
+      for (int sl = 0; sl < kMxMaxSlots; ++sl) {
+        const bool in = sl < p.S && b < nb;
+        c[sl] = in ? __ldg(q[sl] + b) : make_uint4(0u, 0u, 0u, 0u);
+        sc[sl] = in ? __ldg(e[sl] + b) : 0u;
+      }
+#pragma unroll
+      for (int sl = 0; sl < kMxMaxSlots; ++sl)
+        if (sl < p.S && b < nb)
+          y[sl] = fmaf(mx_block_dot(c[sl], as + sl * sstride + b * kMvXStride), mx_half_scale(sc[sl]), y[sl]);
+    }
+    float acc = p.h[(size_t)t * p.H + row];
+#pragma unroll
+    for (int sl = 0; sl < kMxMaxSlots; ++sl)
+      if (sl < p.S) acc = fmaf(sl < p.k ? p.w[t * p.k + sl] : p.sg[t], warp_sum(y[sl]), acc);
+    if (lane == 0) p.h[(size_t)t * p.H + row] = acc;
+  }
+}
+
+cudaError_t launch_mx_layer(const MxLayerParams& p, cudaStream_t s) {
+  const size_t sg = sizeof(float) * (size_t)(p.H / 32) * kMvXStride;
+  const size_t sd = sizeof(float) * (size_t)p.S * (p.I / 32) * kMvXStride;
+  cudaError_t e = cudaFuncSetAttribute((const void*)mx_gateup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sg);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute((const void*)mx_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sd);
+  if (e != cudaSuccess) return e;
+  const int per = kMxLWarps * kMxGuItems;
+  mx_gateup_kernel<<<dim3((p.S * p.I + per - 1) / per, p.T), kMxLWarps * 32, sg, s>>>(p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int rows = kMxLWarps * kMxDnRows;
+  mx_down_kernel<<<dim3((p.H + rows - 1) / rows, p.T), kMxLWarps * 32, sd, s>>>(p);
+  return cudaGetLastError();
+}
+
 }  // namespace qmoe

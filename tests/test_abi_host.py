@@ -81,7 +81,9 @@ def test_workspace_size_and_layer_validation():
     rc4, n4 = ws_size(fake_layer(), T=4)
     assert rc4 == 0 and n4 > n
     assert ws_size(fake_layer(bits=3))[0] == 2            # unsupported bits
-    assert ws_size(fake_layer(group=32))[0] == 2          # unsupported group
+    assert ws_size(fake_layer(group=16))[0] == 2          # unsupported group
+    assert ws_size(fake_layer(group=32, bits=2))[0] == 2  # group 32 is the MXFP4 codec: 4-bit only
+    assert ws_size(fake_layer(group=32, bits=4))[0] == 0  # MXFP4 experts
     assert ws_size(fake_layer(top_k=9))[0] == 1           # k > 8
     assert ws_size(fake_layer(n_experts=2, top_k=3))[0] == 1   # k > E
     assert ws_size(fake_layer(hidden=4000))[0] == 1       # not a multiple of 128

@@ -139,3 +139,94 @@ def test_gemm_rejects_bad_shapes_before_launch(dev):
     with pytest.raises(qm.MoeError) as ex:   # R not a multiple of 128
         qm.moe_expert_gemm_mxfp4(qm.MxMat(W.q[:200], W.scales[:200]), x, y, ws=ws)
     assert ex.value.code == 2
+
+
+# ------------------------------------------------------------------ a decode layer of MXFP4 experts
+import fixtures  # noqa: E402
+
+
+def mx_layer(name, E, dev, scale=(116, 120)):
+    """The router, gamma and shared-gate vectors of a fixture layer with MXFP4 experts (seeded)."""
+    base = fixtures.CONFIGS[name]
+    cfg = base if E == base.E else fixtures.Config(base.name, H=base.H, E=E, k=base.k, I=base.I, bits=4,
+                                                   scale_sigma=base.scale_sigma)
+    Wr, rb, gs, gamma = fixtures.layer_vectors(cfg, 0)
+    H, I = cfg.H, cfg.I
+    host = [tuple(gen.mx_matrix(1000 + 3 * e + m, *((I, H) if m < 2 else (H, I)), *scale) for m in range(3))
+            for e in range(E + 1)]
+
+    def dev_expert(ex):
+        return qm.Expert(*[qm.QMat(torch.from_numpy(q.view(np.int32)).to(dev), torch.from_numpy(e).to(dev), None)
+                           for q, e in ex])
+
+    def t16(a):
+        return torch.from_numpy(a.view(np.int16)).to(dev)
+
+    layer = qm.Layer(hidden=H, inter=I, top_k=cfg.k, bits=4, group=32, router_w=t16(Wr),
+                     experts=[dev_expert(ex) for ex in host[:E]], rms_gamma=t16(gamma), shared=dev_expert(host[E]),
+                     shared_gate_w=t16(gs), router_bias=torch.from_numpy(rb).to(dev) if rb is not None else None,
+                     rms_eps=cfg.rms_eps)
+    return cfg, layer, host, (Wr, rb, gs, gamma)
+
+
+def run_mx_layer(cfg, layer, x, h0, dev):
+    T, H = x.shape
+    ws = qm.new_workspace(layer, T)
+    h = torch.from_numpy(h0.astype(np.float32)).to(dev)
+    xo = torch.empty((T, H), dtype=torch.int16, device=dev)
+    xf = torch.empty((T, H), dtype=torch.float32, device=dev)
+    idx = torch.empty((T, cfg.k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, cfg.k), dtype=torch.float32, device=dev)
+    qm.moe_layer_forward(layer, torch.from_numpy(x.view(np.int16)).to(dev), h, xo, xf, idx, w, ws=ws)
+    assert qm.moe_poll_status(ws) == 0
+    return h.cpu().numpy(), xf.cpu().numpy(), xo.cpu().numpy(), idx.cpu().numpy(), w.cpu().numpy()
+
+
+@pytest.mark.parametrize("name,E,T", [("tiny", 16, 1), ("tiny", 16, 3), ("tiny", 16, 8), ("layer_q4", 64, 1),
+                                      ("layer_q4", 64, 4)])
+def test_mx_layer_matches_oracle(dev, name, E, T):
+    """Router, top-k, MXFP4 gate/up + SwiGLU, down + weighted combine + residual, RMSNorm: routing
+    bit-exact, outputs within the layer tolerance of the oracle's composition of its own steps
+    (hidden 256 / 16 experts, and hidden 4096 / intermediate 1024 / 64 experts, top-3 + shared)."""
+    cfg, layer, host, (Wr, rb, gs, gamma) = mx_layer(name, E, dev)
+    x = gen.x_tokens(cfg, 31 + T, T=T)
+    h0 = gen.bf16_bits_to_f32(x).astype(np.float64) * 0.5
+    h, xf, xo, idx, w = run_mx_layer(cfg, layer, x, h0, dev)
+    ref = oracle.mx_layer(x, h0, Wr, gamma, host[:E], host[E], k=cfg.k, eps=cfg.rms_eps, router_bias=rb, gs=gs)
+    np.testing.assert_array_equal(idx, ref["idx"])
+    np.testing.assert_allclose(w, ref["w"], rtol=1e-6, atol=1e-7)
+    eh, ex_ = normwise(h, ref["h_out"]), normwise(xf, ref["x_out"])
+    assert eh <= 2e-3 and ex_ <= 2e-3, (eh, ex_)
+    assert eh <= 1e-4 and ex_ <= 1e-4, (eh, ex_)   # fp32 sums of exact products: far inside the bar
+    assert np.array_equal(xo.view(np.uint16), gen.f32_to_bf16_bits(xf))   # x_out is the RNE of x_out_f32
+    print(f"mxfp4 layer {name} E={E} T={T}: h' {eh:.2e}, x_out {ex_:.2e}")
+
+
+def test_mx_layer_path_and_limits(dev):
+    cfg, layer, _, _ = mx_layer("tiny", 16, dev)
+    path, nev = C_int(), C_int()
+    assert qm.lib().moe_layer_path(layer.cref(), 4, C.byref(path), C.byref(nev)) == 0
+    assert (path.value, nev.value) == (4, 5)
+    assert qm.lib().moe_layer_path(layer.cref(), 9, C.byref(path), C.byref(nev)) == 2   # decode only
+
+
+def test_mx_stack_equals_layer_by_layer(dev):
+    """Two MXFP4 layers through moe_stack_forward equal two moe_layer_forward calls, bit for bit."""
+    cfg, l0, _, _ = mx_layer("tiny", 16, dev)
+    _, l1, _, _ = mx_layer("tiny", 16, dev, scale=(115, 119))
+    x = gen.x_tokens(cfg, 5, T=1)
+    h0 = gen.bf16_bits_to_f32(x).astype(np.float32)
+    ws = qm.new_workspace(l0, 1)
+    h = torch.from_numpy(h0.copy()).to(dev)
+    xo = torch.empty((1, cfg.H), dtype=torch.int16, device=dev)
+    idx_all = torch.empty((2, cfg.k), dtype=torch.int32, device=dev)
+    qm.moe_stack_forward([l0, l1], torch.from_numpy(x.view(np.int16)).to(dev), h, xo, idx_all, ws=ws)
+    a = run_mx_layer(cfg, l0, x, h0, dev)
+    b = run_mx_layer(cfg, l1, a[2].view(np.uint16), a[0], dev)
+    np.testing.assert_array_equal(h.cpu().numpy(), b[0])
+    np.testing.assert_array_equal(xo.cpu().numpy(), b[2])
+    np.testing.assert_array_equal(idx_all.cpu().numpy(), np.stack([a[3][0], b[3][0]]))
+
+
+import ctypes as C  # noqa: E402
+C_int = C.c_int32
