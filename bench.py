@@ -40,7 +40,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=480)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="layer_q4",
-                    choices=["layer_q4", "layer_q2", "prefill_q4", "stack_q4", "cached_q4"],
+                    choices=["layer_q4", "layer_q2", "prefill_q4", "stack_q4", "cached_q4", "mxfp4_q4"],
                     help="prefill_q4: one step = one 512-token forward of the layer (the prefill path); "
                          "cached_q4: decode of layer_q4 with its routed experts in host memory and an HBM cache")
     ap.add_argument("--cache-slots", type=int, default=64, help="cached_q4: experts the HBM cache holds")
@@ -827,9 +827,203 @@ def ours_cached(args, cfg):
         print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ MXFP4 experts (--config mxfp4_q4)
+MX_METRIC = "MoE-layer decode tokens/s, MXFP4 experts (E2M1 + E8M0 per 32), 1 B200"
+
+
+def mx_bytes_per_expert(cfg) -> int:
+    return 3 * (cfg.I * cfg.H // 2 + cfg.I * cfg.H // 32)
+
+
+def mx_oracle_sample(cfg, seconds: float, max_tokens: int = 10 ** 9, warmup: int = 1, threads: int = 0):
+    """The oracle's MXFP4 layer on decode tokens of this workload (the touched experts regenerated
+    on the host before timing); returns (tokens/s, tokens, threads, seconds)."""
+    import numpy as np
+
+    import fixtures
+    import oracle
+    from fixtures import gen
+
+    threads = oracle.set_threads(threads if threads > 0 else (os.cpu_count() or 1))
+    Wr, rb, gs, gamma = fixtures.layer_vectors(cfg, 0)
+    cache = {}
+
+    def ex(e):
+        if e not in cache:
+            cache[e] = gen.mx_expert(e, cfg.H, cfg.I)
+        return cache[e]
+
+    shared = ex(cfg.E)
+    done, elapsed, s = 0, 0.0, 0
+    for timed in [False] * warmup + [True] * (10 ** 9):
+        if timed and (done >= max_tokens or (elapsed >= seconds and done >= 2)):
+            break
+        x = gen.x_tokens(cfg, 500 + s, T=1)
+        s += 1
+        idx, _, _ = oracle.route(x, Wr, cfg.k, bias=rb, gs=gs)
+        experts = {int(e): ex(int(e)) for e in idx[0]}
+        h0 = gen.bf16_bits_to_f32(x).astype(np.float64)
+        table = [experts.get(e) for e in range(cfg.E)]
+        t0 = time.perf_counter()
+        oracle.mx_layer(x, h0, Wr, gamma, table, shared, k=cfg.k, eps=cfg.rms_eps, router_bias=rb, gs=gs)
+        if timed:
+            elapsed += time.perf_counter() - t0
+            done += 1
+        if len(cache) > 48:
+            cache = {cfg.E: shared}
+    return done / elapsed, done, threads, elapsed
+
+
+def ours_mx(args, cfg):
+    """Decode of one 512-expert hidden-4096 layer whose experts are MXFP4 (moe_layer group 32): router,
+    certified top-k, MXFP4 gate/up + SwiGLU and down + combine + residual, RMSNorm. Tokens rotate over
+    64 inputs; the 3.4 GB expert pool is larger than L2."""
+    import numpy as np
+    import torch
+
+    import fixtures
+    import quantized_expert_decode_moe_b200 as qm
+    from fixtures import gen
+
+    world, rank, local = dist_info()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    qm.lib()
+    Wr, rb, gs, gamma = fixtures.layer_vectors(cfg, 0)
+
+    def t16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev)
+
+    experts = []
+    for e in range(cfg.E + 1):
+        mats = [qm.QMat(torch.from_numpy(q.view(np.int32)).to(dev), torch.from_numpy(sc).to(dev), None)
+                for q, sc in gen.mx_expert(e, cfg.H, cfg.I)]
+        experts.append(qm.Expert(*mats))
+    layer = qm.Layer(hidden=cfg.H, inter=cfg.I, top_k=cfg.k, bits=4, group=32, router_w=t16(Wr),
+                     experts=experts[:cfg.E], rms_gamma=t16(gamma), shared=experts[cfg.E], shared_gate_w=t16(gs),
+                     router_bias=torch.from_numpy(rb).to(dev) if rb is not None else None, rms_eps=cfg.rms_eps)
+    P = 64
+    x_host = gen.x_tokens(cfg, 900, T=P)
+    xs = torch.from_numpy(x_host.view(np.int16)).to(dev)
+    h0 = torch.from_numpy(gen.bf16_bits_to_f32(x_host).astype(np.float32)).to(dev)
+    hs = h0.clone()
+    xo = torch.empty((P, cfg.H), dtype=torch.int16, device=dev)
+    ws = qm.new_workspace(layer, 1)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(i):
+        qm.moe_layer_forward(layer, xs[i:i + 1], hs[i:i + 1], xo[i:i + 1], ws=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(P):
+            step(i)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(P):
+                step(i)
+        for _ in range(max(args.warmup, 3) // P + 1):
+            g.replay()
+    stream.synchronize()
+    assert qm.moe_poll_status(ws, stream) == 0
+    reps = max(1, args.steps // P)
+    steps = reps * P
+    gpu_uuid = str(getattr(torch.cuda.get_device_properties(dev), "uuid", "") or "")
+    clocks = Clocks(("GPU-" + gpu_uuid) if gpu_uuid and not gpu_uuid.startswith("GPU-") else (gpu_uuid or str(local)))
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        busy(g.replay, stream)
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+        busy(g.replay, stream)
+    e1.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    assert qm.moe_poll_status(ws, stream) == 0
+    # stages, timed one by one: router, top-k, MXFP4 experts (gate/up + down), RMSNorm
+    path, nev = qm.moe_layer_path(layer, 1)
+    nst = nev - 1
+    prof_n = min(args.prof_steps, 256)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(prof_n)]
+    with torch.cuda.stream(stream):
+        for row in evs:
+            for e in row:
+                e.record(stream)
+        for s in range(prof_n):
+            i = s % P
+            qm.moe_layer_forward_timed(layer, xs[i:i + 1], hs[i:i + 1], xo[i:i + 1], ws=ws, events=evs[s],
+                                       stream=stream)
+    stream.synchronize()
+    names = ["route_logits", "topk", "mx_gateup+mx_down", "norm"]
+    dur = [sum(evs[s][j].elapsed_time(evs[s][j + 1]) for s in range(prof_n)) / prof_n for j in range(nst)]
+    # end to end with host buffers: x and h in, x_out back, every step
+    e2e_n = min(args.e2e_steps, steps, 512)
+    inh, ind, xdev, hdev = packed_inputs(x_host.reshape(P, 1, cfg.H), h0.cpu().numpy().reshape(P, 1, cfg.H), dev)
+    outh = torch.empty((P, cfg.H), dtype=torch.int16).pin_memory()
+    odev = torch.empty((1, cfg.H), dtype=torch.int16, device=dev)
+    with torch.cuda.stream(stream):
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for s in range(e2e_n):
+            i = s % P
+            ind.copy_(inh[i], non_blocking=True)
+            qm.moe_layer_forward(layer, xdev, hdev, odev, ws=ws, stream=stream)
+            outh[i:i + 1].copy_(odev, non_blocking=True)
+        f1.record(stream)
+    f1.synchronize()
+    e2e_ms = f0.elapsed_time(f1)
+    peaks, peak_kind = measured_peaks()
+    per_tok = (cfg.k + 1) * mx_bytes_per_expert(cfg)
+    achieved = per_tok / (dur[2] * 1e-3) / 1e9
+    line = {
+        "metric": MX_METRIC, "value": steps / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world, "steps": steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms / steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "E2M1 codes x fp32 activations, fp32 block sums times E8M0 scales; router logits f64",
+        "data": "synthetic (seeded; no model weights)",
+        "config": {"workload": "one 512-expert hidden-4096 layer of MXFP4 experts, decode batch 1", "H": cfg.H,
+                   "E": cfg.E, "top_k": cfg.k, "shared": 1, "I": cfg.I, "codec": "mxfp4", "T": 1,
+                   "l2": "inputs larger than L2: 3.4 GB expert pool, 64 rotating tokens"},
+        "hbm_gbs": per_tok * steps / (ms * 1e-3) / 1e9, "active_bytes_per_token": per_tok,
+        "stage_ms": dict(zip(names, dur)),
+        "roofline": {"bound": "hbm", "kernel": "mx_gateup_kernel + mx_down_kernel", "achieved": achieved,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "algorithmic_bytes": per_tok, "peak_kind": peak_kind},
+        "e2e": {"value": e2e_n / (e2e_ms * 1e-3), "unit": "tokens/s", "steps": e2e_n,
+                "h2d_bytes_per_step": cfg.H * 6, "d2h_bytes_per_step": cfg.H * 2},
+        "gpu_launches": 5 * steps, "path": path, "clocks": clk,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        rate, n, threads, el = mx_oracle_sample(cfg, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                "sample": f"{n} decode tokens of this workload ({el:.1f} s of oracle time)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     import fixtures
+    if args.config == "mxfp4_q4":
+        cfg = fixtures.CONFIGS["layer_q4"]
+        if args.impl == "reference":
+            rate, n, threads, el = mx_oracle_sample(cfg, max(args.cpu_seconds, 5.0), max_tokens=max(1, args.steps))
+            line = {"impl": "reference", "metric": MX_METRIC, "value": rate, "unit": "tokens/s", "n_gpus": args.gpus,
+                    "steps": n, "warmup": max(args.warmup, 3), "ms_per_step": 1e3 * el / n,
+                    "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                    "data": "synthetic (seeded; no model weights)",
+                    "config": {"workload": "one 512-expert hidden-4096 layer of MXFP4 experts, decode batch 1"},
+                    "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                     "sample": f"{n} decode tokens"},
+                    "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            if dist_info()[1] == 0:
+                print(json.dumps(line), flush=True)
+        else:
+            ours_mx(args, cfg)
+        return
     if args.config == "cached_q4":
         cfg = fixtures.CONFIGS["layer_q4"]
         if args.impl == "reference":

@@ -261,3 +261,9 @@ def mx_matrix(seed: int, R: int, K: int, scale_lo: int = 118, scale_hi: int = 12
 def mx_tokens(seed: int, T: int, K: int, sigma: float = 1.0) -> np.ndarray:
     """T rows of K normal bf16 activations (bit patterns, uint16 [T][K])."""
     return normal_bf16(key_of(seed, 0, T_X, 7), T * K, sigma).reshape(T, K)
+
+
+def mx_expert(e: int, H: int, I: int, scale_lo: int = 116, scale_hi: int = 120):
+    """Expert e of a synthetic MXFP4 layer: ((qg, eg), (qu, eu), (qd, ed)), gate and up [I][H],
+    down [H][I] (scale bytes 116..120: 2^-11 .. 2^-7)."""
+    return tuple(mx_matrix(1000 + 3 * e + m, *((I, H) if m < 2 else (H, I)), scale_lo, scale_hi) for m in range(3))

@@ -193,7 +193,7 @@ def moe_workspace_size(layer: Layer, max_tokens: int) -> int:
     return n.value
 
 
-PATHS = {1: "fused", 2: "chain", 3: "prefill"}
+PATHS = {1: "fused", 2: "chain", 3: "prefill", 4: "mxfp4"}
 
 
 def moe_layer_path(layer: Layer, T: int):

@@ -152,8 +152,7 @@ def mx_layer(name, E, dev, scale=(116, 120)):
                                                    scale_sigma=base.scale_sigma)
     Wr, rb, gs, gamma = fixtures.layer_vectors(cfg, 0)
     H, I = cfg.H, cfg.I
-    host = [tuple(gen.mx_matrix(1000 + 3 * e + m, *((I, H) if m < 2 else (H, I)), *scale) for m in range(3))
-            for e in range(E + 1)]
+    host = [gen.mx_expert(e, H, I, *scale) for e in range(E + 1)]
 
     def dev_expert(ex):
         return qm.Expert(*[qm.QMat(torch.from_numpy(q.view(np.int32)).to(dev), torch.from_numpy(e).to(dev), None)
