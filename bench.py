@@ -211,6 +211,7 @@ DECODE_SOURCES = ("common.cuh", "kernels.cuh", "decode.cu", "stage.cuh", "sync.c
 ROUTER_SOURCES = ("common.cuh", "kernels.cu", "kernels.cuh", "topk.cuh")                           # router, norm
 FUSED_SOURCES = ("common.cuh", "kernels.cuh", "fused.cu", "stage.cuh", "sync.cuh", "topk.cuh")
 PREFILL_SOURCES = ("common.cuh", "kernels.cuh", "prefill.cu")
+MX_SOURCES = ("common.cuh", "kernels.cuh", "mx.cu")
 SOURCES_OF = {"route_logits_kernel": ROUTER_SOURCES, "norm_kernel": ROUTER_SOURCES,
               "fused_decode_kernel": FUSED_SOURCES}
 
@@ -990,7 +991,8 @@ def ours_mx(args, cfg):
         "hbm_gbs": per_tok * steps / (ms * 1e-3) / 1e9, "active_bytes_per_token": per_tok,
         "stage_ms": dict(zip(names, dur)),
         "roofline": {"bound": "hbm", "kernel": "mx_gateup_kernel + mx_down_kernel", "achieved": achieved,
-                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": recorded_traffic("mx_experts", "mxfp4_q4", MX_SOURCES),
                      "algorithmic_bytes": per_tok, "peak_kind": peak_kind},
         "e2e": {"value": e2e_n / (e2e_ms * 1e-3), "unit": "tokens/s", "steps": e2e_n,
                 "h2d_bytes_per_step": cfg.H * 6, "d2h_bytes_per_step": cfg.H * 2},
