@@ -9,10 +9,13 @@
 //
 // Two entry points:
 //  * mx_gemv_kernel: y = W x (decode). A warp per row, a lane per 32-element
-//    block: the 16 code bytes of the block in one load, each nibble decoded to
-//    2|v| by a byte permutation (the eight magnitudes 0..12 as a byte table),
-//    the sign bit moved into the float, an fp32 FMA with x (staged in shared
-//    memory), the block sum times 2^(byte - 128).
+//    block: the 16 code bytes of the block in one load. A code's magnitude
+//    field f, shifted to bit 22 of an fp32 word, is |v| 2^-126 exactly (f = 1,
+//    the subnormal E2M1 value 0.5, lands on the fp32 subnormal 2^-127), and its
+//    sign bit goes to bit 31: three integer operations per element, then
+//    packed fp32x2 FMAs against x staged per block as x 2^s (the block's
+//    largest |x| brought near 2^50, so every product is a normal float); the
+//    block sum times 2^(126 - s) and the E8M0 scale 2^(byte - 127).
 //  * mx_gemm_kernel: Y = X W^T for many tokens on the tcgen05 tensor cores,
 //    kind::mxf4 with block scaling: the weight codes go from HBM to shared
 //    memory unchanged (TMA tiles of 16 bytes x 128 rows, i.e. one MX block of
@@ -41,30 +44,98 @@ namespace qmoe {
 constexpr int kMvWarps = 8;
 constexpr int kMvXStride = 36;   // floats per 32-element block of x in shared memory (padded)
 
-// 2^(byte - 128): the block scale times 1/2, as the nibbles decode to 2|v|; NaN for 0xFF
-__device__ __forceinline__ float mx_half_scale(unsigned byte) {
-  return byte == 0xFFu ? __int_as_float(0x7FC00000) : ldexpf(1.0f, (int)byte - 128);
+// 2^n for n in [-149, 127], from its bits (subnormal below 2^-126)
+__device__ __forceinline__ float mx_pow2(int n) {
+  return n >= -126 ? __int_as_float((n + 127) << 23) : __int_as_float(1 << (n + 149));
 }
 
-// sum over one 32-element block of (2 e2m1(code_k)) x_k; xs: the block's 32 values of x
+// the E8M0 scale 2^(byte - 127); NaN for 0xFF
+__device__ __forceinline__ float mx_scale(unsigned byte) {
+  return byte == 0xFFu ? __int_as_float(0x7FC00000) : mx_pow2((int)byte - 127);
+}
+
+// packed fp32x2 arithmetic (two values in one 64-bit register, the first in the low half)
+__device__ __forceinline__ unsigned long long f2_pack(uint32_t lo, uint32_t hi) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b,
+                                                     unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ float f2_sum(unsigned long long v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return lo + hi;
+}
+
+// element j of a code word as the fp32 bits of |v| 2^-126 with v's sign: the magnitude field
+// at bit 22 (field 1, the subnormal value 0.5, is the fp32 subnormal 2^-127), the sign at bit 31
+__device__ __forceinline__ uint32_t mx_code_bits(uint32_t w, int j) {
+  const uint32_t mag = j <= 5 ? (w << (22 - 4 * j)) : (w >> (4 * j - 22));
+  return ((w << (28 - 4 * j)) & 0x80000000u) | (mag & 0x01C00000u);
+}
+
+// sum over one 32-element block of e2m1(code_k) x_k; xs: the block as mx_stage_block left it
+// (32 values x_k 2^s, then the factor 2^(126 - s) in slot 32)
 __device__ __forceinline__ float mx_block_dot(const uint4 c, const float* xs) {
   const uint32_t w[4] = {c.x, c.y, c.z, c.w};
-  float s = 0.f;
+  unsigned long long acc = 0ull;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const float4 xa = *(const float4*)(xs + 8 * i), xb = *(const float4*)(xs + 8 * i + 4);
-    const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-    // byte table of 2|v| for the magnitude fields 0..7: 0, 1, 2, 3, 4, 6, 8, 12
-    const uint32_t lo = __byte_perm(0x03020100u, 0x0C080604u, w[i] & 0x7777u);
-    const uint32_t hi = __byte_perm(0x03020100u, 0x0C080604u, (w[i] >> 16) & 0x7777u);
+    const ulonglong2 xa = *(const ulonglong2*)(xs + 8 * i), xb = *(const ulonglong2*)(xs + 8 * i + 4);
+    acc = f2_fma(f2_pack(mx_code_bits(w[i], 0), mx_code_bits(w[i], 1)), xa.x, acc);
+    acc = f2_fma(f2_pack(mx_code_bits(w[i], 2), mx_code_bits(w[i], 3)), xa.y, acc);
+    acc = f2_fma(f2_pack(mx_code_bits(w[i], 4), mx_code_bits(w[i], 5)), xb.x, acc);
+    acc = f2_fma(f2_pack(mx_code_bits(w[i], 6), mx_code_bits(w[i], 7)), xb.y, acc);
+  }
+  return f2_sum(acc) * xs[32];
+}
+
+// Stages one 32-value block: x 2^s, with s the power of two that brings the block's largest |x|
+// into [2^50, 2^51) (clamped to [-1, 126], so 2^s and the factor 2^(126 - s) are normal floats),
+// then the factor in slot 32. Exact: scaling by powers of two.
+__device__ __forceinline__ void mx_stage_block(const float (&v)[32], float* dst) {
+  float m = 0.f;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const uint32_t mag = ((j < 4 ? lo : hi) >> (8 * (j & 3))) & 0xFFu;
-      const uint32_t sgn = (w[i] << (28 - 4 * j)) & 0x80000000u;   // bit 4j+3 -> bit 31
-      s = fmaf(__uint_as_float(__float_as_uint((float)mag) ^ sgn), xv[j], s);
+  for (int k = 0; k < 32; ++k) m = fmaxf(m, fabsf(v[k]));
+  int sc = 0;
+  if (m > 0.f) {
+    const int e = m >= 0x1p-126f ? (int)((__float_as_uint(m) >> 23) & 0xFFu) - 127 : -127;   // floor(log2 m)
+    sc = min(126, max(-1, 50 - e));
+  }
+  const float up = mx_pow2(sc);
+#pragma unroll
+  for (int k = 0; k < 32; k += 4)
+    *(float4*)(dst + k) = make_float4(v[k] * up, v[k + 1] * up, v[k + 2] * up, v[k + 3] * up);
+  dst[32] = mx_pow2(126 - sc);
+}
+// one block of 32 fp32 / 32 bf16 values from global memory into shared memory
+__device__ __forceinline__ void mx_stage_f32(const float* src, float* dst) {
+  float v[32];
+#pragma unroll
+  for (int k = 0; k < 32; k += 4) {
+    const float4 q = __ldg((const float4*)(src + k));
+    v[k] = q.x; v[k + 1] = q.y; v[k + 2] = q.z; v[k + 3] = q.w;
+  }
+  mx_stage_block(v, dst);
+}
+__device__ __forceinline__ void mx_stage_bf16(const uint16_t* src, float* dst) {
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 u = __ldg((const uint4*)src + i);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      v[8 * i + 2 * h] = bf16lo(w[h]);
+      v[8 * i + 2 * h + 1] = bf16hi(w[h]);
     }
   }
-  return s;
+  mx_stage_block(v, dst);
 }
 
 // grid ceil(R / kMvWarps), block 32 kMvWarps: warp w of CTA b computes row b kMvWarps + w.
@@ -73,10 +144,7 @@ __global__ void __launch_bounds__(kMvWarps * 32) mx_gemv_kernel(const uint32_t* 
                                                                 const float* __restrict__ x, float* __restrict__ y) {
   extern __shared__ __align__(16) float xs[];   // [K/32][kMvXStride]
   const int nb = K / 32;
-  for (int i = threadIdx.x; i < K / 4; i += blockDim.x) {
-    const float4 v = __ldg((const float4*)x + i);
-    *(float4*)(xs + (i >> 3) * kMvXStride + 4 * (i & 7)) = v;
-  }
+  for (int b = threadIdx.x; b < nb; b += blockDim.x) mx_stage_f32(x + 32 * b, xs + b * kMvXStride);
   __syncthreads();
   const int lane = threadIdx.x & 31, r = blockIdx.x * kMvWarps + (threadIdx.x >> 5);
   if (r >= R) return;
@@ -95,7 +163,7 @@ __global__ void __launch_bounds__(kMvWarps * 32) mx_gemv_kernel(const uint32_t* 
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int b = b0 + 32 * u + lane;
-      if (b < nb) acc = fmaf(mx_block_dot(c[u], xs + b * kMvXStride), mx_half_scale(sb[u]), acc);
+      if (b < nb) acc = fmaf(mx_block_dot(c[u], xs + b * kMvXStride), mx_scale(sb[u]), acc);
     }
   }
   acc = warp_sum(acc);
@@ -136,11 +204,6 @@ static_assert(kMxN + kMxStages * kMxSfCols <= 256, "accumulator and scales fit 2
 // column m1 of lane m0 of every 32-lane group, the layout the block-scaled
 // MMA reads (scale j of the word selected by the descriptor's scale id).
 __host__ __device__ __forceinline__ int mx_sf_off(int m, int j) { return (m & 31) * 16 + (m >> 5) * 4 + j; }
-
-// 2^n for n in [-149, 127], from its bits (subnormal below 2^-126)
-__device__ __forceinline__ float mx_pow2(int n) {
-  return n >= -126 ? __int_as_float((n + 127) << 23) : __int_as_float(1 << (n + 149));
-}
 
 // grid T_pad + ceil(R nstg / kMxPrepThreads), block kMxPrepThreads.
 //  CTA t < T_pad: token row t (zeros beyond T); thread i takes the 32-element
@@ -458,119 +521,129 @@ cudaError_t launch_mx_gemm(const uint32_t* q, const uint8_t* e, int R, int K, co
 // The expert descriptors are the layer's: moe_qmat.q the codes, moe_qmat.scales
 // the E8M0 bytes [R][K/32] (uint8), biases unused.
 constexpr int kMxLWarps = 8;
-constexpr int kMxGuItems = 1;    // (slot, row) pairs per warp in gate/up
-constexpr int kMxDnRows = 1;     // hidden rows per warp in down
 constexpr int kMxMaxSlots = kMaxSlots;
 
-// dots of two MXFP4 rows (nb blocks each) with one staged vector (blocks of kMvXStride floats):
-// each lane's blocks of both rows are loaded before any is used; all lanes get both sums
-__device__ __forceinline__ float2 mx_row_dot2(const uint32_t* qa, const uint8_t* ea, const uint32_t* qb,
-                                              const uint8_t* eb, int nb, const float* xs, int lane) {
-  float2 acc = make_float2(0.f, 0.f);
-  for (int b0 = 0; b0 < nb; b0 += 4 * 32) {
-    uint4 ca[4], cb[4];
-    unsigned sa[4], sb[4];
+// One lane's share of a 128-block chunk of two MXFP4 rows: blocks b0 + 32 u + lane, u < 4.
+struct MxChunk2 {
+  uint4 ca[4], cb[4];
+  unsigned sa[4], sb[4];
+};
+__device__ __forceinline__ void mx_load2(MxChunk2& c, const uint32_t* qa, const uint8_t* ea, const uint32_t* qb,
+                                         const uint8_t* eb, int b0, int nb, int lane) {
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int b = b0 + 32 * u + lane;
-      const bool in = b < nb;
-      ca[u] = in ? __ldg((const uint4*)qa + b) : make_uint4(0u, 0u, 0u, 0u);
-      cb[u] = in ? __ldg((const uint4*)qb + b) : make_uint4(0u, 0u, 0u, 0u);
-      sa[u] = in ? __ldg(ea + b) : 0u;
-      sb[u] = in ? __ldg(eb + b) : 0u;
-    }
+  for (int u = 0; u < 4; ++u) {
+    const int b = b0 + 32 * u + lane;
+    const bool in = b < nb;
+    c.ca[u] = in ? __ldg((const uint4*)qa + b) : make_uint4(0u, 0u, 0u, 0u);
+    c.cb[u] = in ? __ldg((const uint4*)qb + b) : make_uint4(0u, 0u, 0u, 0u);
+    c.sa[u] = in ? __ldg(ea + b) : 0u;
+    c.sb[u] = in ? __ldg(eb + b) : 0u;
+  }
+}
+__device__ __forceinline__ void mx_dot2(const MxChunk2& c, int b0, int nb, const float* xs, int lane, float2& acc) {
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int b = b0 + 32 * u + lane;
-      if (b < nb) {
-        acc.x = fmaf(mx_block_dot(ca[u], xs + b * kMvXStride), mx_half_scale(sa[u]), acc.x);
-        acc.y = fmaf(mx_block_dot(cb[u], xs + b * kMvXStride), mx_half_scale(sb[u]), acc.y);
-      }
+  for (int u = 0; u < 4; ++u) {
+    const int b = b0 + 32 * u + lane;
+    if (b < nb) {
+      acc.x = fmaf(mx_block_dot(c.ca[u], xs + b * kMvXStride), mx_scale(c.sa[u]), acc.x);
+      acc.y = fmaf(mx_block_dot(c.cb[u], xs + b * kMvXStride), mx_scale(c.sb[u]), acc.y);
     }
   }
-  return make_float2(warp_sum(acc.x), warp_sum(acc.y));
 }
 
 __device__ __forceinline__ void mx_stage(float* dst, const float* src, int n) {   // n floats, n % 32 == 0
-  for (int i = threadIdx.x; i < n / 4; i += blockDim.x)
-    *(float4*)(dst + (i >> 3) * kMvXStride + 4 * (i & 7)) = *(const float4*)(src + 4 * i);
+  for (int b = threadIdx.x; b < n / 32; b += blockDim.x) mx_stage_f32(src + 32 * b, dst + b * kMvXStride);
 }
 
-// grid (ceil(S I / (kMxLWarps kMxGuItems)), T), block 32 kMxLWarps: a[t][s][i] = silu(G x_t)_i (U x_t)_i
-// for the expert of slot s (slot k = the shared expert).
+// grid (ceil(S I / kMxLWarps), T), block 32 kMxLWarps: a[t][s][i] = silu(G x_t)_i (U x_t)_i for the
+// expert of slot s (slot k = the shared expert), one (slot, row) per warp. Each warp resolves its
+// expert and requests its rows' first blocks before the CTA stages x_t, so the dependent loads
+// (selection, descriptor, codes) overlap the staging.
 __global__ void __launch_bounds__(kMxLWarps * 32) mx_gateup_kernel(MxLayerParams p) {
   extern __shared__ __align__(16) float xs[];   // x_t, [H/32][kMvXStride]
   const int t = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const uint16_t* xt = p.x + (size_t)t * p.H;
-  for (int i = threadIdx.x; i < p.H / 8; i += blockDim.x) {   // bf16 -> fp32, 8 values per thread
-    const uint4 v = __ldg((const uint4*)xt + i);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    float* d = xs + (i >> 2) * kMvXStride + 8 * (i & 3);
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      d[2 * h] = bf16lo(w[h]);
-      d[2 * h + 1] = bf16hi(w[h]);
-    }
-  }
-  __syncthreads();
   const int nb = p.H / 32;
-  for (int j = 0; j < kMxGuItems; ++j) {
-    const int item = (blockIdx.x * kMxLWarps + warp) * kMxGuItems + j;
-    if (item >= p.S * p.I) break;
-    const int sl = item / p.I, i = item % p.I;
+  const int item = blockIdx.x * kMxLWarps + warp;
+  const bool has = item < p.S * p.I;
+  const int sl = has ? item / p.I : 0, i = has ? item % p.I : 0;
+  const uint32_t *gq = nullptr, *uq = nullptr;
+  const uint8_t *ge = nullptr, *ue = nullptr;
+  MxChunk2 c;
+  if (has) {
     const moe_expert* ex = sl < p.k ? p.experts + p.idx[t * p.k + sl] : &p.shared;
-    const moe_qmat G = ex->gate, U = ex->up;
-    const size_t qo = (size_t)i * (p.H / 8), eo = (size_t)i * nb;
-    const float2 gu = mx_row_dot2(G.q + qo, (const uint8_t*)G.scales + eo, U.q + qo, (const uint8_t*)U.scales + eo,
-                                  nb, xs, lane);
-    if (lane == 0) p.a[((size_t)t * p.S + sl) * p.I + i] = gu.x / (1.f + expf(-gu.x)) * gu.y;
+    gq = ex->gate.q + (size_t)i * (p.H / 8);
+    uq = ex->up.q + (size_t)i * (p.H / 8);
+    ge = (const uint8_t*)ex->gate.scales + (size_t)i * nb;
+    ue = (const uint8_t*)ex->up.scales + (size_t)i * nb;
+    mx_load2(c, gq, ge, uq, ue, 0, nb, lane);
   }
+  const uint16_t* xt = p.x + (size_t)t * p.H;
+  for (int b = threadIdx.x; b < nb; b += blockDim.x) mx_stage_bf16(xt + 32 * b, xs + b * kMvXStride);
+  __syncthreads();
+  if (!has) return;
+  float2 acc = make_float2(0.f, 0.f);
+  for (int b0 = 0;;) {
+    mx_dot2(c, b0, nb, xs, lane, acc);
+    b0 += 4 * 32;
+    if (b0 >= nb) break;
+    mx_load2(c, gq, ge, uq, ue, b0, nb, lane);
+  }
+  const float g = warp_sum(acc.x), u = warp_sum(acc.y);
+  if (lane == 0) p.a[((size_t)t * p.S + sl) * p.I + i] = g / (1.f + expf(-g)) * u;
 }
 
-// grid (ceil(H / (kMxLWarps kMxDnRows)), T), block 32 kMxLWarps:
+// grid (ceil(H / kMxLWarps), T), block 32 kMxLWarps, a hidden row per warp:
 // h[t][j] += sum_{s<k} w[t][s] (D_s a[t][s])_j + sg[t] (D_shared a[t][k])_j, in that order.
-__global__ void __launch_bounds__(kMxLWarps * 32) mx_down_kernel(MxLayerParams p) {
+// Each warp requests every slot's first blocks of its row before the CTA stages a[t].
+__global__ void __launch_bounds__(kMxLWarps * 32, 2) mx_down_kernel(MxLayerParams p) {
   extern __shared__ __align__(16) float as[];   // a[t][s], s < S: [S][I/32][kMvXStride]
   const int t = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nb = p.I / 32, sstride = nb * kMvXStride;
+  const int row = blockIdx.x * kMxLWarps + warp;
+  const bool has = row < p.H;
+  const uint4* q[kMxMaxSlots];
+  const uint8_t* e[kMxMaxSlots];
+  uint4 c[kMxMaxSlots];
+  unsigned sc[kMxMaxSlots];
+#pragma unroll
+  for (int sl = 0; sl < kMxMaxSlots; ++sl) {
+    q[sl] = nullptr;
+    e[sl] = nullptr;
+    if (has && sl < p.S) {
+      const moe_qmat D = sl < p.k ? p.experts[p.idx[t * p.k + sl]].down : p.shared.down;
+      q[sl] = (const uint4*)(D.q + (size_t)row * (p.I / 8));
+      e[sl] = (const uint8_t*)D.scales + (size_t)row * nb;
+    }
+    const bool in = q[sl] && lane < nb;
+    c[sl] = in ? __ldg(q[sl] + lane) : make_uint4(0u, 0u, 0u, 0u);
+    sc[sl] = in ? __ldg(e[sl] + lane) : 0u;
+  }
   for (int sl = 0; sl < p.S; ++sl) mx_stage(as + sl * sstride, p.a + ((size_t)t * p.S + sl) * p.I, p.I);
   __syncthreads();
-  for (int j = 0; j < kMxDnRows; ++j) {
-    const int row = (blockIdx.x * kMxLWarps + warp) * kMxDnRows + j;
-    if (row >= p.H) break;
-    const uint4* q[kMxMaxSlots];
-    const uint8_t* e[kMxMaxSlots];
+  if (!has) return;
+  float y[kMxMaxSlots];
+#pragma unroll
+  for (int sl = 0; sl < kMxMaxSlots; ++sl) y[sl] = 0.f;
+  for (int b0 = 0;;) {   // every slot's block b0 + lane in flight at once
+    const int b = b0 + lane;
 #pragma unroll
     for (int sl = 0; sl < kMxMaxSlots; ++sl)
-      if (sl < p.S) {
-        const moe_qmat D = sl < p.k ? p.experts[p.idx[t * p.k + sl]].down : p.shared.down;
-        q[sl] = (const uint4*)(D.q + (size_t)row * (p.I / 8));
-        e[sl] = (const uint8_t*)D.scales + (size_t)row * nb;
-      }
-    float y[kMxMaxSlots];
+      if (sl < p.S && b < nb)
+        y[sl] = fmaf(mx_block_dot(c[sl], as + sl * sstride + b * kMvXStride), mx_scale(sc[sl]), y[sl]);
+    b0 += 32;
+    if (b0 >= nb) break;
 #pragma unroll
-    for (int sl = 0; sl < kMxMaxSlots; ++sl) y[sl] = 0.f;
-    for (int b0 = 0; b0 < nb; b0 += 32) {   // every slot's block b in flight at once
-      const int b = b0 + lane;
-      uint4 c[kMxMaxSlots];
-      unsigned sc[kMxMaxSlots];
-#pragma unroll
-      for (int sl = 0; sl < kMxMaxSlots; ++sl) {
-        const bool in = sl < p.S && b < nb;
-        c[sl] = in ? __ldg(q[sl] + b) : make_uint4(0u, 0u, 0u, 0u);
-        sc[sl] = in ? __ldg(e[sl] + b) : 0u;
-      }
-#pragma unroll
-      for (int sl = 0; sl < kMxMaxSlots; ++sl)
-        if (sl < p.S && b < nb)
-          y[sl] = fmaf(mx_block_dot(c[sl], as + sl * sstride + b * kMvXStride), mx_half_scale(sc[sl]), y[sl]);
+    for (int sl = 0; sl < kMxMaxSlots; ++sl) {
+      const bool in = sl < p.S && b0 + lane < nb;
+      c[sl] = in ? __ldg(q[sl] + b0 + lane) : make_uint4(0u, 0u, 0u, 0u);
+      sc[sl] = in ? __ldg(e[sl] + b0 + lane) : 0u;
     }
-    float acc = p.h[(size_t)t * p.H + row];
-#pragma unroll
-    for (int sl = 0; sl < kMxMaxSlots; ++sl)
-      if (sl < p.S) acc = fmaf(sl < p.k ? p.w[t * p.k + sl] : p.sg[t], warp_sum(y[sl]), acc);
-    if (lane == 0) p.h[(size_t)t * p.H + row] = acc;
   }
+  float acc = p.h[(size_t)t * p.H + row];
+#pragma unroll
+  for (int sl = 0; sl < kMxMaxSlots; ++sl)
+    if (sl < p.S) acc = fmaf(sl < p.k ? p.w[t * p.k + sl] : p.sg[t], warp_sum(y[sl]), acc);
+  if (lane == 0) p.h[(size_t)t * p.H + row] = acc;
 }
 
 cudaError_t launch_mx_layer(const MxLayerParams& p, cudaStream_t s) {
@@ -580,11 +653,9 @@ cudaError_t launch_mx_layer(const MxLayerParams& p, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute((const void*)mx_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sd);
   if (e != cudaSuccess) return e;
-  const int per = kMxLWarps * kMxGuItems;
-  mx_gateup_kernel<<<dim3((p.S * p.I + per - 1) / per, p.T), kMxLWarps * 32, sg, s>>>(p);
+  mx_gateup_kernel<<<dim3((p.S * p.I + kMxLWarps - 1) / kMxLWarps, p.T), kMxLWarps * 32, sg, s>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const int rows = kMxLWarps * kMxDnRows;
-  mx_down_kernel<<<dim3((p.H + rows - 1) / rows, p.T), kMxLWarps * 32, sd, s>>>(p);
+  mx_down_kernel<<<dim3((p.H + kMxLWarps - 1) / kMxLWarps, p.T), kMxLWarps * 32, sd, s>>>(p);
   return cudaGetLastError();
 }
 
