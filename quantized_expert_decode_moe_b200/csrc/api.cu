@@ -207,6 +207,7 @@ moe_status decode_chain(const moe_layer* L, const uint16_t* x_in, float* h, int 
 moe_status mx_chain(const moe_layer* L, const uint16_t* x_in, float* h, int T, uint16_t* x_out, float* x_out_f32,
                     int32_t* topk_idx, float* topk_w, void* ws, cudaStream_t s, void* const* events = nullptr,
                     uint16_t* x_rec = nullptr, float* h_rec = nullptr) {
+  const bool pdl = events == nullptr && !topk_idx && !topk_w;   // programmatic launches between the kernels
   auto mark = [&](int i) { if (events) cudaEventRecord((cudaEvent_t)events[i], s); };
   mark(0);
   const int H = L->hidden, I = L->inter, E = L->n_experts, k = L->top_k, S = slots_of(L);
@@ -217,7 +218,7 @@ moe_status mx_chain(const moe_layer* L, const uint16_t* x_in, float* h, int T, u
   rp.logits = at<double>(ws, W.logits);
   rp.bound = at<float>(ws, W.bound);
   rp.h = h; rp.x_rec = x_rec; rp.h_rec = h_rec;
-  if (launch_route(rp, s, false) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_route(rp, s, pdl) != cudaSuccess) return MOE_ERR_CUDA;
   mark(1);
   TopkParams tp{};
   tp.E = E; tp.k = k; tp.T = T; tp.has_shared = L->has_shared; tp.H = H;
@@ -225,7 +226,7 @@ moe_status mx_chain(const moe_layer* L, const uint16_t* x_in, float* h, int T, u
   tp.x = x_in; tp.router_w = L->router_w; tp.router_bias = L->router_bias;
   tp.idx = at<int32_t>(ws, W.pidx); tp.w = at<float>(ws, W.pw); tp.sg = L->has_shared ? at<float>(ws, W.psg) : nullptr;
   tp.rechecks = at<uint32_t>(ws, 16);
-  if (launch_topk(tp, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_topk(tp, s, pdl) != cudaSuccess) return MOE_ERR_CUDA;
   const size_t sel = sizeof(int32_t) * (size_t)T * k;
   if (topk_idx && cudaMemcpyAsync(topk_idx, tp.idx, sel, cudaMemcpyDeviceToDevice, s) != cudaSuccess) return MOE_ERR_CUDA;
   if (topk_w && cudaMemcpyAsync(topk_w, tp.w, sel, cudaMemcpyDeviceToDevice, s) != cudaSuccess) return MOE_ERR_CUDA;
@@ -235,12 +236,12 @@ moe_status mx_chain(const moe_layer* L, const uint16_t* x_in, float* h, int T, u
   mp.x = x_in; mp.experts = L->experts; mp.shared = L->shared;
   mp.idx = tp.idx; mp.w = tp.w; mp.sg = tp.sg;
   mp.a = at<float>(ws, W.a); mp.h = h;
-  if (launch_mx_layer(mp, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_mx_layer(mp, s, pdl) != cudaSuccess) return MOE_ERR_CUDA;
   mark(3);
   NormParams np{};
   np.H = H; np.k = 0; np.T = T;
   np.h = h; np.gamma = L->rms_gamma; np.eps = L->rms_eps; np.x_out = x_out; np.x_out_f32 = x_out_f32;
-  if (launch_norm(np, false, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_norm(np, pdl, s) != cudaSuccess) return MOE_ERR_CUDA;
   mark(4);
   return MOE_OK;
 }

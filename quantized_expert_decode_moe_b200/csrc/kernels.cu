@@ -199,6 +199,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_logits_kernel(RouteParams
 __global__ void __launch_bounds__(kThreads) topk_kernel(TopkParams p) {
   __shared__ TopkSmem ts;
   const int t = blockIdx.x, tid = threadIdx.x;
+  griddep_wait();   // the logits' kernel has completed (no-op without a programmatic launch)
+  griddep_launch_dependents();
   const RouterRef rr{p.x + (size_t)t * p.H, p.router_w, p.router_bias, p.H};
   block_topk(p.logits + (size_t)t * (p.E + 1), p.bound ? p.bound + (size_t)t * (p.E + 1) : nullptr, p.E, p.k,
              p.has_shared, rr, ts);
@@ -507,12 +509,12 @@ cudaError_t launch_route(const RouteParams& p, cudaStream_t s, bool pdl) {
   return launch_ex((const void*)route_logits_kernel, grid, dim3(kRouteThreads), sm, s, pdl, args);
 }
 
-cudaError_t launch_topk(const TopkParams& p, cudaStream_t s) {
+cudaError_t launch_topk(const TopkParams& p, cudaStream_t s, bool pdl) {
   cudaError_t e = set_smem((const void*)topk_kernel, 0);
   if (e != cudaSuccess) return e;
   TopkParams q = p;
   void* args[] = {&q};
-  return launch_ex((const void*)topk_kernel, dim3(p.T), dim3(kThreads), 0, s, false, args);
+  return launch_ex((const void*)topk_kernel, dim3(p.T), dim3(kThreads), 0, s, pdl, args);
 }
 
 static int smem_optin() {

@@ -246,7 +246,7 @@ cudaError_t launch_route_gemm(const RouteParams& p, cudaStream_t s);   // many t
 // router rows and tokens, padded to the tcgen05 router's 128 x 128 tiles
 __host__ __device__ inline size_t route_tc_rows_w(int E) { return (size_t)((E + 127) / 128) * 128; }
 __host__ __device__ inline size_t route_tc_rows_x(int T) { return (size_t)((T + 127) / 128) * 128; }
-cudaError_t launch_topk(const TopkParams& p, cudaStream_t s);
+cudaError_t launch_topk(const TopkParams& p, cudaStream_t s, bool pdl = false);
 // MXFP4 experts (mx.cu): mat-vec, and the many-token product on tcgen05 (kind::mxf4)
 cudaError_t launch_mx_gemv(const uint32_t* q, const uint8_t* e, int R, int K, const float* x, float* y, cudaStream_t s);
 cudaError_t launch_mx_gemm(const uint32_t* q, const uint8_t* e, int R, int K, const uint16_t* x, int T, float* y,
@@ -262,7 +262,7 @@ struct MxLayerParams {
   float* a;                    // [T][S][I]
   float* h;                    // [T][H], in place: h + the weighted expert outputs
 };
-cudaError_t launch_mx_layer(const MxLayerParams& p, cudaStream_t s);
+cudaError_t launch_mx_layer(const MxLayerParams& p, cudaStream_t s, bool pdl = false);
 cudaError_t launch_gateup(const GateUpParams& p, int bits, int T, bool pdl, cudaStream_t s);
 cudaError_t launch_down(const DownParams& p, int bits, int T, bool pdl, cudaStream_t s);
 cudaError_t launch_norm(const NormParams& p, bool pdl, cudaStream_t s);

@@ -556,9 +556,9 @@ __device__ __forceinline__ void mx_stage(float* dst, const float* src, int n) { 
 }
 
 // grid (ceil(S I / kMxLWarps), T), block 32 kMxLWarps: a[t][s][i] = silu(G x_t)_i (U x_t)_i for the
-// expert of slot s (slot k = the shared expert), one (slot, row) per warp. Each warp resolves its
-// expert and requests its rows' first blocks before the CTA stages x_t, so the dependent loads
-// (selection, descriptor, codes) overlap the staging.
+// expert of slot s (slot k = the shared expert), one (slot, row) per warp. Under a programmatic
+// launch the CTA stages x_t (the layer input, complete since the router passed its own wait)
+// before waiting for the top-k; then each warp resolves its expert and requests its rows.
 __global__ void __launch_bounds__(kMxLWarps * 32) mx_gateup_kernel(MxLayerParams p) {
   extern __shared__ __align__(16) float xs[];   // x_t, [H/32][kMvXStride]
   const int t = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -569,6 +569,10 @@ __global__ void __launch_bounds__(kMxLWarps * 32) mx_gateup_kernel(MxLayerParams
   const uint32_t *gq = nullptr, *uq = nullptr;
   const uint8_t *ge = nullptr, *ue = nullptr;
   MxChunk2 c;
+  const uint16_t* xt = p.x + (size_t)t * p.H;
+  for (int b = threadIdx.x; b < nb; b += blockDim.x) mx_stage_bf16(xt + 32 * b, xs + b * kMvXStride);
+  griddep_wait();   // the top-k has completed
+  griddep_launch_dependents();
   if (has) {
     const moe_expert* ex = sl < p.k ? p.experts + p.idx[t * p.k + sl] : &p.shared;
     gq = ex->gate.q + (size_t)i * (p.H / 8);
@@ -577,8 +581,6 @@ __global__ void __launch_bounds__(kMxLWarps * 32) mx_gateup_kernel(MxLayerParams
     ue = (const uint8_t*)ex->up.scales + (size_t)i * nb;
     mx_load2(c, gq, ge, uq, ue, 0, nb, lane);
   }
-  const uint16_t* xt = p.x + (size_t)t * p.H;
-  for (int b = threadIdx.x; b < nb; b += blockDim.x) mx_stage_bf16(xt + 32 * b, xs + b * kMvXStride);
   __syncthreads();
   if (!has) return;
   float2 acc = make_float2(0.f, 0.f);
@@ -594,7 +596,8 @@ __global__ void __launch_bounds__(kMxLWarps * 32) mx_gateup_kernel(MxLayerParams
 
 // grid (ceil(H / kMxLWarps), T), block 32 kMxLWarps, a hidden row per warp:
 // h[t][j] += sum_{s<k} w[t][s] (D_s a[t][s])_j + sg[t] (D_shared a[t][k])_j, in that order.
-// Each warp requests every slot's first blocks of its row before the CTA stages a[t].
+// Each warp resolves every slot's expert (the selection is complete: the top-k ran before the
+// gate/up kernel passed its wait) and requests its row's first blocks, then waits for a[t].
 __global__ void __launch_bounds__(kMxLWarps * 32, 2) mx_down_kernel(MxLayerParams p) {
   extern __shared__ __align__(16) float as[];   // a[t][s], s < S: [S][I/32][kMvXStride]
   const int t = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -618,6 +621,8 @@ __global__ void __launch_bounds__(kMxLWarps * 32, 2) mx_down_kernel(MxLayerParam
     c[sl] = in ? __ldg(q[sl] + lane) : make_uint4(0u, 0u, 0u, 0u);
     sc[sl] = in ? __ldg(e[sl] + lane) : 0u;
   }
+  griddep_wait();   // the gate/up kernel has completed: a is final
+  griddep_launch_dependents();
   for (int sl = 0; sl < p.S; ++sl) mx_stage(as + sl * sstride, p.a + ((size_t)t * p.S + sl) * p.I, p.I);
   __syncthreads();
   if (!has) return;
@@ -646,17 +651,37 @@ __global__ void __launch_bounds__(kMxLWarps * 32, 2) mx_down_kernel(MxLayerParam
   if (lane == 0) p.h[(size_t)t * p.H + row] = acc;
 }
 
-cudaError_t launch_mx_layer(const MxLayerParams& p, cudaStream_t s) {
+static cudaError_t mx_launch(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
+                             void** args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  if (pdl) {
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+  }
+  return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
+cudaError_t launch_mx_layer(const MxLayerParams& p, cudaStream_t s, bool pdl) {
   const size_t sg = sizeof(float) * (size_t)(p.H / 32) * kMvXStride;
   const size_t sd = sizeof(float) * (size_t)p.S * (p.I / 32) * kMvXStride;
   cudaError_t e = cudaFuncSetAttribute((const void*)mx_gateup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sg);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute((const void*)mx_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sd);
   if (e != cudaSuccess) return e;
-  mx_gateup_kernel<<<dim3((p.S * p.I + kMxLWarps - 1) / kMxLWarps, p.T), kMxLWarps * 32, sg, s>>>(p);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  mx_down_kernel<<<dim3((p.H + kMxLWarps - 1) / kMxLWarps, p.T), kMxLWarps * 32, sd, s>>>(p);
-  return cudaGetLastError();
+  MxLayerParams q = p;
+  void* args[] = {&q};
+  e = mx_launch((const void*)mx_gateup_kernel, dim3((p.S * p.I + kMxLWarps - 1) / kMxLWarps, p.T), dim3(kMxLWarps * 32),
+                sg, s, pdl, args);
+  if (e != cudaSuccess) return e;
+  return mx_launch((const void*)mx_down_kernel, dim3((p.H + kMxLWarps - 1) / kMxLWarps, p.T), dim3(kMxLWarps * 32), sd,
+                   s, pdl, args);
 }
 
 }  // namespace qmoe
