@@ -40,7 +40,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=480)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="layer_q4",
-                    choices=["layer_q4", "layer_q2", "prefill_q4", "stack_q4", "cached_q4", "mxfp4_q4"],
+                    choices=["layer_q4", "layer_q2", "prefill_q4", "stack_q4", "cached_q4", "mxfp4_q4", "mxfp4_gemm"],
                     help="prefill_q4: one step = one 512-token forward of the layer (the prefill path); "
                          "cached_q4: decode of layer_q4 with its routed experts in host memory and an HBM cache")
     ap.add_argument("--cache-slots", type=int, default=64, help="cached_q4: experts the HBM cache holds")
@@ -1006,9 +1006,140 @@ def ours_mx(args, cfg):
         print(json.dumps(line), flush=True)
 
 
+def ours_mxgemm(args):
+    """The many-token MXFP4 product on tcgen05 (kind::mxf4 with block scaling): Y = X W^T for the
+    512 tokens of the prefill workload and a 2048 x 4096 MXFP4 matrix (the shared expert's gate and
+    up rows); one step = one moe_expert_gemm_mxfp4 call (prep of the activation terms, the
+    block-scaled product, the sum of the column splits). 48 rotating weight copies (214 MB, larger
+    than L2)."""
+    import numpy as np
+    import torch
+
+    import oracle
+    import quantized_expert_decode_moe_b200 as qm
+    from fixtures import gen
+
+    world, rank, local = dist_info()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    qm.lib()
+    R, K, T, C = 2048, 4096, 512, 48
+    q, e = gen.mx_matrix(5, R, K)
+    qd = torch.from_numpy(q.view(np.int32)).to(dev)
+    ed = torch.from_numpy(e).to(dev)
+    mats = [qm.MxMat(qd.clone(), ed.clone()) for _ in range(C)]
+    x_host = gen.mx_tokens(6, T, K)
+    xd = torch.from_numpy(x_host.view(np.int16)).to(dev)
+    y = torch.empty((T, R), device=dev)
+    ws = qm.new_mx_workspace(R, K, T)
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        for c in range(C):
+            qm.moe_expert_gemm_mxfp4(mats[c], xd, y, ws=ws, stream=stream)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for c in range(C):
+                qm.moe_expert_gemm_mxfp4(mats[c], xd, y, ws=ws, stream=stream)
+        for _ in range(max(1, max(args.warmup, 3) // C + 1)):
+            g.replay()
+    stream.synchronize()
+    assert qm.moe_poll_status(ws, stream) == 0
+    reps = max(1, args.steps // C)
+    steps = reps * C
+    gpu_uuid = str(getattr(torch.cuda.get_device_properties(dev), "uuid", "") or "")
+    clocks = Clocks(("GPU-" + gpu_uuid) if gpu_uuid and not gpu_uuid.startswith("GPU-") else (gpu_uuid or str(local)))
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        busy(g.replay, stream)
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+        busy(g.replay, stream)
+    e1.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    assert qm.moe_poll_status(ws, stream) == 0
+    # end to end: x in from page-locked host memory, Y back, every step
+    xh = torch.from_numpy(x_host.view(np.int16)).pin_memory()
+    yh = torch.empty((T, R), dtype=torch.float32).pin_memory()
+    e2e_n = min(args.e2e_steps, steps, 96)
+    with torch.cuda.stream(stream):
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for i in range(e2e_n):
+            xd.copy_(xh, non_blocking=True)
+            qm.moe_expert_gemm_mxfp4(mats[i % C], xd, y, ws=ws, stream=stream)
+            yh.copy_(y, non_blocking=True)
+        f1.record(stream)
+    f1.synchronize()
+    e2e_ms = f0.elapsed_time(f1)
+    peaks, peak_kind = measured_peaks()
+    fp4_peak = 4.0 * peaks["bf16_tflops"]   # dense fp4 = 4 x dense bf16 (nominal 9 / 2.25 PFLOP/s)
+    flops = 2.0 * R * K * T
+    per_step_ms = ms / steps
+    achieved = flops / (per_step_ms * 1e-3) / 1e12
+    line = {
+        "metric": "MXFP4 expert product, tokens/s (512-token batch, 2048 x 4096 MXFP4 matrix), tcgen05 kind::mxf4, 1 B200",
+        "value": T * steps / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world, "steps": steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": per_step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "E2M1 weights x five E2M1 terms of the bf16 activations (E8M0 block scales), fp32 in tensor memory",
+        "data": "synthetic (seeded; no model weights)",
+        "config": {"workload": "512 tokens x one 2048 x 4096 MXFP4 matrix (the shared expert's gate and up rows)",
+                   "R": R, "K": K, "T": T, "copies": C, "l2": "48 rotating weight copies (214 MB), larger than L2"},
+        "tflops": achieved,
+        "roofline": {"bound": "tensor", "kernel": "moe_expert_gemm_mxfp4 (prep + mx_gemm_kernel + split sum)",
+                     "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s", "frac": achieved / fp4_peak,
+                     "traffic": None, "algorithmic_flops": flops,
+                     "peak_kind": f"{peak_kind} bf16 x 4 (fp4 / bf16 nominal ratio); achieved counts the product once, "
+                                  f"the five activation terms issue 5x these fp4 MMA flops"},
+        "e2e": {"value": T * e2e_n / (e2e_ms * 1e-3), "unit": "tokens/s", "steps": e2e_n,
+                "h2d_bytes_per_step": T * K * 2, "d2h_bytes_per_step": T * R * 4},
+        "gpu_launches": 3 * steps, "clocks": clk,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        n = 16
+        t0 = time.perf_counter()
+        oracle.mx_gemm(q, e, x_host[:n], K)
+        el = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": n / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                "sample": f"{n} tokens of this workload ({el:.1f} s: dequantisation and one numpy "
+                                          f"matrix product in double)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     import fixtures
+    if args.config == "mxfp4_gemm":
+        if args.impl == "reference":
+            if dist_info()[1] == 0:
+                import oracle
+                from fixtures import gen
+                R, K, n = 2048, 4096, max(1, min(args.steps, 64))
+                q, e = gen.mx_matrix(5, R, K)
+                x = gen.mx_tokens(6, n, K)
+                t0 = time.perf_counter()
+                oracle.mx_gemm(q, e, x, K)
+                el = time.perf_counter() - t0
+                rate = n / el
+                print(json.dumps({
+                    "impl": "reference", "metric": "MXFP4 expert product, tokens/s (512-token batch, 2048 x 4096 MXFP4 "
+                    "matrix), tcgen05 kind::mxf4, 1 B200", "value": rate, "unit": "tokens/s", "n_gpus": args.gpus,
+                    "steps": n, "warmup": 0, "ms_per_step": 1e3 * el / n, "higher_is_better": True, "scaling": "weak",
+                    "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded; no model weights)",
+                    "config": {"workload": "512 tokens x one 2048 x 4096 MXFP4 matrix", "tokens_timed": n},
+                    "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                     "sample": f"{n} tokens"},
+                    "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+                    flush=True)
+        else:
+            ours_mxgemm(args)
+        return
     if args.config == "mxfp4_q4":
         cfg = fixtures.CONFIGS["layer_q4"]
         if args.impl == "reference":

@@ -205,12 +205,15 @@ static_assert(kMxN + kMxStages * kMxSfCols <= 256, "accumulator and scales fit 2
 // MMA reads (scale j of the word selected by the descriptor's scale id).
 __host__ __device__ __forceinline__ int mx_sf_off(int m, int j) { return (m & 31) * 16 + (m >> 5) * 4 + j; }
 
-// grid T_pad + ceil(R nstg / kMxPrepThreads), block kMxPrepThreads.
-//  CTA t < T_pad: token row t (zeros beyond T); thread i takes the 32-element
-//   blocks b = i + kMxPrepThreads n and writes, per term, the 16 code bytes at
-//   bq[(((t/128) nstg + b/4) kMxTerms + term) kMxChunk 4 + (b%4) kMxChunk + (t%128) 16]
-//   and the scale byte at bsf[(((t/128) nstg + b/4) kMxTerms + term) 512 + mx_sf_off(t%128, b%4)].
-//  CTA T_pad + s: scale words i = s kMxPrepThreads + thread (row i / nstg, stage
+// grid T_pad q + ceil(R nstg / kMxPrepThreads) with q = ceil(4 (K/32) / kMxPrepThreads),
+// block kMxPrepThreads.
+//  CTA t q + j (t < T_pad): token row t (zeros beyond T). Four adjacent threads take one
+//   32-element block b (thread i of the CTA: task j kMxPrepThreads + i, block task / 4, quarter
+//   task % 4 = elements 8 quarter .. +7, one code word); the block's maximum per term is reduced
+//   over the four with shuffles. Per term the code word goes to
+//   bq[(((t/128) nstg + b/4) kMxTerms + term) kMxTileA + (b%4) kMxChunk + (t%128) 16 + 4 quarter]
+//   and (quarter 0) the scale byte to bsf[(((t/128) nstg + b/4) kMxTerms + term) 512 + mx_sf_off(t%128, b%4)].
+//  CTA T_pad q + s: scale words i = s kMxPrepThreads + thread (row i / nstg, stage
 //   i % nstg: the row's four scales of that stage), rearranged into the same
 //   512-byte blocks, asf[((row/128) nstg + stage) 512 + mx_sf_off(row%128, 0)].
 __global__ void __launch_bounds__(kMxPrepThreads) mx_prep_kernel(const uint16_t* __restrict__ x, int T, int Tpad,
@@ -218,63 +221,65 @@ __global__ void __launch_bounds__(kMxPrepThreads) mx_prep_kernel(const uint16_t*
                                                                  uint8_t* __restrict__ bq, uint8_t* __restrict__ bsf,
                                                                  uint8_t* __restrict__ asf) {
   const int nb = K / 32, nstg = K / kMxKS;
-  if ((int)blockIdx.x >= Tpad) {   // weight scales: one 4-byte word (4 blocks, K % 128 == 0) per thread
-    const size_t i = (size_t)(blockIdx.x - Tpad) * kMxPrepThreads + threadIdx.x;
+  const int q = (4 * nb + kMxPrepThreads - 1) / kMxPrepThreads;
+  if ((int)blockIdx.x >= Tpad * q) {   // weight scales: one 4-byte word (4 blocks, K % 128 == 0) per thread
+    const size_t i = (size_t)(blockIdx.x - Tpad * q) * kMxPrepThreads + threadIdx.x;
     if (i >= (size_t)R * nstg) return;
     const int r = (int)(i / nstg), g = (int)(i % nstg);
     const uint32_t w = __ldg((const uint32_t*)e + i);
     *(uint32_t*)(asf + ((size_t)(r / kMxM) * nstg + g) * kMxSf + mx_sf_off(r % kMxM, 0)) = w;
     return;
   }
-  const int t = blockIdx.x, tt = t / kMxN, rr = t % kMxN;
-  for (int b = threadIdx.x; b < nb; b += kMxPrepThreads) {
-    float v[32];
-    if (t < T) {
-      const uint4* src = (const uint4*)(x + (size_t)t * K + 32 * b);
+  const int t = blockIdx.x / q, task = (blockIdx.x % q) * kMxPrepThreads + threadIdx.x;
+  const int b = task >> 2, qt = task & 3, tt = t / kMxN, rr = t % kMxN;
+  // every thread of a group of four takes part in the shuffles; a group past the row's last block
+  // has no block (b >= nb) and stores nothing
+  const bool in = b < nb;
+  float v[8];
+  if (in && t < T) {
+    const uint4 u = __ldg((const uint4*)(x + (size_t)t * K + 32 * b + 8 * qt));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint4 u = __ldg(src + i);
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          v[8 * i + 2 * h] = bf16lo(w[h]);
-          v[8 * i + 2 * h + 1] = bf16hi(w[h]);
-        }
-      }
-    } else {
-#pragma unroll
-      for (int k = 0; k < 32; ++k) v[k] = 0.f;
+    for (int h = 0; h < 4; ++h) {
+      v[2 * h] = bf16lo(w[h]);
+      v[2 * h + 1] = bf16hi(w[h]);
     }
-    const int g = b / 4, c = b % 4;
+  } else {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = 0.f;
+  }
+  const int g = b / 4, c = b % 4;
 #pragma unroll 1
-    for (int term = 0; term < kMxTerms; ++term) {
-      float m = 0.f;
+  for (int term = 0; term < kMxTerms; ++term) {
+    float m = 0.f;
 #pragma unroll
-      for (int k = 0; k < 32; ++k) m = fmaxf(m, fabsf(v[k]));
-      // the smallest power 2^u with m <= 6 2^u, no smaller than 2^-127 (every m below 2^-126 takes
-      // u = -127): with m = f 2^E, f in [0.5, 1), u = E - 3 if f <= 0.75, else E - 2
-      int u = -127;
-      if (m >= 0x1p-126f) {
-        const uint32_t bits = __float_as_uint(m);
-        const int E = (int)((bits >> 23) & 0xFFu) - 126;
-        u = max(-127, (bits & 0x7FFFFFu) <= 0x400000u ? E - 3 : E - 2);
-      }
-      const float down = mx_pow2(-u), up = mx_pow2(u - 1);   // 2^-u; 2^(u-1), the unit of 2|E2M1 value|
-      uint32_t code[4] = {0u, 0u, 0u, 0u};
+    for (int k = 0; k < 8; ++k) m = fmaxf(m, fabsf(v[k]));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    // the smallest power 2^u with m <= 6 2^u, no smaller than 2^-127 (every m below 2^-126 takes
+    // u = -127): with m = f 2^E, f in [0.5, 1), u = E - 3 if f <= 0.75, else E - 2
+    int u = -127;
+    if (m >= 0x1p-126f) {
+      const uint32_t bits = __float_as_uint(m);
+      const int E = (int)((bits >> 23) & 0xFFu) - 126;
+      u = max(-127, (bits & 0x7FFFFFu) <= 0x400000u ? E - 3 : E - 2);
+    }
+    const float down = mx_pow2(-u), up = mx_pow2(u - 1);   // 2^-u; 2^(u-1), the unit of 2|E2M1 value|
+    uint32_t code = 0u;
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        const float a = fabsf(v[k] * down);   // exact unless it underflows, far below 0.25
-        const int idx = (a > 0.25f) + (a > 0.75f) + (a > 1.25f) + (a > 1.75f) + (a > 2.5f) + (a > 3.5f) + (a > 5.f);
-        const int twice = idx <= 4 ? idx : (idx == 5 ? 6 : (idx == 6 ? 8 : 12));   // 2 |E2M1 value|
-        const bool neg = v[k] < 0.f;
-        const float val = (float)(neg ? -twice : twice) * up;   // exact: a small integer times 2^(u-1)
-        v[k] -= val;   // exact: 0, or within a factor of two of v[k]
-        code[k >> 3] |= (uint32_t)(idx | (neg ? 8 : 0)) << (4 * (k & 7));
-      }
+    for (int k = 0; k < 8; ++k) {
+      const float a = fabsf(v[k] * down);   // exact unless it underflows, far below 0.25
+      const int idx = (a > 0.25f) + (a > 0.75f) + (a > 1.25f) + (a > 1.75f) + (a > 2.5f) + (a > 3.5f) + (a > 5.f);
+      const int twice = idx <= 4 ? idx : (idx == 5 ? 6 : (idx == 6 ? 8 : 12));   // 2 |E2M1 value|
+      const bool neg = v[k] < 0.f;
+      const float val = (float)(neg ? -twice : twice) * up;   // exact: a small integer times 2^(u-1)
+      v[k] -= val;   // exact: 0, or within a factor of two of v[k]
+      code |= (uint32_t)(idx | (neg ? 8 : 0)) << (4 * k);
+    }
+    if (in) {
       const size_t blk = ((size_t)tt * nstg + g) * kMxTerms + term;
-      *(uint4*)(bq + blk * kMxTileA + (size_t)c * kMxChunk + (size_t)rr * 16) =
-          make_uint4(code[0], code[1], code[2], code[3]);
-      bsf[blk * kMxSf + mx_sf_off(rr, c)] = (uint8_t)(u + 127);
+      *(uint32_t*)(bq + blk * kMxTileA + (size_t)c * kMxChunk + (size_t)rr * 16 + 4 * qt) = code;
+      if (qt == 0) bsf[blk * kMxSf + mx_sf_off(rr, c)] = (uint8_t)(u + 127);
     }
   }
 }
@@ -482,7 +487,8 @@ cudaError_t launch_mx_gemm(const uint32_t* q, const uint8_t* e, int R, int K, co
   const int tpad = (T + kMxN - 1) / kMxN * kMxN;
   uint8_t* base = (uint8_t*)ws;
   const int nscale = (int)(((size_t)R * (K / kMxKS) + kMxPrepThreads - 1) / kMxPrepThreads);
-  mx_prep_kernel<<<tpad + nscale, kMxPrepThreads, 0, s>>>(x, T, tpad, e, R, K, base + W.bq, base + W.bsf,
+  const int qrow = (4 * (K / 32) + kMxPrepThreads - 1) / kMxPrepThreads;
+  mx_prep_kernel<<<tpad * qrow + nscale, kMxPrepThreads, 0, s>>>(x, T, tpad, e, R, K, base + W.bq, base + W.bsf,
                                                              base + W.asf);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
