@@ -264,16 +264,23 @@ __global__ void __launch_bounds__(kMxPrepThreads) mx_prep_kernel(const uint16_t*
       const int E = (int)((bits >> 23) & 0xFFu) - 126;
       u = max(-127, (bits & 0x7FFFFFu) <= 0x400000u ? E - 3 : E - 2);
     }
-    const float down = mx_pow2(-u), up = mx_pow2(u - 1);   // 2^-u; 2^(u-1), the unit of 2|E2M1 value|
+    const float down = mx_pow2(-u), up = mx_pow2(u);   // 2^-u, 2^u
     uint32_t code = 0u;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const float a = fabsf(v[k] * down);   // exact unless it underflows, far below 0.25
-      const int idx = (a > 0.25f) + (a > 0.75f) + (a > 1.25f) + (a > 1.75f) + (a > 2.5f) + (a > 3.5f) + (a > 5.f);
-      const int twice = idx <= 4 ? idx : (idx == 5 ? 6 : (idx == 6 ? 8 : 12));   // 2 |E2M1 value|
+      // a = |v| 2^-u in [0, 6] (exact unless it underflows, far below 0.25), rounded to the nearest
+      // E2M1 value: from 1 up, one mantissa bit (add half of it to the float's bits, then drop the
+      // rest: 1, 1.5, 2, 3, 4, 6; code 2 (exponent + 1) + mantissa bit); below 1, rint(2a) halves
+      // (0, 0.5, 1; code = rint(2a))
+      const float a = fabsf(v[k] * down);
+      const uint32_t rb = (__float_as_uint(a) + 0x200000u) & 0xFFC00000u;
+      const int hi_code = (int)(((rb >> 23) - 126u) << 1 | ((rb >> 22) & 1u));
+      const int lo_code = __float2int_rn(2.f * a);
+      const bool big = a >= 1.f;
+      const int idx = big ? hi_code : lo_code;
+      const float r = big ? __uint_as_float(rb) : 0.5f * (float)lo_code;
       const bool neg = v[k] < 0.f;
-      const float val = (float)(neg ? -twice : twice) * up;   // exact: a small integer times 2^(u-1)
-      v[k] -= val;   // exact: 0, or within a factor of two of v[k]
+      v[k] -= (neg ? -r : r) * up;   // exact: r has two significant bits and is 0 or within a factor of two of a
       code |= (uint32_t)(idx | (neg ? 8 : 0)) << (4 * k);
     }
     if (in) {
