@@ -40,7 +40,7 @@
  *      T > 8     the grouped prefill kernels (two stages of their ring of
  *                weight tiles must fit and their row tiles must divide the
  *                matrices);
- *      MXFP4    (group 32) T <= 8: the down kernel stages every slot's SwiGLU
+ *      MXFP4    (group 32), any T: the down kernel stages every slot's SwiGLU
  *                output in shared memory: (top_k + shared) * I <= 51,200;
  *    and H, I <= 8192 throughout. With MOE_DECODE_KERNEL=fused in the
  *    environment (read once), single-token calls and stacks take the fused
@@ -101,9 +101,11 @@ typedef struct {
  *   bits in {2,4}, group = 64, has_shared in {0,1}, rms_eps > 0.
  *   bits = 4 with group = 32 selects MXFP4 experts (see moe_mxmat): each
  *   moe_qmat's q holds the E2M1 codes, its scales pointer the E8M0 bytes
- *   uint8 [R][K/32], its biases are not read (may be NULL); decode only
- *   (T <= 8; MOE_ERR_UNSUPPORTED above), through moe_layer_forward,
- *   moe_layer_forward_timed, moe_layer_forward_noalloc and moe_stack_forward.
+ *   uint8 [R][K/32], its biases are not read (may be NULL); through
+ *   moe_layer_forward and moe_layer_forward_timed (any T: above 8 tokens the
+ *   router is the many-token one and the expert kernels run per token, each
+ *   expert's rows read once per token that chooses it), and
+ *   moe_layer_forward_noalloc and moe_stack_forward (T <= 8 / T = 1).
  *   router_w    bf16 [E][H]
  *   router_bias fp32 [E] or NULL: added to the logits before softmax/top-k
  *   experts     device array [E] of moe_expert

@@ -94,10 +94,11 @@ bool fused_requested() {
   }
   return v == 1;
 }
-// MXFP4 layers: decode (up to 8 tokens); the down kernel stages every slot's
+// MXFP4 layers, any number of tokens; the down kernel stages every slot's
 // SwiGLU output (S I floats, padded by 9/8) in shared memory.
 bool mx_supported(const moe_layer* L, int T) {
-  return T <= kDecodeMaxT && (size_t)slots_of(L) * (L->inter / 32) * 36 * sizeof(float) <= 227 * 1024;
+  (void)T;
+  return (size_t)slots_of(L) * (L->inter / 32) * 36 * sizeof(float) <= 227 * 1024;
 }
 
 Path path_of(const moe_layer* L, int T) {
@@ -207,7 +208,8 @@ moe_status decode_chain(const moe_layer* L, const uint16_t* x_in, float* h, int 
 moe_status mx_chain(const moe_layer* L, const uint16_t* x_in, float* h, int T, uint16_t* x_out, float* x_out_f32,
                     int32_t* topk_idx, float* topk_w, void* ws, cudaStream_t s, void* const* events = nullptr,
                     uint16_t* x_rec = nullptr, float* h_rec = nullptr) {
-  const bool pdl = events == nullptr && !topk_idx && !topk_w;   // programmatic launches between the kernels
+  // programmatic launches between the kernels (decode: the router of up to 8 tokens supports them)
+  const bool pdl = events == nullptr && !topk_idx && !topk_w && T <= kDecodeMaxT;
   auto mark = [&](int i) { if (events) cudaEventRecord((cudaEvent_t)events[i], s); };
   mark(0);
   const int H = L->hidden, I = L->inter, E = L->n_experts, k = L->top_k, S = slots_of(L);
@@ -218,7 +220,15 @@ moe_status mx_chain(const moe_layer* L, const uint16_t* x_in, float* h, int T, u
   rp.logits = at<double>(ws, W.logits);
   rp.bound = at<float>(ws, W.bound);
   rp.h = h; rp.x_rec = x_rec; rp.h_rec = h_rec;
-  if (launch_route(rp, s, pdl) != cudaSuccess) return MOE_ERR_CUDA;
+  if (T > kDecodeMaxT) {   // many tokens: the exact integer router on tcgen05
+    rp.lpart = at<long long>(ws, W.lpart);
+    rp.wdig = at<int8_t>(ws, W.wdig); rp.xdig = at<int8_t>(ws, W.xdig);
+    rp.wst = at<double>(ws, W.wst); rp.xst = at<double>(ws, W.xst);
+    rp.status = at<uint32_t>(ws, W.status); rp.wait_ns = wait_bound_ns();
+    if (launch_route_gemm(rp, s) != cudaSuccess) return MOE_ERR_CUDA;
+  } else if (launch_route(rp, s, pdl) != cudaSuccess) {
+    return MOE_ERR_CUDA;
+  }
   mark(1);
   TopkParams tp{};
   tp.E = E; tp.k = k; tp.T = T; tp.has_shared = L->has_shared; tp.H = H;
