@@ -94,11 +94,11 @@ bool fused_requested() {
   }
   return v == 1;
 }
-// MXFP4 layers, any number of tokens; the down kernel stages every slot's
-// SwiGLU output (S I floats, padded by 9/8) in shared memory.
+// MXFP4 layers, any number of tokens; the down kernel holds the digit blocks of
+// every slot's SwiGLU output in shared memory (112 bytes per 32 values).
 bool mx_supported(const moe_layer* L, int T) {
   (void)T;
-  return (size_t)slots_of(L) * (L->inter / 32) * 36 * sizeof(float) <= 227 * 1024;
+  return (size_t)slots_of(L) * (L->inter / 32) * 112 <= 227 * 1024;
 }
 
 Path path_of(const moe_layer* L, int T) {
@@ -214,6 +214,8 @@ moe_status mx_chain(const moe_layer* L, const uint16_t* x_in, float* h, int T, u
   mark(0);
   const int H = L->hidden, I = L->inter, E = L->n_experts, k = L->top_k, S = slots_of(L);
   const WsLayout W = layout_of(L, T);
+  // the digit blocks of x first (the gate/up kernel reads them before its own wait)
+  if (launch_mx_digits(x_in, true, T, H, at<uint8_t>(ws, W.mxx), s, pdl) != cudaSuccess) return MOE_ERR_CUDA;
   RouteParams rp{};
   rp.H = H; rp.E = E; rp.T = T; rp.has_shared = L->has_shared;
   rp.x = x_in; rp.router_w = L->router_w; rp.router_bias = L->router_bias; rp.gate_w = L->shared_gate_w;
@@ -246,6 +248,7 @@ moe_status mx_chain(const moe_layer* L, const uint16_t* x_in, float* h, int T, u
   mp.x = x_in; mp.experts = L->experts; mp.shared = L->shared;
   mp.idx = tp.idx; mp.w = tp.w; mp.sg = tp.sg;
   mp.a = at<float>(ws, W.a); mp.h = h;
+  mp.xdig = at<uint8_t>(ws, W.mxx); mp.adig = at<uint8_t>(ws, W.mxa);
   if (launch_mx_layer(mp, s, pdl) != cudaSuccess) return MOE_ERR_CUDA;
   mark(3);
   NormParams np{};

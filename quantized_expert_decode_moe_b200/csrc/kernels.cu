@@ -25,6 +25,8 @@ WsLayout ws_layout(int H, int I, int E, int k, int S, int T) {
   L.gpart = o; o = align256(o + sizeof(float) * (size_t)kMaxCtas);
   L.a = o; o = align256(o + sizeof(float) * (size_t)T * S * I);
   L.hacc = o; o = align256(o + sizeof(float) * (size_t)T * H);
+  L.mxx = o; o = align256(o + (size_t)T * (H / 32) * 112);
+  L.mxa = o; o = align256(o + (size_t)T * S * (I / 32) * 112);
   L.counts = o; o = align256(o + sizeof(int32_t) * (size_t)E);
   L.offsets = o; o = align256(o + sizeof(int32_t) * (size_t)(E + 1));
   L.perm = o; o = align256(o + sizeof(int32_t) * (size_t)T * k);

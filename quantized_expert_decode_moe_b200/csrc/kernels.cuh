@@ -25,6 +25,7 @@ struct WsLayout {
   size_t gpart;       // float [kMaxCtas] per-CTA partial sums (fused decode)
   size_t a;           // float [T][S][I]  silu(gate) * up of each slot (slot S-1 = shared expert)
   size_t hacc;        // float [T][H]     h + weighted expert outputs
+  size_t mxx, mxa;    // MXFP4 layers: digit blocks of x [T][H/32][112 B] and of a [T][S][I/32][112 B]
   // prefill
   size_t counts;      // int32 [E]
   size_t offsets;     // int32 [E+1]
@@ -261,7 +262,11 @@ struct MxLayerParams {
   const int32_t* idx; const float* w; const float* sg;   // [T][k], [T][k], [T]
   float* a;                    // [T][S][I]
   float* h;                    // [T][H], in place: h + the weighted expert outputs
+  const uint8_t* xdig;         // [T][H/32] digit blocks of x (launch_mx_digits, before the router)
+  uint8_t* adig;               // [T][S][I/32] digit blocks of a (written between gate/up and down)
 };
+// digit blocks of rows of K values (bf16 or fp32) for the MXFP4 layer kernels: 112 bytes per 32
+cudaError_t launch_mx_digits(const void* src, bool bf16, int rows, int K, uint8_t* dst, cudaStream_t s, bool pdl);
 cudaError_t launch_mx_layer(const MxLayerParams& p, cudaStream_t s, bool pdl = false);
 cudaError_t launch_gateup(const GateUpParams& p, int bits, int T, bool pdl, cudaStream_t s);
 cudaError_t launch_down(const DownParams& p, int bits, int T, bool pdl, cudaStream_t s);

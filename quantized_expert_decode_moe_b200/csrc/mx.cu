@@ -138,6 +138,111 @@ __device__ __forceinline__ void mx_stage_bf16(const uint16_t* src, float* dst) {
   mx_stage_block(v, dst);
 }
 
+// ---- digit blocks (the layer kernels): a 32-value block of x or a as 22-bit fixed point with
+// its own power of two, X = rint(v 2^p), max |v| 2^p < 2^22, split exactly into three balanced
+// signed 8-bit digits (three 32-byte planes), then the factor 2^-(p+1) as a float at byte 96
+// (the 1/2 undoes the codes' 2 e2m1); bf16 values within 2^-14 of the block's largest are
+// exact, others round within 2^-23 of it. Written once per call by mx_digits_kernel.
+constexpr int kMxDig = 112;   // bytes per digit block (96 digits, the factor, padding to 16)
+
+__device__ __forceinline__ void mx_digit_block(const float (&v)[32], uint8_t* dst) {
+  float m = 0.f;
+#pragma unroll
+  for (int k = 0; k < 32; ++k) m = fmaxf(m, fabsf(v[k]));
+  int p = 0;
+  if (m > 0.f) {   // m = f 2^E, f in [0.5, 1); below 2^-126 treated as 2^-126
+    const int E = m >= 0x1p-126f ? (int)((__float_as_uint(m) >> 23) & 0xFFu) - 126 : -125;
+    p = 22 - E;
+  }
+  const float u1 = mx_pow2(p / 2), u2 = mx_pow2(p - p / 2);   // 2^p as two normal factors
+  uint32_t pl[3][8] = {};
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    const int X = __float2int_rn(v[k] * u1 * u2);   // |X| <= 2^22
+    const int d0 = ((X + 128) & 255) - 128;
+    const int X1 = (X - d0) / 256;
+    const int d1 = ((X1 + 128) & 255) - 128;
+    const int d2 = (X1 - d1) / 256;
+    pl[0][k >> 2] |= (uint32_t)(d0 & 255) << (8 * (k & 3));
+    pl[1][k >> 2] |= (uint32_t)(d1 & 255) << (8 * (k & 3));
+    pl[2][k >> 2] |= (uint32_t)(d2 & 255) << (8 * (k & 3));
+  }
+  uint4* dp = (uint4*)dst;
+#pragma unroll
+  for (int q = 0; q < 3; ++q) {
+    dp[2 * q] = make_uint4(pl[q][0], pl[q][1], pl[q][2], pl[q][3]);
+    dp[2 * q + 1] = make_uint4(pl[q][4], pl[q][5], pl[q][6], pl[q][7]);
+  }
+  dp[6] = make_uint4(__float_as_uint(-p - 1 >= -149 ? mx_pow2(-p - 1) : 0.f), 0u, 0u, 0u);
+}
+
+// The signed bytes 2 e2m1(code) (-12 .. 12) of the four codes in the low 16 bits of h: the
+// magnitude field indexes a byte table of the values and one of their negations (a byte
+// permutation each), the sign bit picks between them.
+__device__ __forceinline__ uint32_t mx_q4(uint32_t h) {
+  const uint32_t sel = h & 0x7777u;
+  const uint32_t pos = __byte_perm(0x03020100u, 0x0C080604u, sel);    //  0,  1,  2,  3 |  4,  6,  8,  12
+  const uint32_t neg = __byte_perm(0xFDFEFF00u, 0xF4F8FAFCu, sel);    // -0, -1, -2, -3 | -4, -6, -8, -12
+  const uint32_t msk = __byte_perm(0u, 0xFFFFFFFFu, (h >> 1) & 0x4444u);   // 0xFF where the sign bit is set
+  return (pos & ~msk) | (neg & msk);
+}
+
+// Sum over one 32-element block of e2m1(code_k) x_k, x as a digit block: the integer sums of the
+// codes (as 2 e2m1) times each digit plane (dp4a, four products an instruction) are exact; the
+// three are combined in fp32 and scaled by the block's factor.
+__device__ __forceinline__ float mx_block_dot_dig(const uint4 c, const uint8_t* d) {
+  const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+  const uint4* dp = (const uint4*)d;
+  const uint4 p0a = dp[0], p0b = dp[1], p1a = dp[2], p1b = dp[3], p2a = dp[4], p2b = dp[5];
+  const uint32_t d0[8] = {p0a.x, p0a.y, p0a.z, p0a.w, p0b.x, p0b.y, p0b.z, p0b.w};
+  const uint32_t d1[8] = {p1a.x, p1a.y, p1a.z, p1a.w, p1b.x, p1b.y, p1b.z, p1b.w};
+  const uint32_t d2[8] = {p2a.x, p2a.y, p2a.z, p2a.w, p2b.x, p2b.y, p2b.z, p2b.w};
+  int s0 = 0, s1 = 0, s2 = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int lo = (int)mx_q4(w[i]), hi = (int)mx_q4(w[i] >> 16);   // elements 8i..8i+3, 8i+4..8i+7
+    s0 = __dp4a(lo, (int)d0[2 * i], s0); s0 = __dp4a(hi, (int)d0[2 * i + 1], s0);
+    s1 = __dp4a(lo, (int)d1[2 * i], s1); s1 = __dp4a(hi, (int)d1[2 * i + 1], s1);
+    s2 = __dp4a(lo, (int)d2[2 * i], s2); s2 = __dp4a(hi, (int)d2[2 * i + 1], s2);
+  }
+  return ((float)s2 * 65536.f + (float)s1 * 256.f + (float)s0) * __uint_as_float(((const uint32_t*)d)[24]);
+}
+
+// grid ceil(rows K/32 / 128), block 128: the digit blocks of rows of K values (bf16 when
+// bf16 != 0, else fp32), one block per thread: dst[row][K/32][kMxDig]. Under a programmatic
+// launch it first waits for the kernel that wrote the rows.
+__global__ void __launch_bounds__(128) mx_digits_kernel(const void* __restrict__ src, int bf16, int rows, int K,
+                                                        uint8_t* __restrict__ dst) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int nb = K / 32;
+  if (i >= (size_t)rows * nb) return;
+  const size_t row = i / nb, b = i % nb;
+  float v[32];
+  if (bf16) {
+    const uint4* sp = (const uint4*)((const uint16_t*)src + row * K + 32 * b);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint4 u = __ldg(sp + j);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        v[8 * j + 2 * h] = bf16lo(w[h]);
+        v[8 * j + 2 * h + 1] = bf16hi(w[h]);
+      }
+    }
+  } else {
+    const float4* sp = (const float4*)((const float*)src + row * K + 32 * b);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float4 q = __ldcg(sp + j);
+      v[4 * j] = q.x; v[4 * j + 1] = q.y; v[4 * j + 2] = q.z; v[4 * j + 3] = q.w;
+    }
+  }
+  mx_digit_block(v, dst + i * kMxDig);
+}
+
 // grid ceil(R / kMvWarps), block 32 kMvWarps: warp w of CTA b computes row b kMvWarps + w.
 __global__ void __launch_bounds__(kMvWarps * 32) mx_gemv_kernel(const uint32_t* __restrict__ q,
                                                                 const uint8_t* __restrict__ e, int R, int K,
@@ -553,13 +658,13 @@ __device__ __forceinline__ void mx_load2(MxChunk2& c, const uint32_t* qa, const 
     c.sb[u] = in ? __ldg(eb + b) : 0u;
   }
 }
-__device__ __forceinline__ void mx_dot2(const MxChunk2& c, int b0, int nb, const float* xs, int lane, float2& acc) {
+__device__ __forceinline__ void mx_dot2(const MxChunk2& c, int b0, int nb, const uint8_t* xd, int lane, float2& acc) {
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     const int b = b0 + 32 * u + lane;
     if (b < nb) {
-      acc.x = fmaf(mx_block_dot(c.ca[u], xs + b * kMvXStride), mx_scale(c.sa[u]), acc.x);
-      acc.y = fmaf(mx_block_dot(c.cb[u], xs + b * kMvXStride), mx_scale(c.sb[u]), acc.y);
+      acc.x = fmaf(mx_block_dot_dig(c.ca[u], xd + b * kMxDig), mx_scale(c.sa[u]), acc.x);
+      acc.y = fmaf(mx_block_dot_dig(c.cb[u], xd + b * kMxDig), mx_scale(c.sb[u]), acc.y);
     }
   }
 }
@@ -570,10 +675,11 @@ __device__ __forceinline__ void mx_stage(float* dst, const float* src, int n) { 
 
 // grid (ceil(S I / kMxLWarps), T), block 32 kMxLWarps: a[t][s][i] = silu(G x_t)_i (U x_t)_i for the
 // expert of slot s (slot k = the shared expert), one (slot, row) per warp. Under a programmatic
-// launch the CTA stages x_t (the layer input, complete since the router passed its own wait)
-// before waiting for the top-k; then each warp resolves its expert and requests its rows.
+// launch the CTA copies x_t's digit blocks (written before the router ran, so complete once this
+// kernel starts) before waiting for the top-k; then each warp resolves its expert and requests
+// its rows.
 __global__ void __launch_bounds__(kMxLWarps * 32) mx_gateup_kernel(MxLayerParams p) {
-  extern __shared__ __align__(16) float xs[];   // x_t, [H/32][kMvXStride]
+  extern __shared__ __align__(16) unsigned char xd[];   // x_t's digit blocks, [H/32][kMxDig]
   const int t = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nb = p.H / 32;
   const int item = blockIdx.x * kMxLWarps + warp;
@@ -582,8 +688,8 @@ __global__ void __launch_bounds__(kMxLWarps * 32) mx_gateup_kernel(MxLayerParams
   const uint32_t *gq = nullptr, *uq = nullptr;
   const uint8_t *ge = nullptr, *ue = nullptr;
   MxChunk2 c;
-  const uint16_t* xt = p.x + (size_t)t * p.H;
-  for (int b = threadIdx.x; b < nb; b += blockDim.x) mx_stage_bf16(xt + 32 * b, xs + b * kMvXStride);
+  const uint4* xsrc = (const uint4*)(p.xdig + (size_t)t * nb * kMxDig);
+  for (int q = threadIdx.x; q < nb * (kMxDig / 16); q += blockDim.x) ((uint4*)xd)[q] = __ldcg(xsrc + q);
   griddep_wait();   // the top-k has completed
   griddep_launch_dependents();
   if (has) {
@@ -598,7 +704,7 @@ __global__ void __launch_bounds__(kMxLWarps * 32) mx_gateup_kernel(MxLayerParams
   if (!has) return;
   float2 acc = make_float2(0.f, 0.f);
   for (int b0 = 0;;) {
-    mx_dot2(c, b0, nb, xs, lane, acc);
+    mx_dot2(c, b0, nb, xd, lane, acc);
     b0 += 4 * 32;
     if (b0 >= nb) break;
     mx_load2(c, gq, ge, uq, ue, b0, nb, lane);
@@ -610,11 +716,12 @@ __global__ void __launch_bounds__(kMxLWarps * 32) mx_gateup_kernel(MxLayerParams
 // grid (ceil(H / kMxLWarps), T), block 32 kMxLWarps, a hidden row per warp:
 // h[t][j] += sum_{s<k} w[t][s] (D_s a[t][s])_j + sg[t] (D_shared a[t][k])_j, in that order.
 // Each warp resolves every slot's expert (the selection is complete: the top-k ran before the
-// gate/up kernel passed its wait) and requests its row's first blocks, then waits for a[t].
+// gate/up kernel passed its wait) and requests its row's first blocks, then waits for the digit
+// blocks of a[t] and copies them.
 __global__ void __launch_bounds__(kMxLWarps * 32, 2) mx_down_kernel(MxLayerParams p) {
-  extern __shared__ __align__(16) float as[];   // a[t][s], s < S: [S][I/32][kMvXStride]
+  extern __shared__ __align__(16) unsigned char ad[];   // a[t][s]'s digit blocks, [S][I/32][kMxDig]
   const int t = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int nb = p.I / 32, sstride = nb * kMvXStride;
+  const int nb = p.I / 32, sstride = nb * kMxDig;
   const int row = blockIdx.x * kMxLWarps + warp;
   const bool has = row < p.H;
   const uint4* q[kMxMaxSlots];
@@ -634,9 +741,10 @@ __global__ void __launch_bounds__(kMxLWarps * 32, 2) mx_down_kernel(MxLayerParam
     c[sl] = in ? __ldg(q[sl] + lane) : make_uint4(0u, 0u, 0u, 0u);
     sc[sl] = in ? __ldg(e[sl] + lane) : 0u;
   }
-  griddep_wait();   // the gate/up kernel has completed: a is final
+  griddep_wait();   // the digit blocks of a are complete
   griddep_launch_dependents();
-  for (int sl = 0; sl < p.S; ++sl) mx_stage(as + sl * sstride, p.a + ((size_t)t * p.S + sl) * p.I, p.I);
+  const uint4* asrc = (const uint4*)(p.adig + (size_t)t * p.S * sstride);
+  for (int qq = threadIdx.x; qq < p.S * sstride / 16; qq += blockDim.x) ((uint4*)ad)[qq] = __ldcg(asrc + qq);
   __syncthreads();
   if (!has) return;
   float y[kMxMaxSlots];
@@ -647,7 +755,7 @@ __global__ void __launch_bounds__(kMxLWarps * 32, 2) mx_down_kernel(MxLayerParam
 #pragma unroll
     for (int sl = 0; sl < kMxMaxSlots; ++sl)
       if (sl < p.S && b < nb)
-        y[sl] = fmaf(mx_block_dot(c[sl], as + sl * sstride + b * kMvXStride), mx_scale(sc[sl]), y[sl]);
+        y[sl] = fmaf(mx_block_dot_dig(c[sl], ad + sl * sstride + b * kMxDig), mx_scale(sc[sl]), y[sl]);
     b0 += 32;
     if (b0 >= nb) break;
 #pragma unroll
@@ -681,9 +789,18 @@ static cudaError_t mx_launch(const void* fn, dim3 grid, dim3 block, size_t smem,
   return cudaLaunchKernelExC(&cfg, fn, args);
 }
 
+cudaError_t launch_mx_digits(const void* src, bool bf16, int rows, int K, uint8_t* dst, cudaStream_t s, bool pdl) {
+  const size_t n = (size_t)rows * (K / 32);
+  const void* sp = src;
+  int b16 = bf16 ? 1 : 0;
+  void* args[] = {(void*)&sp, &b16, &rows, &K, &dst};
+  return mx_launch((const void*)mx_digits_kernel, dim3((unsigned)((n + 127) / 128)), dim3(128), 0, s, pdl, args);
+}
+
+// gate/up, the digit blocks of a, down
 cudaError_t launch_mx_layer(const MxLayerParams& p, cudaStream_t s, bool pdl) {
-  const size_t sg = sizeof(float) * (size_t)(p.H / 32) * kMvXStride;
-  const size_t sd = sizeof(float) * (size_t)p.S * (p.I / 32) * kMvXStride;
+  const size_t sg = (size_t)(p.H / 32) * kMxDig;
+  const size_t sd = (size_t)p.S * (p.I / 32) * kMxDig;
   cudaError_t e = cudaFuncSetAttribute((const void*)mx_gateup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sg);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute((const void*)mx_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sd);
@@ -692,6 +809,8 @@ cudaError_t launch_mx_layer(const MxLayerParams& p, cudaStream_t s, bool pdl) {
   void* args[] = {&q};
   e = mx_launch((const void*)mx_gateup_kernel, dim3((p.S * p.I + kMxLWarps - 1) / kMxLWarps, p.T), dim3(kMxLWarps * 32),
                 sg, s, pdl, args);
+  if (e != cudaSuccess) return e;
+  e = launch_mx_digits(p.a, false, p.T * p.S, p.I, p.adig, s, pdl);
   if (e != cudaSuccess) return e;
   return mx_launch((const void*)mx_down_kernel, dim3((p.H + kMxLWarps - 1) / kMxLWarps, p.T), dim3(kMxLWarps * 32), sd,
                    s, pdl, args);
