@@ -958,7 +958,7 @@ def ours_mx(args, cfg):
             qm.moe_layer_forward_timed(layer, xs[i:i + 1], hs[i:i + 1], xo[i:i + 1], ws=ws, events=evs[s],
                                        stream=stream)
     stream.synchronize()
-    names = ["route_logits", "topk", "mx_gateup+mx_down", "norm"]
+    names = ["digits_x+route_logits", "topk", "mx_gateup+digits_a+mx_down", "norm"]
     dur = [sum(evs[s][j].elapsed_time(evs[s][j + 1]) for s in range(prof_n)) / prof_n for j in range(nst)]
     # end to end with host buffers: x and h in, x_out back, every step
     e2e_n = min(args.e2e_steps, steps, 512)
@@ -990,13 +990,14 @@ def ours_mx(args, cfg):
                    "l2": "inputs larger than L2: 3.4 GB expert pool, 64 rotating tokens"},
         "hbm_gbs": per_tok * steps / (ms * 1e-3) / 1e9, "active_bytes_per_token": per_tok,
         "stage_ms": dict(zip(names, dur)),
-        "roofline": {"bound": "hbm", "kernel": "mx_gateup_kernel + mx_down_kernel", "achieved": achieved,
+        "roofline": {"bound": "hbm", "kernel": "mx_gateup_kernel + mx_digits_kernel (a) + mx_down_kernel",
+                     "achieved": achieved,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                      "traffic": recorded_traffic("mx_experts", "mxfp4_q4", MX_SOURCES),
                      "algorithmic_bytes": per_tok, "peak_kind": peak_kind},
         "e2e": {"value": e2e_n / (e2e_ms * 1e-3), "unit": "tokens/s", "steps": e2e_n,
                 "h2d_bytes_per_step": cfg.H * 6, "d2h_bytes_per_step": cfg.H * 2},
-        "gpu_launches": 5 * steps, "path": path, "clocks": clk,
+        "gpu_launches": 7 * steps, "path": path, "clocks": clk,
     }
     if rank == 0 and not args.no_cpu_baseline:
         rate, n, threads, el = mx_oracle_sample(cfg, args.cpu_seconds)
