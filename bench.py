@@ -113,6 +113,30 @@ class Clocks:
         return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(smax), "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ------------------------------------------------------------------ end-to-end timing
+E2E_REPS = 3
+
+
+def e2e_ms(step, n, stream, warm=4):
+    """Milliseconds for n calls of step(s) (host copies in, the public call, the result back) on
+    stream, after warm untimed calls: the median of E2E_REPS timed runs of the same loop."""
+    import torch
+    with torch.cuda.stream(stream):
+        for s in range(warm):
+            step(s)
+        stream.synchronize()
+        runs = []
+        for _ in range(E2E_REPS):
+            f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            f0.record(stream)
+            for s in range(n):
+                step(s)
+            f1.record(stream)
+            f1.synchronize()
+            runs.append(f0.elapsed_time(f1))
+    return sorted(runs)[len(runs) // 2]
+
+
 # ------------------------------------------------------------------ host buffers
 def packed_inputs(x_bits, h, dev):
     """Pinned host rows holding a step's x (bf16 bits) and h (fp32) back to back, and a device twin
@@ -436,25 +460,17 @@ def ours(args, cfg):
                                          W["h0"].cpu().numpy().reshape(P, 1, cfg.H), dev)
     outh = torch.empty((P, cfg.H), dtype=torch.int16).pin_memory()
     odev = torch.empty((1, cfg.H), dtype=torch.int16, device=dev)
-    with torch.cuda.stream(stream):
-        for s in range(8):
-            i = s % P
-            ind.copy_(inh[i], non_blocking=True)
-            qm.moe_layer_forward(layers[s % C], xdev, hdev, odev, ws=ws, stream=stream)
-            outh[i:i + 1].copy_(odev, non_blocking=True)
-        stream.synchronize()
-        if dist:
-            dist.barrier()
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        f0.record(stream)
-        for s in range(e2e_n):
-            i = s % P
-            ind.copy_(inh[i], non_blocking=True)   # x and h of the step, one copy
-            qm.moe_layer_forward(layers[s % C], xdev, hdev, odev, ws=ws, stream=stream)
-            outh[i:i + 1].copy_(odev, non_blocking=True)
-        f1.record(stream)
-    f1.synchronize()
-    e2e_ms = max_over_ranks(f0.elapsed_time(f1), dist, dev)
+    def e2e_step(s):
+        i = s % P
+        ind.copy_(inh[i], non_blocking=True)   # x and h of the step, one copy
+        qm.moe_layer_forward(layers[s % C], xdev, hdev, odev, ws=ws, stream=stream)
+        outh[i:i + 1].copy_(odev, non_blocking=True)
+
+    e2e_step(0)
+    stream.synchronize()
+    if dist:
+        dist.barrier()
+    e2e_ms_ = max_over_ranks(e2e_ms(e2e_step, e2e_n, stream, warm=8), dist, dev)
 
     peaks, peak_kind = measured_peaks()
     active = cfg.active_bytes_per_token                      # expert bytes per token (4 experts)
@@ -482,7 +498,7 @@ def ours(args, cfg):
         "roofline": {"bound": "hbm", "kernel": names[j_dom], "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
                      "algorithmic_bytes": dom_bytes, "peak_kind": peak_kind},
-        "e2e": {"value": job_throughput(world, e2e_n, e2e_ms), "unit": UNIT, "steps": e2e_n,
+        "e2e": {"value": job_throughput(world, e2e_n, e2e_ms_), "unit": UNIT, "steps": e2e_n, "reps": E2E_REPS,
                 "h2d_bytes_per_step": cfg.H * 2 + cfg.H * 4, "d2h_bytes_per_step": cfg.H * 2},
         "gpu_launches": nk * args.steps, "path": path,
         "clocks": clk,
@@ -571,16 +587,12 @@ def ours_prefill(args, cfg):
     inh, ind, xd, hd = packed_inputs(np.stack(xs_host), np.stack([h.cpu().numpy() for h in hs]), dev)
     outh = torch.empty((T, cfg.H), dtype=torch.int16).pin_memory()
     e2e_n = min(steps, 32)
-    with torch.cuda.stream(stream):
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        f0.record(stream)
-        for i in range(e2e_n):
-            ind.copy_(inh[i % NB], non_blocking=True)   # x and h of the batch, one copy
-            qm.moe_layer_forward(layer, xd, hd, xo, ws=ws, stream=stream)
-            outh.copy_(xo, non_blocking=True)
-        f1.record(stream)
-    f1.synchronize()
-    e2e_ms = f0.elapsed_time(f1)
+    def e2e_step(i):
+        ind.copy_(inh[i % NB], non_blocking=True)   # x and h of the batch, one copy
+        qm.moe_layer_forward(layer, xd, hd, xo, ws=ws, stream=stream)
+        outh.copy_(xo, non_blocking=True)
+
+    e2e_ms_ = e2e_ms(e2e_step, e2e_n, stream, warm=2)
     peaks, peak_kind = measured_peaks()
     shared_tc = cfg.T >= 64 and os.environ.get("MOE_PREFILL_SHARED", "") != "mma" or \
         os.environ.get("MOE_PREFILL_SHARED", "") == "tc"
@@ -608,7 +620,7 @@ def ours_prefill(args, cfg):
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                      "traffic": recorded_traffic("prefill_grouped_gateup", cfg.name, PREFILL_SOURCES),
                      "algorithmic_bytes": gu_bytes, "peak_kind": peak_kind},
-        "e2e": {"value": T * e2e_n / (e2e_ms * 1e-3), "unit": "tokens/s", "steps": e2e_n,
+        "e2e": {"value": T * e2e_n / (e2e_ms_ * 1e-3), "unit": "tokens/s", "steps": e2e_n, "reps": E2E_REPS,
                 "h2d_bytes_per_step": T * cfg.H * (2 + 4), "d2h_bytes_per_step": T * cfg.H * 2},
         # router (GEMM, norms, combine), top-k, grouping, digits of x, gate/up, digits of a, down,
         # combine + norm; with the shared expert on tcgen05 also its tables of x, gate/up, tables of a, down
@@ -699,17 +711,13 @@ def ours_stack(args, cfg):
     outh = torch.empty((P, cfg.H), dtype=torch.int16).pin_memory()
     od = torch.empty(cfg.H, dtype=torch.int16, device=dev)
     e2e_n = min(steps, 256)
-    with torch.cuda.stream(stream):
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        f0.record(stream)
-        for s in range(e2e_n):
-            i = s % P
-            ind.copy_(inh[i], non_blocking=True)   # x and h of the step, one copy
-            qm.moe_stack_forward(arr, xd, hd, od, ws=ws, stream=stream)
-            outh[i].copy_(od, non_blocking=True)
-        f1.record(stream)
-    f1.synchronize()
-    e2e_ms = f0.elapsed_time(f1)
+    def e2e_step(s):
+        i = s % P
+        ind.copy_(inh[i], non_blocking=True)   # x and h of the step, one copy
+        qm.moe_stack_forward(arr, xd, hd, od, ws=ws, stream=stream)
+        outh[i].copy_(od, non_blocking=True)
+
+    e2e_ms_ = e2e_ms(e2e_step, e2e_n, stream)
     peaks, peak_kind = measured_peaks()
     active = cfg.active_bytes_per_token               # 24 layers x 4 experts
     tok_s = steps / (ms * 1e-3)
@@ -731,7 +739,7 @@ def ours_stack(args, cfg):
         "roofline": {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
                      "algorithmic_bytes": dom_bytes, "peak_kind": peak_kind},
-        "e2e": {"value": e2e_n / (e2e_ms * 1e-3), "unit": UNIT, "steps": e2e_n,
+        "e2e": {"value": e2e_n / (e2e_ms_ * 1e-3), "unit": UNIT, "steps": e2e_n, "reps": E2E_REPS,
                 "h2d_bytes_per_step": cfg.H * (2 + 4), "d2h_bytes_per_step": cfg.H * 2},
         "gpu_launches": (1 if path == "fused" else 4 * cfg.layers) * steps, "clocks": clk,
     }
@@ -958,24 +966,20 @@ def ours_mx(args, cfg):
             qm.moe_layer_forward_timed(layer, xs[i:i + 1], hs[i:i + 1], xo[i:i + 1], ws=ws, events=evs[s],
                                        stream=stream)
     stream.synchronize()
-    names = ["digits_x+route_logits", "topk", "mx_gateup+digits_a+mx_down", "norm"]
+    names = ["route_logits+digits_x", "topk", "mx_gateup+mx_down", "norm"]
     dur = [sum(evs[s][j].elapsed_time(evs[s][j + 1]) for s in range(prof_n)) / prof_n for j in range(nst)]
     # end to end with host buffers: x and h in, x_out back, every step
     e2e_n = min(args.e2e_steps, steps, 512)
     inh, ind, xdev, hdev = packed_inputs(x_host.reshape(P, 1, cfg.H), h0.cpu().numpy().reshape(P, 1, cfg.H), dev)
     outh = torch.empty((P, cfg.H), dtype=torch.int16).pin_memory()
     odev = torch.empty((1, cfg.H), dtype=torch.int16, device=dev)
-    with torch.cuda.stream(stream):
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        f0.record(stream)
-        for s in range(e2e_n):
-            i = s % P
-            ind.copy_(inh[i], non_blocking=True)
-            qm.moe_layer_forward(layer, xdev, hdev, odev, ws=ws, stream=stream)
-            outh[i:i + 1].copy_(odev, non_blocking=True)
-        f1.record(stream)
-    f1.synchronize()
-    e2e_ms = f0.elapsed_time(f1)
+    def e2e_step(s):
+        i = s % P
+        ind.copy_(inh[i], non_blocking=True)
+        qm.moe_layer_forward(layer, xdev, hdev, odev, ws=ws, stream=stream)
+        outh[i:i + 1].copy_(odev, non_blocking=True)
+
+    e2e_ms_ = e2e_ms(e2e_step, e2e_n, stream, warm=8)
     peaks, peak_kind = measured_peaks()
     per_tok = (cfg.k + 1) * mx_bytes_per_expert(cfg)
     achieved = per_tok / (dur[2] * 1e-3) / 1e9
@@ -990,14 +994,14 @@ def ours_mx(args, cfg):
                    "l2": "inputs larger than L2: 3.4 GB expert pool, 64 rotating tokens"},
         "hbm_gbs": per_tok * steps / (ms * 1e-3) / 1e9, "active_bytes_per_token": per_tok,
         "stage_ms": dict(zip(names, dur)),
-        "roofline": {"bound": "hbm", "kernel": "mx_gateup_kernel + mx_digits_kernel (a) + mx_down_kernel",
+        "roofline": {"bound": "hbm", "kernel": "mx_gateup_kernel + mx_down_kernel",
                      "achieved": achieved,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                      "traffic": recorded_traffic("mx_experts", "mxfp4_q4", MX_SOURCES),
                      "algorithmic_bytes": per_tok, "peak_kind": peak_kind},
-        "e2e": {"value": e2e_n / (e2e_ms * 1e-3), "unit": "tokens/s", "steps": e2e_n,
+        "e2e": {"value": e2e_n / (e2e_ms_ * 1e-3), "unit": "tokens/s", "steps": e2e_n, "reps": E2E_REPS,
                 "h2d_bytes_per_step": cfg.H * 6, "d2h_bytes_per_step": cfg.H * 2},
-        "gpu_launches": 7 * steps, "path": path, "clocks": clk,
+        "gpu_launches": 6 * steps, "path": path, "clocks": clk,
     }
     if rank == 0 and not args.no_cpu_baseline:
         rate, n, threads, el = mx_oracle_sample(cfg, args.cpu_seconds)
@@ -1067,16 +1071,12 @@ def ours_mxgemm(args):
     xh = torch.from_numpy(x_host.view(np.int16)).pin_memory()
     yh = torch.empty((T, R), dtype=torch.float32).pin_memory()
     e2e_n = min(args.e2e_steps, steps, 96)
-    with torch.cuda.stream(stream):
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        f0.record(stream)
-        for i in range(e2e_n):
-            xd.copy_(xh, non_blocking=True)
-            qm.moe_expert_gemm_mxfp4(mats[i % C], xd, y, ws=ws, stream=stream)
-            yh.copy_(y, non_blocking=True)
-        f1.record(stream)
-    f1.synchronize()
-    e2e_ms = f0.elapsed_time(f1)
+    def e2e_step(i):
+        xd.copy_(xh, non_blocking=True)
+        qm.moe_expert_gemm_mxfp4(mats[i % C], xd, y, ws=ws, stream=stream)
+        yh.copy_(y, non_blocking=True)
+
+    e2e_ms_ = e2e_ms(e2e_step, e2e_n, stream, warm=2)
     peaks, peak_kind = measured_peaks()
     fp4_peak = 4.0 * peaks["bf16_tflops"]   # dense fp4 = 4 x dense bf16 (nominal 9 / 2.25 PFLOP/s)
     flops = 2.0 * R * K * T
@@ -1097,7 +1097,7 @@ def ours_mxgemm(args):
                      "traffic": None, "algorithmic_flops": flops,
                      "peak_kind": f"{peak_kind} bf16 x 4 (fp4 / bf16 nominal ratio); achieved counts the product once, "
                                   f"the five activation terms issue 5x these fp4 MMA flops"},
-        "e2e": {"value": T * e2e_n / (e2e_ms * 1e-3), "unit": "tokens/s", "steps": e2e_n,
+        "e2e": {"value": T * e2e_n / (e2e_ms_ * 1e-3), "unit": "tokens/s", "steps": e2e_n, "reps": E2E_REPS,
                 "h2d_bytes_per_step": T * K * 2, "d2h_bytes_per_step": T * R * 4},
         "gpu_launches": 3 * steps, "clocks": clk,
     }

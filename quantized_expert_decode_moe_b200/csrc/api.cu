@@ -214,8 +214,6 @@ moe_status mx_chain(const moe_layer* L, const uint16_t* x_in, float* h, int T, u
   mark(0);
   const int H = L->hidden, I = L->inter, E = L->n_experts, k = L->top_k, S = slots_of(L);
   const WsLayout W = layout_of(L, T);
-  // the digit blocks of x first (the gate/up kernel reads them before its own wait)
-  if (launch_mx_digits(x_in, true, T, H, at<uint8_t>(ws, W.mxx), s, pdl) != cudaSuccess) return MOE_ERR_CUDA;
   RouteParams rp{};
   rp.H = H; rp.E = E; rp.T = T; rp.has_shared = L->has_shared;
   rp.x = x_in; rp.router_w = L->router_w; rp.router_bias = L->router_bias; rp.gate_w = L->shared_gate_w;
@@ -231,6 +229,8 @@ moe_status mx_chain(const moe_layer* L, const uint16_t* x_in, float* h, int T, u
   } else if (launch_route(rp, s, pdl) != cudaSuccess) {
     return MOE_ERR_CUDA;
   }
+  // the digit blocks of x, beside the router (the gate/up kernel reads them before its own wait)
+  if (launch_mx_digits(x_in, T, H, at<uint8_t>(ws, W.mxx), s, pdl) != cudaSuccess) return MOE_ERR_CUDA;
   mark(1);
   TopkParams tp{};
   tp.E = E; tp.k = k; tp.T = T; tp.has_shared = L->has_shared; tp.H = H;
@@ -247,7 +247,7 @@ moe_status mx_chain(const moe_layer* L, const uint16_t* x_in, float* h, int T, u
   mp.H = H; mp.I = I; mp.k = k; mp.S = S; mp.T = T;
   mp.x = x_in; mp.experts = L->experts; mp.shared = L->shared;
   mp.idx = tp.idx; mp.w = tp.w; mp.sg = tp.sg;
-  mp.a = at<float>(ws, W.a); mp.h = h;
+  mp.h = h;
   mp.xdig = at<uint8_t>(ws, W.mxx); mp.adig = at<uint8_t>(ws, W.mxa);
   if (launch_mx_layer(mp, s, pdl) != cudaSuccess) return MOE_ERR_CUDA;
   mark(3);

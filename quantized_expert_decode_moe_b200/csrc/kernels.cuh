@@ -260,13 +260,12 @@ struct MxLayerParams {
   const moe_expert* experts;   // device [E]: q codes, scales E8M0 bytes [R][K/32]
   moe_expert shared;           // slot k when S > k
   const int32_t* idx; const float* w; const float* sg;   // [T][k], [T][k], [T]
-  float* a;                    // [T][S][I]
   float* h;                    // [T][H], in place: h + the weighted expert outputs
-  const uint8_t* xdig;         // [T][H/32] digit blocks of x (launch_mx_digits, before the router)
-  uint8_t* adig;               // [T][S][I/32] digit blocks of a (written between gate/up and down)
+  const uint8_t* xdig;         // [T][H/32] digit blocks of x (launch_mx_digits, after the router)
+  uint8_t* adig;               // [T][S][I/32] digit blocks of a (written by the gate/up kernel)
 };
-// digit blocks of rows of K values (bf16 or fp32) for the MXFP4 layer kernels: 112 bytes per 32
-cudaError_t launch_mx_digits(const void* src, bool bf16, int rows, int K, uint8_t* dst, cudaStream_t s, bool pdl);
+// digit blocks of rows of K bf16 values for the MXFP4 layer kernels: 112 bytes per 32
+cudaError_t launch_mx_digits(const uint16_t* src, int rows, int K, uint8_t* dst, cudaStream_t s, bool pdl);
 cudaError_t launch_mx_layer(const MxLayerParams& p, cudaStream_t s, bool pdl = false);
 cudaError_t launch_gateup(const GateUpParams& p, int bits, int T, bool pdl, cudaStream_t s);
 cudaError_t launch_down(const DownParams& p, int bits, int T, bool pdl, cudaStream_t s);

@@ -33,12 +33,16 @@
 #include <cudaTypedefs.h>
 #include <math.h>
 
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "kernels.cuh"
 #include "sync.cuh"
 #include "tc.cuh"
 
 namespace qmoe {
+
+namespace cg = cooperative_groups;
 
 // ------------------------------------------------------------------ mat-vec (decode)
 constexpr int kMvWarps = 8;
@@ -145,37 +149,6 @@ __device__ __forceinline__ void mx_stage_bf16(const uint16_t* src, float* dst) {
 // exact, others round within 2^-23 of it. Written once per call by mx_digits_kernel.
 constexpr int kMxDig = 112;   // bytes per digit block (96 digits, the factor, padding to 16)
 
-__device__ __forceinline__ void mx_digit_block(const float (&v)[32], uint8_t* dst) {
-  float m = 0.f;
-#pragma unroll
-  for (int k = 0; k < 32; ++k) m = fmaxf(m, fabsf(v[k]));
-  int p = 0;
-  if (m > 0.f) {   // m = f 2^E, f in [0.5, 1); below 2^-126 treated as 2^-126
-    const int E = m >= 0x1p-126f ? (int)((__float_as_uint(m) >> 23) & 0xFFu) - 126 : -125;
-    p = 22 - E;
-  }
-  const float u1 = mx_pow2(p / 2), u2 = mx_pow2(p - p / 2);   // 2^p as two normal factors
-  uint32_t pl[3][8] = {};
-#pragma unroll
-  for (int k = 0; k < 32; ++k) {
-    const int X = __float2int_rn(v[k] * u1 * u2);   // |X| <= 2^22
-    const int d0 = ((X + 128) & 255) - 128;
-    const int X1 = (X - d0) / 256;
-    const int d1 = ((X1 + 128) & 255) - 128;
-    const int d2 = (X1 - d1) / 256;
-    pl[0][k >> 2] |= (uint32_t)(d0 & 255) << (8 * (k & 3));
-    pl[1][k >> 2] |= (uint32_t)(d1 & 255) << (8 * (k & 3));
-    pl[2][k >> 2] |= (uint32_t)(d2 & 255) << (8 * (k & 3));
-  }
-  uint4* dp = (uint4*)dst;
-#pragma unroll
-  for (int q = 0; q < 3; ++q) {
-    dp[2 * q] = make_uint4(pl[q][0], pl[q][1], pl[q][2], pl[q][3]);
-    dp[2 * q + 1] = make_uint4(pl[q][4], pl[q][5], pl[q][6], pl[q][7]);
-  }
-  dp[6] = make_uint4(__float_as_uint(-p - 1 >= -149 ? mx_pow2(-p - 1) : 0.f), 0u, 0u, 0u);
-}
-
 // The signed bytes 2 e2m1(code) (-12 .. 12) of the four codes in the low 16 bits of h: the
 // magnitude field indexes a byte table of the values and one of their negations (a byte
 // permutation each), the sign bit picks between them.
@@ -208,39 +181,40 @@ __device__ __forceinline__ float mx_block_dot_dig(const uint4 c, const uint8_t* 
   return ((float)s2 * 65536.f + (float)s1 * 256.f + (float)s0) * __uint_as_float(((const uint32_t*)d)[24]);
 }
 
-// grid ceil(rows K/32 / 128), block 128: the digit blocks of rows of K values (bf16 when
-// bf16 != 0, else fp32), one block per thread: dst[row][K/32][kMxDig]. Under a programmatic
-// launch it first waits for the kernel that wrote the rows.
-__global__ void __launch_bounds__(128) mx_digits_kernel(const void* __restrict__ src, int bf16, int rows, int K,
-                                                        uint8_t* __restrict__ dst) {
-  griddep_wait();
-  griddep_launch_dependents();
-  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int nb = K / 32;
-  if (i >= (size_t)rows * nb) return;
-  const size_t row = i / nb, b = i % nb;
-  float v[32];
-  if (bf16) {
-    const uint4* sp = (const uint4*)((const uint16_t*)src + row * K + 32 * b);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint4 u = __ldg(sp + j);
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        v[8 * j + 2 * h] = bf16lo(w[h]);
-        v[8 * j + 2 * h + 1] = bf16hi(w[h]);
-      }
-    }
-  } else {
-    const float4* sp = (const float4*)((const float*)src + row * K + 32 * b);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float4 q = __ldcg(sp + j);
-      v[4 * j] = q.x; v[4 * j + 1] = q.y; v[4 * j + 2] = q.z; v[4 * j + 3] = q.w;
-    }
+// The digit block of 32 values held one per lane (lane k: value k), written to o; the whole warp
+// calls it. The block's largest magnitude by warp shuffles, each lane's three digit bytes stored
+// directly, the factor and the padding by lane 0.
+__device__ __forceinline__ void mx_digit_lanes(float v, int lane, uint8_t* o) {
+  const float m = warp_max(fabsf(v));
+  int p = 0;
+  if (m > 0.f) {   // m = f 2^E, f in [0.5, 1); below 2^-126 treated as 2^-126
+    const int E = m >= 0x1p-126f ? (int)((__float_as_uint(m) >> 23) & 0xFFu) - 126 : -125;
+    p = 22 - E;
   }
-  mx_digit_block(v, dst + i * kMxDig);
+  const int X = __float2int_rn(v * mx_pow2(p / 2) * mx_pow2(p - p / 2));   // |X| <= 2^22
+  const int d0 = ((X + 128) & 255) - 128;
+  const int X1 = (X - d0) / 256;
+  const int d1 = ((X1 + 128) & 255) - 128;
+  const int d2 = (X1 - d1) / 256;
+  o[lane] = (uint8_t)(d0 & 255);
+  o[32 + lane] = (uint8_t)(d1 & 255);
+  o[64 + lane] = (uint8_t)(d2 & 255);
+  if (lane == 0) *(uint4*)(o + 96) = make_uint4(__float_as_uint(-p - 1 >= -149 ? mx_pow2(-p - 1) : 0.f), 0u, 0u, 0u);
+}
+
+// grid ceil(rows K/32 / 8), block 256: the digit blocks of rows of K bf16 values,
+// dst[row][K/32][kMxDig], a warp per block. It reads the rows without waiting: under a
+// programmatic launch it follows a kernel that triggered its dependents only after its own wait
+// (so the rows' writer, two launches back, has completed). It waits for that kernel before it
+// exits, so that whatever waits for this one also finds that one complete.
+__global__ void __launch_bounds__(256) mx_digits_kernel(const uint16_t* __restrict__ src, int rows, int K,
+                                                        uint8_t* __restrict__ dst) {
+  griddep_launch_dependents();
+  const size_t wi = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;   // the warp's block
+  const int lane = threadIdx.x & 31, nb = K / 32;
+  if (wi < (size_t)rows * nb)   // whole warps
+    mx_digit_lanes(bf16_to_f32(__ldg(src + (wi / nb) * K + (wi % nb) * 32 + lane)), lane, dst + wi * kMxDig);
+  griddep_wait();
 }
 
 // grid ceil(R / kMvWarps), block 32 kMvWarps: warp w of CTA b computes row b kMvWarps + w.
@@ -673,35 +647,40 @@ __device__ __forceinline__ void mx_stage(float* dst, const float* src, int n) { 
   for (int b = threadIdx.x; b < n / 32; b += blockDim.x) mx_stage_f32(src + 32 * b, dst + b * kMvXStride);
 }
 
-// grid (ceil(S I / kMxLWarps), T), block 32 kMxLWarps: a[t][s][i] = silu(G x_t)_i (U x_t)_i for the
-// expert of slot s (slot k = the shared expert), one (slot, row) per warp. Under a programmatic
-// launch the CTA copies x_t's digit blocks (written before the router ran, so complete once this
-// kernel starts) before waiting for the top-k; then each warp resolves its expert and requests
+// grid (S I / kMxLWarps, T), block 32 kMxLWarps, clusters of kMxGuCluster CTAs: a[t][s][i] =
+// silu(G x_t)_i (U x_t)_i for the expert of slot s (slot k = the shared expert), one (slot, row)
+// per warp; a cluster's warps hold the 32 rows of one block of a, which they gather in the shared
+// memory of the cluster's first CTA, whose first warp writes the block's digit block to adig.
+// Under a programmatic launch the CTA copies x_t's digit blocks (complete once this kernel
+// starts: their kernel ran two launches before, and the top-k triggered this launch only after
+// its own wait) before waiting for the top-k; then each warp resolves its expert and requests
 // its rows.
-__global__ void __launch_bounds__(kMxLWarps * 32) mx_gateup_kernel(MxLayerParams p) {
+constexpr int kMxGuCluster = 32 / kMxLWarps;
+__global__ void __cluster_dims__(kMxGuCluster, 1, 1) __launch_bounds__(kMxLWarps * 32)
+mx_gateup_kernel(MxLayerParams p) {
   extern __shared__ __align__(16) unsigned char xd[];   // x_t's digit blocks, [H/32][kMxDig]
+  __shared__ float ablk[32];                             // the cluster's block of a (first CTA)
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
   const int t = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nb = p.H / 32;
-  const int item = blockIdx.x * kMxLWarps + warp;
-  const bool has = item < p.S * p.I;
-  const int sl = has ? item / p.I : 0, i = has ? item % p.I : 0;
-  const uint32_t *gq = nullptr, *uq = nullptr;
-  const uint8_t *ge = nullptr, *ue = nullptr;
+  const int item = blockIdx.x * kMxLWarps + warp;   // < S I: the grid is exact
+  // first phase of the cluster barrier: passed below once every CTA of the cluster runs, before
+  // any writes into the first CTA's shared memory
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+  const int sl = item / p.I, i = item % p.I;
   MxChunk2 c;
   const uint4* xsrc = (const uint4*)(p.xdig + (size_t)t * nb * kMxDig);
   for (int q = threadIdx.x; q < nb * (kMxDig / 16); q += blockDim.x) ((uint4*)xd)[q] = __ldcg(xsrc + q);
   griddep_wait();   // the top-k has completed
   griddep_launch_dependents();
-  if (has) {
-    const moe_expert* ex = sl < p.k ? p.experts + p.idx[t * p.k + sl] : &p.shared;
-    gq = ex->gate.q + (size_t)i * (p.H / 8);
-    uq = ex->up.q + (size_t)i * (p.H / 8);
-    ge = (const uint8_t*)ex->gate.scales + (size_t)i * nb;
-    ue = (const uint8_t*)ex->up.scales + (size_t)i * nb;
-    mx_load2(c, gq, ge, uq, ue, 0, nb, lane);
-  }
+  const moe_expert* ex = sl < p.k ? p.experts + p.idx[t * p.k + sl] : &p.shared;
+  const uint32_t* gq = ex->gate.q + (size_t)i * (p.H / 8);
+  const uint32_t* uq = ex->up.q + (size_t)i * (p.H / 8);
+  const uint8_t* ge = (const uint8_t*)ex->gate.scales + (size_t)i * nb;
+  const uint8_t* ue = (const uint8_t*)ex->up.scales + (size_t)i * nb;
+  mx_load2(c, gq, ge, uq, ue, 0, nb, lane);
   __syncthreads();
-  if (!has) return;
   float2 acc = make_float2(0.f, 0.f);
   for (int b0 = 0;;) {
     mx_dot2(c, b0, nb, xd, lane, acc);
@@ -710,7 +689,11 @@ __global__ void __launch_bounds__(kMxLWarps * 32) mx_gateup_kernel(MxLayerParams
     mx_load2(c, gq, ge, uq, ue, b0, nb, lane);
   }
   const float g = warp_sum(acc.x), u = warp_sum(acc.y);
-  if (lane == 0) p.a[((size_t)t * p.S + sl) * p.I + i] = g / (1.f + expf(-g)) * u;
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+  if (lane == 0) *cluster.map_shared_rank(&ablk[rank * kMxLWarps + warp], 0) = g / (1.f + expf(-g)) * u;
+  cluster.sync();   // the block is complete; nobody touches another CTA's shared memory after this
+  if (rank == 0 && warp == 0)   // item is the block's first row
+    mx_digit_lanes(ablk[lane], lane, p.adig + (((size_t)t * p.S + sl) * (p.I / 32) + i / 32) * kMxDig);
 }
 
 // grid (ceil(H / kMxLWarps), T), block 32 kMxLWarps, a hidden row per warp:
@@ -789,15 +772,14 @@ static cudaError_t mx_launch(const void* fn, dim3 grid, dim3 block, size_t smem,
   return cudaLaunchKernelExC(&cfg, fn, args);
 }
 
-cudaError_t launch_mx_digits(const void* src, bool bf16, int rows, int K, uint8_t* dst, cudaStream_t s, bool pdl) {
+cudaError_t launch_mx_digits(const uint16_t* src, int rows, int K, uint8_t* dst, cudaStream_t s, bool pdl) {
   const size_t n = (size_t)rows * (K / 32);
-  const void* sp = src;
-  int b16 = bf16 ? 1 : 0;
-  void* args[] = {(void*)&sp, &b16, &rows, &K, &dst};
-  return mx_launch((const void*)mx_digits_kernel, dim3((unsigned)((n + 127) / 128)), dim3(128), 0, s, pdl, args);
+  const uint16_t* sp = src;
+  void* args[] = {(void*)&sp, &rows, &K, &dst};
+  return mx_launch((const void*)mx_digits_kernel, dim3((unsigned)((n + 7) / 8)), dim3(256), 0, s, pdl, args);
 }
 
-// gate/up, the digit blocks of a, down
+// gate/up (writing the digit blocks of a), down
 cudaError_t launch_mx_layer(const MxLayerParams& p, cudaStream_t s, bool pdl) {
   const size_t sg = (size_t)(p.H / 32) * kMxDig;
   const size_t sd = (size_t)p.S * (p.I / 32) * kMxDig;
@@ -807,10 +789,8 @@ cudaError_t launch_mx_layer(const MxLayerParams& p, cudaStream_t s, bool pdl) {
   if (e != cudaSuccess) return e;
   MxLayerParams q = p;
   void* args[] = {&q};
-  e = mx_launch((const void*)mx_gateup_kernel, dim3((p.S * p.I + kMxLWarps - 1) / kMxLWarps, p.T), dim3(kMxLWarps * 32),
-                sg, s, pdl, args);
-  if (e != cudaSuccess) return e;
-  e = launch_mx_digits(p.a, false, p.T * p.S, p.I, p.adig, s, pdl);
+  // S I / kMxLWarps CTAs: a multiple of the cluster size, since 32 divides I
+  e = mx_launch((const void*)mx_gateup_kernel, dim3(p.S * p.I / kMxLWarps, p.T), dim3(kMxLWarps * 32), sg, s, pdl, args);
   if (e != cudaSuccess) return e;
   return mx_launch((const void*)mx_down_kernel, dim3((p.H + kMxLWarps - 1) / kMxLWarps, p.T), dim3(kMxLWarps * 32), sd,
                    s, pdl, args);
