@@ -744,9 +744,9 @@ cudaError_t launch_fused(const FusedParams& p, int bits, cudaStream_t s) {
   const size_t sm = fused_smem_bytes(p.H, p.I, p.S, bits);
   if (sm > (size_t)fu_optin_smem()) return cudaErrorInvalidConfiguration;
   const void* fn = bits == 4 ? (const void*)fused_decode_kernel<4> : (const void*)fused_decode_kernel<2>;
-  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  cudaError_t e = set_func_attr(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e != cudaSuccess) return e;
-  if ((e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm)) != cudaSuccess) return e;
+  if ((e = set_func_attr(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm)) != cudaSuccess) return e;
   // the grid-wide barriers need every CTA resident at once: at most one wave
   int per_sm = 0;
   if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, sm)) != cudaSuccess) return e;

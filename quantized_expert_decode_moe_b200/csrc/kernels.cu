@@ -4,6 +4,9 @@
 // (token, rank) pairs by expert.
 #include <math.h>
 
+#include <mutex>
+#include <vector>
+
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -78,6 +81,29 @@ int num_sms() {
     if (n <= 0) n = 148;
   }
   return n;
+}
+
+// cudaFuncSetAttribute once per kernel, device, attribute and value: a launch
+// that repeats the last value set skips the driver call.
+cudaError_t set_func_attr(const void* fn, cudaFuncAttribute attr, int value) {
+  struct Entry {
+    const void* fn;
+    int dev, attr, value;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> seen;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (Entry& x : seen)
+    if (x.fn == fn && x.dev == dev && x.attr == (int)attr) {
+      if (x.value == value) return cudaSuccess;
+      if ((e = cudaFuncSetAttribute(fn, attr, value)) == cudaSuccess) x.value = value;
+      return e;
+    }
+  if ((e = cudaFuncSetAttribute(fn, attr, value)) == cudaSuccess) seen.push_back({fn, dev, (int)attr, value});
+  return e;
 }
 
 // CTA count for a split-unit kernel: every CTA range >= nspans units (a tile
@@ -494,10 +520,10 @@ static cudaError_t launch_ex(const void* fn, dim3 grid, dim3 block, size_t smem,
 // to be drained to change its L1/shared split between kernels of a chain
 // (a dependent kernel can then start next to its predecessor).
 static cudaError_t set_smem(const void* fn, size_t bytes) {
-  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  cudaError_t e = set_func_attr(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e != cudaSuccess) return e;
   if (bytes <= 48 * 1024) return cudaSuccess;
-  return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  return set_func_attr(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
 cudaError_t launch_route(const RouteParams& p, cudaStream_t s, bool pdl) {

@@ -282,6 +282,8 @@ cudaError_t launch_prefill_down(const PrefillParams& p, int bits, cudaStream_t s
 cudaError_t launch_selftest_wait(uint32_t* status, unsigned long long bound_ns, cudaStream_t s);
 cudaError_t launch_selftest_grid(unsigned* hdr, unsigned long long bound_ns, cudaStream_t s);
 int num_sms();
+// cudaFuncSetAttribute, skipped when the kernel already has that value on the current device
+cudaError_t set_func_attr(const void* fn, cudaFuncAttribute attr, int value);
 bool fused_supported(int H, int I, int E, int k, int has_shared, int bits);
 int fused_ctas(int H, int I);
 size_t fused_smem_bytes(int H, int I, int S, int bits);

@@ -149,20 +149,29 @@ __device__ __forceinline__ void mx_stage_bf16(const uint16_t* src, float* dst) {
 // exact, others round within 2^-23 of it. Written once per call by mx_digits_kernel.
 constexpr int kMxDig = 112;   // bytes per digit block (96 digits, the factor, padding to 16)
 
-// The signed bytes 2 e2m1(code) (-12 .. 12) of the four codes in the low 16 bits of h: the
-// magnitude field indexes a byte table of the values and one of their negations (a byte
-// permutation each), the sign bit picks between them.
-__device__ __forceinline__ uint32_t mx_q4(uint32_t h) {
-  const uint32_t sel = h & 0x7777u;
-  const uint32_t pos = __byte_perm(0x03020100u, 0x0C080604u, sel);    //  0,  1,  2,  3 |  4,  6,  8,  12
-  const uint32_t neg = __byte_perm(0xFDFEFF00u, 0xF4F8FAFCu, sel);    // -0, -1, -2, -3 | -4, -6, -8, -12
-  const uint32_t msk = __byte_perm(0u, 0xFFFFFFFFu, (h >> 1) & 0x4444u);   // 0xFF where the sign bit is set
-  return (pos & ~msk) | (neg & msk);
+// prmt.b32 in its generic mode: byte n of the result is byte (c >> 4n) & 7 of b:a, or, where bit
+// 4n + 3 of c is set, that byte's sign bit replicated; only the low 16 bits of c are read.
+__device__ __forceinline__ uint32_t prmt_b32(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// The signed bytes 2 e2m1(code) (-12 .. 12) of the four codes in the low 16 bits of s, given sn =
+// s with every code's sign bit flipped. The code itself selects from a byte table of the values
+// 2 e2m1 (all below 0x80): a set sign bit turns its byte into 0, so p holds the positive codes'
+// values; the flipped codes give the negative codes' magnitudes n; 0x80 - n per byte never
+// borrows (n <= 12) and, with the top bit flipped back, is -n as a byte.
+__device__ __forceinline__ uint32_t mx_q4(uint32_t s, uint32_t sn) {
+  const uint32_t p = prmt_b32(0x03020100u, 0x0C080604u, s);    //  0, 1, 2, 3 | 4, 6, 8, 12
+  const uint32_t n = prmt_b32(0x03020100u, 0x0C080604u, sn);
+  return p | ((0x80808080u - n) ^ 0x80808080u);
 }
 
 // Sum over one 32-element block of e2m1(code_k) x_k, x as a digit block: the integer sums of the
-// codes (as 2 e2m1) times each digit plane (dp4a, four products an instruction) are exact; the
-// three are combined in fp32 and scaled by the block's factor.
+// codes (as 2 e2m1) times each digit plane (dp4a, four products an instruction) combine exactly
+// in 32 bits (|sum of 2 e2m1(c) X| <= 32 * 12 * 2^22 < 2^31), then one conversion and the block's
+// factor.
 __device__ __forceinline__ float mx_block_dot_dig(const uint4 c, const uint8_t* d) {
   const uint32_t w[4] = {c.x, c.y, c.z, c.w};
   const uint4* dp = (const uint4*)d;
@@ -173,12 +182,13 @@ __device__ __forceinline__ float mx_block_dot_dig(const uint4 c, const uint8_t* 
   int s0 = 0, s1 = 0, s2 = 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int lo = (int)mx_q4(w[i]), hi = (int)mx_q4(w[i] >> 16);   // elements 8i..8i+3, 8i+4..8i+7
+    const uint32_t wn = w[i] ^ 0x88888888u;
+    const int lo = (int)mx_q4(w[i], wn), hi = (int)mx_q4(w[i] >> 16, wn >> 16);   // elements 8i..8i+3, 8i+4..8i+7
     s0 = __dp4a(lo, (int)d0[2 * i], s0); s0 = __dp4a(hi, (int)d0[2 * i + 1], s0);
     s1 = __dp4a(lo, (int)d1[2 * i], s1); s1 = __dp4a(hi, (int)d1[2 * i + 1], s1);
     s2 = __dp4a(lo, (int)d2[2 * i], s2); s2 = __dp4a(hi, (int)d2[2 * i + 1], s2);
   }
-  return ((float)s2 * 65536.f + (float)s1 * 256.f + (float)s0) * __uint_as_float(((const uint32_t*)d)[24]);
+  return (float)(s0 + s1 * 256 + s2 * 65536) * __uint_as_float(((const uint32_t*)d)[24]);
 }
 
 // The digit block of 32 values held one per lane (lane k: value k), written to o; the whole warp
@@ -252,7 +262,7 @@ __global__ void __launch_bounds__(kMvWarps * 32) mx_gemv_kernel(const uint32_t* 
 cudaError_t launch_mx_gemv(const uint32_t* q, const uint8_t* e, int R, int K, const float* x, float* y,
                            cudaStream_t s) {
   const size_t sm = sizeof(float) * (size_t)(K / 32) * kMvXStride;
-  cudaError_t err = cudaFuncSetAttribute((const void*)mx_gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t err = set_func_attr((const void*)mx_gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)sm);
   if (err != cudaSuccess) return err;
   mx_gemv_kernel<<<(R + kMvWarps - 1) / kMvWarps, kMvWarps * 32, sm, s>>>(q, e, R, K, x, y);
@@ -597,7 +607,7 @@ cudaError_t launch_mx_gemm(const uint32_t* q, const uint8_t* e, int R, int K, co
   p.status = (uint32_t*)ws;
   p.wait_ns = wait_ns;
   const size_t sm = (size_t)kMxStages * kMxStageBytes + sizeof(MxSmem);
-  err = cudaFuncSetAttribute((const void*)mx_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  err = set_func_attr((const void*)mx_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (err != cudaSuccess) return err;
   mx_gemm_kernel<<<dim3(R / kMxM, tpad / kMxN, W.splits), 128, sm, s>>>(map, p);
   err = cudaGetLastError();
@@ -655,8 +665,10 @@ __device__ __forceinline__ void mx_stage(float* dst, const float* src, int n) { 
 // starts: their kernel ran two launches before, and the top-k triggered this launch only after
 // its own wait) before waiting for the top-k; then each warp resolves its expert and requests
 // its rows.
+// 64 registers (4 CTAs per SM): the 512 CTAs of 4 slots x intermediate 1024 run in one wave on
+// 148 SMs, which pays for the few spilled bytes.
 constexpr int kMxGuCluster = 32 / kMxLWarps;
-__global__ void __cluster_dims__(kMxGuCluster, 1, 1) __launch_bounds__(kMxLWarps * 32)
+__global__ void __cluster_dims__(kMxGuCluster, 1, 1) __launch_bounds__(kMxLWarps * 32, 4)
 mx_gateup_kernel(MxLayerParams p) {
   extern __shared__ __align__(16) unsigned char xd[];   // x_t's digit blocks, [H/32][kMxDig]
   __shared__ float ablk[32];                             // the cluster's block of a (first CTA)
@@ -700,19 +712,21 @@ mx_gateup_kernel(MxLayerParams p) {
 // h[t][j] += sum_{s<k} w[t][s] (D_s a[t][s])_j + sg[t] (D_shared a[t][k])_j, in that order.
 // Each warp resolves every slot's expert (the selection is complete: the top-k ran before the
 // gate/up kernel passed its wait) and requests its row's first blocks, then waits for the digit
-// blocks of a[t] and copies them.
-__global__ void __launch_bounds__(kMxLWarps * 32, 2) mx_down_kernel(MxLayerParams p) {
+// blocks of a[t] and copies them. NS >= S bounds the slots held in registers; with up to 4 slots
+// the kernel fits 64 registers, so 4 CTAs per SM hold all 512 CTAs of hidden 4096 in one wave.
+template <int NS>
+__global__ void __launch_bounds__(kMxLWarps * 32, NS <= 4 ? 4 : 2) mx_down_kernel(MxLayerParams p) {
   extern __shared__ __align__(16) unsigned char ad[];   // a[t][s]'s digit blocks, [S][I/32][kMxDig]
   const int t = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nb = p.I / 32, sstride = nb * kMxDig;
   const int row = blockIdx.x * kMxLWarps + warp;
   const bool has = row < p.H;
-  const uint4* q[kMxMaxSlots];
-  const uint8_t* e[kMxMaxSlots];
-  uint4 c[kMxMaxSlots];
-  unsigned sc[kMxMaxSlots];
+  const uint4* q[NS];
+  const uint8_t* e[NS];
+  uint4 c[NS];
+  unsigned sc[NS];
 #pragma unroll
-  for (int sl = 0; sl < kMxMaxSlots; ++sl) {
+  for (int sl = 0; sl < NS; ++sl) {
     q[sl] = nullptr;
     e[sl] = nullptr;
     if (has && sl < p.S) {
@@ -730,19 +744,19 @@ __global__ void __launch_bounds__(kMxLWarps * 32, 2) mx_down_kernel(MxLayerParam
   for (int qq = threadIdx.x; qq < p.S * sstride / 16; qq += blockDim.x) ((uint4*)ad)[qq] = __ldcg(asrc + qq);
   __syncthreads();
   if (!has) return;
-  float y[kMxMaxSlots];
+  float y[NS];
 #pragma unroll
-  for (int sl = 0; sl < kMxMaxSlots; ++sl) y[sl] = 0.f;
+  for (int sl = 0; sl < NS; ++sl) y[sl] = 0.f;
   for (int b0 = 0;;) {   // every slot's block b0 + lane in flight at once
     const int b = b0 + lane;
 #pragma unroll
-    for (int sl = 0; sl < kMxMaxSlots; ++sl)
+    for (int sl = 0; sl < NS; ++sl)
       if (sl < p.S && b < nb)
         y[sl] = fmaf(mx_block_dot_dig(c[sl], ad + sl * sstride + b * kMxDig), mx_scale(sc[sl]), y[sl]);
     b0 += 32;
     if (b0 >= nb) break;
 #pragma unroll
-    for (int sl = 0; sl < kMxMaxSlots; ++sl) {
+    for (int sl = 0; sl < NS; ++sl) {
       const bool in = sl < p.S && b0 + lane < nb;
       c[sl] = in ? __ldg(q[sl] + b0 + lane) : make_uint4(0u, 0u, 0u, 0u);
       sc[sl] = in ? __ldg(e[sl] + b0 + lane) : 0u;
@@ -750,7 +764,7 @@ __global__ void __launch_bounds__(kMxLWarps * 32, 2) mx_down_kernel(MxLayerParam
   }
   float acc = p.h[(size_t)t * p.H + row];
 #pragma unroll
-  for (int sl = 0; sl < kMxMaxSlots; ++sl)
+  for (int sl = 0; sl < NS; ++sl)
     if (sl < p.S) acc = fmaf(sl < p.k ? p.w[t * p.k + sl] : p.sg[t], warp_sum(y[sl]), acc);
   if (lane == 0) p.h[(size_t)t * p.H + row] = acc;
 }
@@ -783,17 +797,19 @@ cudaError_t launch_mx_digits(const uint16_t* src, int rows, int K, uint8_t* dst,
 cudaError_t launch_mx_layer(const MxLayerParams& p, cudaStream_t s, bool pdl) {
   const size_t sg = (size_t)(p.H / 32) * kMxDig;
   const size_t sd = (size_t)p.S * (p.I / 32) * kMxDig;
-  cudaError_t e = cudaFuncSetAttribute((const void*)mx_gateup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sg);
+  cudaError_t e = set_func_attr((const void*)mx_gateup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sg);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute((const void*)mx_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sd);
+  const void* down = p.S <= 2 ? (const void*)mx_down_kernel<2>
+                   : p.S <= 4 ? (const void*)mx_down_kernel<4>
+                   : p.S <= 6 ? (const void*)mx_down_kernel<6> : (const void*)mx_down_kernel<kMxMaxSlots>;
+  e = set_func_attr(down, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sd);
   if (e != cudaSuccess) return e;
   MxLayerParams q = p;
   void* args[] = {&q};
   // S I / kMxLWarps CTAs: a multiple of the cluster size, since 32 divides I
   e = mx_launch((const void*)mx_gateup_kernel, dim3(p.S * p.I / kMxLWarps, p.T), dim3(kMxLWarps * 32), sg, s, pdl, args);
   if (e != cudaSuccess) return e;
-  return mx_launch((const void*)mx_down_kernel, dim3((p.H + kMxLWarps - 1) / kMxLWarps, p.T), dim3(kMxLWarps * 32), sd,
-                   s, pdl, args);
+  return mx_launch(down, dim3((p.H + kMxLWarps - 1) / kMxLWarps, p.T), dim3(kMxLWarps * 32), sd, s, pdl, args);
 }
 
 }  // namespace qmoe

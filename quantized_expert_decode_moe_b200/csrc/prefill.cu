@@ -573,7 +573,7 @@ size_t pf_max_chunks(int T, int k, int E, int chunk) {
 
 cudaError_t launch_group(const GroupParams& p, cudaStream_t s) {
   const size_t sm = sizeof(int) * 3 * (size_t)p.E;
-  cudaError_t e = cudaFuncSetAttribute((const void*)group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  cudaError_t e = set_func_attr((const void*)group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   GroupParams q = p;
   void* args[] = {&q};
@@ -584,9 +584,9 @@ cudaError_t launch_group(const GroupParams& p, cudaStream_t s) {
 int pf_chunk_tokens(int H, int I) { return (H > 4096 || I > 4096) ? 4 : 8; }
 
 static cudaError_t pf_prepare(const void* fn, size_t bytes) {
-  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  cudaError_t e = set_func_attr(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  return set_func_attr(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
 // Launch configuration of a grouped kernel (gate/up or down) of a layer shape:

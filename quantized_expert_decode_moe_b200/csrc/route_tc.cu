@@ -344,7 +344,7 @@ cudaError_t launch_route_gemm(const RouteParams& p, cudaStream_t s) {
   splits = splits < 1 ? 1 : (splits > kRtSplitMax ? kRtSplitMax : splits);
   splits = splits > nstg ? nstg : splits;
   const size_t sm = (size_t)kRtStages * kRtStageBytes + sizeof(RtSmem);
-  e = cudaFuncSetAttribute((const void*)route_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  e = set_func_attr((const void*)route_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   void* args2[] = {&q, &splits};
   e = cudaLaunchKernel((const void*)route_tc_kernel, dim3(rw / kRtM, rx / kRtN, splits), dim3(128), args2, sm, s);

@@ -557,7 +557,7 @@ cudaError_t launch_tc_dense(const TcParams& p, cudaStream_t s) {
   if (!q.nst || p.M % kTcM || p.K % kGroup || p.Tpad != tc_pad16(p.T)) return cudaErrorInvalidConfiguration;
   const size_t sm = tc_geom(q.nt, q.hilo, q.nst).total;
   const void* fn = p.bits == 4 ? (const void*)tc_dense_kernel<4> : (const void*)tc_dense_kernel<2>;
-  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  cudaError_t e = set_func_attr(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   void* args[] = {&q};
   const dim3 grid(p.M / kTcM, (q.Tpad + q.nt - 1) / q.nt, q.splits);

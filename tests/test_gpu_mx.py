@@ -145,11 +145,12 @@ def test_gemm_rejects_bad_shapes_before_launch(dev):
 import fixtures  # noqa: E402
 
 
-def mx_layer(name, E, dev, scale=(116, 120)):
+def mx_layer(name, E, dev, scale=(116, 120), k=None, shared=True):
     """The router, gamma and shared-gate vectors of a fixture layer with MXFP4 experts (seeded)."""
     base = fixtures.CONFIGS[name]
-    cfg = base if E == base.E else fixtures.Config(base.name, H=base.H, E=E, k=base.k, I=base.I, bits=4,
-                                                   scale_sigma=base.scale_sigma)
+    k = base.k if k is None else k
+    cfg = base if (E, k, shared) == (base.E, base.k, True) else fixtures.Config(
+        base.name, H=base.H, E=E, k=k, I=base.I, bits=4, scale_sigma=base.scale_sigma, has_shared=shared)
     Wr, rb, gs, gamma = fixtures.layer_vectors(cfg, 0)
     H, I = cfg.H, cfg.I
     host = [gen.mx_expert(e, H, I, *scale) for e in range(E + 1)]
@@ -162,9 +163,9 @@ def mx_layer(name, E, dev, scale=(116, 120)):
         return torch.from_numpy(a.view(np.int16)).to(dev)
 
     layer = qm.Layer(hidden=H, inter=I, top_k=cfg.k, bits=4, group=32, router_w=t16(Wr),
-                     experts=[dev_expert(ex) for ex in host[:E]], rms_gamma=t16(gamma), shared=dev_expert(host[E]),
-                     shared_gate_w=t16(gs), router_bias=torch.from_numpy(rb).to(dev) if rb is not None else None,
-                     rms_eps=cfg.rms_eps)
+                     experts=[dev_expert(ex) for ex in host[:E]], rms_gamma=t16(gamma),
+                     shared=dev_expert(host[E]) if shared else None, shared_gate_w=t16(gs) if shared else None,
+                     router_bias=torch.from_numpy(rb).to(dev) if rb is not None else None, rms_eps=cfg.rms_eps)
     return cfg, layer, host, (Wr, rb, gs, gamma)
 
 
@@ -200,6 +201,23 @@ def test_mx_layer_matches_oracle(dev, name, E, T):
     assert eh <= 1e-4 and ex_ <= 1e-4, (eh, ex_)   # fp32 sums of exact products: far inside the bar
     assert np.array_equal(xo.view(np.uint16), gen.f32_to_bf16_bits(xf))   # x_out is the RNE of x_out_f32
     print(f"mxfp4 layer {name} E={E} T={T}: h' {eh:.2e}, x_out {ex_:.2e}")
+
+
+@pytest.mark.parametrize("k,shared,T", [(1, False, 1), (5, True, 2), (8, True, 1), (8, True, 12)])
+def test_mx_layer_slot_counts(dev, k, shared, T):
+    """1 to 9 expert slots per token (top-1 without the shared expert, top-5 and top-8 with it): the
+    down kernel holds up to 2, 6 or 9 slots in registers; routing bit-exact, outputs within the
+    layer tolerance of the oracle."""
+    cfg, layer, host, (Wr, rb, gs, gamma) = mx_layer("tiny", 16, dev, k=k, shared=shared)
+    x = gen.x_tokens(cfg, 77 + k, T=T)
+    h0 = gen.bf16_bits_to_f32(x).astype(np.float64) * 0.5
+    h, xf, xo, idx, w = run_mx_layer(cfg, layer, x, h0, dev)
+    ref = oracle.mx_layer(x, h0, Wr, gamma, host[:16], host[16] if shared else None, k=k, eps=cfg.rms_eps,
+                          router_bias=rb, gs=gs if shared else None)
+    np.testing.assert_array_equal(idx, ref["idx"])
+    np.testing.assert_allclose(w, ref["w"], rtol=1e-6, atol=1e-7)
+    eh, ex_ = normwise(h, ref["h_out"]), normwise(xf, ref["x_out"])
+    assert eh <= 1e-4 and ex_ <= 1e-4, (eh, ex_)
 
 
 def test_mx_layer_path_and_limits(dev):
