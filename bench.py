@@ -208,7 +208,13 @@ def busy(fn, stream, seconds: float = 0.25):
 
 # kernels of each decode path, in launch order
 KERNELS = {"fused": ["fused_decode_kernel"],
-           "chain": ["route_logits_kernel", "gateup_decode_kernel", "down_decode_kernel", "norm_kernel"]}
+           "chain": ["route_logits_kernel", "gateup_decode_kernel", "down_decode_kernel", "norm_kernel"],
+           "digit": ["route_logits_kernel+mx_digits_kernel", "topk_kernel", "mx_gateup_kernel+mx_down_kernel",
+                     "norm_cluster_kernel"]}
+LAUNCHES = {"fused": 1, "chain": 4, "digit": 6}   # kernels per decode step
+DTYPES = {"fused": "u4 codes x s8 activation digits on int8 tensor cores (s32), fp32 scale+accumulate",
+          "chain": "u4 codes x s8 activation digits on int8 tensor cores (s32), fp32 scale+accumulate",
+          "digit": "u4/u2 codes x s8 digits of 22-bit fixed-point activations by dp4a (s32), fp32 scale+bias"}
 
 
 def kernel_bytes(cfg, name: str, layers: int = 1) -> int:
@@ -225,7 +231,11 @@ def kernel_bytes(cfg, name: str, layers: int = 1) -> int:
            "route_logits_kernel": router + 2 * cfg.H,
            "gateup_decode_kernel": gu + 2 * cfg.H,
            "down_decode_kernel": dn + 4 * cfg.H * (S + 2),
-           "norm_kernel": 6 * cfg.H * 4}[name]
+           "norm_kernel": 6 * cfg.H * 4,
+           "route_logits_kernel+mx_digits_kernel": router + 2 * cfg.H,
+           "topk_kernel": 12 * (cfg.E + 1),
+           "mx_gateup_kernel+mx_down_kernel": gu + dn + 2 * 4 * cfg.H,
+           "norm_cluster_kernel": 6 * cfg.H * 4}[name]
     return per * layers
 
 
@@ -237,7 +247,8 @@ FUSED_SOURCES = ("common.cuh", "kernels.cuh", "fused.cu", "stage.cuh", "sync.cuh
 PREFILL_SOURCES = ("common.cuh", "kernels.cuh", "prefill.cu")
 MX_SOURCES = ("common.cuh", "kernels.cuh", "mx.cu")
 SOURCES_OF = {"route_logits_kernel": ROUTER_SOURCES, "norm_kernel": ROUTER_SOURCES,
-              "fused_decode_kernel": FUSED_SOURCES}
+              "fused_decode_kernel": FUSED_SOURCES, "mx_gateup_kernel+mx_down_kernel": MX_SOURCES}
+TRAFFIC_KEY = {"mx_gateup_kernel+mx_down_kernel": "mx_experts"}   # name of a stage's record in traffic.txt
 
 
 def kernel_src_sha(files=DECODE_SOURCES):
@@ -482,11 +493,12 @@ def ours(args, cfg):
     j_dom = max(range(nk), key=lambda j: dur[j])
     dom_bytes = kernel_bytes(cfg, names[j_dom])
     achieved = dom_bytes / (dur[j_dom] * 1e-3) / 1e9
-    traffic = recorded_traffic(names[j_dom], cfg.name, SOURCES_OF.get(names[j_dom], DECODE_SOURCES))
+    traffic = recorded_traffic(TRAFFIC_KEY.get(names[j_dom], names[j_dom]), cfg.name,
+                               SOURCES_OF.get(names[j_dom], DECODE_SOURCES))
     line = {
         "metric": METRIC, "value": tok_s, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "u4 codes x s8 activation digits on int8 tensor cores (s32), fp32 scale+accumulate",
+        "scaling": "weak", "vs_baseline": None, "dtype": DTYPES[path],
         "data": "synthetic (seeded; no model weights)",
         "config": {"workload": cfg.note, "H": cfg.H, "E": cfg.E, "top_k": cfg.k, "shared": 1, "I": cfg.I,
                    "bits": cfg.bits, "group": cfg.G, "T": 1, "parallelism": f"replicas x{world}",
@@ -500,7 +512,7 @@ def ours(args, cfg):
                      "algorithmic_bytes": dom_bytes, "peak_kind": peak_kind},
         "e2e": {"value": job_throughput(world, e2e_n, e2e_ms_), "unit": UNIT, "steps": e2e_n, "reps": E2E_REPS,
                 "h2d_bytes_per_step": cfg.H * 2 + cfg.H * 4, "d2h_bytes_per_step": cfg.H * 2},
-        "gpu_launches": nk * args.steps, "path": path,
+        "gpu_launches": LAUNCHES[path] * args.steps, "path": path,
         "clocks": clk,
     }
     if rank == 0 and not args.no_cpu_baseline:
@@ -728,7 +740,7 @@ def ours_stack(args, cfg):
         "metric": "24-layer MoE decode tokens/s and achieved HBM GB/s (% of 8 TB/s), 4-bit experts, 1 B200",
         "value": tok_s, "unit": UNIT, "n_gpus": world, "steps": steps, "warmup": max(args.warmup, 3),
         "ms_per_step": ms / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "u4 codes x s8 activation digits on int8 tensor cores (s32), fp32 scale+accumulate",
+        "dtype": DTYPES[path],
         "data": "synthetic (seeded; no model weights)",
         "config": {"workload": cfg.note, "H": cfg.H, "E": cfg.E, "top_k": cfg.k, "shared": 1, "I": cfg.I,
                    "bits": cfg.bits, "layers": cfg.layers, "T": 1,
@@ -741,7 +753,7 @@ def ours_stack(args, cfg):
                      "algorithmic_bytes": dom_bytes, "peak_kind": peak_kind},
         "e2e": {"value": e2e_n / (e2e_ms_ * 1e-3), "unit": UNIT, "steps": e2e_n, "reps": E2E_REPS,
                 "h2d_bytes_per_step": cfg.H * (2 + 4), "d2h_bytes_per_step": cfg.H * 2},
-        "gpu_launches": (1 if path == "fused" else 4 * cfg.layers) * steps, "clocks": clk,
+        "gpu_launches": (1 if path == "fused" else LAUNCHES[path] * cfg.layers) * steps, "clocks": clk,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -284,15 +284,26 @@ moe_status moe_stack_forward(const moe_layer* layers, int32_t L, const uint16_t*
 
 /*
  * The kernel path that serves a call of T tokens on `layer` (host only,
- * launches nothing): MOE_PATH_FUSED (the fused decode kernel, T = 1),
- * MOE_PATH_CHAIN (the four-kernel decode chain, T <= 8), MOE_PATH_PREFILL
- * (T > 8) or MOE_PATH_MXFP4 (a layer of MXFP4 experts: router, top-k,
- * gate/up + SwiGLU and down + combine, RMSNorm), and in *n_events the number of events moe_layer_forward_timed
- * records on that path (its stages + 1). Either output may be NULL.
+ * launches nothing): MOE_PATH_DIGIT (decode of an affine layer, T <= 8, the
+ * default: router, top-k, gate/up + SwiGLU and down + combine on digit
+ * blocks of x and of the SwiGLU outputs, RMSNorm), MOE_PATH_CHAIN (the
+ * four-kernel decode chain, T <= 8), MOE_PATH_FUSED (the fused decode
+ * kernel, T = 1), MOE_PATH_PREFILL (T > 8) or MOE_PATH_MXFP4 (a layer of
+ * MXFP4 experts, the kernels of MOE_PATH_DIGIT with E2M1 codes), and in
+ * *n_events the number of events moe_layer_forward_timed records on that
+ * path (its stages + 1). Either output may be NULL. For affine decode,
+ * MOE_DECODE_KERNEL=chain in the environment (read at every call) selects
+ * the chain and MOE_DECODE_KERNEL=fused the fused kernel where it fits.
  * Errors: those of moe_workspace_size's layer checks; MOE_ERR_UNSUPPORTED
  * when no path fits (see "Supported shapes").
  */
-typedef enum { MOE_PATH_FUSED = 1, MOE_PATH_CHAIN = 2, MOE_PATH_PREFILL = 3, MOE_PATH_MXFP4 = 4 } moe_path;
+typedef enum {
+  MOE_PATH_FUSED = 1,
+  MOE_PATH_CHAIN = 2,
+  MOE_PATH_PREFILL = 3,
+  MOE_PATH_MXFP4 = 4,
+  MOE_PATH_DIGIT = 5
+} moe_path;
 moe_status moe_layer_path(const moe_layer* layer, int32_t T, int32_t* path, int32_t* n_events);
 
 /*
@@ -336,7 +347,7 @@ moe_status moe_layer_forward_timed(const moe_layer* layer, const uint16_t* x_in,
  * different host threads) race on the array: order them on one stream.
  * Arguments and errors are otherwise those of moe_layer_forward.
  */
-#define MOE_NOALLOC_SCRATCH_BYTES (4u << 20)
+#define MOE_NOALLOC_SCRATCH_BYTES (8u << 20)
 moe_status moe_layer_forward_noalloc(const moe_layer* layer, const uint16_t* x_in, float* h, int32_t T,
                                      uint16_t* x_out, float* x_out_f32, int32_t* topk_idx, float* topk_w,
                                      void* stream);

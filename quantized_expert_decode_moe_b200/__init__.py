@@ -193,7 +193,8 @@ def moe_workspace_size(layer: Layer, max_tokens: int) -> int:
     return n.value
 
 
-PATHS = {1: "fused", 2: "chain", 3: "prefill", 4: "mxfp4"}
+PATHS = {1: "fused", 2: "chain", 3: "prefill", 4: "mxfp4", 5: "digit"}
+NOALLOC_SCRATCH_BYTES = 8 << 20   # MOE_NOALLOC_SCRATCH_BYTES of include/moe.h
 
 
 def moe_layer_path(layer: Layer, T: int):

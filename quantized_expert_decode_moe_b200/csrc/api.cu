@@ -79,35 +79,44 @@ int slots_of(const moe_layer* L) { return L->top_k + (L->has_shared ? 1 : 0); }
 // launch: the fused single-kernel layer for one token, the four-kernel chain
 // for up to 8 tokens, the grouped prefill path above that.
 //
-// Decode defaults to the four-kernel chain: on B200 it measured 24.9 us per
-// 4-bit hidden-4096 layer-token against 44.6 us for the fused kernel, whose
-// phases run one after another inside each CTA while the chain overlaps
-// them across kernels. MOE_DECODE_KERNEL=fused in the environment (read
-// once) selects the fused kernel for single-token calls and stacks wherever
-// it fits.
-enum class Path { kNone, kFused, kChain, kPrefill, kMx };
-bool fused_requested() {
-  static int v = -1;
-  if (v < 0) {
-    const char* e = getenv("MOE_DECODE_KERNEL");
-    v = (e && strcmp(e, "fused") == 0) ? 1 : 0;
-  }
-  return v == 1;
+// Decode of affine layers defaults to the digit-block kernels (mx.cu, the
+// kernels of the MXFP4 layers with the affine codecs): on B200 the four-kernel
+// chain measured 24.4 us per 4-bit hidden-4096 layer-token and the fused
+// kernel 44.6 us, whose phases run one after another inside each CTA.
+// MOE_DECODE_KERNEL in the environment (read at every call) overrides it:
+// "chain" selects the four-kernel chain, "fused" the fused kernel for
+// single-token calls and stacks wherever it fits (the chain otherwise).
+enum class Path { kNone, kFused, kChain, kPrefill, kMx, kDigit };
+enum class DecodeKernel { kDefault, kFused, kChain };
+DecodeKernel decode_kernel_env() {
+  const char* e = getenv("MOE_DECODE_KERNEL");
+  if (e && strcmp(e, "fused") == 0) return DecodeKernel::kFused;
+  if (e && strcmp(e, "chain") == 0) return DecodeKernel::kChain;
+  return DecodeKernel::kDefault;
 }
-// MXFP4 layers, any number of tokens; the down kernel holds the digit blocks of
-// every slot's SwiGLU output in shared memory (112 bytes per 32 values).
+// The digit-block layer kernels (MXFP4 layers at any number of tokens, affine
+// ones up to 8): the down kernel holds the digit blocks of every slot's SwiGLU
+// output in shared memory (112 bytes per 32 values).
+bool digit_smem_fits(const moe_layer* L) { return (size_t)slots_of(L) * (L->inter / 32) * 112 <= 227 * 1024; }
 bool mx_supported(const moe_layer* L, int T) {
   (void)T;
-  return (size_t)slots_of(L) * (L->inter / 32) * 112 <= 227 * 1024;
+  return digit_smem_fits(L);
 }
+int codec_of(const moe_layer* L) { return is_mx(L) ? kCodecMx : L->bits; }
 
 Path path_of(const moe_layer* L, int T) {
   if (is_mx(L)) return mx_supported(L, T) ? Path::kMx : Path::kNone;
-  if (T > kDecodeMaxT) return prefill_supported(L->hidden, L->inter, L->bits) ? Path::kPrefill : Path::kNone;
+  if (T > kDecodeMaxT)   // the grouped prefill, else the digit-block kernels token by token
+    return prefill_supported(L->hidden, L->inter, L->bits) ? Path::kPrefill
+                                                           : (digit_smem_fits(L) ? Path::kDigit : Path::kNone);
   const bool fused = fused_supported(L->hidden, L->inter, L->n_experts, L->top_k, L->has_shared, L->bits);
   const bool chain = chain_supported(L->hidden, L->inter, L->top_k, L->has_shared, L->bits);
-  if (T == 1 && fused && (fused_requested() || !chain)) return Path::kFused;
+  const bool digit = digit_smem_fits(L);
+  const DecodeKernel env = decode_kernel_env();
+  if (T == 1 && fused && (env == DecodeKernel::kFused || (!chain && !digit))) return Path::kFused;
+  if (digit && env == DecodeKernel::kDefault) return Path::kDigit;
   if (chain) return Path::kChain;
+  if (digit) return Path::kDigit;
   return Path::kNone;
 }
 
@@ -203,8 +212,9 @@ moe_status decode_chain(const moe_layer* L, const uint16_t* x_in, float* h, int 
   return MOE_OK;
 }
 
-// A decode layer of MXFP4 experts: router, certified top-k, gate/up with SwiGLU, down with the
-// weighted combine and the residual (mx.cu), RMSNorm.
+// A layer on the digit-block kernels (MXFP4 experts at any number of tokens, affine ones in
+// decode): router, certified top-k, gate/up with SwiGLU, down with the weighted combine and the
+// residual (mx.cu), RMSNorm.
 moe_status mx_chain(const moe_layer* L, const uint16_t* x_in, float* h, int T, uint16_t* x_out, float* x_out_f32,
                     int32_t* topk_idx, float* topk_w, void* ws, cudaStream_t s, void* const* events = nullptr,
                     uint16_t* x_rec = nullptr, float* h_rec = nullptr) {
@@ -230,7 +240,8 @@ moe_status mx_chain(const moe_layer* L, const uint16_t* x_in, float* h, int T, u
     return MOE_ERR_CUDA;
   }
   // the digit blocks of x, beside the router (the gate/up kernel reads them before its own wait)
-  if (launch_mx_digits(x_in, T, H, at<uint8_t>(ws, W.mxx), s, pdl) != cudaSuccess) return MOE_ERR_CUDA;
+  const int codec = codec_of(L);
+  if (launch_mx_digits(x_in, T, H, at<uint8_t>(ws, W.mxx), codec, s, pdl) != cudaSuccess) return MOE_ERR_CUDA;
   mark(1);
   TopkParams tp{};
   tp.E = E; tp.k = k; tp.T = T; tp.has_shared = L->has_shared; tp.H = H;
@@ -244,7 +255,7 @@ moe_status mx_chain(const moe_layer* L, const uint16_t* x_in, float* h, int T, u
   if (topk_w && cudaMemcpyAsync(topk_w, tp.w, sel, cudaMemcpyDeviceToDevice, s) != cudaSuccess) return MOE_ERR_CUDA;
   mark(2);
   MxLayerParams mp{};
-  mp.H = H; mp.I = I; mp.k = k; mp.S = S; mp.T = T;
+  mp.H = H; mp.I = I; mp.k = k; mp.S = S; mp.T = T; mp.codec = codec;
   mp.x = x_in; mp.experts = L->experts; mp.shared = L->shared;
   mp.idx = tp.idx; mp.w = tp.w; mp.sg = tp.sg;
   mp.h = h;
@@ -430,6 +441,7 @@ moe_status moe_layer_path(const moe_layer* layer, int32_t T, int32_t* path, int3
     case Path::kChain: code = MOE_PATH_CHAIN; ev = 5; break;
     case Path::kPrefill: code = MOE_PATH_PREFILL; ev = 6; break;
     case Path::kMx: code = MOE_PATH_MXFP4; ev = 5; break;
+    case Path::kDigit: code = MOE_PATH_DIGIT; ev = 5; break;
     default: return MOE_ERR_UNSUPPORTED;
   }
   if (path) *path = code;
@@ -565,7 +577,8 @@ moe_status moe_layer_forward(const moe_layer* layer, const uint16_t* x_in, float
     case Path::kFused:
       return fused_forward(layer, 1, x_in, h, x_out, x_out_f32, topk_idx, topk_w, nullptr, nullptr, ws, s);
     case Path::kChain: return decode_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, s);
-    case Path::kMx: return mx_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, s);
+    case Path::kMx:
+    case Path::kDigit: return mx_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, s);
     default: return MOE_ERR_UNSUPPORTED;
   }
 }
@@ -588,7 +601,8 @@ moe_status moe_layer_forward_timed(const moe_layer* layer, const uint16_t* x_in,
   cudaStream_t s = (cudaStream_t)stream;
   if (path == Path::kPrefill)
     return prefill_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, s, events);
-  if (path == Path::kMx) return mx_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, s, events);
+  if (path == Path::kMx || path == Path::kDigit)
+    return mx_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, s, events);
   if (path == Path::kFused) {
     if (cudaEventRecord((cudaEvent_t)events[0], s) != cudaSuccess) return MOE_ERR_CUDA;
     if ((st = fused_forward(layer, 1, x_in, h, x_out, x_out_f32, topk_idx, topk_w, nullptr, nullptr, ws, s)))
@@ -629,7 +643,7 @@ moe_status moe_stack_forward(const moe_layer* layers, int32_t L, const uint16_t*
   }
   for (int l = 0; l < L; ++l) {
     const uint16_t* xin = l == 0 ? x_in : x_out;
-    if (path == Path::kMx) {
+    if (path == Path::kMx || path == Path::kDigit) {
       if ((st = mx_chain(&layers[l], xin, h, 1, x_out, nullptr, topk_idx_all ? topk_idx_all + (size_t)l * k : nullptr,
                          nullptr, ws, s, nullptr, layer_inputs ? layer_inputs + (size_t)l * H : nullptr,
                          layer_h ? layer_h + (size_t)l * H : nullptr)))
@@ -692,7 +706,7 @@ moe_status moe_layer_forward_noalloc(const moe_layer* layer, const uint16_t* x_i
   // moe_noalloc_poll_status reads it. The kernels clear their own accumulators.
   if (path == Path::kFused)
     return fused_forward(layer, 1, x_in, h, x_out, x_out_f32, topk_idx, topk_w, nullptr, nullptr, ws, s);
-  if (path == Path::kMx) return mx_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, s);
+  if (path == Path::kMx || path == Path::kDigit) return mx_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, s);
   return decode_chain(layer, x_in, h, T, x_out, x_out_f32, topk_idx, topk_w, ws, s);
 }
 

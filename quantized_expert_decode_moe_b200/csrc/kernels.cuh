@@ -253,19 +253,24 @@ cudaError_t launch_mx_gemv(const uint32_t* q, const uint8_t* e, int R, int K, co
 cudaError_t launch_mx_gemm(const uint32_t* q, const uint8_t* e, int R, int K, const uint16_t* x, int T, float* y,
                            void* ws, unsigned long long wait_ns, cudaStream_t s);
 size_t mx_gemm_ws_bytes(int R, int K, int T);
-// a decode layer of MXFP4 experts, after the router and the top-k
+// Codecs of the digit-block layer kernels: MXFP4 (E2M1 codes, E8M0 scale per 32), affine 4-bit
+// and 2-bit codes with a bf16 scale and bias per 64 (w = q s + b).
+constexpr int kCodecMx = 0, kCodecQ4 = 4, kCodecQ2 = 2;
+// a decode layer on digit blocks (MXFP4 or affine 4-/2-bit experts), after the router and the top-k
 struct MxLayerParams {
   int H, I, k, S, T;
+  int codec;                   // 0 MXFP4, 4 affine 4-bit, 2 affine 2-bit
   const uint16_t* x;           // [T][H] bf16
-  const moe_expert* experts;   // device [E]: q codes, scales E8M0 bytes [R][K/32]
+  const moe_expert* experts;   // device [E]: q codes; scales E8M0 bytes [R][K/32] (MXFP4) or bf16 scales
+                               // and biases [R][K/64] (affine)
   moe_expert shared;           // slot k when S > k
   const int32_t* idx; const float* w; const float* sg;   // [T][k], [T][k], [T]
   float* h;                    // [T][H], in place: h + the weighted expert outputs
   const uint8_t* xdig;         // [T][H/32] digit blocks of x (launch_mx_digits, after the router)
   uint8_t* adig;               // [T][S][I/32] digit blocks of a (written by the gate/up kernel)
 };
-// digit blocks of rows of K bf16 values for the MXFP4 layer kernels: 112 bytes per 32
-cudaError_t launch_mx_digits(const uint16_t* src, int rows, int K, uint8_t* dst, cudaStream_t s, bool pdl);
+// digit blocks of rows of K bf16 values for the layer kernels of a codec: 112 bytes per 32
+cudaError_t launch_mx_digits(const uint16_t* src, int rows, int K, uint8_t* dst, int codec, cudaStream_t s, bool pdl);
 cudaError_t launch_mx_layer(const MxLayerParams& p, cudaStream_t s, bool pdl = false);
 cudaError_t launch_gateup(const GateUpParams& p, int bits, int T, bool pdl, cudaStream_t s);
 cudaError_t launch_down(const DownParams& p, int bits, int T, bool pdl, cudaStream_t s);

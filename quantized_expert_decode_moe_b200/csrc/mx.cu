@@ -145,9 +145,22 @@ __device__ __forceinline__ void mx_stage_bf16(const uint16_t* src, float* dst) {
 // ---- digit blocks (the layer kernels): a 32-value block of x or a as 22-bit fixed point with
 // its own power of two, X = rint(v 2^p), max |v| 2^p < 2^22, split exactly into three balanced
 // signed 8-bit digits (three 32-byte planes), then the factor 2^-(p+1) as a float at byte 96
-// (the 1/2 undoes the codes' 2 e2m1); bf16 values within 2^-14 of the block's largest are
-// exact, others round within 2^-23 of it. Written once per call by mx_digits_kernel.
-constexpr int kMxDig = 112;   // bytes per digit block (96 digits, the factor, padding to 16)
+// (the 1/2 undoes the MXFP4 codes' 2 e2m1; the affine kernels double it back) and the exact
+// sum of the block's X as an int32 at byte 100 (|sum| <= 2^27; the affine bias term). bf16
+// values within 2^-14 of the block's largest are exact, others round within 2^-23 of it.
+// Within a plane the digits follow the order in which the matrix codes expand to bytes
+// (mx_dig_pos). Written once per call by mx_digits_kernel.
+constexpr int kMxDig = 112;   // bytes per digit block (96 digits, the factor, the sum, padding to 16)
+
+// Byte of element k (0..31) of a block within a digit plane. MXFP4: element order (a half-word
+// of codes expands to elements 8i..8i+3). 4-bit: per 8 elements, the even ones then the odd
+// ones (the low and the high nibbles of a code word, masked). 2-bit: per 16 elements, stride 4
+// (code word w shifted by 2j and masked holds elements j, j+4, j+8, j+12).
+__device__ __forceinline__ int mx_dig_pos(int k, int codec) {
+  if (codec == kCodecQ4) return (k & ~7) | ((k & 1) << 2) | ((k >> 1) & 3);
+  if (codec == kCodecQ2) return (k & ~15) | ((k & 3) << 2) | ((k >> 2) & 3);
+  return k;
+}
 
 // prmt.b32 in its generic mode: byte n of the result is byte (c >> 4n) & 7 of b:a, or, where bit
 // 4n + 3 of c is set, that byte's sign bit replicated; only the low 16 bits of c are read.
@@ -191,10 +204,57 @@ __device__ __forceinline__ float mx_block_dot_dig(const uint4 c, const uint8_t* 
   return (float)(s0 + s1 * 256 + s2 * 65536) * __uint_as_float(((const uint32_t*)d)[24]);
 }
 
+// The digit planes of a block as 8 words each.
+struct MxPlanes {
+  uint32_t d0[8], d1[8], d2[8];
+};
+__device__ __forceinline__ MxPlanes mx_planes(const uint8_t* d) {
+  const uint4* dp = (const uint4*)d;
+  const uint4 p0a = dp[0], p0b = dp[1], p1a = dp[2], p1b = dp[3], p2a = dp[4], p2b = dp[5];
+  return MxPlanes{{p0a.x, p0a.y, p0a.z, p0a.w, p0b.x, p0b.y, p0b.z, p0b.w},
+                  {p1a.x, p1a.y, p1a.z, p1a.w, p1b.x, p1b.y, p1b.z, p1b.w},
+                  {p2a.x, p2a.y, p2a.z, p2a.w, p2b.x, p2b.y, p2b.z, p2b.w}};
+}
+
+// Sum over one 32-element block of q_k X_k for 4-bit codes q (0..15) and a digit block in the
+// 4-bit order: the low and the high nibbles of each code word, masked, are four unsigned bytes
+// each (elements 8i + 0, 2, 4, 6 and 8i + 1, 3, 5, 7); exact in 32 bits (32 * 15 * 2^22 < 2^31).
+__device__ __forceinline__ int dq4_block_dot(const uint4 c, const uint8_t* d) {
+  const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+  const MxPlanes P = mx_planes(d);
+  int s0 = 0, s1 = 0, s2 = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int lo = (int)(w[i] & 0x0F0F0F0Fu), hi = (int)((w[i] >> 4) & 0x0F0F0F0Fu);
+    s0 = __dp4a(lo, (int)P.d0[2 * i], s0); s0 = __dp4a(hi, (int)P.d0[2 * i + 1], s0);
+    s1 = __dp4a(lo, (int)P.d1[2 * i], s1); s1 = __dp4a(hi, (int)P.d1[2 * i + 1], s1);
+    s2 = __dp4a(lo, (int)P.d2[2 * i], s2); s2 = __dp4a(hi, (int)P.d2[2 * i + 1], s2);
+  }
+  return s0 + s1 * 256 + s2 * 65536;
+}
+
+// The same for 2-bit codes (two words per block): word i shifted by 2j and masked holds
+// elements 16i + j, + 4, + 8, + 12, the 2-bit order of the digit block.
+__device__ __forceinline__ int dq2_block_dot(const uint2 c, const uint8_t* d) {
+  const uint32_t w[2] = {c.x, c.y};
+  const MxPlanes P = mx_planes(d);
+  int s0 = 0, s1 = 0, s2 = 0;
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int r = (int)((w[i] >> (2 * j)) & 0x03030303u);
+      s0 = __dp4a(r, (int)P.d0[4 * i + j], s0);
+      s1 = __dp4a(r, (int)P.d1[4 * i + j], s1);
+      s2 = __dp4a(r, (int)P.d2[4 * i + j], s2);
+    }
+  return s0 + s1 * 256 + s2 * 65536;
+}
+
 // The digit block of 32 values held one per lane (lane k: value k), written to o; the whole warp
 // calls it. The block's largest magnitude by warp shuffles, each lane's three digit bytes stored
 // directly, the factor and the padding by lane 0.
-__device__ __forceinline__ void mx_digit_lanes(float v, int lane, uint8_t* o) {
+__device__ __forceinline__ void mx_digit_lanes(float v, int lane, uint8_t* o, int codec) {
   const float m = warp_max(fabsf(v));
   int p = 0;
   if (m > 0.f) {   // m = f 2^E, f in [0.5, 1); below 2^-126 treated as 2^-126
@@ -206,10 +266,13 @@ __device__ __forceinline__ void mx_digit_lanes(float v, int lane, uint8_t* o) {
   const int X1 = (X - d0) / 256;
   const int d1 = ((X1 + 128) & 255) - 128;
   const int d2 = (X1 - d1) / 256;
-  o[lane] = (uint8_t)(d0 & 255);
-  o[32 + lane] = (uint8_t)(d1 & 255);
-  o[64 + lane] = (uint8_t)(d2 & 255);
-  if (lane == 0) *(uint4*)(o + 96) = make_uint4(__float_as_uint(-p - 1 >= -149 ? mx_pow2(-p - 1) : 0.f), 0u, 0u, 0u);
+  const int at = mx_dig_pos(lane, codec);
+  o[at] = (uint8_t)(d0 & 255);
+  o[32 + at] = (uint8_t)(d1 & 255);
+  o[64 + at] = (uint8_t)(d2 & 255);
+  const int sum = __reduce_add_sync(0xffffffffu, X);
+  if (lane == 0)
+    *(uint4*)(o + 96) = make_uint4(__float_as_uint(-p - 1 >= -149 ? mx_pow2(-p - 1) : 0.f), (uint32_t)sum, 0u, 0u);
 }
 
 // grid ceil(rows K/32 / 8), block 256: the digit blocks of rows of K bf16 values,
@@ -218,12 +281,12 @@ __device__ __forceinline__ void mx_digit_lanes(float v, int lane, uint8_t* o) {
 // (so the rows' writer, two launches back, has completed). It waits for that kernel before it
 // exits, so that whatever waits for this one also finds that one complete.
 __global__ void __launch_bounds__(256) mx_digits_kernel(const uint16_t* __restrict__ src, int rows, int K,
-                                                        uint8_t* __restrict__ dst) {
+                                                        uint8_t* __restrict__ dst, int codec) {
   griddep_launch_dependents();
   const size_t wi = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;   // the warp's block
   const int lane = threadIdx.x & 31, nb = K / 32;
   if (wi < (size_t)rows * nb)   // whole warps
-    mx_digit_lanes(bf16_to_f32(__ldg(src + (wi / nb) * K + (wi % nb) * 32 + lane)), lane, dst + wi * kMxDig);
+    mx_digit_lanes(bf16_to_f32(__ldg(src + (wi / nb) * K + (wi % nb) * 32 + lane)), lane, dst + wi * kMxDig, codec);
   griddep_wait();
 }
 
@@ -617,50 +680,69 @@ cudaError_t launch_mx_gemm(const uint32_t* q, const uint8_t* e, int R, int K, co
   return cudaGetLastError();
 }
 
-// ------------------------------------------------------------------ a decode layer of MXFP4 experts
-// After the router and the top-k (kernels.cu): gate/up with SwiGLU, then down
-// with the weighted combine and the residual, then the RMSNorm (kernels.cu).
-// The expert descriptors are the layer's: moe_qmat.q the codes, moe_qmat.scales
-// the E8M0 bytes [R][K/32] (uint8), biases unused.
+// ------------------------------------------------------------------ decode layer kernels on digit blocks
+// After the router and the top-k (kernels.cu): gate/up with SwiGLU, then down with the weighted
+// combine and the residual, then the RMSNorm (kernels.cu), for two kinds of expert matrices:
+//  * MXFP4 (kCodecMx): moe_qmat.q the E2M1 codes, scales the E8M0 bytes [R][K/32], biases unused;
+//  * affine 4-bit and 2-bit codes (kCodecQ4, kCodecQ2): q the codes, scales and biases bf16
+//    [R][K/64], w = q s + b per group of 64 consecutive k.
+// A lane takes whole 32-element blocks of a row (16 bytes of codes, 8 for 2-bit codes, and the
+// block's scale, or its group's scale and bias) against x or a as digit blocks whose planes
+// follow the order in which the codes expand to bytes.
 constexpr int kMxLWarps = 8;
 constexpr int kMxMaxSlots = kMaxSlots;
 
-// One lane's share of a 128-block chunk of two MXFP4 rows: blocks b0 + 32 u + lane, u < 4.
-struct MxChunk2 {
-  uint4 ca[4], cb[4];
-  unsigned sa[4], sb[4];
-};
-__device__ __forceinline__ void mx_load2(MxChunk2& c, const uint32_t* qa, const uint8_t* ea, const uint32_t* qb,
-                                         const uint8_t* eb, int b0, int nb, int lane) {
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int b = b0 + 32 * u + lane;
-    const bool in = b < nb;
-    c.ca[u] = in ? __ldg((const uint4*)qa + b) : make_uint4(0u, 0u, 0u, 0u);
-    c.cb[u] = in ? __ldg((const uint4*)qb + b) : make_uint4(0u, 0u, 0u, 0u);
-    c.sa[u] = in ? __ldg(ea + b) : 0u;
-    c.sb[u] = in ? __ldg(eb + b) : 0u;
-  }
+template <int CODEC> struct MxBlk;                               // one block's codes and scale words
+template <> struct MxBlk<kCodecMx> { uint4 c; unsigned e; };
+template <> struct MxBlk<kCodecQ4> { uint4 c; unsigned sb; };   // sb: scale bits | bias bits << 16
+template <> struct MxBlk<kCodecQ2> { uint2 c; unsigned sb; };
+
+// Block b of row `row` of a K-column matrix M (nothing read when !in).
+template <int CODEC>
+__device__ __forceinline__ MxBlk<CODEC> mx_blk_load(const moe_qmat& M, size_t row, int K, int b, bool in);
+template <>
+__device__ __forceinline__ MxBlk<kCodecMx> mx_blk_load<kCodecMx>(const moe_qmat& M, size_t row, int K, int b, bool in) {
+  const size_t at = row * (K / 32) + b;
+  return MxBlk<kCodecMx>{in ? __ldg((const uint4*)M.q + at) : make_uint4(0u, 0u, 0u, 0u),
+                         in ? (unsigned)__ldg((const uint8_t*)M.scales + at) : 0u};
 }
-__device__ __forceinline__ void mx_dot2(const MxChunk2& c, int b0, int nb, const uint8_t* xd, int lane, float2& acc) {
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int b = b0 + 32 * u + lane;
-    if (b < nb) {
-      acc.x = fmaf(mx_block_dot_dig(c.ca[u], xd + b * kMxDig), mx_scale(c.sa[u]), acc.x);
-      acc.y = fmaf(mx_block_dot_dig(c.cb[u], xd + b * kMxDig), mx_scale(c.sb[u]), acc.y);
-    }
-  }
+__device__ __forceinline__ unsigned mx_sb_load(const moe_qmat& M, size_t row, int K, int b, bool in) {
+  const size_t g = row * (K / 64) + b / 2;
+  return in ? (unsigned)__ldg(M.scales + g) | ((unsigned)__ldg(M.biases + g) << 16) : 0u;
+}
+template <>
+__device__ __forceinline__ MxBlk<kCodecQ4> mx_blk_load<kCodecQ4>(const moe_qmat& M, size_t row, int K, int b, bool in) {
+  return MxBlk<kCodecQ4>{in ? __ldg((const uint4*)M.q + row * (K / 32) + b) : make_uint4(0u, 0u, 0u, 0u),
+                         mx_sb_load(M, row, K, b, in)};
+}
+template <>
+__device__ __forceinline__ MxBlk<kCodecQ2> mx_blk_load<kCodecQ2>(const moe_qmat& M, size_t row, int K, int b, bool in) {
+  return MxBlk<kCodecQ2>{in ? __ldg((const uint2*)M.q + row * (K / 32) + b) : make_uint2(0u, 0u),
+                         mx_sb_load(M, row, K, b, in)};
 }
 
-__device__ __forceinline__ void mx_stage(float* dst, const float* src, int n) {   // n floats, n % 32 == 0
-  for (int b = threadIdx.x; b < n / 32; b += blockDim.x) mx_stage_f32(src + 32 * b, dst + b * kMvXStride);
+// The block's share of the row's dot product with the values of digit block d. Affine codes:
+// s sum q X + b sum X, both sums exact integers, times 2^-p (twice the stored factor).
+__device__ __forceinline__ float mx_blk_value(const MxBlk<kCodecMx>& k, const uint8_t* d) {
+  return mx_block_dot_dig(k.c, d) * mx_scale(k.e);
+}
+__device__ __forceinline__ float mx_affine(int sq, unsigned sb, const uint8_t* d) {
+  const float f = 2.f * __uint_as_float(((const uint32_t*)d)[24]);
+  const int sx = ((const int*)d)[25];
+  return f * fmaf((float)sq, bf16lo(sb), (float)sx * bf16hi(sb));
+}
+__device__ __forceinline__ float mx_blk_value(const MxBlk<kCodecQ4>& k, const uint8_t* d) {
+  return mx_affine(dq4_block_dot(k.c, d), k.sb, d);
+}
+__device__ __forceinline__ float mx_blk_value(const MxBlk<kCodecQ2>& k, const uint8_t* d) {
+  return mx_affine(dq2_block_dot(k.c, d), k.sb, d);
 }
 
 // grid (S I / kMxLWarps, T), block 32 kMxLWarps, clusters of kMxGuCluster CTAs: a[t][s][i] =
 // silu(G x_t)_i (U x_t)_i for the expert of slot s (slot k = the shared expert), one (slot, row)
-// per warp; a cluster's warps hold the 32 rows of one block of a, which they gather in the shared
-// memory of the cluster's first CTA, whose first warp writes the block's digit block to adig.
+// per warp, every lane's 4 blocks of the gate and up rows requested at once; a cluster's warps
+// hold the 32 rows of one block of a, which they gather in the shared memory of the cluster's
+// first CTA, whose first warp writes the block's digit block to adig.
 // Under a programmatic launch the CTA copies x_t's digit blocks (complete once this kernel
 // starts: their kernel ran two launches before, and the top-k triggered this launch only after
 // its own wait) before waiting for the top-k; then each warp resolves its expert and requests
@@ -668,6 +750,7 @@ __device__ __forceinline__ void mx_stage(float* dst, const float* src, int n) { 
 // 64 registers (4 CTAs per SM): the 512 CTAs of 4 slots x intermediate 1024 run in one wave on
 // 148 SMs, which pays for the few spilled bytes.
 constexpr int kMxGuCluster = 32 / kMxLWarps;
+template <int CODEC>
 __global__ void __cluster_dims__(kMxGuCluster, 1, 1) __launch_bounds__(kMxLWarps * 32, 4)
 mx_gateup_kernel(MxLayerParams p) {
   extern __shared__ __align__(16) unsigned char xd[];   // x_t's digit blocks, [H/32][kMxDig]
@@ -681,31 +764,42 @@ mx_gateup_kernel(MxLayerParams p) {
   // any writes into the first CTA's shared memory
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
   const int sl = item / p.I, i = item % p.I;
-  MxChunk2 c;
   const uint4* xsrc = (const uint4*)(p.xdig + (size_t)t * nb * kMxDig);
   for (int q = threadIdx.x; q < nb * (kMxDig / 16); q += blockDim.x) ((uint4*)xd)[q] = __ldcg(xsrc + q);
   griddep_wait();   // the top-k has completed
   griddep_launch_dependents();
-  const moe_expert* ex = sl < p.k ? p.experts + p.idx[t * p.k + sl] : &p.shared;
-  const uint32_t* gq = ex->gate.q + (size_t)i * (p.H / 8);
-  const uint32_t* uq = ex->up.q + (size_t)i * (p.H / 8);
-  const uint8_t* ge = (const uint8_t*)ex->gate.scales + (size_t)i * nb;
-  const uint8_t* ue = (const uint8_t*)ex->up.scales + (size_t)i * nb;
-  mx_load2(c, gq, ge, uq, ue, 0, nb, lane);
+  MxBlk<CODEC> ga[4], ua[4];
+  auto load = [&](int b0) {   // the expert's descriptor read again for every chunk of 128 blocks
+    const moe_expert* ex = sl < p.k ? p.experts + p.idx[t * p.k + sl] : &p.shared;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int b = b0 + 32 * u + lane;
+      ga[u] = mx_blk_load<CODEC>(ex->gate, i, p.H, b, b < nb);
+      ua[u] = mx_blk_load<CODEC>(ex->up, i, p.H, b, b < nb);
+    }
+  };
+  load(0);
   __syncthreads();
   float2 acc = make_float2(0.f, 0.f);
   for (int b0 = 0;;) {
-    mx_dot2(c, b0, nb, xd, lane, acc);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int b = b0 + 32 * u + lane;
+      if (b < nb) {
+        acc.x += mx_blk_value(ga[u], xd + b * kMxDig);
+        acc.y += mx_blk_value(ua[u], xd + b * kMxDig);
+      }
+    }
     b0 += 4 * 32;
     if (b0 >= nb) break;
-    mx_load2(c, gq, ge, uq, ue, b0, nb, lane);
+    load(b0);
   }
   const float g = warp_sum(acc.x), u = warp_sum(acc.y);
   asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
   if (lane == 0) *cluster.map_shared_rank(&ablk[rank * kMxLWarps + warp], 0) = g / (1.f + expf(-g)) * u;
   cluster.sync();   // the block is complete; nobody touches another CTA's shared memory after this
   if (rank == 0 && warp == 0)   // item is the block's first row
-    mx_digit_lanes(ablk[lane], lane, p.adig + (((size_t)t * p.S + sl) * (p.I / 32) + i / 32) * kMxDig);
+    mx_digit_lanes(ablk[lane], lane, p.adig + (((size_t)t * p.S + sl) * (p.I / 32) + i / 32) * kMxDig, CODEC);
 }
 
 // grid (ceil(H / kMxLWarps), T), block 32 kMxLWarps, a hidden row per warp:
@@ -714,30 +808,24 @@ mx_gateup_kernel(MxLayerParams p) {
 // gate/up kernel passed its wait) and requests its row's first blocks, then waits for the digit
 // blocks of a[t] and copies them. NS >= S bounds the slots held in registers; with up to 4 slots
 // the kernel fits 64 registers, so 4 CTAs per SM hold all 512 CTAs of hidden 4096 in one wave.
-template <int NS>
+template <int CODEC, int NS>
 __global__ void __launch_bounds__(kMxLWarps * 32, NS <= 4 ? 4 : 2) mx_down_kernel(MxLayerParams p) {
   extern __shared__ __align__(16) unsigned char ad[];   // a[t][s]'s digit blocks, [S][I/32][kMxDig]
   const int t = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nb = p.I / 32, sstride = nb * kMxDig;
   const int row = blockIdx.x * kMxLWarps + warp;
   const bool has = row < p.H;
-  const uint4* q[NS];
-  const uint8_t* e[NS];
-  uint4 c[NS];
-  unsigned sc[NS];
+  MxBlk<CODEC> c[NS];
+  auto load = [&](int b0) {   // every slot's block b0 + lane (descriptors read again per chunk)
 #pragma unroll
-  for (int sl = 0; sl < NS; ++sl) {
-    q[sl] = nullptr;
-    e[sl] = nullptr;
-    if (has && sl < p.S) {
-      const moe_qmat D = sl < p.k ? p.experts[p.idx[t * p.k + sl]].down : p.shared.down;
-      q[sl] = (const uint4*)(D.q + (size_t)row * (p.I / 8));
-      e[sl] = (const uint8_t*)D.scales + (size_t)row * nb;
+    for (int sl = 0; sl < NS; ++sl) {
+      const bool in = has && sl < p.S && b0 + lane < nb;
+      moe_qmat D{};
+      if (in) D = sl < p.k ? p.experts[p.idx[t * p.k + sl]].down : p.shared.down;
+      c[sl] = mx_blk_load<CODEC>(D, row, p.I, b0 + lane, in);
     }
-    const bool in = q[sl] && lane < nb;
-    c[sl] = in ? __ldg(q[sl] + lane) : make_uint4(0u, 0u, 0u, 0u);
-    sc[sl] = in ? __ldg(e[sl] + lane) : 0u;
-  }
+  };
+  load(0);
   griddep_wait();   // the digit blocks of a are complete
   griddep_launch_dependents();
   const uint4* asrc = (const uint4*)(p.adig + (size_t)t * p.S * sstride);
@@ -751,16 +839,10 @@ __global__ void __launch_bounds__(kMxLWarps * 32, NS <= 4 ? 4 : 2) mx_down_kerne
     const int b = b0 + lane;
 #pragma unroll
     for (int sl = 0; sl < NS; ++sl)
-      if (sl < p.S && b < nb)
-        y[sl] = fmaf(mx_block_dot_dig(c[sl], ad + sl * sstride + b * kMxDig), mx_scale(sc[sl]), y[sl]);
+      if (sl < p.S && b < nb) y[sl] += mx_blk_value(c[sl], ad + sl * sstride + b * kMxDig);
     b0 += 32;
     if (b0 >= nb) break;
-#pragma unroll
-    for (int sl = 0; sl < NS; ++sl) {
-      const bool in = sl < p.S && b0 + lane < nb;
-      c[sl] = in ? __ldg(q[sl] + b0 + lane) : make_uint4(0u, 0u, 0u, 0u);
-      sc[sl] = in ? __ldg(e[sl] + b0 + lane) : 0u;
-    }
+    load(b0);
   }
   float acc = p.h[(size_t)t * p.H + row];
 #pragma unroll
@@ -786,30 +868,42 @@ static cudaError_t mx_launch(const void* fn, dim3 grid, dim3 block, size_t smem,
   return cudaLaunchKernelExC(&cfg, fn, args);
 }
 
-cudaError_t launch_mx_digits(const uint16_t* src, int rows, int K, uint8_t* dst, cudaStream_t s, bool pdl) {
+cudaError_t launch_mx_digits(const uint16_t* src, int rows, int K, uint8_t* dst, int codec, cudaStream_t s,
+                             bool pdl) {
   const size_t n = (size_t)rows * (K / 32);
   const uint16_t* sp = src;
-  void* args[] = {(void*)&sp, &rows, &K, &dst};
+  void* args[] = {(void*)&sp, &rows, &K, &dst, &codec};
   return mx_launch((const void*)mx_digits_kernel, dim3((unsigned)((n + 7) / 8)), dim3(256), 0, s, pdl, args);
 }
 
 // gate/up (writing the digit blocks of a), down
-cudaError_t launch_mx_layer(const MxLayerParams& p, cudaStream_t s, bool pdl) {
+template <int CODEC>
+static cudaError_t mx_layer_launch(const MxLayerParams& p, cudaStream_t s, bool pdl) {
   const size_t sg = (size_t)(p.H / 32) * kMxDig;
   const size_t sd = (size_t)p.S * (p.I / 32) * kMxDig;
-  cudaError_t e = set_func_attr((const void*)mx_gateup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sg);
+  const void* gateup = (const void*)mx_gateup_kernel<CODEC>;
+  const void* down = p.S <= 2 ? (const void*)mx_down_kernel<CODEC, 2>
+                   : p.S <= 4 ? (const void*)mx_down_kernel<CODEC, 4>
+                   : p.S <= 6 ? (const void*)mx_down_kernel<CODEC, 6> : (const void*)mx_down_kernel<CODEC, kMxMaxSlots>;
+  cudaError_t e = set_func_attr(gateup, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sg);
   if (e != cudaSuccess) return e;
-  const void* down = p.S <= 2 ? (const void*)mx_down_kernel<2>
-                   : p.S <= 4 ? (const void*)mx_down_kernel<4>
-                   : p.S <= 6 ? (const void*)mx_down_kernel<6> : (const void*)mx_down_kernel<kMxMaxSlots>;
   e = set_func_attr(down, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sd);
   if (e != cudaSuccess) return e;
   MxLayerParams q = p;
   void* args[] = {&q};
   // S I / kMxLWarps CTAs: a multiple of the cluster size, since 32 divides I
-  e = mx_launch((const void*)mx_gateup_kernel, dim3(p.S * p.I / kMxLWarps, p.T), dim3(kMxLWarps * 32), sg, s, pdl, args);
+  e = mx_launch(gateup, dim3(p.S * p.I / kMxLWarps, p.T), dim3(kMxLWarps * 32), sg, s, pdl, args);
   if (e != cudaSuccess) return e;
   return mx_launch(down, dim3((p.H + kMxLWarps - 1) / kMxLWarps, p.T), dim3(kMxLWarps * 32), sd, s, pdl, args);
+}
+
+cudaError_t launch_mx_layer(const MxLayerParams& p, cudaStream_t s, bool pdl) {
+  switch (p.codec) {
+    case kCodecMx: return mx_layer_launch<kCodecMx>(p, s, pdl);
+    case kCodecQ4: return mx_layer_launch<kCodecQ4>(p, s, pdl);
+    case kCodecQ2: return mx_layer_launch<kCodecQ2>(p, s, pdl);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace qmoe

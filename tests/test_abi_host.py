@@ -160,16 +160,25 @@ def test_entry_points_reject_bad_arguments_before_launch():
     assert L.moe_selftest_wait_timeout(ws, n, 20 * 10 ** 9, None) == 1
 
 
-def test_unlaunchable_decode_shapes_are_rejected_before_launch():
-    """Hidden 8192, intermediate 3072, 4-bit, top-3 + shared: the decode
-    kernels' staging of a CTA's rows does not fit one CTA's shared memory, so
-    every decode entry point refuses the layer with MOE_ERR_UNSUPPORTED for
-    every token count from 1 to 8. On a machine without a GPU any launch
-    would fail with MOE_ERR_CUDA instead, so these codes also show that
-    nothing was launched. The grouped prefill path (T > 8) still takes the
-    layer, and the largest shapes each decode path accepts pass the checks."""
+def layer_path(layer, T):
+    p, n = C.c_int32(), C.c_int32()
+    rc = qm.lib().moe_layer_path(C.byref(layer), T, C.byref(p), C.byref(n))
+    return rc, qm.PATHS.get(p.value) if rc == 0 else None
+
+
+def test_unlaunchable_decode_shapes_are_rejected_before_launch(monkeypatch):
+    """Hidden 8192, intermediate 8192, 4-bit, top-8 + shared: the digit-block
+    down kernel would hold 9 slots x 256 digit blocks of 112 bytes, more than
+    one CTA's shared memory, and the chain's and the fused kernel's staging
+    does not fit either, so every decode entry point refuses the layer with
+    MOE_ERR_UNSUPPORTED for every token count from 1 to 8. On a machine
+    without a GPU any launch would fail with MOE_ERR_CUDA instead, so these
+    codes also show that nothing was launched. The grouped prefill path
+    (T > 8) still takes the layer, and the largest shapes each decode path
+    accepts pass the checks."""
+    monkeypatch.delenv("MOE_DECODE_KERNEL", raising=False)
     L = qm.lib()
-    bad = fake_layer(hidden=8192, inter=3072)
+    bad = fake_layer(hidden=8192, inter=8192, top_k=8)
     p = C.c_void_p(0x200000)
     ws = C.c_void_p(0x400000)
     for T in (1, 8):
@@ -183,13 +192,23 @@ def test_unlaunchable_decode_shapes_are_rejected_before_launch():
         assert L.moe_layer_forward_noalloc(C.byref(bad), p, p, T, p, None, None, None, None) == 2
     lays = (qm._Layer * 3)(bad, bad, bad)
     assert L.moe_stack_forward(lays, 3, p, p, p, None, None, None, ws, n, None) == 2
-    # the limits: fused (T = 1) up to hidden 4096 / inter 1152; the chain up to hidden 7552 / inter 2688 (4-bit)
-    assert ws_size(fake_layer(hidden=4096, inter=1152), 1)[0] == 0
-    assert ws_size(fake_layer(hidden=7552, inter=2688), 1)[0] == 0
-    assert ws_size(fake_layer(hidden=7552, inter=2688), 8)[0] == 0
-    assert ws_size(fake_layer(hidden=7680, inter=1024), 8)[0] == 2
-    assert ws_size(fake_layer(hidden=4096, inter=2816), 8)[0] == 2
-    assert ws_size(fake_layer(hidden=8192, inter=2048, bits=2), 8)[0] == 0
+    # the digit-block kernels (default for decode): 9 slots up to intermediate 7296
+    assert layer_path(fake_layer(hidden=8192, inter=7296, top_k=8), 8) == (0, "digit")
+    assert layer_path(fake_layer(hidden=8192, inter=7424, top_k=8), 8)[0] == 2
+    assert layer_path(fake_layer(), 1) == (0, "digit") and layer_path(fake_layer(), 9) == (0, "prefill")
+    # a shape the grouped prefill cannot take runs the digit-block kernels token by token
+    assert layer_path(fake_layer(hidden=4096, inter=2816), 9) == (0, "digit")
+    # MOE_DECODE_KERNEL=chain: the chain up to hidden 7552 / inter 2688 (4-bit), else the digit kernels
+    monkeypatch.setenv("MOE_DECODE_KERNEL", "chain")
+    assert layer_path(fake_layer(hidden=7552, inter=2688), 1) == (0, "chain")
+    assert layer_path(fake_layer(hidden=7552, inter=2688), 8) == (0, "chain")
+    assert layer_path(fake_layer(hidden=7680, inter=1024), 8) == (0, "digit")
+    assert layer_path(fake_layer(hidden=4096, inter=2816), 8) == (0, "digit")
+    assert layer_path(fake_layer(hidden=8192, inter=2048, bits=2), 8) == (0, "chain")
+    # MOE_DECODE_KERNEL=fused: the fused kernel (T = 1) up to hidden 4096 / inter 1152
+    monkeypatch.setenv("MOE_DECODE_KERNEL", "fused")
+    assert layer_path(fake_layer(hidden=4096, inter=1152), 1) == (0, "fused")
+    assert layer_path(fake_layer(hidden=4096, inter=1152), 2) == (0, "chain")
 
 
 def test_wait_bound_and_header_words_documented():

@@ -13,8 +13,9 @@ So the ids must equal the oracle's bit for bit:
     exact tie. These must take the exact recheck, which the workspace header
     counts.
 The same ids and layer outputs are checked through the decode layer (the
-four-kernel chain, or the fused kernel when MOE_DECODE_KERNEL=fused) and the
-prefill path, and the decode paths run at the largest shapes they accept.
+digit-block kernels by default; the four-kernel chain when
+MOE_DECODE_KERNEL=chain, the fused kernel when MOE_DECODE_KERNEL=fused) and
+the prefill path, and the decode paths run at the largest shapes they accept.
 """
 import os
 
@@ -250,7 +251,7 @@ def _layer_vs_oracle(cfg, T, dev, calls=2):
 def test_fused_layer_at_its_largest_shape(dev, bits):
     """hidden 4096 and intermediate 1152 = 8 rows x 148 SMs (rounded to a span):
     the largest shape whose per-SM gate/up and down rows fit the fused kernel
-    (which runs it when MOE_DECODE_KERNEL=fused; the chain otherwise)."""
+    (which runs it when MOE_DECODE_KERNEL=fused; the decode path of the environment otherwise)."""
     cfg = fixtures.Config("fused_max", H=4096, E=16, k=3, I=1152, bits=bits,
                           scale_sigma=0.02 if bits == 4 else 0.05)
     _layer_vs_oracle(cfg, 1, dev)
@@ -277,10 +278,16 @@ def test_odd_span_counts(dev, bits):
 
 
 def test_decode_path_is_the_one_requested(dev):
-    """Single-token calls take the four-kernel chain unless MOE_DECODE_KERNEL=fused."""
+    """Decode calls take the digit-block kernels, the four-kernel chain with
+    MOE_DECODE_KERNEL=chain, the fused kernel (one token) with =fused."""
     t = fxg.device_layer(NT, 0)
     layer = qm.layer_from_tensors(NT, t)
-    want = "fused" if os.environ.get("MOE_DECODE_KERNEL") == "fused" else "chain"
-    assert qm.moe_layer_path(layer, 1) == (want, 2 if want == "fused" else 5)
-    assert qm.moe_layer_path(layer, 2) == ("chain", 5)
+    env = os.environ.get("MOE_DECODE_KERNEL")
+    if env == "fused":
+        assert qm.moe_layer_path(layer, 1) == ("fused", 2)
+        assert qm.moe_layer_path(layer, 2) == ("chain", 5)
+    else:
+        want = "chain" if env == "chain" else "digit"
+        assert qm.moe_layer_path(layer, 1) == (want, 5)
+        assert qm.moe_layer_path(layer, 8) == (want, 5)
     assert qm.moe_layer_path(layer, 9) == ("prefill", 6)

@@ -49,8 +49,8 @@ def test_wait_timeout_is_latched_and_the_context_stays_usable():
 def test_grid_barrier_timeout_is_latched_and_the_workspace_recovers():
     """The fused decode kernel's grid-wide barrier: one CTA arrives at a round
     sized for two, its bounded wait runs out and leaves the arrival counter at
-    1. After moe_poll_status the same workspace serves fused single-token
-    layer calls whose routing and outputs match the oracle."""
+    1. After moe_poll_status the same workspace serves single-token layer
+    calls whose routing and outputs match the oracle."""
     assert torch.cuda.is_available()
     dev = torch.device("cuda")
     cfg = fixtures.CONFIGS["tiny"]

@@ -80,16 +80,18 @@ def test_noalloc_scratch_covers_largest_decode_shape():
     L = qm.lib()
     p = 0x100000
     ex = qm._Expert(*[qm._QMat(p, p, p) for _ in range(3)])
-    cases = [(4, 3, 7552, 2688), (4, 8, 7552, 2176), (2, 3, 8192, 4352), (2, 8, 8192, 3328)]
+    # the digit-block kernels take hidden and intermediate up to 8192 with top-3 + shared, and
+    # intermediate up to 7296 with top-8 + shared (their down kernel's digit blocks of a)
+    cases = [(4, 3, 8192, 8192), (4, 8, 8192, 7296), (2, 3, 8192, 8192), (2, 8, 8192, 7296)]
     for bits, k, H, I in cases:
         lay = qm._Layer(H, I, 4096, k, bits, 64, 1, 1e-6, p, None, p, ex, p, p)
         n = C.c_size_t(0)
         assert L.moe_workspace_size(C.byref(lay), 8, C.byref(n)) == 0, (bits, k, H, I)
-        assert 0 < n.value <= (4 << 20)
-        big = qm._Layer(H, I + 128 * (1 if bits == 4 else 8), 4096, k, bits, 64, 1, 1e-6, p, None, p, ex, p, p)
+        assert 0 < n.value <= qm.NOALLOC_SCRATCH_BYTES
+        big = qm._Layer(H, I + 128, 4096, k, bits, 64, 1, 1e-6, p, None, p, ex, p, p)
         assert L.moe_workspace_size(C.byref(big), 8, C.byref(n)) == 2   # one span more: no longer fits
     pp = C.c_void_p(0x200000)
     lay = qm._Layer(4096, 1024, 512, 3, 4, 64, 1, 1e-6, p, None, p, ex, p, p)
     assert L.moe_layer_forward_noalloc(C.byref(lay), pp, pp, 9, pp, None, None, None, None) == 2   # MOE_ERR_UNSUPPORTED
-    bad = qm._Layer(8192, 3072, 512, 3, 4, 64, 1, 1e-6, p, None, p, ex, p, p)
+    bad = qm._Layer(8192, 7424, 512, 8, 4, 64, 1, 1e-6, p, None, p, ex, p, p)
     assert L.moe_layer_forward_noalloc(C.byref(bad), pp, pp, 1, pp, None, None, None, None) == 2
