@@ -209,9 +209,8 @@ def busy(fn, stream, seconds: float = 0.25):
 # kernels of each decode path, in launch order
 KERNELS = {"fused": ["fused_decode_kernel"],
            "chain": ["route_logits_kernel", "gateup_decode_kernel", "down_decode_kernel", "norm_kernel"],
-           "digit": ["route_logits_kernel+mx_digits_kernel", "topk_kernel", "mx_gateup_kernel+mx_down_kernel",
-                     "norm_cluster_kernel"]}
-LAUNCHES = {"fused": 1, "chain": 4, "digit": 6}   # kernels per decode step
+           "digit": ["route_logits_kernel", "topk_kernel", "mx_gateup_kernel+mx_down_kernel", "norm_cluster_kernel"]}
+LAUNCHES = {"fused": 1, "chain": 4, "digit": 5}   # kernels per decode step
 DTYPES = {"fused": "u4 codes x s8 activation digits on int8 tensor cores (s32), fp32 scale+accumulate",
           "chain": "u4 codes x s8 activation digits on int8 tensor cores (s32), fp32 scale+accumulate",
           "digit": "u4/u2 codes x s8 digits of 22-bit fixed-point activations by dp4a (s32), fp32 scale+bias"}
@@ -232,7 +231,6 @@ def kernel_bytes(cfg, name: str, layers: int = 1) -> int:
            "gateup_decode_kernel": gu + 2 * cfg.H,
            "down_decode_kernel": dn + 4 * cfg.H * (S + 2),
            "norm_kernel": 6 * cfg.H * 4,
-           "route_logits_kernel+mx_digits_kernel": router + 2 * cfg.H,
            "topk_kernel": 12 * (cfg.E + 1),
            "mx_gateup_kernel+mx_down_kernel": gu + dn + 2 * 4 * cfg.H,
            "norm_cluster_kernel": 6 * cfg.H * 4}[name]
@@ -242,10 +240,10 @@ def kernel_bytes(cfg, name: str, layers: int = 1) -> int:
 # the files that define each kernel (its translation unit and the headers it includes); recorded
 # ncu traffic is tied to their hash
 DECODE_SOURCES = ("common.cuh", "kernels.cuh", "decode.cu", "stage.cuh", "sync.cuh", "topk.cuh")   # gate/up, down
-ROUTER_SOURCES = ("common.cuh", "kernels.cu", "kernels.cuh", "topk.cuh")                           # router, norm
+ROUTER_SOURCES = ("common.cuh", "kernels.cu", "kernels.cuh", "topk.cuh", "digits.cuh")             # router, norm
 FUSED_SOURCES = ("common.cuh", "kernels.cuh", "fused.cu", "stage.cuh", "sync.cuh", "topk.cuh")
 PREFILL_SOURCES = ("common.cuh", "kernels.cuh", "prefill.cu")
-MX_SOURCES = ("common.cuh", "kernels.cuh", "mx.cu")
+MX_SOURCES = ("common.cuh", "kernels.cuh", "digits.cuh", "mx.cu")
 SOURCES_OF = {"route_logits_kernel": ROUTER_SOURCES, "norm_kernel": ROUTER_SOURCES,
               "fused_decode_kernel": FUSED_SOURCES, "mx_gateup_kernel+mx_down_kernel": MX_SOURCES}
 TRAFFIC_KEY = {"mx_gateup_kernel+mx_down_kernel": "mx_experts"}   # name of a stage's record in traffic.txt
@@ -842,7 +840,7 @@ def ours_cached(args, cfg):
                      "peak_kind": "measured in this run (256 MB page-locked copy)"},
         "e2e": {"value": steps / (ms * 1e-3), "unit": "tokens/s", "steps": steps,
                 "h2d_bytes_per_step": copied, "d2h_bytes_per_step": 4 * cfg.k},
-        "gpu_launches": 6 * steps, "clocks": clk,
+        "gpu_launches": (2 + LAUNCHES[qm.moe_layer_path(layer, 1)[0]]) * steps, "clocks": clk,   # routing, then the layer
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -978,7 +976,7 @@ def ours_mx(args, cfg):
             qm.moe_layer_forward_timed(layer, xs[i:i + 1], hs[i:i + 1], xo[i:i + 1], ws=ws, events=evs[s],
                                        stream=stream)
     stream.synchronize()
-    names = ["route_logits+digits_x", "topk", "mx_gateup+mx_down", "norm"]
+    names = ["route_logits (+ digit blocks of x)", "topk", "mx_gateup+mx_down", "norm"]
     dur = [sum(evs[s][j].elapsed_time(evs[s][j + 1]) for s in range(prof_n)) / prof_n for j in range(nst)]
     # end to end with host buffers: x and h in, x_out back, every step
     e2e_n = min(args.e2e_steps, steps, 512)
@@ -1013,7 +1011,7 @@ def ours_mx(args, cfg):
                      "algorithmic_bytes": per_tok, "peak_kind": peak_kind},
         "e2e": {"value": e2e_n / (e2e_ms_ * 1e-3), "unit": "tokens/s", "steps": e2e_n, "reps": E2E_REPS,
                 "h2d_bytes_per_step": cfg.H * 6, "d2h_bytes_per_step": cfg.H * 2},
-        "gpu_launches": 6 * steps, "path": path, "clocks": clk,
+        "gpu_launches": 5 * steps, "path": path, "clocks": clk,
     }
     if rank == 0 and not args.no_cpu_baseline:
         rate, n, threads, el = mx_oracle_sample(cfg, args.cpu_seconds)

@@ -230,18 +230,20 @@ moe_status mx_chain(const moe_layer* L, const uint16_t* x_in, float* h, int T, u
   rp.logits = at<double>(ws, W.logits);
   rp.bound = at<float>(ws, W.bound);
   rp.h = h; rp.x_rec = x_rec; rp.h_rec = h_rec;
+  const int codec = codec_of(L);
   if (T > kDecodeMaxT) {   // many tokens: the exact integer router on tcgen05
     rp.lpart = at<long long>(ws, W.lpart);
     rp.wdig = at<int8_t>(ws, W.wdig); rp.xdig = at<int8_t>(ws, W.xdig);
     rp.wst = at<double>(ws, W.wst); rp.xst = at<double>(ws, W.xst);
     rp.status = at<uint32_t>(ws, W.status); rp.wait_ns = wait_bound_ns();
     if (launch_route_gemm(rp, s) != cudaSuccess) return MOE_ERR_CUDA;
-  } else if (launch_route(rp, s, pdl) != cudaSuccess) {
-    return MOE_ERR_CUDA;
+    // the digit blocks of x after the router
+    if (launch_mx_digits(x_in, T, H, at<uint8_t>(ws, W.mxx), codec, s, false) != cudaSuccess) return MOE_ERR_CUDA;
+  } else {   // decode: the router writes the digit blocks of x (the gate/up kernel reads them before its own wait)
+    rp.xblocks = at<uint8_t>(ws, W.mxx);
+    rp.codec = codec;
+    if (launch_route(rp, s, pdl) != cudaSuccess) return MOE_ERR_CUDA;
   }
-  // the digit blocks of x, beside the router (the gate/up kernel reads them before its own wait)
-  const int codec = codec_of(L);
-  if (launch_mx_digits(x_in, T, H, at<uint8_t>(ws, W.mxx), codec, s, pdl) != cudaSuccess) return MOE_ERR_CUDA;
   mark(1);
   TopkParams tp{};
   tp.E = E; tp.k = k; tp.T = T; tp.has_shared = L->has_shared; tp.H = H;

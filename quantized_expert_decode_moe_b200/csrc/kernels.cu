@@ -11,6 +11,7 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "digits.cuh"
 #include "topk.cuh"
 
 namespace cg = cooperative_groups;
@@ -150,8 +151,10 @@ constexpr int kRouteThreads = kRouteRows * kRouteSplit * 32;
 constexpr int kRouteChunks = 4;   // 16-byte weight chunks per lane per pass
 
 // The router's weights do not depend on the previous kernel and are loaded
-// before griddepcontrol.wait; x after it. Side job of the decode chain (CTAs
-// of token row 0): optionally record the layer's inputs x and h.
+// before griddepcontrol.wait; x after it. Side jobs: optionally record the
+// layer's inputs x and h (CTAs of token row 0), and write x's digit blocks
+// for the digit-block layer kernels (a warp per 32-value block, from the x
+// staged in shared memory).
 __global__ void __launch_bounds__(kRouteThreads) route_logits_kernel(RouteParams p) {
   extern __shared__ __align__(128) unsigned char smem[];
   uint4* xs = (uint4*)smem;                                  // [H/8]
@@ -198,6 +201,12 @@ __global__ void __launch_bounds__(kRouteThreads) route_logits_kernel(RouteParams
         }
       }
       __syncthreads();
+      if (p.xblocks) {   // warp-uniform: every lane of a warp takes the same blocks
+        const int nb = p.H / 32, nw = kRouteThreads / 32;
+        for (int b = blockIdx.x * nw + warp; b < nb; b += gridDim.x * nw)
+          mx_digit_lanes(bf16_to_f32(((const uint16_t*)xs)[b * 32 + lane]), lane,
+                         p.xblocks + ((size_t)t * nb + b) * kMxDig, p.codec);
+      }
     }
 #pragma unroll
     for (int i = 0; i < kRouteChunks; ++i) {

@@ -68,6 +68,9 @@ struct RouteParams {
   uint32_t* status; unsigned long long wait_ns;   // bound of the tcgen05 router's waits
   // side job of the decode chain (null when unused): copies of the layer's inputs x, h ([T][H])
   const float* h; uint16_t* x_rec; float* h_rec;
+  // side job for the digit-block layer kernels (null when unused): x's digit blocks
+  // [T][H/32][112 bytes] in the order of codec `codec`
+  uint8_t* xblocks; int codec;
 };
 
 struct TopkParams {
