@@ -29,24 +29,25 @@
  *    environment (read once, clamped to 1 ms .. 10 s), latches
  *    MOE_ERR_TIMEOUT and skips the remaining waits of the call: the outputs
  *    of a call that latched a timeout are invalid.
- *  - Supported shapes. The decode kernels stage each CTA's rows of the active
- *    experts in shared memory, one CTA per SM. A layer call is rejected with
- *    MOE_ERR_UNSUPPORTED, before any launch, when no kernel path fits the
- *    device:
- *      T <= 8    the four-kernel decode chain (also for T = 1, by default): gate/up stages 3 experts x 8 rows x H
- *                and down up to 4 experts x 32 rows x I in one CTA (227 KB
- *                per CTA, top_k 3 + shared: H <= 7552 and I <= 2688 at 4
- *                bits, I <= 4352 at 2 bits);
+ *  - Supported shapes. A layer call is rejected with MOE_ERR_UNSUPPORTED,
+ *    before any launch, when no kernel path fits the device:
+ *      T <= 8    the digit-block decode kernels (the default): the down
+ *                kernel holds every slot's SwiGLU output as digit blocks
+ *                (112 bytes per 32 values) in one CTA's shared memory,
+ *                (top_k + shared) * I <= 51,200 (227 KB per CTA);
  *      T > 8     the grouped prefill kernels (two stages of their ring of
  *                weight tiles must fit and their row tiles must divide the
- *                matrices);
- *      MXFP4    (group 32), any T: the down kernel stages every slot's SwiGLU
- *                output in shared memory: (top_k + shared) * I <= 51,200;
- *    and H, I <= 8192 throughout. With MOE_DECODE_KERNEL=fused in the
- *    environment (read once), single-token calls and stacks take the fused
- *    single-kernel layer where it fits: H <= 4096, top_k <= 3 (top_k +
- *    shared <= 4), E <= 4096, I <= 8 n and H <= 32 n with n = min(SMs, I, H)
- *    (148 SMs: I <= 1152); otherwise the chain.
+ *                matrices), else the digit-block kernels token by token;
+ *      MXFP4    (group 32), any T: the digit-block kernels, same rule;
+ *    and H, I <= 8192 throughout. MOE_DECODE_KERNEL in the environment (read
+ *    at every call) selects other decode kernels where they fit (the
+ *    digit-block kernels otherwise): =chain the four-kernel chain, whose
+ *    gate/up stages 3 experts x 8 rows x H and down up to 4 experts x 32 rows
+ *    x I in one CTA (top_k 3 + shared: H <= 7552 and I <= 2688 at 4 bits,
+ *    I <= 4352 at 2 bits); =fused, for single-token calls and stacks, the
+ *    fused single-kernel layer: H <= 4096, top_k <= 3 (top_k + shared <= 4),
+ *    E <= 4096, I <= 8 n and H <= 32 n with n = min(SMs, I, H) (148 SMs:
+ *    I <= 1152), else the chain.
  *    moe_layer_forward_noalloc and moe_stack_forward apply the same rules
  *    (T = 1 for the stack), and moe_workspace_size applies the rule of
  *    T = max_tokens.
@@ -253,12 +254,14 @@ moe_status moe_group_tokens(int32_t T, int32_t k, int32_t E, const int32_t* topk
 /*
  * Whole MoE layer for T tokens: router, expert gate/up + SwiGLU, down, combine
  * with the shared-expert gate, residual and RMSNorm, all on the device with
- * no host round trip. T = 1..8 runs the four-kernel decode chain (router,
- * gate/up + SwiGLU, down + combine, RMSNorm, linked by programmatic
- * dependent launch), or for T = 1 on request the fused decode kernel (the
- * whole layer in one persistent launch, grid-wide barriers between its
- * phases); larger T the prefill kernels (grouping by expert, grouped dequant
- * GEMM). See "Supported shapes" above.
+ * no host round trip. T = 1..8 runs the digit-block decode kernels (router,
+ * which also writes x as exact fixed-point digit planes; certified top-k;
+ * gate/up + SwiGLU, which writes the SwiGLU outputs' digit planes; down +
+ * combine + residual; RMSNorm; five launches linked by programmatic
+ * dependent launch), or on request the four-kernel decode chain or, for
+ * T = 1, the fused decode kernel (the whole layer in one persistent launch,
+ * grid-wide barriers between its phases); larger T the prefill kernels
+ * (grouping by expert, grouped dequant GEMM). See "Supported shapes" above.
  *   x_in bf16 [T][H]; h fp32 [T][H] residual in, h' out; x_out bf16 [T][H];
  *   x_out_f32 fp32 [T][H] or NULL; topk_idx int32 [T][k] or NULL;
  *   topk_w fp32 [T][k] or NULL.
@@ -269,7 +272,8 @@ moe_status moe_layer_forward(const moe_layer* layer, const uint16_t* x_in, float
 
 /*
  * L layers in sequence for one decode token: layer l's x_out feeds layer l+1
- * and h is carried in fp32 ("Deferred GPU expert compute"). With the fused
+ * and h is carried in fp32 ("Deferred GPU expert compute"); each layer runs
+ * the decode kernels of moe_layer_forward at T = 1. With the fused
  * kernel (MOE_DECODE_KERNEL=fused), up to 24 layers run in one launch: x and
  * h stay on the chip between layers, and the next layer's router rows and
  * shared expert are requested while the current layer finishes.
@@ -311,9 +315,10 @@ moe_status moe_layer_path(const moe_layer* layer, int32_t T, int32_t* path, int3
  * recorded before the first and after each of the kernels of the layer, so a
  * caller can time them one by one. events: host array of n_events created
  * cudaEvent_t handles (passed as void*); n_events must be at least the number
- * of recorded stages + 1 (moe_layer_path reports it): decode chain 5
- * (router, gate/up, down, norm); fused decode 2 (the one kernel); prefill 6 (router, top-k + grouping, gate/up, down,
- * combine + norm). The kernels run without programmatic overlap between
+ * of recorded stages + 1 (moe_layer_path reports it): digit-block decode
+ * and MXFP4 5 (router, top-k, gate/up + down, norm); decode chain 5 (router,
+ * gate/up, down, norm); fused decode 2 (the one kernel); prefill 6 (router,
+ * top-k + grouping, gate/up, down, combine + norm). The kernels run without programmatic overlap between
  * them. Same arguments and errors otherwise.
  */
 moe_status moe_layer_forward_timed(const moe_layer* layer, const uint16_t* x_in, float* h, int32_t T,
