@@ -262,21 +262,12 @@ moe_status mx_chain(const moe_layer* L, const uint16_t* x_in, float* h, int T, u
   mp.idx = tp.idx; mp.w = tp.w; mp.sg = tp.sg;
   mp.h = h;
   mp.xdig = at<uint8_t>(ws, W.mxx); mp.adig = at<uint8_t>(ws, W.mxa);
-  // decode: the RMSNorm in the down kernel's last CTA per token (timed calls keep it a kernel of
-  // its own, so that its stage is measured)
-  const bool fold = T <= kDecodeMaxT && !events;
-  if (fold) {
-    mp.norm_done = at<unsigned>(ws, kNormDoneOffset);
-    mp.gamma = L->rms_gamma; mp.eps = L->rms_eps; mp.x_out = x_out; mp.x_out_f32 = x_out_f32;
-  }
   if (launch_mx_layer(mp, s, pdl) != cudaSuccess) return MOE_ERR_CUDA;
   mark(3);
-  if (!fold) {
-    NormParams np{};
-    np.H = H; np.k = 0; np.T = T;
-    np.h = h; np.gamma = L->rms_gamma; np.eps = L->rms_eps; np.x_out = x_out; np.x_out_f32 = x_out_f32;
-    if (launch_norm(np, pdl, s) != cudaSuccess) return MOE_ERR_CUDA;
-  }
+  NormParams np{};
+  np.H = H; np.k = 0; np.T = T;
+  np.h = h; np.gamma = L->rms_gamma; np.eps = L->rms_eps; np.x_out = x_out; np.x_out_f32 = x_out_f32;
+  if (launch_norm(np, pdl, s) != cudaSuccess) return MOE_ERR_CUDA;
   mark(4);
   return MOE_OK;
 }

@@ -15,8 +15,7 @@ constexpr size_t kSelFlagOffset = 80;   // byte offset of the decode chain's sel
 
 // Workspace carve-up for T tokens of one layer shape. The first 256 bytes are
 // the header: the status word (word 0), the count of top-k selections that
-// needed the exact recheck (word 4), the digit-block down kernel's per-token
-// counts of finished CTAs (words 8..15), the grid-barrier arrival counters
+// needed the exact recheck (word 4), the grid-barrier arrival counters
 // (words 16..19), the decode chain's per-token selection flags (words
 // 20..27) and the grid-barrier generations (words 32, 40, 48, 56).
 struct WsLayout {
@@ -270,15 +269,9 @@ struct MxLayerParams {
   moe_expert shared;           // slot k when S > k
   const int32_t* idx; const float* w; const float* sg;   // [T][k], [T][k], [T]
   float* h;                    // [T][H], in place: h + the weighted expert outputs
-  const uint8_t* xdig;         // [T][H/32] digit blocks of x (the router or launch_mx_digits)
+  const uint8_t* xdig;         // [T][H/32] digit blocks of x (launch_mx_digits, after the router)
   uint8_t* adig;               // [T][S][I/32] digit blocks of a (written by the gate/up kernel)
-  // RMSNorm folded into the down kernel (null norm_done: a separate norm kernel runs): per-token
-  // counts of finished CTAs [T] (zero between calls; the last CTA of a token resets its count),
-  // gamma bf16 [H], x_out bf16 [T][H], x_out_f32 fp32 [T][H] or null
-  unsigned* norm_done;
-  const uint16_t* gamma; float eps; uint16_t* x_out; float* x_out_f32;
 };
-constexpr size_t kNormDoneOffset = 32;   // byte offset of the folded RMSNorm's counts (8 words)
 // digit blocks of rows of K bf16 values for the layer kernels of a codec: 112 bytes per 32
 cudaError_t launch_mx_digits(const uint16_t* src, int rows, int K, uint8_t* dst, int codec, cudaStream_t s, bool pdl);
 cudaError_t launch_mx_layer(const MxLayerParams& p, cudaStream_t s, bool pdl = false);

@@ -754,35 +754,8 @@ mx_gateup_kernel(MxLayerParams p) {
     mx_digit_lanes(ablk[lane], lane, p.adig + (((size_t)t * p.S + sl) * (p.I / 32) + i / 32) * kMxDig, CODEC);
 }
 
-// The RMSNorm of token t's h' (complete in global memory) by one CTA: x_out = h' / sqrt(mean h'^2
-// + eps) * gamma, in bf16 (and fp32 when asked).
-__device__ __forceinline__ void mx_norm_token(const MxLayerParams& p, int t) {
-  __shared__ float red[kMxLWarps];
-  const float* hr = p.h + (size_t)t * p.H;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  float ss = 0.f;
-  for (int j = threadIdx.x; j < p.H; j += blockDim.x) {
-    const float v = __ldcg(hr + j);
-    ss = fmaf(v, v, ss);
-  }
-  ss = warp_sum(ss);
-  if (lane == 0) red[warp] = ss;
-  __syncthreads();
-  float tot = 0.f;
-#pragma unroll
-  for (int w = 0; w < kMxLWarps; ++w) tot += red[w];
-  const float inv = 1.f / sqrtf(tot / (float)p.H + p.eps);
-  for (int j = threadIdx.x; j < p.H; j += blockDim.x) {
-    const float xo = __ldcg(hr + j) * inv * bf16_to_f32(p.gamma[j]);
-    p.x_out[(size_t)t * p.H + j] = f32_to_bf16(xo);
-    if (p.x_out_f32) p.x_out_f32[(size_t)t * p.H + j] = xo;
-  }
-}
-
 // grid (ceil(H / kMxLWarps), T), block 32 kMxLWarps, a hidden row per warp:
 // h[t][j] += sum_{s<k} w[t][s] (D_s a[t][s])_j + sg[t] (D_shared a[t][k])_j, in that order.
-// With norm_done set, the CTA that finishes a token's rows last (a count per token, after a
-// device-scope fence of every row it wrote) normalises the token's h' and resets the count.
 // Each warp resolves every slot's expert (the selection is complete: the top-k ran before the
 // gate/up kernel passed its wait) and requests its row's first blocks, then waits for the digit
 // blocks of a[t] and copies them. NS >= S bounds the slots held in registers; with up to 4 slots
@@ -810,39 +783,24 @@ __global__ void __launch_bounds__(kMxLWarps * 32, NS <= 4 ? 4 : 2) mx_down_kerne
   const uint4* asrc = (const uint4*)(p.adig + (size_t)t * p.S * sstride);
   for (int qq = threadIdx.x; qq < p.S * sstride / 16; qq += blockDim.x) ((uint4*)ad)[qq] = __ldcg(asrc + qq);
   __syncthreads();
-  if (has) {
-    float y[NS];
+  if (!has) return;
+  float y[NS];
 #pragma unroll
-    for (int sl = 0; sl < NS; ++sl) y[sl] = 0.f;
-    for (int b0 = 0;;) {   // every slot's block b0 + lane in flight at once
-      const int b = b0 + lane;
-#pragma unroll
-      for (int sl = 0; sl < NS; ++sl)
-        if (sl < p.S && b < nb) y[sl] += mx_blk_value(c[sl], ad + sl * sstride + b * kMxDig);
-      b0 += 32;
-      if (b0 >= nb) break;
-      load(b0);
-    }
-    float acc = p.h[(size_t)t * p.H + row];
+  for (int sl = 0; sl < NS; ++sl) y[sl] = 0.f;
+  for (int b0 = 0;;) {   // every slot's block b0 + lane in flight at once
+    const int b = b0 + lane;
 #pragma unroll
     for (int sl = 0; sl < NS; ++sl)
-      if (sl < p.S) acc = fmaf(sl < p.k ? p.w[t * p.k + sl] : p.sg[t], warp_sum(y[sl]), acc);
-    if (lane == 0) {
-      p.h[(size_t)t * p.H + row] = acc;
-      __threadfence();   // this row before the token's count
-    }
+      if (sl < p.S && b < nb) y[sl] += mx_blk_value(c[sl], ad + sl * sstride + b * kMxDig);
+    b0 += 32;
+    if (b0 >= nb) break;
+    load(b0);
   }
-  if (p.norm_done) {
-    __shared__ unsigned last;
-    __syncthreads();
-    if (threadIdx.x == 0) last = atomicAdd(p.norm_done + t, 1u) == gridDim.x - 1 ? 1u : 0u;
-    __syncthreads();
-    if (last) {
-      __threadfence();   // every other CTA's rows, counted before this one, are visible
-      mx_norm_token(p, t);
-      if (threadIdx.x == 0) p.norm_done[t] = 0u;
-    }
-  }
+  float acc = p.h[(size_t)t * p.H + row];
+#pragma unroll
+  for (int sl = 0; sl < NS; ++sl)
+    if (sl < p.S) acc = fmaf(sl < p.k ? p.w[t * p.k + sl] : p.sg[t], warp_sum(y[sl]), acc);
+  if (lane == 0) p.h[(size_t)t * p.H + row] = acc;
 }
 
 static cudaError_t mx_launch(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
