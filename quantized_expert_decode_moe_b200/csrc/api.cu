@@ -212,9 +212,9 @@ moe_status decode_chain(const moe_layer* L, const uint16_t* x_in, float* h, int 
   return MOE_OK;
 }
 
-// A layer on the digit-block kernels (MXFP4 experts at any number of tokens, affine ones in
-// decode): router, certified top-k, gate/up with SwiGLU, down with the weighted combine and the
-// residual (mx.cu), RMSNorm.
+// A layer on the digit-block kernels (MXFP4 experts at any number of tokens; affine ones in decode,
+// and above 8 tokens where the grouped prefill cannot take the shape): router, certified top-k,
+// gate/up with SwiGLU, down with the weighted combine and the residual (mx.cu), RMSNorm.
 moe_status mx_chain(const moe_layer* L, const uint16_t* x_in, float* h, int T, uint16_t* x_out, float* x_out_f32,
                     int32_t* topk_idx, float* topk_w, void* ws, cudaStream_t s, void* const* events = nullptr,
                     uint16_t* x_rec = nullptr, float* h_rec = nullptr) {

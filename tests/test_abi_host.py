@@ -244,3 +244,13 @@ def test_mxfp4_entry_points_check_arguments_on_the_host():
     assert L.moe_expert_gemm_mxfp4(None, 128, 128, *args, need, None) == 1
     assert L.moe_expert_gemm_mxfp4(C.byref(W), 128, 128, C.c_void_p(0x1000), 4, C.c_void_p(0x1000),
                                    C.c_void_p(0x10010), need, None) == 1      # workspace not 256-byte aligned
+
+
+def test_binding_constants_match_the_header():
+    """The binding's copies of header constants: the no-alloc scratch size and the path codes."""
+    hdr = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "moe.h")).read()
+    m = re.search(r"#define MOE_NOALLOC_SCRATCH_BYTES \((\d+)u << (\d+)\)", hdr)
+    assert m and int(m.group(1)) << int(m.group(2)) == qm.NOALLOC_SCRATCH_BYTES
+    codes = dict((int(v), k) for k, v in re.findall(r"MOE_PATH_(\w+) = (\d+)", hdr))
+    assert {c: n.lower() for c, n in codes.items()} == {1: "fused", 2: "chain", 3: "prefill", 4: "mxfp4", 5: "digit"}
+    assert qm.PATHS == {1: "fused", 2: "chain", 3: "prefill", 4: "mxfp4", 5: "digit"}
